@@ -1,0 +1,456 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+No test here compares the oracle with itself: each checks it against an
+independent statement -- a hand-derived fixture, numpy dense attention over
+contiguous K/V, a closed form, or a paging invariant (the block table changes
+where K/V live, never what attention computes: ipipp.com vLLM article, section
+"二、PagedAttention分页原理深度剖析"; shared prefix blocks with copy-on-write:
+"vLLM 深读", section "先看浪费在哪里").
+"""
+import glob
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+BS = 16
+
+
+# ---------------------------------------------------------------- helpers ----
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def place_blocks(K: np.ndarray, table, num_blocks: int, fill=np.nan) -> np.ndarray:
+    """Put contiguous rows K[L][Hkv][D] into a pool [NB][Hkv][16][D] block by block:
+    logical block i (rows 16i..16i+15) becomes physical block table[i]."""
+    L, hkv, d = K.shape
+    nblk = (L + BS - 1) // BS
+    padded = np.full((nblk * BS, hkv, d), fill, dtype=K.dtype)
+    padded[:L] = K
+    blocks = padded.reshape(nblk, BS, hkv, d).transpose(0, 2, 1, 3)
+    pool = np.full((num_blocks, hkv, BS, d), fill, dtype=K.dtype)
+    for i in range(nblk):
+        pool[table[i]] = blocks[i]
+    return pool
+
+
+def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndarray:
+    """numpy float64 softmax(scale q K^T) V for one sequence.
+    q [Hq][D]; K, V [L][Hkv][D]; query head h reads kv head h // (Hq/Hkv)."""
+    hq = q.shape[0]
+    hkv = K.shape[1]
+    g = hq // hkv
+    out = np.zeros(q.shape, dtype=np.float64)
+    for h in range(hq):
+        Kh = K[:, h // g, :].astype(np.float64)
+        Vh = V[:, h // g, :].astype(np.float64)
+        z = float(np.float32(scale)) * (Kh @ q[h].astype(np.float64))
+        w = np.exp(z - z.max())
+        out[h] = (w[:, None] * Vh).sum(0) / w.sum()
+    return out
+
+
+def random_paged(rng, lens, hq, hkv, d, num_blocks=None, dtype="f32"):
+    """Contiguous per-sequence K/V plus the same data paged into a scattered pool."""
+    nblk = [(L + BS - 1) // BS for L in lens]
+    nb = num_blocks or sum(nblk) + 5
+    perm = rng.permutation(nb)
+    tables, used = [], 0
+    for n in nblk:
+        tables.append(perm[used:used + n].tolist())
+        used += n
+    mb = max(nblk + [1])
+    bt = np.full((len(lens), mb), -1, dtype=np.int32)
+    for s, t in enumerate(tables):
+        bt[s, :len(t)] = t
+    Ks = [rng.standard_normal((L, hkv, d)).astype(np.float32) for L in lens]
+    Vs = [rng.standard_normal((L, hkv, d)).astype(np.float32) for L in lens]
+    q = rng.standard_normal((len(lens), hq, d)).astype(np.float32)
+    kpool = np.full((nb, hkv, BS, d), np.nan, dtype=np.float32)
+    vpool = np.full((nb, hkv, BS, d), np.nan, dtype=np.float32)
+    for s in range(len(lens)):
+        kp = place_blocks(Ks[s], tables[s], nb)
+        vp = place_blocks(Vs[s], tables[s], nb)
+        for b in tables[s]:
+            kpool[b] = kp[b]
+            vpool[b] = vp[b]
+    if dtype == "bf16":
+        Ks = [bf16_bits_to_f64(to_bf16_bits(K)) for K in Ks]
+        Vs = [bf16_bits_to_f64(to_bf16_bits(V)) for V in Vs]
+        return (to_bf16_bits(q), to_bf16_bits(kpool), to_bf16_bits(vpool), bt,
+                np.array(lens, dtype=np.int32), Ks, Vs, bf16_bits_to_f64(to_bf16_bits(q)))
+    return q, kpool, vpool, bt, np.array(lens, dtype=np.int32), Ks, Vs, q
+
+
+# --------------------------------------------------------- golden fixtures ----
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_golden_fixture_files_have_citations():
+    files = sorted(glob.glob(os.path.join(GOLDEN, "*.json")))
+    assert len(files) >= 7
+    for f in files:
+        data = json.load(open(f))
+        assert data.get("citation") and data.get("derivation"), f
+
+
+def test_golden_slot_mapping():
+    g = _golden("slot_mapping_example.json")
+    pos = np.array(g["positions"], dtype=np.int32)
+    seq = np.zeros_like(pos)
+    slots = oracle.slot_mapping(np.array(g["block_tables"], dtype=np.int32), seq, pos,
+                                g["block_size"])
+    assert slots.tolist() == g["expected_slots"]
+
+
+@pytest.mark.parametrize("name", ["attention_two_tokens.json", "attention_uniform_keys.json",
+                                  "attention_gqa_two_heads.json",
+                                  "paged_gather_twenty_tokens.json"])
+def test_golden_attention(name):
+    g = _golden(name)
+    L, d = g["context_len"], g["head_dim"]
+    hq, hkv = g["num_q_heads"], g["num_kv_heads"]
+    if g["k_tokens"] == "j":
+        K = np.arange(L, dtype=np.float32).reshape(L, 1, 1)
+        V = (np.arange(L, dtype=np.float32) + 1).reshape(L, 1, 1)
+    else:
+        K = np.array(g["k_tokens"], dtype=np.float32)
+        V = np.array(g["v_tokens"], dtype=np.float32)
+    kpool = place_blocks(K, g["block_table"], g["num_blocks"])
+    vpool = place_blocks(V, g["block_table"], g["num_blocks"])
+    q = np.array(g["q"], dtype=np.float32).reshape(1, hq, d)
+    out = oracle.paged_decode(q, kpool, vpool, np.array([g["block_table"]], dtype=np.int32),
+                              np.array([L], dtype=np.int32), g["scale"])
+    np.testing.assert_allclose(out[0], np.array(g["expected"]), rtol=0, atol=g["atol"])
+
+
+def test_golden_lse_merge():
+    g = _golden("lse_merge_two_parts.json")
+    out = oracle.lse_merge(np.array(g["m"]), np.array(g["l"]), np.array(g["o"]))
+    np.testing.assert_allclose(out, g["expected"], rtol=0, atol=g["atol"])
+
+
+def test_golden_copy_blocks():
+    g = _golden("copy_blocks_example.json")
+    nb = g["num_blocks"]
+    base = (100.0 * np.arange(nb)).reshape(nb, 1, 1, 1)
+    k = (base + np.arange(BS).reshape(1, 1, BS, 1)).astype(np.float32)
+    v = -k
+    oracle.copy_blocks(k, v, np.array(g["pairs"]))
+    for b, b0 in enumerate(g["expected_block_base"]):
+        assert np.array_equal(k[b, 0, :, 0], b0 + np.arange(BS, dtype=np.float32))
+        assert np.array_equal(v[b, 0, :, 0], -(b0 + np.arange(BS, dtype=np.float32)))
+
+
+# ------------------------------------------------------- dense reduction ----
+@pytest.mark.parametrize("d", [4, 8, 64])
+@pytest.mark.parametrize("hq,hkv", [(1, 1), (4, 1), (8, 2), (6, 3)])
+def test_dense_reduction_fp32(d, hq, hkv):
+    rng = np.random.default_rng(1000 * d + 10 * hq + hkv)
+    lens = [1, 15, 16, 17, 33, 64]
+    q, kp, vp, bt, cl, Ks, Vs, qf = random_paged(rng, lens, hq, hkv, d)
+    scale = 1.0 / math.sqrt(d)
+    out = oracle.paged_decode(q, kp, vp, bt, cl, scale)
+    for s in range(len(lens)):
+        ref = dense_attention(qf[s], Ks[s], Vs[s], scale)
+        np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
+
+
+def test_dense_reduction_bf16():
+    rng = np.random.default_rng(7)
+    lens = [3, 16, 40, 64]
+    q, kp, vp, bt, cl, Ks, Vs, qf = random_paged(rng, lens, 8, 2, 64, dtype="bf16")
+    out = oracle.paged_decode(q, kp, vp, bt, cl, 0.125)
+    for s in range(len(lens)):
+        ref = dense_attention(qf[s], Ks[s], Vs[s], 0.125)
+        np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
+
+
+def test_dense_reduction_c1_config():
+    """The tiny fp32 configuration against numpy dense attention over the contiguous K/V
+    read back block by block from the generator's pool."""
+    b = workloads.c1_tiny_fp32()
+    h = b.host()
+    out = oracle.paged_decode(h["q"], h["k_cache"], h["v_cache"], b.block_tables,
+                              b.context_lens, b.scale)
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        nblk = (L + BS - 1) // BS
+        blocks = h["k_cache"][b.block_tables[s, :nblk]]          # [nblk][Hkv][16][D]
+        K = blocks.transpose(0, 2, 1, 3).reshape(nblk * BS, b.num_kv_heads, b.head_dim)[:L]
+        blocks = h["v_cache"][b.block_tables[s, :nblk]]
+        V = blocks.transpose(0, 2, 1, 3).reshape(nblk * BS, b.num_kv_heads, b.head_dim)[:L]
+        assert np.isfinite(K).all() and np.isfinite(V).all()
+        ref = dense_attention(h["q"][s], K, V, b.scale)
+        np.testing.assert_allclose(out[s], ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ closed forms ----
+def test_single_token_returns_its_value_exactly():
+    rng = np.random.default_rng(3)
+    q, kp, vp, bt, cl, Ks, Vs, _ = random_paged(rng, [1, 1], 4, 2, 64)
+    out = oracle.paged_decode(q, kp, vp, bt, cl, 0.125)
+    for s in range(2):
+        for h in range(4):
+            assert np.array_equal(out[s, h], Vs[s][0, h // 2].astype(np.float64))
+
+
+def test_zero_scale_gives_mean_of_values():
+    rng = np.random.default_rng(4)
+    lens = [5, 31, 48]
+    q, kp, vp, bt, cl, Ks, Vs, _ = random_paged(rng, lens, 2, 2, 8)
+    out = oracle.paged_decode(q, kp, vp, bt, cl, 0.0)
+    for s, L in enumerate(lens):
+        np.testing.assert_allclose(out[s], Vs[s].astype(np.float64).mean(0), rtol=0, atol=1e-12)
+
+
+def test_equal_keys_give_mean_of_values():
+    rng = np.random.default_rng(5)
+    L, d = 37, 8
+    K = np.repeat(rng.standard_normal((1, 1, d)).astype(np.float32), L, axis=0)
+    V = rng.standard_normal((L, 1, d)).astype(np.float32)
+    table = [4, 0, 2]
+    q = rng.standard_normal((1, 1, d)).astype(np.float32)
+    out = oracle.paged_decode(q, place_blocks(K, table, 5), place_blocks(V, table, 5),
+                              np.array([table], dtype=np.int32), np.array([L], dtype=np.int32),
+                              0.7)
+    np.testing.assert_allclose(out[0, 0], V[:, 0].astype(np.float64).mean(0), rtol=0, atol=1e-12)
+
+
+def test_dominant_key_selects_its_value():
+    rng = np.random.default_rng(6)
+    L, d, j_star = 45, 16, 29
+    K = rng.standard_normal((L, 1, d)).astype(np.float32)
+    q = rng.standard_normal((1, 1, d)).astype(np.float32)
+    K[j_star, 0] = 64.0 * q[0, 0]            # its score exceeds all others by far more than 60
+    V = rng.standard_normal((L, 1, d)).astype(np.float32)
+    table = [2, 0, 1]
+    scale = 1.0
+    z = (K[:, 0].astype(np.float64) @ q[0, 0].astype(np.float64)) * scale
+    assert z[j_star] - np.delete(z, j_star).max() > 60
+    out = oracle.paged_decode(q, place_blocks(K, table, 3), place_blocks(V, table, 3),
+                              np.array([table], dtype=np.int32), np.array([L], dtype=np.int32),
+                              scale)
+    np.testing.assert_allclose(out[0, 0], V[j_star, 0].astype(np.float64), rtol=0, atol=1e-12)
+
+
+def test_empty_context_gives_zero():
+    rng = np.random.default_rng(8)
+    q, kp, vp, bt, cl, _, _, _ = random_paged(rng, [0, 20], 2, 1, 8)
+    out = oracle.paged_decode(q, kp, vp, bt, cl, 0.3)
+    assert np.array_equal(out[0], np.zeros((2, 8)))
+    assert np.isfinite(out[1]).all()
+
+
+# --------------------------------------------------------------- GQA ----
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    rng = np.random.default_rng(9)
+    lens = [7, 40, 65]
+    q, kp, vp, bt, cl, _, _, _ = random_paged(rng, lens, 8, 2, 16)
+    gqa = oracle.paged_decode(q, kp, vp, bt, cl, 0.25)
+    kp_mha = np.repeat(kp, 4, axis=1)     # kv head k serves query heads 4k..4k+3
+    vp_mha = np.repeat(vp, 4, axis=1)
+    mha = oracle.paged_decode(q, np.ascontiguousarray(kp_mha), np.ascontiguousarray(vp_mha),
+                              bt, cl, 0.25)
+    assert np.array_equal(gqa, mha)
+
+
+def test_gqa_head_mapping_is_not_interleaved():
+    """Query heads 0..g-1 read kv head 0 (a reading; an interleaved h % Hkv mapping would fail)."""
+    rng = np.random.default_rng(10)
+    q, kp, vp, bt, cl, Ks, Vs, qf = random_paged(rng, [1], 4, 2, 8)
+    out = oracle.paged_decode(q, kp, vp, bt, cl, 1.0)
+    assert np.array_equal(out[0, 1], Vs[0][0, 0].astype(np.float64))
+    assert np.array_equal(out[0, 2], Vs[0][0, 1].astype(np.float64))
+
+
+# ------------------------------------------------------- paging invariants ----
+def test_block_placement_permutation_is_bitwise_invariant():
+    b = workloads.random_batch(11, [3, 16, 17, 100, 250], 8, 2, 32, "bf16", device="cpu")
+    p = workloads.permute_placement(b, seed=12)
+    assert not np.array_equal(b.block_tables, p.block_tables)
+    hb, hp = b.host(), p.host()
+    ob = oracle.paged_decode(hb["q"], hb["k_cache"], hb["v_cache"], b.block_tables,
+                             b.context_lens, b.scale)
+    op = oracle.paged_decode(hp["q"], hp["k_cache"], hp["v_cache"], p.block_tables,
+                             p.context_lens, p.scale)
+    assert np.array_equal(ob, op)
+
+
+def _apply_step_oracle(b: workloads.Batch):
+    """Copy-on-write copies, then the new tokens' writes, on host copies of the pool."""
+    h = b.host()
+    k, v = h["k_cache"].copy(), h["v_cache"].copy()
+    oracle.copy_blocks(k, v, b.cow_pairs)
+    slots = oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos)
+    oracle.reshape_and_cache(h["new_k"], h["new_v"], k, v, slots)
+    return h, k, v
+
+
+def test_shared_prefix_equals_private_copies():
+    b = workloads.c4_shared_prefix(prompts=3, samples=4, prefix=64, max_tail=40, num_blocks=200)
+    assert b.cow_pairs.shape[0] > 0
+    h, k, v = _apply_step_oracle(b)
+    shared = oracle.paged_decode(h["q"], k, v, b.block_tables, b.context_lens, b.scale)
+    assert np.isfinite(shared).all()
+    after = workloads.Batch(b.name, b.seed, b.dtype, b.num_q_heads, b.num_kv_heads, b.head_dim,
+                            b.num_blocks, b.context_lens, b.block_tables, b.scale, b.q,
+                            torch.from_numpy(k.view(np.int16)).view(torch.bfloat16),
+                            torch.from_numpy(v.view(np.int16)).view(torch.bfloat16),
+                            b.new_k, b.new_v, b.new_seq, b.new_pos, b.cow_pairs)
+    priv = workloads.private_copy(after)
+    assert priv.num_blocks > b.num_blocks          # some blocks really were shared
+    hp = priv.host()
+    private = oracle.paged_decode(hp["q"], hp["k_cache"], hp["v_cache"], priv.block_tables,
+                                  priv.context_lens, priv.scale)
+    assert np.array_equal(shared, private)
+
+
+def test_padding_is_never_read():
+    """NaN in every slot past the context, in unreferenced blocks and -1 table padding:
+    the result is finite and equal to the run with finite values there."""
+    b = workloads.random_batch(13, [1, 15, 17, 47, 64], 4, 2, 16, "f32", device="cpu",
+                               extra_table=3)
+    h = b.host()
+    assert np.isnan(h["k_cache"]).any()
+    poisoned = oracle.paged_decode(h["q"], h["k_cache"], h["v_cache"], b.block_tables,
+                                   b.context_lens, b.scale)
+    assert np.isfinite(poisoned).all()
+    k = np.where(np.isnan(h["k_cache"]), np.float32(3.0), h["k_cache"])
+    v = np.where(np.isnan(h["v_cache"]), np.float32(-7.0), h["v_cache"])
+    bt = np.where(b.block_tables < 0, 0, b.block_tables).astype(np.int32)
+    clean = oracle.paged_decode(h["q"], k, v, bt, b.context_lens, b.scale)
+    assert np.array_equal(poisoned, clean)
+
+
+# --------------------------------------------------- partition and merge ----
+@pytest.mark.parametrize("part", [16, 48, 512, None])
+def test_partition_merge_equals_single_pass(part):
+    rng = np.random.default_rng(14)
+    lens = [1, 16, 47, 600, 1100]
+    q, kp, vp, bt, cl, _, _, _ = random_paged(rng, lens, 4, 2, 8)
+    full = oracle.paged_decode(q, kp, vp, bt, cl, 0.3)
+    for s, L in enumerate(lens):
+        P = part or L
+        for h in range(4):
+            ms, ls, os_ = [], [], []
+            for t0 in range(0, max(L, 1), P):
+                m, l, o = oracle.partition_stats(q, kp, vp, bt, cl, 0.3, s, h, t0, min(L, t0 + P))
+                ms.append(m)
+                ls.append(l)
+                os_.append(o)
+            merged = oracle.lse_merge(np.array(ms), np.array(ls), np.array(os_))
+            np.testing.assert_allclose(merged, full[s, h], rtol=0, atol=1e-12)
+
+
+def test_merge_ignores_empty_parts():
+    m = np.array([-np.inf, 0.5, -np.inf])
+    l = np.array([0.0, 2.0, 0.0])
+    o = np.array([[np.nan, np.nan], [1.0, -2.0], [0.0, 0.0]])
+    assert np.array_equal(oracle.lse_merge(m, l, o), np.array([1.0, -2.0]))
+    assert np.array_equal(oracle.lse_merge(m[[0]], l[[0]], o[[0]]), np.zeros(2))
+
+
+# ------------------------------------------------- reshape_and_cache, slots ----
+def test_reshape_then_decode_equals_dense():
+    """Write a whole context token by token through slot_mapping + reshape_and_cache into a
+    NaN pool, then decode: the result is dense attention over the tokens written."""
+    rng = np.random.default_rng(15)
+    lens = [5, 16, 33]
+    hq, hkv, d = 4, 2, 8
+    nb = 12
+    perm = rng.permutation(nb)
+    tables, used = [], 0
+    for L in lens:
+        n = (L + BS - 1) // BS
+        tables.append(perm[used:used + n].tolist())
+        used += n
+    bt = np.full((len(lens), 3), -1, dtype=np.int32)
+    for s, t in enumerate(tables):
+        bt[s, :len(t)] = t
+    kpool = np.full((nb, hkv, BS, d), np.nan, dtype=np.float32)
+    vpool = np.full((nb, hkv, BS, d), np.nan, dtype=np.float32)
+    seq = np.concatenate([np.full(L, s) for s, L in enumerate(lens)]).astype(np.int32)
+    pos = np.concatenate([np.arange(L) for L in lens]).astype(np.int32)
+    order = rng.permutation(seq.shape[0])           # write order does not matter
+    seq, pos = seq[order], pos[order]
+    knew = rng.standard_normal((seq.shape[0], hkv, d)).astype(np.float32)
+    vnew = rng.standard_normal((seq.shape[0], hkv, d)).astype(np.float32)
+    slots = oracle.slot_mapping(bt, seq, pos)
+    assert len(set(slots.tolist())) == len(slots)
+    oracle.reshape_and_cache(knew, vnew, kpool, vpool, slots)
+    q = rng.standard_normal((len(lens), hq, d)).astype(np.float32)
+    cl = np.array(lens, dtype=np.int32)
+    out = oracle.paged_decode(q, kpool, vpool, bt, cl, 0.4)
+    for s, L in enumerate(lens):
+        K = np.zeros((L, hkv, d), dtype=np.float32)
+        V = np.zeros((L, hkv, d), dtype=np.float32)
+        for t in np.nonzero(seq == s)[0]:
+            K[pos[t]] = knew[t]
+            V[pos[t]] = vnew[t]
+        np.testing.assert_allclose(out[s], dense_attention(q[s], K, V, 0.4), rtol=0, atol=1e-12)
+    # exactly the written rows changed: T tokens x Hkv heads rows of D values
+    assert np.isfinite(kpool).all(axis=-1).sum() == seq.shape[0] * hkv
+
+
+def test_reshape_skips_negative_slots_and_rejects_out_of_range():
+    k = np.ones((2, 1, 4), dtype=np.float32)
+    kc = np.zeros((2, 1, BS, 4), dtype=np.float32)
+    vc = np.zeros_like(kc)
+    oracle.reshape_and_cache(k, k, kc, vc, np.array([-1, 17]))
+    assert kc[1, 0, 1].tolist() == [1, 1, 1, 1] and kc.sum() == 4
+    with pytest.raises(oracle.OracleError):
+        oracle.reshape_and_cache(k, k, kc, vc, np.array([0, 32]))
+
+
+def test_copy_blocks_snapshot_semantics():
+    nb = 3
+    k = np.arange(nb * BS * 2, dtype=np.float32).reshape(nb, 1, BS, 2)
+    v = k + 0.5
+    k0, v0 = k.copy(), v.copy()
+    oracle.copy_blocks(k, v, np.array([[0, 1], [1, 2]]))   # a chain: reads happen first
+    assert np.array_equal(k[1], k0[0]) and np.array_equal(k[2], k0[1])
+    assert np.array_equal(v[1], v0[0]) and np.array_equal(v[2], v0[1])
+    assert np.array_equal(k[0], k0[0])
+    with pytest.raises(oracle.OracleError):
+        oracle.copy_blocks(k, v, np.array([[0, 3]]))
+
+
+def test_bad_table_entry_and_length_are_errors():
+    rng = np.random.default_rng(16)
+    q, kp, vp, bt, cl, _, _, _ = random_paged(rng, [20], 1, 1, 4)
+    bad = bt.copy()
+    bad[0, 1] = kp.shape[0]
+    with pytest.raises(oracle.OracleError):
+        oracle.paged_decode(q, kp, vp, bad, cl, 1.0)
+    with pytest.raises(oracle.OracleError):
+        oracle.paged_decode(q, kp, vp, bt, np.array([33], dtype=np.int32), 1.0)
+
+
+# -------------------------------------------------------- tolerance sanity ----
+def test_bf16_rounding_of_exact_output_meets_the_tolerance():
+    """The bf16 tolerance (|e| <= 2e-2 + 1e-2 |ref|) is attainable: rounding the exact
+    output to bf16 alone stays far inside it."""
+    b = workloads.random_batch(17, [100, 1000, 2000], 32, 8, 128, "bf16", device="cpu")
+    h = b.host()
+    ref = oracle.paged_decode(h["q"], h["k_cache"], h["v_cache"], b.block_tables,
+                              b.context_lens, b.scale)
+    rounded = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+    err = np.abs(rounded - ref)
+    assert (err <= 2e-2 + 1e-2 * np.abs(ref)).all()
+    assert err.max() <= 2.0 ** -8 * np.abs(ref).max()
