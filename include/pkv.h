@@ -1,0 +1,210 @@
+/*
+ * pkv.h -- C ABI of the B200 (sm_100a) paged KV-cache decode library.
+ *
+ * The operations are those of PagedAttention decode as the pages state the
+ * problem:
+ *  - the KV cache is cut into fixed-size blocks of 16 tokens; a per-sequence
+ *    block table maps each logical block to a physical block of one shared
+ *    pool, and attention visits the sequence block by block, looking up each
+ *    block and loading it (ipipp.com vLLM article, section
+ *    "二、PagedAttention分页原理深度剖析");
+ *  - new tokens reach their physical slot through slot_mapping ("vLLM" wiki
+ *    entry, wiki.bytelighting.cn, section "Flattened 布局与 slot_mapping");
+ *  - blocks shared by several sequences are reference counted and copied on
+ *    write ("vLLM 深读：用 PagedAttention 撑起高并发 LLM 推理", section
+ *    "先看浪费在哪里").
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless the argument says "host".  The caller
+ *    owns every buffer; the library never allocates device memory.  Scratch
+ *    memory (the decode workspace) is passed in by the caller.
+ *  - Every call is asynchronous on `cuda_stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  A returned PKV_OK means the work was validated
+ *    and enqueued, not that it has finished.
+ *  - The return value reports what the host can see: bad arguments, an
+ *    unsupported shape, a workspace that is too small, a failed launch.
+ *  - Indices the host cannot see (block-table entries, slots, copy pairs,
+ *    context lengths, all in device memory) are checked by the kernels.  An
+ *    invalid one is skipped -- never dereferenced -- and a bit is set in a
+ *    per-device error word; pkv_check_device_error() reads and clears it.  No
+ *    kernel traps, asserts or waits without a bound: every internal wait gives
+ *    up after about four seconds and reports PKV_DEVERR_TIMEOUT.
+ *  - All device pointers must be 16-byte aligned.
+ *
+ * Layouts (row-major, innermost last):
+ *  - q, out         [num_seqs][num_q_heads][head_dim], dtype of the cache
+ *  - k, v (new)     [num_tokens][num_kv_heads][head_dim]
+ *  - k_cache,v_cache[num_blocks][num_kv_heads][16][head_dim]  ("HND": one
+ *                   (block, kv head) tile of 16 tokens is contiguous)
+ *  - block_tables   int32 [num_seqs][max_blocks_per_seq]; entries at or past
+ *                   ceil(context_len/16) are never read
+ *  - context_lens   int32 [num_seqs]; the length includes the token being
+ *                   decoded; 0 is allowed and gives a zero output
+ *  - slot_mapping   int64 [num_tokens]; slot = block*16 + offset; negative
+ *                   slots mark padding tokens and are skipped
+ *  - pairs          int64 [num_pairs][2] = (src block, dst block)
+ *  - query head h reads kv head h / (num_q_heads / num_kv_heads).
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_NULL = 1,          /* a required pointer is NULL */
+    PKV_ERR_SHAPE = 2,         /* inconsistent sizes (e.g. Hq % Hkv != 0, negative counts) */
+    PKV_ERR_UNSUPPORTED = 3,   /* block_size != 16, head_dim not 64/128, group > 16, dtype */
+    PKV_ERR_WORKSPACE = 4,     /* workspace NULL, misaligned or smaller than required */
+    PKV_ERR_PAIRS = 5,         /* copy pairs: out of range, repeated dst, or dst also a src */
+    PKV_ERR_CUDA = 6,          /* a CUDA runtime call or a launch failed */
+    PKV_ERR_DEVICE_INDEX = 7,  /* a kernel met an invalid index (see the error bits) */
+    PKV_ERR_ALIGN = 8,         /* a pointer is not 16-byte aligned */
+    PKV_ERR_DEVICE_TIMEOUT = 9 /* a kernel's bounded wait expired */
+} pkv_status;
+
+typedef enum pkv_dtype {
+    PKV_F32 = 0,   /* IEEE binary32 */
+    PKV_BF16 = 1   /* bfloat16; arithmetic in fp32, output rounded to nearest even */
+} pkv_dtype;
+
+/* Bits of the per-device error word. */
+#define PKV_DEVERR_BLOCK   0x1u   /* block-table entry outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT    0x2u   /* slot beyond num_blocks*16 */
+#define PKV_DEVERR_LEN     0x4u   /* context length < 0 or > max_blocks_per_seq*16 or > max_context_len */
+#define PKV_DEVERR_PAIR    0x8u   /* copy pair outside [0, num_blocks) */
+#define PKV_DEVERR_POS     0x10u  /* slot-mapping position outside the block table */
+#define PKV_DEVERR_TIMEOUT 0x20u  /* a bounded wait gave up */
+
+typedef struct pkv_dims {
+    int32_t num_seqs;            /* B */
+    int32_t num_q_heads;         /* Hq */
+    int32_t num_kv_heads;        /* Hkv; Hq % Hkv == 0, Hq/Hkv <= 16 */
+    int32_t head_dim;            /* D: 64 or 128 */
+    int32_t block_size;          /* must be 16 */
+    int32_t num_blocks;          /* NB, physical blocks in each of the K and V pools */
+    int32_t max_blocks_per_seq;  /* MB, width of block_tables */
+    pkv_dtype dtype;             /* of q, out, k, v and both caches */
+} pkv_dims;
+
+/*
+ * Partition size the decode will use for `partition_tokens` (0 = automatic):
+ * a multiple of 16.  A sequence longer than the partition is split into
+ * partitions computed independently and merged by log-sum-exp.  When the
+ * result is >= max_context_len the decode runs single-pass.
+ * Returns 0 for invalid dims.
+ */
+int32_t pkv_decode_partition_tokens(const pkv_dims *dims, int32_t max_context_len,
+                                    int32_t partition_tokens);
+
+/*
+ * Bytes of device workspace pkv_paged_attention_decode needs for these
+ * arguments (work list, scheduling counters and, when sequences are split,
+ * the per-partition partial results).  Returns 0 for invalid dims.
+ */
+size_t pkv_decode_workspace_bytes(const pkv_dims *dims, int32_t max_context_len,
+                                  int32_t partition_tokens);
+
+/*
+ * Offsets inside the workspace of the split-K partial results, for tests that
+ * inspect them: part_o is float [B][Hq][max_parts][D] (each partition's
+ * normalised output), part_ml is float [B][Hq][max_parts][2] = (m, l) with m
+ * the partition's max of scale*q.k and l = sum exp(scale*q.k - m).  Only
+ * partitions of sequences with more than one partition are written.
+ * Returns PKV_ERR_SHAPE when the decode would run single-pass.
+ */
+pkv_status pkv_decode_workspace_layout(const pkv_dims *dims, int32_t max_context_len,
+                                       int32_t partition_tokens, int32_t *max_parts,
+                                       size_t *part_o_offset, size_t *part_ml_offset);
+
+/*
+ * Paged decode attention: for each sequence s and query head h,
+ *   out[s][h] = softmax_j(scale * q[s][h] . K_j) V_j   over j < context_lens[s],
+ * with K_j, V_j read from physical block block_tables[s][j/16], slot j%16,
+ * kv head h/(Hq/Hkv).  One query token per sequence.
+ *
+ * max_context_len (host) must be >= every context length; it sizes the
+ * partitions and the workspace (a larger value is always safe; a length above
+ * it is clamped and flagged PKV_DEVERR_LEN).  partition_tokens: 0 = automatic,
+ * else a multiple of 16 (e.g. 512).  workspace: device scratch of at least
+ * pkv_decode_workspace_bytes() bytes, 256-byte aligned, not shared with a
+ * decode that may run concurrently.  Launches a planning kernel, the decode
+ * kernel and, when some sequence is split, the merge kernel, in that order.
+ */
+pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_tables,
+                                      const int32_t *context_lens, float scale,
+                                      const pkv_dims *dims, int32_t max_context_len,
+                                      int32_t partition_tokens, void *workspace,
+                                      size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * reshape_and_cache: for every token t with slot_mapping[t] >= 0, copy the
+ * bytes of k[t][h][:] and v[t][h][:] to k_cache / v_cache at block
+ * slot/16, kv head h, offset slot%16, for every kv head h.  The copy is
+ * bit-exact (no conversion).  Negative slots are skipped; a slot >=
+ * num_blocks*16 is skipped and flagged PKV_DEVERR_SLOT.  Two tokens with the
+ * same non-negative slot in one call leave that slot unspecified.
+ * dims->num_seqs and dims->max_blocks_per_seq are not used.
+ */
+pkv_status pkv_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache,
+                                 const int64_t *slot_mapping, int32_t num_tokens,
+                                 const pkv_dims *dims, void *cuda_stream);
+
+/*
+ * copy_blocks (copy-on-write): for each pair (src, dst) copy every byte of K
+ * block src to K block dst and of V block src to V block dst (all kv heads,
+ * all 16 slots).  Pairs are applied as if every source were read before any
+ * destination is written; that is only guaranteed when no destination repeats
+ * and no destination is also a source, which pkv_validate_copy_pairs() checks
+ * on a host copy.  A pair outside [0, num_blocks) is skipped and flagged
+ * PKV_DEVERR_PAIR.  dims->num_seqs and dims->max_blocks_per_seq are not used.
+ */
+pkv_status pkv_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs,
+                           int32_t num_pairs, const pkv_dims *dims, void *cuda_stream);
+
+/*
+ * Host-side check of copy pairs (pairs_host is a HOST pointer): every index in
+ * [0, num_blocks), no repeated destination, no destination that is also a
+ * source.  Returns PKV_OK or PKV_ERR_PAIRS.
+ */
+pkv_status pkv_validate_copy_pairs(const int64_t *pairs_host, int32_t num_pairs,
+                                   int32_t num_blocks);
+
+/*
+ * Slot indexing: slot_mapping[t] = block_tables[seq][pos/16]*16 + pos%16 with
+ * seq = token_seq[t] (or t when token_seq is NULL) and pos = token_pos[t] (or
+ * context_lens[seq]-1 when token_pos is NULL: the decode token).  A position
+ * outside the table or a table entry outside [0, num_blocks) gives slot -1
+ * and sets PKV_DEVERR_POS / PKV_DEVERR_BLOCK.  context_lens may be NULL when
+ * token_pos is given.
+ */
+pkv_status pkv_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
+                            const int32_t *context_lens, const int32_t *token_seq,
+                            const int32_t *token_pos, int32_t num_tokens,
+                            const pkv_dims *dims, void *cuda_stream);
+
+/*
+ * Synchronises cuda_stream, then reads and clears the error word of the
+ * current device.  *bits_out (may be NULL) receives the PKV_DEVERR_* bits.
+ * Returns PKV_OK, PKV_ERR_DEVICE_TIMEOUT (timeout bit set),
+ * PKV_ERR_DEVICE_INDEX (other bits) or PKV_ERR_CUDA.
+ */
+pkv_status pkv_check_device_error(void *cuda_stream, uint32_t *bits_out);
+
+/* Static text for a status code. */
+const char *pkv_status_string(pkv_status status);
+
+/* Details of the last non-OK status returned on the calling host thread. */
+const char *pkv_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

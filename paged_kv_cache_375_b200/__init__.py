@@ -1,0 +1,302 @@
+"""Paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI of ``libpkv.so`` (declared in
+``include/pkv.h``).  It only marshals arguments -- shapes, pointers, the
+current CUDA stream and a cached workspace -- every step runs in the library's
+CUDA kernels.  There is no CPU fallback: if the library is missing, importing
+the operations raises.
+
+Operations (the pages' statement of the problem: 16-token blocks, a
+per-sequence block table, slot_mapping, copy-on-write of shared blocks):
+
+  paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens,
+                         scale, num_kv_heads, ...)
+  reshape_and_cache(k, v, k_cache, v_cache, slot_mapping)
+  copy_blocks(k_cache, v_cache, pairs)
+  slot_mapping(block_tables, context_lens=None, token_seq=None, token_pos=None)
+  check_device_error()
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpkv.so")
+
+PKV_F32, PKV_BF16 = 0, 1
+DEVERR_BLOCK, DEVERR_SLOT, DEVERR_LEN, DEVERR_PAIR, DEVERR_POS, DEVERR_TIMEOUT = (
+    0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
+
+STATUS_NAMES = {0: "PKV_OK", 1: "PKV_ERR_NULL", 2: "PKV_ERR_SHAPE", 3: "PKV_ERR_UNSUPPORTED",
+                4: "PKV_ERR_WORKSPACE", 5: "PKV_ERR_PAIRS", 6: "PKV_ERR_CUDA",
+                7: "PKV_ERR_DEVICE_INDEX", 8: "PKV_ERR_ALIGN", 9: "PKV_ERR_DEVICE_TIMEOUT"}
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class PkvDims(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libpkv.so (built in-tree by ``paged_kv_cache_375_b200.build``)."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m paged_kv_cache_375_b200.build` (no CPU fallback exists)")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+        D = ctypes.POINTER(PkvDims)
+        sig = {
+            "pkv_decode_partition_tokens": (i32, [D, i32, i32]),
+            "pkv_decode_workspace_bytes": (sz, [D, i32, i32]),
+            "pkv_decode_workspace_layout": (ctypes.c_int, [D, i32, i32, P, P, P]),
+            "pkv_paged_attention_decode": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P,
+                                                          sz, P]),
+            "pkv_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
+            "pkv_copy_blocks": (ctypes.c_int, [P, P, P, i32, D, P]),
+            "pkv_validate_copy_pairs": (ctypes.c_int, [P, i32, i32]),
+            "pkv_slot_mapping": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
+            "pkv_check_device_error": (ctypes.c_int, [P, P]),
+            "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "pkv_last_error_message": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _check(status: int):
+    if status != 0:
+        lib = load_library()
+        raise PkvError(status, lib.pkv_last_error_message().decode())
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return PKV_BF16
+    if t == torch.float32:
+        return PKV_F32
+    raise TypeError(f"dtype {t} not supported (bfloat16 or float32)")
+
+
+def _stream_ptr(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _p(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def make_dims(num_seqs: int, num_q_heads: int, k_cache: torch.Tensor,
+              max_blocks_per_seq: int) -> PkvDims:
+    nb, hkv, bs, d = k_cache.shape
+    return PkvDims(num_seqs, num_q_heads, hkv, d, bs, nb, max_blocks_per_seq,
+                   _dtype_code(k_cache.dtype))
+
+
+def decode_partition_tokens(dims: PkvDims, max_context_len: int, partition_tokens: int = 0) -> int:
+    return load_library().pkv_decode_partition_tokens(ctypes.byref(dims), max_context_len,
+                                                      partition_tokens)
+
+
+def decode_workspace_bytes(dims: PkvDims, max_context_len: int, partition_tokens: int = 0) -> int:
+    return load_library().pkv_decode_workspace_bytes(ctypes.byref(dims), max_context_len,
+                                                     partition_tokens)
+
+
+def decode_workspace_layout(dims: PkvDims, max_context_len: int, partition_tokens: int = 0):
+    """(max_parts, part_o_offset, part_ml_offset) of the split-K partials in the workspace."""
+    mp = ctypes.c_int32()
+    po = ctypes.c_size_t()
+    pm = ctypes.c_size_t()
+    _check(load_library().pkv_decode_workspace_layout(
+        ctypes.byref(dims), max_context_len, partition_tokens, ctypes.byref(mp),
+        ctypes.byref(po), ctypes.byref(pm)))
+    return mp.value, po.value, pm.value
+
+
+_ws_cache: dict = {}
+
+
+def workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    """A cached uint8 workspace of at least nbytes for (device, current stream).
+
+    Decodes issued on one stream run in order, so they can share it; another
+    stream gets its own.
+    """
+    key = (device, torch.cuda.current_stream(device).cuda_stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                           v_cache: torch.Tensor, block_tables: torch.Tensor,
+                           context_lens: torch.Tensor, scale: float, num_kv_heads: int, *,
+                           max_context_len: int | None = None, partition_tokens: int = 0,
+                           workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
+    """out[s][h] = softmax(scale * q[s][h] . K^T) V over the paged context of sequence s.
+
+    q, out: [B][Hq][D]; k_cache, v_cache: [NB][Hkv][16][D]; block_tables: int32 [B][MB];
+    context_lens: int32 [B].  max_context_len defaults to MB*16 (always safe; a tighter
+    value gives a smaller workspace and better partitioning).
+    """
+    dev = q.device
+    _need(q, "q", device=dev)
+    _need(out, "out", q.dtype, dev)
+    _need(k_cache, "k_cache", q.dtype, dev)
+    _need(v_cache, "v_cache", q.dtype, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must both be [num_blocks][num_kv_heads][16][head_dim]")
+    if k_cache.shape[1] != num_kv_heads:
+        raise ValueError(f"k_cache has {k_cache.shape[1]} kv heads, num_kv_heads={num_kv_heads}")
+    B, hq, d = q.shape
+    if out.shape != q.shape or block_tables.dim() != 2 or block_tables.shape[0] != B \
+            or context_lens.shape != (B,) or k_cache.shape[3] != d:
+        raise ValueError("inconsistent shapes")
+    dims = make_dims(B, hq, k_cache, block_tables.shape[1])
+    mcl = block_tables.shape[1] * k_cache.shape[2] if max_context_len is None else int(max_context_len)
+    need = decode_workspace_bytes(dims, mcl, partition_tokens)
+    if need == 0:
+        raise PkvError(2, load_library().pkv_last_error_message().decode())
+    ws = workspace_tensor if workspace_tensor is not None else workspace(dev, need)
+    _check(load_library().pkv_paged_attention_decode(
+        _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+        float(scale), ctypes.byref(dims), mcl, partition_tokens, _p(ws), ws.numel(),
+        _stream_ptr(dev)))
+    return out
+
+
+def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, slot_mapping: torch.Tensor) -> None:
+    """Write k, v ([T][Hkv][D]) into the caches at slot_mapping (int64 [T]); -1 skips."""
+    dev = k.device
+    _need(k, "k", k_cache.dtype, dev)
+    _need(v, "v", k_cache.dtype, dev)
+    _need(k_cache, "k_cache", device=dev)
+    _need(v_cache, "v_cache", k_cache.dtype, dev)
+    _need(slot_mapping, "slot_mapping", torch.int64, dev)
+    T = slot_mapping.shape[0]
+    if k.shape != v.shape or k.shape[0] != T or k.shape[1:] != (k_cache.shape[1], k_cache.shape[3]):
+        raise ValueError("k, v must be [num_tokens][num_kv_heads][head_dim]")
+    dims = make_dims(0, k_cache.shape[1], k_cache, 1)
+    _check(load_library().pkv_reshape_and_cache(_p(k), _p(v), _p(k_cache), _p(v_cache),
+                                                _p(slot_mapping), T, ctypes.byref(dims),
+                                                _stream_ptr(dev)))
+
+
+def validate_copy_pairs(pairs_host: torch.Tensor, num_blocks: int) -> None:
+    pr = pairs_host.detach().to("cpu", torch.int64).contiguous().reshape(-1, 2)
+    _check(load_library().pkv_validate_copy_pairs(ctypes.c_void_p(pr.data_ptr()), pr.shape[0],
+                                                  num_blocks))
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tensor,
+                validate: bool = True) -> None:
+    """Copy-on-write: copy K and V block src to dst for each (src, dst) row of pairs.
+
+    pairs may live on the CPU (it is validated there, then copied to the device) or on the
+    device (validated only when ``validate`` and after a device-to-host copy).
+    """
+    dev = k_cache.device
+    _need(k_cache, "k_cache", device=dev)
+    _need(v_cache, "v_cache", k_cache.dtype, dev)
+    pr = pairs.reshape(-1, 2)
+    if pr.shape[0] == 0:
+        return
+    if validate:
+        validate_copy_pairs(pr, k_cache.shape[0])
+    pr_dev = pr.to(dev, torch.int64).contiguous()
+    dims = make_dims(0, k_cache.shape[1], k_cache, 1)
+    _check(load_library().pkv_copy_blocks(_p(k_cache), _p(v_cache), _p(pr_dev), pr_dev.shape[0],
+                                          ctypes.byref(dims), _stream_ptr(dev)))
+
+
+def slot_mapping(block_tables: torch.Tensor, num_blocks: int, *,
+                 context_lens: torch.Tensor | None = None, token_seq: torch.Tensor | None = None,
+                 token_pos: torch.Tensor | None = None, num_tokens: int | None = None,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """Slots of tokens: block_tables[seq][pos // 16] * 16 + pos % 16, computed on the GPU.
+
+    Without token_pos the position is context_lens[seq] - 1 (the decode token); without
+    token_seq token t belongs to sequence t.
+    """
+    dev = block_tables.device
+    _need(block_tables, "block_tables", torch.int32, dev)
+    for name, t in (("context_lens", context_lens), ("token_seq", token_seq),
+                    ("token_pos", token_pos)):
+        if t is not None:
+            _need(t, name, torch.int32, dev)
+    B = block_tables.shape[0]
+    if num_tokens is None:
+        num_tokens = token_pos.shape[0] if token_pos is not None else (
+            token_seq.shape[0] if token_seq is not None else B)
+    if out is None:
+        out = torch.empty(num_tokens, dtype=torch.int64, device=dev)
+    dims = PkvDims(B, 1, 1, 64, 16, num_blocks, block_tables.shape[1], PKV_BF16)
+    _check(load_library().pkv_slot_mapping(_p(out), _p(block_tables), _p(context_lens),
+                                           _p(token_seq), _p(token_pos), num_tokens,
+                                           ctypes.byref(dims), _stream_ptr(dev)))
+    return out
+
+
+def check_device_error(device: torch.device | None = None) -> int:
+    """Synchronise the current stream, read and clear the device error bits.
+
+    Raises PkvError when a kernel met an invalid index or a wait timed out.
+    """
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    bits = ctypes.c_uint32()
+    status = load_library().pkv_check_device_error(_stream_ptr(dev), ctypes.byref(bits))
+    if status not in (0, 7, 9):
+        _check(status)
+    if status != 0:
+        raise PkvError(status, f"device error bits 0x{bits.value:x}")
+    return bits.value
+
+
+def device_error_bits(device: torch.device | None = None) -> int:
+    """Like check_device_error, but returns the bits instead of raising."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    bits = ctypes.c_uint32()
+    status = load_library().pkv_check_device_error(_stream_ptr(dev), ctypes.byref(bits))
+    if status not in (0, 7, 9):
+        _check(status)
+    return bits.value

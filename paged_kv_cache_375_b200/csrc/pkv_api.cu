@@ -1,0 +1,485 @@
+// pkv_api.cu -- host side of the C ABI declared in include/pkv.h: argument
+// validation, work planning, TMA tensor-map encoding and kernel launches.
+// Everything is one translation unit so the kernels share the device error
+// word without relocatable device code.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "pkv.h"
+#include "pkv_cache_ops.cuh"
+#include "pkv_decode.cuh"
+#include "pkv_device.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pkv_status fail(pkv_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+pkv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(pkv_dtype t) { return t == PKV_BF16 ? 2 : 4; }
+
+// Checks shared by every call.  `need_seq` also checks the per-sequence fields.
+pkv_status check_dims(const pkv_dims* d, bool need_seq) {
+  if (!d) return fail(PKV_ERR_NULL, "dims is NULL");
+  if (d->dtype != PKV_F32 && d->dtype != PKV_BF16)
+    return fail(PKV_ERR_UNSUPPORTED, "dtype %d not supported (fp32 or bf16)", (int)d->dtype);
+  if (d->block_size != pkv::kBlock)
+    return fail(PKV_ERR_UNSUPPORTED, "block_size %d not supported (16)", d->block_size);
+  if (d->head_dim != 64 && d->head_dim != 128)
+    return fail(PKV_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", d->head_dim);
+  if (d->num_kv_heads <= 0 || d->num_blocks <= 0)
+    return fail(PKV_ERR_SHAPE, "num_kv_heads and num_blocks must be positive");
+  // rows of the pool seen by the TMA tensor map must fit a signed 32-bit coordinate
+  if (static_cast<int64_t>(d->num_blocks) * d->num_kv_heads * pkv::kBlock >= (1ll << 31))
+    return fail(PKV_ERR_SHAPE, "num_blocks * num_kv_heads * 16 must be < 2^31");
+  if (need_seq) {
+    if (d->num_seqs < 0 || d->num_q_heads <= 0 || d->max_blocks_per_seq <= 0)
+      return fail(PKV_ERR_SHAPE, "num_seqs >= 0, num_q_heads > 0, max_blocks_per_seq > 0 required");
+    if (d->num_q_heads % d->num_kv_heads != 0)
+      return fail(PKV_ERR_SHAPE, "num_q_heads %d is not a multiple of num_kv_heads %d",
+                  d->num_q_heads, d->num_kv_heads);
+    if (d->num_q_heads / d->num_kv_heads > 16)
+      return fail(PKV_ERR_UNSUPPORTED, "query heads per kv head %d > 16",
+                  d->num_q_heads / d->num_kv_heads);
+  }
+  return PKV_OK;
+}
+
+int device_sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return sms > 0 ? sms : 148;
+}
+
+struct DecodePlan {
+  int32_t part_tokens = 0;
+  int32_t part_blocks = 0;
+  int32_t max_parts = 0;
+  int32_t max_len = 0;  // lengths above this are clamped (and flagged)
+  size_t items_off = 0, part_o_off = 0, part_ml_off = 0, total = 0;
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Partition choice.  Single pass when there are enough (sequence, kv head)
+// units to fill the GPU several times over and no sequence is very long;
+// otherwise 512-token partitions.
+int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested) {
+  if (requested > 0) return requested;
+  const int32_t single = max_len < pkv::kBlock ? pkv::kBlock
+                                               : static_cast<int32_t>(round_up(max_len, pkv::kBlock));
+  const int64_t units = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
+  const int sms = device_sm_count();
+  if (max_len <= 1024 || (units >= 2ll * sms && max_len <= 8192)) return single;
+  return 512;
+}
+
+pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partition_tokens,
+                     DecodePlan* plan) {
+  pkv_status st = check_dims(d, true);
+  if (st != PKV_OK) return st;
+  if (max_context_len < 0) return fail(PKV_ERR_SHAPE, "max_context_len must be >= 0");
+  if (partition_tokens < 0 || partition_tokens % pkv::kBlock != 0)
+    return fail(PKV_ERR_SHAPE, "partition_tokens must be 0 or a positive multiple of 16");
+  const int64_t table_len = static_cast<int64_t>(d->max_blocks_per_seq) * pkv::kBlock;
+  const int32_t max_len =
+      static_cast<int32_t>(max_context_len < table_len ? max_context_len : table_len);
+  DecodePlan p;
+  p.max_len = max_len;
+  p.part_tokens = choose_partition(d, max_len, partition_tokens);
+  p.part_blocks = p.part_tokens / pkv::kBlock;
+  p.max_parts = max_len <= 0 ? 1 : (max_len + p.part_tokens - 1) / p.part_tokens;
+  const size_t B = static_cast<size_t>(d->num_seqs);
+  const size_t rows = B * d->num_q_heads * p.max_parts;
+  p.items_off = 256;
+  size_t off = round_up(p.items_off + B * p.max_parts * sizeof(pkv::PlanItem), 256);
+  if (p.max_parts > 1) {
+    p.part_o_off = off;
+    off = round_up(off + rows * d->head_dim * sizeof(float), 256);
+    p.part_ml_off = off;
+    off = round_up(off + rows * 2 * sizeof(float), 256);
+  }
+  p.total = off;
+  *plan = p;
+  return PKV_OK;
+}
+
+// cuTensorMapEncodeTiled, resolved from the driver once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+  });
+  return fn;
+}
+
+// A 2-D view of one cache pool: rows = (block, kv head, slot), columns = the
+// head dimension.  The box is 16 rows x 128 bytes with 128-byte swizzling, so
+// one (block, kv head) tile arrives as D*elem/128 swizzled [16][128 B] chunks.
+pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int e = elem_bytes(d->dtype);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d->head_dim),
+                        static_cast<cuuint64_t>(d->num_blocks) * d->num_kv_heads * pkv::kBlock};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d->head_dim) * e};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / e), static_cast<cuuint32_t>(pkv::kBlock)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map,
+                   d->dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   2, const_cast<void*>(pool), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return PKV_OK;
+}
+
+// Kernel configuration per element type.
+template <typename T>
+struct DecodeCfg;
+template <>
+struct DecodeCfg<__nv_bfloat16> {
+  static constexpr int W = 4, S = 4;
+};
+template <>
+struct DecodeCfg<float> {
+  static constexpr int W = 4, S = 2;
+};
+
+// Largest dynamic shared memory already enabled per kernel, per device.
+struct SmemAttr {
+  const void* fn;
+  int device;
+  int bytes;
+};
+std::mutex g_attr_mu;
+std::vector<SmemAttr> g_attr;
+
+cudaError_t ensure_smem(const void* fn, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (auto& a : g_attr) {
+    if (a.fn == fn && a.device == dev) {
+      if (a.bytes >= bytes) return cudaSuccess;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e == cudaSuccess) a.bytes = bytes;
+      return e;
+    }
+  }
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) g_attr.push_back({fn, dev, bytes});
+  return e;
+}
+
+template <typename T, int D, int GMAX>
+pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
+                         const pkv::DecodeParams& prm, int64_t work_units, int g,
+                         cudaStream_t stream) {
+  constexpr int W = DecodeCfg<T>::W, S = DecodeCfg<T>::S;
+  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S>;
+  const int smem = Lay::total_bytes(g);
+  int dev = 0, max_optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (smem > max_optin)
+    return fail(PKV_ERR_UNSUPPORTED, "decode needs %d bytes of shared memory (> %d)", smem,
+                max_optin);
+  auto kern = pkv::decode_kernel<T, D, GMAX, W, S>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, (W + 1) * 32, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "occupancy query (decode)");
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = static_cast<int64_t>(device_sm_count()) * per_sm;
+  if (grid > work_units) grid = work_units;
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<unsigned>(grid), (W + 1) * 32, smem, stream>>>(mk, mv, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status launch_decode_d(const CUtensorMap& mk, const CUtensorMap& mv,
+                           const pkv::DecodeParams& prm, int64_t work_units, int g,
+                           cudaStream_t stream) {
+  if (g <= 8) return launch_decode<T, D, 8>(mk, mv, prm, work_units, g, stream);
+  return launch_decode<T, D, 16>(mk, mv, prm, work_units, g, stream);
+}
+
+template <typename T>
+pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
+                        const int32_t* context_lens, const pkv_dims* d, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(d->num_seqs) * d->num_q_heads;
+  const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
+  const float* po = reinterpret_cast<const float*>(ws + plan.part_o_off);
+  const float* pml = reinterpret_cast<const float*>(ws + plan.part_ml_off);
+  if (d->head_dim == 128) {
+    pkv::merge_kernel<T, 128><<<grid, 128, 0, stream>>>(out, po, pml, context_lens, d->num_seqs,
+                                                        d->num_q_heads, plan.max_parts,
+                                                        plan.max_len, plan.part_tokens);
+  } else {
+    pkv::merge_kernel<T, 64><<<grid, 128, 0, stream>>>(out, po, pml, context_lens, d->num_seqs,
+                                                       d->num_q_heads, plan.max_parts,
+                                                       plan.max_len, plan.part_tokens);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pkv_decode_partition_tokens(const pkv_dims* dims, int32_t max_context_len,
+                                    int32_t partition_tokens) {
+  DecodePlan plan;
+  if (make_plan(dims, max_context_len, partition_tokens, &plan) != PKV_OK) return 0;
+  return plan.part_tokens;
+}
+
+size_t pkv_decode_workspace_bytes(const pkv_dims* dims, int32_t max_context_len,
+                                  int32_t partition_tokens) {
+  DecodePlan plan;
+  if (make_plan(dims, max_context_len, partition_tokens, &plan) != PKV_OK) return 0;
+  return plan.total;
+}
+
+pkv_status pkv_decode_workspace_layout(const pkv_dims* dims, int32_t max_context_len,
+                                       int32_t partition_tokens, int32_t* max_parts,
+                                       size_t* part_o_offset, size_t* part_ml_offset) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (max_parts) *max_parts = plan.max_parts;
+  if (plan.max_parts <= 1) return fail(PKV_ERR_SHAPE, "single-pass decode has no partials");
+  if (part_o_offset) *part_o_offset = plan.part_o_off;
+  if (part_ml_offset) *part_ml_offset = plan.part_ml_off;
+  return PKV_OK;
+}
+
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* context_lens, float scale,
+                                      const pkv_dims* dims, int32_t max_context_len,
+                                      int32_t partition_tokens, void* workspace,
+                                      size_t workspace_bytes, void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  const pkv_dims* d = dims;
+  if (d->num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!workspace) return fail(PKV_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < plan.total)
+    return fail(PKV_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes,
+                plan.total);
+  if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  CUtensorMap mk, mv;
+  if ((st = encode_pool_map(&mk, k_cache, d)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&mv, v_cache, d)) != PKV_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
+  pkv::PlanItem* items = reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off);
+
+  pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, stream>>>(context_lens, d->num_seqs, plan.max_len,
+                                                       plan.part_blocks, items, counters);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "plan launch");
+
+  pkv::DecodeParams prm;
+  prm.out = out;
+  prm.q = q;
+  prm.block_tables = block_tables;
+  prm.items = items;
+  prm.counters = counters;
+  prm.part_o = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_o_off) : nullptr;
+  prm.part_ml = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_ml_off) : nullptr;
+  prm.num_q_heads = d->num_q_heads;
+  prm.num_kv_heads = d->num_kv_heads;
+  prm.group = d->num_q_heads / d->num_kv_heads;
+  prm.max_blocks_per_seq = d->max_blocks_per_seq;
+  prm.num_blocks = d->num_blocks;
+  prm.max_parts = plan.max_parts;
+  prm.part_blocks = plan.part_blocks;
+  prm.qk_scale_log2 = scale * pkv::kLog2e;
+  const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads;
+  if (d->dtype == PKV_BF16) {
+    st = d->head_dim == 128
+             ? launch_decode_d<__nv_bfloat16, 128>(mk, mv, prm, units, prm.group, stream)
+             : launch_decode_d<__nv_bfloat16, 64>(mk, mv, prm, units, prm.group, stream);
+  } else {
+    st = d->head_dim == 128 ? launch_decode_d<float, 128>(mk, mv, prm, units, prm.group, stream)
+                            : launch_decode_d<float, 64>(mk, mv, prm, units, prm.group, stream);
+  }
+  if (st != PKV_OK) return st;
+  if (plan.max_parts > 1) {
+    st = d->dtype == PKV_BF16 ? launch_merge<__nv_bfloat16>(out, plan, ws, context_lens, d, stream)
+                              : launch_merge<float>(out, plan, ws, context_lens, d, stream);
+  }
+  return st;
+}
+
+pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                                 const int64_t* slot_mapping, int32_t num_tokens,
+                                 const pkv_dims* dims, void* cuda_stream) {
+  pkv_status st = check_dims(dims, false);
+  if (st != PKV_OK) return st;
+  if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "k, v and the caches must be 16-byte aligned");
+  const int row_bytes = dims->head_dim * elem_bytes(dims->dtype);
+  const int units = dims->num_kv_heads * row_bytes / 16;
+  int threads = units < 256 ? (units + 31) / 32 * 32 : 256;
+  pkv::reshape_and_cache_kernel<<<num_tokens, threads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
+      static_cast<uint8_t*>(v_cache), slot_mapping, dims->num_kv_heads, row_bytes,
+      static_cast<int64_t>(dims->num_blocks) * pkv::kBlock);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
+  return PKV_OK;
+}
+
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs,
+                           int32_t num_pairs, const pkv_dims* dims, void* cuda_stream) {
+  pkv_status st = check_dims(dims, false);
+  if (st != PKV_OK) return st;
+  if (num_pairs < 0) return fail(PKV_ERR_SHAPE, "num_pairs must be >= 0");
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !pairs) return fail(PKV_ERR_NULL, "a pointer is NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "the caches must be 16-byte aligned");
+  const int64_t block_bytes = static_cast<int64_t>(dims->num_kv_heads) * pkv::kBlock *
+                              dims->head_dim * elem_bytes(dims->dtype);
+  const unsigned chunks =
+      static_cast<unsigned>((block_bytes + pkv::kCopyChunk - 1) / pkv::kCopyChunk);
+  if (chunks > 65535) return fail(PKV_ERR_UNSUPPORTED, "block too large for copy_blocks");
+  dim3 grid(static_cast<unsigned>(num_pairs), chunks, 2);
+  pkv::copy_blocks_kernel<<<grid, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), pairs, block_bytes,
+      dims->num_blocks);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
+  return PKV_OK;
+}
+
+pkv_status pkv_validate_copy_pairs(const int64_t* pairs_host, int32_t num_pairs,
+                                   int32_t num_blocks) {
+  if (num_pairs < 0 || num_blocks <= 0) return fail(PKV_ERR_SHAPE, "bad counts");
+  if (num_pairs == 0) return PKV_OK;
+  if (!pairs_host) return fail(PKV_ERR_NULL, "pairs_host is NULL");
+  std::vector<uint8_t> role(static_cast<size_t>(num_blocks), 0);  // bit0 src, bit1 dst
+  for (int32_t i = 0; i < num_pairs; ++i) {
+    const int64_t s = pairs_host[2 * i], t = pairs_host[2 * i + 1];
+    if (s < 0 || s >= num_blocks || t < 0 || t >= num_blocks)
+      return fail(PKV_ERR_PAIRS, "pair %d (%lld, %lld) outside [0, %d)", i, (long long)s,
+                  (long long)t, num_blocks);
+    if (role[t] & 2u) return fail(PKV_ERR_PAIRS, "destination %lld repeats", (long long)t);
+    role[s] |= 1u;
+    role[t] |= 2u;
+  }
+  for (int32_t i = 0; i < num_blocks; ++i) {
+    if (role[i] == 3u) return fail(PKV_ERR_PAIRS, "block %d is both a source and a destination", i);
+  }
+  return PKV_OK;
+}
+
+pkv_status pkv_slot_mapping(int64_t* slot_mapping, const int32_t* block_tables,
+                            const int32_t* context_lens, const int32_t* token_seq,
+                            const int32_t* token_pos, int32_t num_tokens, const pkv_dims* dims,
+                            void* cuda_stream) {
+  pkv_status st = check_dims(dims, true);
+  if (st != PKV_OK) return st;
+  if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
+  if (num_tokens == 0) return PKV_OK;
+  if (!slot_mapping || !block_tables) return fail(PKV_ERR_NULL, "a pointer is NULL");
+  if (!token_pos && !context_lens)
+    return fail(PKV_ERR_NULL, "context_lens is needed when token_pos is NULL");
+  if (!token_seq && num_tokens > dims->num_seqs)
+    return fail(PKV_ERR_SHAPE, "without token_seq there is one token per sequence");
+  const unsigned grid = static_cast<unsigned>((num_tokens + 255) / 256);
+  pkv::slot_mapping_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      slot_mapping, block_tables, context_lens, token_seq, token_pos, num_tokens, dims->num_seqs,
+      dims->max_blocks_per_seq, dims->num_blocks);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "slot_mapping launch");
+  return PKV_OK;
+}
+
+pkv_status pkv_check_device_error(void* cuda_stream, uint32_t* bits_out) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int bits = 0;
+  e = cudaMemcpyFromSymbol(&bits, pkv::g_device_error, sizeof bits);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  const unsigned int zero = 0;
+  e = cudaMemcpyToSymbol(pkv::g_device_error, &zero, sizeof zero);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+  if (bits_out) *bits_out = bits;
+  if (bits & PKV_DEVERR_TIMEOUT) return fail(PKV_ERR_DEVICE_TIMEOUT, "device wait timed out (bits 0x%x)", bits);
+  if (bits) return fail(PKV_ERR_DEVICE_INDEX, "device index error (bits 0x%x)", bits);
+  return PKV_OK;
+}
+
+const char* pkv_status_string(pkv_status status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_NULL: return "null pointer";
+    case PKV_ERR_SHAPE: return "inconsistent shape";
+    case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case PKV_ERR_PAIRS: return "invalid copy pairs";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_DEVICE_INDEX: return "invalid index met on the device";
+    case PKV_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* pkv_last_error_message(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,118 @@
+// pkv_cache_ops.cuh -- the kernels that maintain the paged KV cache on sm_100a:
+// slot indexing, reshape_and_cache (scatter of new tokens into their slots)
+// and copy_blocks (copy-on-write of shared blocks).
+//
+//  * Slots: a token at position j of a sequence lives in logical block j/16
+//    at offset j%16; the block table names the physical block ("vLLM" wiki
+//    entry, wiki.bytelighting.cn, "Flattened 布局与 slot_mapping"; ipipp.com
+//    vLLM article, "二、PagedAttention分页原理深度剖析").
+//  * copy_blocks serves copy-on-write of blocks shared by several sequences
+//    ("vLLM 深读：用 PagedAttention 撑起高并发 LLM 推理", "先看浪费在哪里").
+//
+// These are byte movers: the element type only fixes the row size.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+// ---------------------------------------------------------------- slot mapping
+__global__ void __launch_bounds__(256)
+    slot_mapping_kernel(int64_t* __restrict__ slots, const int32_t* __restrict__ block_tables,
+                        const int32_t* __restrict__ context_lens,
+                        const int32_t* __restrict__ token_seq,
+                        const int32_t* __restrict__ token_pos, int32_t num_tokens,
+                        int32_t num_seqs, int32_t max_blocks_per_seq, int32_t num_blocks) {
+  const int32_t t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= num_tokens) return;
+  const int32_t seq = token_seq ? token_seq[t] : t;
+  int64_t slot = -1;
+  if (seq < 0 || seq >= num_seqs) {
+    raise_error(PKV_DEVERR_POS);
+  } else {
+    const int32_t pos = token_pos ? token_pos[t] : context_lens[seq] - 1;
+    if (pos < 0 || pos / kBlock >= max_blocks_per_seq) {
+      raise_error(PKV_DEVERR_POS);
+    } else {
+      const int32_t phys =
+          block_tables[static_cast<int64_t>(seq) * max_blocks_per_seq + pos / kBlock];
+      if (phys < 0 || phys >= num_blocks) {
+        raise_error(PKV_DEVERR_BLOCK);
+      } else {
+        slot = static_cast<int64_t>(phys) * kBlock + pos % kBlock;
+      }
+    }
+  }
+  slots[t] = slot;
+}
+
+// ----------------------------------------------------------- reshape_and_cache
+// One CTA per token.  Each thread moves 16-byte units of the token's K row
+// block ([Hkv][D]) and V row block to their (block, head, offset) rows.
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                             uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
+                             const int64_t* __restrict__ slot_mapping, int32_t num_kv_heads,
+                             int32_t row_bytes, int64_t num_slots) {
+  const int32_t t = blockIdx.x;
+  const int64_t slot = slot_mapping[t];
+  if (slot < 0) return;  // padding token
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0) raise_error(PKV_DEVERR_SLOT);
+    return;
+  }
+  const int64_t block = slot / kBlock;
+  const int32_t offset = static_cast<int32_t>(slot % kBlock);
+  const int32_t units_per_row = row_bytes / 16;
+  const int32_t units = num_kv_heads * units_per_row;
+  const uint4* ksrc = k + static_cast<int64_t>(t) * units;
+  const uint4* vsrc = v + static_cast<int64_t>(t) * units;
+  for (int32_t u = threadIdx.x; u < units; u += blockDim.x) {
+    const int32_t h = u / units_per_row;
+    const int32_t within = u % units_per_row;
+    const int64_t dst =
+        ((block * num_kv_heads + h) * kBlock + offset) * row_bytes + within * 16;
+    const uint4 kv = ksrc[u];
+    const uint4 vv = vsrc[u];
+    *reinterpret_cast<uint4*>(k_cache + dst) = kv;
+    *reinterpret_cast<uint4*>(v_cache + dst) = vv;
+  }
+}
+
+// ------------------------------------------------------------------ copy_blocks
+// Grid: (pair, chunk, cache).  One thread moves one chunk of a block with the
+// bulk-copy (TMA) engine: global -> shared, then shared -> global.
+constexpr int kCopyChunk = 16384;
+
+__global__ void __launch_bounds__(32)
+    copy_blocks_kernel(uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
+                       const int64_t* __restrict__ pairs, int64_t block_bytes,
+                       int32_t num_blocks) {
+  __shared__ __align__(128) uint8_t buf[kCopyChunk];
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const int64_t src = pairs[2 * blockIdx.x];
+  const int64_t dst = pairs[2 * blockIdx.x + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (blockIdx.y == 0 && blockIdx.z == 0) raise_error(PKV_DEVERR_PAIR);
+    return;
+  }
+  const int64_t off = static_cast<int64_t>(blockIdx.y) * kCopyChunk;
+  if (off >= block_bytes) return;
+  const uint32_t bytes = static_cast<uint32_t>(
+      block_bytes - off < kCopyChunk ? block_bytes - off : kCopyChunk);
+  uint8_t* cache = blockIdx.z == 0 ? k_cache : v_cache;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_arrive_expect_tx(&bar, bytes);
+  bulk_load(buf, cache + src * block_bytes + off, bytes, &bar);
+  if (!mbar_wait(&bar, 0)) {
+    return;  // timeout already flagged; nothing was issued after the load
+  }
+  fence_proxy_async_smem();
+  bulk_store(cache + dst * block_bytes + off, buf, bytes);
+  bulk_commit();
+  bulk_wait_all();
+}
+
+}  // namespace pkv

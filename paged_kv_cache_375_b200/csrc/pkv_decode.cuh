@@ -1,0 +1,808 @@
+// pkv_decode.cuh -- paged decode attention for sm_100a.
+//
+// What is computed (ipipp.com vLLM article, section
+// "二、PagedAttention分页原理深度剖析"): for every sequence and query head,
+// softmax(scale * q . K^T) V over the sequence's context, where the context is
+// stored in 16-token blocks scattered over one pool and found block by block
+// through the sequence's block table.
+//
+// How it runs on a B200:
+//  * A planning kernel turns context_lens into a work list of items
+//    (sequence, partition), longest first.  A partition is at most
+//    `part_blocks` blocks; a sequence longer than one partition is split
+//    (split-K) and its partial results are merged by log-sum-exp afterwards.
+//  * The decode kernel is persistent (one CTA per SM).  Items (x every kv
+//    head) are handed out through an atomic counter.  Inside a CTA one
+//    producer warp walks the block table and issues a TMA tensor load per
+//    128-byte column chunk of each 16-token K and V tile (the tile of one
+//    (block, kv head) is contiguous in the HND pool) into 128B-swizzled
+//    shared memory, signalling an mbarrier; W consumer warps take the blocks
+//    of an item round-robin, each keeping its own online-softmax state, and
+//    merge their states at the end of the item.  The producer runs ahead
+//    across item boundaries, so the next item's tiles are already in flight
+//    while the current one is merged.
+//  * bf16: all query heads of a GQA group (g <= 16 rows) form the M side of
+//    mma.sync m16n8k16: S = Q K^T per 16-token tile, then O += P V.  Every KV
+//    tile is read from HBM once per group.
+//  * fp32: the same pipeline with a CUDA-core consumer (fp32 has no exact
+//    tensor-core path; TF32 would break the fp32 tolerance).
+//  * Padding slots of the last block are never used: their scores are
+//    selected to -inf and their V values are masked to zero before the MMA
+//    (0 * NaN would otherwise poison the output).
+#pragma once
+
+#include <type_traits>
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr int kRing = 4;          // items in flight between producer and consumers
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// One unit of planned work: tokens [p*part_blocks*16, ...) of sequence s.
+struct PlanItem {
+  int32_t seq;
+  int32_t part;
+  int32_t len;     // context length of the sequence, after validation
+  int32_t nparts;  // partitions of the sequence
+};
+
+// Context length after validation against the table width and the host's
+// max_context_len hint; out-of-range values are clamped and flagged.
+__device__ __forceinline__ int32_t checked_len(int32_t L, int32_t max_len) {
+  if (L < 0 || L > max_len) {
+    raise_error(PKV_DEVERR_LEN);
+    L = L < 0 ? 0 : max_len;
+  }
+  return L;
+}
+
+__device__ __forceinline__ int32_t num_parts(int32_t L, int32_t part_tokens) {
+  int32_t n = (L + part_tokens - 1) / part_tokens;
+  return n < 1 ? 1 : n;
+}
+
+// ----------------------------------------------------------------- planning
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 1024;  // item sizes in blocks; larger sizes share the top bucket
+
+__device__ __forceinline__ int plan_bucket(int32_t blocks) {
+  return blocks < kPlanBuckets - 1 ? blocks : kPlanBuckets - 1;
+}
+
+__device__ __forceinline__ int32_t part_size_blocks(int32_t L, int32_t p, int32_t part_blocks) {
+  int32_t total = (L + kBlock - 1) / kBlock;
+  int32_t rest = total - p * part_blocks;
+  return rest < part_blocks ? rest : part_blocks;
+}
+
+// Single CTA.  counters[0] = work counter (zeroed here), counters[1] = items.
+__global__ void __launch_bounds__(kPlanThreads)
+    plan_kernel(const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t max_len,
+                int32_t part_blocks, PlanItem* __restrict__ items,
+                uint32_t* __restrict__ counters) {
+  __shared__ uint32_t hist[kPlanBuckets];
+  __shared__ uint32_t warp_sums[kPlanThreads / 32];
+  const int tid = threadIdx.x;
+  const int32_t part_tokens = part_blocks * kBlock;
+  for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
+  __syncthreads();
+  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
+    int32_t L = checked_len(context_lens[s], max_len);
+    int32_t n = num_parts(L, part_tokens);
+    for (int32_t p = 0; p < n; ++p) atomicAdd(&hist[plan_bucket(part_size_blocks(L, p, part_blocks))], 1u);
+  }
+  __syncthreads();
+  // Exclusive scan in descending bucket order: thread i owns bucket B-1-i.
+  const int bucket = kPlanBuckets - 1 - tid;
+  uint32_t v = hist[bucket];
+  uint32_t incl = v;
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const uint32_t base = (warp > 0 ? warp_sums[warp - 1] : 0u) + incl - v;
+  __syncthreads();
+  hist[bucket] = base;  // becomes the write cursor of the bucket
+  if (tid == kPlanThreads - 1) {
+    counters[1] = warp_sums[kPlanThreads / 32 - 1];
+    counters[0] = 0u;
+  }
+  __syncthreads();
+  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
+    int32_t L = context_lens[s];
+    L = L < 0 ? 0 : (L > max_len ? max_len : L);
+    int32_t n = num_parts(L, part_tokens);
+    for (int32_t p = 0; p < n; ++p) {
+      uint32_t pos = atomicAdd(&hist[plan_bucket(part_size_blocks(L, p, part_blocks))], 1u);
+      items[pos] = PlanItem{s, p, L, n};
+    }
+  }
+}
+
+// ------------------------------------------------------------ decode kernel
+struct DecodeParams {
+  void* out;                     // [B][Hq][D], dtype of the cache
+  const void* q;                 // [B][Hq][D]
+  const int32_t* block_tables;   // [B][MB]
+  const PlanItem* items;         // planned work, longest first
+  uint32_t* counters;            // [0] work counter, [1] number of items
+  float* part_o;                 // [B][Hq][max_parts][D]
+  float* part_ml;                // [B][Hq][max_parts][2]
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t group;                 // Hq / Hkv
+  int32_t max_blocks_per_seq;
+  int32_t num_blocks;
+  int32_t max_parts;
+  int32_t part_blocks;
+  float qk_scale_log2;           // scale * log2(e)
+};
+
+// Shared-memory map of the decode kernel (offsets from a 1024-aligned base).
+template <int ELEM, int D, int GMAX, int W, int S>
+struct DecodeLayout {
+  static constexpr int kTileBytes = kBlock * D * ELEM;       // one K (or V) tile
+  static constexpr int kChunks = D * ELEM / 128;             // 128-byte column chunks
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kQBytes = ((GMAX * D * ELEM) + 127) / 128 * 128;
+  static constexpr int kStagesOff = 0;
+  static constexpr int kRingOff = kStagesOff + W * S * kStageBytes;
+  static constexpr int kMergeOff = kRingOff + kRing * kQBytes;
+  // merge area: 2 buffers x W warps x (g*D + 2g rounded up to 4) floats, g
+  // chosen at run time; every warp's slot starts 16-byte aligned.
+  __host__ __device__ static int merge_floats_per_warp(int g) { return g * D + (2 * g + 3) / 4 * 4; }
+  __host__ __device__ static int meta_off(int g) {
+    return kMergeOff + 2 * W * merge_floats_per_warp(g) * 4;
+  }
+  static constexpr int kMetaBytes = kRing * 32;
+  __host__ __device__ static int bars_off(int g) { return (meta_off(g) + kMetaBytes + 7) / 8 * 8; }
+  static constexpr int kNumBars = 2 * W * S + 2 * kRing + 2;
+  __host__ __device__ static int flags_off(int g) { return bars_off(g) + kNumBars * 8; }
+  __host__ __device__ static int total_bytes(int g) {
+    return flags_off(g) + (W * S + 4) * 4 + 1024;  // + slack for 1024-byte alignment
+  }
+};
+
+struct ItemMeta {
+  int32_t seq, kv_head, part, len, nparts, blk_begin, nblk, pad;
+};
+
+// ---- consumer state for bf16 (tensor cores) ----
+template <int D, int GMAX>
+struct Bf16State {
+  static constexpr int KS = D / 16;  // k-steps of Q K^T
+  static constexpr int NT = D / 8;   // n-tiles of P V
+  static constexpr bool kTwoRowHalves = GMAX > 8;
+  uint32_t qa[KS][4];
+  float o[NT][4];
+  float m[2], l[2];
+};
+
+template <int D, int GMAX>
+__device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const uint8_t* qs,
+                                                int g, int lane) {
+  const int r0 = lane >> 2, qd = (lane & 3) * 2;
+  const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qs);
+#pragma unroll
+  for (int ks = 0; ks < Bf16State<D, GMAX>::KS; ++ks) {
+    const int c = ks * 16 + qd;
+    st.qa[ks][0] = r0 < g ? *reinterpret_cast<const uint32_t*>(q16 + r0 * D + c) : 0u;
+    st.qa[ks][2] = r0 < g ? *reinterpret_cast<const uint32_t*>(q16 + r0 * D + c + 8) : 0u;
+    if constexpr (Bf16State<D, GMAX>::kTwoRowHalves) {
+      const int r1 = r0 + 8;
+      st.qa[ks][1] = r1 < g ? *reinterpret_cast<const uint32_t*>(q16 + r1 * D + c) : 0u;
+      st.qa[ks][3] = r1 < g ? *reinterpret_cast<const uint32_t*>(q16 + r1 * D + c + 8) : 0u;
+    } else {
+      st.qa[ks][1] = 0u;
+      st.qa[ks][3] = 0u;
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < Bf16State<D, GMAX>::NT; ++nt) {
+    st.o[nt][0] = st.o[nt][1] = st.o[nt][2] = st.o[nt][3] = 0.f;
+  }
+  st.m[0] = st.m[1] = -INFINITY;
+  st.l[0] = st.l[1] = 0.f;
+}
+
+// One 16-token tile: scores, online softmax, P V.  `valid` tokens (0..16) of
+// the tile belong to the context.
+template <int D, int GMAX>
+__device__ __forceinline__ void bf16_block(Bf16State<D, GMAX>& st, const uint8_t* ktile,
+                                           const uint8_t* vtile, int valid, float sc,
+                                           int lane) {
+  using St = Bf16State<D, GMAX>;
+  constexpr bool kTwo = St::kTwoRowHalves;
+  const uint32_t kt = smem_addr(ktile), vt = smem_addr(vtile);
+  // ---- S = Q K^T (two independent accumulation chains per n-tile) ----
+  float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  {
+    const int mi = lane >> 3, ri = lane & 7;
+    const uint32_t t = (mi >> 1) * 8 + ri;      // token row this lane addresses
+    const uint32_t gsel = mi & 1;               // low / high 8 columns of the k-step
+    const uint32_t rowbase = kt + t * 128u;
+#pragma unroll
+    for (int ks = 0; ks < St::KS; ++ks) {
+      const uint32_t c = ks >> 2, j = (ks & 3) * 2;
+      const uint32_t addr = rowbase + c * (kBlock * 128u) + (((j + gsel) ^ (t & 7u)) << 4);
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4(addr, b0, b1, b2, b3);
+      if (ks & 1) {
+        mma_bf16_16816(sb[0], st.qa[ks], b0, b1);
+        mma_bf16_16816(sb[1], st.qa[ks], b2, b3);
+      } else {
+        mma_bf16_16816(sa[0], st.qa[ks], b0, b1);
+        mma_bf16_16816(sa[1], st.qa[ks], b2, b3);
+      }
+    }
+  }
+  // ---- scale, mask, online softmax ----
+  const int qd = (lane & 3) * 2;
+  float z[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tok = nt * 8 + qd + (i & 1);
+      const float v = (sa[nt][i] + sb[nt][i]) * sc;
+      z[nt][i] = tok < valid ? v : -INFINITY;
+    }
+  }
+  float p[2][4];
+#pragma unroll
+  for (int rh = 0; rh < (kTwo ? 2 : 1); ++rh) {
+    float mx = fmaxf(fmaxf(z[0][2 * rh], z[0][2 * rh + 1]), fmaxf(z[1][2 * rh], z[1][2 * rh + 1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(st.m[rh], mx);
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = exp2f(st.m[rh] - m_use);
+    st.m[rh] = m_new;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      p[nt][2 * rh] = exp2f(z[nt][2 * rh] - m_use);
+      p[nt][2 * rh + 1] = exp2f(z[nt][2 * rh + 1] - m_use);
+    }
+#pragma unroll
+    for (int nt = 0; nt < St::NT; ++nt) {
+      st.o[nt][2 * rh] *= alpha;
+      st.o[nt][2 * rh + 1] *= alpha;
+    }
+    st.l[rh] *= alpha;
+  }
+  uint32_t pa[4];
+  pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+  pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+  st.l[0] += (bf16lo_to_f32(pa[0]) + bf16hi_to_f32(pa[0])) +
+             (bf16lo_to_f32(pa[2]) + bf16hi_to_f32(pa[2]));
+  if constexpr (kTwo) {
+    pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+    pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+    st.l[1] += (bf16lo_to_f32(pa[1]) + bf16hi_to_f32(pa[1])) +
+               (bf16lo_to_f32(pa[3]) + bf16hi_to_f32(pa[3]));
+  } else {
+    pa[1] = 0u;
+    pa[3] = 0u;
+  }
+  // ---- O += P V ----
+  uint32_t mk0 = 0xffffffffu, mk1 = 0xffffffffu;
+  const bool partial = valid < kBlock;
+  if (partial) {
+    mk0 = (qd < valid ? 0x0000ffffu : 0u) | (qd + 1 < valid ? 0xffff0000u : 0u);
+    mk1 = (qd + 8 < valid ? 0x0000ffffu : 0u) | (qd + 9 < valid ? 0xffff0000u : 0u);
+  }
+  {
+    const int mi = lane >> 3, ri = lane & 7;
+    const uint32_t t = (mi & 1) * 8 + ri;
+    const uint32_t gsel = mi >> 1;
+    const uint32_t rowbase = vt + t * 128u;
+#pragma unroll
+    for (int dt = 0; dt < St::NT / 2; ++dt) {
+      const uint32_t c = dt >> 2, j = (dt & 3) * 2;
+      const uint32_t addr = rowbase + c * (kBlock * 128u) + (((j + gsel) ^ (t & 7u)) << 4);
+      uint32_t v0, v1, v2, v3;
+      ldmatrix_x4_trans(addr, v0, v1, v2, v3);
+      if (partial) {
+        v0 &= mk0;
+        v1 &= mk1;
+        v2 &= mk0;
+        v3 &= mk1;
+      }
+      mma_bf16_16816(st.o[2 * dt], pa, v0, v1);
+      mma_bf16_16816(st.o[2 * dt + 1], pa, v2, v3);
+    }
+  }
+}
+
+// Write this warp's (m, l, O) rows into its slot of the merge area.
+template <int D, int GMAX>
+__device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot, int g,
+                                             int lane) {
+  using St = Bf16State<D, GMAX>;
+  const int r0 = lane >> 2, qd = (lane & 3) * 2;
+  float* O = slot;
+  float* M = slot + g * D;
+  float* L = M + g;
+#pragma unroll
+  for (int rh = 0; rh < (St::kTwoRowHalves ? 2 : 1); ++rh) {
+    float l = st.l[rh];
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    const int row = r0 + 8 * rh;
+    if (row < g) {
+#pragma unroll
+      for (int nt = 0; nt < St::NT; ++nt) {
+        *reinterpret_cast<float2*>(O + row * D + nt * 8 + qd) =
+            make_float2(st.o[nt][2 * rh], st.o[nt][2 * rh + 1]);
+      }
+      if ((lane & 3) == 0) {
+        M[row] = st.m[rh];
+        L[row] = l;
+      }
+    }
+  }
+}
+
+// ---- consumer state for fp32 (CUDA cores) ----
+template <int D, int GMAX>
+struct F32State {
+  static constexpr int NV = D / 32;  // output columns per lane
+  float o[GMAX][NV];
+  float m[GMAX], l[GMAX];
+};
+
+template <int D, int GMAX>
+__device__ __forceinline__ void f32_begin_item(F32State<D, GMAX>& st) {
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) {
+    st.m[h] = -INFINITY;
+    st.l[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < F32State<D, GMAX>::NV; ++i) st.o[h][i] = 0.f;
+  }
+}
+
+template <int D, int GMAX>
+__device__ __forceinline__ void f32_block(F32State<D, GMAX>& st, const float* qs,
+                                          const uint8_t* ktile, const uint8_t* vtile, int valid,
+                                          float sc, int g, int lane) {
+  constexpr int NV = F32State<D, GMAX>::NV;
+  const int t = lane & 15, hf = lane >> 4;
+  float acc[GMAX];
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) acc[h] = 0.f;
+#pragma unroll
+  for (int dd = 0; dd < D / 8; ++dd) {
+    const int d0 = hf * (D / 2) + dd * 4;
+    const uint32_t byte = d0 * 4;
+    const float4 kv = *reinterpret_cast<const float4*>(
+        ktile + (byte >> 7) * (kBlock * 128) + swz128(t, byte & 127));
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < g) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + h * D + d0);
+        acc[h] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, acc[h]))));
+      }
+    }
+  }
+  float pr[GMAX];
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) {
+    if (h < g) {
+      float a = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 16);
+      const float z = t < valid ? a * sc : -INFINITY;
+      float mx = z;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      const float m_new = fmaxf(st.m[h], mx);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = exp2f(st.m[h] - m_use);
+      const float pz = exp2f(z - m_use);
+      float ps = pz;
+      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+      st.m[h] = m_new;
+      st.l[h] = st.l[h] * alpha + ps;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) st.o[h][i] *= alpha;
+      pr[h] = pz;
+    }
+  }
+  for (int tt = 0; tt < valid; ++tt) {
+    float v[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      v[i] = *reinterpret_cast<const float*>(vtile + i * (kBlock * 128) +
+                                             swz128(tt, (lane * 4) & 127));
+    }
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+      if (h < g) {
+        const float pt = __shfl_sync(0xffffffffu, pr[h], tt);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) st.o[h][i] = fmaf(pt, v[i], st.o[h][i]);
+      }
+    }
+  }
+}
+
+template <int D, int GMAX>
+__device__ __forceinline__ void f32_publish(F32State<D, GMAX>& st, float* slot, int g,
+                                            int lane) {
+  float* O = slot;
+  float* M = slot + g * D;
+  float* L = M + g;
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) {
+    if (h < g) {
+#pragma unroll
+      for (int i = 0; i < F32State<D, GMAX>::NV; ++i) O[h * D + lane + 32 * i] = st.o[h][i];
+      if (lane == 0) {
+        M[h] = st.m[h];
+        L[h] = st.l[h];
+      }
+    }
+  }
+}
+
+// ---- combine the W warps' states of one item and store the result ----
+template <typename T, int D, int W>
+__device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const ItemMeta& it,
+                                                  const float* merge, int per_warp, int g,
+                                                  int warp, int lane) {
+  const int tid = warp * 32 + lane;
+  const int row0 = it.seq * prm.num_q_heads + it.kv_head * g;  // first q-head row of the group
+  for (int e = tid * 4; e < g * D; e += W * 32 * 4) {
+    const int h = e / D, d = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < W; ++w) M = fmaxf(M, merge[w * per_warp + g * D + h]);
+    float lsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const float* slot = merge + w * per_warp;
+        const float f = exp2f(slot[g * D + h] - M);
+        lsum = fmaf(slot[g * D + g + h], f, lsum);
+        const float4 ov = *reinterpret_cast<const float4*>(slot + h * D + d);
+        acc.x = fmaf(ov.x, f, acc.x);
+        acc.y = fmaf(ov.y, f, acc.y);
+        acc.z = fmaf(ov.z, f, acc.z);
+        acc.w = fmaf(ov.w, f, acc.w);
+      }
+      const float inv = 1.f / lsum;
+      acc.x *= inv;
+      acc.y *= inv;
+      acc.z *= inv;
+      acc.w *= inv;
+    }
+    const size_t row = static_cast<size_t>(row0 + h);
+    if (it.nparts == 1) {
+      if constexpr (sizeof(T) == 2) {
+        uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(prm.out) + row * D + d) = packed;
+      } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.out) + row * D + d) = acc;
+      }
+    } else {
+      const size_t prow = row * prm.max_parts + it.part;
+      *reinterpret_cast<float4*>(prm.part_o + prow * D + d) = acc;
+      if (d == 0) {
+        prm.part_ml[prow * 2 + 0] = M == -INFINITY ? -INFINITY : M * kLn2;
+        prm.part_ml[prow * 2 + 1] = lsum;
+      }
+    }
+  }
+}
+
+// The persistent decode kernel.  Warps 0..W-1 consume, warp W produces.
+template <typename T, int D, int GMAX, int W, int S>
+__global__ void __launch_bounds__((W + 1) * 32, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
+  constexpr int ELEM = sizeof(T);
+  using Lay = DecodeLayout<ELEM, D, GMAX, W, S>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int g = prm.group;
+  uint8_t* stages = smem + Lay::kStagesOff;
+  uint8_t* ring = smem + Lay::kRingOff;
+  float* merge = reinterpret_cast<float*>(smem + Lay::kMergeOff);
+  ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + Lay::meta_off(g));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off(g));
+  uint64_t* full = bars;                       // [W][S]
+  uint64_t* empty = bars + W * S;              // [W][S]
+  uint64_t* item_full = bars + 2 * W * S;      // [kRing]
+  uint64_t* item_empty = item_full + kRing;    // [kRing]
+  uint64_t* merge_bar = item_empty + kRing;    // [2]
+  uint32_t* stage_ok = reinterpret_cast<uint32_t*>(smem + Lay::flags_off(g));  // [W][S]
+  volatile uint32_t* abort_flag = stage_ok + W * S;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < W * S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_empty[i], W);
+    }
+    mbar_init(&merge_bar[0], W);
+    mbar_init(&merge_bar[1], W);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int32_t hkv = prm.num_kv_heads;
+  if (warp == W) {
+    // ================================ producer ================================
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_k);
+      prefetch_tensormap(&tmap_v);
+    }
+    const uint32_t total = prm.counters[1] * static_cast<uint32_t>(hkv);
+    const uint64_t policy = l2_policy_evict_first();
+    uint32_t stage_ctr[W];
+#pragma unroll
+    for (int w = 0; w < W; ++w) stage_ctr[w] = 0;
+    uint32_t next = 0;
+    if (lane == 0) next = atomicAdd(&prm.counters[0], 1u);
+    next = __shfl_sync(0xffffffffu, next, 0);
+    bool ok = true;
+    for (uint32_t item_seq = 0;; ++item_seq) {
+      const int r = item_seq % kRing;
+      if (item_seq >= kRing) {
+        if (lane == 0) ok = mbar_wait(&item_empty[r], ((item_seq / kRing) - 1) & 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok || *abort_flag) break;
+      }
+      const uint32_t widx = next;
+      if (widx >= total) {
+        if (lane == 0) {
+          meta[r].seq = -1;
+          mbar_arrive(&item_full[r]);
+        }
+        break;
+      }
+      if (lane == 0) next = atomicAdd(&prm.counters[0], 1u);
+      next = __shfl_sync(0xffffffffu, next, 0);
+      const PlanItem pi = prm.items[widx / hkv];
+      const int32_t kvh = static_cast<int32_t>(widx % hkv);
+      const int32_t blk_begin = pi.part * prm.part_blocks;
+      const int32_t nblk_total = (pi.len + kBlock - 1) / kBlock;
+      int32_t nblk = nblk_total - blk_begin;
+      nblk = nblk < prm.part_blocks ? nblk : prm.part_blocks;
+      nblk = nblk < 0 ? 0 : nblk;
+      if (lane == 0) {
+        ItemMeta& mt = meta[r];
+        mt.seq = pi.seq;
+        mt.kv_head = kvh;
+        mt.part = pi.part;
+        mt.len = pi.len;
+        mt.nparts = pi.nparts;
+        mt.blk_begin = blk_begin;
+        mt.nblk = nblk;
+        const uint32_t qbytes = static_cast<uint32_t>(g * D * ELEM);
+        mbar_arrive_expect_tx(&item_full[r], qbytes);
+        const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(prm.q) +
+                              (static_cast<size_t>(pi.seq) * prm.num_q_heads + kvh * g) * D * ELEM;
+        bulk_load(ring + r * Lay::kQBytes, qsrc, qbytes, &item_full[r]);
+      }
+      const int32_t* table = prm.block_tables +
+                             static_cast<size_t>(pi.seq) * prm.max_blocks_per_seq + blk_begin;
+      int32_t tbl = (lane < nblk) ? table[lane] : -1;
+      for (int32_t b = 0; b < nblk; ++b) {
+        if ((b & 31) == 0 && b > 0) tbl = (b + lane < nblk) ? table[b + lane] : -1;
+        const int32_t entry = __shfl_sync(0xffffffffu, tbl, b & 31);
+        const int w = b % W;
+        uint32_t ctr = 0;
+#pragma unroll
+        for (int x = 0; x < W; ++x) ctr = (x == w) ? stage_ctr[x] : ctr;
+        const int st = ctr % S;
+        if (lane == 0) {
+          if (ctr >= S) ok = mbar_wait(&empty[w * S + st], ((ctr / S) - 1) & 1);
+          if (ok) {
+            const bool valid = entry >= 0 && entry < prm.num_blocks;
+            stage_ok[w * S + st] = valid ? 1u : 0u;
+            uint8_t* kdst = stages + (w * S + st) * Lay::kStageBytes;
+            uint8_t* vdst = kdst + Lay::kTileBytes;
+            if (valid) {
+              mbar_arrive_expect_tx(&full[w * S + st], 2 * Lay::kTileBytes);
+              const int32_t y = (entry * hkv + kvh) * kBlock;
+#pragma unroll
+              for (int c = 0; c < Lay::kChunks; ++c) {
+                tma_load_2d_hint(kdst + c * (kBlock * 128), &tmap_k, c * (128 / ELEM), y,
+                                 &full[w * S + st], policy);
+                tma_load_2d_hint(vdst + c * (kBlock * 128), &tmap_v, c * (128 / ELEM), y,
+                                 &full[w * S + st], policy);
+              }
+            } else {
+              raise_error(PKV_DEVERR_BLOCK);
+              mbar_arrive(&full[w * S + st]);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+#pragma unroll
+        for (int x = 0; x < W; ++x) stage_ctr[x] += (x == w) ? 1u : 0u;
+      }
+      if (!ok || *abort_flag) break;
+    }
+    if (!ok) {
+      // A wait gave up: tell the consumers, then wait (briefly, bounded) for
+      // the tile copies this warp issued, so none lands after the CTA exits.
+      *abort_flag = 1u;
+      if (lane == 0) {
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+#pragma unroll
+          for (int s2 = 0; s2 < S; ++s2) {
+            const uint32_t c = stage_ctr[w];
+            if (c > static_cast<uint32_t>(s2)) {
+              const uint32_t issues = (c - 1 - s2) / S + 1;
+              mbar_wait(&full[w * S + s2], (issues - 1) & 1, 100000000ull);
+            }
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ================================ consumers ================================
+  using Bst = Bf16State<D, GMAX>;
+  using Fst = F32State<D, GMAX>;
+  constexpr bool kBf16 = sizeof(T) == 2;
+  typename std::conditional<kBf16, Bst, Fst>::type st;
+  uint32_t stage_ctr = 0;
+  const float sc = prm.qk_scale_log2;
+  const int per_warp = Lay::merge_floats_per_warp(g);
+  for (uint32_t item_seq = 0;; ++item_seq) {
+    const int r = item_seq % kRing;
+    if (!mbar_wait(&item_full[r], (item_seq / kRing) & 1)) {
+      *abort_flag = 1u;
+      break;
+    }
+    const ItemMeta it = meta[r];
+    if (it.seq < 0) break;
+    const uint8_t* qs = ring + r * Lay::kQBytes;
+    if constexpr (kBf16) {
+      bf16_begin_item<D, GMAX>(st, qs, g, lane);
+    } else {
+      f32_begin_item<D, GMAX>(st);
+    }
+    bool ok = true;
+    for (int32_t b = warp; b < it.nblk; b += W) {
+      const int s_idx = stage_ctr % S;
+      ok = mbar_wait(&full[warp * S + s_idx], (stage_ctr / S) & 1);
+      if (!ok) break;
+      int valid = it.len - (it.blk_begin + b) * kBlock;
+      valid = valid > kBlock ? kBlock : valid;
+      if (!stage_ok[warp * S + s_idx]) valid = 0;
+      const uint8_t* kt = stages + (warp * S + s_idx) * Lay::kStageBytes;
+      if constexpr (kBf16) {
+        bf16_block<D, GMAX>(st, kt, kt + Lay::kTileBytes, valid, sc, lane);
+      } else {
+        f32_block<D, GMAX>(st, reinterpret_cast<const float*>(qs), kt, kt + Lay::kTileBytes, valid,
+                           sc, g, lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[warp * S + s_idx]);
+      ++stage_ctr;
+    }
+    if (!ok) {
+      *abort_flag = 1u;
+      break;
+    }
+    // The q tile and the metadata have been read: free the ring slot.
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[r]);
+    // ---- merge the W warps' states ----
+    const int mb = item_seq & 1;
+    float* mslot = merge + (mb * W + warp) * per_warp;
+    if constexpr (kBf16) {
+      bf16_publish<D, GMAX>(st, mslot, g, lane);
+    } else {
+      f32_publish<D, GMAX>(st, mslot, g, lane);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&merge_bar[mb]);
+    if (!mbar_wait(&merge_bar[mb], (item_seq >> 1) & 1)) {
+      *abort_flag = 1u;
+      break;
+    }
+    combine_and_store<T, D, W>(prm, it, merge + mb * W * per_warp, per_warp, g, warp, lane);
+  }
+}
+
+// ------------------------------------------------------------- merge kernel
+// One warp per (sequence, query head) row whose sequence was split: combine
+// the partitions' (m, l, o) by log-sum-exp and store the final output.
+template <typename T, int D>
+__global__ void __launch_bounds__(128)
+    merge_kernel(void* __restrict__ out, const float* __restrict__ part_o,
+                 const float* __restrict__ part_ml, const int32_t* __restrict__ context_lens,
+                 int32_t num_seqs, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
+                 int32_t part_tokens) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
+  const int32_t s = static_cast<int32_t>(row / num_q_heads);
+  int32_t L = context_lens[s];
+  L = L < 0 ? 0 : (L > max_len ? max_len : L);
+  const int32_t n = num_parts(L, part_tokens);
+  if (n <= 1) return;  // the decode kernel wrote this row directly
+  const float* ml = part_ml + row * max_parts * 2;
+  float M = -INFINITY;
+  for (int p = lane; p < n; p += 32) M = fmaxf(M, ml[2 * p]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  constexpr int VEC = D / 32;  // floats per lane
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+  const float* po = part_o + row * max_parts * D + lane * VEC;
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int p = 0; p < n; ++p) {
+      const float lp = ml[2 * p + 1];
+      const float w = lp > 0.f ? lp * exp2f((ml[2 * p] - M) * kLog2e) : 0.f;
+      wsum += w;
+      if constexpr (VEC == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(po + static_cast<size_t>(p) * D);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]);
+        acc[3] = fmaf(w, v.w, acc[3]);
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(po + static_cast<size_t>(p) * D);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  if constexpr (sizeof(T) == 2) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + row * D + lane * VEC;
+    if constexpr (VEC == 4) {
+      *reinterpret_cast<uint2*>(o) =
+          make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    } else {
+      *reinterpret_cast<uint32_t*>(o) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
+  } else {
+    float* o = reinterpret_cast<float*>(out) + row * D + lane * VEC;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) o[i] = acc[i] * inv;
+  }
+}
+
+}  // namespace pkv

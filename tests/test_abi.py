@@ -1,0 +1,147 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+its host-side logic (argument checks, workspace sizing, partition choice,
+copy-pair validation) behaves as documented.  No GPU is needed: nothing here
+launches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_cache_375_b200 as pkv
+from paged_kv_cache_375_b200 import build as pkv_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkv_build.build()
+    return pkv.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pkv_paged_attention_decode", "pkv_reshape_and_cache", "pkv_copy_blocks",
+                     "pkv_slot_mapping", "pkv_check_device_error", "pkv_decode_workspace_bytes"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pkv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_library_is_built_for_sm100a_only(lib):
+    # the build flags pin the architecture; the ELF carries the sm_100a cubin
+    assert "arch=compute_100a,code=sm_100a" in " ".join(pkv_build.NVCC_FLAGS)
+
+
+def test_status_strings(lib):
+    for code in range(10):
+        assert lib.pkv_status_string(code).decode() != "unknown status"
+    assert lib.pkv_status_string(99).decode() == "unknown status"
+
+
+def dims(B=4, hq=8, hkv=2, d=128, bs=16, nb=100, mb=8, dtype=pkv.PKV_BF16):
+    return pkv.PkvDims(B, hq, hkv, d, bs, nb, mb, dtype)
+
+
+def test_workspace_single_pass_has_no_partials():
+    d = dims(B=256, hq=32, hkv=8, nb=40000, mb=512)
+    assert pkv.decode_partition_tokens(d, 8192) >= 8192
+    n = pkv.decode_workspace_bytes(d, 8192)
+    assert 0 < n < 64 * 1024
+    with pytest.raises(pkv.PkvError):
+        pkv.decode_workspace_layout(d, 8192)
+
+
+def test_workspace_split_k_sizes():
+    d = dims(B=8, hq=64, hkv=8, nb=81920, mb=8192)
+    P = pkv.decode_partition_tokens(d, 131072)
+    assert P == 512
+    max_parts, po, pm = pkv.decode_workspace_layout(d, 131072)
+    assert max_parts == 256
+    assert po % 256 == 0 and pm % 256 == 0 and pm >= po + 8 * 64 * 256 * 128 * 4
+    assert pkv.decode_workspace_bytes(d, 131072) >= pm + 8 * 64 * 256 * 2 * 4
+
+
+def test_explicit_partition_is_honoured():
+    d = dims()
+    assert pkv.decode_partition_tokens(d, 100, 32) == 32
+    mp, _, _ = pkv.decode_workspace_layout(d, 100, 32)
+    assert mp == 4
+
+
+@pytest.mark.parametrize("bad", [
+    dict(bs=8), dict(d=96), dict(hq=6, hkv=4), dict(hq=34, hkv=2), dict(nb=0),
+    dict(dtype=7), dict(mb=0), dict(B=-1)])
+def test_bad_dims_are_rejected(bad):
+    assert pkv.decode_workspace_bytes(dims(**bad), 64) == 0
+
+
+def test_bad_partition_is_rejected():
+    assert pkv.decode_workspace_bytes(dims(), 64, 24) == 0
+
+
+def test_decode_rejects_null_and_small_workspace(lib):
+    d = dims()
+    null = ctypes.c_void_p(0)
+    st = lib.pkv_paged_attention_decode(null, null, null, null, null, null, 1.0,
+                                        ctypes.byref(d), 64, 0, null, 0, null)
+    assert pkv.STATUS_NAMES[st] == "PKV_ERR_NULL"
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any launch
+    st = lib.pkv_paged_attention_decode(fake, fake, fake, fake, fake, fake, 1.0,
+                                        ctypes.byref(d), 64, 0, fake, 16, null)
+    assert pkv.STATUS_NAMES[st] == "PKV_ERR_WORKSPACE"
+    assert b"needed" in lib.pkv_last_error_message()
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    st = lib.pkv_paged_attention_decode(odd, fake, fake, fake, fake, fake, 1.0,
+                                        ctypes.byref(d), 64, 0, fake, 1 << 20, null)
+    assert pkv.STATUS_NAMES[st] == "PKV_ERR_ALIGN"
+
+
+def test_empty_batch_is_a_no_op(lib):
+    d = dims(B=0)
+    null = ctypes.c_void_p(0)
+    assert lib.pkv_paged_attention_decode(null, null, null, null, null, null, 1.0,
+                                          ctypes.byref(d), 0, 0, null, 0, null) == 0
+    assert lib.pkv_reshape_and_cache(null, null, null, null, null, 0, ctypes.byref(d), null) == 0
+    assert lib.pkv_copy_blocks(null, null, null, 0, ctypes.byref(d), null) == 0
+
+
+def _validate(pairs, nb):
+    import torch
+    t = torch.tensor(pairs, dtype=torch.int64).reshape(-1, 2)
+    return pkv.validate_copy_pairs(t, nb)
+
+
+def test_copy_pair_validation():
+    _validate([[0, 1], [2, 3]], 4)
+    _validate([], 4)
+    for bad in ([[0, 4]], [[-1, 2]], [[0, 1], [2, 1]], [[0, 1], [1, 2]], [[0, 1], [2, 0]]):
+        with pytest.raises(pkv.PkvError) as e:
+            _validate(bad, 4)
+        assert e.value.status == 5
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The binding and the CUDA sources never import, include or link the oracle."""
+    pkg = os.path.join(ROOT, "paged_kv_cache_375_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), f
