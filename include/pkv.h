@@ -134,7 +134,8 @@ pkv_status pkv_decode_workspace_layout(const pkv_dims *dims, int32_t max_context
  * else a multiple of 16 (e.g. 512).  workspace: device scratch of at least
  * pkv_decode_workspace_bytes() bytes, 256-byte aligned, not shared with a
  * decode that may run concurrently.  Launches a planning kernel, the decode
- * kernel and, when some sequence is split, the merge kernel, in that order.
+ * kernel and, when some sequence is split, the merge kernel, in that order
+ * (pkv_decode_plan followed by pkv_decode_run).
  */
 pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_cache,
                                       const void *v_cache, const int32_t *block_tables,
@@ -142,6 +143,29 @@ pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_ca
                                       const pkv_dims *dims, int32_t max_context_len,
                                       int32_t partition_tokens, void *workspace,
                                       size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * The two halves of pkv_paged_attention_decode, for callers that decode
+ * several layers (several cache pools) with the same context lengths: plan
+ * once per step, run once per layer.
+ *
+ * pkv_decode_plan launches the planning kernel: it reads context_lens and
+ * writes the work list into the workspace.  pkv_decode_run launches the
+ * decode kernel (and the merge kernel when some sequence is split) using the
+ * plan found in the workspace; every argument it shares with the plan call
+ * (dims, max_context_len, partition_tokens, the workspace and context_lens'
+ * contents) must be the same as at planning time, and runs using one plan
+ * must not overlap on the GPU.  After a device error, plan again.
+ */
+pkv_status pkv_decode_plan(const int32_t *context_lens, const pkv_dims *dims,
+                           int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                           size_t workspace_bytes, void *cuda_stream);
+
+pkv_status pkv_decode_run(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, const int32_t *context_lens, float scale,
+                          const pkv_dims *dims, int32_t max_context_len,
+                          int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                          void *cuda_stream);
 
 /*
  * reshape_and_cache: for every token t with slot_mapping[t] >= 0, copy the

@@ -71,6 +71,8 @@ def load_library() -> ctypes.CDLL:
             "pkv_decode_workspace_layout": (ctypes.c_int, [D, i32, i32, P, P, P]),
             "pkv_paged_attention_decode": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P,
                                                           sz, P]),
+            "pkv_decode_plan": (ctypes.c_int, [P, D, i32, i32, P, sz, P]),
+            "pkv_decode_run": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P, sz, P]),
             "pkv_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
             "pkv_copy_blocks": (ctypes.c_int, [P, P, P, i32, D, P]),
             "pkv_validate_copy_pairs": (ctypes.c_int, [P, i32, i32]),
@@ -202,6 +204,53 @@ def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Te
         float(scale), ctypes.byref(dims), mcl, partition_tokens, _p(ws), ws.numel(),
         _stream_ptr(dev)))
     return out
+
+
+class DecodePlan:
+    """A decode plan for one step: the work list built from context_lens, kept in a
+    workspace.  ``run`` decodes one layer's cache pools with it; plan once per step, run
+    once per layer (the context lengths are the same for every layer)."""
+
+    def __init__(self, block_tables: torch.Tensor, context_lens: torch.Tensor, num_q_heads: int,
+                 k_cache: torch.Tensor, *, max_context_len: int | None = None,
+                 partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None):
+        dev = context_lens.device
+        _need(block_tables, "block_tables", torch.int32, dev)
+        _need(context_lens, "context_lens", torch.int32, dev)
+        self.block_tables, self.context_lens = block_tables, context_lens
+        self.dims = make_dims(context_lens.shape[0], num_q_heads, k_cache, block_tables.shape[1])
+        self.max_context_len = (block_tables.shape[1] * k_cache.shape[2] if max_context_len is None
+                                else int(max_context_len))
+        self.partition_tokens = partition_tokens
+        need = decode_workspace_bytes(self.dims, self.max_context_len, partition_tokens)
+        if need == 0:
+            raise PkvError(2, load_library().pkv_last_error_message().decode())
+        if workspace_tensor is None:
+            workspace_tensor = torch.empty(need, dtype=torch.uint8, device=dev)
+        if workspace_tensor.numel() < need:
+            raise ValueError(f"workspace_tensor has {workspace_tensor.numel()} bytes, {need} needed")
+        self.workspace = workspace_tensor
+        _check(load_library().pkv_decode_plan(_p(context_lens), ctypes.byref(self.dims),
+                                              self.max_context_len, partition_tokens,
+                                              _p(self.workspace), self.workspace.numel(),
+                                              _stream_ptr(dev)))
+
+    def run(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+            v_cache: torch.Tensor, scale: float) -> torch.Tensor:
+        dev = q.device
+        _need(q, "q", device=dev)
+        _need(out, "out", q.dtype, dev)
+        _need(k_cache, "k_cache", q.dtype, dev)
+        _need(v_cache, "v_cache", q.dtype, dev)
+        if out.shape != q.shape or q.shape[0] != self.dims.num_seqs \
+                or tuple(k_cache.shape) != (self.dims.num_blocks, self.dims.num_kv_heads, 16,
+                                            self.dims.head_dim) or v_cache.shape != k_cache.shape:
+            raise ValueError("inconsistent shapes")
+        _check(load_library().pkv_decode_run(
+            _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
+            _p(self.context_lens), float(scale), ctypes.byref(self.dims), self.max_context_len,
+            self.partition_tokens, _p(self.workspace), self.workspace.numel(), _stream_ptr(dev)))
+        return out
 
 
 def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,

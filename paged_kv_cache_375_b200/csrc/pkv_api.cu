@@ -240,6 +240,15 @@ pkv_status launch_decode_d(const CUtensorMap& mk, const CUtensorMap& mv,
   return launch_decode<T, D, 16>(mk, mv, prm, work_units, g, stream);
 }
 
+pkv_status check_workspace(const DecodePlan& plan, const void* workspace, size_t bytes) {
+  if (!workspace) return fail(PKV_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (bytes < plan.total)
+    return fail(PKV_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", bytes, plan.total);
+  return PKV_OK;
+}
+
 template <typename T>
 pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
                         const int32_t* context_lens, const pkv_dims* d, cudaStream_t stream) {
@@ -292,12 +301,29 @@ pkv_status pkv_decode_workspace_layout(const pkv_dims* dims, int32_t max_context
   return PKV_OK;
 }
 
-pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
-                                      const void* v_cache, const int32_t* block_tables,
-                                      const int32_t* context_lens, float scale,
-                                      const pkv_dims* dims, int32_t max_context_len,
-                                      int32_t partition_tokens, void* workspace,
-                                      size_t workspace_bytes, void* cuda_stream) {
+pkv_status pkv_decode_plan(const int32_t* context_lens, const pkv_dims* dims,
+                           int32_t max_context_len, int32_t partition_tokens, void* workspace,
+                           size_t workspace_bytes, void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (dims->num_seqs == 0) return PKV_OK;
+  if (!context_lens) return fail(PKV_ERR_NULL, "context_lens is NULL");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
+      context_lens, dims->num_seqs, plan.max_len, plan.part_blocks,
+      reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off), reinterpret_cast<uint32_t*>(ws));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "plan launch");
+  return PKV_OK;
+}
+
+pkv_status pkv_decode_run(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens, float scale,
+                          const pkv_dims* dims, int32_t max_context_len,
+                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                          void* cuda_stream) {
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
@@ -305,14 +331,9 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   if (d->num_seqs == 0) return PKV_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
     return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
-  if (!workspace) return fail(PKV_ERR_WORKSPACE, "workspace is NULL");
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  if (workspace_bytes < plan.total)
-    return fail(PKV_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes,
-                plan.total);
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
   if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
   CUtensorMap mk, mv;
   if ((st = encode_pool_map(&mk, k_cache, d)) != PKV_OK) return st;
@@ -321,11 +342,6 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
   pkv::PlanItem* items = reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off);
-
-  pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, stream>>>(context_lens, d->num_seqs, plan.max_len,
-                                                       plan.part_blocks, items, counters);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "plan launch");
 
   pkv::DecodeParams prm;
   prm.out = out;
@@ -358,6 +374,31 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
                               : launch_merge<float>(out, plan, ws, context_lens, d, stream);
   }
   return st;
+}
+
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* context_lens, float scale,
+                                      const pkv_dims* dims, int32_t max_context_len,
+                                      int32_t partition_tokens, void* workspace,
+                                      size_t workspace_bytes, void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (dims->num_seqs == 0) return PKV_OK;
+  // Check everything the run needs before launching the plan.
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  st = pkv_decode_plan(context_lens, dims, max_context_len, partition_tokens, workspace,
+                       workspace_bytes, cuda_stream);
+  if (st != PKV_OK) return st;
+  return pkv_decode_run(out, q, k_cache, v_cache, block_tables, context_lens, scale, dims,
+                        max_context_len, partition_tokens, workspace, workspace_bytes,
+                        cuda_stream);
 }
 
 pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,

@@ -78,7 +78,9 @@ __device__ __forceinline__ int32_t part_size_blocks(int32_t L, int32_t p, int32_
   return rest < part_blocks ? rest : part_blocks;
 }
 
-// Single CTA.  counters[0] = work counter (zeroed here), counters[1] = items.
+// Single CTA.  counters[0] = work counter, counters[1] = items, counters[2] =
+// CTAs finished; the work and finish counters are zeroed here, and the decode
+// kernel's last CTA zeroes them again, so one plan serves any number of runs.
 __global__ void __launch_bounds__(kPlanThreads)
     plan_kernel(const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t max_len,
                 int32_t part_blocks, PlanItem* __restrict__ items,
@@ -123,6 +125,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   if (tid == kPlanThreads - 1) {
     counters[1] = warp_sums[kPlanThreads / 32 - 1];
     counters[0] = 0u;
+    counters[2] = 0u;
   }
   __syncthreads();
   for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
@@ -142,7 +145,7 @@ struct DecodeParams {
   const void* q;                 // [B][Hq][D]
   const int32_t* block_tables;   // [B][MB]
   const PlanItem* items;         // planned work, longest first
-  uint32_t* counters;            // [0] work counter, [1] number of items
+  uint32_t* counters;            // [0] work counter, [1] number of items, [2] CTAs done
   float* part_o;                 // [B][Hq][max_parts][D]
   float* part_ml;                // [B][Hq][max_parts][2]
   int32_t num_q_heads;
@@ -587,6 +590,13 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         if (lane == 0) {
           meta[r].seq = -1;
           mbar_arrive(&item_full[r]);
+          // Every CTA has made its last fetch once it gets here; the last one
+          // to finish rearms the counters for the next run of the same plan.
+          __threadfence();
+          if (atomicAdd(&prm.counters[2], 1u) == gridDim.x - 1) {
+            prm.counters[0] = 0u;
+            prm.counters[2] = 0u;
+          }
         }
         break;
       }
