@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one pass of the whole path over one synthetic batch, with every
+input already resident in HBM:
+  slot indexing of the new tokens -> reshape_and_cache -> decode plan ->
+  decode (-> log-sum-exp merge when sequences are split)
+(the shared-prefix workload also runs copy_blocks first).
+
+The default workload is the Llama-3-8B-shaped GQA batch (256 sequences, 32 q /
+8 kv heads, head_dim 128, bf16, lognormal context lengths with median 1000),
+the batched bf16 GQA configuration the throughput target is stated on.  The
+KV pools (about 2.3 GB) are far larger than the 126 MB L2, so no flush is
+needed between steps.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c5]
+  python bench.py --impl reference ...      # the float64 CPU oracle, timed
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+decodes its own replica of the batch (the path has no exchange step), the
+timed region is bracketed by barriers and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attn: KV-read GB/s (% of B200 HBM peak), seqs/s at batch"
+UNIT = "GB/s"
+WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shared_prefix",
+             "c5": "c5_long_splitk", "c1": "c1_tiny_fp32"}
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+
+
+# ------------------------------------------------------------------ helpers
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_375_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
+    the current decode sources and this workload; else None."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = rec.get(workload)
+    if not entry or entry.get("source_hash") != decode_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def algorithmic_bytes(b: workloads.Batch) -> dict:
+    """Bytes a decode launch must move at least: every context token's K and V once per kv
+    head, q, out, the block-table entries in use and the context lengths."""
+    lens = b.context_lens.astype(np.int64)
+    table = int(((lens + 15) // 16).sum()) * 4
+    qo = 2 * b.num_seqs * b.num_q_heads * b.head_dim * b.elem_bytes
+    kv = b.kv_bytes()
+    return {"kv": kv, "q_out": qo, "table": table, "lens": 4 * b.num_seqs,
+            "total": kv + qo + table + 4 * b.num_seqs}
+
+
+class ClockSampler:
+    """Samples the GPU's SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, local_rank: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.period = [], 0, period_s
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            index = int(vis.split(",")[local_rank]) if vis else local_rank
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report no clocks rather than fail the run
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                get = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                self.reasons |= get(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of x over all ranks (the slowest rank sets the job's time)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_rank: float, world: int, seconds: float) -> float:
+    """Aggregate throughput: units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / seconds
+
+
+# ------------------------------------------------------------------ our arm
+class Step:
+    """The hot path over one batch through the public API (device-resident inputs)."""
+
+    def __init__(self, b: workloads.Batch, partition_tokens: int):
+        import paged_kv_cache_375_b200 as pkv
+        self.pkv, self.b = pkv, b
+        dev = b.q.device
+        self.dev = dev
+        self.bt = torch.from_numpy(b.block_tables).to(dev)
+        self.cl = torch.from_numpy(b.context_lens).to(dev)
+        self.out = torch.empty_like(b.q)
+        self.mcl = max(b.max_context_len, 1)
+        self.partition = partition_tokens
+        self.dims = pkv.make_dims(b.num_seqs, b.num_q_heads, b.k_cache, b.max_blocks_per_seq)
+        self.part_tokens = pkv.decode_partition_tokens(self.dims, self.mcl, partition_tokens)
+        self.split = self.part_tokens < self.mcl
+        ws = pkv.decode_workspace_bytes(self.dims, self.mcl, partition_tokens)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.T = int(b.new_seq.shape[0])
+        self.decode_mode = self.T == b.num_seqs and np.array_equal(b.new_seq, np.arange(b.num_seqs)) \
+            and np.array_equal(b.new_pos, b.context_lens - 1)
+        self.seq = torch.from_numpy(b.new_seq).to(dev)
+        self.pos = torch.from_numpy(b.new_pos).to(dev)
+        self.slots = torch.empty(max(self.T, 1), dtype=torch.int64, device=dev)
+        self.pairs = torch.from_numpy(b.cow_pairs).to(dev) if b.cow_pairs.shape[0] else None
+        if self.pairs is not None:
+            pkv.validate_copy_pairs(torch.from_numpy(b.cow_pairs), b.num_blocks)
+
+    def launches_per_step(self) -> int:
+        n = 2 + (1 if self.split else 0)              # plan, decode (, merge)
+        n += 2 if self.T else 0                        # slot indexing, reshape_and_cache
+        n += 1 if self.pairs is not None else 0        # copy_blocks
+        return n
+
+    def cache_ops(self):
+        pkv, b = self.pkv, self.b
+        if self.pairs is not None:
+            pkv.copy_blocks(b.k_cache, b.v_cache, self.pairs, validate=False)
+        if self.T:
+            if self.decode_mode:
+                pkv.slot_mapping(self.bt, b.num_blocks, context_lens=self.cl, out=self.slots)
+            else:
+                pkv.slot_mapping(self.bt, b.num_blocks, token_seq=self.seq, token_pos=self.pos,
+                                 out=self.slots)
+            pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, self.slots[:self.T])
+
+    def plan(self):
+        self.plan_obj = self.pkv.DecodePlan(self.bt, self.cl, self.b.num_q_heads, self.b.k_cache,
+                                            max_context_len=self.mcl,
+                                            partition_tokens=self.partition,
+                                            workspace_tensor=self.ws)
+
+    def decode(self):
+        self.plan_obj.run(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.b.scale)
+
+    def __call__(self):
+        self.cache_ops()
+        self.plan()
+        self.decode()
+
+
+def run_ours(args, world, rank, local):
+    import paged_kv_cache_375_b200 as pkv
+    from paged_kv_cache_375_b200 import build as pkv_build
+    if not pkv_build.up_to_date():
+        pkv_build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    name = WORKLOADS[args.workload]
+    b = workloads.BUILDERS[name](device=dev)
+    step = Step(b, args.partition)
+    alg = algorithmic_bytes(b)
+    kv_bytes = b.kv_bytes() if name != "c4_shared_prefix" else b.unique_kv_bytes()
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    pkv.check_device_error(dev)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            step.cache_ops()
+            ev[i][1].record(stream)
+            step.plan()
+            ev[i][2].record(stream)
+            step.decode()
+            ev[i][3].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    pkv.check_device_error(dev)
+    total_ms = start.elapsed_time(end)
+    cache_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    plan_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / K
+    seconds = total_ms / 1e3
+    value = whole_job_value(kv_bytes * K / 1e9, world, seconds)
+    peak, peak_kind = hbm_peak()
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(step, args, world, dev, kv_bytes)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": b.dtype, "data": "synthetic",
+        "config": {
+            "workload": f"{name}: {workloads.CONFIGS[name]}",
+            "batch": b.num_seqs, "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads,
+            "head_dim": b.head_dim, "block_size": 16, "num_blocks": b.num_blocks,
+            "context_tokens": int(b.context_lens.sum()), "max_context_len": b.max_context_len,
+            "new_tokens_per_step": step.T, "cow_pairs_per_step": int(b.cow_pairs.shape[0]),
+            "partition_tokens": step.part_tokens, "split_k": step.split,
+            "kv_bytes_per_step": kv_bytes,
+            "l2": "inputs larger than L2 (KV pools >> 126 MB); no flush between steps",
+            "parallelism": f"replicas x{world} (no data-path collective)",
+        },
+        "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
+        "seqs_per_s": round(whole_job_value(b.num_seqs * K, world, seconds), 1),
+        "breakdown_ms": {"cache_ops": round(cache_ms, 5), "plan": round(plan_ms, 5),
+                         "decode": round(decode_ms, 5)},
+        "roofline": {
+            "kernel": "decode_kernel" + (" + merge_kernel" if step.split else ""),
+            "bound": "hbm", "achieved": round(alg["total"] / (decode_ms / 1e3) / 1e9, 2),
+            "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)",
+            "unit": "GB/s", "frac": round(alg["total"] / (decode_ms / 1e3) / 1e9 / peak, 4),
+            "traffic": recorded_traffic(args.workload),
+            "algorithmic_bytes_per_launch": alg,
+        },
+        "gpu_launches": step.launches_per_step() * K,
+        "clocks": sampler.summary(),
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
+    return result
+
+
+def run_e2e(step: Step, args, world, dev, kv_bytes):
+    """Same step, but every step copies its inputs from pinned host memory to the device
+    (q, the new tokens' K/V, context lengths, block tables) and reads the output back to
+    pinned host memory, synchronising on it."""
+    b = step.b
+    host = {name: t.detach().cpu().pin_memory() for name, t in (
+        ("q", b.q), ("new_k", b.new_k), ("new_v", b.new_v), ("cl", step.cl), ("bt", step.bt))}
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        b.q.copy_(host["q"], non_blocking=True)
+        b.new_k.copy_(host["new_k"], non_blocking=True)
+        b.new_v.copy_(host["new_v"], non_blocking=True)
+        step.cl.copy_(host["cl"], non_blocking=True)
+        step.bt.copy_(host["bt"], non_blocking=True)
+        step()
+        out_host.copy_(step.out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(max(3, args.warmup // 4)):
+        one()
+    K = max(3, args.steps // 4)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(K):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world, dev)
+    return {"value": round(whole_job_value(kv_bytes * K / 1e9, world, ms / 1e3), 2), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": round(ms / K, 5), "host_sync_per_step": True}
+
+
+# ------------------------------------------------------------ oracle (CPU)
+def oracle_step(b: workloads.Batch, host: dict, seqs: np.ndarray | None, threads: int):
+    """The oracle's pass over (a sample of) the step: copies, writes, attention."""
+    import oracle
+    k, v = host["k_cache"], host["v_cache"]
+    if b.cow_pairs.shape[0]:
+        oracle.copy_blocks(k, v, b.cow_pairs)
+    if b.new_seq.shape[0]:
+        oracle.reshape_and_cache(host["new_k"], host["new_v"], k, v,
+                                 oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos))
+    if seqs is None:
+        return oracle.paged_decode(host["q"], k, v, b.block_tables, b.context_lens, b.scale,
+                                   threads=threads)
+    tasks = np.array([(s, h) for s in seqs for h in range(b.num_q_heads)], dtype=np.int32)
+    return oracle.paged_decode(host["q"], k, v, b.block_tables, b.context_lens, b.scale,
+                               tasks=tasks, threads=threads)
+
+
+def cpu_baseline(b: workloads.Batch, seconds: float) -> dict:
+    """The oracle, as it stands, on the host cores: whole steps of the workload repeated
+    for about `seconds` (at least once)."""
+    threads = len(os.sched_getaffinity(0))
+    host = b.host()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(b, host, None, threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    kv = b.kv_bytes()
+    return {"value": round(kv * reps / el / 1e9, 4), "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"{reps} full step(s) of {b.name} ({b.num_seqs} seqs x {b.num_q_heads} "
+                      f"q heads, fp64) in {el:.1f} s",
+            "seqs_per_s": round(b.num_seqs * reps / el, 2)}
+
+
+def run_reference(args, world, rank, local):
+    """The reference arm: the float64 oracle timed on the host cores, on this workload, each
+    step a bounded sample of sequences so that the whole run takes a few minutes."""
+    name = WORKLOADS[args.workload]
+    b = workloads.BUILDERS[name](device="cpu")
+    threads = len(os.sched_getaffinity(0))
+    host = b.host()
+    # size the per-step sample: calibrate on one sequence, aim at ~150 s for the whole run
+    t0 = time.perf_counter()
+    oracle_step(b, host, np.array([int(np.argmax(b.context_lens))]), threads)
+    per_seq = max((time.perf_counter() - t0) * float(b.context_lens.mean())
+                  / float(b.context_lens.max()), 1e-4)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = int(min(b.num_seqs, max(1, budget / per_seq)))
+    rng = np.random.default_rng(0)
+    sample = np.sort(rng.choice(b.num_seqs, size=n, replace=False))
+    sample_kv = int(b.context_lens[sample].astype(np.int64).sum()) * b.num_kv_heads * \
+        b.head_dim * b.elem_bytes * 2
+    for _ in range(args.warmup):
+        oracle_step(b, host, sample, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(b, host, sample, threads)
+    el = time.perf_counter() - t0
+    value = sample_kv * args.steps / el / 1e9
+    peak, _ = hbm_peak()
+    desc = f"{n} of {b.num_seqs} sequences (seeded choice) x {b.num_q_heads} q heads per step"
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": f"{name}: {workloads.CONFIGS[name]}", "batch": b.num_seqs,
+                   "sample_per_step": desc},
+        "pct_of_hbm_peak": round(100.0 * value / peak, 4),
+        "seqs_per_s": round(n * args.steps / el, 3),
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c3")
+    ap.add_argument("--partition", type=int, default=0, help="partition tokens (0 = automatic)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # rank 0 alone times the CPU oracle; other ranks have nothing to do
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        print(json.dumps(run_reference(args, world, 0, 0)), flush=True)
+        return 0
+    world, rank, local = dist_init()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    try:
+        result = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
