@@ -131,7 +131,8 @@ pkv_status pkv_decode_workspace_layout(const pkv_dims *dims, int32_t max_context
  * max_context_len (host) must be >= every context length; it sizes the
  * partitions and the workspace (a larger value is always safe; a length above
  * it is clamped and flagged PKV_DEVERR_LEN).  partition_tokens: 0 = automatic,
- * else a multiple of 16 (e.g. 512).  workspace: device scratch of at least
+ * else a multiple of 16 no larger than 8192 (e.g. 512); a sequence longer
+ * than 8192 tokens is therefore always split.  workspace: device scratch of at least
  * pkv_decode_workspace_bytes() bytes, 256-byte aligned, not shared with a
  * decode that may run concurrently.  Launches a planning kernel, the decode
  * kernel and, when some sequence is split, the merge kernel, in that order

@@ -92,7 +92,9 @@ int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested) 
                                                : static_cast<int32_t>(round_up(max_len, pkv::kBlock));
   const int64_t units = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
   const int sms = device_sm_count();
-  if (max_len <= 1024 || (units >= 2ll * sms && max_len <= 8192)) return single;
+  if (single <= pkv::kMaxItemBlocks * pkv::kBlock &&
+      (max_len <= 1024 || units >= 2ll * sms))
+    return single;
   return 512;
 }
 
@@ -103,6 +105,9 @@ pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partiti
   if (max_context_len < 0) return fail(PKV_ERR_SHAPE, "max_context_len must be >= 0");
   if (partition_tokens < 0 || partition_tokens % pkv::kBlock != 0)
     return fail(PKV_ERR_SHAPE, "partition_tokens must be 0 or a positive multiple of 16");
+  if (partition_tokens > pkv::kMaxItemBlocks * pkv::kBlock)
+    return fail(PKV_ERR_UNSUPPORTED, "partition_tokens must be <= %d",
+                pkv::kMaxItemBlocks * pkv::kBlock);
   const int64_t table_len = static_cast<int64_t>(d->max_blocks_per_seq) * pkv::kBlock;
   const int32_t max_len =
       static_cast<int32_t>(max_context_len < table_len ? max_context_len : table_len);
@@ -164,16 +169,16 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d
   return PKV_OK;
 }
 
-// Kernel configuration per element type.
-template <typename T>
-struct DecodeCfg;
-template <>
-struct DecodeCfg<__nv_bfloat16> {
+// Kernel configuration: W decode warps per CTA, S tile stages per warp.
+// fp32 tiles are twice as large, so fp32 keeps fewer stages (one for the
+// largest group size at head_dim 128, where shared memory is the limit).
+template <typename T, int D, int GMAX>
+struct DecodeCfg {
   static constexpr int W = 4, S = 4;
 };
-template <>
-struct DecodeCfg<float> {
-  static constexpr int W = 4, S = 2;
+template <int D, int GMAX>
+struct DecodeCfg<float, D, GMAX> {
+  static constexpr int W = 4, S = (D == 128 && GMAX == 16) ? 1 : 2;
 };
 
 // Largest dynamic shared memory already enabled per kernel, per device.
@@ -207,7 +212,7 @@ template <typename T, int D, int GMAX>
 pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
                          const pkv::DecodeParams& prm, int64_t work_units, int g,
                          cudaStream_t stream) {
-  constexpr int W = DecodeCfg<T>::W, S = DecodeCfg<T>::S;
+  constexpr int W = DecodeCfg<T, D, GMAX>::W, S = DecodeCfg<T, D, GMAX>::S;
   using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S>;
   const int smem = Lay::total_bytes(g);
   int dev = 0, max_optin = 0;

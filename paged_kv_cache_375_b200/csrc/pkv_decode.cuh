@@ -158,6 +158,10 @@ struct DecodeParams {
   float qk_scale_log2;           // scale * log2(e)
 };
 
+// Largest partition (in blocks) the decode kernel handles; the block-table
+// slice of every item in flight is staged in shared memory.
+constexpr int kMaxItemBlocks = 512;
+
 // Shared-memory map of the decode kernel (offsets from a 1024-aligned base).
 template <int ELEM, int D, int GMAX, int W, int S>
 struct DecodeLayout {
@@ -167,7 +171,8 @@ struct DecodeLayout {
   static constexpr int kQBytes = ((GMAX * D * ELEM) + 127) / 128 * 128;
   static constexpr int kStagesOff = 0;
   static constexpr int kRingOff = kStagesOff + W * S * kStageBytes;
-  static constexpr int kMergeOff = kRingOff + kRing * kQBytes;
+  static constexpr int kTablesOff = kRingOff + kRing * kQBytes;
+  static constexpr int kMergeOff = kTablesOff + kRing * kMaxItemBlocks * 4;
   // merge area: 2 buffers x W warps x (g*D + 2g rounded up to 4) floats, g
   // chosen at run time; every warp's slot starts 16-byte aligned.
   __host__ __device__ static int merge_floats_per_warp(int g) { return g * D + (2 * g + 3) / 4 * 4; }
@@ -176,7 +181,7 @@ struct DecodeLayout {
   }
   static constexpr int kMetaBytes = kRing * 32;
   __host__ __device__ static int bars_off(int g) { return (meta_off(g) + kMetaBytes + 7) / 8 * 8; }
-  static constexpr int kNumBars = 2 * W * S + 2 * kRing + 2;
+  static constexpr int kNumBars = W * S + 2 * kRing + 2;
   __host__ __device__ static int flags_off(int g) { return bars_off(g) + kNumBars * 8; }
   __host__ __device__ static int total_bytes(int g) {
     return flags_off(g) + (W * S + 4) * 4 + 1024;  // + slack for 1024-byte alignment
@@ -521,9 +526,17 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
   }
 }
 
-// The persistent decode kernel.  Warps 0..W-1 consume, warp W produces.
+// The persistent decode kernel.  Warps 0..W-1 decode; warp W schedules.
+//
+// The scheduler warp fetches items from the global work counter and
+// publishes each into a ring slot: its metadata, its q tile (one bulk copy)
+// and the slice of the block table it covers.  Every decode warp owns S tile
+// stages and is its own TMA producer: it keeps up to S of its blocks in
+// flight, following its share of the items (blocks w, w+W, ... of each) and
+// running ahead into the next items while it computes.  At the end of an item
+// the W warps combine their online-softmax states through shared memory.
 template <typename T, int D, int GMAX, int W, int S>
-__global__ void __launch_bounds__((W + 1) * 32, 1)
+__global__ void __launch_bounds__((W + 1) * 32)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
   constexpr int ELEM = sizeof(T);
@@ -534,12 +547,12 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   const int g = prm.group;
   uint8_t* stages = smem + Lay::kStagesOff;
   uint8_t* ring = smem + Lay::kRingOff;
+  int32_t* tables = reinterpret_cast<int32_t*>(smem + Lay::kTablesOff);  // [kRing][kMaxItemBlocks]
   float* merge = reinterpret_cast<float*>(smem + Lay::kMergeOff);
   ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + Lay::meta_off(g));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off(g));
   uint64_t* full = bars;                       // [W][S]
-  uint64_t* empty = bars + W * S;              // [W][S]
-  uint64_t* item_full = bars + 2 * W * S;      // [kRing]
+  uint64_t* item_full = bars + W * S;          // [kRing]
   uint64_t* item_empty = item_full + kRing;    // [kRing]
   uint64_t* merge_bar = item_empty + kRing;    // [2]
   uint32_t* stage_ok = reinterpret_cast<uint32_t*>(smem + Lay::flags_off(g));  // [W][S]
@@ -547,10 +560,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < W * S; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
+    for (int i = 0; i < W * S; ++i) mbar_init(&full[i], 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], W);
@@ -564,28 +574,20 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
   const int32_t hkv = prm.num_kv_heads;
   if (warp == W) {
-    // ================================ producer ================================
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_k);
-      prefetch_tensormap(&tmap_v);
-    }
+    // ================================ scheduler ================================
     const uint32_t total = prm.counters[1] * static_cast<uint32_t>(hkv);
-    const uint64_t policy = l2_policy_evict_first();
-    uint32_t stage_ctr[W];
-#pragma unroll
-    for (int w = 0; w < W; ++w) stage_ctr[w] = 0;
     uint32_t next = 0;
     if (lane == 0) next = atomicAdd(&prm.counters[0], 1u);
-    next = __shfl_sync(0xffffffffu, next, 0);
+    uint32_t item_seq = 0;
     bool ok = true;
-    for (uint32_t item_seq = 0;; ++item_seq) {
+    for (;; ++item_seq) {
       const int r = item_seq % kRing;
       if (item_seq >= kRing) {
         if (lane == 0) ok = mbar_wait(&item_empty[r], ((item_seq / kRing) - 1) & 1);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok || *abort_flag) break;
       }
-      const uint32_t widx = next;
+      const uint32_t widx = __shfl_sync(0xffffffffu, next, 0);
       if (widx >= total) {
         if (lane == 0) {
           meta[r].seq = -1;
@@ -598,17 +600,22 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
             prm.counters[2] = 0u;
           }
         }
+        ++item_seq;
         break;
       }
+      // fetch the following item now; its value is only needed next time round
       if (lane == 0) next = atomicAdd(&prm.counters[0], 1u);
-      next = __shfl_sync(0xffffffffu, next, 0);
       const PlanItem pi = prm.items[widx / hkv];
       const int32_t kvh = static_cast<int32_t>(widx % hkv);
       const int32_t blk_begin = pi.part * prm.part_blocks;
-      const int32_t nblk_total = (pi.len + kBlock - 1) / kBlock;
-      int32_t nblk = nblk_total - blk_begin;
+      int32_t nblk = (pi.len + kBlock - 1) / kBlock - blk_begin;
       nblk = nblk < prm.part_blocks ? nblk : prm.part_blocks;
       nblk = nblk < 0 ? 0 : nblk;
+      const int32_t* src = prm.block_tables +
+                           static_cast<size_t>(pi.seq) * prm.max_blocks_per_seq + blk_begin;
+      int32_t* dst = tables + r * kMaxItemBlocks;
+      for (int32_t j = lane; j < nblk; j += 32) dst[j] = src[j];
+      __syncwarp();
       if (lane == 0) {
         ItemMeta& mt = meta[r];
         mt.seq = pi.seq;
@@ -624,80 +631,98 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                               (static_cast<size_t>(pi.seq) * prm.num_q_heads + kvh * g) * D * ELEM;
         bulk_load(ring + r * Lay::kQBytes, qsrc, qbytes, &item_full[r]);
       }
-      const int32_t* table = prm.block_tables +
-                             static_cast<size_t>(pi.seq) * prm.max_blocks_per_seq + blk_begin;
-      int32_t tbl = (lane < nblk) ? table[lane] : -1;
-      for (int32_t b = 0; b < nblk; ++b) {
-        if ((b & 31) == 0 && b > 0) tbl = (b + lane < nblk) ? table[b + lane] : -1;
-        const int32_t entry = __shfl_sync(0xffffffffu, tbl, b & 31);
-        const int w = b % W;
-        uint32_t ctr = 0;
-#pragma unroll
-        for (int x = 0; x < W; ++x) ctr = (x == w) ? stage_ctr[x] : ctr;
-        const int st = ctr % S;
-        if (lane == 0) {
-          if (ctr >= S) ok = mbar_wait(&empty[w * S + st], ((ctr / S) - 1) & 1);
-          if (ok) {
-            const bool valid = entry >= 0 && entry < prm.num_blocks;
-            stage_ok[w * S + st] = valid ? 1u : 0u;
-            uint8_t* kdst = stages + (w * S + st) * Lay::kStageBytes;
-            uint8_t* vdst = kdst + Lay::kTileBytes;
-            if (valid) {
-              mbar_arrive_expect_tx(&full[w * S + st], 2 * Lay::kTileBytes);
-              const int32_t y = (entry * hkv + kvh) * kBlock;
-#pragma unroll
-              for (int c = 0; c < Lay::kChunks; ++c) {
-                tma_load_2d_hint(kdst + c * (kBlock * 128), &tmap_k, c * (128 / ELEM), y,
-                                 &full[w * S + st], policy);
-                tma_load_2d_hint(vdst + c * (kBlock * 128), &tmap_v, c * (128 / ELEM), y,
-                                 &full[w * S + st], policy);
-              }
-            } else {
-              raise_error(PKV_DEVERR_BLOCK);
-              mbar_arrive(&full[w * S + st]);
-            }
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-#pragma unroll
-        for (int x = 0; x < W; ++x) stage_ctr[x] += (x == w) ? 1u : 0u;
-      }
-      if (!ok || *abort_flag) break;
     }
     if (!ok) {
-      // A wait gave up: tell the consumers, then wait (briefly, bounded) for
-      // the tile copies this warp issued, so none lands after the CTA exits.
+      // A wait gave up: tell the decode warps, then wait (bounded) for the q
+      // copies still in flight into the ring, so none lands after exit.
       *abort_flag = 1u;
       if (lane == 0) {
-#pragma unroll
-        for (int w = 0; w < W; ++w) {
-#pragma unroll
-          for (int s2 = 0; s2 < S; ++s2) {
-            const uint32_t c = stage_ctr[w];
-            if (c > static_cast<uint32_t>(s2)) {
-              const uint32_t issues = (c - 1 - s2) / S + 1;
-              mbar_wait(&full[w * S + s2], (issues - 1) & 1, 100000000ull);
-            }
-          }
+        for (uint32_t j = item_seq > kRing ? item_seq - kRing : 0; j < item_seq; ++j) {
+          mbar_wait(&item_full[j % kRing], (j / kRing) & 1, kDrainLimitCycles);
         }
       }
     }
     return;
   }
 
-  // ================================ consumers ================================
+  // ================================ decode warps ================================
   using Bst = Bf16State<D, GMAX>;
   using Fst = F32State<D, GMAX>;
   constexpr bool kBf16 = sizeof(T) == 2;
   typename std::conditional<kBf16, Bst, Fst>::type st;
-  uint32_t stage_ctr = 0;
   const float sc = prm.qk_scale_log2;
   const int per_warp = Lay::merge_floats_per_warp(g);
-  for (uint32_t item_seq = 0;; ++item_seq) {
-    const int r = item_seq % kRing;
-    if (!mbar_wait(&item_full[r], (item_seq / kRing) & 1)) {
-      *abort_flag = 1u;
+  uint64_t* my_full = full + warp * S;
+  uint32_t* my_ok = stage_ok + warp * S;
+  uint8_t* my_stages = stages + warp * S * Lay::kStageBytes;
+
+  // Producer cursor over this warp's blocks: item p_item, block p_blk of it.
+  uint32_t cctr = 0, pctr = 0;       // blocks consumed / issued by this warp
+  uint32_t c_item = 0;               // item being consumed
+  uint32_t p_item = 0;
+  int32_t p_blk = warp;
+  bool p_known = false, p_end = false;
+  ItemMeta pm{};
+  bool ok = true;
+
+  // Issue this warp's next blocks until S are in flight.  With `blocking` the
+  // wait for an item's metadata may block (only when the block is needed now).
+  auto produce = [&](bool blocking) {
+    while (pctr < cctr + S && !p_end) {
+      if (!p_known) {
+        if (p_item >= c_item + kRing) return;          // that slot still holds an older item
+        const int r = p_item % kRing;
+        const uint32_t par = (p_item / kRing) & 1;
+        if (blocking) {
+          if (!mbar_wait(&item_full[r], par)) {
+            ok = false;
+            return;
+          }
+        } else if (!mbar_try_wait(&item_full[r], par)) {
+          return;
+        }
+        pm = meta[r];
+        if (pm.seq < 0) {
+          p_end = true;
+          return;
+        }
+        p_known = true;
+      }
+      if (p_blk >= pm.nblk) {
+        ++p_item;
+        p_blk = warp;
+        p_known = false;
+        continue;
+      }
+      const int s_idx = pctr % S;
+      const int32_t entry = tables[(p_item % kRing) * kMaxItemBlocks + p_blk];
+      if (lane == 0) {
+        const bool valid = entry >= 0 && entry < prm.num_blocks;
+        my_ok[s_idx] = valid ? 1u : 0u;
+        uint8_t* kdst = my_stages + s_idx * Lay::kStageBytes;
+        uint8_t* vdst = kdst + Lay::kTileBytes;
+        if (valid) {
+          mbar_arrive_expect_tx(&my_full[s_idx], 2 * Lay::kTileBytes);
+          const int32_t y = (entry * hkv + pm.kv_head) * kBlock;
+#pragma unroll
+          for (int c = 0; c < Lay::kChunks; ++c) {
+            tma_load_2d(kdst + c * (kBlock * 128), &tmap_k, c * (128 / ELEM), y, &my_full[s_idx]);
+            tma_load_2d(vdst + c * (kBlock * 128), &tmap_v, c * (128 / ELEM), y, &my_full[s_idx]);
+          }
+        } else {
+          raise_error(PKV_DEVERR_BLOCK);
+          mbar_arrive(&my_full[s_idx]);
+        }
+      }
+      p_blk += W;
+      ++pctr;
+    }
+  };
+
+  for (;; ++c_item) {
+    const int r = c_item % kRing;
+    if (!mbar_wait(&item_full[r], (c_item / kRing) & 1)) {
+      ok = false;
       break;
     }
     const ItemMeta it = meta[r];
@@ -708,15 +733,23 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     } else {
       f32_begin_item<D, GMAX>(st);
     }
-    bool ok = true;
     for (int32_t b = warp; b < it.nblk; b += W) {
-      const int s_idx = stage_ctr % S;
-      ok = mbar_wait(&full[warp * S + s_idx], (stage_ctr / S) & 1);
-      if (!ok) break;
+      if (cctr == pctr) {
+        produce(true);
+        if (!ok || cctr == pctr) {
+          ok = false;
+          break;
+        }
+      }
+      const int s_idx = cctr % S;
+      if (!mbar_wait(&my_full[s_idx], (cctr / S) & 1)) {
+        ok = false;
+        break;
+      }
       int valid = it.len - (it.blk_begin + b) * kBlock;
       valid = valid > kBlock ? kBlock : valid;
-      if (!stage_ok[warp * S + s_idx]) valid = 0;
-      const uint8_t* kt = stages + (warp * S + s_idx) * Lay::kStageBytes;
+      if (!my_ok[s_idx]) valid = 0;
+      const uint8_t* kt = my_stages + s_idx * Lay::kStageBytes;
       if constexpr (kBf16) {
         bf16_block<D, GMAX>(st, kt, kt + Lay::kTileBytes, valid, sc, lane);
       } else {
@@ -724,18 +757,16 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                            sc, g, lane);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[warp * S + s_idx]);
-      ++stage_ctr;
+      ++cctr;
+      produce(false);
     }
-    if (!ok) {
-      *abort_flag = 1u;
-      break;
-    }
-    // The q tile and the metadata have been read: free the ring slot.
+    if (!ok) break;
+    // The q tile, metadata and table slice of this item are no longer needed.
     __syncwarp();
     if (lane == 0) mbar_arrive(&item_empty[r]);
+    produce(false);
     // ---- merge the W warps' states ----
-    const int mb = item_seq & 1;
+    const int mb = c_item & 1;
     float* mslot = merge + (mb * W + warp) * per_warp;
     if constexpr (kBf16) {
       bf16_publish<D, GMAX>(st, mslot, g, lane);
@@ -744,11 +775,19 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&merge_bar[mb]);
-    if (!mbar_wait(&merge_bar[mb], (item_seq >> 1) & 1)) {
-      *abort_flag = 1u;
+    if (!mbar_wait(&merge_bar[mb], (c_item >> 1) & 1)) {
+      ok = false;
       break;
     }
     combine_and_store<T, D, W>(prm, it, merge + mb * W * per_warp, per_warp, g, warp, lane);
+  }
+  if (!ok) {
+    // A wait gave up: raise the abort flag and wait (bounded) for the copies
+    // this warp still has in flight.
+    *abort_flag = 1u;
+    for (uint32_t k = cctr; k < pctr; ++k) {
+      mbar_wait(&my_full[k % S], (k / S) & 1, kDrainLimitCycles);
+    }
   }
 }
 

@@ -22,14 +22,11 @@ __device__ __forceinline__ void raise_error(unsigned int bits) {
   atomicOr(&g_device_error, bits);
 }
 
-// Every wait on the GPU gives up after this many nanoseconds of %globaltimer.
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;
-
-__device__ __forceinline__ unsigned long long global_timer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
+// Every wait on the GPU gives up after this many SM clock cycles (about four
+// seconds at the B200's 1.965 GHz boost clock; longer at lower clocks).
+constexpr long long kWaitLimitCycles = 8000000000ll;
+// Shorter bound used when draining copies after a wait has already failed.
+constexpr long long kDrainLimitCycles = 200000000ll;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -79,16 +76,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// raises PKV_DEVERR_TIMEOUT) if it has not completed within limit_ns.
+// raises PKV_DEVERR_TIMEOUT) if it has not completed within limit_cycles SM
+// cycles.  The clock is only read after a burst of fast polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          unsigned long long limit_ns = kWaitLimitNs) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_timer_ns();
+                                          long long limit_cycles = kWaitLimitCycles) {
+#pragma unroll 1
+  for (int i = 0; i < 256; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+  }
+  const long long t0 = clock64();
   for (;;) {
-    for (int i = 0; i < 64; ++i) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i) {
       if (mbar_try_wait(bar, parity)) return true;
     }
-    if (global_timer_ns() - t0 > limit_ns) {
+    if (clock64() - t0 > limit_cycles) {
       raise_error(PKV_DEVERR_TIMEOUT);
       return false;
     }
