@@ -29,7 +29,11 @@
  *    per-device error word; pkv_check_device_error() reads and clears it.  No
  *    kernel traps, asserts or waits without a bound: every internal wait gives
  *    up after about four seconds and reports PKV_DEVERR_TIMEOUT.
- *  - All device pointers must be 16-byte aligned.
+ *  - All device pointers must be 16-byte aligned.  Calls that launch work make
+ *    the device owning their output buffer current (the library carries its
+ *    own CUDA runtime, so the caller's current device is not seen); a host
+ *    pointer where device memory is expected is rejected with PKV_ERR_SHAPE.
+ *    The stream must belong to that device.
  *
  * Layouts (row-major, innermost last):
  *  - q, out         [num_seqs][num_q_heads][head_dim], dtype of the cache
@@ -216,7 +220,8 @@ pkv_status pkv_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
 
 /*
  * Synchronises cuda_stream, then reads and clears the error word of the
- * current device.  *bits_out (may be NULL) receives the PKV_DEVERR_* bits.
+ * device that owns the stream (the library's current device for a NULL
+ * stream).  *bits_out (may be NULL) receives the PKV_DEVERR_* bits.
  * Returns PKV_OK, PKV_ERR_DEVICE_TIMEOUT (timeout bit set),
  * PKV_ERR_DEVICE_INDEX (other bits) or PKV_ERR_CUDA.
  */

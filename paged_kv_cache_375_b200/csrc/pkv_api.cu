@@ -37,6 +37,29 @@ pkv_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Make the device that owns `p` current for this library's runtime.  The
+// library carries its own CUDA runtime, whose current device is independent
+// of the caller's (e.g. PyTorch's), so every call that launches work binds
+// the device of its output buffer first.  Also rejects host pointers.
+pkv_status bind_device(const void* p, const char* what) {
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(e, "cudaPointerGetAttributes");
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(PKV_ERR_SHAPE, "%s is not device memory", what);
+  int cur = -1;
+  e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (cur != a.device) {
+    e = cudaSetDevice(a.device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  }
+  return PKV_OK;
+}
+
 int elem_bytes(pkv_dtype t) { return t == PKV_BF16 ? 2 : 4; }
 
 // Checks shared by every call.  `need_seq` also checks the per-sequence fields.
@@ -315,6 +338,7 @@ pkv_status pkv_decode_plan(const int32_t* context_lens, const pkv_dims* dims,
   if (dims->num_seqs == 0) return PKV_OK;
   if (!context_lens) return fail(PKV_ERR_NULL, "context_lens is NULL");
   if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  if ((st = bind_device(workspace, "workspace")) != PKV_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
       context_lens, dims->num_seqs, plan.max_len, plan.part_blocks,
@@ -340,6 +364,7 @@ pkv_status pkv_decode_run(void* out, const void* q, const void* k_cache, const v
     return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
   if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
   if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  if ((st = bind_device(out, "out")) != PKV_OK) return st;
   CUtensorMap mk, mv;
   if ((st = encode_pool_map(&mk, k_cache, d)) != PKV_OK) return st;
   if ((st = encode_pool_map(&mv, v_cache, d)) != PKV_OK) return st;
@@ -417,6 +442,7 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, vo
     return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
   if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
     return fail(PKV_ERR_ALIGN, "k, v and the caches must be 16-byte aligned");
+  if ((st = bind_device(k_cache, "k_cache")) != PKV_OK) return st;
   const int row_bytes = dims->head_dim * elem_bytes(dims->dtype);
   const int units = dims->num_kv_heads * row_bytes / 16;
   int threads = units < 256 ? (units + 31) / 32 * 32 : 256;
@@ -438,6 +464,7 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs,
   if (!k_cache || !v_cache || !pairs) return fail(PKV_ERR_NULL, "a pointer is NULL");
   if (!aligned16(k_cache) || !aligned16(v_cache))
     return fail(PKV_ERR_ALIGN, "the caches must be 16-byte aligned");
+  if ((st = bind_device(k_cache, "k_cache")) != PKV_OK) return st;
   const int64_t block_bytes = static_cast<int64_t>(dims->num_kv_heads) * pkv::kBlock *
                               dims->head_dim * elem_bytes(dims->dtype);
   const unsigned chunks =
@@ -486,6 +513,7 @@ pkv_status pkv_slot_mapping(int64_t* slot_mapping, const int32_t* block_tables,
     return fail(PKV_ERR_NULL, "context_lens is needed when token_pos is NULL");
   if (!token_seq && num_tokens > dims->num_seqs)
     return fail(PKV_ERR_SHAPE, "without token_seq there is one token per sequence");
+  if ((st = bind_device(slot_mapping, "slot_mapping")) != PKV_OK) return st;
   const unsigned grid = static_cast<unsigned>((num_tokens + 255) / 256);
   pkv::slot_mapping_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
       slot_mapping, block_tables, context_lens, token_seq, token_pos, num_tokens, dims->num_seqs,
@@ -496,7 +524,18 @@ pkv_status pkv_slot_mapping(int64_t* slot_mapping, const int32_t* block_tables,
 }
 
 pkv_status pkv_check_device_error(void* cuda_stream, uint32_t* bits_out) {
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  cudaError_t e;
+  if (cuda_stream) {
+    // read the error word of the device that owns the stream
+    int dev = -1, cur = -1;
+    e = cudaStreamGetDevice(static_cast<cudaStream_t>(cuda_stream), &dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamGetDevice");
+    if (cudaGetDevice(&cur) == cudaSuccess && cur != dev) {
+      e = cudaSetDevice(dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    }
+  }
+  e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   unsigned int bits = 0;
   e = cudaMemcpyFromSymbol(&bits, pkv::g_device_error, sizeof bits);
