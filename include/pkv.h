@@ -173,6 +173,37 @@ pkv_status pkv_decode_run(void *out, const void *q, const void *k_cache, const v
                           void *cuda_stream);
 
 /*
+ * Decode with built-in scratch, for callers that cannot allocate device
+ * memory.  There is no counterpart in the paper: it is a convenience of this
+ * library.  Some callers cannot call cudaMalloc themselves -- for instance an
+ * engine that hands almost all HBM to its KV-cache pool at start-up and lets
+ * nothing else allocate, or a host runtime that reaches this library only
+ * through the C ABI and owns no device allocator.  This entry point takes the
+ * same arguments as pkv_paged_attention_decode minus the workspace: the
+ * scratch is a fixed array of PKV_STATIC_WORKSPACE_BYTES inside the library,
+ * reserved on every GPU that loads the library until the process exits.
+ *  - The call allocates nothing.  The first call on a device looks up that
+ *    array's device address (cudaGetSymbolAddress, with that device current)
+ *    and caches it; make that first call before any stream capture.
+ *  - A decode whose pkv_decode_workspace_bytes() exceeds
+ *    PKV_STATIC_WORKSPACE_BYTES is rejected with PKV_ERR_WORKSPACE (the
+ *    message gives both sizes); use pkv_paged_attention_decode with a
+ *    caller-provided workspace instead.
+ *  - All calls in the process share the one array per device, and each call
+ *    leaves its contents behind.  Nothing in it needs to start at zero (the
+ *    planning kernel resets the counters it uses), but calls that overlap on
+ *    the GPU -- on different streams, or from different host threads -- race
+ *    on it and must be serialised by the caller.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (32u << 20)
+
+pkv_status pkv_paged_attention_decode_static(void *out, const void *q, const void *k_cache,
+                                             const void *v_cache, const int32_t *block_tables,
+                                             const int32_t *context_lens, float scale,
+                                             const pkv_dims *dims, int32_t max_context_len,
+                                             int32_t partition_tokens, void *cuda_stream);
+
+/*
  * reshape_and_cache: for every token t with slot_mapping[t] >= 0, copy the
  * bytes of k[t][h][:] and v[t][h][:] to k_cache / v_cache at block
  * slot/16, kv head h, offset slot%16, for every kv head h.  The copy is

@@ -298,6 +298,33 @@ pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
   return PKV_OK;
 }
 
+// Scratch for pkv_paged_attention_decode_static: callers that cannot
+// allocate device memory use this fixed array instead of a workspace of their
+// own.  Every device that loads the library holds it until the process exits.
+static __device__ __align__(256) uint8_t g_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mu;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device (host code cannot use the array's name as a device pointer).
+pkv_status static_workspace(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_ws_mu);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    g_static_ws_ptr[dev] = p;
+  }
+  *ptr = g_static_ws_ptr[dev];
+  return PKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -429,6 +456,26 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   return pkv_decode_run(out, q, k_cache, v_cache, block_tables, context_lens, scale, dims,
                         max_context_len, partition_tokens, workspace, workspace_bytes,
                         cuda_stream);
+}
+
+pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_cache,
+                                             const void* v_cache, const int32_t* block_tables,
+                                             const int32_t* context_lens, float scale,
+                                             const pkv_dims* dims, int32_t max_context_len,
+                                             int32_t partition_tokens, void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (plan.total > PKV_STATIC_WORKSPACE_BYTES)
+    return fail(PKV_ERR_WORKSPACE,
+                "this decode needs %zu bytes of scratch but the built-in scratch holds %u; "
+                "call pkv_paged_attention_decode with a workspace of your own",
+                plan.total, (unsigned)PKV_STATIC_WORKSPACE_BYTES);
+  void* ws = nullptr;
+  if ((st = static_workspace(&ws)) != PKV_OK) return st;
+  return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                    dims, max_context_len, partition_tokens, ws,
+                                    PKV_STATIC_WORKSPACE_BYTES, cuda_stream);
 }
 
 pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
