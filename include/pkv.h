@@ -117,9 +117,12 @@ size_t pkv_decode_workspace_bytes(const pkv_dims *dims, int32_t max_context_len,
 /*
  * Offsets inside the workspace of the split-K partial results, for tests that
  * inspect them: part_o is float [B][Hq][max_parts][D] (each partition's
- * normalised output), part_ml is float [B][Hq][max_parts][2] = (m, l) with m
- * the partition's max of scale*q.k and l = sum exp(scale*q.k - m).  Only
- * partitions of sequences with more than one partition are written.
+ * normalised output), part_ml is float [B][Hq][max_parts][2] = (m, l) with
+ * l = sum exp(scale*q.k - m) over the partition.  m is the partition's max of
+ * scale*q.k for fp32; for bf16 it is a reference value at most 8 ln 2 below
+ * that max (the kernel only moves its running max when it grows by more than
+ * that), which the merge treats the same way.  Only partitions of sequences
+ * with more than one partition are written.
  * Returns PKV_ERR_SHAPE when the decode would run single-pass.
  */
 pkv_status pkv_decode_workspace_layout(const pkv_dims *dims, int32_t max_context_len,

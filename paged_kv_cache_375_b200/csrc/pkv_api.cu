@@ -35,6 +35,25 @@ pkv_status cuda_fail(cudaError_t e, const char* what) {
   return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// Launch with programmatic stream serialisation, so the kernel can begin while
+// the previous kernel in the stream drains (every kernel here waits for its
+// prerequisites with griddepcontrol.wait before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Make the device that owns `p` current for this library's runtime.  The
@@ -106,19 +125,20 @@ struct DecodePlan {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Partition choice.  Single pass when there are enough (sequence, kv head)
-// units to fill the GPU several times over and no sequence is very long;
-// otherwise 512-token partitions.
+// Partition choice.  Aim at about 16 items of work per SM at the longest
+// length: P = the power of two >= B*Hkv*max_len / (16*SMs), within
+// [512, 8192] tokens.  When that covers the longest sequence the decode is
+// single-pass (the planner then orders whole sequences longest first).
 int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested) {
   if (requested > 0) return requested;
-  const int32_t single = max_len < pkv::kBlock ? pkv::kBlock
-                                               : static_cast<int32_t>(round_up(max_len, pkv::kBlock));
   const int64_t units = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
-  const int sms = device_sm_count();
-  if (single <= pkv::kMaxItemBlocks * pkv::kBlock &&
-      (max_len <= 1024 || units >= 2ll * sms))
-    return single;
-  return 512;
+  const int64_t target = units * max_len / (16ll * device_sm_count());
+  int64_t p = 512;
+  while (p < target && p < pkv::kMaxItemBlocks * pkv::kBlock) p *= 2;
+  if (p >= max_len)
+    return max_len < pkv::kBlock ? pkv::kBlock
+                                 : static_cast<int32_t>(round_up(max_len, pkv::kBlock));
+  return static_cast<int32_t>(p);
 }
 
 pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partition_tokens,
@@ -192,12 +212,16 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d
   return PKV_OK;
 }
 
-// Kernel configuration: W decode warps per CTA, S tile stages per warp.
-// fp32 tiles are twice as large, so fp32 keeps fewer stages (one for the
-// largest group size at head_dim 128, where shared memory is the limit).
+// Kernel configuration: W decode warps per CTA (one CTA per SM), S tile
+// stages per warp.  Eight decode warps with two stages each hide the latency
+// of the per-tile math best (measured on B200); groups of more than 8 query
+// heads at head_dim 128 need a merge area too large for that, and use four
+// warps with four stages.  fp32 tiles are twice as large, so fp32 keeps
+// fewer stages (one for the largest group at head_dim 128).
 template <typename T, int D, int GMAX>
 struct DecodeCfg {
-  static constexpr int W = 4, S = 4;
+  static constexpr bool kBig = (D == 128 && GMAX == 16);
+  static constexpr int W = kBig ? 4 : 8, S = kBig ? 4 : 2;
 };
 template <int D, int GMAX>
 struct DecodeCfg<float, D, GMAX> {
@@ -254,8 +278,8 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
   int64_t grid = static_cast<int64_t>(device_sm_count()) * per_sm;
   if (grid > work_units) grid = work_units;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), (W + 1) * 32, smem, stream>>>(mk, mv, prm);
-  e = cudaGetLastError();
+  e = launch(kern, dim3(static_cast<unsigned>(grid)), dim3((W + 1) * 32), smem, stream, mk, mv,
+             prm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return PKV_OK;
 }
@@ -284,16 +308,10 @@ pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
   const float* po = reinterpret_cast<const float*>(ws + plan.part_o_off);
   const float* pml = reinterpret_cast<const float*>(ws + plan.part_ml_off);
-  if (d->head_dim == 128) {
-    pkv::merge_kernel<T, 128><<<grid, 128, 0, stream>>>(out, po, pml, context_lens, d->num_seqs,
-                                                        d->num_q_heads, plan.max_parts,
-                                                        plan.max_len, plan.part_tokens);
-  } else {
-    pkv::merge_kernel<T, 64><<<grid, 128, 0, stream>>>(out, po, pml, context_lens, d->num_seqs,
-                                                       d->num_q_heads, plan.max_parts,
-                                                       plan.max_len, plan.part_tokens);
-  }
-  cudaError_t e = cudaGetLastError();
+  auto kern = d->head_dim == 128 ? pkv::merge_kernel<T, 128> : pkv::merge_kernel<T, 64>;
+  cudaError_t e = launch(kern, dim3(grid), dim3(128), 0, stream, out, po, pml, context_lens,
+                         d->num_seqs, d->num_q_heads, plan.max_parts, plan.max_len,
+                         plan.part_tokens);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return PKV_OK;
 }
@@ -367,10 +385,11 @@ pkv_status pkv_decode_plan(const int32_t* context_lens, const pkv_dims* dims,
   if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
   if ((st = bind_device(workspace, "workspace")) != PKV_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  pkv::plan_kernel<<<1, pkv::kPlanThreads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
-      context_lens, dims->num_seqs, plan.max_len, plan.part_blocks,
-      reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off), reinterpret_cast<uint32_t*>(ws));
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch(pkv::plan_kernel, dim3(1), dim3(pkv::kPlanThreads), 0,
+                         static_cast<cudaStream_t>(cuda_stream), context_lens, dims->num_seqs,
+                         plan.max_len, plan.part_blocks,
+                         reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off),
+                         reinterpret_cast<uint32_t*>(ws));
   if (e != cudaSuccess) return cuda_fail(e, "plan launch");
   return PKV_OK;
 }
@@ -493,11 +512,11 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, vo
   const int row_bytes = dims->head_dim * elem_bytes(dims->dtype);
   const int units = dims->num_kv_heads * row_bytes / 16;
   int threads = units < 256 ? (units + 31) / 32 * 32 : 256;
-  pkv::reshape_and_cache_kernel<<<num_tokens, threads, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
-      static_cast<uint8_t*>(v_cache), slot_mapping, dims->num_kv_heads, row_bytes,
-      static_cast<int64_t>(dims->num_blocks) * pkv::kBlock);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch(pkv::reshape_and_cache_kernel, dim3(num_tokens), dim3(threads), 0,
+                         static_cast<cudaStream_t>(cuda_stream), static_cast<const uint4*>(k),
+                         static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
+                         static_cast<uint8_t*>(v_cache), slot_mapping, dims->num_kv_heads,
+                         row_bytes, static_cast<int64_t>(dims->num_blocks) * pkv::kBlock);
   if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
   return PKV_OK;
 }
@@ -518,10 +537,9 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs,
       static_cast<unsigned>((block_bytes + pkv::kCopyChunk - 1) / pkv::kCopyChunk);
   if (chunks > 65535) return fail(PKV_ERR_UNSUPPORTED, "block too large for copy_blocks");
   dim3 grid(static_cast<unsigned>(num_pairs), chunks, 2);
-  pkv::copy_blocks_kernel<<<grid, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
-      static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), pairs, block_bytes,
-      dims->num_blocks);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch(pkv::copy_blocks_kernel, grid, dim3(32), 0,
+                         static_cast<cudaStream_t>(cuda_stream), static_cast<uint8_t*>(k_cache),
+                         static_cast<uint8_t*>(v_cache), pairs, block_bytes, dims->num_blocks);
   if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
   return PKV_OK;
 }
@@ -562,10 +580,10 @@ pkv_status pkv_slot_mapping(int64_t* slot_mapping, const int32_t* block_tables,
     return fail(PKV_ERR_SHAPE, "without token_seq there is one token per sequence");
   if ((st = bind_device(slot_mapping, "slot_mapping")) != PKV_OK) return st;
   const unsigned grid = static_cast<unsigned>((num_tokens + 255) / 256);
-  pkv::slot_mapping_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(
-      slot_mapping, block_tables, context_lens, token_seq, token_pos, num_tokens, dims->num_seqs,
-      dims->max_blocks_per_seq, dims->num_blocks);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch(pkv::slot_mapping_kernel, dim3(grid), dim3(256), 0,
+                         static_cast<cudaStream_t>(cuda_stream), slot_mapping, block_tables,
+                         context_lens, token_seq, token_pos, num_tokens, dims->num_seqs,
+                         dims->max_blocks_per_seq, dims->num_blocks);
   if (e != cudaSuccess) return cuda_fail(e, "slot_mapping launch");
   return PKV_OK;
 }

@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(256)
                         const int32_t* __restrict__ token_seq,
                         const int32_t* __restrict__ token_pos, int32_t num_tokens,
                         int32_t num_seqs, int32_t max_blocks_per_seq, int32_t num_blocks) {
+  pdl_wait();
+  pdl_trigger();
   const int32_t t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= num_tokens) return;
   const int32_t seq = token_seq ? token_seq[t] : t;
@@ -54,6 +56,8 @@ __global__ void __launch_bounds__(256)
                              uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
                              const int64_t* __restrict__ slot_mapping, int32_t num_kv_heads,
                              int32_t row_bytes, int64_t num_slots) {
+  pdl_wait();
+  pdl_trigger();
   const int32_t t = blockIdx.x;
   const int64_t slot = slot_mapping[t];
   if (slot < 0) return;  // padding token
@@ -90,6 +94,8 @@ __global__ void __launch_bounds__(32)
                        int32_t num_blocks) {
   __shared__ __align__(128) uint8_t buf[kCopyChunk];
   __shared__ __align__(8) uint64_t bar;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x != 0) return;
   const int64_t src = pairs[2 * blockIdx.x];
   const int64_t dst = pairs[2 * blockIdx.x + 1];

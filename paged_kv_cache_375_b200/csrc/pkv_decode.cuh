@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kPlanThreads)
   const int tid = threadIdx.x;
   const int32_t part_tokens = part_blocks * kBlock;
   for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
   for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
     int32_t L = checked_len(context_lens[s], max_len);
@@ -193,149 +195,179 @@ struct ItemMeta {
 };
 
 // ---- consumer state for bf16 (tensor cores) ----
+//
+// Per 16-token tile the scores are computed transposed, S^T = K Q^T, with the
+// tile's tokens as the MMA's M (16) and the group's query heads as N (8 per
+// n-tile), so one m16n8k16 covers a k-step of the whole group.  The output is
+// kept transposed too, O^T += V^T P^T (M = head_dim in tiles of 16, N = the
+// heads, K = the tile's tokens); P^T reaches the B-fragment layout through
+// movmatrix.  Two tiles are processed per step for instruction-level
+// parallelism.  The running max only moves when it grows by more than
+// kRescaleSlack (log2 units): weights then stay below 2^kRescaleSlack and the
+// accumulators are rescaled rarely (a warp vote decides).
+constexpr float kRescaleSlack = 8.f;
+
 template <int D, int GMAX>
 struct Bf16State {
-  static constexpr int KS = D / 16;  // k-steps of Q K^T
-  static constexpr int NT = D / 8;   // n-tiles of P V
-  static constexpr bool kTwoRowHalves = GMAX > 8;
-  uint32_t qa[KS][4];
-  float o[NT][4];
-  float m[2], l[2];
+  static constexpr int KS = D / 16;    // k-steps of S^T = K Q^T
+  static constexpr int MT = D / 16;    // m-tiles of O^T
+  static constexpr int NH = GMAX / 8;  // n-tiles of query heads
+  uint32_t qb[NH][KS][2];              // B fragments of Q^T
+  float o[NH][MT][4];                  // O^T accumulators
+  float m[NH][2];                      // running max of heads 8nh + 2(lane%4) + {0,1}
+  float l[NH][2];                      // this lane's part of the softmax denominators
 };
 
 template <int D, int GMAX>
 __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const uint8_t* qs,
                                                 int g, int lane) {
-  const int r0 = lane >> 2, qd = (lane & 3) * 2;
+  using St = Bf16State<D, GMAX>;
+  const int r = lane >> 2, qd = (lane & 3) * 2;
   const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qs);
 #pragma unroll
-  for (int ks = 0; ks < Bf16State<D, GMAX>::KS; ++ks) {
-    const int c = ks * 16 + qd;
-    st.qa[ks][0] = r0 < g ? *reinterpret_cast<const uint32_t*>(q16 + r0 * D + c) : 0u;
-    st.qa[ks][2] = r0 < g ? *reinterpret_cast<const uint32_t*>(q16 + r0 * D + c + 8) : 0u;
-    if constexpr (Bf16State<D, GMAX>::kTwoRowHalves) {
-      const int r1 = r0 + 8;
-      st.qa[ks][1] = r1 < g ? *reinterpret_cast<const uint32_t*>(q16 + r1 * D + c) : 0u;
-      st.qa[ks][3] = r1 < g ? *reinterpret_cast<const uint32_t*>(q16 + r1 * D + c + 8) : 0u;
-    } else {
-      st.qa[ks][1] = 0u;
-      st.qa[ks][3] = 0u;
-    }
-  }
-#pragma unroll
-  for (int nt = 0; nt < Bf16State<D, GMAX>::NT; ++nt) {
-    st.o[nt][0] = st.o[nt][1] = st.o[nt][2] = st.o[nt][3] = 0.f;
-  }
-  st.m[0] = st.m[1] = -INFINITY;
-  st.l[0] = st.l[1] = 0.f;
-}
-
-// One 16-token tile: scores, online softmax, P V.  `valid` tokens (0..16) of
-// the tile belong to the context.
-template <int D, int GMAX>
-__device__ __forceinline__ void bf16_block(Bf16State<D, GMAX>& st, const uint8_t* ktile,
-                                           const uint8_t* vtile, int valid, float sc,
-                                           int lane) {
-  using St = Bf16State<D, GMAX>;
-  constexpr bool kTwo = St::kTwoRowHalves;
-  const uint32_t kt = smem_addr(ktile), vt = smem_addr(vtile);
-  // ---- S = Q K^T (two independent accumulation chains per n-tile) ----
-  float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  {
-    const int mi = lane >> 3, ri = lane & 7;
-    const uint32_t t = (mi >> 1) * 8 + ri;      // token row this lane addresses
-    const uint32_t gsel = mi & 1;               // low / high 8 columns of the k-step
-    const uint32_t rowbase = kt + t * 128u;
+  for (int nh = 0; nh < St::NH; ++nh) {
+    const int head = nh * 8 + r;
 #pragma unroll
     for (int ks = 0; ks < St::KS; ++ks) {
-      const uint32_t c = ks >> 2, j = (ks & 3) * 2;
-      const uint32_t addr = rowbase + c * (kBlock * 128u) + (((j + gsel) ^ (t & 7u)) << 4);
-      uint32_t b0, b1, b2, b3;
-      ldmatrix_x4(addr, b0, b1, b2, b3);
-      if (ks & 1) {
-        mma_bf16_16816(sb[0], st.qa[ks], b0, b1);
-        mma_bf16_16816(sb[1], st.qa[ks], b2, b3);
-      } else {
-        mma_bf16_16816(sa[0], st.qa[ks], b0, b1);
-        mma_bf16_16816(sa[1], st.qa[ks], b2, b3);
-      }
-    }
-  }
-  // ---- scale, mask, online softmax ----
-  const int qd = (lane & 3) * 2;
-  float z[2][4];
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int tok = nt * 8 + qd + (i & 1);
-      const float v = (sa[nt][i] + sb[nt][i]) * sc;
-      z[nt][i] = tok < valid ? v : -INFINITY;
-    }
-  }
-  float p[2][4];
-#pragma unroll
-  for (int rh = 0; rh < (kTwo ? 2 : 1); ++rh) {
-    float mx = fmaxf(fmaxf(z[0][2 * rh], z[0][2 * rh + 1]), fmaxf(z[1][2 * rh], z[1][2 * rh + 1]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(st.m[rh], mx);
-    const float m_use = m_new == -INFINITY ? 0.f : m_new;
-    const float alpha = exp2f(st.m[rh] - m_use);
-    st.m[rh] = m_new;
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      p[nt][2 * rh] = exp2f(z[nt][2 * rh] - m_use);
-      p[nt][2 * rh + 1] = exp2f(z[nt][2 * rh + 1] - m_use);
+      const int c = ks * 16 + qd;
+      st.qb[nh][ks][0] = head < g ? *reinterpret_cast<const uint32_t*>(q16 + head * D + c) : 0u;
+      st.qb[nh][ks][1] = head < g ? *reinterpret_cast<const uint32_t*>(q16 + head * D + c + 8) : 0u;
     }
 #pragma unroll
-    for (int nt = 0; nt < St::NT; ++nt) {
-      st.o[nt][2 * rh] *= alpha;
-      st.o[nt][2 * rh + 1] *= alpha;
+    for (int mt = 0; mt < St::MT; ++mt) {
+      st.o[nh][mt][0] = st.o[nh][mt][1] = st.o[nh][mt][2] = st.o[nh][mt][3] = 0.f;
     }
-    st.l[rh] *= alpha;
+    st.m[nh][0] = st.m[nh][1] = -INFINITY;
+    st.l[nh][0] = st.l[nh][1] = 0.f;
   }
-  uint32_t pa[4];
-  pa[0] = pack_bf16x2(p[0][0], p[0][1]);
-  pa[2] = pack_bf16x2(p[1][0], p[1][1]);
-  st.l[0] += (bf16lo_to_f32(pa[0]) + bf16hi_to_f32(pa[0])) +
-             (bf16lo_to_f32(pa[2]) + bf16hi_to_f32(pa[2]));
-  if constexpr (kTwo) {
-    pa[1] = pack_bf16x2(p[0][2], p[0][3]);
-    pa[3] = pack_bf16x2(p[1][2], p[1][3]);
-    st.l[1] += (bf16lo_to_f32(pa[1]) + bf16hi_to_f32(pa[1])) +
-               (bf16lo_to_f32(pa[3]) + bf16hi_to_f32(pa[3]));
-  } else {
-    pa[1] = 0u;
-    pa[3] = 0u;
-  }
-  // ---- O += P V ----
-  uint32_t mk0 = 0xffffffffu, mk1 = 0xffffffffu;
-  const bool partial = valid < kBlock;
-  if (partial) {
-    mk0 = (qd < valid ? 0x0000ffffu : 0u) | (qd + 1 < valid ? 0xffff0000u : 0u);
-    mk1 = (qd + 8 < valid ? 0x0000ffffu : 0u) | (qd + 9 < valid ? 0xffff0000u : 0u);
-  }
+}
+
+// Two 16-token tiles (the second may be absent: valid1 = 0 and its pointers
+// equal the first's).  validX tokens of tile X belong to the context.
+template <int D, int GMAX>
+__device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t* k0,
+                                          const uint8_t* v0, int valid0, const uint8_t* k1,
+                                          const uint8_t* v1, int valid1, float sc, int lane) {
+  using St = Bf16State<D, GMAX>;
+  constexpr int NH = St::NH;
+  const int r = lane >> 2, qd = (lane & 3) * 2;
+  // ---- S^T = K Q^T for both tiles (two accumulation chains each) ----
+  float s[2][2][NH][4];
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) s[t][c][nh][0] = s[t][c][nh][1] = s[t][c][nh][2] = s[t][c][nh][3] = 0.f;
   {
-    const int mi = lane >> 3, ri = lane & 7;
-    const uint32_t t = (mi & 1) * 8 + ri;
-    const uint32_t gsel = mi >> 1;
-    const uint32_t rowbase = vt + t * 128u;
+    // ldmatrix.x4 rows: lanes 0-7 tokens 0-7 / low 8 columns, 8-15 tokens 8-15 / low,
+    // 16-23 tokens 0-7 / high, 24-31 tokens 8-15 / high -> A fragments a0..a3.
+    const uint32_t tok = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const uint32_t gsel = lane >> 4;
+    const uint32_t base0 = smem_addr(k0) + tok * 128u, base1 = smem_addr(k1) + tok * 128u;
 #pragma unroll
-    for (int dt = 0; dt < St::NT / 2; ++dt) {
-      const uint32_t c = dt >> 2, j = (dt & 3) * 2;
-      const uint32_t addr = rowbase + c * (kBlock * 128u) + (((j + gsel) ^ (t & 7u)) << 4);
-      uint32_t v0, v1, v2, v3;
-      ldmatrix_x4_trans(addr, v0, v1, v2, v3);
-      if (partial) {
-        v0 &= mk0;
-        v1 &= mk1;
-        v2 &= mk0;
-        v3 &= mk1;
+    for (int ks = 0; ks < St::KS; ++ks) {
+      const uint32_t off = (ks >> 2) * (kBlock * 128u) + (((((ks & 3) * 2) + gsel) ^ (tok & 7u)) << 4);
+      uint32_t a[4], b[4];
+      ldmatrix_x4(base0 + off, a[0], a[1], a[2], a[3]);
+      ldmatrix_x4(base1 + off, b[0], b[1], b[2], b[3]);
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) {
+        mma_bf16_16816(s[0][ks & 1][nh], a, st.qb[nh][ks][0], st.qb[nh][ks][1]);
+        mma_bf16_16816(s[1][ks & 1][nh], b, st.qb[nh][ks][0], st.qb[nh][ks][1]);
       }
-      mma_bf16_16816(st.o[2 * dt], pa, v0, v1);
-      mma_bf16_16816(st.o[2 * dt + 1], pa, v2, v3);
+    }
+  }
+  // ---- scale and mask; element i of a C fragment is token r + 8(i>>1), head 2q + (i&1) ----
+  float z[2][NH][4];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int valid = t ? valid1 : valid0;
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float v = (s[t][0][nh][i] + s[t][1][nh][i]) * sc;
+        z[t][nh][i] = (r + 8 * (i >> 1)) < valid ? v : -INFINITY;
+      }
+  }
+  // ---- running max per head column, lazy rescale ----
+  bool grow = false;
+  float m_new[NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      float mx = fmaxf(fmaxf(z[0][nh][hc], z[0][nh][hc + 2]), fmaxf(z[1][nh][hc], z[1][nh][hc + 2]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      m_new[nh][hc] = mx;
+      grow |= mx > st.m[nh][hc] + kRescaleSlack;
+    }
+  if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        if (m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack) {
+          const float alpha = fast_exp2(st.m[nh][hc] - m_new[nh][hc]);  // 0 when m was -inf
+          st.m[nh][hc] = m_new[nh][hc];
+          st.l[nh][hc] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < St::MT; ++mt) {
+            st.o[nh][mt][hc] *= alpha;
+            st.o[nh][mt][hc + 2] *= alpha;
+          }
+        }
+      }
+  }
+  // ---- P = exp2(z - m) in bf16, transposed into B fragments ----
+  uint32_t pb[2][NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    const float mu0 = st.m[nh][0] == -INFINITY ? 0.f : st.m[nh][0];
+    const float mu1 = st.m[nh][1] == -INFINITY ? 0.f : st.m[nh][1];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t lo = pack_bf16x2(fast_exp2(z[t][nh][0] - mu0), fast_exp2(z[t][nh][1] - mu1));
+      const uint32_t hi = pack_bf16x2(fast_exp2(z[t][nh][2] - mu0), fast_exp2(z[t][nh][3] - mu1));
+      st.l[nh][0] += bf16lo_to_f32(lo) + bf16lo_to_f32(hi);
+      st.l[nh][1] += bf16hi_to_f32(lo) + bf16hi_to_f32(hi);
+      pb[t][nh][0] = movmatrix_trans(lo);
+      pb[t][nh][1] = movmatrix_trans(hi);
+    }
+  }
+  // ---- O^T += V^T P^T ----
+  {
+    // ldmatrix.x4.trans rows: lanes 0-7 tokens 0-7 / low 8 d, 8-15 tokens 0-7 / high,
+    // 16-23 tokens 8-15 / low, 24-31 tokens 8-15 / high -> A fragments a0..a3 of V^T.
+    const uint32_t tok = (lane >> 4) * 8 + (lane & 7);
+    const uint32_t gsel = (lane >> 3) & 1;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int valid = t ? valid1 : valid0;
+      const uint32_t base = smem_addr(t ? v1 : v0) + tok * 128u;
+      uint32_t mk0 = 0xffffffffu, mk1 = 0xffffffffu;
+      const bool partial = valid < kBlock;
+      if (partial) {
+        mk0 = (qd < valid ? 0x0000ffffu : 0u) | (qd + 1 < valid ? 0xffff0000u : 0u);
+        mk1 = (qd + 8 < valid ? 0x0000ffffu : 0u) | (qd + 9 < valid ? 0xffff0000u : 0u);
+      }
+#pragma unroll
+      for (int mt = 0; mt < St::MT; ++mt) {
+        const uint32_t off = (mt >> 2) * (kBlock * 128u) + (((((mt & 3) * 2) + gsel) ^ (tok & 7u)) << 4);
+        uint32_t a[4];
+        ldmatrix_x4_trans(base + off, a[0], a[1], a[2], a[3]);
+        if (partial) {
+          a[0] &= mk0;
+          a[1] &= mk0;
+          a[2] &= mk1;
+          a[3] &= mk1;
+        }
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) mma_bf16_16816(st.o[nh][mt], a, pb[t][nh][0], pb[t][nh][1]);
+      }
     }
   }
 }
@@ -345,28 +377,31 @@ template <int D, int GMAX>
 __device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot, int g,
                                              int lane) {
   using St = Bf16State<D, GMAX>;
-  const int r0 = lane >> 2, qd = (lane & 3) * 2;
+  const int r = lane >> 2, qd = (lane & 3) * 2;
   float* O = slot;
   float* M = slot + g * D;
   float* L = M + g;
 #pragma unroll
-  for (int rh = 0; rh < (St::kTwoRowHalves ? 2 : 1); ++rh) {
-    float l = st.l[rh];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const int row = r0 + 8 * rh;
-    if (row < g) {
+  for (int nh = 0; nh < St::NH; ++nh)
 #pragma unroll
-      for (int nt = 0; nt < St::NT; ++nt) {
-        *reinterpret_cast<float2*>(O + row * D + nt * 8 + qd) =
-            make_float2(st.o[nt][2 * rh], st.o[nt][2 * rh + 1]);
-      }
-      if ((lane & 3) == 0) {
-        M[row] = st.m[rh];
-        L[row] = l;
+    for (int hc = 0; hc < 2; ++hc) {
+      float l = st.l[nh][hc];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      const int head = nh * 8 + qd + hc;
+      if (head < g) {
+#pragma unroll
+        for (int mt = 0; mt < St::MT; ++mt) {
+          O[head * D + mt * 16 + r] = st.o[nh][mt][hc];
+          O[head * D + mt * 16 + r + 8] = st.o[nh][mt][hc + 2];
+        }
+        if (r == 0) {
+          M[head] = st.m[nh][hc];
+          L[head] = l;
+        }
       }
     }
-  }
 }
 
 // ---- consumer state for fp32 (CUDA cores) ----
@@ -571,6 +606,7 @@ __global__ void __launch_bounds__((W + 1) * 32)
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();  // the plan and the cache writes before this launch are complete
 
   const int32_t hkv = prm.num_kv_heads;
   if (warp == W) {
@@ -589,6 +625,7 @@ __global__ void __launch_bounds__((W + 1) * 32)
       }
       const uint32_t widx = __shfl_sync(0xffffffffu, next, 0);
       if (widx >= total) {
+        pdl_trigger();  // this CTA's work is all handed out: let the next kernel launch
         if (lane == 0) {
           meta[r].seq = -1;
           mbar_arrive(&item_full[r]);
@@ -733,31 +770,40 @@ __global__ void __launch_bounds__((W + 1) * 32)
     } else {
       f32_begin_item<D, GMAX>(st);
     }
-    for (int32_t b = warp; b < it.nblk; b += W) {
-      if (cctr == pctr) {
+    // bf16 consumes this warp's blocks two at a time (b and b + W), fp32 one at a time.
+    constexpr int kStep = kBf16 ? 2 : 1;
+    for (int32_t b = warp; b < it.nblk; b += kStep * W) {
+      const int n = (kStep == 2 && b + W < it.nblk) ? 2 : 1;
+      if (pctr < cctr + n) {
         produce(true);
-        if (!ok || cctr == pctr) {
+        if (!ok || pctr < cctr + n) {
           ok = false;
           break;
         }
       }
-      const int s_idx = cctr % S;
-      if (!mbar_wait(&my_full[s_idx], (cctr / S) & 1)) {
-        ok = false;
-        break;
+      int valid[2] = {0, 0};
+      const uint8_t* kt[2];
+#pragma unroll
+      for (int x = 0; x < kStep; ++x) {
+        const uint32_t k = cctr + (x < n ? x : 0);
+        const int s_idx = k % S;
+        if (x < n && !mbar_wait(&my_full[s_idx], (k / S) & 1)) ok = false;
+        kt[x] = my_stages + s_idx * Lay::kStageBytes;
+        if (x < n && my_ok[s_idx]) {
+          const int v = it.len - (it.blk_begin + b + x * W) * kBlock;
+          valid[x] = v > kBlock ? kBlock : v;
+        }
       }
-      int valid = it.len - (it.blk_begin + b) * kBlock;
-      valid = valid > kBlock ? kBlock : valid;
-      if (!my_ok[s_idx]) valid = 0;
-      const uint8_t* kt = my_stages + s_idx * Lay::kStageBytes;
+      if (!ok) break;
       if constexpr (kBf16) {
-        bf16_block<D, GMAX>(st, kt, kt + Lay::kTileBytes, valid, sc, lane);
+        bf16_step<D, GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], kt[1],
+                           kt[1] + Lay::kTileBytes, valid[1], sc, lane);
       } else {
-        f32_block<D, GMAX>(st, reinterpret_cast<const float*>(qs), kt, kt + Lay::kTileBytes, valid,
-                           sc, g, lane);
+        f32_block<D, GMAX>(st, reinterpret_cast<const float*>(qs), kt[0], kt[0] + Lay::kTileBytes,
+                           valid[0], sc, g, lane);
       }
       __syncwarp();
-      ++cctr;
+      cctr += n;
       produce(false);
     }
     if (!ok) break;
@@ -800,6 +846,8 @@ __global__ void __launch_bounds__(128)
                  const float* __restrict__ part_ml, const int32_t* __restrict__ context_lens,
                  int32_t num_seqs, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
                  int32_t part_tokens) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
   if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;

@@ -69,13 +69,26 @@ def test_workspace_single_pass_has_no_partials():
 
 
 def test_workspace_split_k_sizes():
+    # long contexts, few sequences: about 16 items per SM -> 4096-token partitions
     d = dims(B=8, hq=64, hkv=8, nb=81920, mb=8192)
     P = pkv.decode_partition_tokens(d, 131072)
-    assert P == 512
+    assert P == 4096
     max_parts, po, pm = pkv.decode_workspace_layout(d, 131072)
+    assert max_parts == 32
+    assert po % 256 == 0 and pm % 256 == 0 and pm >= po + 8 * 64 * 32 * 128 * 4
+    assert pkv.decode_workspace_bytes(d, 131072) >= pm + 8 * 64 * 32 * 2 * 4
+    max_parts, _, _ = pkv.decode_workspace_layout(d, 131072, 512)
     assert max_parts == 256
-    assert po % 256 == 0 and pm % 256 == 0 and pm >= po + 8 * 64 * 256 * 128 * 4
-    assert pkv.decode_workspace_bytes(d, 131072) >= pm + 8 * 64 * 256 * 2 * 4
+
+
+def test_partition_rule_is_a_power_of_two_in_range():
+    for B, mcl in ((1, 131072), (4, 20000), (64, 2048), (256, 8192), (2, 100)):
+        d = dims(B=B, hq=32, hkv=8, nb=81920, mb=8192)
+        P = pkv.decode_partition_tokens(d, mcl)
+        if P < mcl:
+            assert P in (512, 1024, 2048, 4096, 8192)
+        else:
+            assert P % 16 == 0 and P < mcl + 16
 
 
 def test_explicit_partition_is_honoured():
