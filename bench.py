@@ -263,8 +263,15 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     pkv.check_device_error(dev)
 
+    # Timed region: K steps back to back.  Events between launches would break
+    # the overlap of consecutive launches (programmatic dependent launch), so
+    # only every SAMPLE-th step has its decode launch bracketed by events; those
+    # give the decode kernel's duration for the roofline (slightly pessimistic:
+    # a bracketed launch cannot overlap the plan kernel before it).
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    SAMPLE = 8
+    ev = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for i in range(0, K, SAMPLE)}
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -273,21 +280,21 @@ def run_ours(args, world, rank, local):
     with sampler:
         start.record(stream)
         for i in range(K):
-            ev[i][0].record(stream)
             step.cache_ops()
-            ev[i][1].record(stream)
             step.plan()
-            ev[i][2].record(stream)
-            step.decode()
-            ev[i][3].record(stream)
+            if i in ev:
+                ev[i][0].record(stream)
+                step.decode()
+                ev[i][1].record(stream)
+            else:
+                step.decode()
         end.record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
     pkv.check_device_error(dev)
     total_ms = start.elapsed_time(end)
-    cache_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    plan_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
-    decode_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    decode_ms = statistics.mean(a.elapsed_time(z) for a, z in ev.values())
+    ops = None if args.no_breakdown else breakdown(step, stream, dev)
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / K
     seconds = total_ms / 1e3
@@ -316,8 +323,9 @@ def run_ours(args, world, rank, local):
         },
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
         "seqs_per_s": round(whole_job_value(b.num_seqs * K, world, seconds), 1),
-        "breakdown_ms": {"cache_ops": round(cache_ms, 5), "plan": round(plan_ms, 5),
-                         "decode": round(decode_ms, 5)},
+        "breakdown": {"decode_ms_sampled": round(decode_ms, 5), "ops_alone": ops,
+                      "note": "decode: every 8th step of the timed region bracketed by events; "
+                              "other ops: each timed alone (50 launches) after the timed region"},
         "roofline": {
             "kernel": "decode_kernel" + (" + merge_kernel" if step.split else ""),
             "bound": "hbm", "achieved": round(alg["total"] / (decode_ms / 1e3) / 1e9, 2),
@@ -334,6 +342,61 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
     return result
+
+
+def op_bytes(step: Step) -> dict:
+    """Algorithmic bytes of each cache-maintenance op of one step (read + write)."""
+    b = step.b
+    row = b.num_kv_heads * b.head_dim * b.elem_bytes           # one token's K (or V) rows
+    block = row * 16                                            # one K (or V) block
+    T, P = step.T, int(b.cow_pairs.shape[0])
+    return {
+        "slot_mapping": T * (4 + 4 + 8) + (4 * b.num_seqs if step.decode_mode else 8 * T),
+        "reshape_and_cache": 2 * 2 * T * row + 8 * T,           # K and V, read and write
+        "copy_blocks": 2 * 2 * P * block + 16 * P,              # K and V, read and write
+        # reads the lengths, writes one 16-byte work item per (sequence, partition)
+        "plan": 4 * b.num_seqs + 16 * int(np.maximum(
+            1, (b.context_lens.astype(np.int64) + step.part_tokens - 1) // step.part_tokens).sum()),
+    }
+
+
+def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
+    """Each op of the step timed alone with events after the timed region (launches
+    here do not overlap), with achieved bandwidth against the HBM peak."""
+    pkv, b = step.pkv, step.b
+    ops = {"plan": step.plan}
+    if step.T:
+        if step.decode_mode:
+            ops["slot_mapping"] = lambda: pkv.slot_mapping(step.bt, b.num_blocks,
+                                                           context_lens=step.cl, out=step.slots)
+        else:
+            ops["slot_mapping"] = lambda: pkv.slot_mapping(step.bt, b.num_blocks,
+                                                           token_seq=step.seq, token_pos=step.pos,
+                                                           out=step.slots)
+        ops["reshape_and_cache"] = lambda: pkv.reshape_and_cache(
+            b.new_k, b.new_v, b.k_cache, b.v_cache, step.slots[:step.T])
+    if step.pairs is not None:
+        ops["copy_blocks"] = lambda: pkv.copy_blocks(b.k_cache, b.v_cache, step.pairs,
+                                                     validate=False)
+    nbytes = op_bytes(step)
+    peak, _ = hbm_peak()
+    out = {}
+    for name, fn in ops.items():
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(z) / n
+        gbs = nbytes[name] / (ms / 1e3) / 1e9
+        out[name] = {"ms": round(ms, 5), "bytes": nbytes[name], "GBps": round(gbs, 1),
+                     "frac_of_hbm_peak": round(gbs / peak, 4)}
+    step()  # leave a consistent state behind
+    torch.cuda.synchronize(dev)
+    return out
 
 
 def run_e2e(step: Step, args, world, dev, kv_bytes):
@@ -469,6 +532,8 @@ def main(argv=None):
     ap.add_argument("--partition", type=int, default=0, help="partition tokens (0 = automatic)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true",
+                    help="skip timing the cache ops and the plan alone after the timed region")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

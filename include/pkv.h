@@ -28,7 +28,7 @@
  *    invalid one is skipped -- never dereferenced -- and a bit is set in a
  *    per-device error word; pkv_check_device_error() reads and clears it.  No
  *    kernel traps, asserts or waits without a bound: every internal wait gives
- *    up after about four seconds and reports PKV_DEVERR_TIMEOUT.
+ *    up after about one second and reports PKV_DEVERR_TIMEOUT.
  *  - All device pointers must be 16-byte aligned.  Calls that launch work make
  *    the device owning their output buffer current (the library carries its
  *    own CUDA runtime, so the caller's current device is not seen); a host
@@ -260,6 +260,15 @@ pkv_status pkv_slot_mapping(int64_t *slot_mapping, const int32_t *block_tables,
  * PKV_ERR_DEVICE_INDEX (other bits) or PKV_ERR_CUDA.
  */
 pkv_status pkv_check_device_error(void *cuda_stream, uint32_t *bits_out);
+
+/*
+ * Diagnostic: launches one warp that waits, with the kernels' own bounded
+ * wait, on a barrier nothing completes.  After about a second the wait gives
+ * up and sets PKV_DEVERR_TIMEOUT; the kernel then returns and the context
+ * stays usable.  Shows that a stalled wait turns into an error status
+ * rather than a hang.  Asynchronous on cuda_stream.
+ */
+pkv_status pkv_selftest_wait_timeout(void *cuda_stream);
 
 /* Static text for a status code. */
 const char *pkv_status_string(pkv_status status);

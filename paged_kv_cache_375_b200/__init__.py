@@ -78,6 +78,7 @@ def load_library() -> ctypes.CDLL:
             "pkv_validate_copy_pairs": (ctypes.c_int, [P, i32, i32]),
             "pkv_slot_mapping": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
             "pkv_check_device_error": (ctypes.c_int, [P, P]),
+            "pkv_selftest_wait_timeout": (ctypes.c_int, [P]),
             "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "pkv_last_error_message": (ctypes.c_char_p, []),
         }
@@ -349,3 +350,10 @@ def device_error_bits(device: torch.device | None = None) -> int:
     if status not in (0, 7, 9):
         _check(status)
     return bits.value
+
+
+def selftest_wait_timeout(device: torch.device | None = None) -> None:
+    """Launch the bounded-wait self-test (about one second); read the result with
+    device_error_bits()."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    _check(load_library().pkv_selftest_wait_timeout(_stream_ptr(dev)))

@@ -588,6 +588,13 @@ pkv_status pkv_slot_mapping(int64_t* slot_mapping, const int32_t* block_tables,
   return PKV_OK;
 }
 
+pkv_status pkv_selftest_wait_timeout(void* cuda_stream) {
+  cudaError_t e = launch(pkv::wait_timeout_selftest_kernel, dim3(1), dim3(32), 0,
+                         static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return PKV_OK;
+}
+
 pkv_status pkv_check_device_error(void* cuda_stream, uint32_t* bits_out) {
   cudaError_t e;
   if (cuda_stream) {

@@ -121,4 +121,19 @@ __global__ void __launch_bounds__(32)
   bulk_wait_all();
 }
 
+// ------------------------------------------------------------ wait self-test
+// One warp waits, with the same bounded wait the decode kernel uses, on an
+// mbarrier phase that nothing completes.  The wait expires, raises
+// PKV_DEVERR_TIMEOUT and the kernel returns normally.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  mbar_wait(&bar, 0);
+}
+
 }  // namespace pkv

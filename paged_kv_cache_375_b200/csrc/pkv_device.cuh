@@ -22,9 +22,10 @@ __device__ __forceinline__ void raise_error(unsigned int bits) {
   atomicOr(&g_device_error, bits);
 }
 
-// Every wait on the GPU gives up after this many SM clock cycles (about four
-// seconds at the B200's 1.965 GHz boost clock; longer at lower clocks).
-constexpr long long kWaitLimitCycles = 8000000000ll;
+// Every wait on the GPU gives up after this many SM clock cycles (about one
+// second at the B200's 1.965 GHz boost clock; a little longer at lower
+// clocks).  A healthy wait in these kernels lasts microseconds.
+constexpr long long kWaitLimitCycles = 2000000000ll;
 // Shorter bound used when draining copies after a wait has already failed.
 constexpr long long kDrainLimitCycles = 200000000ll;
 

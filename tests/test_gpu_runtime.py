@@ -1,0 +1,75 @@
+"""Runtime behaviour on the GPU: a plan reused for several runs (several layers'
+pools), back-to-back decodes on one stream, and the bounded-wait failure path
+(a wait that nothing completes turns into an error status, and the context
+stays usable)."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_375_b200 as pkv
+import workloads
+from gpu_util import check_close, dev_i32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("partition", [0, 256])
+def test_one_plan_serves_several_runs(cuda_device, partition):
+    lens = [3, 100, 640, 1999, 16, 700]
+    b = workloads.random_batch(71, lens, 32, 8, 128, "bf16", device=cuda_device)
+    # a second "layer": other pools and queries with the same tables and lengths
+    gen = torch.Generator(device=cuda_device).manual_seed(72)
+    k2 = torch.randn(b.k_cache.shape, generator=gen, device=cuda_device).to(torch.bfloat16)
+    v2 = torch.randn(b.v_cache.shape, generator=gen, device=cuda_device).to(torch.bfloat16)
+    q2 = torch.randn(b.q.shape, generator=gen, device=cuda_device).to(torch.bfloat16)
+    bt = dev_i32(b.block_tables, cuda_device)
+    cl = dev_i32(b.context_lens, cuda_device)
+    mcl = b.max_context_len
+    plan = pkv.DecodePlan(bt, cl, b.num_q_heads, b.k_cache, max_context_len=mcl,
+                          partition_tokens=partition)
+    outs = []
+    for _ in range(3):
+        for q, k, v in ((b.q, b.k_cache, b.v_cache), (q2, k2, v2)):
+            outs.append(plan.run(torch.empty_like(q), q, k, v, b.scale))
+    ref1 = pkv.paged_attention_decode(torch.empty_like(b.q), b.q, b.k_cache, b.v_cache, bt, cl,
+                                      b.scale, 8, max_context_len=mcl, partition_tokens=partition)
+    ref2 = pkv.paged_attention_decode(torch.empty_like(q2), q2, k2, v2, bt, cl, b.scale, 8,
+                                      max_context_len=mcl, partition_tokens=partition)
+    assert pkv.device_error_bits() == 0
+    for i, o in enumerate(outs):
+        ref = ref1 if i % 2 == 0 else ref2
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16)), f"run {i}"
+
+
+def test_back_to_back_decodes_are_deterministic(cuda_device):
+    b = workloads.random_batch(73, list(range(1, 400, 7)), 16, 2, 128, "bf16", device=cuda_device)
+    bt = dev_i32(b.block_tables, cuda_device)
+    cl = dev_i32(b.context_lens, cuda_device)
+    outs = [pkv.paged_attention_decode(torch.empty_like(b.q), b.q, b.k_cache, b.v_cache, bt, cl,
+                                       b.scale, 2, max_context_len=b.max_context_len)
+            for _ in range(20)]
+    assert pkv.device_error_bits() == 0
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_expired_wait_reports_timeout_and_context_survives(cuda_device):
+    assert pkv.device_error_bits() == 0
+    pkv.selftest_wait_timeout(cuda_device)
+    bits = pkv.device_error_bits()
+    assert bits & pkv.DEVERR_TIMEOUT
+    with pytest.raises(pkv.PkvError):
+        pkv.selftest_wait_timeout(cuda_device)
+        pkv.check_device_error(cuda_device)
+    # the context is still usable: a decode afterwards is correct
+    b = workloads.c1_tiny_fp32(device=cuda_device)
+    host = b.host()
+    import oracle
+    out = torch.empty_like(b.q)
+    pkv.paged_attention_decode(out, b.q, b.k_cache, b.v_cache, dev_i32(b.block_tables, cuda_device),
+                               dev_i32(b.context_lens, cuda_device), b.scale, b.num_kv_heads,
+                               max_context_len=b.max_context_len)
+    ref = oracle.paged_decode(host["q"], host["k_cache"], host["v_cache"], b.block_tables,
+                              b.context_lens, b.scale)
+    check_close(out, ref, "f32", "after timeout")
+    assert pkv.device_error_bits() == 0
