@@ -46,7 +46,7 @@ WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shar
              "c5": "c5_long_splitk", "c1": "c1_tiny_fp32"}
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")  # JSON text
 
 
 # ------------------------------------------------------------------ helpers
@@ -82,14 +82,15 @@ def recorded_traffic(workload: str):
 
 
 def algorithmic_bytes(b: workloads.Batch) -> dict:
-    """Bytes a decode launch must move at least: every context token's K and V once per kv
-    head, q, out, the block-table entries in use and the context lengths."""
+    """Bytes a decode launch must move from HBM at least: every context token's K and V once
+    per kv head (slots shared by several sequences once), q, out, the block-table entries
+    in use and the context lengths."""
     lens = b.context_lens.astype(np.int64)
     table = int(((lens + 15) // 16).sum()) * 4
     qo = 2 * b.num_seqs * b.num_q_heads * b.head_dim * b.elem_bytes
-    kv = b.kv_bytes()
-    return {"kv": kv, "q_out": qo, "table": table, "lens": 4 * b.num_seqs,
-            "total": kv + qo + table + 4 * b.num_seqs}
+    kv = b.unique_kv_bytes() if b.cow_pairs.shape[0] or b.name == "c4_shared_prefix" else b.kv_bytes()
+    return {"kv": kv, "kv_logical": b.kv_bytes(), "q_out": qo, "table": table,
+            "lens": 4 * b.num_seqs, "total": kv + qo + table + 4 * b.num_seqs}
 
 
 class ClockSampler:

@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(32)
   fence_proxy_async_smem();
   bulk_store(cache + dst * block_bytes + off, buf, bytes);
   bulk_commit();
-  bulk_wait_all();
+  bulk_wait_read_all();  // keep the shared buffer alive until the store has read it
 }
 
 // ------------------------------------------------------------ wait self-test

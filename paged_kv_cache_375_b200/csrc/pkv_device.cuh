@@ -168,9 +168,10 @@ __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
-// Wait until every committed bulk store has completed (writes performed).
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+// Wait until every committed bulk store has finished reading its shared-memory
+// source (the global writes complete by the end of the kernel).
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // Order prior generic-proxy accesses to shared memory before later
