@@ -422,23 +422,55 @@ def run_e2e(step: Step, args, world, dev, kv_bytes):
         out_host.copy_(step.out, non_blocking=True)
         stream.synchronize()
 
-    for _ in range(max(3, args.warmup // 4)):
-        one()
+    def timed(fn, K):
+        for _ in range(max(3, args.warmup // 4)):
+            fn()
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(K):
+            fn()
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        return max_over_ranks(s.elapsed_time(e), world, dev)
+
     K = max(3, args.steps // 4)
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    s = torch.cuda.Event(enable_timing=True)
-    e = torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(K):
-        one()
-    e.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    ms = max_over_ranks(s.elapsed_time(e), world, dev)
-    return {"value": round(whole_job_value(kv_bytes * K / 1e9, world, ms / 1e3), 2), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
-            "ms_per_step": round(ms / K, 5), "host_sync_per_step": True}
+    ms = timed(one, K)
+    result = {"value": round(whole_job_value(kv_bytes * K / 1e9, world, ms / 1e3), 2),
+              "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+              "ms_per_step": round(ms / K, 5), "host_sync_per_step": True}
+    # The same step captured once into a CUDA graph (copies in, kernels, copy out) and
+    # replayed every step: what a serving loop that replays a captured step would see.
+    try:
+        graph_stream = torch.cuda.Stream(device=dev)
+        graph_stream.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(graph_stream):
+            with torch.cuda.graph(g, stream=graph_stream):
+                b.q.copy_(host["q"], non_blocking=True)
+                b.new_k.copy_(host["new_k"], non_blocking=True)
+                b.new_v.copy_(host["new_v"], non_blocking=True)
+                step.cl.copy_(host["cl"], non_blocking=True)
+                step.bt.copy_(host["bt"], non_blocking=True)
+                step()
+                out_host.copy_(step.out, non_blocking=True)
+        torch.cuda.synchronize(dev)
+
+        def replay():
+            g.replay()
+            torch.cuda.current_stream(dev).synchronize()
+
+        gms = timed(replay, K)
+        result["graph_replay"] = {
+            "value": round(whole_job_value(kv_bytes * K / 1e9, world, gms / 1e3), 2),
+            "ms_per_step": round(gms / K, 5)}
+        del g
+    except RuntimeError as ex:  # report, do not fail the bench
+        result["graph_replay"] = {"error": str(ex)[:200]}
+    return result
 
 
 # ------------------------------------------------------------ oracle (CPU)

@@ -73,3 +73,46 @@ def test_expired_wait_reports_timeout_and_context_survives(cuda_device):
                               b.context_lens, b.scale)
     check_close(out, ref, "f32", "after timeout")
     assert pkv.device_error_bits() == 0
+
+
+def test_decode_step_captured_in_a_cuda_graph_matches_eager(cuda_device):
+    """Slot indexing, reshape_and_cache, plan and decode captured once into a CUDA graph
+    and replayed give bit-identical results to eager launches."""
+    b = workloads.random_batch(74, [5, 17, 300, 1200, 2100], 32, 8, 128, "bf16",
+                               device=cuda_device, new_token=True)
+    bt = dev_i32(b.block_tables, cuda_device)
+    cl = dev_i32(b.context_lens, cuda_device)
+    mcl = b.max_context_len
+    ws = torch.empty(pkv.decode_workspace_bytes(
+        pkv.make_dims(b.num_seqs, b.num_q_heads, b.k_cache, b.max_blocks_per_seq), mcl, 512),
+        dtype=torch.uint8, device=cuda_device)
+    slots = torch.empty(b.num_seqs, dtype=torch.int64, device=cuda_device)
+    out = torch.empty_like(b.q)
+
+    def step():
+        pkv.slot_mapping(bt, b.num_blocks, context_lens=cl, out=slots)
+        pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, slots)
+        plan = pkv.DecodePlan(bt, cl, b.num_q_heads, b.k_cache, max_context_len=mcl,
+                              partition_tokens=512, workspace_tensor=ws)
+        plan.run(out, b.q, b.k_cache, b.v_cache, b.scale)
+
+    step()
+    torch.cuda.synchronize()
+    eager = out.clone()
+    out.zero_()
+    s = torch.cuda.Stream(device=cuda_device)
+    s.wait_stream(torch.cuda.current_stream(cuda_device))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        step()                                   # warm the per-kernel settings outside capture
+        torch.cuda.synchronize()
+        out.zero_()
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    assert pkv.device_error_bits() == 0
