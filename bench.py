@@ -340,6 +340,8 @@ def run_ours(args, world, rank, local):
     }
     if e2e is not None:
         result["e2e"] = e2e
+    if rank == 0 and not args.no_breakdown:
+        result["host_block_manager"] = host_block_manager_cost(b)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
     return result
@@ -398,6 +400,32 @@ def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
     step()  # leave a consistent state behind
     torch.cuda.synchronize(dev)
     return out
+
+
+def host_block_manager_cost(b: workloads.Batch, steps: int = 50) -> dict:
+    """Host time of the native block manager for one decode step of this batch: append
+    one token to every sequence (slots, copy-on-write pairs) and export the block tables
+    and lengths the decode call takes.  CPU only."""
+    import paged_kv_cache_375_b200 as pkv
+    rng = np.random.default_rng(0)
+    bm = pkv.BlockManager(b.num_blocks, 16, seed=1, prefix_caching=True)
+    ids = np.arange(b.num_seqs, dtype=np.int64)
+    for s in range(b.num_seqs):
+        bm.add_sequence(int(s), rng.integers(0, 32000, size=int(b.context_lens[s]) - 1))
+    width = b.max_blocks_per_seq + (steps + 15) // 16 + 1
+    toks = rng.integers(0, 32000, size=(steps, b.num_seqs)).astype(np.int32)
+    slots = np.empty(b.num_seqs, dtype=np.int64)
+    tables = np.empty((b.num_seqs, width), dtype=np.int32)
+    lens = np.empty(b.num_seqs, dtype=np.int32)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        bm.append_tokens(ids, toks[i], out=slots)
+        bm.take_copies()
+        bm.block_tables(ids, width, tables=tables, lens=lens)
+    el = time.perf_counter() - t0
+    bm.close()
+    return {"us_per_step": round(1e6 * el / steps, 2), "sequences": b.num_seqs,
+            "what": "append one token per sequence + take copies + export tables and lengths"}
 
 
 def run_e2e(step: Step, args, world, dev, kv_bytes):

@@ -69,7 +69,9 @@ typedef enum pkv_status {
     PKV_ERR_CUDA = 6,          /* a CUDA runtime call or a launch failed */
     PKV_ERR_DEVICE_INDEX = 7,  /* a kernel met an invalid index (see the error bits) */
     PKV_ERR_ALIGN = 8,         /* a pointer is not 16-byte aligned */
-    PKV_ERR_DEVICE_TIMEOUT = 9 /* a kernel's bounded wait expired */
+    PKV_ERR_DEVICE_TIMEOUT = 9,/* a kernel's bounded wait expired */
+    PKV_ERR_NO_BLOCKS = 10,    /* block manager: the pool has no block left */
+    PKV_ERR_NOT_FOUND = 11     /* block manager: unknown (or already used) sequence id */
 } pkv_status;
 
 typedef enum pkv_dtype {

@@ -33,7 +33,8 @@ DEVERR_BLOCK, DEVERR_SLOT, DEVERR_LEN, DEVERR_PAIR, DEVERR_POS, DEVERR_TIMEOUT =
 
 STATUS_NAMES = {0: "PKV_OK", 1: "PKV_ERR_NULL", 2: "PKV_ERR_SHAPE", 3: "PKV_ERR_UNSUPPORTED",
                 4: "PKV_ERR_WORKSPACE", 5: "PKV_ERR_PAIRS", 6: "PKV_ERR_CUDA",
-                7: "PKV_ERR_DEVICE_INDEX", 8: "PKV_ERR_ALIGN", 9: "PKV_ERR_DEVICE_TIMEOUT"}
+                7: "PKV_ERR_DEVICE_INDEX", 8: "PKV_ERR_ALIGN", 9: "PKV_ERR_DEVICE_TIMEOUT",
+                10: "PKV_ERR_NO_BLOCKS", 11: "PKV_ERR_NOT_FOUND"}
 
 
 class PkvError(RuntimeError):
@@ -80,6 +81,17 @@ def load_library() -> ctypes.CDLL:
             "pkv_check_device_error": (ctypes.c_int, [P, P]),
             "pkv_selftest_wait_timeout": (ctypes.c_int, [P]),
             "pkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "pkv_bm_create": (P, [i32, i32, ctypes.c_uint64, i32]),
+            "pkv_bm_destroy": (None, [P]),
+            "pkv_bm_add_sequence": (ctypes.c_int, [P, ctypes.c_int64, P, i32, P]),
+            "pkv_bm_fork": (ctypes.c_int, [P, ctypes.c_int64, ctypes.c_int64]),
+            "pkv_bm_append_tokens": (ctypes.c_int, [P, P, P, i32, P]),
+            "pkv_bm_slots": (ctypes.c_int, [P, ctypes.c_int64, i32, i32, P]),
+            "pkv_bm_free_sequence": (ctypes.c_int, [P, ctypes.c_int64]),
+            "pkv_bm_take_copies": (i32, [P, P, i32]),
+            "pkv_bm_block_tables": (ctypes.c_int, [P, P, i32, i32, P, P]),
+            "pkv_bm_stats": (ctypes.c_int, [P, P, P, P, P]),
+            "pkv_bm_refcount": (i32, [P, i32]),
             "pkv_last_error_message": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -357,3 +369,110 @@ def selftest_wait_timeout(device: torch.device | None = None) -> None:
     device_error_bits()."""
     dev = device or torch.device("cuda", torch.cuda.current_device())
     _check(load_library().pkv_selftest_wait_timeout(_stream_ptr(dev)))
+
+
+class BlockManager:
+    """Host-side KV-block bookkeeping (the library's native block manager).
+
+    Hands out blocks of ``block_size`` tokens from a scattered pool, keeps block tables,
+    shares blocks between forked sequences with reference counts and emits copy-on-write
+    pairs, and (with ``prefix_caching``) reuses cached full prompt blocks found through a
+    chain of block hashes, evicting unreferenced cached blocks least recently used first.
+    Take the queued copies (``take_copies``) after each append call, before sequences
+    are freed, and apply them with ``copy_blocks`` before the step's writes.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int = 16, seed: int = 0,
+                 prefix_caching: bool = False):
+        import numpy as np
+        self._np = np
+        self._lib = load_library()
+        self._h = self._lib.pkv_bm_create(num_blocks, block_size, seed, int(prefix_caching))
+        if not self._h:
+            raise PkvError(2, "invalid block manager sizes")
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def close(self):
+        if self._h:
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _arr(self, a, dtype):
+        a = self._np.ascontiguousarray(a, dtype=dtype)
+        return a, a.ctypes.data_as(ctypes.c_void_p)
+
+    def add_sequence(self, seq_id: int, tokens) -> int:
+        """Start a sequence with its prompt; returns the number of prompt tokens found cached."""
+        t, tp = self._arr(tokens, self._np.int32)
+        cached = ctypes.c_int32(0)
+        _bm_check(self._lib.pkv_bm_add_sequence(self._h, seq_id, tp, t.shape[0],
+                                                ctypes.byref(cached)))
+        return cached.value
+
+    def fork(self, parent: int, child: int) -> None:
+        _bm_check(self._lib.pkv_bm_fork(self._h, parent, child))
+
+    def append_tokens(self, seq_ids, tokens, out=None):
+        """Append one token to each sequence; returns the int64 slots of the new tokens
+        (written into ``out`` when given)."""
+        s, sp = self._arr(seq_ids, self._np.int64)
+        t, tp = self._arr(tokens, self._np.int32)
+        assert s.shape == t.shape
+        if out is None:
+            out = self._np.empty(s.shape[0], dtype=self._np.int64)
+        assert out.dtype == self._np.int64 and out.flags["C_CONTIGUOUS"] and out.shape == s.shape
+        _bm_check(self._lib.pkv_bm_append_tokens(self._h, sp, tp, s.shape[0],
+                                                 out.ctypes.data_as(ctypes.c_void_p)))
+        return out
+
+    def slots(self, seq_id: int, pos_begin: int, pos_end: int):
+        out = self._np.empty(max(0, pos_end - pos_begin), dtype=self._np.int64)
+        _bm_check(self._lib.pkv_bm_slots(self._h, seq_id, pos_begin, pos_end,
+                                         out.ctypes.data_as(ctypes.c_void_p)))
+        return out
+
+    def free_sequence(self, seq_id: int) -> None:
+        _bm_check(self._lib.pkv_bm_free_sequence(self._h, seq_id))
+
+    def take_copies(self):
+        """The queued (src, dst) copy-on-write pairs, as int64 [P][2]."""
+        n = -self._lib.pkv_bm_take_copies(self._h, None, 0)
+        out = self._np.empty((max(n, 0), 2), dtype=self._np.int64)
+        got = self._lib.pkv_bm_take_copies(self._h, out.ctypes.data_as(ctypes.c_void_p), n)
+        return out[:max(got, 0)]
+
+    def block_tables(self, seq_ids, max_blocks: int, tables=None, lens=None):
+        """(tables int32 [n][max_blocks] padded with -1, context lengths int32 [n]); written
+        into ``tables`` / ``lens`` when given (e.g. pinned buffers reused every step)."""
+        s, sp = self._arr(seq_ids, self._np.int64)
+        if tables is None:
+            tables = self._np.empty((s.shape[0], max_blocks), dtype=self._np.int32)
+        if lens is None:
+            lens = self._np.empty(s.shape[0], dtype=self._np.int32)
+        assert tables.dtype == self._np.int32 and tables.shape == (s.shape[0], max_blocks)
+        assert lens.dtype == self._np.int32 and lens.shape == (s.shape[0],)
+        assert tables.flags["C_CONTIGUOUS"] and lens.flags["C_CONTIGUOUS"]
+        _bm_check(self._lib.pkv_bm_block_tables(self._h, sp, s.shape[0], max_blocks,
+                                                tables.ctypes.data_as(ctypes.c_void_p),
+                                                lens.ctypes.data_as(ctypes.c_void_p)))
+        return tables, lens
+
+    def stats(self) -> dict:
+        v = [ctypes.c_int32() for _ in range(4)]
+        _bm_check(self._lib.pkv_bm_stats(self._h, *[ctypes.byref(x) for x in v]))
+        return dict(zip(("free", "evictable", "used", "sequences"), (x.value for x in v)))
+
+    def refcount(self, block: int) -> int:
+        return self._lib.pkv_bm_refcount(self._h, block)
+
+
+def _bm_check(status: int):
+    if status != 0:
+        name = STATUS_NAMES.get(status, status)
+        raise PkvError(status, load_library().pkv_status_string(status).decode() + f" ({name})")

@@ -13,8 +13,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpkv.so")
-SOURCES = ["pkv_api.cu"]
+SOURCES = ["pkv_api.cu", "pkv_block_manager.cpp"]
 DEPS = SOURCES + ["pkv_device.cuh", "pkv_decode.cuh", "pkv_cache_ops.cuh"]
+HEADERS = ["pkv.h", "pkv_block_manager.h"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
@@ -36,7 +37,7 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in DEPS] + [os.path.join(INCLUDE, "pkv.h")]
+    deps = [os.path.join(CSRC, f) for f in DEPS] + [os.path.join(INCLUDE, h) for h in HEADERS]
     return all(os.path.getmtime(p) <= t for p in deps)
 
 

@@ -633,6 +633,8 @@ const char* pkv_status_string(pkv_status status) {
     case PKV_ERR_DEVICE_INDEX: return "invalid index met on the device";
     case PKV_ERR_ALIGN: return "pointer not 16-byte aligned";
     case PKV_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case PKV_ERR_NO_BLOCKS: return "no KV block left in the pool";
+    case PKV_ERR_NOT_FOUND: return "unknown or duplicate sequence id";
   }
   return "unknown status";
 }

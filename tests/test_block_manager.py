@@ -1,0 +1,192 @@
+"""The native host block manager (include/pkv_block_manager.h), on the CPU.
+
+The main check simulates the KV pool: every token is written to the slot the
+manager hands out, every copy-on-write pair copies a whole block, and then
+every live sequence, read back through its block table, must return exactly
+its own tokens -- paging changes where K/V live, never what a sequence sees
+(ipipp.com vLLM article, "二、PagedAttention分页原理深度剖析").  Reference counts
+must equal the number of table entries pointing at each block, and the pool
+must account for every block.  Prefix caching is checked against what the
+wiki entry's "Automatic Prefix Caching" section fixes: chained hashes of full
+blocks, exact block-by-block matching, full blocks only, LRU eviction.
+"""
+import numpy as np
+import pytest
+
+import paged_kv_cache_375_b200 as pkv
+
+BS = 16
+
+
+class SimPool:
+    """Token ids stored per physical slot, updated exactly as the device would be."""
+
+    def __init__(self, num_blocks):
+        self.slots = np.full(num_blocks * BS, -1, dtype=np.int64)
+
+    def write(self, slots, tokens):
+        self.slots[np.asarray(slots)] = np.asarray(tokens)
+
+    def copy(self, pairs):
+        snap = self.slots.copy()
+        for src, dst in pairs:
+            self.slots[dst * BS:(dst + 1) * BS] = snap[src * BS:(src + 1) * BS]
+
+    def read(self, table, length):
+        pos = np.arange(length)
+        return self.slots[table[pos // BS] * BS + pos % BS]
+
+
+def check_invariants(bm, pool, seqs, num_blocks):
+    ids = sorted(seqs)
+    if ids:
+        tables, lens = bm.block_tables(ids, max_blocks=256)
+        refs = np.zeros(num_blocks, dtype=np.int64)
+        for i, s in enumerate(ids):
+            assert lens[i] == len(seqs[s])
+            n = (lens[i] + BS - 1) // BS
+            assert (tables[i, n:] == -1).all()
+            row = tables[i, :n]
+            assert len(set(row.tolist())) == n            # a sequence never repeats a block
+            refs[row] += 1
+            got = pool.read(row, lens[i])
+            assert np.array_equal(got, np.array(seqs[s])), f"sequence {s} reads wrong tokens"
+        for b in range(num_blocks):
+            assert bm.refcount(b) == refs[b]
+    st = bm.stats()
+    assert st["free"] + st["evictable"] + st["used"] == num_blocks
+    assert st["sequences"] == len(seqs)
+
+
+@pytest.mark.parametrize("prefix_caching", [False, True])
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_random_operations_keep_every_sequence_intact(prefix_caching, seed):
+    rng = np.random.default_rng(seed)
+    num_blocks = 400
+    bm = pkv.BlockManager(num_blocks, BS, seed=seed, prefix_caching=prefix_caching)
+    pool = SimPool(num_blocks)
+    seqs = {}
+    prompts = [rng.integers(0, 50, size=int(rng.integers(1, 90))).tolist() for _ in range(6)]
+    next_id = 0
+    for it in range(600):
+        op = rng.random()
+        if op < 0.2 or not seqs:
+            prompt = list(prompts[rng.integers(len(prompts))])
+            if rng.random() < 0.5:
+                prompt += rng.integers(0, 50, size=int(rng.integers(0, 40))).tolist()
+            try:
+                cached = bm.add_sequence(next_id, prompt)
+            except pkv.PkvError as e:
+                assert e.status == 10
+                continue
+            assert cached % BS == 0 and cached <= len(prompt)
+            if not prefix_caching:
+                assert cached == 0
+            # the caller writes the K/V of the prompt tokens that were not cached
+            pool.write(bm.slots(next_id, cached, len(prompt)), prompt[cached:])
+            seqs[next_id] = prompt
+            next_id += 1
+        elif op < 0.35:
+            parent = int(rng.choice(list(seqs)))
+            bm.fork(parent, next_id)
+            seqs[next_id] = list(seqs[parent])
+            next_id += 1
+        elif op < 0.85:
+            ids = rng.choice(list(seqs), size=min(len(seqs), int(rng.integers(1, 6))),
+                             replace=False).tolist()
+            toks = rng.integers(0, 50, size=len(ids)).tolist()
+            try:
+                slots = bm.append_tokens(ids, toks)
+            except pkv.PkvError as e:
+                assert e.status == 10
+                check_invariants(bm, pool, seqs, num_blocks)   # nothing changed
+                continue
+            pool.copy(bm.take_copies())                          # copies before writes
+            pool.write(slots, toks)
+            for s, t in zip(ids, toks):
+                seqs[s].append(t)
+        else:
+            s = int(rng.choice(list(seqs)))
+            bm.free_sequence(s)
+            del seqs[s]
+        if it % 25 == 0:
+            check_invariants(bm, pool, seqs, num_blocks)
+    check_invariants(bm, pool, seqs, num_blocks)
+    for s in list(seqs):
+        bm.free_sequence(s)
+    st = bm.stats()
+    assert st["used"] == 0 and st["sequences"] == 0
+
+
+def test_fork_then_append_copies_the_shared_partial_block_once():
+    bm = pkv.BlockManager(50, BS, seed=4)
+    bm.add_sequence(0, list(range(20)))          # 2 blocks, the second partial
+    for c in range(1, 4):
+        bm.fork(0, c)
+    tables, _ = bm.block_tables([0], 8)
+    shared_tail = int(tables[0, 1])
+    assert bm.refcount(shared_tail) == 4
+    bm.append_tokens([1, 2, 3, 0], [7, 7, 7, 7])
+    pairs = bm.take_copies()
+    assert pairs.shape == (3, 2) and (pairs[:, 0] == shared_tail).all()
+    assert bm.refcount(shared_tail) == 1         # the last holder writes in place
+    # full shared blocks are never copied: appending into a fresh block needs no copy
+    bm2 = pkv.BlockManager(50, BS, seed=5)
+    bm2.add_sequence(0, list(range(32)))
+    bm2.fork(0, 1)
+    bm2.append_tokens([0, 1], [1, 2])
+    assert bm2.take_copies().shape == (0, 2)
+
+
+def test_prefix_cache_reuses_full_blocks_only_and_matches_exactly():
+    bm = pkv.BlockManager(100, BS, seed=6, prefix_caching=True)
+    prompt = list(range(100, 150))               # 3 full blocks + 2 tokens
+    assert bm.add_sequence(0, prompt) == 0
+    assert bm.add_sequence(1, prompt) == 48      # full blocks reused, not the partial one
+    t, _ = bm.block_tables([0, 1], 8)
+    assert (t[0, :3] == t[1, :3]).all() and t[0, 3] != t[1, 3]
+    # a difference inside block 1 stops the match after block 0
+    other = list(prompt)
+    other[20] = -5
+    assert bm.add_sequence(2, other) == 16
+    # same tokens, different prefix: the chained hash does not match
+    shifted = [7] * 16 + prompt[16:]
+    assert bm.add_sequence(3, shifted) == 0
+
+
+def test_prefix_cache_survives_free_and_evicts_least_recently_used():
+    nb = 8
+    bm = pkv.BlockManager(nb, BS, seed=7, prefix_caching=True)
+    a = list(range(32))                          # 2 full blocks
+    b = list(range(1000, 1032))
+    bm.add_sequence(0, a)
+    bm.free_sequence(0)
+    bm.add_sequence(1, b)
+    bm.free_sequence(1)
+    st = bm.stats()
+    assert st["evictable"] == 4 and st["used"] == 0
+    assert bm.add_sequence(2, a) == 32           # still cached after its owner ended
+    bm.free_sequence(2)                          # a is now more recently used than b
+    # use up the pool: 4 free blocks, then the oldest cached blocks (b's) go first
+    bm.add_sequence(3, list(range(5000, 5000 + 16 * 6)))
+    assert bm.stats()["evictable"] == 2
+    bm.free_sequence(3)
+    assert bm.add_sequence(4, a) == 32           # a survived
+    assert bm.add_sequence(5, b) == 0            # b was evicted
+
+
+def test_exhaustion_is_reported_and_changes_nothing():
+    bm = pkv.BlockManager(3, BS, seed=8)
+    bm.add_sequence(0, list(range(40)))          # all 3 blocks
+    before = bm.stats()
+    with pytest.raises(pkv.PkvError) as e:
+        bm.add_sequence(1, [1])
+    assert e.value.status == 10
+    with pytest.raises(pkv.PkvError):
+        bm.append_tokens([0] * 9, [1] * 9)       # 8 fit in the last block, the 9th needs a new one
+    assert bm.stats() == before
+    with pytest.raises(pkv.PkvError) as e:
+        bm.fork(5, 6)
+    assert e.value.status == 11
+    with pytest.raises(pkv.PkvError):
+        bm.add_sequence(0, [1])                  # id already in use
