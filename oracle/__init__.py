@@ -79,9 +79,11 @@ def _load():
                                                    i32, i64, i32, f32, i32, i32, i32, i32,
                                                    P, P, P]
             lib.oracle_lse_merge.argtypes = [P, P, P, i32, i32, P]
+            lib.oracle_paged_multi.argtypes = [P, P, P, P, i32, P, P, P, i32, i32, i32, i32,
+                                               i32, i64, i32, f32, i32]
             lib.oracle_lse_merge_f32.argtypes = [P, P, P, i32, i32, P]
             for name in ("oracle_slot_mapping", "oracle_reshape_and_cache",
-                         "oracle_copy_blocks", "oracle_paged_decode",
+                         "oracle_copy_blocks", "oracle_paged_decode", "oracle_paged_multi",
                          "oracle_partition_stats", "oracle_lse_merge",
                          "oracle_lse_merge_f32"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -164,6 +166,30 @@ def paged_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
     _check(_load().oracle_paged_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), code,
                                        _ptr(bt), _ptr(cl), B, Hq, Hkv, D, BS, NB, bt.shape[1],
                                        float(scale), tp, n, threads))
+    return out
+
+
+def paged_multi(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                block_tables: np.ndarray, context_lens: np.ndarray,
+                query_start_loc: np.ndarray, scale: float, threads: int | None = None) -> np.ndarray:
+    """Float64 output of several causal query tokens per sequence.
+
+    q: [T][Hq][D] (sequence s owns rows query_start_loc[s] .. query_start_loc[s+1]-1);
+    returns [T][Hq][D] doubles.
+    """
+    code = _dtype_code(k_cache)
+    assert q.dtype == k_cache.dtype == v_cache.dtype
+    T, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_cache.shape
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+    assert qsl.shape[0] == cl.shape[0] + 1 and qsl[-1] <= T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    threads = threads or len(os.sched_getaffinity(0))
+    _check(_load().oracle_paged_multi(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), code,
+                                      _ptr(bt), _ptr(cl), _ptr(qsl), cl.shape[0], Hq, Hkv, D, BS,
+                                      NB, bt.shape[1], float(scale), threads))
     return out
 
 

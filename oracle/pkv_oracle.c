@@ -409,6 +409,126 @@ int oracle_paged_decode(double *out, const void *q, const void *k_cache,
 }
 
 /* ------------------------------------------------------------------------- */
+/* Several query tokens per sequence (a chunk of new tokens, e.g. speculative
+ * tokens being verified or a slice of a prompt).  The chunk of sequence s is
+ * q rows query_start_loc[s] .. query_start_loc[s+1]-1; its i-th token sits at
+ * position L - n + i (L = context_lens[s] includes the chunk, n = chunk
+ * length) and attends causally: to keys j <= L - n + i.  The layout of the
+ * flattened query rows follows the wiki's "Flattened 布局与 slot_mapping"
+ * (cu_seqlens separate the requests); causality is the plain reading of
+ * autoregressive attention.  With n = 1 this is oracle_paged_decode. */
+typedef struct {
+    const problem *pb;
+    const int32_t *query_start_loc;
+    double *out;
+    int64_t next;
+    int status;
+} multi_pool;
+
+static void *multi_worker(void *arg)
+{
+    multi_pool *mp = arg;
+    const problem *pb = mp->pb;
+    const int32_t D = pb->head_dim;
+    const int32_t group = pb->num_q_heads / pb->num_kv_heads;
+    for (;;) {
+        int64_t task = __atomic_fetch_add(&mp->next, 1, __ATOMIC_RELAXED);
+        if (task >= (int64_t)pb->num_seqs * pb->num_kv_heads) {
+            break;
+        }
+        int32_t seq = (int32_t)(task / pb->num_kv_heads);
+        int32_t kv_head = (int32_t)(task % pb->num_kv_heads);
+        int32_t L, st;
+        st = checked_len(pb, seq, &L);
+        int32_t q0 = mp->query_start_loc[seq], n = mp->query_start_loc[seq + 1] - q0;
+        if (st == ORACLE_OK && (n < 0 || n > L)) {
+            st = ORACLE_BAD_LEN;
+        }
+        double *K = NULL, *V = NULL, *qrow = NULL;
+        if (st == ORACLE_OK) {
+            K = malloc(sizeof(double) * ((size_t)L * D + 1));
+            V = malloc(sizeof(double) * ((size_t)L * D + 1));
+            qrow = malloc(sizeof(double) * (size_t)D);
+            if (!K || !V || !qrow) {
+                st = ORACLE_NO_MEMORY;
+            } else {
+                st = gather_context(pb, seq, kv_head, L, K, V);
+            }
+        }
+        if (st == ORACLE_OK) {
+            for (int32_t i = 0; i < n; ++i) {
+                const int32_t visible = L - n + i + 1;      /* keys 0 .. L-n+i */
+                for (int32_t hg = 0; hg < group; ++hg) {
+                    const int32_t h = kv_head * group + hg;
+                    const int64_t row = (int64_t)(q0 + i) * pb->num_q_heads + h;
+                    for (int32_t d = 0; d < D; ++d) {
+                        qrow[d] = widen(pb->q, row * D + d, pb->dtype);
+                    }
+                    double m, l;
+                    attend_range(qrow, K, V, D, pb->scale, 0, visible, &m, &l, mp->out + row * D);
+                }
+            }
+        } else {
+            int expected = ORACLE_OK;
+            __atomic_compare_exchange_n(&mp->status, &expected, st, 0, __ATOMIC_RELAXED,
+                                        __ATOMIC_RELAXED);
+        }
+        free(K);
+        free(V);
+        free(qrow);
+    }
+    return NULL;
+}
+
+/* out: [num_q_tokens][num_q_heads][head_dim] doubles, q: [num_q_tokens][Hq][D]. */
+int oracle_paged_multi(double *out, const void *q, const void *k_cache, const void *v_cache,
+                       int32_t dtype, const int32_t *block_tables, const int32_t *context_lens,
+                       const int32_t *query_start_loc, int32_t num_seqs, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                       int64_t num_blocks, int32_t max_blocks_per_seq, float scale,
+                       int32_t num_threads)
+{
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
+        !query_start_loc || (dtype != ORACLE_F32 && dtype != ORACLE_BF16) || num_seqs < 0 ||
+        num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+        head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0) {
+        return ORACLE_BAD_ARG;
+    }
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        if (query_start_loc[s + 1] < query_start_loc[s]) {
+            return ORACLE_BAD_ARG;
+        }
+    }
+    problem pb = {q, k_cache, v_cache, dtype, block_tables, context_lens,
+                  num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                  num_blocks, max_blocks_per_seq, (double)scale};
+    multi_pool mp = {&pb, query_start_loc, out, 0, ORACLE_OK};
+    if (num_threads <= 1) {
+        multi_worker(&mp);
+        return mp.status;
+    }
+    pthread_t *threads = malloc(sizeof(pthread_t) * (size_t)num_threads);
+    if (!threads) {
+        return ORACLE_NO_MEMORY;
+    }
+    int started = 0;
+    for (int i = 0; i < num_threads; ++i) {
+        if (pthread_create(&threads[i], NULL, multi_worker, &mp) != 0) {
+            break;
+        }
+        ++started;
+    }
+    if (started == 0) {
+        multi_worker(&mp);
+    }
+    for (int i = 0; i < started; ++i) {
+        pthread_join(threads[i], NULL);
+    }
+    free(threads);
+    return mp.status;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Partitioned attention and the log-sum-exp merge.
  *
  * The pages name online softmax only as a topic; the merge of partial softmax

@@ -36,6 +36,10 @@ MUTANTS = {
                               "memcpy((char *)k_cache + (size_t)pairs[2 * i + 1] * block_bytes,\n               (const char *)k_cache + (size_t)src * block_bytes, (size_t)block_bytes);\n        memcpy(snap_k + (size_t)i * block_bytes,\n               (const char *)k_cache + (size_t)src * block_bytes, (size_t)block_bytes);"),
     "bf16_widen_shift": ("uint32_t bits = (uint32_t)((const uint16_t *)base)[index] << 16;",
                          "uint32_t bits = (uint32_t)((const uint16_t *)base)[index] << 15;"),
+    "multi_not_causal": ("const int32_t visible = L - n + i + 1;      /* keys 0 .. L-n+i */",
+                         "const int32_t visible = L;"),
+    "multi_causal_off_by_one": ("const int32_t visible = L - n + i + 1;      /* keys 0 .. L-n+i */",
+                                "const int32_t visible = L - n + i;"),
     "q_row_of_wrong_head": ("qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + q_head) * D + d, pb->dtype);",
                             "qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + kv_head) * D + d, pb->dtype);"),
 }

@@ -454,3 +454,52 @@ def test_bf16_rounding_of_exact_output_meets_the_tolerance():
     err = np.abs(rounded - ref)
     assert (err <= 2e-2 + 1e-2 * np.abs(ref)).all()
     assert err.max() <= 2.0 ** -8 * np.abs(ref).max()
+
+
+# ------------------------------------------------------- several query tokens ----
+def _multi_case(rng, lens, chunks, hq, hkv, d):
+    q1, kp, vp, bt, cl, Ks, Vs, _ = random_paged(rng, lens, hq, hkv, d)
+    qsl = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    q = rng.standard_normal((int(qsl[-1]), hq, d)).astype(np.float32)
+    return q, kp, vp, bt, cl, Ks, Vs, qsl
+
+
+def test_multi_with_one_token_per_sequence_is_decode():
+    rng = np.random.default_rng(20)
+    lens = [1, 16, 37, 90]
+    q, kp, vp, bt, cl, _, _, _ = random_paged(rng, lens, 8, 2, 16)
+    qsl = np.arange(len(lens) + 1, dtype=np.int32)
+    assert np.array_equal(oracle.paged_multi(q, kp, vp, bt, cl, qsl, 0.3),
+                          oracle.paged_decode(q, kp, vp, bt, cl, 0.3))
+
+
+def test_multi_matches_dense_causal_attention():
+    rng = np.random.default_rng(21)
+    lens, chunks = [5, 33, 64, 70], [5, 4, 1, 16]
+    q, kp, vp, bt, cl, Ks, Vs, qsl = _multi_case(rng, lens, chunks, 8, 2, 16)
+    out = oracle.paged_multi(q, kp, vp, bt, cl, qsl, 0.25)
+    for s, (L, n) in enumerate(zip(lens, chunks)):
+        for i in range(n):
+            p = L - n + i                                  # this token's position
+            row = qsl[s] + i
+            ref = dense_attention(q[row], Ks[s][:p + 1], Vs[s][:p + 1], 0.25)
+            np.testing.assert_allclose(out[row], ref, rtol=0, atol=1e-12)
+
+
+def test_multi_last_token_sees_the_whole_context_and_first_prompt_token_only_itself():
+    rng = np.random.default_rng(22)
+    lens, chunks = [20, 48], [20, 3]               # the first chunk is a whole prompt
+    q, kp, vp, bt, cl, Ks, Vs, qsl = _multi_case(rng, lens, chunks, 4, 4, 8)
+    out = oracle.paged_multi(q, kp, vp, bt, cl, qsl, 0.5)
+    last = qsl[1:] - 1
+    assert np.array_equal(out[last], oracle.paged_decode(np.ascontiguousarray(q[last]), kp, vp,
+                                                         bt, cl, 0.5))
+    for h in range(4):                             # position 0 attends to key 0 alone
+        assert np.array_equal(out[0, h], Vs[0][0, h].astype(np.float64))
+
+
+def test_multi_rejects_chunks_longer_than_the_context():
+    rng = np.random.default_rng(23)
+    q, kp, vp, bt, cl, _, _, qsl = _multi_case(rng, [4], [5], 1, 1, 8)
+    with pytest.raises(oracle.OracleError):
+        oracle.paged_multi(q, kp, vp, bt, cl, qsl, 1.0)
