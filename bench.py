@@ -43,7 +43,7 @@ import workloads  # noqa: E402
 METRIC = "paged decode attn: KV-read GB/s (% of B200 HBM peak), seqs/s at batch"
 UNIT = "GB/s"
 WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shared_prefix",
-             "c5": "c5_long_splitk", "c1": "c1_tiny_fp32"}
+             "c5": "c5_long_splitk", "c1": "c1_tiny_fp32", "c3spec": "c3_spec_decode"}
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")  # JSON text
@@ -87,7 +87,7 @@ def algorithmic_bytes(b: workloads.Batch) -> dict:
     in use and the context lengths."""
     lens = b.context_lens.astype(np.int64)
     table = int(((lens + 15) // 16).sum()) * 4
-    qo = 2 * b.num_seqs * b.num_q_heads * b.head_dim * b.elem_bytes
+    qo = 2 * b.q.shape[0] * b.num_q_heads * b.head_dim * b.elem_bytes
     kv = b.unique_kv_bytes() if b.cow_pairs.shape[0] or b.name == "c4_shared_prefix" else b.kv_bytes()
     return {"kv": kv, "kv_logical": b.kv_bytes(), "q_out": qo, "table": table,
             "lens": 4 * b.num_seqs, "total": kv + qo + table + 4 * b.num_seqs}
@@ -200,11 +200,18 @@ class Step:
         self.dims = pkv.make_dims(b.num_seqs, b.num_q_heads, b.k_cache, b.max_blocks_per_seq)
         self.part_tokens = pkv.decode_partition_tokens(self.dims, self.mcl, partition_tokens)
         self.split = self.part_tokens < self.mcl
-        ws = pkv.decode_workspace_bytes(self.dims, self.mcl, partition_tokens)
+        self.multi = b.query_start_loc is not None
+        if self.multi:
+            self.qsl = torch.from_numpy(b.query_start_loc).to(dev)
+            ws = pkv.load_library().pkv_multi_workspace_bytes(
+                __import__("ctypes").byref(self.dims), b.q.shape[0], self.mcl, partition_tokens)
+        else:
+            ws = pkv.decode_workspace_bytes(self.dims, self.mcl, partition_tokens)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.T = int(b.new_seq.shape[0])
-        self.decode_mode = self.T == b.num_seqs and np.array_equal(b.new_seq, np.arange(b.num_seqs)) \
-            and np.array_equal(b.new_pos, b.context_lens - 1)
+        self.decode_mode = (self.T == b.num_seqs
+                            and np.array_equal(b.new_seq, np.arange(b.num_seqs))
+                            and np.array_equal(b.new_pos, b.context_lens - 1))
         self.seq = torch.from_numpy(b.new_seq).to(dev)
         self.pos = torch.from_numpy(b.new_pos).to(dev)
         self.slots = torch.empty(max(self.T, 1), dtype=torch.int64, device=dev)
@@ -237,7 +244,11 @@ class Step:
                                             workspace_tensor=self.ws)
 
     def decode(self):
-        self.plan_obj.run(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.b.scale)
+        if self.multi:
+            self.plan_obj.run_multi(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.qsl,
+                                    self.b.max_query_len, self.b.scale)
+        else:
+            self.plan_obj.run(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.b.scale)
 
     def __call__(self):
         self.cache_ops()

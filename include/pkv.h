@@ -155,6 +155,47 @@ pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_ca
                                       size_t workspace_bytes, void *cuda_stream);
 
 /*
+ * Several query tokens per sequence: chunks of new tokens (tokens proposed by
+ * speculative decoding and being verified, or a slice of a prompt).  The
+ * chunk of sequence s is rows query_start_loc[s] .. query_start_loc[s+1]-1
+ * of q and out (int32 [num_seqs+1], device, non-decreasing, the cu_seqlens of
+ * the flattened layout); its i-th token sits at position L - n + i, where
+ * L = context_lens[s] already counts the chunk (its K/V written by
+ * reshape_and_cache first) and n is the chunk length, and attends causally
+ * to keys 0 .. L - n + i:
+ *   out[row][h] = softmax_{j <= L-n+i}(scale * q[row][h] . K_j) V_j.
+ * q, out: [num_q_tokens][Hq][D].  max_query_len (host) bounds every chunk;
+ * max_query_len x (Hq/Hkv) must be at most 16 (the query rows of one kv head
+ * share an MMA tile).  A chunk longer than max_query_len or than its context
+ * is clamped, and a chunk reaching outside rows [0, num_q_tokens) is skipped;
+ * both are flagged PKV_DEVERR_LEN.  With n = 1 everywhere this is
+ * pkv_paged_attention_decode.  Workspace: pkv_multi_workspace_bytes().
+ */
+size_t pkv_multi_workspace_bytes(const pkv_dims *dims, int32_t num_q_tokens,
+                                 int32_t max_context_len, int32_t partition_tokens);
+
+pkv_status pkv_paged_attention_multi(void *out, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *block_tables,
+                                     const int32_t *context_lens, const int32_t *query_start_loc,
+                                     int32_t num_q_tokens, int32_t max_query_len, float scale,
+                                     const pkv_dims *dims, int32_t max_context_len,
+                                     int32_t partition_tokens, void *workspace,
+                                     size_t workspace_bytes, void *cuda_stream);
+
+/*
+ * The run half of pkv_paged_attention_multi, over a plan made by
+ * pkv_decode_plan (the plan depends only on the context lengths); the same
+ * rules as pkv_decode_run apply, with the workspace sized by
+ * pkv_multi_workspace_bytes.
+ */
+pkv_status pkv_multi_run(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, const int32_t *context_lens,
+                         const int32_t *query_start_loc, int32_t num_q_tokens,
+                         int32_t max_query_len, float scale, const pkv_dims *dims,
+                         int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                         size_t workspace_bytes, void *cuda_stream);
+
+/*
  * The two halves of pkv_paged_attention_decode, for callers that decode
  * several layers (several cache pools) with the same context lengths: plan
  * once per step, run once per layer.

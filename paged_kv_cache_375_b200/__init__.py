@@ -73,6 +73,11 @@ def load_library() -> ctypes.CDLL:
             "pkv_paged_attention_decode": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P,
                                                           sz, P]),
             "pkv_decode_plan": (ctypes.c_int, [P, D, i32, i32, P, sz, P]),
+            "pkv_multi_workspace_bytes": (sz, [D, i32, i32, i32]),
+            "pkv_multi_run": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, D, i32, i32, P,
+                                             sz, P]),
+            "pkv_paged_attention_multi": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, D,
+                                                         i32, i32, P, sz, P]),
             "pkv_decode_run": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P, sz, P]),
             "pkv_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
             "pkv_copy_blocks": (ctypes.c_int, [P, P, P, i32, D, P]),
@@ -219,6 +224,46 @@ def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Te
     return out
 
 
+def paged_attention_multi(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                          v_cache: torch.Tensor, block_tables: torch.Tensor,
+                          context_lens: torch.Tensor, query_start_loc: torch.Tensor,
+                          scale: float, num_kv_heads: int, max_query_len: int, *,
+                          max_context_len: int | None = None, partition_tokens: int = 0,
+                          workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
+    """Causal attention of several query tokens per sequence over the paged context.
+
+    q, out: [T][Hq][D]; query_start_loc: int32 [B+1] (sequence s owns rows
+    query_start_loc[s] .. query_start_loc[s+1]-1, at positions L-n .. L-1 of its context,
+    L = context_lens[s] including the chunk).  max_query_len * (Hq/Hkv) <= 16.
+    """
+    dev = q.device
+    _need(q, "q", device=dev)
+    _need(out, "out", q.dtype, dev)
+    _need(k_cache, "k_cache", q.dtype, dev)
+    _need(v_cache, "v_cache", q.dtype, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    _need(query_start_loc, "query_start_loc", torch.int32, dev)
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape or k_cache.shape[1] != num_kv_heads:
+        raise ValueError("k_cache and v_cache must be [num_blocks][num_kv_heads][16][head_dim]")
+    T, hq, d = q.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or query_start_loc.shape != (B + 1,) or block_tables.shape[0] != B:
+        raise ValueError("inconsistent shapes")
+    dims = make_dims(B, hq, k_cache, block_tables.shape[1])
+    mcl = block_tables.shape[1] * k_cache.shape[2] if max_context_len is None else int(max_context_len)
+    lib = load_library()
+    need = lib.pkv_multi_workspace_bytes(ctypes.byref(dims), T, mcl, partition_tokens)
+    if need == 0:
+        raise PkvError(2, lib.pkv_last_error_message().decode())
+    ws = workspace_tensor if workspace_tensor is not None else workspace(dev, need)
+    _check(lib.pkv_paged_attention_multi(
+        _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+        _p(query_start_loc), T, int(max_query_len), float(scale), ctypes.byref(dims), mcl,
+        partition_tokens, _p(ws), ws.numel(), _stream_ptr(dev)))
+    return out
+
+
 class DecodePlan:
     """A decode plan for one step: the work list built from context_lens, kept in a
     workspace.  ``run`` decodes one layer's cache pools with it; plan once per step, run
@@ -247,6 +292,27 @@ class DecodePlan:
                                               self.max_context_len, partition_tokens,
                                               _p(self.workspace), self.workspace.numel(),
                                               _stream_ptr(dev)))
+
+    def run_multi(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor, query_start_loc: torch.Tensor, max_query_len: int,
+                  scale: float) -> torch.Tensor:
+        """Several causal query tokens per sequence (see paged_attention_multi) over this
+        plan; the plan's workspace must hold pkv_multi_workspace_bytes for q's rows."""
+        dev = q.device
+        _need(q, "q", device=dev)
+        _need(out, "out", q.dtype, dev)
+        _need(query_start_loc, "query_start_loc", torch.int32, dev)
+        need = load_library().pkv_multi_workspace_bytes(ctypes.byref(self.dims), q.shape[0],
+                                                        self.max_context_len,
+                                                        self.partition_tokens)
+        if need == 0 or self.workspace.numel() < need:
+            raise PkvError(4, f"workspace too small for {q.shape[0]} query rows ({need} bytes)")
+        _check(load_library().pkv_multi_run(
+            _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
+            _p(self.context_lens), _p(query_start_loc), q.shape[0], int(max_query_len),
+            float(scale), ctypes.byref(self.dims), self.max_context_len, self.partition_tokens,
+            _p(self.workspace), self.workspace.numel(), _stream_ptr(dev)))
+        return out
 
     def run(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
             v_cache: torch.Tensor, scale: float) -> torch.Tensor:

@@ -119,7 +119,8 @@ struct DecodePlan {
   int32_t part_tokens = 0;
   int32_t part_blocks = 0;
   int32_t max_parts = 0;
-  int32_t max_len = 0;  // lengths above this are clamped (and flagged)
+  int32_t max_len = 0;       // lengths above this are clamped (and flagged)
+  int32_t num_q_tokens = 0;  // query rows of q and out (num_seqs for decode)
   size_t items_off = 0, part_o_off = 0, part_ml_off = 0, total = 0;
 };
 
@@ -141,8 +142,9 @@ int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested) 
   return static_cast<int32_t>(p);
 }
 
+// num_q_tokens < 0: one query token per sequence (decode).
 pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partition_tokens,
-                     DecodePlan* plan) {
+                     DecodePlan* plan, int32_t num_q_tokens = -1) {
   pkv_status st = check_dims(d, true);
   if (st != PKV_OK) return st;
   if (max_context_len < 0) return fail(PKV_ERR_SHAPE, "max_context_len must be >= 0");
@@ -156,11 +158,12 @@ pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partiti
       static_cast<int32_t>(max_context_len < table_len ? max_context_len : table_len);
   DecodePlan p;
   p.max_len = max_len;
+  p.num_q_tokens = num_q_tokens < 0 ? d->num_seqs : num_q_tokens;
   p.part_tokens = choose_partition(d, max_len, partition_tokens);
   p.part_blocks = p.part_tokens / pkv::kBlock;
   p.max_parts = max_len <= 0 ? 1 : (max_len + p.part_tokens - 1) / p.part_tokens;
   const size_t B = static_cast<size_t>(d->num_seqs);
-  const size_t rows = B * d->num_q_heads * p.max_parts;
+  const size_t rows = static_cast<size_t>(p.num_q_tokens) * d->num_q_heads * p.max_parts;
   p.items_off = 256;
   size_t off = round_up(p.items_off + B * p.max_parts * sizeof(pkv::PlanItem), 256);
   if (p.max_parts > 1) {
@@ -213,19 +216,17 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d
 }
 
 // Kernel configuration: W decode warps per CTA (one CTA per SM), S tile
-// stages per warp.  Eight decode warps with two stages each hide the latency
-// of the per-tile math best (measured on B200); groups of more than 8 query
-// heads at head_dim 128 need a merge area too large for that, and use four
-// warps with four stages.  fp32 tiles are twice as large, so fp32 keeps
-// fewer stages (one for the largest group at head_dim 128).
+// stages per warp, MB merge buffers.  Eight decode warps with two stages each
+// hide the latency of the per-tile math best (measured on B200).  With 16
+// query rows per kv head at head_dim 128 a second merge buffer does not fit,
+// so that case keeps one.  fp32 tiles are twice as large: four warps.
 template <typename T, int D, int GMAX>
 struct DecodeCfg {
-  static constexpr bool kBig = (D == 128 && GMAX == 16);
-  static constexpr int W = kBig ? 4 : 8, S = kBig ? 4 : 2;
+  static constexpr int W = 8, S = 2, MB = (D == 128 && GMAX == 16) ? 1 : 2;
 };
 template <int D, int GMAX>
 struct DecodeCfg<float, D, GMAX> {
-  static constexpr int W = 4, S = (D == 128 && GMAX == 16) ? 1 : 2;
+  static constexpr int W = 4, S = 2, MB = (D == 128 && GMAX == 16) ? 1 : 2;
 };
 
 // Largest dynamic shared memory already enabled per kernel, per device.
@@ -257,18 +258,19 @@ cudaError_t ensure_smem(const void* fn, int bytes) {
 
 template <typename T, int D, int GMAX>
 pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
-                         const pkv::DecodeParams& prm, int64_t work_units, int g,
+                         const pkv::DecodeParams& prm, int64_t work_units, int rows_max,
                          cudaStream_t stream) {
   constexpr int W = DecodeCfg<T, D, GMAX>::W, S = DecodeCfg<T, D, GMAX>::S;
-  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S>;
-  const int smem = Lay::total_bytes(g);
+  constexpr int MB = DecodeCfg<T, D, GMAX>::MB;
+  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S, MB>;
+  const int smem = Lay::total_bytes(rows_max);
   int dev = 0, max_optin = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (smem > max_optin)
     return fail(PKV_ERR_UNSUPPORTED, "decode needs %d bytes of shared memory (> %d)", smem,
                 max_optin);
-  auto kern = pkv::decode_kernel<T, D, GMAX, W, S>;
+  auto kern = pkv::decode_kernel<T, D, GMAX, W, S, MB>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   int per_sm = 0;
@@ -284,12 +286,16 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
   return PKV_OK;
 }
 
+// The query rows of an item (chunk length x group) go on the MMA's N side:
+// up to 8 or up to 16 rows.
 template <typename T, int D>
 pkv_status launch_decode_d(const CUtensorMap& mk, const CUtensorMap& mv,
-                           const pkv::DecodeParams& prm, int64_t work_units, int g,
+                           const pkv::DecodeParams& prm, int64_t work_units, int rows_max,
                            cudaStream_t stream) {
-  if (g <= 8) return launch_decode<T, D, 8>(mk, mv, prm, work_units, g, stream);
-  return launch_decode<T, D, 16>(mk, mv, prm, work_units, g, stream);
+  if (rows_max <= 8) return launch_decode<T, D, 8>(mk, mv, prm, work_units, rows_max, stream);
+  if (rows_max <= 16) return launch_decode<T, D, 16>(mk, mv, prm, work_units, rows_max, stream);
+  return fail(PKV_ERR_UNSUPPORTED, "query rows per kv head (chunk length x group = %d) > 16",
+              rows_max);
 }
 
 pkv_status check_workspace(const DecodePlan& plan, const void* workspace, size_t bytes) {
@@ -303,15 +309,16 @@ pkv_status check_workspace(const DecodePlan& plan, const void* workspace, size_t
 
 template <typename T>
 pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
-                        const int32_t* context_lens, const pkv_dims* d, cudaStream_t stream) {
-  const int64_t rows = static_cast<int64_t>(d->num_seqs) * d->num_q_heads;
+                        const int32_t* context_lens, const int32_t* query_start_loc,
+                        const pkv_dims* d, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(plan.num_q_tokens) * d->num_q_heads;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
   const float* po = reinterpret_cast<const float*>(ws + plan.part_o_off);
   const float* pml = reinterpret_cast<const float*>(ws + plan.part_ml_off);
   auto kern = d->head_dim == 128 ? pkv::merge_kernel<T, 128> : pkv::merge_kernel<T, 64>;
   cudaError_t e = launch(kern, dim3(grid), dim3(128), 0, stream, out, po, pml, context_lens,
-                         d->num_seqs, d->num_q_heads, plan.max_parts, plan.max_len,
-                         plan.part_tokens);
+                         query_start_loc, d->num_seqs, plan.num_q_tokens, d->num_q_heads,
+                         plan.max_parts, plan.max_len, plan.part_tokens);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return PKV_OK;
 }
@@ -341,6 +348,72 @@ pkv_status static_workspace(void** ptr) {
   }
   *ptr = g_static_ws_ptr[dev];
   return PKV_OK;
+}
+
+// Decode (and merge) over a plan already in the workspace.  query_start_loc
+// NULL: one query token per sequence; otherwise chunks of up to max_query_len
+// causal query tokens.
+pkv_status run_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens,
+                      const int32_t* query_start_loc, int32_t max_query_len, float scale,
+                      const pkv_dims* d, const DecodePlan& plan, void* workspace,
+                      size_t workspace_bytes, void* cuda_stream) {
+  pkv_status st;
+  if (d->num_seqs == 0 || plan.num_q_tokens == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  if (max_query_len < 1) return fail(PKV_ERR_SHAPE, "max_query_len must be >= 1");
+  const int group = d->num_q_heads / d->num_kv_heads;
+  const int rows_max = max_query_len * group;
+  if (rows_max > 16)
+    return fail(PKV_ERR_UNSUPPORTED, "chunk length x group = %d > 16 query rows per kv head",
+                rows_max);
+  if ((st = bind_device(out, "out")) != PKV_OK) return st;
+  CUtensorMap mk, mv;
+  if ((st = encode_pool_map(&mk, k_cache, d)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&mv, v_cache, d)) != PKV_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  pkv::DecodeParams prm;
+  prm.out = out;
+  prm.q = q;
+  prm.block_tables = block_tables;
+  prm.items = reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off);
+  prm.counters = reinterpret_cast<uint32_t*>(ws);
+  prm.part_o = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_o_off) : nullptr;
+  prm.part_ml = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_ml_off) : nullptr;
+  prm.query_start_loc = query_start_loc;
+  prm.max_query_len = max_query_len;
+  prm.num_q_tokens = plan.num_q_tokens;
+  prm.num_q_heads = d->num_q_heads;
+  prm.num_kv_heads = d->num_kv_heads;
+  prm.group = group;
+  prm.max_blocks_per_seq = d->max_blocks_per_seq;
+  prm.num_blocks = d->num_blocks;
+  prm.max_parts = plan.max_parts;
+  prm.part_blocks = plan.part_blocks;
+  prm.qk_scale_log2 = scale * pkv::kLog2e;
+  const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads;
+  if (d->dtype == PKV_BF16) {
+    st = d->head_dim == 128
+             ? launch_decode_d<__nv_bfloat16, 128>(mk, mv, prm, units, rows_max, stream)
+             : launch_decode_d<__nv_bfloat16, 64>(mk, mv, prm, units, rows_max, stream);
+  } else {
+    st = d->head_dim == 128 ? launch_decode_d<float, 128>(mk, mv, prm, units, rows_max, stream)
+                            : launch_decode_d<float, 64>(mk, mv, prm, units, rows_max, stream);
+  }
+  if (st != PKV_OK) return st;
+  if (plan.max_parts > 1) {
+    st = d->dtype == PKV_BF16
+             ? launch_merge<__nv_bfloat16>(out, plan, ws, context_lens, query_start_loc, d, stream)
+             : launch_merge<float>(out, plan, ws, context_lens, query_start_loc, d, stream);
+  }
+  return st;
 }
 
 }  // namespace
@@ -402,54 +475,8 @@ pkv_status pkv_decode_run(void* out, const void* q, const void* k_cache, const v
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
-  const pkv_dims* d = dims;
-  if (d->num_seqs == 0) return PKV_OK;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
-    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
-  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
-    return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
-  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
-  if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
-  if ((st = bind_device(out, "out")) != PKV_OK) return st;
-  CUtensorMap mk, mv;
-  if ((st = encode_pool_map(&mk, k_cache, d)) != PKV_OK) return st;
-  if ((st = encode_pool_map(&mv, v_cache, d)) != PKV_OK) return st;
-  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(ws);
-  pkv::PlanItem* items = reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off);
-
-  pkv::DecodeParams prm;
-  prm.out = out;
-  prm.q = q;
-  prm.block_tables = block_tables;
-  prm.items = items;
-  prm.counters = counters;
-  prm.part_o = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_o_off) : nullptr;
-  prm.part_ml = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_ml_off) : nullptr;
-  prm.num_q_heads = d->num_q_heads;
-  prm.num_kv_heads = d->num_kv_heads;
-  prm.group = d->num_q_heads / d->num_kv_heads;
-  prm.max_blocks_per_seq = d->max_blocks_per_seq;
-  prm.num_blocks = d->num_blocks;
-  prm.max_parts = plan.max_parts;
-  prm.part_blocks = plan.part_blocks;
-  prm.qk_scale_log2 = scale * pkv::kLog2e;
-  const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads;
-  if (d->dtype == PKV_BF16) {
-    st = d->head_dim == 128
-             ? launch_decode_d<__nv_bfloat16, 128>(mk, mv, prm, units, prm.group, stream)
-             : launch_decode_d<__nv_bfloat16, 64>(mk, mv, prm, units, prm.group, stream);
-  } else {
-    st = d->head_dim == 128 ? launch_decode_d<float, 128>(mk, mv, prm, units, prm.group, stream)
-                            : launch_decode_d<float, 64>(mk, mv, prm, units, prm.group, stream);
-  }
-  if (st != PKV_OK) return st;
-  if (plan.max_parts > 1) {
-    st = d->dtype == PKV_BF16 ? launch_merge<__nv_bfloat16>(out, plan, ws, context_lens, d, stream)
-                              : launch_merge<float>(out, plan, ws, context_lens, d, stream);
-  }
-  return st;
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
+                    dims, plan, workspace, workspace_bytes, cuda_stream);
 }
 
 pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_cache,
@@ -475,6 +502,53 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   return pkv_decode_run(out, q, k_cache, v_cache, block_tables, context_lens, scale, dims,
                         max_context_len, partition_tokens, workspace, workspace_bytes,
                         cuda_stream);
+}
+
+size_t pkv_multi_workspace_bytes(const pkv_dims* dims, int32_t num_q_tokens,
+                                 int32_t max_context_len, int32_t partition_tokens) {
+  DecodePlan plan;
+  if (num_q_tokens < 0) return 0;
+  if (make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens) != PKV_OK) return 0;
+  return plan.total;
+}
+
+pkv_status pkv_multi_run(void* out, const void* q, const void* k_cache, const void* v_cache,
+                         const int32_t* block_tables, const int32_t* context_lens,
+                         const int32_t* query_start_loc, int32_t num_q_tokens,
+                         int32_t max_query_len, float scale, const pkv_dims* dims,
+                         int32_t max_context_len, int32_t partition_tokens, void* workspace,
+                         size_t workspace_bytes, void* cuda_stream) {
+  if (num_q_tokens < 0) return fail(PKV_ERR_SHAPE, "num_q_tokens must be >= 0");
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
+  if (st != PKV_OK) return st;
+  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
+  if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                    max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream);
+}
+
+pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, const int32_t* query_start_loc,
+                                     int32_t num_q_tokens, int32_t max_query_len, float scale,
+                                     const pkv_dims* dims, int32_t max_context_len,
+                                     int32_t partition_tokens, void* workspace,
+                                     size_t workspace_bytes, void* cuda_stream) {
+  if (num_q_tokens < 0) return fail(PKV_ERR_SHAPE, "num_q_tokens must be >= 0");
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
+  if (st != PKV_OK) return st;
+  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
+  if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
+  if (max_query_len < 1 || (max_query_len * (dims->num_q_heads / dims->num_kv_heads)) > 16)
+    return fail(PKV_ERR_UNSUPPORTED, "max_query_len x group must be in [1, 16]");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  st = pkv_decode_plan(context_lens, dims, max_context_len, partition_tokens, workspace,
+                       workspace_bytes, cuda_stream);
+  if (st != PKV_OK) return st;
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                    max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream);
 }
 
 pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_cache,

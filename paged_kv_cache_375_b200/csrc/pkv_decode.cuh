@@ -143,13 +143,18 @@ __global__ void __launch_bounds__(kPlanThreads)
 
 // ------------------------------------------------------------ decode kernel
 struct DecodeParams {
-  void* out;                     // [B][Hq][D], dtype of the cache
-  const void* q;                 // [B][Hq][D]
+  void* out;                     // [T][Hq][D], dtype of the cache (T query tokens)
+  const void* q;                 // [T][Hq][D]
   const int32_t* block_tables;   // [B][MB]
   const PlanItem* items;         // planned work, longest first
   uint32_t* counters;            // [0] work counter, [1] number of items, [2] CTAs done
-  float* part_o;                 // [B][Hq][max_parts][D]
-  float* part_ml;                // [B][Hq][max_parts][2]
+  float* part_o;                 // [T][Hq][max_parts][D]
+  float* part_ml;                // [T][Hq][max_parts][2]
+  // Query tokens of sequence s: rows query_start_loc[s] .. query_start_loc[s+1]-1
+  // at positions L-n .. L-1 (causal); NULL means one token per sequence, row s.
+  const int32_t* query_start_loc;
+  int32_t max_query_len;         // longest chunk; chunk length x group <= GMAX
+  int32_t num_q_tokens;          // rows of q and out
   int32_t num_q_heads;
   int32_t num_kv_heads;
   int32_t group;                 // Hq / Hkv
@@ -165,7 +170,10 @@ struct DecodeParams {
 constexpr int kMaxItemBlocks = 512;
 
 // Shared-memory map of the decode kernel (offsets from a 1024-aligned base).
-template <int ELEM, int D, int GMAX, int W, int S>
+// MB merge buffers: with two, consecutive items alternate buffers and one
+// barrier per item suffices; with one (when two do not fit), a second
+// barrier keeps the next item's states out until the current one is combined.
+template <int ELEM, int D, int GMAX, int W, int S, int MB = 2>
 struct DecodeLayout {
   static constexpr int kTileBytes = kBlock * D * ELEM;       // one K (or V) tile
   static constexpr int kChunks = D * ELEM / 128;             // 128-byte column chunks
@@ -179,9 +187,9 @@ struct DecodeLayout {
   // chosen at run time; every warp's slot starts 16-byte aligned.
   __host__ __device__ static int merge_floats_per_warp(int g) { return g * D + (2 * g + 3) / 4 * 4; }
   __host__ __device__ static int meta_off(int g) {
-    return kMergeOff + 2 * W * merge_floats_per_warp(g) * 4;
+    return kMergeOff + MB * W * merge_floats_per_warp(g) * 4;
   }
-  static constexpr int kMetaBytes = kRing * 32;
+  static constexpr int kMetaBytes = kRing * 64;
   __host__ __device__ static int bars_off(int g) { return (meta_off(g) + kMetaBytes + 7) / 8 * 8; }
   static constexpr int kNumBars = W * S + 2 * kRing + 2;
   __host__ __device__ static int flags_off(int g) { return bars_off(g) + kNumBars * 8; }
@@ -191,7 +199,8 @@ struct DecodeLayout {
 };
 
 struct ItemMeta {
-  int32_t seq, kv_head, part, len, nparts, blk_begin, nblk, pad;
+  int32_t seq, kv_head, part, len, nparts, blk_begin, nblk;
+  int32_t q_start, q_len;        // query rows of the chunk and its length
 };
 
 // ---- consumer state for bf16 (tensor cores) ----
@@ -214,13 +223,16 @@ struct Bf16State {
   static constexpr int NH = GMAX / 8;  // n-tiles of query heads
   uint32_t qb[NH][KS][2];              // B fragments of Q^T
   float o[NH][MT][4];                  // O^T accumulators
-  float m[NH][2];                      // running max of heads 8nh + 2(lane%4) + {0,1}
+  float m[NH][2];                      // running max of rows 8nh + 2(lane%4) + {0,1}
   float l[NH][2];                      // this lane's part of the softmax denominators
+  int32_t lim[NH][2];                  // last key position those rows may see (causal)
 };
 
+// Query rows of an item: row n = i*g + h is chunk token i (at position
+// len - q_len + i) and query head h of the group; `rows` = q_len * g.
 template <int D, int GMAX>
 __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const uint8_t* qs,
-                                                int g, int lane) {
+                                                int rows, int g, int len, int q_len, int lane) {
   using St = Bf16State<D, GMAX>;
   const int r = lane >> 2, qd = (lane & 3) * 2;
   const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qs);
@@ -230,8 +242,13 @@ __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const ui
 #pragma unroll
     for (int ks = 0; ks < St::KS; ++ks) {
       const int c = ks * 16 + qd;
-      st.qb[nh][ks][0] = head < g ? *reinterpret_cast<const uint32_t*>(q16 + head * D + c) : 0u;
-      st.qb[nh][ks][1] = head < g ? *reinterpret_cast<const uint32_t*>(q16 + head * D + c + 8) : 0u;
+      st.qb[nh][ks][0] = head < rows ? *reinterpret_cast<const uint32_t*>(q16 + head * D + c) : 0u;
+      st.qb[nh][ks][1] = head < rows ? *reinterpret_cast<const uint32_t*>(q16 + head * D + c + 8) : 0u;
+    }
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int n = nh * 8 + qd + hc;
+      st.lim[nh][hc] = n < rows ? len - q_len + n / g : -1;
     }
 #pragma unroll
     for (int mt = 0; mt < St::MT; ++mt) {
@@ -243,11 +260,13 @@ __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const ui
 }
 
 // Two 16-token tiles (the second may be absent: valid1 = 0 and its pointers
-// equal the first's).  validX tokens of tile X belong to the context.
+// equal the first's).  validX tokens of tile X belong to the context; its
+// first token sits at position posX.
 template <int D, int GMAX>
 __device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t* k0,
-                                          const uint8_t* v0, int valid0, const uint8_t* k1,
-                                          const uint8_t* v1, int valid1, float sc, int lane) {
+                                          const uint8_t* v0, int valid0, int pos0,
+                                          const uint8_t* k1, const uint8_t* v1, int valid1,
+                                          int pos1, float sc, int lane) {
   using St = Bf16State<D, GMAX>;
   constexpr int NH = St::NH;
   const int r = lane >> 2, qd = (lane & 3) * 2;
@@ -283,12 +302,14 @@ __device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t*
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int valid = t ? valid1 : valid0;
+    const int pos = t ? pos1 : pos0;
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        const int tok = r + 8 * (i >> 1);
         const float v = (s[t][0][nh][i] + s[t][1][nh][i]) * sc;
-        z[t][nh][i] = (r + 8 * (i >> 1)) < valid ? v : -INFINITY;
+        z[t][nh][i] = (tok < valid && pos + tok <= st.lim[nh][i & 1]) ? v : -INFINITY;
       }
   }
   // ---- running max per head column, lazy rescale ----
@@ -374,8 +395,9 @@ __device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t*
 
 // Write this warp's (m, l, O) rows into its slot of the merge area.
 template <int D, int GMAX>
-__device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot, int g,
+__device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot, int rows,
                                              int lane) {
+  const int g = rows;  // the slot holds `rows` rows
   using St = Bf16State<D, GMAX>;
   const int r = lane >> 2, qd = (lane & 3) * 2;
   float* O = slot;
@@ -410,12 +432,15 @@ struct F32State {
   static constexpr int NV = D / 32;  // output columns per lane
   float o[GMAX][NV];
   float m[GMAX], l[GMAX];
+  int32_t lim[GMAX];                 // last key position each row may see (causal)
 };
 
 template <int D, int GMAX>
-__device__ __forceinline__ void f32_begin_item(F32State<D, GMAX>& st) {
+__device__ __forceinline__ void f32_begin_item(F32State<D, GMAX>& st, int rows, int g, int len,
+                                               int q_len) {
 #pragma unroll
   for (int h = 0; h < GMAX; ++h) {
+    st.lim[h] = h < rows ? len - q_len + h / g : -1;
     st.m[h] = -INFINITY;
     st.l[h] = 0.f;
 #pragma unroll
@@ -426,7 +451,7 @@ __device__ __forceinline__ void f32_begin_item(F32State<D, GMAX>& st) {
 template <int D, int GMAX>
 __device__ __forceinline__ void f32_block(F32State<D, GMAX>& st, const float* qs,
                                           const uint8_t* ktile, const uint8_t* vtile, int valid,
-                                          float sc, int g, int lane) {
+                                          int pos, float sc, int g, int lane) {
   constexpr int NV = F32State<D, GMAX>::NV;
   const int t = lane & 15, hf = lane >> 4;
   float acc[GMAX];
@@ -451,7 +476,7 @@ __device__ __forceinline__ void f32_block(F32State<D, GMAX>& st, const float* qs
   for (int h = 0; h < GMAX; ++h) {
     if (h < g) {
       float a = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 16);
-      const float z = t < valid ? a * sc : -INFINITY;
+      const float z = (t < valid && pos + t <= st.lim[h]) ? a * sc : -INFINITY;
       float mx = z;
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
@@ -511,13 +536,14 @@ __device__ __forceinline__ void f32_publish(F32State<D, GMAX>& st, float* slot, 
 }
 
 // ---- combine the W warps' states of one item and store the result ----
+// The item's `rows` rows are chunk token i = n / group, head n % group.
 template <typename T, int D, int W>
 __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const ItemMeta& it,
-                                                  const float* merge, int per_warp, int g,
+                                                  const float* merge, int per_warp, int rows,
                                                   int warp, int lane) {
   const int tid = warp * 32 + lane;
-  const int row0 = it.seq * prm.num_q_heads + it.kv_head * g;  // first q-head row of the group
-  for (int e = tid * 4; e < g * D; e += W * 32 * 4) {
+  const int g = rows;  // merge-slot layout: rows x D outputs, then rows maxima and sums
+  for (int e = tid * 4; e < rows * D; e += W * 32 * 4) {
     const int h = e / D, d = e % D;
     float M = -INFINITY;
 #pragma unroll
@@ -542,7 +568,9 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
       acc.z *= inv;
       acc.w *= inv;
     }
-    const size_t row = static_cast<size_t>(row0 + h);
+    const int group = prm.group;
+    const size_t row = static_cast<size_t>(it.q_start + h / group) * prm.num_q_heads +
+                       it.kv_head * group + h % group;
     if (it.nparts == 1) {
       if constexpr (sizeof(T) == 2) {
         uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
@@ -570,27 +598,28 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
 // flight, following its share of the items (blocks w, w+W, ... of each) and
 // running ahead into the next items while it computes.  At the end of an item
 // the W warps combine their online-softmax states through shared memory.
-template <typename T, int D, int GMAX, int W, int S>
-__global__ void __launch_bounds__((W + 1) * 32)
+template <typename T, int D, int GMAX, int W, int S, int MB>
+__global__ void __launch_bounds__((W + 1) * 32, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
   constexpr int ELEM = sizeof(T);
-  using Lay = DecodeLayout<ELEM, D, GMAX, W, S>;
+  using Lay = DecodeLayout<ELEM, D, GMAX, W, S, MB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int g = prm.group;
+  const int rows_max = prm.max_query_len * g;  // query rows of the largest item
   uint8_t* stages = smem + Lay::kStagesOff;
   uint8_t* ring = smem + Lay::kRingOff;
   int32_t* tables = reinterpret_cast<int32_t*>(smem + Lay::kTablesOff);  // [kRing][kMaxItemBlocks]
   float* merge = reinterpret_cast<float*>(smem + Lay::kMergeOff);
-  ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + Lay::meta_off(g));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off(g));
+  ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + Lay::meta_off(rows_max));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off(rows_max));
   uint64_t* full = bars;                       // [W][S]
   uint64_t* item_full = bars + W * S;          // [kRing]
   uint64_t* item_empty = item_full + kRing;    // [kRing]
   uint64_t* merge_bar = item_empty + kRing;    // [2]
-  uint32_t* stage_ok = reinterpret_cast<uint32_t*>(smem + Lay::flags_off(g));  // [W][S]
+  uint32_t* stage_ok = reinterpret_cast<uint32_t*>(smem + Lay::flags_off(rows_max));  // [W][S]
   volatile uint32_t* abort_flag = stage_ok + W * S;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -652,6 +681,22 @@ __global__ void __launch_bounds__((W + 1) * 32)
                            static_cast<size_t>(pi.seq) * prm.max_blocks_per_seq + blk_begin;
       int32_t* dst = tables + r * kMaxItemBlocks;
       for (int32_t j = lane; j < nblk; j += 32) dst[j] = src[j];
+      // the chunk of query tokens: one per sequence unless query_start_loc is given
+      int32_t q_start = pi.seq, q_len = 1;
+      if (prm.query_start_loc) {
+        q_start = prm.query_start_loc[pi.seq];
+        q_len = prm.query_start_loc[pi.seq + 1] - q_start;
+        const int32_t cap = pi.len < prm.max_query_len ? pi.len : prm.max_query_len;
+        if (q_len < 0 || q_len > cap) {
+          if (lane == 0 && kvh == 0 && pi.part == 0) raise_error(PKV_DEVERR_LEN);
+          q_len = q_len < 0 ? 0 : cap;
+        }
+        if (q_start < 0 || q_start + q_len > prm.num_q_tokens) {  // rows outside q / out
+          if (lane == 0 && kvh == 0 && pi.part == 0) raise_error(PKV_DEVERR_LEN);
+          q_start = 0;
+          q_len = 0;
+        }
+      }
       __syncwarp();
       if (lane == 0) {
         ItemMeta& mt = meta[r];
@@ -662,11 +707,20 @@ __global__ void __launch_bounds__((W + 1) * 32)
         mt.nparts = pi.nparts;
         mt.blk_begin = blk_begin;
         mt.nblk = nblk;
-        const uint32_t qbytes = static_cast<uint32_t>(g * D * ELEM);
-        mbar_arrive_expect_tx(&item_full[r], qbytes);
-        const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(prm.q) +
-                              (static_cast<size_t>(pi.seq) * prm.num_q_heads + kvh * g) * D * ELEM;
-        bulk_load(ring + r * Lay::kQBytes, qsrc, qbytes, &item_full[r]);
+        mt.q_start = q_start;
+        mt.q_len = q_len;
+        const uint32_t row_bytes = static_cast<uint32_t>(g * D * ELEM);  // one token's group
+        if (q_len > 0) {
+          mbar_arrive_expect_tx(&item_full[r], row_bytes * q_len);
+          for (int32_t i = 0; i < q_len; ++i) {
+            const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(prm.q) +
+                                  (static_cast<size_t>(q_start + i) * prm.num_q_heads + kvh * g) *
+                                      D * ELEM;
+            bulk_load(ring + r * Lay::kQBytes + i * row_bytes, qsrc, row_bytes, &item_full[r]);
+          }
+        } else {
+          mbar_arrive(&item_full[r]);
+        }
       }
     }
     if (!ok) {
@@ -688,7 +742,7 @@ __global__ void __launch_bounds__((W + 1) * 32)
   constexpr bool kBf16 = sizeof(T) == 2;
   typename std::conditional<kBf16, Bst, Fst>::type st;
   const float sc = prm.qk_scale_log2;
-  const int per_warp = Lay::merge_floats_per_warp(g);
+  const int per_warp = Lay::merge_floats_per_warp(rows_max);
   uint64_t* my_full = full + warp * S;
   uint32_t* my_ok = stage_ok + warp * S;
   uint8_t* my_stages = stages + warp * S * Lay::kStageBytes;
@@ -765,10 +819,11 @@ __global__ void __launch_bounds__((W + 1) * 32)
     const ItemMeta it = meta[r];
     if (it.seq < 0) break;
     const uint8_t* qs = ring + r * Lay::kQBytes;
+    const int rows = it.q_len * g;  // query rows of this item
     if constexpr (kBf16) {
-      bf16_begin_item<D, GMAX>(st, qs, g, lane);
+      bf16_begin_item<D, GMAX>(st, qs, rows, g, it.len, it.q_len, lane);
     } else {
-      f32_begin_item<D, GMAX>(st);
+      f32_begin_item<D, GMAX>(st, rows, g, it.len, it.q_len);
     }
     // bf16 consumes this warp's blocks two at a time (b and b + W), fp32 one at a time.
     constexpr int kStep = kBf16 ? 2 : 1;
@@ -795,12 +850,13 @@ __global__ void __launch_bounds__((W + 1) * 32)
         }
       }
       if (!ok) break;
+      const int pos0 = (it.blk_begin + b) * kBlock;  // position of the first tile's token 0
       if constexpr (kBf16) {
-        bf16_step<D, GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], kt[1],
-                           kt[1] + Lay::kTileBytes, valid[1], sc, lane);
+        bf16_step<D, GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
+                           kt[1] + Lay::kTileBytes, valid[1], pos0 + W * kBlock, sc, lane);
       } else {
         f32_block<D, GMAX>(st, reinterpret_cast<const float*>(qs), kt[0], kt[0] + Lay::kTileBytes,
-                           valid[0], sc, g, lane);
+                           valid[0], pos0, sc, rows, lane);
       }
       __syncwarp();
       cctr += n;
@@ -812,20 +868,31 @@ __global__ void __launch_bounds__((W + 1) * 32)
     if (lane == 0) mbar_arrive(&item_empty[r]);
     produce(false);
     // ---- merge the W warps' states ----
-    const int mb = c_item & 1;
-    float* mslot = merge + (mb * W + warp) * per_warp;
-    if constexpr (kBf16) {
-      bf16_publish<D, GMAX>(st, mslot, g, lane);
-    } else {
-      f32_publish<D, GMAX>(st, mslot, g, lane);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&merge_bar[mb]);
-    if (!mbar_wait(&merge_bar[mb], (c_item >> 1) & 1)) {
+    // two buffers: item c uses buffer c & 1 and merge_bar[c & 1];
+    // one buffer: merge_bar[0] = states published, merge_bar[1] = combined.
+    const int mb = MB == 2 ? (c_item & 1) : 0;
+    const uint32_t pub_parity = MB == 2 ? ((c_item >> 1) & 1) : (c_item & 1);
+    if (MB == 1 && c_item > 0 && !mbar_wait(&merge_bar[1], (c_item - 1) & 1)) {
       ok = false;
       break;
     }
-    combine_and_store<T, D, W>(prm, it, merge + mb * W * per_warp, per_warp, g, warp, lane);
+    float* mslot = merge + (mb * W + warp) * per_warp;
+    if constexpr (kBf16) {
+      bf16_publish<D, GMAX>(st, mslot, rows, lane);
+    } else {
+      f32_publish<D, GMAX>(st, mslot, rows, lane);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&merge_bar[mb]);
+    if (!mbar_wait(&merge_bar[mb], pub_parity)) {
+      ok = false;
+      break;
+    }
+    combine_and_store<T, D, W>(prm, it, merge + mb * W * per_warp, per_warp, rows, warp, lane);
+    if constexpr (MB == 1) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&merge_bar[1]);
+    }
   }
   if (!ok) {
     // A wait gave up: raise the abort flag and wait (bounded) for the copies
@@ -838,20 +905,32 @@ __global__ void __launch_bounds__((W + 1) * 32)
 }
 
 // ------------------------------------------------------------- merge kernel
-// One warp per (sequence, query head) row whose sequence was split: combine
-// the partitions' (m, l, o) by log-sum-exp and store the final output.
+// One warp per (query token, query head) row whose sequence was split:
+// combine the partitions' (m, l, o) by log-sum-exp and store the final
+// output.  Partitions a causal row cannot see carry l = 0 and no weight.
 template <typename T, int D>
 __global__ void __launch_bounds__(128)
     merge_kernel(void* __restrict__ out, const float* __restrict__ part_o,
                  const float* __restrict__ part_ml, const int32_t* __restrict__ context_lens,
-                 int32_t num_seqs, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
+                 const int32_t* __restrict__ query_start_loc, int32_t num_seqs,
+                 int32_t num_q_tokens, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
                  int32_t part_tokens) {
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
-  if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
-  const int32_t s = static_cast<int32_t>(row / num_q_heads);
+  if (row >= static_cast<int64_t>(num_q_tokens) * num_q_heads) return;
+  const int32_t t = static_cast<int32_t>(row / num_q_heads);  // query token
+  int32_t s = t;                                                // its sequence
+  if (query_start_loc) {  // the last sequence whose chunk starts at or before t
+    int32_t lo = 0, hi = num_seqs - 1;
+    while (lo < hi) {
+      const int32_t mid = (lo + hi + 1) / 2;
+      if (query_start_loc[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+    if (t >= query_start_loc[num_seqs]) return;  // rows past the last chunk
+  }
   int32_t L = context_lens[s];
   L = L < 0 ? 0 : (L > max_len ? max_len : L);
   const int32_t n = num_parts(L, part_tokens);

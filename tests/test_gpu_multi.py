@@ -1,0 +1,123 @@
+"""GPU parity of several causal query tokens per sequence (through the C ABI)
+against the float64 oracle: chunks of new tokens written by reshape_and_cache,
+each with its query row attending to the context up to its own position."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_375_b200 as pkv
+import workloads
+from gpu_util import check_close, compact_for_tasks, dev_i32, host_bits, oracle_caches_after_step
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_multi(b, partition_tokens=0, max_query_len=None):
+    dev = b.q.device
+    bt = dev_i32(b.block_tables, dev)
+    cl = dev_i32(b.context_lens, dev)
+    qsl = dev_i32(b.query_start_loc, dev)
+    if b.new_seq.shape[0]:
+        slots = pkv.slot_mapping(bt, b.num_blocks, token_seq=dev_i32(b.new_seq, dev),
+                                 token_pos=dev_i32(b.new_pos, dev))
+        pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, slots)
+    out = torch.empty_like(b.q)
+    pkv.paged_attention_multi(out, b.q, b.k_cache, b.v_cache, bt, cl, qsl, b.scale,
+                              b.num_kv_heads, max_query_len or b.max_query_len,
+                              max_context_len=max(b.max_context_len, 1),
+                              partition_tokens=partition_tokens)
+    return out
+
+
+def run_and_check(b, partition_tokens=0, what=""):
+    host = b.host()
+    out = gpu_multi(b, partition_tokens)
+    assert pkv.device_error_bits() == 0
+    k, v = oracle_caches_after_step(b, host)
+    ref = oracle.paged_multi(host["q"], k, v, b.block_tables, b.context_lens,
+                             b.query_start_loc, b.scale)
+    check_close(out, ref, b.dtype, what)
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 4), (8, 8, 16), (16, 2, 2), (6, 2, 5),
+                                             (8, 4, 8)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_random_chunks(cuda_device, dtype, hq, hkv, max_chunk, d):
+    rng = np.random.default_rng(hq * 100 + hkv * 10 + max_chunk + d)
+    lens = np.array([1, 2, 15, 16, 17, 33, 64, 100, 257, 300, 31, 48])
+    chunks = np.minimum(rng.integers(1, max_chunk + 1, size=lens.shape[0]), lens)
+    b = workloads.chunked_batch(500 + d, lens, chunks, hq, hkv, d, dtype, device=cuda_device,
+                                extra_table=2)
+    run_and_check(b, what=f"{dtype} {hq}/{hkv} chunks<={max_chunk} d{d}")
+
+
+@pytest.mark.parametrize("partition", [16, 64, 256])
+def test_chunks_with_split_k(cuda_device, partition):
+    lens = np.array([40, 300, 1000, 2100, 5])
+    chunks = np.array([4, 3, 4, 1, 2])
+    b = workloads.chunked_batch(600 + partition, lens, chunks, 32, 8, 128, "bf16",
+                                device=cuda_device)
+    run_and_check(b, partition, f"split {partition}")
+
+
+def test_one_token_chunks_equal_decode_bitwise(cuda_device):
+    lens = np.array([3, 16, 17, 600, 1500])
+    b = workloads.chunked_batch(700, lens, np.ones(5, dtype=np.int64), 32, 8, 128, "bf16",
+                                device=cuda_device)
+    multi = gpu_multi(b)
+    out = torch.empty_like(b.q)
+    pkv.paged_attention_decode(out, b.q, b.k_cache, b.v_cache,
+                               dev_i32(b.block_tables, cuda_device),
+                               dev_i32(b.context_lens, cuda_device), b.scale, b.num_kv_heads,
+                               max_context_len=b.max_context_len)
+    assert torch.equal(multi.view(torch.int16), out.view(torch.int16))
+
+
+def test_empty_chunks_and_zero_length_sequences(cuda_device):
+    lens = np.array([0, 20, 7, 0, 33])
+    chunks = np.array([0, 3, 0, 0, 2])
+    b = workloads.chunked_batch(701, lens, chunks, 8, 2, 64, "bf16", device=cuda_device)
+    run_and_check(b, what="empty chunks")
+
+
+def test_chunk_longer_than_its_context_is_flagged(cuda_device):
+    lens = np.array([10, 40])
+    b = workloads.chunked_batch(702, lens, np.array([2, 3]), 8, 8, 64, "bf16", device=cuda_device)
+    b.query_start_loc = np.array([0, 2, 5], dtype=np.int32)
+    gpu_multi(b, max_query_len=2)     # the second chunk (3 tokens) exceeds max_query_len
+    assert pkv.device_error_bits() & pkv.DEVERR_LEN
+
+
+def test_spec_decode_workload_sampled(cuda_device):
+    """The full Llama-3-8B-shaped batch verifying 4 draft tokens per sequence; sampled
+    query rows recomputed by the oracle."""
+    b = workloads.c3_spec_decode(device=cuda_device)
+    out = gpu_multi(b)
+    assert pkv.device_error_bits() == 0
+    assert torch.isfinite(out).all()
+    rng = np.random.default_rng(5)
+    seqs = np.unique(np.concatenate([[int(np.argmax(b.context_lens))],
+                                     rng.integers(0, b.num_seqs, 6)]))
+    # the oracle on the sampled sequences only, over their compacted blocks
+    tasks = np.array([(s, 0) for s in seqs], dtype=np.int32)
+    kh, vh, bt = compact_for_tasks(b, b.k_cache, b.v_cache, tasks)
+    sub_bt = bt[seqs]
+    sub_cl = b.context_lens[seqs]
+    qsl = b.query_start_loc
+    rows = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in seqs])
+    sub_qsl = np.concatenate([[0], np.cumsum(qsl[seqs + 1] - qsl[seqs])]).astype(np.int32)
+    q_rows = host_bits(b.q)[rows]
+    ref = oracle.paged_multi(np.ascontiguousarray(q_rows), kh, vh, sub_bt, sub_cl, sub_qsl,
+                             b.scale, threads=4)
+    check_close(out[torch.from_numpy(rows).long()], ref, "bf16", "spec decode")
+
+
+def test_chunk_outside_the_query_rows_is_skipped_and_flagged(cuda_device):
+    lens = np.array([10, 40])
+    b = workloads.chunked_batch(703, lens, np.array([2, 3]), 8, 8, 64, "bf16", device=cuda_device)
+    b.query_start_loc = np.array([0, 2, 9], dtype=np.int32)   # rows 2..8 but q has 5 rows
+    gpu_multi(b, max_query_len=16)
+    assert pkv.device_error_bits() & pkv.DEVERR_LEN

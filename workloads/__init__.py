@@ -113,6 +113,8 @@ class Batch:
     new_pos: np.ndarray             # int32 [T] position of each new token
     cow_pairs: np.ndarray           # int64 [P][2] (src, dst), applied before the writes
     meta: dict = field(default_factory=dict)
+    # several query tokens per sequence: rows query_start_loc[s] .. [s+1]-1 of q
+    query_start_loc: np.ndarray | None = None
 
     @property
     def num_seqs(self) -> int:
@@ -125,6 +127,12 @@ class Batch:
     @property
     def max_blocks_per_seq(self) -> int:
         return int(self.block_tables.shape[1])
+
+    @property
+    def max_query_len(self) -> int:
+        if self.query_start_loc is None:
+            return 1
+        return int(np.diff(self.query_start_loc).max()) if self.num_seqs else 1
 
     @property
     def max_context_len(self) -> int:
@@ -151,8 +159,8 @@ class Batch:
 
     def io_bytes(self) -> int:
         """q + out + block-table + context-length bytes of one decode step."""
-        B, Hq, D = self.num_seqs, self.num_q_heads, self.head_dim
-        return 2 * B * Hq * D * self.elem_bytes + self.block_tables.nbytes + self.context_lens.nbytes
+        T, Hq, D = self.q.shape[0], self.num_q_heads, self.head_dim
+        return 2 * T * Hq * D * self.elem_bytes + self.block_tables.nbytes + self.context_lens.nbytes
 
     def host(self) -> dict:
         """Host numpy copies: float32 arrays, or uint16 arrays holding bf16 bits."""
@@ -170,7 +178,8 @@ class Batch:
                      self.block_tables.copy(), self.scale, self.q.to(device),
                      self.k_cache.to(device), self.v_cache.to(device), self.new_k.to(device),
                      self.new_v.to(device), self.new_seq.copy(), self.new_pos.copy(),
-                     self.cow_pairs.copy(), dict(self.meta))
+                     self.cow_pairs.copy(), dict(self.meta),
+                     None if self.query_start_loc is None else self.query_start_loc.copy())
 
 
 def torch_dtype(dtype: str) -> torch.dtype:
@@ -319,6 +328,53 @@ def c3_llama3_8b_gqa(device="cpu", num_seqs: int = 256) -> Batch:
     return b
 
 
+def chunked_batch(seed: int, lens, chunks, hq: int, hkv: int, d: int, dtype: str = "bf16",
+                  num_blocks: int | None = None, device="cpu", name: str = "chunked",
+                  extra_table: int = 0) -> Batch:
+    """Each sequence ends with a chunk of new tokens (chunks[s] of them, its last
+    positions): their K/V are the new tokens to write before attention and each gets a
+    query row; query_start_loc separates the chunks."""
+    lens = np.asarray(lens, dtype=np.int64)
+    chunks = np.asarray(chunks, dtype=np.int64)
+    assert (chunks <= lens).all()
+    rng = np.random.default_rng(seed)
+    need = int(sum((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE for L in lens))
+    nb = num_blocks if num_blocks is not None else max(need + 8, 16)
+    bm = BlockManager(nb, rng)
+    tables = [bm.allocate((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE) for L in lens]
+    new_seq = np.concatenate([np.full(int(c), s) for s, c in enumerate(chunks)] + [np.zeros(0)])
+    new_pos = np.concatenate([np.arange(int(L - c), int(L)) for L, c in zip(lens, chunks)]
+                             + [np.zeros(0)])
+    b = _assemble(name, seed, dtype, hq, hkv, d, nb, lens, tables, tables, lens - chunks,
+                  new_seq.astype(np.int64), new_pos.astype(np.int64), [], device,
+                  {"blocks_in_use": bm.blocks_in_use()})
+    T = int(chunks.sum())
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 7919)
+    b.q = _randn((T, hq, d), gen, device, dtype)
+    b.query_start_loc = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    width = max(b.block_tables.shape[1], 1) + extra_table
+    if b.block_tables.shape[1] < width:
+        bt = np.full((b.num_seqs, width), -1, dtype=np.int32)
+        bt[:, :b.block_tables.shape[1]] = b.block_tables
+        b.block_tables = bt
+    return b
+
+
+def c3_spec_decode(device="cpu", num_seqs: int = 256, draft: int = 4) -> Batch:
+    """The Llama-3-8B-shaped GQA batch verifying `draft` speculative tokens per sequence:
+    the draft tokens are the last positions of each context (lognormal lengths as in the
+    decode batch, at least `draft`), written by reshape_and_cache, each with its query
+    row, attending causally."""
+    lens = np.maximum(c3_lens(num_seqs), draft)
+    need = int(sum((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE for L in lens))
+    b = chunked_batch(CONFIG_SEEDS["c3_llama3_8b_gqa"] + 100, lens, np.full(num_seqs, draft),
+                      32, 8, 128, "bf16", num_blocks=max(32768, int(math.ceil(1.25 * need))),
+                      device=device, name="c3_spec_decode")
+    b.meta["draft_tokens"] = draft
+    return b
+
+
 def c4_shared_prefix(device="cpu", prompts: int = 32, samples: int = 8, prefix: int = 1024,
                      max_tail: int = 512, num_blocks: int | None = None) -> Batch:
     """Parallel sampling with a shared prefix.
@@ -380,8 +436,12 @@ def c5_long_splitk(device="cpu", num_seqs: int = 8) -> Batch:
                         name="c5_long_splitk")
 
 
+CONFIGS["c3_spec_decode"] = ("Llama-3-8B-shaped GQA bf16, batch 256, verifying 4 speculative tokens "
+                              "per sequence (causal, 16 query rows per kv head)")
+
 BUILDERS = {
     "c1_tiny_fp32": c1_tiny_fp32,
+    "c3_spec_decode": c3_spec_decode,
     "c2_llama2_13b_mha": c2_llama2_13b_mha,
     "c3_llama3_8b_gqa": c3_llama3_8b_gqa,
     "c4_shared_prefix": c4_shared_prefix,
