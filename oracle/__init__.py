@@ -28,6 +28,7 @@ _lib = None
 
 F32 = 0
 BF16 = 1
+E4M3 = 2
 
 _STATUS = {
     0: "ok",
@@ -81,9 +82,17 @@ def _load():
             lib.oracle_lse_merge.argtypes = [P, P, P, i32, i32, P]
             lib.oracle_paged_multi.argtypes = [P, P, P, P, i32, P, P, P, i32, i32, i32, i32,
                                                i32, i64, i32, f32, i32]
+            lib.oracle_paged_decode_fp8.argtypes = [P, P, P, P, f32, f32, P, P, i32, i32, i32,
+                                                    i32, i32, i64, i32, f32, P, i64, i32]
+            lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i64,
+                                                         f32, f32]
+            lib.oracle_e4m3_quantize.argtypes = [P, i64, f32, P]
+            lib.oracle_e4m3_values.argtypes = [P, i64, P]
             lib.oracle_lse_merge_f32.argtypes = [P, P, P, i32, i32, P]
             for name in ("oracle_slot_mapping", "oracle_reshape_and_cache",
                          "oracle_copy_blocks", "oracle_paged_decode", "oracle_paged_multi",
+                         "oracle_paged_decode_fp8", "oracle_reshape_and_cache_fp8",
+                         "oracle_e4m3_quantize", "oracle_e4m3_values",
                          "oracle_partition_stats", "oracle_lse_merge",
                          "oracle_lse_merge_f32"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -190,6 +199,59 @@ def paged_multi(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
     _check(_load().oracle_paged_multi(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), code,
                                       _ptr(bt), _ptr(cl), _ptr(qsl), cl.shape[0], Hq, Hkv, D, BS,
                                       NB, bt.shape[1], float(scale), threads))
+    return out
+
+
+def e4m3_quantize(x: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """uint8 e4m3 codes of float32 x / scale (the division in float32)."""
+    xf = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(xf.shape, dtype=np.uint8)
+    _check(_load().oracle_e4m3_quantize(_ptr(xf), xf.size, float(scale), _ptr(out)))
+    return out
+
+
+def e4m3_values(codes: np.ndarray) -> np.ndarray:
+    """Exact values of e4m3 codes (no scale), as float64."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _check(_load().oracle_e4m3_values(_ptr(c), c.size, _ptr(out)))
+    return out
+
+
+def reshape_and_cache_fp8(k: np.ndarray, v: np.ndarray, k_cache: np.ndarray,
+                          v_cache: np.ndarray, slot_mapping_: np.ndarray, k_scale: float,
+                          v_scale: float) -> None:
+    """In place on uint8 e4m3 pools [NB][Hkv][BS][D]; k, v are bf16 bits [T][Hkv][D]."""
+    sm = np.ascontiguousarray(slot_mapping_, dtype=np.int64)
+    nb, hkv, bs, d = k_cache.shape
+    assert k.dtype == np.uint16 and k_cache.dtype == np.uint8 and k.shape[1:] == (hkv, d)
+    _check(_load().oracle_reshape_and_cache_fp8(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
+                                                _ptr(sm), sm.shape[0], hkv, d, bs, nb,
+                                                float(k_scale), float(v_scale)))
+
+
+def paged_decode_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_scale: float,
+                     v_scale: float, block_tables: np.ndarray, context_lens: np.ndarray,
+                     scale: float, tasks: np.ndarray | None = None,
+                     threads: int | None = None) -> np.ndarray:
+    """Float64 decode over e4m3 pools (uint8 codes times the pool's scale); q is bf16 bits."""
+    assert q.dtype == np.uint16 and k_cache.dtype == np.uint8 == v_cache.dtype
+    B, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_cache.shape
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    threads = threads or len(os.sched_getaffinity(0))
+    if tasks is None:
+        out = np.empty((B, Hq, D), dtype=np.float64)
+        tp, n = None, B * Hq
+    else:
+        tk = np.ascontiguousarray(tasks, dtype=np.int32).reshape(-1, 2)
+        out = np.empty((tk.shape[0], D), dtype=np.float64)
+        tp, n = _ptr(tk), tk.shape[0]
+    _check(_load().oracle_paged_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                           float(k_scale), float(v_scale), _ptr(bt), _ptr(cl),
+                                           B, Hq, Hkv, D, BS, NB, bt.shape[1], float(scale), tp,
+                                           n, threads))
     return out
 
 

@@ -58,15 +58,98 @@ enum {
     ORACLE_NO_MEMORY = 6
 };
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
+
+/* ------------------------------------------------------------------------- */
+/* FP8 E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; exponent 15 with mantissa 7 is NaN, so the largest finite value
+ * is 1.75 * 2^8 = 448; exponent 0 holds the subnormals m * 2^-9).  A KV cache
+ * in this format stores code = e4m3(x / scale) with one scale per pool; the
+ * reading of "quantise" used here: divide in single precision, round to the
+ * nearest representable value with ties to even, saturate to +-448 instead of
+ * overflowing, keep NaN. */
+static double e4m3_value(uint8_t code)
+{
+    const int sign = code >> 7, exp = (code >> 3) & 15, man = code & 7;
+    double v;
+    if (exp == 15 && man == 7) {
+        return NAN;
+    }
+    if (exp == 0) {
+        v = ldexp((double)man, -9);
+    } else {
+        v = ldexp(1.0 + man / 8.0, exp - 7);
+    }
+    return sign ? -v : v;
+}
+
+static uint8_t e4m3_encode(float y)
+{
+    if (isnan(y)) {
+        return 0x7f;
+    }
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a >= 448.0) {
+        return sign | 0x7e;                       /* saturate */
+    }
+    int e;
+    frexp(a, &e);                                 /* a = f * 2^e, 0.5 <= f < 1 */
+    int unbiased = e - 1;                         /* a in [2^unbiased, 2^(unbiased+1)) */
+    if (a == 0.0 || unbiased < -6) {
+        unbiased = -6;                            /* subnormal range: steps of 2^-9 */
+    }
+    /* number of 2^(unbiased-3) steps, rounded to nearest, ties to even (rint
+     * under the default rounding mode) */
+    double steps = rint(ldexp(a, 3 - unbiased));
+    if (steps >= 16.0) {                          /* rounded up into the next binade */
+        unbiased += 1;
+        steps = 8.0;
+    }
+    if (unbiased > 8 || (unbiased == 8 && steps > 14.0)) {
+        return sign | 0x7e;                       /* beyond 448 after rounding */
+    }
+    if (steps < 8.0) {                            /* subnormal */
+        return sign | (uint8_t)steps;
+    }
+    return sign | (uint8_t)(((unbiased + 7) << 3) | ((int)steps - 8));
+}
+
+/* Encode n floats: out[i] = e4m3(x[i] / scale), the division in float. */
+int oracle_e4m3_quantize(const float *x, int64_t n, float scale, uint8_t *out)
+{
+    if ((!x || !out) && n > 0) {
+        return 1;
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        out[i] = e4m3_encode(x[i] / scale);
+    }
+    return 0;
+}
+
+/* Decode n codes to doubles (the exact values, without any scale). */
+int oracle_e4m3_values(const uint8_t *codes, int64_t n, double *out)
+{
+    if ((!codes || !out) && n > 0) {
+        return 1;
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        out[i] = e4m3_value(codes[i]);
+    }
+    return 0;
+}
 
 /* Widen one stored element to double.  bf16 is the upper half of an IEEE
  * binary32, so shifting its 16 bits up gives the exact float, and float to
- * double is exact. */
+ * double is exact.  An e4m3 code widens to its exact value (the pool's scale
+ * is applied by the caller). */
 static double widen(const void *base, int64_t index, int dtype)
 {
     if (dtype == ORACLE_F32) {
         return (double)((const float *)base)[index];
+    }
+    if (dtype == ORACLE_E4M3) {
+        return e4m3_value(((const uint8_t *)base)[index]);
     }
     uint32_t bits = (uint32_t)((const uint16_t *)base)[index] << 16;
     float f;
@@ -139,6 +222,43 @@ int oracle_reshape_and_cache(const void *k, const void *v, void *k_cache,
     return status;
 }
 
+/* reshape_and_cache into FP8 (e4m3) pools: token t's bf16 K and V values are
+ * quantised (code = e4m3(value / scale), the division in float) and written
+ * at slot_mapping[t]. */
+int oracle_reshape_and_cache_fp8(const uint16_t *k, const uint16_t *v, uint8_t *k_cache,
+                                 uint8_t *v_cache, const int64_t *slot_mapping,
+                                 int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int64_t num_blocks, float k_scale,
+                                 float v_scale)
+{
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping || num_tokens < 0 ||
+        num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0) {
+        return ORACLE_BAD_ARG;
+    }
+    int status = ORACLE_OK;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) {
+            continue;
+        }
+        if (slot >= num_blocks * block_size) {
+            status = ORACLE_BAD_SLOT;
+            continue;
+        }
+        int64_t block = slot / block_size, offset = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            for (int32_t d = 0; d < head_dim; ++d) {
+                size_t src = ((size_t)t * num_kv_heads + h) * head_dim + d;
+                size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) *
+                                 head_dim + d;
+                k_cache[dst] = e4m3_encode((float)widen(k, (int64_t)src, ORACLE_BF16) / k_scale);
+                v_cache[dst] = e4m3_encode((float)widen(v, (int64_t)src, ORACLE_BF16) / v_scale);
+            }
+        }
+    }
+    return status;
+}
+
 /* ------------------------------------------------------------------------- */
 /* copy_blocks: for each pair (src, dst) the whole K block and the whole V block
  * of src (all kv heads, all slots) are copied to dst.  Sources are taken from a
@@ -196,7 +316,14 @@ typedef struct {
     int64_t num_blocks;
     int32_t max_blocks_per_seq;
     double scale;
+    /* FP8 caches: q is bf16, each cache element is code * its pool's scale */
+    double k_scale, v_scale;
 } problem;
+
+static int q_dtype(const problem *pb)
+{
+    return pb->dtype == ORACLE_E4M3 ? ORACLE_BF16 : pb->dtype;
+}
 
 /* Gather the contiguous K and V rows [0, len) of (seq, kv_head) by walking the
  * block table one logical block at a time.  Returns ORACLE_BAD_BLOCK if an
@@ -216,8 +343,8 @@ static int gather_context(const problem *pb, int32_t seq, int32_t kv_head,
         int64_t row =
             ((physical_block * pb->num_kv_heads + kv_head) * pb->block_size + offset) * D;
         for (int32_t d = 0; d < D; ++d) {
-            K[(int64_t)j * D + d] = widen(pb->k_cache, row + d, pb->dtype);
-            V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype);
+            K[(int64_t)j * D + d] = widen(pb->k_cache, row + d, pb->dtype) * pb->k_scale;
+            V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype) * pb->v_scale;
         }
     }
     return ORACLE_OK;
@@ -299,7 +426,7 @@ static int decode_one(const problem *pb, int32_t seq, int32_t q_head, double *ou
         return ORACLE_NO_MEMORY;
     }
     for (int32_t d = 0; d < D; ++d) {
-        qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + q_head) * D + d, pb->dtype);
+        qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + q_head) * D + d, q_dtype(pb));
     }
     st = gather_context(pb, seq, kv_head, L, K, V);
     if (st == ORACLE_OK) {
@@ -348,6 +475,14 @@ static void *decode_worker(void *arg)
     return NULL;
 }
 
+static int paged_decode_scaled(double *out, const void *q, const void *k_cache,
+                               const void *v_cache, int32_t dtype, float k_scale, float v_scale,
+                               const int32_t *block_tables, const int32_t *context_lens,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                               int32_t max_blocks_per_seq, float scale,
+                               const int32_t *tasks, int64_t num_tasks, int32_t num_threads);
+
 /*
  * out: [num_tasks][head_dim] doubles.  With tasks == NULL every (seq, q_head)
  * is computed in row-major order (num_tasks must then be num_seqs*num_q_heads),
@@ -361,11 +496,41 @@ int oracle_paged_decode(double *out, const void *q, const void *k_cache,
                         int32_t max_blocks_per_seq, float scale,
                         const int32_t *tasks, int64_t num_tasks, int32_t num_threads)
 {
+    return paged_decode_scaled(out, q, k_cache, v_cache, dtype, 1.0f, 1.0f, block_tables,
+                               context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                               block_size, num_blocks, max_blocks_per_seq, scale, tasks,
+                               num_tasks, num_threads);
+}
+
+/* The same for an FP8 (e4m3) cache: q is bf16; each cached element is its
+ * code's value times k_scale (K pool) or v_scale (V pool). */
+int oracle_paged_decode_fp8(double *out, const void *q, const void *k_cache,
+                            const void *v_cache, float k_scale, float v_scale,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                            int32_t max_blocks_per_seq, float scale,
+                            const int32_t *tasks, int64_t num_tasks, int32_t num_threads)
+{
+    return paged_decode_scaled(out, q, k_cache, v_cache, ORACLE_E4M3, k_scale, v_scale,
+                               block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
+                               tasks, num_tasks, num_threads);
+}
+
+static int paged_decode_scaled(double *out, const void *q, const void *k_cache,
+                               const void *v_cache, int32_t dtype, float k_scale, float v_scale,
+                               const int32_t *block_tables, const int32_t *context_lens,
+                               int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                               int32_t max_blocks_per_seq, float scale,
+                               const int32_t *tasks, int64_t num_tasks, int32_t num_threads)
+{
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
-        (dtype != ORACLE_F32 && dtype != ORACLE_BF16) || num_seqs < 0 ||
-        num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
-        head_dim <= 0 || block_size <= 0 || num_blocks <= 0 ||
-        max_blocks_per_seq <= 0 || num_tasks < 0) {
+        (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && dtype != ORACLE_E4M3) ||
+        num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || num_tasks < 0) {
         return ORACLE_BAD_ARG;
     }
     if (!tasks && num_tasks != (int64_t)num_seqs * num_q_heads) {
@@ -381,7 +546,8 @@ int oracle_paged_decode(double *out, const void *q, const void *k_cache,
     }
     problem pb = {q, k_cache, v_cache, dtype, block_tables, context_lens,
                   num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                  num_blocks, max_blocks_per_seq, (double)scale};
+                  num_blocks, max_blocks_per_seq, (double)scale, (double)k_scale,
+                  (double)v_scale};
     task_pool tp = {&pb, out, tasks, num_tasks, 0, ORACLE_OK};
     if (num_threads <= 1) {
         decode_worker(&tp);
@@ -462,7 +628,7 @@ static void *multi_worker(void *arg)
                     const int32_t h = kv_head * group + hg;
                     const int64_t row = (int64_t)(q0 + i) * pb->num_q_heads + h;
                     for (int32_t d = 0; d < D; ++d) {
-                        qrow[d] = widen(pb->q, row * D + d, pb->dtype);
+                        qrow[d] = widen(pb->q, row * D + d, q_dtype(pb));
                     }
                     double m, l;
                     attend_range(qrow, K, V, D, pb->scale, 0, visible, &m, &l, mp->out + row * D);
@@ -501,7 +667,7 @@ int oracle_paged_multi(double *out, const void *q, const void *k_cache, const vo
     }
     problem pb = {q, k_cache, v_cache, dtype, block_tables, context_lens,
                   num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                  num_blocks, max_blocks_per_seq, (double)scale};
+                  num_blocks, max_blocks_per_seq, (double)scale, 1.0, 1.0};
     multi_pool mp = {&pb, query_start_loc, out, 0, ORACLE_OK};
     if (num_threads <= 1) {
         multi_worker(&mp);
@@ -555,7 +721,7 @@ int oracle_partition_stats(const void *q, const void *k_cache, const void *v_cac
     }
     problem pb = {q, k_cache, v_cache, dtype, block_tables, context_lens,
                   num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                  num_blocks, max_blocks_per_seq, (double)scale};
+                  num_blocks, max_blocks_per_seq, (double)scale, 1.0, 1.0};
     int32_t L;
     int st = checked_len(&pb, seq, &L);
     if (st != ORACLE_OK) {
@@ -576,7 +742,8 @@ int oracle_partition_stats(const void *q, const void *k_cache, const void *v_cac
     }
     const int32_t kv_head = q_head / (num_q_heads / num_kv_heads);
     for (int32_t d = 0; d < D; ++d) {
-        qrow[d] = widen(q, ((int64_t)seq * num_q_heads + q_head) * D + d, dtype);
+        qrow[d] = widen(q, ((int64_t)seq * num_q_heads + q_head) * D + d,
+                        dtype == ORACLE_E4M3 ? ORACLE_BF16 : dtype);
     }
     st = gather_context(&pb, seq, kv_head, L, K, V);
     if (st == ORACLE_OK) {

@@ -40,8 +40,16 @@ MUTANTS = {
                          "const int32_t visible = L;"),
     "multi_causal_off_by_one": ("const int32_t visible = L - n + i + 1;      /* keys 0 .. L-n+i */",
                                 "const int32_t visible = L - n + i;"),
-    "q_row_of_wrong_head": ("qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + q_head) * D + d, pb->dtype);",
-                            "qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + kv_head) * D + d, pb->dtype);"),
+    "q_row_of_wrong_head": ("qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + q_head) * D + d, q_dtype(pb));",
+                            "qrow[d] = widen(pb->q, ((int64_t)seq * pb->num_q_heads + kv_head) * D + d, q_dtype(pb));"),
+    "e4m3_ties_away": ("double steps = rint(ldexp(a, 3 - unbiased));",
+                       "double steps = floor(ldexp(a, 3 - unbiased) + 0.5);"),
+    "e4m3_bias_off_by_one": ("return sign | (uint8_t)(((unbiased + 7) << 3) | ((int)steps - 8));",
+                             "return sign | (uint8_t)(((unbiased + 8) << 3) | ((int)steps - 8));"),
+    "e4m3_no_saturation": ("        return sign | 0x7e;                       /* saturate */",
+                           "        return sign | 0x7f;                       /* saturate */"),
+    "fp8_scale_dropped": ("V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype) * pb->v_scale;",
+                          "V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype);"),
 }
 
 

@@ -503,3 +503,78 @@ def test_multi_rejects_chunks_longer_than_the_context():
     q, kp, vp, bt, cl, _, _, qsl = _multi_case(rng, [4], [5], 1, 1, 8)
     with pytest.raises(oracle.OracleError):
         oracle.paged_multi(q, kp, vp, bt, cl, qsl, 1.0)
+
+
+# ------------------------------------------------------------- FP8 (e4m3) ----
+def test_golden_e4m3_examples():
+    g = _golden("e4m3_examples.json")
+    codes = oracle.e4m3_quantize(np.array(g["values"], dtype=np.float32))
+    assert codes.tolist() == g["codes"]
+
+
+def test_e4m3_every_finite_code_round_trips():
+    codes = np.array([c for c in range(256) if c & 0x7f != 0x7f], dtype=np.uint8)
+    vals = oracle.e4m3_values(codes)
+    assert np.isfinite(vals).all() and np.abs(vals).max() == 448.0
+    assert np.array_equal(oracle.e4m3_quantize(vals.astype(np.float32)), codes)
+    assert np.isnan(oracle.e4m3_values(np.array([0x7f, 0xff], dtype=np.uint8))).all()
+
+
+def test_e4m3_rounds_to_the_nearest_value_ties_to_even():
+    rng = np.random.default_rng(30)
+    x = np.concatenate([rng.standard_normal(4000) * 10.0 ** rng.uniform(-4, 2.5, 4000),
+                        rng.uniform(-500, 500, 200)]).astype(np.float32)
+    codes = oracle.e4m3_quantize(x)
+    grid_codes = np.array([c for c in range(256) if c & 0x7f != 0x7f], dtype=np.uint8)
+    grid = oracle.e4m3_values(grid_codes)
+    for xi, ci in zip(x.astype(np.float64), codes):
+        if abs(xi) >= 448.0:
+            assert oracle.e4m3_values(np.array([ci]))[0] == np.copysign(448.0, xi)
+            continue
+        d = np.abs(grid - xi)
+        best = grid_codes[d == d.min()]
+        if len(best) > 1:                                   # a tie: the even mantissa wins
+            best = [c for c in best if (c & 1) == 0 and (c & 0x80) == (ci & 0x80)] or best
+        assert ci in best, (xi, ci, best)
+
+
+def test_e4m3_divides_by_the_scale_in_float():
+    x = np.array([1.0, 3.0, -7.5], dtype=np.float32)
+    assert np.array_equal(oracle.e4m3_quantize(x, 0.5), oracle.e4m3_quantize(x / np.float32(0.5)))
+
+
+def test_fp8_decode_matches_dense_attention_on_dequantised_values():
+    rng = np.random.default_rng(31)
+    lens = [1, 16, 33, 70]
+    hq, hkv, d = 8, 2, 64
+    q32, kp32, vp32, bt, cl, Ks, Vs, _ = random_paged(rng, lens, hq, hkv, d)
+    k_scale, v_scale = np.float32(0.05), np.float32(0.02)
+    kc = oracle.e4m3_quantize(np.nan_to_num(kp32), k_scale)
+    vc = oracle.e4m3_quantize(np.nan_to_num(vp32), v_scale)
+    qb = to_bf16_bits(q32)
+    out = oracle.paged_decode_fp8(qb, kc, vc, k_scale, v_scale, bt, cl, 0.125)
+    qf = bf16_bits_to_f64(qb)
+    kd = oracle.e4m3_values(kc) * float(k_scale)
+    vd = oracle.e4m3_values(vc) * float(v_scale)
+    for s, L in enumerate(lens):
+        n = (L + BS - 1) // BS
+        K = kd[bt[s, :n]].transpose(0, 2, 1, 3).reshape(n * BS, hkv, d)[:L]
+        V = vd[bt[s, :n]].transpose(0, 2, 1, 3).reshape(n * BS, hkv, d)[:L]
+        np.testing.assert_allclose(out[s], dense_attention(qf[s], K, V, 0.125), rtol=0,
+                                   atol=1e-12)
+
+
+def test_fp8_reshape_quantises_into_the_slot():
+    rng = np.random.default_rng(32)
+    hkv, d, nb = 2, 64, 4
+    k = to_bf16_bits(rng.standard_normal((3, hkv, d)).astype(np.float32))
+    v = to_bf16_bits(rng.standard_normal((3, hkv, d)).astype(np.float32))
+    kc = np.zeros((nb, hkv, BS, d), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    slots = np.array([5, -1, 50])
+    oracle.reshape_and_cache_fp8(k, v, kc, vc, slots, 0.1, 0.3)
+    kf = bf16_bits_to_f64(k).astype(np.float32)
+    vf = bf16_bits_to_f64(v).astype(np.float32)
+    assert np.array_equal(kc[0, :, 5], oracle.e4m3_quantize(kf[0], 0.1))
+    assert np.array_equal(vc[3, :, 2], oracle.e4m3_quantize(vf[2], 0.3))
+    assert kc.astype(np.int64).sum() == oracle.e4m3_quantize(kf[[0, 2]], 0.1).astype(np.int64).sum()
