@@ -43,7 +43,8 @@ import workloads  # noqa: E402
 METRIC = "paged decode attn: KV-read GB/s (% of B200 HBM peak), seqs/s at batch"
 UNIT = "GB/s"
 WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shared_prefix",
-             "c5": "c5_long_splitk", "c1": "c1_tiny_fp32", "c3spec": "c3_spec_decode"}
+             "c5": "c5_long_splitk", "c1": "c1_tiny_fp32", "c3spec": "c3_spec_decode",
+             "c3fp8": "c3_fp8"}
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")  # JSON text
@@ -87,7 +88,7 @@ def algorithmic_bytes(b: workloads.Batch) -> dict:
     in use and the context lengths."""
     lens = b.context_lens.astype(np.int64)
     table = int(((lens + 15) // 16).sum()) * 4
-    qo = 2 * b.q.shape[0] * b.num_q_heads * b.head_dim * b.elem_bytes
+    qo = 2 * b.q.shape[0] * b.num_q_heads * b.head_dim * b.q_elem_bytes
     kv = b.unique_kv_bytes() if b.cow_pairs.shape[0] or b.name == "c4_shared_prefix" else b.kv_bytes()
     return {"kv": kv, "kv_logical": b.kv_bytes(), "q_out": qo, "table": table,
             "lens": 4 * b.num_seqs, "total": kv + qo + table + 4 * b.num_seqs}
@@ -235,7 +236,15 @@ class Step:
             else:
                 pkv.slot_mapping(self.bt, b.num_blocks, token_seq=self.seq, token_pos=self.pos,
                                  out=self.slots)
-            pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, self.slots[:self.T])
+            self.write_new(self.slots[:self.T])
+
+    def write_new(self, slots):
+        b = self.b
+        if b.dtype == "fp8":
+            self.pkv.reshape_and_cache_fp8(b.new_k, b.new_v, b.k_cache, b.v_cache, slots,
+                                           b.k_scale, b.v_scale)
+        else:
+            self.pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, slots)
 
     def plan(self):
         self.plan_obj = self.pkv.DecodePlan(self.bt, self.cl, self.b.num_q_heads, self.b.k_cache,
@@ -247,6 +256,9 @@ class Step:
         if self.multi:
             self.plan_obj.run_multi(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.qsl,
                                     self.b.max_query_len, self.b.scale)
+        elif self.b.dtype == "fp8":
+            self.plan_obj.run_fp8(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.b.scale,
+                                  self.b.k_scale, self.b.v_scale)
         else:
             self.plan_obj.run(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.b.scale)
 
@@ -361,12 +373,13 @@ def run_ours(args, world, rank, local):
 def op_bytes(step: Step) -> dict:
     """Algorithmic bytes of each cache-maintenance op of one step (read + write)."""
     b = step.b
-    row = b.num_kv_heads * b.head_dim * b.elem_bytes           # one token's K (or V) rows
+    row = b.num_kv_heads * b.head_dim * b.elem_bytes           # one token's cached K (or V)
+    row_in = b.num_kv_heads * b.head_dim * b.q_elem_bytes      # one new token's K (or V)
     block = row * 16                                            # one K (or V) block
     T, P = step.T, int(b.cow_pairs.shape[0])
     return {
         "slot_mapping": T * (4 + 4 + 8) + (4 * b.num_seqs if step.decode_mode else 8 * T),
-        "reshape_and_cache": 2 * 2 * T * row + 8 * T,           # K and V, read and write
+        "reshape_and_cache": 2 * T * (row_in + row) + 8 * T,    # K and V, read and write
         "copy_blocks": 2 * 2 * P * block + 16 * P,              # K and V, read and write
         # reads the lengths, writes one 16-byte work item per (sequence, partition)
         "plan": 4 * b.num_seqs + 16 * int(np.maximum(
@@ -387,8 +400,7 @@ def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
             ops["slot_mapping"] = lambda: pkv.slot_mapping(step.bt, b.num_blocks,
                                                            token_seq=step.seq, token_pos=step.pos,
                                                            out=step.slots)
-        ops["reshape_and_cache"] = lambda: pkv.reshape_and_cache(
-            b.new_k, b.new_v, b.k_cache, b.v_cache, step.slots[:step.T])
+        ops["reshape_and_cache"] = lambda: step.write_new(step.slots[:step.T])
     if step.pairs is not None:
         ops["copy_blocks"] = lambda: pkv.copy_blocks(b.k_cache, b.v_cache, step.pairs,
                                                      validate=False)
@@ -519,13 +531,19 @@ def oracle_step(b: workloads.Batch, host: dict, seqs: np.ndarray | None, threads
     k, v = host["k_cache"], host["v_cache"]
     if b.cow_pairs.shape[0]:
         oracle.copy_blocks(k, v, b.cow_pairs)
+    fp8 = b.dtype == "fp8"
     if b.new_seq.shape[0]:
-        oracle.reshape_and_cache(host["new_k"], host["new_v"], k, v,
-                                 oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos))
-    if seqs is None:
-        return oracle.paged_decode(host["q"], k, v, b.block_tables, b.context_lens, b.scale,
-                                   threads=threads)
-    tasks = np.array([(s, h) for s in seqs for h in range(b.num_q_heads)], dtype=np.int32)
+        slots = oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos)
+        if fp8:
+            oracle.reshape_and_cache_fp8(host["new_k"], host["new_v"], k, v, slots, b.k_scale,
+                                         b.v_scale)
+        else:
+            oracle.reshape_and_cache(host["new_k"], host["new_v"], k, v, slots)
+    tasks = None if seqs is None else np.array([(s, h) for s in seqs
+                                                for h in range(b.num_q_heads)], dtype=np.int32)
+    if fp8:
+        return oracle.paged_decode_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
+                                       b.context_lens, b.scale, tasks=tasks, threads=threads)
     return oracle.paged_decode(host["q"], k, v, b.block_tables, b.context_lens, b.scale,
                                tasks=tasks, threads=threads)
 

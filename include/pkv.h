@@ -75,8 +75,10 @@ typedef enum pkv_status {
 } pkv_status;
 
 typedef enum pkv_dtype {
-    PKV_F32 = 0,   /* IEEE binary32 */
-    PKV_BF16 = 1   /* bfloat16; arithmetic in fp32, output rounded to nearest even */
+    PKV_F32 = 0,       /* IEEE binary32 */
+    PKV_BF16 = 1,      /* bfloat16; arithmetic in fp32, output rounded to nearest even */
+    PKV_FP8_E4M3 = 2   /* caches hold FP8 e4m3 codes (one byte; value = code x the pool's
+                          scale); q, out and the new K/V are bf16; head_dim 128 only */
 } pkv_dtype;
 
 /* Bits of the per-device error word. */
@@ -248,6 +250,41 @@ pkv_status pkv_paged_attention_decode_static(void *out, const void *q, const voi
                                              const int32_t *context_lens, float scale,
                                              const pkv_dims *dims, int32_t max_context_len,
                                              int32_t partition_tokens, void *cuda_stream);
+
+/*
+ * FP8 KV cache.  The pages list FP8 among the quantisation formats and note
+ * that memory saved holds more KV blocks ("vLLM 深读", section "引擎的分层结构";
+ * "vllm" by vampireachao, "第三层：图、核、量化"); here the cache itself is FP8:
+ * each pool has one scale, a cached element is code x scale.
+ *  - pkv_reshape_and_cache_fp8: k, v are bf16 [T][Hkv][D]; each value x is
+ *    stored as code = e4m3(x / scale) (division in float, round to nearest
+ *    even, saturate to +-448); slots as in pkv_reshape_and_cache.
+ *  - pkv_paged_attention_decode_fp8 / pkv_decode_run_fp8: as the bf16 calls,
+ *    over e4m3 pools with their k_scale and v_scale; q and out are bf16.
+ *    Arithmetic: codes are widened exactly to f16, q is rounded to f16
+ *    (|q| above 65504 saturates), products accumulate in fp32.
+ * dims->dtype must be PKV_FP8_E4M3 (the plain calls reject it); copy_blocks,
+ * slot mapping and the planner work on FP8 pools unchanged.
+ */
+pkv_status pkv_reshape_and_cache_fp8(const void *k, const void *v, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int32_t num_tokens,
+                                     float k_scale, float v_scale, const pkv_dims *dims,
+                                     void *cuda_stream);
+
+pkv_status pkv_paged_attention_decode_fp8(void *out, const void *q, const void *k_cache,
+                                          const void *v_cache, const int32_t *block_tables,
+                                          const int32_t *context_lens, float scale,
+                                          float k_scale, float v_scale, const pkv_dims *dims,
+                                          int32_t max_context_len, int32_t partition_tokens,
+                                          void *workspace, size_t workspace_bytes,
+                                          void *cuda_stream);
+
+pkv_status pkv_decode_run_fp8(void *out, const void *q, const void *k_cache,
+                              const void *v_cache, const int32_t *block_tables,
+                              const int32_t *context_lens, float scale, float k_scale,
+                              float v_scale, const pkv_dims *dims, int32_t max_context_len,
+                              int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                              void *cuda_stream);
 
 /*
  * reshape_and_cache: for every token t with slot_mapping[t] >= 0, copy the

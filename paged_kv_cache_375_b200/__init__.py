@@ -27,7 +27,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpkv.so")
 
-PKV_F32, PKV_BF16 = 0, 1
+PKV_F32, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2
 DEVERR_BLOCK, DEVERR_SLOT, DEVERR_LEN, DEVERR_PAIR, DEVERR_POS, DEVERR_TIMEOUT = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
 
@@ -80,6 +80,11 @@ def load_library() -> ctypes.CDLL:
                                                          i32, i32, P, sz, P]),
             "pkv_decode_run": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P, sz, P]),
             "pkv_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
+            "pkv_reshape_and_cache_fp8": (ctypes.c_int, [P, P, P, P, P, i32, f32, f32, D, P]),
+            "pkv_paged_attention_decode_fp8": (ctypes.c_int, [P, P, P, P, P, P, f32, f32, f32, D,
+                                                              i32, i32, P, sz, P]),
+            "pkv_decode_run_fp8": (ctypes.c_int, [P, P, P, P, P, P, f32, f32, f32, D, i32, i32,
+                                                  P, sz, P]),
             "pkv_copy_blocks": (ctypes.c_int, [P, P, P, i32, D, P]),
             "pkv_validate_copy_pairs": (ctypes.c_int, [P, i32, i32]),
             "pkv_slot_mapping": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
@@ -118,7 +123,9 @@ def _dtype_code(t: torch.dtype) -> int:
         return PKV_BF16
     if t == torch.float32:
         return PKV_F32
-    raise TypeError(f"dtype {t} not supported (bfloat16 or float32)")
+    if t == torch.float8_e4m3fn:
+        return PKV_FP8_E4M3
+    raise TypeError(f"dtype {t} not supported (bfloat16, float32 or float8_e4m3fn caches)")
 
 
 def _stream_ptr(device: torch.device):
@@ -264,6 +271,45 @@ def paged_attention_multi(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Ten
     return out
 
 
+def _check_fp8_decode(out, q, k_cache, v_cache, block_tables, context_lens):
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
+    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must both be [num_blocks][num_kv_heads][16][head_dim]")
+    B, hq, d = q.shape
+    if out.shape != q.shape or block_tables.dim() != 2 or block_tables.shape[0] != B \
+            or context_lens.shape != (B,) or k_cache.shape[3] != d:
+        raise ValueError("inconsistent shapes")
+
+
+def paged_attention_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                               v_cache: torch.Tensor, block_tables: torch.Tensor,
+                               context_lens: torch.Tensor, scale: float, k_scale: float,
+                               v_scale: float, *, max_context_len: int | None = None,
+                               partition_tokens: int = 0,
+                               workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
+    """paged_attention_decode over FP8 (float8_e4m3fn) caches whose elements stand for
+    code * k_scale and code * v_scale; q and out are bfloat16, head_dim 128."""
+    _check_fp8_decode(out, q, k_cache, v_cache, block_tables, context_lens)
+    dev = q.device
+    dims = make_dims(q.shape[0], q.shape[1], k_cache, block_tables.shape[1])
+    mcl = block_tables.shape[1] * k_cache.shape[2] if max_context_len is None else int(max_context_len)
+    need = decode_workspace_bytes(dims, mcl, partition_tokens)
+    if need == 0:
+        raise PkvError(2, load_library().pkv_last_error_message().decode())
+    ws = workspace_tensor if workspace_tensor is not None else workspace(dev, need)
+    _check(load_library().pkv_paged_attention_decode_fp8(
+        _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+        float(scale), float(k_scale), float(v_scale), ctypes.byref(dims), mcl, partition_tokens,
+        _p(ws), ws.numel(), _stream_ptr(dev)))
+    return out
+
+
 class DecodePlan:
     """A decode plan for one step: the work list built from context_lens, kept in a
     workspace.  ``run`` decodes one layer's cache pools with it; plan once per step, run
@@ -331,6 +377,22 @@ class DecodePlan:
             self.partition_tokens, _p(self.workspace), self.workspace.numel(), _stream_ptr(dev)))
         return out
 
+    def run_fp8(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, scale: float, k_scale: float,
+                v_scale: float) -> torch.Tensor:
+        """``run`` over FP8 caches (see paged_attention_decode_fp8)."""
+        _check_fp8_decode(out, q, k_cache, v_cache, self.block_tables, self.context_lens)
+        if q.shape[0] != self.dims.num_seqs or tuple(k_cache.shape) != (
+                self.dims.num_blocks, self.dims.num_kv_heads, 16, self.dims.head_dim):
+            raise ValueError("inconsistent shapes")
+        dims = PkvDims(*[getattr(self.dims, f) for f, _ in PkvDims._fields_[:-1]], PKV_FP8_E4M3)
+        _check(load_library().pkv_decode_run_fp8(
+            _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
+            _p(self.context_lens), float(scale), float(k_scale), float(v_scale),
+            ctypes.byref(dims), self.max_context_len, self.partition_tokens, _p(self.workspace),
+            self.workspace.numel(), _stream_ptr(q.device)))
+        return out
+
 
 def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
                       v_cache: torch.Tensor, slot_mapping: torch.Tensor) -> None:
@@ -348,6 +410,28 @@ def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
     _check(load_library().pkv_reshape_and_cache(_p(k), _p(v), _p(k_cache), _p(v_cache),
                                                 _p(slot_mapping), T, ctypes.byref(dims),
                                                 _stream_ptr(dev)))
+
+
+def reshape_and_cache_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
+                          v_cache: torch.Tensor, slot_mapping: torch.Tensor, k_scale: float,
+                          v_scale: float) -> None:
+    """Quantise bf16 k, v ([T][Hkv][128]) to e4m3 codes (value / scale, nearest even,
+    saturated) and write them into the float8_e4m3fn caches at slot_mapping; -1 skips."""
+    dev = k.device
+    _need(k, "k", torch.bfloat16, dev)
+    _need(v, "v", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
+    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need(slot_mapping, "slot_mapping", torch.int64, dev)
+    T = slot_mapping.shape[0]
+    if k.shape != v.shape or k.shape[0] != T or k.shape[1:] != (k_cache.shape[1], k_cache.shape[3]) \
+            or v_cache.shape != k_cache.shape:
+        raise ValueError("k, v must be [num_tokens][num_kv_heads][head_dim]")
+    dims = make_dims(0, k_cache.shape[1], k_cache, 1)
+    _check(load_library().pkv_reshape_and_cache_fp8(_p(k), _p(v), _p(k_cache), _p(v_cache),
+                                                    _p(slot_mapping), T, float(k_scale),
+                                                    float(v_scale), ctypes.byref(dims),
+                                                    _stream_ptr(dev)))
 
 
 def validate_copy_pairs(pairs_host: torch.Tensor, num_blocks: int) -> None:

@@ -79,13 +79,16 @@ pkv_status bind_device(const void* p, const char* what) {
   return PKV_OK;
 }
 
-int elem_bytes(pkv_dtype t) { return t == PKV_BF16 ? 2 : 4; }
+int elem_bytes(pkv_dtype t) { return t == PKV_BF16 ? 2 : (t == PKV_FP8_E4M3 ? 1 : 4); }
 
 // Checks shared by every call.  `need_seq` also checks the per-sequence fields.
 pkv_status check_dims(const pkv_dims* d, bool need_seq) {
   if (!d) return fail(PKV_ERR_NULL, "dims is NULL");
-  if (d->dtype != PKV_F32 && d->dtype != PKV_BF16)
-    return fail(PKV_ERR_UNSUPPORTED, "dtype %d not supported (fp32 or bf16)", (int)d->dtype);
+  if (d->dtype != PKV_F32 && d->dtype != PKV_BF16 && d->dtype != PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "dtype %d not supported (fp32, bf16, fp8 e4m3)",
+                (int)d->dtype);
+  if (d->dtype == PKV_FP8_E4M3 && d->head_dim != 128)
+    return fail(PKV_ERR_UNSUPPORTED, "FP8 caches need head_dim 128");
   if (d->block_size != pkv::kBlock)
     return fail(PKV_ERR_UNSUPPORTED, "block_size %d not supported (16)", d->block_size);
   if (d->head_dim != 64 && d->head_dim != 128)
@@ -206,8 +209,9 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d
   cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / e), static_cast<cuuint32_t>(pkv::kBlock)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map,
-                   d->dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   d->dtype == PKV_BF16       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                   : d->dtype == PKV_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                    2, const_cast<void*>(pool), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -227,6 +231,12 @@ struct DecodeCfg {
 template <int D, int GMAX>
 struct DecodeCfg<float, D, GMAX> {
   static constexpr int W = 4, S = 2, MB = (D == 128 && GMAX == 16) ? 1 : 2;
+};
+// FP8 tiles are half the size of bf16 ones: twice the stages for the same
+// bytes in flight.
+template <int D, int GMAX>
+struct DecodeCfg<pkv::Fp8Kv, D, GMAX> {
+  static constexpr int W = 8, S = 4, MB = GMAX == 16 ? 1 : 2;
 };
 
 // Largest dynamic shared memory already enabled per kernel, per device.
@@ -262,7 +272,7 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
                          cudaStream_t stream) {
   constexpr int W = DecodeCfg<T, D, GMAX>::W, S = DecodeCfg<T, D, GMAX>::S;
   constexpr int MB = DecodeCfg<T, D, GMAX>::MB;
-  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S, MB>;
+  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S, MB, pkv::q_elem_bytes<T>()>;
   const int smem = Lay::total_bytes(rows_max);
   int dev = 0, max_optin = 0;
   cudaGetDevice(&dev);
@@ -357,7 +367,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
                       const int32_t* block_tables, const int32_t* context_lens,
                       const int32_t* query_start_loc, int32_t max_query_len, float scale,
                       const pkv_dims* d, const DecodePlan& plan, void* workspace,
-                      size_t workspace_bytes, void* cuda_stream) {
+                      size_t workspace_bytes, void* cuda_stream, float k_scale = 1.f,
+                      float v_scale = 1.f) {
   pkv_status st;
   if (d->num_seqs == 0 || plan.num_q_tokens == 0) return PKV_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
@@ -366,6 +377,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
   if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
   if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
   if (max_query_len < 1) return fail(PKV_ERR_SHAPE, "max_query_len must be >= 1");
   const int group = d->num_q_heads / d->num_kv_heads;
   const int rows_max = max_query_len * group;
@@ -397,9 +410,12 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.num_blocks = d->num_blocks;
   prm.max_parts = plan.max_parts;
   prm.part_blocks = plan.part_blocks;
-  prm.qk_scale_log2 = scale * pkv::kLog2e;
+  prm.qk_scale_log2 = scale * pkv::kLog2e * k_scale;
+  prm.out_scale = v_scale;
   const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads;
-  if (d->dtype == PKV_BF16) {
+  if (d->dtype == PKV_FP8_E4M3) {
+    st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
+  } else if (d->dtype == PKV_BF16) {
     st = d->head_dim == 128
              ? launch_decode_d<__nv_bfloat16, 128>(mk, mv, prm, units, rows_max, stream)
              : launch_decode_d<__nv_bfloat16, 64>(mk, mv, prm, units, rows_max, stream);
@@ -409,7 +425,7 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   }
   if (st != PKV_OK) return st;
   if (plan.max_parts > 1) {
-    st = d->dtype == PKV_BF16
+    st = d->dtype != PKV_F32
              ? launch_merge<__nv_bfloat16>(out, plan, ws, context_lens, query_start_loc, d, stream)
              : launch_merge<float>(out, plan, ws, context_lens, query_start_loc, d, stream);
   }
@@ -475,6 +491,8 @@ pkv_status pkv_decode_run(void* out, const void* q, const void* k_cache, const v
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
+  if (dims->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "FP8 caches need their scales: use pkv_decode_run_fp8");
   return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
                     dims, plan, workspace, workspace_bytes, cuda_stream);
 }
@@ -488,6 +506,9 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
+  if (dims->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED,
+                "FP8 caches need their scales: use pkv_paged_attention_decode_fp8");
   if (dims->num_seqs == 0) return PKV_OK;
   // Check everything the run needs before launching the plan.
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
@@ -551,6 +572,70 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
                     max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream);
 }
 
+pkv_status pkv_decode_run_fp8(void* out, const void* q, const void* k_cache,
+                              const void* v_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, float scale, float k_scale,
+                              float v_scale, const pkv_dims* dims, int32_t max_context_len,
+                              int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                              void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
+                    dims, plan, workspace, workspace_bytes, cuda_stream, k_scale, v_scale);
+}
+
+pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_cache,
+                                          const void* v_cache, const int32_t* block_tables,
+                                          const int32_t* context_lens, float scale,
+                                          float k_scale, float v_scale, const pkv_dims* dims,
+                                          int32_t max_context_len, int32_t partition_tokens,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+  if (dims->num_seqs == 0) return PKV_OK;
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  st = pkv_decode_plan(context_lens, dims, max_context_len, partition_tokens, workspace,
+                       workspace_bytes, cuda_stream);
+  if (st != PKV_OK) return st;
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
+                    dims, plan, workspace, workspace_bytes, cuda_stream, k_scale, v_scale);
+}
+
+pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                                     const int64_t* slot_mapping, int32_t num_tokens,
+                                     float k_scale, float v_scale, const pkv_dims* dims,
+                                     void* cuda_stream) {
+  pkv_status st = check_dims(dims, false);
+  if (st != PKV_OK) return st;
+  if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+  if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
+  if (num_tokens == 0) return PKV_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "k, v and the caches must be 16-byte aligned");
+  if ((st = bind_device(k_cache, "k_cache")) != PKV_OK) return st;
+  const int units = dims->num_kv_heads * dims->head_dim / 8;
+  const int threads = units < 256 ? (units + 31) / 32 * 32 : 256;
+  cudaError_t e = launch(pkv::reshape_and_cache_fp8_kernel, dim3(num_tokens), dim3(threads), 0,
+                         static_cast<cudaStream_t>(cuda_stream), static_cast<const uint4*>(k),
+                         static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
+                         static_cast<uint8_t*>(v_cache), slot_mapping, dims->num_kv_heads,
+                         dims->head_dim, static_cast<int64_t>(dims->num_blocks) * pkv::kBlock,
+                         k_scale, v_scale);
+  if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache_fp8 launch");
+  return PKV_OK;
+}
+
 pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_cache,
                                              const void* v_cache, const int32_t* block_tables,
                                              const int32_t* context_lens, float scale,
@@ -576,6 +661,8 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, vo
                                  const pkv_dims* dims, void* cuda_stream) {
   pkv_status st = check_dims(dims, false);
   if (st != PKV_OK) return st;
+  if (dims->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "FP8 caches quantise on write: use pkv_reshape_and_cache_fp8");
   if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
   if (num_tokens == 0) return PKV_OK;
   if (!k || !v || !k_cache || !v_cache || !slot_mapping)

@@ -83,6 +83,52 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ------------------------------------------------ reshape_and_cache into FP8
+// One CTA per token: each thread turns 8 bf16 values of the token's K (and V)
+// into 8 e4m3 codes, code = e4m3(value / scale) with the division in float,
+// rounded to nearest even and saturated to +-448, and stores them at the slot.
+__global__ void __launch_bounds__(256)
+    reshape_and_cache_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                 uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
+                                 const int64_t* __restrict__ slot_mapping, int32_t num_kv_heads,
+                                 int32_t head_dim, int64_t num_slots, float k_scale,
+                                 float v_scale) {
+  pdl_wait();
+  pdl_trigger();
+  const int32_t t = blockIdx.x;
+  const int64_t slot = slot_mapping[t];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (threadIdx.x == 0) raise_error(PKV_DEVERR_SLOT);
+    return;
+  }
+  const int64_t block = slot / kBlock;
+  const int32_t offset = static_cast<int32_t>(slot % kBlock);
+  const int32_t units_per_row = head_dim / 8;
+  const int32_t units = num_kv_heads * units_per_row;
+  for (int32_t u = threadIdx.x; u < units; u += blockDim.x) {
+    const int32_t h = u / units_per_row;
+    const int32_t within = u % units_per_row;
+    const int64_t dst = ((block * num_kv_heads + h) * kBlock + offset) * head_dim + within * 8;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const uint4 x = (c ? v : k)[static_cast<int64_t>(t) * units + u];
+      const float sc = c ? v_scale : k_scale;
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t codes[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t p0 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i]), sc),
+                                            __fdiv_rn(bf16hi_to_f32(w[2 * i]), sc));
+        const uint32_t p1 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i + 1]), sc),
+                                            __fdiv_rn(bf16hi_to_f32(w[2 * i + 1]), sc));
+        codes[i] = p0 | (p1 << 16);
+      }
+      *reinterpret_cast<uint2*>((c ? v_cache : k_cache) + dst) = make_uint2(codes[0], codes[1]);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ copy_blocks
 // Grid: (pair, chunk, cache).  One thread moves one chunk of a block with the
 // bulk-copy (TMA) engine: global -> shared, then shared -> global.

@@ -162,8 +162,18 @@ struct DecodeParams {
   int32_t num_blocks;
   int32_t max_parts;
   int32_t part_blocks;
-  float qk_scale_log2;           // scale * log2(e)
+  float qk_scale_log2;           // scale * log2(e) (times the K scale for FP8 caches)
+  float out_scale;               // 1, or the V scale for FP8 caches
 };
+
+// Tag type of an FP8 (e4m3) cache: one-byte codes, bf16 q and out.
+struct Fp8Kv {};
+
+// Bytes per q / out element for a cache element type.
+template <typename T>
+constexpr int q_elem_bytes() {
+  return sizeof(T) == 4 ? 4 : 2;
+}
 
 // Largest partition (in blocks) the decode kernel handles; the block-table
 // slice of every item in flight is staged in shared memory.
@@ -173,12 +183,12 @@ constexpr int kMaxItemBlocks = 512;
 // MB merge buffers: with two, consecutive items alternate buffers and one
 // barrier per item suffices; with one (when two do not fit), a second
 // barrier keeps the next item's states out until the current one is combined.
-template <int ELEM, int D, int GMAX, int W, int S, int MB = 2>
+template <int ELEM, int D, int GMAX, int W, int S, int MB = 2, int QELEM = ELEM>
 struct DecodeLayout {
   static constexpr int kTileBytes = kBlock * D * ELEM;       // one K (or V) tile
   static constexpr int kChunks = D * ELEM / 128;             // 128-byte column chunks
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kQBytes = ((GMAX * D * ELEM) + 127) / 128 * 128;
+  static constexpr int kQBytes = ((GMAX * D * QELEM) + 127) / 128 * 128;
   static constexpr int kStagesOff = 0;
   static constexpr int kRingOff = kStagesOff + W * S * kStageBytes;
   static constexpr int kTablesOff = kRingOff + kRing * kQBytes;
@@ -426,6 +436,228 @@ __device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot
     }
 }
 
+// ---- consumer state for an FP8 (e4m3) cache (f16 tensor cores) ----
+//
+// Tiles hold one-byte codes [16 tokens][128 d].  K fragments come from
+// ldmatrix on 16-bit units, so a lane holds four consecutive d-values of a
+// token; the k-order of S^T = K Q^T is permuted to match (k-slots 2q, 2q+1,
+// 2q+8, 2q+9 of a 16-wide step are d 4q .. 4q+3 of that step) and Q's
+// fragments are built in the same order.  V fragments come from
+// ldmatrix.trans on 16-bit units (pairs of d-values); a byte permute splits
+// the pairs, so row r of an output m-tile is d = 16mt + 2r and row r+8 is
+// d = 16mt + 2r + 1.  Codes become f16 exactly (cvt.f16x2.e4m3x2); the K
+// scale is folded into the score scale and the V scale into the output.
+template <int GMAX>
+struct Fp8State {
+  static constexpr int D = 128;
+  static constexpr int KS = 8, MT = 8, NH = GMAX / 8;
+  uint32_t qb[NH][KS][2];  // f16 B fragments of Q^T in the permuted k-order
+  float o[NH][MT][4];
+  float m[NH][2], l[NH][2];
+  int32_t lim[NH][2];
+};
+
+template <int GMAX>
+__device__ __forceinline__ void fp8_begin_item(Fp8State<GMAX>& st, const uint8_t* qs, int rows,
+                                               int g, int len, int q_len, int lane) {
+  using St = Fp8State<GMAX>;
+  const int r = lane >> 2, q4 = (lane & 3) * 4, qd = (lane & 3) * 2;
+  const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qs);  // bf16 rows of 128
+#pragma unroll
+  for (int nh = 0; nh < St::NH; ++nh) {
+    const int row = nh * 8 + r;
+#pragma unroll
+    for (int ks = 0; ks < St::KS; ++ks) {
+      if (row < rows) {
+        const uint2 w = *reinterpret_cast<const uint2*>(q16 + row * 128 + ks * 16 + q4);
+        st.qb[nh][ks][0] = pack_f16x2(bf16lo_to_f32(w.x), bf16hi_to_f32(w.x));
+        st.qb[nh][ks][1] = pack_f16x2(bf16lo_to_f32(w.y), bf16hi_to_f32(w.y));
+      } else {
+        st.qb[nh][ks][0] = st.qb[nh][ks][1] = 0u;
+      }
+    }
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      const int n = nh * 8 + qd + hc;
+      st.lim[nh][hc] = n < rows ? len - q_len + n / g : -1;
+    }
+#pragma unroll
+    for (int mt = 0; mt < St::MT; ++mt) {
+      st.o[nh][mt][0] = st.o[nh][mt][1] = st.o[nh][mt][2] = st.o[nh][mt][3] = 0.f;
+    }
+    st.m[nh][0] = st.m[nh][1] = -INFINITY;
+    st.l[nh][0] = st.l[nh][1] = 0.f;
+  }
+}
+
+template <int GMAX>
+__device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
+                                         const uint8_t* v0, int valid0, int pos0,
+                                         const uint8_t* k1, const uint8_t* v1, int valid1,
+                                         int pos1, float sc, int lane) {
+  using St = Fp8State<GMAX>;
+  constexpr int NH = St::NH;
+  const int r = lane >> 2, qd = (lane & 3) * 2;
+  // ldmatrix.x4 rows: lanes 0-7 tokens 0-7 / granule 2p, 8-15 tokens 8-15 / 2p,
+  // 16-23 tokens 0-7 / 2p+1, 24-31 tokens 8-15 / 2p+1 (a granule = 16 codes).
+  const uint32_t tok = ((lane >> 3) & 1) * 8 + (lane & 7);
+  const uint32_t gsel = lane >> 4;
+  // ---- S^T = K Q^T ----
+  float s[2][2][NH][4];
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) s[t][c][nh][0] = s[t][c][nh][1] = s[t][c][nh][2] = s[t][c][nh][3] = 0.f;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const uint32_t base = smem_addr(t ? k1 : k0) + tok * 128u;
+#pragma unroll
+    for (int kp = 0; kp < St::KS / 2; ++kp) {
+      const uint32_t off = ((((kp * 2) + gsel) ^ (tok & 7u)) << 4);
+      uint32_t m0, m1, m2, m3;
+      ldmatrix_x4(base + off, m0, m1, m2, m3);
+      const uint32_t a_lo[4] = {e4m3x2_to_f16x2(m0), e4m3x2_to_f16x2(m1),
+                                e4m3x2_to_f16x2(m0 >> 16), e4m3x2_to_f16x2(m1 >> 16)};
+      const uint32_t a_hi[4] = {e4m3x2_to_f16x2(m2), e4m3x2_to_f16x2(m3),
+                                e4m3x2_to_f16x2(m2 >> 16), e4m3x2_to_f16x2(m3 >> 16)};
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh) {
+        mma_f16_16816(s[t][0][nh], a_lo, st.qb[nh][2 * kp][0], st.qb[nh][2 * kp][1]);
+        mma_f16_16816(s[t][1][nh], a_hi, st.qb[nh][2 * kp + 1][0], st.qb[nh][2 * kp + 1][1]);
+      }
+    }
+  }
+  // ---- scale and mask; element i of a C fragment is token r + 8(i>>1), row 2q + (i&1) ----
+  float z[2][NH][4];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int valid = t ? valid1 : valid0;
+    const int pos = t ? pos1 : pos0;
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tk = r + 8 * (i >> 1);
+        const float v = (s[t][0][nh][i] + s[t][1][nh][i]) * sc;
+        z[t][nh][i] = (tk < valid && pos + tk <= st.lim[nh][i & 1]) ? v : -INFINITY;
+      }
+  }
+  // ---- running max, lazy rescale (as for bf16) ----
+  bool grow = false;
+  float m_new[NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      float mx = fmaxf(fmaxf(z[0][nh][hc], z[0][nh][hc + 2]), fmaxf(z[1][nh][hc], z[1][nh][hc + 2]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      m_new[nh][hc] = mx;
+      grow |= mx > st.m[nh][hc] + kRescaleSlack;
+    }
+  if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        if (m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack) {
+          const float alpha = fast_exp2(st.m[nh][hc] - m_new[nh][hc]);
+          st.m[nh][hc] = m_new[nh][hc];
+          st.l[nh][hc] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < St::MT; ++mt) {
+            st.o[nh][mt][hc] *= alpha;
+            st.o[nh][mt][hc + 2] *= alpha;
+          }
+        }
+      }
+  }
+  // ---- P = exp2(z - m) in f16, transposed into B fragments ----
+  uint32_t pb[2][NH][2];
+#pragma unroll
+  for (int nh = 0; nh < NH; ++nh) {
+    const float mu0 = st.m[nh][0] == -INFINITY ? 0.f : st.m[nh][0];
+    const float mu1 = st.m[nh][1] == -INFINITY ? 0.f : st.m[nh][1];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint32_t lo = pack_f16x2(fast_exp2(z[t][nh][0] - mu0), fast_exp2(z[t][nh][1] - mu1));
+      const uint32_t hi = pack_f16x2(fast_exp2(z[t][nh][2] - mu0), fast_exp2(z[t][nh][3] - mu1));
+      st.l[nh][0] += f16lo_to_f32(lo) + f16lo_to_f32(hi);
+      st.l[nh][1] += f16hi_to_f32(lo) + f16hi_to_f32(hi);
+      pb[t][nh][0] = movmatrix_trans(lo);
+      pb[t][nh][1] = movmatrix_trans(hi);
+    }
+  }
+  // ---- O^T += V^T P^T (m-tile rows interleave d: r -> 2r, r+8 -> 2r+1) ----
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int valid = t ? valid1 : valid0;
+    const uint32_t base = smem_addr(t ? v1 : v0) + tok * 128u;
+    uint32_t mk0 = 0xffffffffu, mk1 = 0xffffffffu;
+    const bool partial = valid < kBlock;
+    if (partial) {
+      mk0 = (qd < valid ? 0x0000ffffu : 0u) | (qd + 1 < valid ? 0xffff0000u : 0u);
+      mk1 = (qd + 8 < valid ? 0x0000ffffu : 0u) | (qd + 9 < valid ? 0xffff0000u : 0u);
+    }
+#pragma unroll
+    for (int mp = 0; mp < St::MT / 2; ++mp) {
+      const uint32_t off = ((((mp * 2) + gsel) ^ (tok & 7u)) << 4);
+      uint32_t m0, m1, m2, m3;
+      ldmatrix_x4_trans(base + off, m0, m1, m2, m3);
+      // m0 / m1: tokens 0-7 / 8-15 of granule 2mp; m2 / m3: of granule 2mp+1
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const uint32_t ya = __byte_perm(hlf ? m2 : m0, 0u, 0x3120u);
+        const uint32_t yb = __byte_perm(hlf ? m3 : m1, 0u, 0x3120u);
+        uint32_t a[4] = {e4m3x2_to_f16x2(ya), e4m3x2_to_f16x2(ya >> 16),
+                         e4m3x2_to_f16x2(yb), e4m3x2_to_f16x2(yb >> 16)};
+        if (partial) {
+          a[0] &= mk0;
+          a[1] &= mk0;
+          a[2] &= mk1;
+          a[3] &= mk1;
+        }
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) mma_f16_16816(st.o[nh][2 * mp + hlf], a, pb[t][nh][0], pb[t][nh][1]);
+      }
+    }
+  }
+}
+
+template <int GMAX>
+__device__ __forceinline__ void fp8_publish(Fp8State<GMAX>& st, float* slot, int rows, int lane) {
+  using St = Fp8State<GMAX>;
+  constexpr int D = 128;
+  const int r = lane >> 2, qd = (lane & 3) * 2;
+  float* O = slot;
+  float* M = slot + rows * D;
+  float* L = M + rows;
+#pragma unroll
+  for (int nh = 0; nh < St::NH; ++nh)
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      float l = st.l[nh][hc];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      const int row = nh * 8 + qd + hc;
+      if (row < rows) {
+#pragma unroll
+        for (int mt = 0; mt < St::MT; ++mt) {
+          O[row * D + mt * 16 + 2 * r] = st.o[nh][mt][hc];
+          O[row * D + mt * 16 + 2 * r + 1] = st.o[nh][mt][hc + 2];
+        }
+        if (r == 0) {
+          M[row] = st.m[nh][hc];
+          L[row] = l;
+        }
+      }
+    }
+}
+
 // ---- consumer state for fp32 (CUDA cores) ----
 template <int D, int GMAX>
 struct F32State {
@@ -562,7 +794,7 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
         acc.z = fmaf(ov.z, f, acc.z);
         acc.w = fmaf(ov.w, f, acc.w);
       }
-      const float inv = 1.f / lsum;
+      const float inv = prm.out_scale / lsum;
       acc.x *= inv;
       acc.y *= inv;
       acc.z *= inv;
@@ -572,7 +804,7 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
     const size_t row = static_cast<size_t>(it.q_start + h / group) * prm.num_q_heads +
                        it.kv_head * group + h % group;
     if (it.nparts == 1) {
-      if constexpr (sizeof(T) == 2) {
+      if constexpr (sizeof(T) != 4) {  // bf16 output (bf16 and FP8 caches)
         uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
         *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(prm.out) + row * D + d) = packed;
       } else {
@@ -602,8 +834,9 @@ template <typename T, int D, int GMAX, int W, int S, int MB>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
-  constexpr int ELEM = sizeof(T);
-  using Lay = DecodeLayout<ELEM, D, GMAX, W, S, MB>;
+  constexpr int ELEM = sizeof(T);            // cache bytes per element (1 for FP8)
+  constexpr int QELEM = q_elem_bytes<T>();   // q bytes per element
+  using Lay = DecodeLayout<ELEM, D, GMAX, W, S, MB, QELEM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -709,13 +942,13 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         mt.nblk = nblk;
         mt.q_start = q_start;
         mt.q_len = q_len;
-        const uint32_t row_bytes = static_cast<uint32_t>(g * D * ELEM);  // one token's group
+        const uint32_t row_bytes = static_cast<uint32_t>(g * D * QELEM);  // one token's group
         if (q_len > 0) {
           mbar_arrive_expect_tx(&item_full[r], row_bytes * q_len);
           for (int32_t i = 0; i < q_len; ++i) {
             const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(prm.q) +
                                   (static_cast<size_t>(q_start + i) * prm.num_q_heads + kvh * g) *
-                                      D * ELEM;
+                                      D * QELEM;
             bulk_load(ring + r * Lay::kQBytes + i * row_bytes, qsrc, row_bytes, &item_full[r]);
           }
         } else {
@@ -739,8 +972,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   // ================================ decode warps ================================
   using Bst = Bf16State<D, GMAX>;
   using Fst = F32State<D, GMAX>;
+  constexpr bool kFp8 = std::is_same<T, Fp8Kv>::value;
   constexpr bool kBf16 = sizeof(T) == 2;
-  typename std::conditional<kBf16, Bst, Fst>::type st;
+  typename std::conditional<kFp8, Fp8State<GMAX>,
+                            typename std::conditional<kBf16, Bst, Fst>::type>::type st;
   const float sc = prm.qk_scale_log2;
   const int per_warp = Lay::merge_floats_per_warp(rows_max);
   uint64_t* my_full = full + warp * S;
@@ -820,13 +1055,15 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     if (it.seq < 0) break;
     const uint8_t* qs = ring + r * Lay::kQBytes;
     const int rows = it.q_len * g;  // query rows of this item
-    if constexpr (kBf16) {
+    if constexpr (kFp8) {
+      fp8_begin_item<GMAX>(st, qs, rows, g, it.len, it.q_len, lane);
+    } else if constexpr (kBf16) {
       bf16_begin_item<D, GMAX>(st, qs, rows, g, it.len, it.q_len, lane);
     } else {
       f32_begin_item<D, GMAX>(st, rows, g, it.len, it.q_len);
     }
     // bf16 consumes this warp's blocks two at a time (b and b + W), fp32 one at a time.
-    constexpr int kStep = kBf16 ? 2 : 1;
+    constexpr int kStep = (kBf16 || kFp8) ? 2 : 1;
     for (int32_t b = warp; b < it.nblk; b += kStep * W) {
       const int n = (kStep == 2 && b + W < it.nblk) ? 2 : 1;
       if (pctr < cctr + n) {
@@ -851,7 +1088,10 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
       }
       if (!ok) break;
       const int pos0 = (it.blk_begin + b) * kBlock;  // position of the first tile's token 0
-      if constexpr (kBf16) {
+      if constexpr (kFp8) {
+        fp8_step<GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
+                       kt[1] + Lay::kTileBytes, valid[1], pos0 + W * kBlock, sc, lane);
+      } else if constexpr (kBf16) {
         bf16_step<D, GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
                            kt[1] + Lay::kTileBytes, valid[1], pos0 + W * kBlock, sc, lane);
       } else {
@@ -877,7 +1117,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
       break;
     }
     float* mslot = merge + (mb * W + warp) * per_warp;
-    if constexpr (kBf16) {
+    if constexpr (kFp8) {
+      fp8_publish<GMAX>(st, mslot, rows, lane);
+    } else if constexpr (kBf16) {
       bf16_publish<D, GMAX>(st, mslot, rows, lane);
     } else {
       f32_publish<D, GMAX>(st, mslot, rows, lane);

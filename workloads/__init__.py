@@ -96,7 +96,7 @@ class Batch:
 
     name: str
     seed: int
-    dtype: str                      # "f32" or "bf16"
+    dtype: str                      # "f32", "bf16" or "fp8" (e4m3 caches, bf16 q and new K/V)
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
@@ -115,6 +115,9 @@ class Batch:
     meta: dict = field(default_factory=dict)
     # several query tokens per sequence: rows query_start_loc[s] .. [s+1]-1 of q
     query_start_loc: np.ndarray | None = None
+    # FP8 caches: a cached code c stands for c * k_scale (K) or c * v_scale (V)
+    k_scale: float = 1.0
+    v_scale: float = 1.0
 
     @property
     def num_seqs(self) -> int:
@@ -140,6 +143,12 @@ class Batch:
 
     @property
     def elem_bytes(self) -> int:
+        """Bytes of one cache element."""
+        return {"f32": 4, "bf16": 2, "fp8": 1}[self.dtype]
+
+    @property
+    def q_elem_bytes(self) -> int:
+        """Bytes of one q / out / new K/V element."""
         return 4 if self.dtype == "f32" else 2
 
     def kv_bytes(self) -> int:
@@ -160,14 +169,17 @@ class Batch:
     def io_bytes(self) -> int:
         """q + out + block-table + context-length bytes of one decode step."""
         T, Hq, D = self.q.shape[0], self.num_q_heads, self.head_dim
-        return 2 * T * Hq * D * self.elem_bytes + self.block_tables.nbytes + self.context_lens.nbytes
+        return 2 * T * Hq * D * self.q_elem_bytes + self.block_tables.nbytes + self.context_lens.nbytes
 
     def host(self) -> dict:
-        """Host numpy copies: float32 arrays, or uint16 arrays holding bf16 bits."""
+        """Host numpy copies: float32 arrays, uint16 arrays holding bf16 bits, or uint8
+        arrays holding e4m3 codes."""
         def h(t):
             t = t.detach().contiguous().cpu()
             if t.dtype == torch.bfloat16:
                 return t.view(torch.int16).numpy().view(np.uint16)
+            if t.dtype == torch.float8_e4m3fn:
+                return t.view(torch.uint8).numpy()
             return t.numpy()
         return {"q": h(self.q), "k_cache": h(self.k_cache), "v_cache": h(self.v_cache),
                 "new_k": h(self.new_k), "new_v": h(self.new_v)}
@@ -179,11 +191,38 @@ class Batch:
                      self.k_cache.to(device), self.v_cache.to(device), self.new_k.to(device),
                      self.new_v.to(device), self.new_seq.copy(), self.new_pos.copy(),
                      self.cow_pairs.copy(), dict(self.meta),
-                     None if self.query_start_loc is None else self.query_start_loc.copy())
+                     None if self.query_start_loc is None else self.query_start_loc.copy(),
+                     self.k_scale, self.v_scale)
 
 
 def torch_dtype(dtype: str) -> torch.dtype:
-    return {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
+    """Element type of q / out / new K/V (an FP8 configuration's caches are e4m3)."""
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}[dtype]
+
+
+# Scales of the FP8 configurations' pools (exact in float32, different so that
+# a swapped pair shows).
+FP8_K_SCALE = 1.0 / 64.0
+FP8_V_SCALE = 3.0 / 128.0
+E4M3_NAN_CODE = 0x7F
+
+
+def _random_codes(shape, gen, device, chunk_rows: int | None = None) -> torch.Tensor:
+    """Random e4m3 bit patterns: sign, exponent field 1..15 and mantissa drawn uniformly
+    (magnitudes log-uniform over 2^-6 .. 448); the NaN pattern is replaced by its
+    neighbour 0x7e.  A drawing of codes, not a quantisation."""
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    rows = shape[0]
+    step = chunk_rows or rows
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        sub = (r1 - r0,) + tuple(shape[1:])
+        sign = torch.randint(0, 2, sub, generator=gen, device=device, dtype=torch.uint8)
+        expo = torch.randint(1, 16, sub, generator=gen, device=device, dtype=torch.uint8)
+        mant = torch.randint(0, 8, sub, generator=gen, device=device, dtype=torch.uint8)
+        c = (sign << 7) | (expo << 3) | mant
+        out[r0:r1] = torch.where((c & 0x7F) == E4M3_NAN_CODE, c - 1, c)
+    return out.view(torch.float8_e4m3fn)
 
 
 def default_scale(head_dim: int) -> float:
@@ -222,12 +261,18 @@ def _assemble(name: str, seed: int, dtype: str, hq: int, hkv: int, d: int, num_b
     gen.manual_seed(seed)
     shape = (num_blocks, hkv, BLOCK_SIZE, d)
     chunk = max(1, (1 << 26) // (hkv * BLOCK_SIZE * d))
-    k_cache = _randn(shape, gen, device, dtype, chunk)
-    v_cache = _randn(shape, gen, device, dtype, chunk)
-    q = _randn((B, hq, d), gen, device, dtype)
+    fp8 = dtype == "fp8"
+    vdt = "bf16" if fp8 else dtype
+    if fp8:
+        k_cache = _random_codes(shape, gen, device, chunk)
+        v_cache = _random_codes(shape, gen, device, chunk)
+    else:
+        k_cache = _randn(shape, gen, device, dtype, chunk)
+        v_cache = _randn(shape, gen, device, dtype, chunk)
+    q = _randn((B, hq, d), gen, device, vdt)
     T = int(new_seq.shape[0])
-    new_k = _randn((T, hkv, d), gen, device, dtype)
-    new_v = _randn((T, hkv, d), gen, device, dtype)
+    new_k = _randn((T, hkv, d), gen, device, vdt)
+    new_v = _randn((T, hkv, d), gen, device, vdt)
 
     # Poison: unreferenced blocks, and slots at or past the prefill length.
     referenced = np.zeros(num_blocks, dtype=bool)
@@ -246,18 +291,23 @@ def _assemble(name: str, seed: int, dtype: str, hq: int, hkv: int, d: int, num_b
         else:
             referenced[b] = True
     unref = torch.from_numpy(np.nonzero(~referenced)[0]).to(device)
-    nan = float("nan")
+    # NaN for float pools; the NaN code through a byte view for e4m3 pools
+    kp, vp = (k_cache.view(torch.uint8), v_cache.view(torch.uint8)) if fp8 else (k_cache, v_cache)
+    nan = E4M3_NAN_CODE if fp8 else float("nan")
     if unref.numel():
-        k_cache.index_fill_(0, unref, nan)
-        v_cache.index_fill_(0, unref, nan)
+        kp.index_fill_(0, unref, nan)
+        vp.index_fill_(0, unref, nan)
     for b, rem in partial.items():
-        k_cache[b, :, rem:, :] = nan
-        v_cache[b, :, rem:, :] = nan
+        kp[b, :, rem:, :] = nan
+        vp[b, :, rem:, :] = nan
 
     pairs = np.array(cow_pairs, dtype=np.int64).reshape(-1, 2)
-    return Batch(name, seed, dtype, hq, hkv, d, num_blocks, lens.astype(np.int32), bt,
-                 default_scale(d) if scale is None else scale, q, k_cache, v_cache, new_k, new_v,
-                 new_seq.astype(np.int32), new_pos.astype(np.int32), pairs, meta)
+    b = Batch(name, seed, dtype, hq, hkv, d, num_blocks, lens.astype(np.int32), bt,
+              default_scale(d) if scale is None else scale, q, k_cache, v_cache, new_k, new_v,
+              new_seq.astype(np.int32), new_pos.astype(np.int32), pairs, meta)
+    if fp8:
+        b.k_scale, b.v_scale = FP8_K_SCALE, FP8_V_SCALE
+    return b
 
 
 def random_batch(seed: int, lens, hq: int, hkv: int, d: int, dtype: str = "bf16",
@@ -324,6 +374,19 @@ def c3_llama3_8b_gqa(device="cpu", num_seqs: int = 256) -> Batch:
     nb = max(32768, int(math.ceil(1.25 * need)))
     b = random_batch(seed, lens, 32, 8, 128, "bf16", num_blocks=nb, device=device,
                      new_token=True, name="c3_llama3_8b_gqa")
+    b.meta["lognormal_sigma"] = C3_LOGNORMAL_SIGMA
+    return b
+
+
+def c3_fp8(device="cpu", num_seqs: int = 256) -> Batch:
+    """The Llama-3-8B-shaped GQA decode batch (same lengths and tables) over FP8 e4m3
+    pools with one scale per pool; q and the new tokens' K/V are bf16."""
+    seed = CONFIG_SEEDS["c3_llama3_8b_gqa"]
+    lens = c3_lens(num_seqs)
+    need = int(sum((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE for L in lens))
+    nb = max(32768, int(math.ceil(1.25 * need)))
+    b = random_batch(seed, lens, 32, 8, 128, "fp8", num_blocks=nb, device=device,
+                     new_token=True, name="c3_fp8_llama3_8b_gqa")
     b.meta["lognormal_sigma"] = C3_LOGNORMAL_SIGMA
     return b
 
@@ -438,10 +501,14 @@ def c5_long_splitk(device="cpu", num_seqs: int = 8) -> Batch:
 
 CONFIGS["c3_spec_decode"] = ("Llama-3-8B-shaped GQA bf16, batch 256, verifying 4 speculative tokens "
                               "per sequence (causal, 16 query rows per kv head)")
+CONFIGS["c3_fp8"] = ("Llama-3-8B-shaped GQA over FP8 e4m3 pools (one scale per pool), bf16 q/out: "
+                     "batch 256, 32q/8kv, d128, the same lognormal lens, reshape_and_cache_fp8 "
+                     "of the new token before attention")
 
 BUILDERS = {
     "c1_tiny_fp32": c1_tiny_fp32,
     "c3_spec_decode": c3_spec_decode,
+    "c3_fp8": c3_fp8,
     "c2_llama2_13b_mha": c2_llama2_13b_mha,
     "c3_llama3_8b_gqa": c3_llama3_8b_gqa,
     "c4_shared_prefix": c4_shared_prefix,
