@@ -234,8 +234,9 @@ struct Bf16State {
   uint32_t qb[NH][KS][2];              // B fragments of Q^T
   float o[NH][MT][4];                  // O^T accumulators
   float m[NH][2];                      // running max of rows 8nh + 2(lane%4) + {0,1}
-  float l[NH][2];                      // this lane's part of the softmax denominators
+  float lsum[NH][4];                   // softmax denominators, summed by a tensor-core MMA
   int32_t lim[NH][2];                  // last key position those rows may see (causal)
+  int32_t lim_min;                     // smallest limit over the item's rows
 };
 
 // Query rows of an item: row n = i*g + h is chunk token i (at position
@@ -265,8 +266,9 @@ __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const ui
       st.o[nh][mt][0] = st.o[nh][mt][1] = st.o[nh][mt][2] = st.o[nh][mt][3] = 0.f;
     }
     st.m[nh][0] = st.m[nh][1] = -INFINITY;
-    st.l[nh][0] = st.l[nh][1] = 0.f;
+    st.lsum[nh][0] = st.lsum[nh][1] = st.lsum[nh][2] = st.lsum[nh][3] = 0.f;
   }
+  st.lim_min = len - q_len;
 }
 
 // Two 16-token tiles (the second may be absent: valid1 = 0 and its pointers
@@ -307,22 +309,30 @@ __device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t*
       }
     }
   }
-  // ---- scale and mask; element i of a C fragment is token r + 8(i>>1), head 2q + (i&1) ----
+  // ---- mask (raw scores; element i of a C fragment is token r + 8(i>>1), head 2q + (i&1)).
+  // Tiles that are full and wholly inside every row's causal window need no mask.
   float z[2][NH][4];
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int valid = t ? valid1 : valid0;
-    const int pos = t ? pos1 : pos0;
+  for (int t = 0; t < 2; ++t)
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tok = r + 8 * (i >> 1);
-        const float v = (s[t][0][nh][i] + s[t][1][nh][i]) * sc;
-        z[t][nh][i] = (tok < valid && pos + tok <= st.lim[nh][i & 1]) ? v : -INFINITY;
-      }
+      for (int i = 0; i < 4; ++i) z[t][nh][i] = s[t][0][nh][i] + s[t][1][nh][i];
+  if (!(valid0 == kBlock && valid1 == kBlock && pos1 + kBlock - 1 <= st.lim_min)) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int valid = t ? valid1 : valid0;
+      const int pos = t ? pos1 : pos0;
+#pragma unroll
+      for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tok = r + 8 * (i >> 1);
+          if (!(tok < valid && pos + tok <= st.lim[nh][i & 1])) z[t][nh][i] = -INFINITY;
+        }
+    }
   }
-  // ---- running max per head column, lazy rescale ----
+  // ---- running max per head column (scaled by sc > 0 after the reduction), lazy rescale ----
   bool grow = false;
   float m_new[NH][2];
 #pragma unroll
@@ -333,27 +343,29 @@ __device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t*
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      m_new[nh][hc] = mx;
-      grow |= mx > st.m[nh][hc] + kRescaleSlack;
+      m_new[nh][hc] = mx * sc;
+      grow |= m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack;
     }
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
-        if (m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack) {
-          const float alpha = fast_exp2(st.m[nh][hc] - m_new[nh][hc]);  // 0 when m was -inf
-          st.m[nh][hc] = m_new[nh][hc];
-          st.l[nh][hc] *= alpha;
+        const bool up = m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack;
+        const float alpha = up ? fast_exp2(st.m[nh][hc] - m_new[nh][hc]) : 1.f;  // 0 from -inf
+        st.m[nh][hc] = up ? m_new[nh][hc] : st.m[nh][hc];
+        st.lsum[nh][hc] *= alpha;
+        st.lsum[nh][hc + 2] *= alpha;
 #pragma unroll
-          for (int mt = 0; mt < St::MT; ++mt) {
-            st.o[nh][mt][hc] *= alpha;
-            st.o[nh][mt][hc + 2] *= alpha;
-          }
+        for (int mt = 0; mt < St::MT; ++mt) {
+          st.o[nh][mt][hc] *= alpha;
+          st.o[nh][mt][hc + 2] *= alpha;
         }
       }
   }
-  // ---- P = exp2(z - m) in bf16, transposed into B fragments ----
+  // ---- P = exp2(z sc - m) in bf16, transposed into B fragments; l += ones . P^T ----
+  constexpr uint32_t kOnes = 0x3f803f80u;  // bf16x2 (1, 1)
+  const uint32_t ones[4] = {kOnes, kOnes, kOnes, kOnes};
   uint32_t pb[2][NH][2];
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh) {
@@ -361,12 +373,13 @@ __device__ __forceinline__ void bf16_step(Bf16State<D, GMAX>& st, const uint8_t*
     const float mu1 = st.m[nh][1] == -INFINITY ? 0.f : st.m[nh][1];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      const uint32_t lo = pack_bf16x2(fast_exp2(z[t][nh][0] - mu0), fast_exp2(z[t][nh][1] - mu1));
-      const uint32_t hi = pack_bf16x2(fast_exp2(z[t][nh][2] - mu0), fast_exp2(z[t][nh][3] - mu1));
-      st.l[nh][0] += bf16lo_to_f32(lo) + bf16lo_to_f32(hi);
-      st.l[nh][1] += bf16hi_to_f32(lo) + bf16hi_to_f32(hi);
+      const uint32_t lo = pack_bf16x2(fast_exp2(fmaf(z[t][nh][0], sc, -mu0)),
+                                      fast_exp2(fmaf(z[t][nh][1], sc, -mu1)));
+      const uint32_t hi = pack_bf16x2(fast_exp2(fmaf(z[t][nh][2], sc, -mu0)),
+                                      fast_exp2(fmaf(z[t][nh][3], sc, -mu1)));
       pb[t][nh][0] = movmatrix_trans(lo);
       pb[t][nh][1] = movmatrix_trans(hi);
+      mma_bf16_16816(st.lsum[nh], ones, pb[t][nh][0], pb[t][nh][1]);
     }
   }
   // ---- O^T += V^T P^T ----
@@ -417,10 +430,7 @@ __device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot
   for (int nh = 0; nh < St::NH; ++nh)
 #pragma unroll
     for (int hc = 0; hc < 2; ++hc) {
-      float l = st.l[nh][hc];
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      const float l = st.lsum[nh][hc];  // every row of the ones-MMA holds the full sum
       const int head = nh * 8 + qd + hc;
       if (head < g) {
 #pragma unroll
@@ -441,20 +451,24 @@ __device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot
 // Tiles hold one-byte codes [16 tokens][128 d].  K fragments come from
 // ldmatrix on 16-bit units, so a lane holds four consecutive d-values of a
 // token; the k-order of S^T = K Q^T is permuted to match (k-slots 2q, 2q+1,
-// 2q+8, 2q+9 of a 16-wide step are d 4q .. 4q+3 of that step) and Q's
-// fragments are built in the same order.  V fragments come from
+// 2q+8, 2q+9 of a 16-wide step are d 4q, 4q+1, 4q+2, 4q+3 of that step) and
+// Q's fragments are built in the same order.  V fragments come from
 // ldmatrix.trans on 16-bit units (pairs of d-values); a byte permute splits
 // the pairs, so row r of an output m-tile is d = 16mt + 2r and row r+8 is
 // d = 16mt + 2r + 1.  Codes become f16 exactly (cvt.f16x2.e4m3x2); the K
 // scale is folded into the score scale and the V scale into the output.
+// (The e4m3 m16n8k32 MMA straight on the codes, with q split into two e4m3
+// terms, was measured slower here: more issued instructions per tile.)
 template <int GMAX>
 struct Fp8State {
   static constexpr int D = 128;
   static constexpr int KS = 8, MT = 8, NH = GMAX / 8;
   uint32_t qb[NH][KS][2];  // f16 B fragments of Q^T in the permuted k-order
   float o[NH][MT][4];
-  float m[NH][2], l[NH][2];
+  float m[NH][2];          // running max of the scaled scores (log2 units)
+  float lsum[NH][4];       // running sums of P, accumulated by a tensor-core MMA
   int32_t lim[NH][2];
+  int32_t lim_min;         // smallest limit over the item's rows
 };
 
 template <int GMAX>
@@ -486,8 +500,9 @@ __device__ __forceinline__ void fp8_begin_item(Fp8State<GMAX>& st, const uint8_t
       st.o[nh][mt][0] = st.o[nh][mt][1] = st.o[nh][mt][2] = st.o[nh][mt][3] = 0.f;
     }
     st.m[nh][0] = st.m[nh][1] = -INFINITY;
-    st.l[nh][0] = st.l[nh][1] = 0.f;
+    st.lsum[nh][0] = st.lsum[nh][1] = st.lsum[nh][2] = st.lsum[nh][3] = 0.f;
   }
+  st.lim_min = len - q_len;
 }
 
 template <int GMAX>
@@ -502,80 +517,81 @@ __device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
   // 16-23 tokens 0-7 / 2p+1, 24-31 tokens 8-15 / 2p+1 (a granule = 16 codes).
   const uint32_t tok = ((lane >> 3) & 1) * 8 + (lane & 7);
   const uint32_t gsel = lane >> 4;
-  // ---- S^T = K Q^T ----
-  float s[2][2][NH][4];
+  // ---- S^T = K Q^T, one accumulation chain per tile ----
+  float s[2][NH][4];
 #pragma unroll
   for (int t = 0; t < 2; ++t)
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
+    for (int nh = 0; nh < NH; ++nh) s[t][nh][0] = s[t][nh][1] = s[t][nh][2] = s[t][nh][3] = 0.f;
 #pragma unroll
-      for (int nh = 0; nh < NH; ++nh) s[t][c][nh][0] = s[t][c][nh][1] = s[t][c][nh][2] = s[t][c][nh][3] = 0.f;
+  for (int kp = 0; kp < St::KS / 2; ++kp) {
+    const uint32_t off = ((((kp * 2) + gsel) ^ (tok & 7u)) << 4);
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const uint32_t base = smem_addr(t ? k1 : k0) + tok * 128u;
-#pragma unroll
-    for (int kp = 0; kp < St::KS / 2; ++kp) {
-      const uint32_t off = ((((kp * 2) + gsel) ^ (tok & 7u)) << 4);
+    for (int t = 0; t < 2; ++t) {
       uint32_t m0, m1, m2, m3;
-      ldmatrix_x4(base + off, m0, m1, m2, m3);
-      const uint32_t a_lo[4] = {e4m3x2_to_f16x2(m0), e4m3x2_to_f16x2(m1),
-                                e4m3x2_to_f16x2(m0 >> 16), e4m3x2_to_f16x2(m1 >> 16)};
-      const uint32_t a_hi[4] = {e4m3x2_to_f16x2(m2), e4m3x2_to_f16x2(m3),
-                                e4m3x2_to_f16x2(m2 >> 16), e4m3x2_to_f16x2(m3 >> 16)};
+      ldmatrix_x4(smem_addr(t ? k1 : k0) + tok * 128u + off, m0, m1, m2, m3);
+      uint32_t a_lo[4], a_hi[4];
+      e4m3x4_to_f16x2x2(m0, a_lo[0], a_lo[2]);
+      e4m3x4_to_f16x2x2(m1, a_lo[1], a_lo[3]);
+      e4m3x4_to_f16x2x2(m2, a_hi[0], a_hi[2]);
+      e4m3x4_to_f16x2x2(m3, a_hi[1], a_hi[3]);
 #pragma unroll
       for (int nh = 0; nh < NH; ++nh) {
-        mma_f16_16816(s[t][0][nh], a_lo, st.qb[nh][2 * kp][0], st.qb[nh][2 * kp][1]);
-        mma_f16_16816(s[t][1][nh], a_hi, st.qb[nh][2 * kp + 1][0], st.qb[nh][2 * kp + 1][1]);
+        mma_f16_16816(s[t][nh], a_lo, st.qb[nh][2 * kp][0], st.qb[nh][2 * kp][1]);
+        mma_f16_16816(s[t][nh], a_hi, st.qb[nh][2 * kp + 1][0], st.qb[nh][2 * kp + 1][1]);
       }
     }
   }
-  // ---- scale and mask; element i of a C fragment is token r + 8(i>>1), row 2q + (i&1) ----
-  float z[2][NH][4];
+  // ---- mask (raw scores; element i of a C fragment is token r + 8(i>>1), row 2q + (i&1)).
+  // Tiles that are full and wholly inside every row's causal window need no mask.
+  if (!(valid0 == kBlock && valid1 == kBlock && pos1 + kBlock - 1 <= st.lim_min)) {
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int valid = t ? valid1 : valid0;
-    const int pos = t ? pos1 : pos0;
+    for (int t = 0; t < 2; ++t) {
+      const int valid = t ? valid1 : valid0;
+      const int pos = t ? pos1 : pos0;
 #pragma unroll
-    for (int nh = 0; nh < NH; ++nh)
+      for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int tk = r + 8 * (i >> 1);
-        const float v = (s[t][0][nh][i] + s[t][1][nh][i]) * sc;
-        z[t][nh][i] = (tk < valid && pos + tk <= st.lim[nh][i & 1]) ? v : -INFINITY;
-      }
+        for (int i = 0; i < 4; ++i) {
+          const int tk = r + 8 * (i >> 1);
+          if (!(tk < valid && pos + tk <= st.lim[nh][i & 1])) s[t][nh][i] = -INFINITY;
+        }
+    }
   }
-  // ---- running max, lazy rescale (as for bf16) ----
+  // ---- running max (scaled by sc > 0 after the reduction), lazy rescale ----
   bool grow = false;
   float m_new[NH][2];
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
     for (int hc = 0; hc < 2; ++hc) {
-      float mx = fmaxf(fmaxf(z[0][nh][hc], z[0][nh][hc + 2]), fmaxf(z[1][nh][hc], z[1][nh][hc + 2]));
+      float mx = fmaxf(fmaxf(s[0][nh][hc], s[0][nh][hc + 2]), fmaxf(s[1][nh][hc], s[1][nh][hc + 2]));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      m_new[nh][hc] = mx;
-      grow |= mx > st.m[nh][hc] + kRescaleSlack;
+      m_new[nh][hc] = mx * sc;
+      grow |= m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack;
     }
   if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
     for (int nh = 0; nh < NH; ++nh)
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
-        if (m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack) {
-          const float alpha = fast_exp2(st.m[nh][hc] - m_new[nh][hc]);
-          st.m[nh][hc] = m_new[nh][hc];
-          st.l[nh][hc] *= alpha;
+        const bool up = m_new[nh][hc] > st.m[nh][hc] + kRescaleSlack;
+        const float alpha = up ? fast_exp2(st.m[nh][hc] - m_new[nh][hc]) : 1.f;  // 0 from -inf
+        st.m[nh][hc] = up ? m_new[nh][hc] : st.m[nh][hc];
+        st.lsum[nh][hc] *= alpha;
+        st.lsum[nh][hc + 2] *= alpha;
 #pragma unroll
-          for (int mt = 0; mt < St::MT; ++mt) {
-            st.o[nh][mt][hc] *= alpha;
-            st.o[nh][mt][hc + 2] *= alpha;
-          }
+        for (int mt = 0; mt < St::MT; ++mt) {
+          st.o[nh][mt][hc] *= alpha;
+          st.o[nh][mt][hc + 2] *= alpha;
         }
       }
   }
-  // ---- P = exp2(z - m) in f16, transposed into B fragments ----
+  // ---- P = exp2(s sc - m) in f16, transposed into B fragments; l += ones . P^T ----
+  constexpr uint32_t kOnes = 0x3c003c00u;  // f16x2 (1, 1)
+  const uint32_t ones[4] = {kOnes, kOnes, kOnes, kOnes};
   uint32_t pb[2][NH][2];
 #pragma unroll
   for (int nh = 0; nh < NH; ++nh) {
@@ -583,12 +599,13 @@ __device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
     const float mu1 = st.m[nh][1] == -INFINITY ? 0.f : st.m[nh][1];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      const uint32_t lo = pack_f16x2(fast_exp2(z[t][nh][0] - mu0), fast_exp2(z[t][nh][1] - mu1));
-      const uint32_t hi = pack_f16x2(fast_exp2(z[t][nh][2] - mu0), fast_exp2(z[t][nh][3] - mu1));
-      st.l[nh][0] += f16lo_to_f32(lo) + f16lo_to_f32(hi);
-      st.l[nh][1] += f16hi_to_f32(lo) + f16hi_to_f32(hi);
+      const uint32_t lo = pack_f16x2(fast_exp2(fmaf(s[t][nh][0], sc, -mu0)),
+                                     fast_exp2(fmaf(s[t][nh][1], sc, -mu1)));
+      const uint32_t hi = pack_f16x2(fast_exp2(fmaf(s[t][nh][2], sc, -mu0)),
+                                     fast_exp2(fmaf(s[t][nh][3], sc, -mu1)));
       pb[t][nh][0] = movmatrix_trans(lo);
       pb[t][nh][1] = movmatrix_trans(hi);
+      mma_f16_16816(st.lsum[nh], ones, pb[t][nh][0], pb[t][nh][1]);
     }
   }
   // ---- O^T += V^T P^T (m-tile rows interleave d: r -> 2r, r+8 -> 2r+1) ----
@@ -612,8 +629,9 @@ __device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
       for (int hlf = 0; hlf < 2; ++hlf) {
         const uint32_t ya = __byte_perm(hlf ? m2 : m0, 0u, 0x3120u);
         const uint32_t yb = __byte_perm(hlf ? m3 : m1, 0u, 0x3120u);
-        uint32_t a[4] = {e4m3x2_to_f16x2(ya), e4m3x2_to_f16x2(ya >> 16),
-                         e4m3x2_to_f16x2(yb), e4m3x2_to_f16x2(yb >> 16)};
+        uint32_t a[4];
+        e4m3x4_to_f16x2x2(ya, a[0], a[1]);
+        e4m3x4_to_f16x2x2(yb, a[2], a[3]);
         if (partial) {
           a[0] &= mk0;
           a[1] &= mk0;
@@ -639,10 +657,6 @@ __device__ __forceinline__ void fp8_publish(Fp8State<GMAX>& st, float* slot, int
   for (int nh = 0; nh < St::NH; ++nh)
 #pragma unroll
     for (int hc = 0; hc < 2; ++hc) {
-      float l = st.l[nh][hc];
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
       const int row = nh * 8 + qd + hc;
       if (row < rows) {
 #pragma unroll
@@ -652,7 +666,7 @@ __device__ __forceinline__ void fp8_publish(Fp8State<GMAX>& st, float* slot, int
         }
         if (r == 0) {
           M[row] = st.m[nh][hc];
-          L[row] = l;
+          L[row] = st.lsum[nh][hc];  // every row of the ones-MMA holds the full sum
         }
       }
     }

@@ -243,6 +243,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
   return r;
 }
 
+// Four e4m3 codes to two f16x2 (exact): bytes 0, 1 to `lo`, bytes 2, 3 to `hi`.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t v, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(v));
+}
+
 // Two floats to e4m3x2 codes (round to nearest even, saturating to +-448);
 // `lo` in the low byte of the result.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
