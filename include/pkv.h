@@ -172,6 +172,7 @@ pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_ca
  * is clamped, and a chunk reaching outside rows [0, num_q_tokens) is skipped;
  * both are flagged PKV_DEVERR_LEN.  With n = 1 everywhere this is
  * pkv_paged_attention_decode.  Workspace: pkv_multi_workspace_bytes().
+ * bf16 and fp32 pools only: FP8 pools return PKV_ERR_UNSUPPORTED.
  */
 size_t pkv_multi_workspace_bytes(const pkv_dims *dims, int32_t num_q_tokens,
                                  int32_t max_context_len, int32_t partition_tokens);

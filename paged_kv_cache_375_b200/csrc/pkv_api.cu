@@ -220,29 +220,34 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d
 }
 
 // Kernel configuration: W decode warps per CTA (one CTA per SM), S tile
-// stages per warp, MB merge buffers.  Eight decode warps with two stages each
-// hide the latency of the per-tile math best (measured on B200).  With 16
-// query rows per kv head at head_dim 128 a second merge buffer does not fit,
-// so that case keeps one.  fp32 tiles are twice as large: four warps.
+// stages per stage set, MB merge buffers, SPLIT warps reading each stage set
+// (W / SPLIT sets).  Eight decode warps with two stages each hide the latency
+// of the per-tile math best (measured on B200).  With 16 query rows per kv
+// head at head_dim 128 one warp's state does not fit its registers and a
+// second merge buffer does not fit shared memory: fourteen warps in pairs,
+// each pair sharing the stages of one set and taking 8 rows apiece, one merge
+// buffer (15 warps with the scheduler keep 128 registers per thread: at most
+// four warps per SM sub-partition).  fp32 tiles are twice as large: four warps.
 template <typename T, int D, int GMAX>
 struct DecodeCfg {
-  static constexpr int W = 8, S = 2, MB = (D == 128 && GMAX == 16) ? 1 : 2;
+  static constexpr bool kPairs = D == 128 && GMAX == 16;
+  static constexpr int W = kPairs ? 14 : 8, S = 2, MB = kPairs ? 1 : 2, SPLIT = kPairs ? 2 : 1;
 };
 template <int D, int GMAX>
 struct DecodeCfg<float, D, GMAX> {
-  static constexpr int W = 4, S = 2, MB = (D == 128 && GMAX == 16) ? 1 : 2;
+  static constexpr int W = 4, S = 2, MB = (D == 128 && GMAX == 16) ? 1 : 2, SPLIT = 1;
 };
 // FP8 tiles carry half the bytes of bf16 ones for the same math (plus the
 // code conversions), so the kernel is bound by per-tile latency rather than
 // by HBM: more decode warps hide more of it.  Up to 8 query rows the state
 // fits 128 registers and 15 decode warps run (one merge buffer to fit shared
-// memory); with 16 rows 11 warps at 168 registers (measured on B200: 15
+// memory); with 16 rows 14 warps in pairs as above (measured on B200: 15
 // warps 4.49 TB/s, 11 warps 4.25, 8 warps with 4 stages 3.78 on the
-// Llama-3-8B-shaped batch).  Two stages per warp keep 88-120 KB per SM in
+// Llama-3-8B-shaped batch).  Two stages per warp keep 56-120 KB per SM in
 // flight.
 template <int D, int GMAX>
 struct DecodeCfg<pkv::Fp8Kv, D, GMAX> {
-  static constexpr int W = GMAX == 16 ? 11 : 15, S = 2, MB = 1;
+  static constexpr int W = GMAX == 16 ? 14 : 15, S = 2, MB = 1, SPLIT = GMAX == 16 ? 2 : 1;
 };
 
 // Largest dynamic shared memory already enabled per kernel, per device.
@@ -277,8 +282,8 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
                          const pkv::DecodeParams& prm, int64_t work_units, int rows_max,
                          cudaStream_t stream) {
   constexpr int W = DecodeCfg<T, D, GMAX>::W, S = DecodeCfg<T, D, GMAX>::S;
-  constexpr int MB = DecodeCfg<T, D, GMAX>::MB;
-  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S, MB, pkv::q_elem_bytes<T>()>;
+  constexpr int MB = DecodeCfg<T, D, GMAX>::MB, SPLIT = DecodeCfg<T, D, GMAX>::SPLIT;
+  using Lay = pkv::DecodeLayout<sizeof(T), D, GMAX, W, S, MB, pkv::q_elem_bytes<T>(), SPLIT>;
   const int smem = Lay::total_bytes(rows_max);
   int dev = 0, max_optin = 0;
   cudaGetDevice(&dev);
@@ -286,7 +291,7 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
   if (smem > max_optin)
     return fail(PKV_ERR_UNSUPPORTED, "decode needs %d bytes of shared memory (> %d)", smem,
                 max_optin);
-  auto kern = pkv::decode_kernel<T, D, GMAX, W, S, MB>;
+  auto kern = pkv::decode_kernel<T, D, GMAX, W, S, MB, SPLIT>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
   int per_sm = 0;
@@ -549,6 +554,8 @@ pkv_status pkv_multi_run(void* out, const void* q, const void* k_cache, const vo
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
   if (st != PKV_OK) return st;
+  if (dims->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "several query tokens per sequence need bf16 or fp32 pools");
   if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
   if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
   return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
@@ -566,6 +573,8 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
   if (st != PKV_OK) return st;
+  if (dims->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_UNSUPPORTED, "several query tokens per sequence need bf16 or fp32 pools");
   if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
   if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
   if (max_query_len < 1 || (max_query_len * (dims->num_q_heads / dims->num_kv_heads)) > 16)

@@ -159,7 +159,10 @@ __global__ void __launch_bounds__(32)
   mbar_arrive_expect_tx(&bar, bytes);
   bulk_load(buf, cache + src * block_bytes + off, bytes, &bar);
   if (!mbar_wait(&bar, 0)) {
-    return;  // timeout already flagged; nothing was issued after the load
+    // Timeout (flagged).  Give the load a last, shorter bound to land before
+    // this CTA's shared memory is released; nothing was issued after it.
+    mbar_wait(&bar, 0, kDrainLimitCycles);
+    return;
   }
   fence_proxy_async_smem();
   bulk_store(cache + dst * block_bytes + off, buf, bytes);

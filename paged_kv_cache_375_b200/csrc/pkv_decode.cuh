@@ -183,28 +183,39 @@ constexpr int kMaxItemBlocks = 512;
 // MB merge buffers: with two, consecutive items alternate buffers and one
 // barrier per item suffices; with one (when two do not fit), a second
 // barrier keeps the next item's states out until the current one is combined.
-template <int ELEM, int D, int GMAX, int W, int S, int MB = 2, int QELEM = ELEM>
+// SPLIT warps share one set of tile stages, each taking GMAX / SPLIT of an
+// item's query rows; W / SPLIT "lead" warps own the stages and issue the loads.
+template <int ELEM, int D, int GMAX, int W, int S, int MB = 2, int QELEM = ELEM, int SPLIT = 1>
 struct DecodeLayout {
+  static constexpr int kLead = W / SPLIT;                     // warps owning stages
+  static constexpr int kRowsPerWarp = GMAX / SPLIT;           // query rows one warp holds
   static constexpr int kTileBytes = kBlock * D * ELEM;       // one K (or V) tile
   static constexpr int kChunks = D * ELEM / 128;             // 128-byte column chunks
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kQBytes = ((GMAX * D * QELEM) + 127) / 128 * 128;
   static constexpr int kStagesOff = 0;
-  static constexpr int kRingOff = kStagesOff + W * S * kStageBytes;
+  static constexpr int kRingOff = kStagesOff + kLead * S * kStageBytes;
   static constexpr int kTablesOff = kRingOff + kRing * kQBytes;
   static constexpr int kMergeOff = kTablesOff + kRing * kMaxItemBlocks * 4;
-  // merge area: 2 buffers x W warps x (g*D + 2g rounded up to 4) floats, g
-  // chosen at run time; every warp's slot starts 16-byte aligned.
-  __host__ __device__ static int merge_floats_per_warp(int g) { return g * D + (2 * g + 3) / 4 * 4; }
-  __host__ __device__ static int meta_off(int g) {
-    return kMergeOff + MB * W * merge_floats_per_warp(g) * 4;
+  // Rows of a warp's merge slot when the largest item has rows_max rows.
+  __host__ __device__ static int slot_rows(int rows_max) {
+    return rows_max < kRowsPerWarp ? rows_max : kRowsPerWarp;
+  }
+  // merge area: MB buffers x W warps x (r*D + 2r rounded up to 4) floats for
+  // r slot rows; every warp's slot starts 16-byte aligned.
+  __host__ __device__ static int merge_floats_per_warp(int r) { return r * D + (2 * r + 3) / 4 * 4; }
+  __host__ __device__ static int meta_off(int rows_max) {
+    return kMergeOff + MB * W * merge_floats_per_warp(slot_rows(rows_max)) * 4;
   }
   static constexpr int kMetaBytes = kRing * 64;
-  __host__ __device__ static int bars_off(int g) { return (meta_off(g) + kMetaBytes + 7) / 8 * 8; }
-  static constexpr int kNumBars = W * S + 2 * kRing + 2;
-  __host__ __device__ static int flags_off(int g) { return bars_off(g) + kNumBars * 8; }
-  __host__ __device__ static int total_bytes(int g) {
-    return flags_off(g) + (W * S + 4) * 4 + 1024;  // + slack for 1024-byte alignment
+  __host__ __device__ static int bars_off(int rows_max) {
+    return (meta_off(rows_max) + kMetaBytes + 7) / 8 * 8;
+  }
+  // full[kLead][S], empty[kLead][S], item_full[kRing], item_empty[kRing], merge[2]
+  static constexpr int kNumBars = 2 * kLead * S + 2 * kRing + 2;
+  __host__ __device__ static int flags_off(int rows_max) { return bars_off(rows_max) + kNumBars * 8; }
+  __host__ __device__ static int total_bytes(int rows_max) {
+    return flags_off(rows_max) + (kLead * S + 4) * 4 + 1024;  // + slack for 1024-byte alignment
   }
 };
 
@@ -241,9 +252,12 @@ struct Bf16State {
 
 // Query rows of an item: row n = i*g + h is chunk token i (at position
 // len - q_len + i) and query head h of the group; `rows` = q_len * g.
+// A warp holding rows row0 .. row0 + rows - 1 of the item gets qs pointing at
+// row row0.
 template <int D, int GMAX>
 __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const uint8_t* qs,
-                                                int rows, int g, int len, int q_len, int lane) {
+                                                int rows, int g, int len, int q_len, int lane,
+                                                int row0 = 0) {
   using St = Bf16State<D, GMAX>;
   const int r = lane >> 2, qd = (lane & 3) * 2;
   const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qs);
@@ -259,7 +273,7 @@ __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const ui
 #pragma unroll
     for (int hc = 0; hc < 2; ++hc) {
       const int n = nh * 8 + qd + hc;
-      st.lim[nh][hc] = n < rows ? len - q_len + n / g : -1;
+      st.lim[nh][hc] = n < rows ? len - q_len + (row0 + n) / g : -1;
     }
 #pragma unroll
     for (int mt = 0; mt < St::MT; ++mt) {
@@ -268,7 +282,7 @@ __device__ __forceinline__ void bf16_begin_item(Bf16State<D, GMAX>& st, const ui
     st.m[nh][0] = st.m[nh][1] = -INFINITY;
     st.lsum[nh][0] = st.lsum[nh][1] = st.lsum[nh][2] = st.lsum[nh][3] = 0.f;
   }
-  st.lim_min = len - q_len;
+  st.lim_min = len - q_len + row0 / g;
 }
 
 // Two 16-token tiles (the second may be absent: valid1 = 0 and its pointers
@@ -473,7 +487,8 @@ struct Fp8State {
 
 template <int GMAX>
 __device__ __forceinline__ void fp8_begin_item(Fp8State<GMAX>& st, const uint8_t* qs, int rows,
-                                               int g, int len, int q_len, int lane) {
+                                               int g, int len, int q_len, int lane,
+                                               int row0 = 0) {
   using St = Fp8State<GMAX>;
   const int r = lane >> 2, q4 = (lane & 3) * 4, qd = (lane & 3) * 2;
   const uint16_t* q16 = reinterpret_cast<const uint16_t*>(qs);  // bf16 rows of 128
@@ -493,7 +508,7 @@ __device__ __forceinline__ void fp8_begin_item(Fp8State<GMAX>& st, const uint8_t
 #pragma unroll
     for (int hc = 0; hc < 2; ++hc) {
       const int n = nh * 8 + qd + hc;
-      st.lim[nh][hc] = n < rows ? len - q_len + n / g : -1;
+      st.lim[nh][hc] = n < rows ? len - q_len + (row0 + n) / g : -1;
     }
 #pragma unroll
     for (int mt = 0; mt < St::MT; ++mt) {
@@ -502,7 +517,7 @@ __device__ __forceinline__ void fp8_begin_item(Fp8State<GMAX>& st, const uint8_t
     st.m[nh][0] = st.m[nh][1] = -INFINITY;
     st.lsum[nh][0] = st.lsum[nh][1] = st.lsum[nh][2] = st.lsum[nh][3] = 0.f;
   }
-  st.lim_min = len - q_len;
+  st.lim_min = len - q_len + row0 / g;
 }
 
 template <int GMAX>
@@ -781,28 +796,36 @@ __device__ __forceinline__ void f32_publish(F32State<D, GMAX>& st, float* slot, 
   }
 }
 
-// ---- combine the W warps' states of one item and store the result ----
-// The item's `rows` rows are chunk token i = n / group, head n % group.
-template <typename T, int D, int W>
+// ---- combine the warps' states of one item and store the result ----
+// The item's `rows` rows are chunk token i = n / group, head n % group.  Row
+// n's states sit in the slots of the L = W / SPLIT warps holding it (row
+// n - RPW*half of the warps half*L .. half*L + L - 1, half = n / RPW), each
+// slot laid out as [rh rows x D outputs][rh maxima][rh sums], rh = the rows
+// that half holds.
+template <typename T, int D, int W, int SPLIT, int RPW>
 __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const ItemMeta& it,
                                                   const float* merge, int per_warp, int rows,
                                                   int warp, int lane) {
+  constexpr int L = W / SPLIT;
   const int tid = warp * 32 + lane;
-  const int g = rows;  // merge-slot layout: rows x D outputs, then rows maxima and sums
   for (int e = tid * 4; e < rows * D; e += W * 32 * 4) {
     const int h = e / D, d = e % D;
+    const int half = SPLIT == 1 ? 0 : h / RPW;
+    const int local = h - half * RPW;
+    const int rh = SPLIT == 1 ? rows : (rows - half * RPW < RPW ? rows - half * RPW : RPW);
+    const float* base = merge + half * L * per_warp;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < W; ++w) M = fmaxf(M, merge[w * per_warp + g * D + h]);
+    for (int w = 0; w < L; ++w) M = fmaxf(M, base[w * per_warp + rh * D + local]);
     float lsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        const float* slot = merge + w * per_warp;
-        const float f = exp2f(slot[g * D + h] - M);
-        lsum = fmaf(slot[g * D + g + h], f, lsum);
-        const float4 ov = *reinterpret_cast<const float4*>(slot + h * D + d);
+      for (int w = 0; w < L; ++w) {
+        const float* slot = base + w * per_warp;
+        const float f = exp2f(slot[rh * D + local] - M);
+        lsum = fmaf(slot[rh * D + rh + local], f, lsum);
+        const float4 ov = *reinterpret_cast<const float4*>(slot + local * D + d);
         acc.x = fmaf(ov.x, f, acc.x);
         acc.y = fmaf(ov.y, f, acc.y);
         acc.z = fmaf(ov.z, f, acc.z);
@@ -839,18 +862,24 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
 //
 // The scheduler warp fetches items from the global work counter and
 // publishes each into a ring slot: its metadata, its q tile (one bulk copy)
-// and the slice of the block table it covers.  Every decode warp owns S tile
-// stages and is its own TMA producer: it keeps up to S of its blocks in
-// flight, following its share of the items (blocks w, w+W, ... of each) and
-// running ahead into the next items while it computes.  At the end of an item
+// and the slice of the block table it covers.  Every lead decode warp (the
+// first W / SPLIT) owns S tile stages and is its own TMA producer: it keeps up
+// to S of its blocks in flight, following its share of the items (blocks l,
+// l+L, ... of each, L = W / SPLIT) and running ahead into the next items
+// while it computes.  With SPLIT = 2 a second warp reads the same stages and
+// takes the item's upper query rows; a stage is refilled once both warps have
+// released it (an "empty" barrier with two arrivals).  At the end of an item
 // the W warps combine their online-softmax states through shared memory.
-template <typename T, int D, int GMAX, int W, int S, int MB>
+template <typename T, int D, int GMAX, int W, int S, int MB, int SPLIT>
 __global__ void __launch_bounds__((W + 1) * 32, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
   constexpr int ELEM = sizeof(T);            // cache bytes per element (1 for FP8)
   constexpr int QELEM = q_elem_bytes<T>();   // q bytes per element
-  using Lay = DecodeLayout<ELEM, D, GMAX, W, S, MB, QELEM>;
+  using Lay = DecodeLayout<ELEM, D, GMAX, W, S, MB, QELEM, SPLIT>;
+  constexpr int L = Lay::kLead;              // warps owning stages
+  constexpr int RPW = Lay::kRowsPerWarp;     // query rows per warp
+  static_assert(SPLIT == 1 || (SPLIT == 2 && GMAX == 16 && W % 2 == 0), "row split: 2 x 8 rows");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -862,16 +891,20 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   float* merge = reinterpret_cast<float*>(smem + Lay::kMergeOff);
   ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + Lay::meta_off(rows_max));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::bars_off(rows_max));
-  uint64_t* full = bars;                       // [W][S]
-  uint64_t* item_full = bars + W * S;          // [kRing]
+  uint64_t* full = bars;                       // [L][S]
+  uint64_t* empty = full + L * S;              // [L][S] (SPLIT > 1 only)
+  uint64_t* item_full = empty + L * S;         // [kRing]
   uint64_t* item_empty = item_full + kRing;    // [kRing]
   uint64_t* merge_bar = item_empty + kRing;    // [2]
-  uint32_t* stage_ok = reinterpret_cast<uint32_t*>(smem + Lay::flags_off(rows_max));  // [W][S]
-  volatile uint32_t* abort_flag = stage_ok + W * S;
+  uint32_t* stage_ok = reinterpret_cast<uint32_t*>(smem + Lay::flags_off(rows_max));  // [L][S]
+  volatile uint32_t* abort_flag = stage_ok + L * S;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < W * S; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < L * S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], SPLIT);
+    }
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&item_full[i], 1);
       mbar_init(&item_empty[i], W);
@@ -984,29 +1017,34 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   }
 
   // ================================ decode warps ================================
-  using Bst = Bf16State<D, GMAX>;
+  using Bst = Bf16State<D, RPW>;
   using Fst = F32State<D, GMAX>;
   constexpr bool kFp8 = std::is_same<T, Fp8Kv>::value;
   constexpr bool kBf16 = sizeof(T) == 2;
-  typename std::conditional<kFp8, Fp8State<GMAX>,
+  static_assert(SPLIT == 1 || kFp8 || kBf16, "row split needs the tensor-core states");
+  typename std::conditional<kFp8, Fp8State<RPW>,
                             typename std::conditional<kBf16, Bst, Fst>::type>::type st;
   const float sc = prm.qk_scale_log2;
-  const int per_warp = Lay::merge_floats_per_warp(rows_max);
-  uint64_t* my_full = full + warp * S;
-  uint32_t* my_ok = stage_ok + warp * S;
-  uint8_t* my_stages = stages + warp * S * Lay::kStageBytes;
+  const int per_warp = Lay::merge_floats_per_warp(Lay::slot_rows(rows_max));
+  const int lead = warp % L;         // the stage set this warp reads
+  const int half = warp / L;         // which RPW query rows of an item it holds
+  uint64_t* my_full = full + lead * S;
+  uint64_t* my_empty = empty + lead * S;
+  uint32_t* my_ok = stage_ok + lead * S;
+  uint8_t* my_stages = stages + lead * S * Lay::kStageBytes;
 
-  // Producer cursor over this warp's blocks: item p_item, block p_blk of it.
-  uint32_t cctr = 0, pctr = 0;       // blocks consumed / issued by this warp
+  // Producer cursor over this stage set's blocks: item p_item, block p_blk of it.
+  uint32_t cctr = 0, pctr = 0;       // blocks consumed by this warp / issued by its lead
   uint32_t c_item = 0;               // item being consumed
   uint32_t p_item = 0;
-  int32_t p_blk = warp;
+  int32_t p_blk = lead;
   bool p_known = false, p_end = false;
   ItemMeta pm{};
   bool ok = true;
 
-  // Issue this warp's next blocks until S are in flight.  With `blocking` the
-  // wait for an item's metadata may block (only when the block is needed now).
+  // Issue the stage set's next blocks until S are in flight (lead warps only).
+  // With `blocking` the waits for an item's metadata and for a stage's
+  // release may block (only when the block is needed now).
   auto produce = [&](bool blocking) {
     while (pctr < cctr + S && !p_end) {
       if (!p_known) {
@@ -1035,6 +1073,20 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         continue;
       }
       const int s_idx = pctr % S;
+      if constexpr (SPLIT > 1) {
+        // the stage's previous use must have been released by every warp reading it
+        if (pctr >= static_cast<uint32_t>(S)) {
+          const uint32_t par = ((pctr / S) - 1) & 1;
+          if (blocking) {
+            if (!mbar_wait(&my_empty[s_idx], par)) {
+              ok = false;
+              return;
+            }
+          } else if (!mbar_try_wait(&my_empty[s_idx], par)) {
+            return;
+          }
+        }
+      }
       const int32_t entry = tables[(p_item % kRing) * kMaxItemBlocks + p_blk];
       if (lane == 0) {
         const bool valid = entry >= 0 && entry < prm.num_blocks;
@@ -1054,7 +1106,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
           mbar_arrive(&my_full[s_idx]);
         }
       }
-      p_blk += W;
+      p_blk += L;
       ++pctr;
     }
   };
@@ -1069,18 +1121,23 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     if (it.seq < 0) break;
     const uint8_t* qs = ring + r * Lay::kQBytes;
     const int rows = it.q_len * g;  // query rows of this item
+    // this warp's rows: row0 .. row0 + my_rows - 1
+    const int row0 = half * RPW;
+    const int my_rows = SPLIT == 1 ? rows
+                                   : (rows - row0 < 0 ? 0 : (rows - row0 < RPW ? rows - row0 : RPW));
+    const uint8_t* my_qs = qs + row0 * D * QELEM;
     if constexpr (kFp8) {
-      fp8_begin_item<GMAX>(st, qs, rows, g, it.len, it.q_len, lane);
+      fp8_begin_item<RPW>(st, my_qs, my_rows, g, it.len, it.q_len, lane, row0);
     } else if constexpr (kBf16) {
-      bf16_begin_item<D, GMAX>(st, qs, rows, g, it.len, it.q_len, lane);
+      bf16_begin_item<D, RPW>(st, my_qs, my_rows, g, it.len, it.q_len, lane, row0);
     } else {
       f32_begin_item<D, GMAX>(st, rows, g, it.len, it.q_len);
     }
-    // bf16 consumes this warp's blocks two at a time (b and b + W), fp32 one at a time.
+    // bf16 consumes the blocks two at a time (b and b + L), fp32 one at a time.
     constexpr int kStep = (kBf16 || kFp8) ? 2 : 1;
-    for (int32_t b = warp; b < it.nblk; b += kStep * W) {
-      const int n = (kStep == 2 && b + W < it.nblk) ? 2 : 1;
-      if (pctr < cctr + n) {
+    for (int32_t b = lead; b < it.nblk; b += kStep * L) {
+      const int n = (kStep == 2 && b + L < it.nblk) ? 2 : 1;
+      if (half == 0 && pctr < cctr + n) {
         produce(true);
         if (!ok || pctr < cctr + n) {
           ok = false;
@@ -1096,31 +1153,39 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         if (x < n && !mbar_wait(&my_full[s_idx], (k / S) & 1)) ok = false;
         kt[x] = my_stages + s_idx * Lay::kStageBytes;
         if (x < n && my_ok[s_idx]) {
-          const int v = it.len - (it.blk_begin + b + x * W) * kBlock;
+          const int v = it.len - (it.blk_begin + b + x * L) * kBlock;
           valid[x] = v > kBlock ? kBlock : v;
         }
       }
       if (!ok) break;
       const int pos0 = (it.blk_begin + b) * kBlock;  // position of the first tile's token 0
       if constexpr (kFp8) {
-        fp8_step<GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
-                       kt[1] + Lay::kTileBytes, valid[1], pos0 + W * kBlock, sc, lane);
+        if (my_rows > 0)
+          fp8_step<RPW>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
+                        kt[1] + Lay::kTileBytes, valid[1], pos0 + L * kBlock, sc, lane);
       } else if constexpr (kBf16) {
-        bf16_step<D, GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
-                           kt[1] + Lay::kTileBytes, valid[1], pos0 + W * kBlock, sc, lane);
+        if (my_rows > 0)
+          bf16_step<D, RPW>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
+                            kt[1] + Lay::kTileBytes, valid[1], pos0 + L * kBlock, sc, lane);
       } else {
         f32_block<D, GMAX>(st, reinterpret_cast<const float*>(qs), kt[0], kt[0] + Lay::kTileBytes,
                            valid[0], pos0, sc, rows, lane);
       }
       __syncwarp();
+      if constexpr (SPLIT > 1) {
+        // release the stages to the lead (it refills them once every reader has)
+        if (lane == 0) {
+          for (int x = 0; x < n; ++x) mbar_arrive(&my_empty[(cctr + x) % S]);
+        }
+      }
       cctr += n;
-      produce(false);
+      if (half == 0) produce(false);
     }
     if (!ok) break;
     // The q tile, metadata and table slice of this item are no longer needed.
     __syncwarp();
     if (lane == 0) mbar_arrive(&item_empty[r]);
-    produce(false);
+    if (half == 0) produce(false);
     // ---- merge the W warps' states ----
     // two buffers: item c uses buffer c & 1 and merge_bar[c & 1];
     // one buffer: merge_bar[0] = states published, merge_bar[1] = combined.
@@ -1132,9 +1197,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
     }
     float* mslot = merge + (mb * W + warp) * per_warp;
     if constexpr (kFp8) {
-      fp8_publish<GMAX>(st, mslot, rows, lane);
+      fp8_publish<RPW>(st, mslot, my_rows, lane);
     } else if constexpr (kBf16) {
-      bf16_publish<D, GMAX>(st, mslot, rows, lane);
+      bf16_publish<D, RPW>(st, mslot, my_rows, lane);
     } else {
       f32_publish<D, GMAX>(st, mslot, rows, lane);
     }
@@ -1144,7 +1209,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
       ok = false;
       break;
     }
-    combine_and_store<T, D, W>(prm, it, merge + mb * W * per_warp, per_warp, rows, warp, lane);
+    combine_and_store<T, D, W, SPLIT, RPW>(prm, it, merge + mb * W * per_warp, per_warp, rows,
+                                           warp, lane);
     if constexpr (MB == 1) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&merge_bar[1]);

@@ -218,3 +218,19 @@ def test_c3_fp8_full_size_sampled(cuda_device):
                                   b.context_lens, b.scale, tasks=tasks, threads=8)
     got = out[torch.from_numpy(tasks[:, 0]).long(), torch.from_numpy(tasks[:, 1]).long()]
     check_close(got, ref, "bf16", "c3 fp8 sampled")
+
+
+def test_several_query_tokens_over_fp8_pools_are_rejected(cuda_device):
+    b = workloads.random_batch(980, [20, 30], 8, 2, 128, "fp8", device=cuda_device)
+    bt, cl = dev_i32(b.block_tables, b.q.device), dev_i32(b.context_lens, b.q.device)
+    qsl = torch.tensor([0, 1, 2], dtype=torch.int32, device=b.q.device)
+    out = torch.empty_like(b.q)
+    dims = pkv.make_dims(2, 8, b.k_cache, bt.shape[1])
+    lib = pkv.load_library()
+    need = lib.pkv_multi_workspace_bytes(pkv.ctypes.byref(dims), 2, 30, 0)
+    ws = torch.empty(need, dtype=torch.uint8, device=b.q.device)
+    st = lib.pkv_paged_attention_multi(
+        pkv._p(out), pkv._p(b.q), pkv._p(b.k_cache), pkv._p(b.v_cache), pkv._p(bt), pkv._p(cl),
+        pkv._p(qsl), 2, 1, b.scale, pkv.ctypes.byref(dims), 30, 0, pkv._p(ws), ws.numel(),
+        pkv._stream_ptr(b.q.device))
+    assert st == 3
