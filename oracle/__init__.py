@@ -86,12 +86,15 @@ def _load():
                                                     i32, i32, i64, i32, f32, P, i64, i32]
             lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i64,
                                                          f32, f32]
+            lib.oracle_paged_multi_fp8.argtypes = [P, P, P, P, f32, f32, P, P, P, i32, i32, i32,
+                                                   i32, i32, i64, i32, f32, i32]
             lib.oracle_e4m3_quantize.argtypes = [P, i64, f32, P]
             lib.oracle_e4m3_values.argtypes = [P, i64, P]
             lib.oracle_lse_merge_f32.argtypes = [P, P, P, i32, i32, P]
             for name in ("oracle_slot_mapping", "oracle_reshape_and_cache",
                          "oracle_copy_blocks", "oracle_paged_decode", "oracle_paged_multi",
                          "oracle_paged_decode_fp8", "oracle_reshape_and_cache_fp8",
+                         "oracle_paged_multi_fp8",
                          "oracle_e4m3_quantize", "oracle_e4m3_values",
                          "oracle_partition_stats", "oracle_lse_merge",
                          "oracle_lse_merge_f32"):
@@ -252,6 +255,27 @@ def paged_decode_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_
                                            float(k_scale), float(v_scale), _ptr(bt), _ptr(cl),
                                            B, Hq, Hkv, D, BS, NB, bt.shape[1], float(scale), tp,
                                            n, threads))
+    return out
+
+
+def paged_multi_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_scale: float,
+                    v_scale: float, block_tables: np.ndarray, context_lens: np.ndarray,
+                    query_start_loc: np.ndarray, scale: float,
+                    threads: int | None = None) -> np.ndarray:
+    """paged_multi over e4m3 pools (uint8 codes times the pool's scale); q is bf16 bits."""
+    assert q.dtype == np.uint16 and k_cache.dtype == np.uint8 == v_cache.dtype
+    T, Hq, D = q.shape
+    NB, Hkv, BS, _ = k_cache.shape
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+    assert qsl.shape[0] == cl.shape[0] + 1 and qsl[-1] <= T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    threads = threads or len(os.sched_getaffinity(0))
+    _check(_load().oracle_paged_multi_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                          float(k_scale), float(v_scale), _ptr(bt), _ptr(cl),
+                                          _ptr(qsl), cl.shape[0], Hq, Hkv, D, BS, NB,
+                                          bt.shape[1], float(scale), threads))
     return out
 
 

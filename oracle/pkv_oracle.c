@@ -646,6 +646,14 @@ static void *multi_worker(void *arg)
     return NULL;
 }
 
+static int paged_multi_scaled(double *out, const void *q, const void *k_cache,
+                              const void *v_cache, int32_t dtype, float k_scale, float v_scale,
+                              const int32_t *block_tables, const int32_t *context_lens,
+                              const int32_t *query_start_loc, int32_t num_seqs,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int64_t num_blocks,
+                              int32_t max_blocks_per_seq, float scale, int32_t num_threads);
+
 /* out: [num_q_tokens][num_q_heads][head_dim] doubles, q: [num_q_tokens][Hq][D]. */
 int oracle_paged_multi(double *out, const void *q, const void *k_cache, const void *v_cache,
                        int32_t dtype, const int32_t *block_tables, const int32_t *context_lens,
@@ -654,8 +662,40 @@ int oracle_paged_multi(double *out, const void *q, const void *k_cache, const vo
                        int64_t num_blocks, int32_t max_blocks_per_seq, float scale,
                        int32_t num_threads)
 {
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) {
+        return ORACLE_BAD_ARG;
+    }
+    return paged_multi_scaled(out, q, k_cache, v_cache, dtype, 1.0f, 1.0f, block_tables,
+                              context_lens, query_start_loc, num_seqs, num_q_heads, num_kv_heads,
+                              head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
+                              num_threads);
+}
+
+/* The same over FP8 (e4m3) pools: q is bf16; each cached element is its code's
+ * value times k_scale (K pool) or v_scale (V pool). */
+int oracle_paged_multi_fp8(double *out, const void *q, const void *k_cache, const void *v_cache,
+                           float k_scale, float v_scale, const int32_t *block_tables,
+                           const int32_t *context_lens, const int32_t *query_start_loc,
+                           int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                           int32_t max_blocks_per_seq, float scale, int32_t num_threads)
+{
+    return paged_multi_scaled(out, q, k_cache, v_cache, ORACLE_E4M3, k_scale, v_scale,
+                              block_tables, context_lens, query_start_loc, num_seqs, num_q_heads,
+                              num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                              scale, num_threads);
+}
+
+static int paged_multi_scaled(double *out, const void *q, const void *k_cache,
+                              const void *v_cache, int32_t dtype, float k_scale, float v_scale,
+                              const int32_t *block_tables, const int32_t *context_lens,
+                              const int32_t *query_start_loc, int32_t num_seqs,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int64_t num_blocks,
+                              int32_t max_blocks_per_seq, float scale, int32_t num_threads)
+{
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
-        !query_start_loc || (dtype != ORACLE_F32 && dtype != ORACLE_BF16) || num_seqs < 0 ||
+        !query_start_loc || num_seqs < 0 ||
         num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
         head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0) {
         return ORACLE_BAD_ARG;
@@ -667,7 +707,8 @@ int oracle_paged_multi(double *out, const void *q, const void *k_cache, const vo
     }
     problem pb = {q, k_cache, v_cache, dtype, block_tables, context_lens,
                   num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                  num_blocks, max_blocks_per_seq, (double)scale, 1.0, 1.0};
+                  num_blocks, max_blocks_per_seq, (double)scale, (double)k_scale,
+                  (double)v_scale};
     multi_pool mp = {&pb, query_start_loc, out, 0, ORACLE_OK};
     if (num_threads <= 1) {
         multi_worker(&mp);

@@ -564,6 +564,38 @@ def test_fp8_decode_matches_dense_attention_on_dequantised_values():
                                    atol=1e-12)
 
 
+def test_fp8_multi_matches_dense_causal_attention_on_dequantised_values():
+    """Several causal query tokens over FP8 pools: dense fp64 attention over the widened,
+    scaled codes, each chunk token seeing keys up to its own position; one-token chunks
+    equal FP8 decode."""
+    rng = np.random.default_rng(32)
+    lens, chunks = [4, 16, 33, 70], [4, 1, 5, 16]
+    hq, hkv, d = 8, 2, 32
+    _, kp32, vp32, bt, cl, _, _, _ = random_paged(rng, lens, hq, hkv, d)
+    k_scale, v_scale = np.float32(0.04), np.float32(0.03)
+    kc = oracle.e4m3_quantize(np.nan_to_num(kp32), k_scale)
+    vc = oracle.e4m3_quantize(np.nan_to_num(vp32), v_scale)
+    qsl = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    qb = to_bf16_bits(rng.standard_normal((int(qsl[-1]), hq, d)).astype(np.float32))
+    out = oracle.paged_multi_fp8(qb, kc, vc, k_scale, v_scale, bt, cl, qsl, 0.2)
+    qf = bf16_bits_to_f64(qb)
+    kd = oracle.e4m3_values(kc) * float(k_scale)
+    vd = oracle.e4m3_values(vc) * float(v_scale)
+    for s, (L, n) in enumerate(zip(lens, chunks)):
+        nb = (L + BS - 1) // BS
+        K = kd[bt[s, :nb]].transpose(0, 2, 1, 3).reshape(nb * BS, hkv, d)[:L]
+        V = vd[bt[s, :nb]].transpose(0, 2, 1, 3).reshape(nb * BS, hkv, d)[:L]
+        for i in range(n):
+            p = L - n + i
+            row = qsl[s] + i
+            np.testing.assert_allclose(out[row], dense_attention(qf[row], K[:p + 1], V[:p + 1],
+                                                                 0.2), rtol=0, atol=1e-12)
+    one = np.arange(len(lens) + 1, dtype=np.int32)
+    qd = np.ascontiguousarray(qb[:len(lens)])
+    assert np.array_equal(oracle.paged_multi_fp8(qd, kc, vc, k_scale, v_scale, bt, cl, one, 0.2),
+                          oracle.paged_decode_fp8(qd, kc, vc, k_scale, v_scale, bt, cl, 0.2))
+
+
 def test_fp8_reshape_quantises_into_the_slot():
     rng = np.random.default_rng(32)
     hkv, d, nb = 2, 64, 4
