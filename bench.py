@@ -44,7 +44,7 @@ METRIC = "paged decode attn: KV-read GB/s (% of B200 HBM peak), seqs/s at batch"
 UNIT = "GB/s"
 WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shared_prefix",
              "c5": "c5_long_splitk", "c1": "c1_tiny_fp32", "c3spec": "c3_spec_decode",
-             "c3fp8": "c3_fp8"}
+             "c3fp8": "c3_fp8", "c3specfp8": "c3_spec_fp8"}
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")  # JSON text
@@ -253,7 +253,11 @@ class Step:
                                             workspace_tensor=self.ws)
 
     def decode(self):
-        if self.multi:
+        if self.multi and self.b.dtype == "fp8":
+            self.plan_obj.run_multi_fp8(self.out, self.b.q, self.b.k_cache, self.b.v_cache,
+                                        self.qsl, self.b.max_query_len, self.b.scale,
+                                        self.b.k_scale, self.b.v_scale)
+        elif self.multi:
             self.plan_obj.run_multi(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.qsl,
                                     self.b.max_query_len, self.b.scale)
         elif self.b.dtype == "fp8":
@@ -539,6 +543,17 @@ def oracle_step(b: workloads.Batch, host: dict, seqs: np.ndarray | None, threads
                                          b.v_scale)
         else:
             oracle.reshape_and_cache(host["new_k"], host["new_v"], k, v, slots)
+    if b.query_start_loc is not None:          # several query tokens per sequence
+        sel = np.arange(b.num_seqs) if seqs is None else np.asarray(seqs)
+        qsl = b.query_start_loc
+        rows = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in sel] + [np.zeros(0, int)])
+        sub_qsl = np.concatenate([[0], np.cumsum(qsl[sel + 1] - qsl[sel])]).astype(np.int32)
+        q = np.ascontiguousarray(host["q"][rows])
+        if fp8:
+            return oracle.paged_multi_fp8(q, k, v, b.k_scale, b.v_scale, b.block_tables[sel],
+                                          b.context_lens[sel], sub_qsl, b.scale, threads=threads)
+        return oracle.paged_multi(q, k, v, b.block_tables[sel], b.context_lens[sel], sub_qsl,
+                                  b.scale, threads=threads)
     tasks = None if seqs is None else np.array([(s, h) for s in seqs
                                                 for h in range(b.num_q_heads)], dtype=np.int32)
     if fp8:

@@ -172,7 +172,9 @@ pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_ca
  * is clamped, and a chunk reaching outside rows [0, num_q_tokens) is skipped;
  * both are flagged PKV_DEVERR_LEN.  With n = 1 everywhere this is
  * pkv_paged_attention_decode.  Workspace: pkv_multi_workspace_bytes().
- * bf16 and fp32 pools only: FP8 pools return PKV_ERR_UNSUPPORTED.
+ * bf16 and fp32 pools; FP8 pools go through pkv_paged_attention_multi_fp8
+ * and pkv_multi_run_fp8 (below), which take the pools' scales (the plain
+ * calls return PKV_ERR_UNSUPPORTED for them).
  */
 size_t pkv_multi_workspace_bytes(const pkv_dims *dims, int32_t num_q_tokens,
                                  int32_t max_context_len, int32_t partition_tokens);
@@ -279,6 +281,27 @@ pkv_status pkv_paged_attention_decode_fp8(void *out, const void *q, const void *
                                           int32_t max_context_len, int32_t partition_tokens,
                                           void *workspace, size_t workspace_bytes,
                                           void *cuda_stream);
+
+/* Several causal query tokens per sequence (pkv_paged_attention_multi,
+ * pkv_multi_run) over FP8 pools: q and out bf16, arithmetic as for
+ * pkv_paged_attention_decode_fp8. */
+pkv_status pkv_paged_attention_multi_fp8(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         const int32_t *context_lens,
+                                         const int32_t *query_start_loc, int32_t num_q_tokens,
+                                         int32_t max_query_len, float scale, float k_scale,
+                                         float v_scale, const pkv_dims *dims,
+                                         int32_t max_context_len, int32_t partition_tokens,
+                                         void *workspace, size_t workspace_bytes,
+                                         void *cuda_stream);
+
+pkv_status pkv_multi_run_fp8(void *out, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, const int32_t *context_lens,
+                             const int32_t *query_start_loc, int32_t num_q_tokens,
+                             int32_t max_query_len, float scale, float k_scale, float v_scale,
+                             const pkv_dims *dims, int32_t max_context_len,
+                             int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+                             void *cuda_stream);
 
 pkv_status pkv_decode_run_fp8(void *out, const void *q, const void *k_cache,
                               const void *v_cache, const int32_t *block_tables,

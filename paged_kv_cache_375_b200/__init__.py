@@ -85,6 +85,10 @@ def load_library() -> ctypes.CDLL:
                                                               i32, i32, P, sz, P]),
             "pkv_decode_run_fp8": (ctypes.c_int, [P, P, P, P, P, P, f32, f32, f32, D, i32, i32,
                                                   P, sz, P]),
+            "pkv_paged_attention_multi_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32,
+                                                             f32, f32, D, i32, i32, P, sz, P]),
+            "pkv_multi_run_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, f32, f32, D,
+                                                 i32, i32, P, sz, P]),
             "pkv_copy_blocks": (ctypes.c_int, [P, P, P, i32, D, P]),
             "pkv_validate_copy_pairs": (ctypes.c_int, [P, i32, i32]),
             "pkv_slot_mapping": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
@@ -310,6 +314,44 @@ def paged_attention_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torc
     return out
 
 
+def paged_attention_multi_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                              v_cache: torch.Tensor, block_tables: torch.Tensor,
+                              context_lens: torch.Tensor, query_start_loc: torch.Tensor,
+                              scale: float, k_scale: float, v_scale: float, max_query_len: int,
+                              *, max_context_len: int | None = None, partition_tokens: int = 0,
+                              workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
+    """paged_attention_multi over FP8 (float8_e4m3fn) pools with their scales; q and out
+    are bfloat16, head_dim 128."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
+    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    _need(query_start_loc, "query_start_loc", torch.int32, dev)
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must be [num_blocks][num_kv_heads][16][head_dim]")
+    T, hq, d = q.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or query_start_loc.shape != (B + 1,) or block_tables.shape[0] != B \
+            or k_cache.shape[3] != d:
+        raise ValueError("inconsistent shapes")
+    dims = make_dims(B, hq, k_cache, block_tables.shape[1])
+    mcl = block_tables.shape[1] * k_cache.shape[2] if max_context_len is None else int(max_context_len)
+    lib = load_library()
+    need = lib.pkv_multi_workspace_bytes(ctypes.byref(dims), T, mcl, partition_tokens)
+    if need == 0:
+        raise PkvError(2, lib.pkv_last_error_message().decode())
+    ws = workspace_tensor if workspace_tensor is not None else workspace(dev, need)
+    _check(lib.pkv_paged_attention_multi_fp8(
+        _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+        _p(query_start_loc), T, int(max_query_len), float(scale), float(k_scale),
+        float(v_scale), ctypes.byref(dims), mcl, partition_tokens, _p(ws), ws.numel(),
+        _stream_ptr(dev)))
+    return out
+
+
 class DecodePlan:
     """A decode plan for one step: the work list built from context_lens, kept in a
     workspace.  ``run`` decodes one layer's cache pools with it; plan once per step, run
@@ -358,6 +400,29 @@ class DecodePlan:
             _p(self.context_lens), _p(query_start_loc), q.shape[0], int(max_query_len),
             float(scale), ctypes.byref(self.dims), self.max_context_len, self.partition_tokens,
             _p(self.workspace), self.workspace.numel(), _stream_ptr(dev)))
+        return out
+
+    def run_multi_fp8(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, query_start_loc: torch.Tensor, max_query_len: int,
+                      scale: float, k_scale: float, v_scale: float) -> torch.Tensor:
+        """run_multi over FP8 pools (see paged_attention_multi_fp8)."""
+        dev = q.device
+        _need(q, "q", torch.bfloat16, dev)
+        _need(out, "out", torch.bfloat16, dev)
+        _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
+        _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+        _need(query_start_loc, "query_start_loc", torch.int32, dev)
+        lib = load_library()
+        need = lib.pkv_multi_workspace_bytes(ctypes.byref(self.dims), q.shape[0],
+                                             self.max_context_len, self.partition_tokens)
+        if need == 0 or self.workspace.numel() < need:
+            raise PkvError(4, f"workspace too small for {q.shape[0]} query rows ({need} bytes)")
+        _check(lib.pkv_multi_run_fp8(
+            _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
+            _p(self.context_lens), _p(query_start_loc), q.shape[0], int(max_query_len),
+            float(scale), float(k_scale), float(v_scale), ctypes.byref(self.dims),
+            self.max_context_len, self.partition_tokens, _p(self.workspace),
+            self.workspace.numel(), _stream_ptr(dev)))
         return out
 
     def run(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,

@@ -445,6 +445,68 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
 
 }  // namespace
 
+namespace {
+
+// The run and one-shot calls for several query tokens; `fp8` selects the FP8
+// entry points (FP8 pools and their scales) or the plain ones (bf16 / fp32).
+pkv_status check_multi_pools(const pkv_dims* dims, bool fp8, float k_scale, float v_scale) {
+  if (fp8) {
+    if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+        !std::isfinite(v_scale))
+      return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+  } else if (dims->dtype == PKV_FP8_E4M3) {
+    return fail(PKV_ERR_UNSUPPORTED,
+                "FP8 pools need their scales: use the _fp8 calls for several query tokens");
+  }
+  return PKV_OK;
+}
+
+pkv_status multi_run(void* out, const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, const int32_t* context_lens,
+                     const int32_t* query_start_loc, int32_t num_q_tokens, int32_t max_query_len,
+                     float scale, bool fp8, float k_scale, float v_scale, const pkv_dims* dims,
+                     int32_t max_context_len, int32_t partition_tokens, void* workspace,
+                     size_t workspace_bytes, void* cuda_stream) {
+  if (num_q_tokens < 0) return fail(PKV_ERR_SHAPE, "num_q_tokens must be >= 0");
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
+  if (st != PKV_OK) return st;
+  if ((st = check_multi_pools(dims, fp8, k_scale, v_scale)) != PKV_OK) return st;
+  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
+  if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                    max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream,
+                    k_scale, v_scale);
+}
+
+pkv_status multi_one_shot(void* out, const void* q, const void* k_cache, const void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          const int32_t* query_start_loc, int32_t num_q_tokens,
+                          int32_t max_query_len, float scale, bool fp8, float k_scale,
+                          float v_scale, const pkv_dims* dims, int32_t max_context_len,
+                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                          void* cuda_stream) {
+  if (num_q_tokens < 0) return fail(PKV_ERR_SHAPE, "num_q_tokens must be >= 0");
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
+  if (st != PKV_OK) return st;
+  if ((st = check_multi_pools(dims, fp8, k_scale, v_scale)) != PKV_OK) return st;
+  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
+  if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
+  if (max_query_len < 1 || (max_query_len * (dims->num_q_heads / dims->num_kv_heads)) > 16)
+    return fail(PKV_ERR_UNSUPPORTED, "max_query_len x group must be in [1, 16]");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  st = pkv_decode_plan(context_lens, dims, max_context_len, partition_tokens, workspace,
+                       workspace_bytes, cuda_stream);
+  if (st != PKV_OK) return st;
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                    max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream,
+                    k_scale, v_scale);
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t pkv_decode_partition_tokens(const pkv_dims* dims, int32_t max_context_len,
@@ -544,22 +606,16 @@ size_t pkv_multi_workspace_bytes(const pkv_dims* dims, int32_t num_q_tokens,
   return plan.total;
 }
 
+
 pkv_status pkv_multi_run(void* out, const void* q, const void* k_cache, const void* v_cache,
                          const int32_t* block_tables, const int32_t* context_lens,
                          const int32_t* query_start_loc, int32_t num_q_tokens,
                          int32_t max_query_len, float scale, const pkv_dims* dims,
                          int32_t max_context_len, int32_t partition_tokens, void* workspace,
                          size_t workspace_bytes, void* cuda_stream) {
-  if (num_q_tokens < 0) return fail(PKV_ERR_SHAPE, "num_q_tokens must be >= 0");
-  DecodePlan plan;
-  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
-  if (st != PKV_OK) return st;
-  if (dims->dtype == PKV_FP8_E4M3)
-    return fail(PKV_ERR_UNSUPPORTED, "several query tokens per sequence need bf16 or fp32 pools");
-  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
-  if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
-  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
-                    max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream);
+  return multi_run(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                   num_q_tokens, max_query_len, scale, false, 1.f, 1.f, dims, max_context_len,
+                   partition_tokens, workspace, workspace_bytes, cuda_stream);
 }
 
 pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cache,
@@ -569,22 +625,37 @@ pkv_status pkv_paged_attention_multi(void* out, const void* q, const void* k_cac
                                      const pkv_dims* dims, int32_t max_context_len,
                                      int32_t partition_tokens, void* workspace,
                                      size_t workspace_bytes, void* cuda_stream) {
-  if (num_q_tokens < 0) return fail(PKV_ERR_SHAPE, "num_q_tokens must be >= 0");
-  DecodePlan plan;
-  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, num_q_tokens);
-  if (st != PKV_OK) return st;
-  if (dims->dtype == PKV_FP8_E4M3)
-    return fail(PKV_ERR_UNSUPPORTED, "several query tokens per sequence need bf16 or fp32 pools");
-  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
-  if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
-  if (max_query_len < 1 || (max_query_len * (dims->num_q_heads / dims->num_kv_heads)) > 16)
-    return fail(PKV_ERR_UNSUPPORTED, "max_query_len x group must be in [1, 16]");
-  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
-  st = pkv_decode_plan(context_lens, dims, max_context_len, partition_tokens, workspace,
-                       workspace_bytes, cuda_stream);
-  if (st != PKV_OK) return st;
-  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
-                    max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream);
+  return multi_one_shot(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                        num_q_tokens, max_query_len, scale, false, 1.f, 1.f, dims,
+                        max_context_len, partition_tokens, workspace, workspace_bytes,
+                        cuda_stream);
+}
+
+pkv_status pkv_multi_run_fp8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             const int32_t* query_start_loc, int32_t num_q_tokens,
+                             int32_t max_query_len, float scale, float k_scale, float v_scale,
+                             const pkv_dims* dims, int32_t max_context_len,
+                             int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                             void* cuda_stream) {
+  return multi_run(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                   num_q_tokens, max_query_len, scale, true, k_scale, v_scale, dims,
+                   max_context_len, partition_tokens, workspace, workspace_bytes, cuda_stream);
+}
+
+pkv_status pkv_paged_attention_multi_fp8(void* out, const void* q, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         const int32_t* context_lens,
+                                         const int32_t* query_start_loc, int32_t num_q_tokens,
+                                         int32_t max_query_len, float scale, float k_scale,
+                                         float v_scale, const pkv_dims* dims,
+                                         int32_t max_context_len, int32_t partition_tokens,
+                                         void* workspace, size_t workspace_bytes,
+                                         void* cuda_stream) {
+  return multi_one_shot(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+                        num_q_tokens, max_query_len, scale, true, k_scale, v_scale, dims,
+                        max_context_len, partition_tokens, workspace, workspace_bytes,
+                        cuda_stream);
 }
 
 pkv_status pkv_decode_run_fp8(void* out, const void* q, const void* k_cache,

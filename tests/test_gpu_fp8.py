@@ -220,7 +220,7 @@ def test_c3_fp8_full_size_sampled(cuda_device):
     check_close(got, ref, "bf16", "c3 fp8 sampled")
 
 
-def test_several_query_tokens_over_fp8_pools_are_rejected(cuda_device):
+def test_plain_multi_call_rejects_fp8_pools(cuda_device):
     b = workloads.random_batch(980, [20, 30], 8, 2, 128, "fp8", device=cuda_device)
     bt, cl = dev_i32(b.block_tables, b.q.device), dev_i32(b.context_lens, b.q.device)
     qsl = torch.tensor([0, 1, 2], dtype=torch.int32, device=b.q.device)
@@ -234,3 +234,99 @@ def test_several_query_tokens_over_fp8_pools_are_rejected(cuda_device):
         pkv._p(qsl), 2, 1, b.scale, pkv.ctypes.byref(dims), 30, 0, pkv._p(ws), ws.numel(),
         pkv._stream_ptr(b.q.device))
     assert st == 3
+
+
+def gpu_fp8_multi(b, partition_tokens=0, plan=False):
+    dev = b.q.device
+    bt = dev_i32(b.block_tables, dev)
+    cl = dev_i32(b.context_lens, dev)
+    qsl = dev_i32(b.query_start_loc, dev)
+    if b.new_seq.shape[0]:
+        slots = pkv.slot_mapping(bt, b.num_blocks, token_seq=dev_i32(b.new_seq, dev),
+                                 token_pos=dev_i32(b.new_pos, dev))
+        pkv.reshape_and_cache_fp8(b.new_k, b.new_v, b.k_cache, b.v_cache, slots, b.k_scale,
+                                  b.v_scale)
+    out = torch.empty_like(b.q)
+    mcl = max(b.max_context_len, 1)
+    if plan:
+        dims = pkv.make_dims(b.num_seqs, b.num_q_heads, b.k_cache, bt.shape[1])
+        need = pkv.load_library().pkv_multi_workspace_bytes(pkv.ctypes.byref(dims), b.q.shape[0],
+                                                            mcl, partition_tokens)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        p = pkv.DecodePlan(bt, cl, b.num_q_heads, b.k_cache, max_context_len=mcl,
+                           partition_tokens=partition_tokens, workspace_tensor=ws)
+        p.run_multi_fp8(out, b.q, b.k_cache, b.v_cache, qsl, b.max_query_len, b.scale,
+                        b.k_scale, b.v_scale)
+    else:
+        pkv.paged_attention_multi_fp8(out, b.q, b.k_cache, b.v_cache, bt, cl, qsl, b.scale,
+                                      b.k_scale, b.v_scale, b.max_query_len,
+                                      max_context_len=mcl, partition_tokens=partition_tokens)
+    return out
+
+
+@pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 4), (8, 8, 16), (16, 2, 2), (12, 4, 5),
+                                             (16, 1, 1)])
+def test_fp8_multi_matches_oracle(cuda_device, hq, hkv, max_chunk):
+    rng = np.random.default_rng(hq * 31 + hkv * 7 + max_chunk)
+    lens = np.array([1, 2, 15, 16, 17, 33, 64, 100, 257, 300, 31, 48])
+    chunks = np.minimum(rng.integers(1, max_chunk + 1, size=lens.shape[0]), lens)
+    b = workloads.chunked_batch(990 + hq + max_chunk, lens, chunks, hq, hkv, 128, "fp8",
+                                device=cuda_device, extra_table=2)
+    b.k_scale, b.v_scale = workloads.FP8_K_SCALE, workloads.FP8_V_SCALE
+    host = b.host()
+    out = gpu_fp8_multi(b)
+    assert pkv.device_error_bits() == 0
+    k, v = oracle_fp8_caches(b, host)
+    ref = oracle.paged_multi_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
+                                 b.context_lens, b.query_start_loc, b.scale)
+    check_close(out, ref, "bf16", f"fp8 multi {hq}/{hkv} chunks<={max_chunk}")
+
+
+@pytest.mark.parametrize("partition", [16, 256])
+def test_fp8_multi_split_k_and_plan_run(cuda_device, partition):
+    lens = np.array([40, 300, 1000, 2100, 5])
+    chunks = np.array([4, 3, 4, 1, 2])
+    b = workloads.chunked_batch(995 + partition, lens, chunks, 32, 8, 128, "fp8",
+                                device=cuda_device)
+    b.k_scale, b.v_scale = workloads.FP8_K_SCALE, workloads.FP8_V_SCALE
+    host = b.host()
+    out = gpu_fp8_multi(b, partition)
+    assert pkv.device_error_bits() == 0
+    k, v = oracle_fp8_caches(b, host)
+    ref = oracle.paged_multi_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
+                                 b.context_lens, b.query_start_loc, b.scale)
+    check_close(out, ref, "bf16", f"fp8 multi split {partition}")
+    again = gpu_fp8_multi(b, partition, plan=True)     # the K/V writes are idempotent
+    assert torch.equal(out.view(torch.int16), again.view(torch.int16))
+
+
+def test_fp8_one_token_chunks_equal_fp8_decode_bitwise(cuda_device):
+    lens = np.array([3, 16, 17, 600, 1500])
+    b = workloads.chunked_batch(997, lens, np.ones(5, dtype=np.int64), 32, 8, 128, "fp8",
+                                device=cuda_device)
+    b.k_scale, b.v_scale = workloads.FP8_K_SCALE, workloads.FP8_V_SCALE
+    multi = gpu_fp8_multi(b)
+    out = torch.empty_like(b.q)
+    pkv.paged_attention_decode_fp8(out, b.q, b.k_cache, b.v_cache,
+                                   dev_i32(b.block_tables, cuda_device),
+                                   dev_i32(b.context_lens, cuda_device), b.scale, b.k_scale,
+                                   b.v_scale, max_context_len=b.max_context_len)
+    assert torch.equal(multi.view(torch.int16), out.view(torch.int16))
+
+
+def test_fp8_spec_decode_workload_sampled(cuda_device):
+    b = workloads.c3_spec_fp8(device=cuda_device)
+    out = gpu_fp8_multi(b)
+    assert pkv.device_error_bits() == 0
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(36)
+    seqs = np.unique(np.concatenate([[int(np.argmax(b.context_lens))],
+                                     rng.integers(0, b.num_seqs, 5)]))
+    qsl = b.query_start_loc
+    rows = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in seqs])
+    sub_qsl = np.concatenate([[0], np.cumsum(qsl[seqs + 1] - qsl[seqs])]).astype(np.int32)
+    q = b.q.cpu().view(torch.int16).numpy().view(np.uint16)[rows]
+    ref = oracle.paged_multi_fp8(np.ascontiguousarray(q), codes(b.k_cache), codes(b.v_cache),
+                                 b.k_scale, b.v_scale, b.block_tables[seqs],
+                                 b.context_lens[seqs], sub_qsl, b.scale, threads=8)
+    check_close(out[torch.from_numpy(rows).long()], ref, "bf16", "fp8 spec decode")

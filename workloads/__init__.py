@@ -424,7 +424,8 @@ def chunked_batch(seed: int, lens, chunks, hq: int, hkv: int, d: int, dtype: str
     return b
 
 
-def c3_spec_decode(device="cpu", num_seqs: int = 256, draft: int = 4) -> Batch:
+def c3_spec_decode(device="cpu", num_seqs: int = 256, draft: int = 4,
+                   dtype: str = "bf16") -> Batch:
     """The Llama-3-8B-shaped GQA batch verifying `draft` speculative tokens per sequence:
     the draft tokens are the last positions of each context (lognormal lengths as in the
     decode batch, at least `draft`), written by reshape_and_cache, each with its query
@@ -432,10 +433,16 @@ def c3_spec_decode(device="cpu", num_seqs: int = 256, draft: int = 4) -> Batch:
     lens = np.maximum(c3_lens(num_seqs), draft)
     need = int(sum((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE for L in lens))
     b = chunked_batch(CONFIG_SEEDS["c3_llama3_8b_gqa"] + 100, lens, np.full(num_seqs, draft),
-                      32, 8, 128, "bf16", num_blocks=max(32768, int(math.ceil(1.25 * need))),
-                      device=device, name="c3_spec_decode")
+                      32, 8, 128, dtype, num_blocks=max(32768, int(math.ceil(1.25 * need))),
+                      device=device, name="c3_spec_decode" if dtype == "bf16" else
+                      f"c3_spec_decode_{dtype}")
     b.meta["draft_tokens"] = draft
     return b
+
+
+def c3_spec_fp8(device="cpu", num_seqs: int = 256, draft: int = 4) -> Batch:
+    """The speculative-verification batch over FP8 e4m3 pools (bf16 q and new K/V)."""
+    return c3_spec_decode(device, num_seqs, draft, "fp8")
 
 
 def c4_shared_prefix(device="cpu", prompts: int = 32, samples: int = 8, prefix: int = 1024,
@@ -501,6 +508,8 @@ def c5_long_splitk(device="cpu", num_seqs: int = 8) -> Batch:
 
 CONFIGS["c3_spec_decode"] = ("Llama-3-8B-shaped GQA bf16, batch 256, verifying 4 speculative tokens "
                               "per sequence (causal, 16 query rows per kv head)")
+CONFIGS["c3_spec_fp8"] = ("the speculative-verification batch (256 x 4 draft tokens, causal) over FP8 "
+                          "e4m3 pools, bf16 q/out")
 CONFIGS["c3_fp8"] = ("Llama-3-8B-shaped GQA over FP8 e4m3 pools (one scale per pool), bf16 q/out: "
                      "batch 256, 32q/8kv, d128, the same lognormal lens, reshape_and_cache_fp8 "
                      "of the new token before attention")
@@ -509,6 +518,7 @@ BUILDERS = {
     "c1_tiny_fp32": c1_tiny_fp32,
     "c3_spec_decode": c3_spec_decode,
     "c3_fp8": c3_fp8,
+    "c3_spec_fp8": c3_spec_fp8,
     "c2_llama2_13b_mha": c2_llama2_13b_mha,
     "c3_llama3_8b_gqa": c3_llama3_8b_gqa,
     "c4_shared_prefix": c4_shared_prefix,
