@@ -333,11 +333,13 @@ pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
                         const int32_t* context_lens, const int32_t* query_start_loc,
                         const pkv_dims* d, cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(plan.num_q_tokens) * d->num_q_heads;
-  const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
+  if (rows > 0x7fffffff) return fail(PKV_ERR_UNSUPPORTED, "too many query rows for the merge");
+  const unsigned grid = static_cast<unsigned>(rows);  // one CTA per row
   const float* po = reinterpret_cast<const float*>(ws + plan.part_o_off);
   const float* pml = reinterpret_cast<const float*>(ws + plan.part_ml_off);
   auto kern = d->head_dim == 128 ? pkv::merge_kernel<T, 128> : pkv::merge_kernel<T, 64>;
-  cudaError_t e = launch(kern, dim3(grid), dim3(128), 0, stream, out, po, pml, context_lens,
+  cudaError_t e = launch(kern, dim3(grid), dim3(pkv::kMergeWarps * 32), 0, stream, out, po, pml,
+                         context_lens,
                          query_start_loc, d->num_seqs, plan.num_q_tokens, d->num_q_heads,
                          plan.max_parts, plan.max_len, plan.part_tokens);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");

@@ -1227,42 +1227,49 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 }
 
 // ------------------------------------------------------------- merge kernel
-// One warp per (query token, query head) row whose sequence was split:
-// combine the partitions' (m, l, o) by log-sum-exp and store the final
-// output.  Partitions a causal row cannot see carry l = 0 and no weight.
+// One CTA of kMergeWarps warps per (query token, query head) row whose
+// sequence was split: combine the partitions' (m, l, o) by log-sum-exp and
+// store the final output.  Every warp finds the common maximum M, takes every
+// kMergeWarps-th partition (so a row's partials stream in on several warps at
+// once), and warp 0 adds the warps' sums in a fixed order.  Partitions a causal
+// row cannot see carry l = 0 and no weight.
+constexpr int kMergeWarps = 4;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(void* __restrict__ out, const float* __restrict__ part_o,
                  const float* __restrict__ part_ml, const int32_t* __restrict__ context_lens,
                  const int32_t* __restrict__ query_start_loc, int32_t num_seqs,
                  int32_t num_q_tokens, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
                  int32_t part_tokens) {
+  constexpr int VEC = D / 32;  // floats per lane
+  __shared__ __align__(16) float red[kMergeWarps][D];
+  __shared__ float red_w[kMergeWarps];
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  const int64_t row = blockIdx.x;
   if (row >= static_cast<int64_t>(num_q_tokens) * num_q_heads) return;
   const int32_t t = static_cast<int32_t>(row / num_q_heads);  // query token
   int32_t s = t;                                                // its sequence
   if (query_start_loc) {  // the last sequence whose chunk starts at or before t
+    if (t >= query_start_loc[num_seqs]) return;  // rows past the last chunk
     int32_t lo = 0, hi = num_seqs - 1;
     while (lo < hi) {
       const int32_t mid = (lo + hi + 1) / 2;
       if (query_start_loc[mid] <= t) lo = mid; else hi = mid - 1;
     }
     s = lo;
-    if (t >= query_start_loc[num_seqs]) return;  // rows past the last chunk
   }
   int32_t L = context_lens[s];
   L = L < 0 ? 0 : (L > max_len ? max_len : L);
   const int32_t n = num_parts(L, part_tokens);
-  if (n <= 1) return;  // the decode kernel wrote this row directly
+  if (n <= 1) return;  // the decode kernel wrote this row directly (uniform over the CTA)
   const float* ml = part_ml + row * max_parts * 2;
   float M = -INFINITY;
   for (int p = lane; p < n; p += 32) M = fmaxf(M, ml[2 * p]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  constexpr int VEC = D / 32;  // floats per lane
   float acc[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) acc[i] = 0.f;
@@ -1270,7 +1277,7 @@ __global__ void __launch_bounds__(128)
   const float* po = part_o + row * max_parts * D + lane * VEC;
   if (M != -INFINITY) {
 #pragma unroll 4
-    for (int p = 0; p < n; ++p) {
+    for (int p = warp; p < n; p += kMergeWarps) {
       const float lp = ml[2 * p + 1];
       const float w = lp > 0.f ? lp * exp2f((ml[2 * p] - M) * kLog2e) : 0.f;
       wsum += w;
@@ -1287,7 +1294,22 @@ __global__ void __launch_bounds__(128)
       }
     }
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) red[warp][lane * VEC + i] = acc[i];
+  if (lane == 0) red_w[warp] = wsum;
+  __syncthreads();
+  if (warp != 0) return;
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) tot += red_w[w];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) a += red[w][lane * VEC + i];
+    acc[i] = a;
+  }
+  const float inv = tot > 0.f ? 1.f / tot : 0.f;
   if constexpr (sizeof(T) == 2) {
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + row * D + lane * VEC;
     if constexpr (VEC == 4) {

@@ -498,12 +498,13 @@ def c4_shared_prefix(device="cpu", prompts: int = 32, samples: int = 8, prefix: 
 
 def c5_long_splitk(device="cpu", num_seqs: int = 8) -> Batch:
     """Long-context GQA decode: 64 q / 8 kv heads, d128, lens uniform in [32768, 131072],
-    blocks scattered over an 81,920-block pool; meant for 512-token split-K partitions."""
+    blocks scattered over an 81,920-block pool (10,240 per sequence for other batch
+    sizes); meant for 512-token split-K partitions."""
     seed = CONFIG_SEEDS["c5_long_splitk"]
     rng = np.random.default_rng(seed)
     lens = rng.integers(32768, 131072, size=num_seqs, endpoint=True)
-    return random_batch(seed, lens, 64, 8, 128, "bf16", num_blocks=81920, device=device,
-                        name="c5_long_splitk")
+    return random_batch(seed, lens, 64, 8, 128, "bf16", num_blocks=10240 * num_seqs,
+                        device=device, name="c5_long_splitk")
 
 
 CONFIGS["c3_spec_decode"] = ("Llama-3-8B-shaped GQA bf16, batch 256, verifying 4 speculative tokens "
