@@ -218,10 +218,14 @@ class Step:
         self.pos = torch.from_numpy(b.new_pos).to(dev)
         self.slots = torch.empty(max(self.T, 1), dtype=torch.int64, device=dev)
         self.pairs = torch.from_numpy(b.cow_pairs).to(dev) if b.cow_pairs.shape[0] else None
+        # one new token per sequence at its last position, no copies: the fused prologue
+        self.fused = self.decode_mode and self.pairs is None and not self.multi
         if self.pairs is not None:
             pkv.validate_copy_pairs(torch.from_numpy(b.cow_pairs), b.num_blocks)
 
     def launches_per_step(self) -> int:
+        if self.fused:                                 # prologue, decode (, merge)
+            return 2 + (1 if self.split else 0)
         n = 2 + (1 if self.split else 0)              # plan, decode (, merge)
         n += 2 if self.T else 0                        # slot indexing, reshape_and_cache
         n += 1 if self.pairs is not None else 0        # copy_blocks
@@ -229,6 +233,8 @@ class Step:
 
     def cache_ops(self):
         pkv, b = self.pkv, self.b
+        if self.fused:
+            return                                     # done by the prologue in plan()
         if self.pairs is not None:
             pkv.copy_blocks(b.k_cache, b.v_cache, self.pairs, validate=False)
         if self.T:
@@ -248,10 +254,15 @@ class Step:
             self.pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, slots)
 
     def plan(self):
-        self.plan_obj = self.pkv.DecodePlan(self.bt, self.cl, self.b.num_q_heads, self.b.k_cache,
+        b = self.b
+        extra = {}
+        if self.fused:   # one launch: the new tokens' slots and writes, and the plan
+            extra = dict(new_k=b.new_k, new_v=b.new_v, v_cache=b.v_cache, k_scale=b.k_scale,
+                         v_scale=b.v_scale, slot_mapping_out=self.slots[:self.T])
+        self.plan_obj = self.pkv.DecodePlan(self.bt, self.cl, b.num_q_heads, b.k_cache,
                                             max_context_len=self.mcl,
                                             partition_tokens=self.partition,
-                                            workspace_tensor=self.ws)
+                                            workspace_tensor=self.ws, **extra)
 
     def decode(self):
         if self.multi and self.b.dtype == "fp8":
@@ -402,7 +413,7 @@ def op_bytes(step: Step) -> dict:
     row_in = b.num_kv_heads * b.head_dim * b.q_elem_bytes      # one new token's K (or V)
     block = row * 16                                            # one K (or V) block
     T, P = step.T, int(b.cow_pairs.shape[0])
-    return {
+    out = {
         "slot_mapping": T * (4 + 4 + 8) + (4 * b.num_seqs if step.decode_mode else 8 * T),
         "reshape_and_cache": 2 * T * (row_in + row) + 8 * T,    # K and V, read and write
         "copy_blocks": 2 * 2 * P * block + 16 * P,              # K and V, read and write
@@ -410,13 +421,22 @@ def op_bytes(step: Step) -> dict:
         "plan": 4 * b.num_seqs + 16 * int(np.maximum(
             1, (b.context_lens.astype(np.int64) + step.part_tokens - 1) // step.part_tokens).sum()),
     }
+    out["decode_prologue"] = out["slot_mapping"] + out["reshape_and_cache"] + out["plan"]
+    return out
 
 
 def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
     """Each op of the step timed alone with events after the timed region (launches
     here do not overlap), with achieved bandwidth against the HBM peak."""
     pkv, b = step.pkv, step.b
-    ops = {"plan": step.plan}
+
+    def plan_only():
+        pkv.DecodePlan(step.bt, step.cl, b.num_q_heads, b.k_cache, max_context_len=step.mcl,
+                       partition_tokens=step.partition, workspace_tensor=step.ws)
+
+    ops = {"plan": plan_only}
+    if step.fused:
+        ops["decode_prologue"] = step.plan
     if step.T:
         if step.decode_mode:
             ops["slot_mapping"] = lambda: pkv.slot_mapping(step.bt, b.num_blocks,

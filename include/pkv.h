@@ -255,6 +255,39 @@ pkv_status pkv_paged_attention_decode_static(void *out, const void *q, const voi
                                              int32_t partition_tokens, void *cuda_stream);
 
 /*
+ * The prologue of a decode step in one launch (no counterpart of its own in
+ * the pages: it fuses three of their steps).  For every sequence s with
+ * L = context_lens[s] >= 1 the new token at position L - 1 is written:
+ * slot = block_tables[s][(L-1)/16] * 16 + (L-1) % 16 (slot indexing, the
+ * wiki entry's "Flattened 布局与 slot_mapping"), then k[s], v[s] ([num_seqs]
+ * [Hkv][D], same dtype as the pools) are copied into that slot as
+ * pkv_reshape_and_cache does; and the decode plan is built into `workspace`
+ * exactly as pkv_decode_plan builds it (same arguments, same workspace
+ * size).  The plan is built by one CTA while the others write the tokens.
+ * slot_mapping_out (int64 [num_seqs], may be NULL) receives each sequence's
+ * slot, -1 for L = 0 (no new token, nothing written) or a flagged entry.
+ * Equivalent to pkv_slot_mapping (context-length mode) + pkv_reshape_and_cache
+ * + pkv_decode_plan, except that L = 0 is not an error here.  Device-side
+ * errors: PKV_DEVERR_POS (L - 1 past the table), PKV_DEVERR_BLOCK (entry out
+ * of range), PKV_DEVERR_LEN (lengths, as the plan).  Follow it with
+ * pkv_decode_run (or pkv_decode_run_fp8) on the same workspace.
+ * pkv_decode_prepare_fp8: FP8 pools; k, v are bf16 and quantised as
+ * pkv_reshape_and_cache_fp8 does.
+ */
+pkv_status pkv_decode_prepare(const void *k, const void *v, void *k_cache, void *v_cache,
+                              const int32_t *block_tables, const int32_t *context_lens,
+                              int64_t *slot_mapping_out, const pkv_dims *dims,
+                              int32_t max_context_len, int32_t partition_tokens, void *workspace,
+                              size_t workspace_bytes, void *cuda_stream);
+
+pkv_status pkv_decode_prepare_fp8(const void *k, const void *v, void *k_cache, void *v_cache,
+                                  const int32_t *block_tables, const int32_t *context_lens,
+                                  int64_t *slot_mapping_out, float k_scale, float v_scale,
+                                  const pkv_dims *dims, int32_t max_context_len,
+                                  int32_t partition_tokens, void *workspace,
+                                  size_t workspace_bytes, void *cuda_stream);
+
+/*
  * FP8 KV cache.  The pages list FP8 among the quantisation formats and note
  * that memory saved holds more KV blocks ("vLLM 深读", section "引擎的分层结构";
  * "vllm" by vampireachao, "第三层：图、核、量化"); here the cache itself is FP8:

@@ -73,6 +73,9 @@ def load_library() -> ctypes.CDLL:
             "pkv_paged_attention_decode": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P,
                                                           sz, P]),
             "pkv_decode_plan": (ctypes.c_int, [P, D, i32, i32, P, sz, P]),
+            "pkv_decode_prepare": (ctypes.c_int, [P, P, P, P, P, P, P, D, i32, i32, P, sz, P]),
+            "pkv_decode_prepare_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, f32, f32, D, i32, i32,
+                                                      P, sz, P]),
             "pkv_multi_workspace_bytes": (sz, [D, i32, i32, i32]),
             "pkv_multi_run": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, D, i32, i32, P,
                                              sz, P]),
@@ -355,11 +358,20 @@ def paged_attention_multi_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch
 class DecodePlan:
     """A decode plan for one step: the work list built from context_lens, kept in a
     workspace.  ``run`` decodes one layer's cache pools with it; plan once per step, run
-    once per layer (the context lengths are the same for every layer)."""
+    once per layer (the context lengths are the same for every layer).
+
+    With ``new_k``/``new_v`` ([B][Hkv][D]; bf16 for FP8 pools) and ``v_cache``, the same
+    launch also writes every sequence's new token (position L - 1) into its slot of
+    ``k_cache``/``v_cache`` (quantised with ``k_scale``/``v_scale`` for FP8 pools) and,
+    if given, each slot into ``slot_mapping_out`` (int64 [B]): slot indexing,
+    reshape_and_cache and the plan in one launch."""
 
     def __init__(self, block_tables: torch.Tensor, context_lens: torch.Tensor, num_q_heads: int,
                  k_cache: torch.Tensor, *, max_context_len: int | None = None,
-                 partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None):
+                 partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None,
+                 new_k: torch.Tensor | None = None, new_v: torch.Tensor | None = None,
+                 v_cache: torch.Tensor | None = None, k_scale: float | None = None,
+                 v_scale: float | None = None, slot_mapping_out: torch.Tensor | None = None):
         dev = context_lens.device
         _need(block_tables, "block_tables", torch.int32, dev)
         _need(context_lens, "context_lens", torch.int32, dev)
@@ -376,10 +388,39 @@ class DecodePlan:
         if workspace_tensor.numel() < need:
             raise ValueError(f"workspace_tensor has {workspace_tensor.numel()} bytes, {need} needed")
         self.workspace = workspace_tensor
-        _check(load_library().pkv_decode_plan(_p(context_lens), ctypes.byref(self.dims),
-                                              self.max_context_len, partition_tokens,
-                                              _p(self.workspace), self.workspace.numel(),
-                                              _stream_ptr(dev)))
+        lib = load_library()
+        if new_k is None:
+            _check(lib.pkv_decode_plan(_p(context_lens), ctypes.byref(self.dims),
+                                       self.max_context_len, partition_tokens,
+                                       _p(self.workspace), self.workspace.numel(),
+                                       _stream_ptr(dev)))
+            return
+        fp8 = k_cache.dtype == torch.float8_e4m3fn
+        src = torch.bfloat16 if fp8 else k_cache.dtype
+        _need(new_k, "new_k", src, dev)
+        _need(new_v, "new_v", src, dev)
+        _need(k_cache, "k_cache", device=dev)
+        if v_cache is None:
+            raise ValueError("v_cache is needed to write the new tokens")
+        _need(v_cache, "v_cache", k_cache.dtype, dev)
+        B = context_lens.shape[0]
+        if new_k.shape != (B, k_cache.shape[1], k_cache.shape[3]) or new_v.shape != new_k.shape \
+                or v_cache.shape != k_cache.shape:
+            raise ValueError("new_k, new_v must be [num_seqs][num_kv_heads][head_dim]")
+        if slot_mapping_out is not None:
+            _need(slot_mapping_out, "slot_mapping_out", torch.int64, dev)
+            if slot_mapping_out.shape != (B,):
+                raise ValueError("slot_mapping_out must be int64 [num_seqs]")
+        args = [_p(new_k), _p(new_v), _p(k_cache), _p(v_cache), _p(block_tables),
+                _p(context_lens), _p(slot_mapping_out)]
+        tail = [ctypes.byref(self.dims), self.max_context_len, partition_tokens,
+                _p(self.workspace), self.workspace.numel(), _stream_ptr(dev)]
+        if fp8:
+            if k_scale is None or v_scale is None:
+                raise ValueError("FP8 pools need k_scale and v_scale")
+            _check(lib.pkv_decode_prepare_fp8(*args, float(k_scale), float(v_scale), *tail))
+        else:
+            _check(lib.pkv_decode_prepare(*args, *tail))
 
     def run_multi(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                   v_cache: torch.Tensor, query_start_loc: torch.Tensor, max_query_len: int,

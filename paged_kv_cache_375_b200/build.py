@@ -14,7 +14,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpkv.so")
 SOURCES = ["pkv_api.cu", "pkv_block_manager.cpp"]
-DEPS = SOURCES + ["pkv_device.cuh", "pkv_decode.cuh", "pkv_cache_ops.cuh"]
+DEPS = SOURCES + ["pkv_device.cuh", "pkv_decode.cuh", "pkv_cache_ops.cuh", "pkv_prepare.cuh"]
 HEADERS = ["pkv.h", "pkv_block_manager.h"]
 
 NVCC_FLAGS = [

@@ -16,6 +16,7 @@
 #include "pkv_cache_ops.cuh"
 #include "pkv_decode.cuh"
 #include "pkv_device.cuh"
+#include "pkv_prepare.cuh"
 
 namespace {
 
@@ -449,6 +450,59 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
 
 namespace {
 
+// Slot indexing + the new tokens' writes + the plan in one launch (see
+// pkv_decode_prepare).
+pkv_status decode_prepare(const void* k, const void* v, void* k_cache, void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          int64_t* slot_mapping_out, bool fp8, float k_scale, float v_scale,
+                          const pkv_dims* dims, int32_t max_context_len,
+                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                          void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
+  if (st != PKV_OK) return st;
+  if (fp8) {
+    if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+        !std::isfinite(v_scale))
+      return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+  } else if (dims->dtype == PKV_FP8_E4M3) {
+    return fail(PKV_ERR_UNSUPPORTED, "FP8 pools need their scales: use pkv_decode_prepare_fp8");
+  }
+  if (dims->num_seqs == 0) return PKV_OK;
+  if (!k || !v || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "k, v and the caches must be 16-byte aligned");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  if ((st = bind_device(k_cache, "k_cache")) != PKV_OK) return st;
+  // 16-byte units of one head's source row: bf16 / fp32 rows as stored, FP8
+  // rows as their bf16 inputs
+  const int src_row_bytes = dims->head_dim * (fp8 ? 2 : elem_bytes(dims->dtype));
+  const int units_per_head = src_row_bytes / 16;
+  const int units = dims->num_kv_heads * units_per_head;
+  const int per = units < pkv::kPlanThreads ? units : pkv::kPlanThreads;
+  const int seqs_per_cta = pkv::kPlanThreads / per;
+  const unsigned grid = 1u + static_cast<unsigned>((dims->num_seqs + seqs_per_cta - 1) / seqs_per_cta);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto kern = fp8 ? pkv::decode_prepare_kernel<true> : pkv::decode_prepare_kernel<false>;
+  cudaError_t e = launch(kern, dim3(grid), dim3(pkv::kPlanThreads), 0,
+                         static_cast<cudaStream_t>(cuda_stream), static_cast<const uint4*>(k),
+                         static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
+                         static_cast<uint8_t*>(v_cache), block_tables, context_lens,
+                         slot_mapping_out, dims->num_seqs, dims->num_kv_heads, units_per_head,
+                         dims->max_blocks_per_seq, dims->num_blocks, seqs_per_cta, per, k_scale,
+                         v_scale, plan.max_len, plan.part_blocks,
+                         reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off),
+                         reinterpret_cast<uint32_t*>(ws));
+  if (e != cudaSuccess) return cuda_fail(e, "decode prepare launch");
+  return PKV_OK;
+}
+
+}  // namespace
+
+namespace {
+
 // The run and one-shot calls for several query tokens; `fp8` selects the FP8
 // entry points (FP8 pools and their scales) or the plain ones (bf16 / fp32).
 pkv_status check_multi_pools(const pkv_dims* dims, bool fp8, float k_scale, float v_scale) {
@@ -556,6 +610,27 @@ pkv_status pkv_decode_plan(const int32_t* context_lens, const pkv_dims* dims,
                          reinterpret_cast<uint32_t*>(ws));
   if (e != cudaSuccess) return cuda_fail(e, "plan launch");
   return PKV_OK;
+}
+
+pkv_status pkv_decode_prepare(const void* k, const void* v, void* k_cache, void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int64_t* slot_mapping_out, const pkv_dims* dims,
+                              int32_t max_context_len, int32_t partition_tokens, void* workspace,
+                              size_t workspace_bytes, void* cuda_stream) {
+  return decode_prepare(k, v, k_cache, v_cache, block_tables, context_lens, slot_mapping_out,
+                        false, 1.f, 1.f, dims, max_context_len, partition_tokens, workspace,
+                        workspace_bytes, cuda_stream);
+}
+
+pkv_status pkv_decode_prepare_fp8(const void* k, const void* v, void* k_cache, void* v_cache,
+                                  const int32_t* block_tables, const int32_t* context_lens,
+                                  int64_t* slot_mapping_out, float k_scale, float v_scale,
+                                  const pkv_dims* dims, int32_t max_context_len,
+                                  int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, void* cuda_stream) {
+  return decode_prepare(k, v, k_cache, v_cache, block_tables, context_lens, slot_mapping_out,
+                        true, k_scale, v_scale, dims, max_context_len, partition_tokens,
+                        workspace, workspace_bytes, cuda_stream);
 }
 
 pkv_status pkv_decode_run(void* out, const void* q, const void* k_cache, const void* v_cache,

@@ -78,20 +78,20 @@ __device__ __forceinline__ int32_t part_size_blocks(int32_t L, int32_t p, int32_
   return rest < part_blocks ? rest : part_blocks;
 }
 
-// Single CTA.  counters[0] = work counter, counters[1] = items, counters[2] =
-// CTAs finished; the work and finish counters are zeroed here, and the decode
-// kernel's last CTA zeroes them again, so one plan serves any number of runs.
-__global__ void __launch_bounds__(kPlanThreads)
-    plan_kernel(const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t max_len,
-                int32_t part_blocks, PlanItem* __restrict__ items,
-                uint32_t* __restrict__ counters) {
-  __shared__ uint32_t hist[kPlanBuckets];
-  __shared__ uint32_t warp_sums[kPlanThreads / 32];
+// The plan, run by one CTA of kPlanThreads threads: counts the work items per
+// size, scans, and writes them sorted by size (largest first).  counters[0] =
+// work counter, counters[1] = items, counters[2] = CTAs finished; the work and
+// finish counters are zeroed here, and the decode kernel's last CTA zeroes
+// them again, so one plan serves any number of runs.  The caller has already
+// passed griddepcontrol.wait.
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ context_lens,
+                                          int32_t num_seqs, int32_t max_len, int32_t part_blocks,
+                                          PlanItem* __restrict__ items,
+                                          uint32_t* __restrict__ counters, uint32_t* hist,
+                                          uint32_t* warp_sums) {
   const int tid = threadIdx.x;
   const int32_t part_tokens = part_blocks * kBlock;
   for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
-  pdl_wait();
-  pdl_trigger();
   __syncthreads();
   for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
     int32_t L = checked_len(context_lens[s], max_len);
@@ -139,6 +139,18 @@ __global__ void __launch_bounds__(kPlanThreads)
       items[pos] = PlanItem{s, p, L, n};
     }
   }
+}
+
+// Single CTA: the plan alone.
+__global__ void __launch_bounds__(kPlanThreads)
+    plan_kernel(const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t max_len,
+                int32_t part_blocks, PlanItem* __restrict__ items,
+                uint32_t* __restrict__ counters) {
+  __shared__ uint32_t hist[kPlanBuckets];
+  __shared__ uint32_t warp_sums[kPlanThreads / 32];
+  pdl_wait();
+  pdl_trigger();
+  plan_body(context_lens, num_seqs, max_len, part_blocks, items, counters, hist, warp_sums);
 }
 
 // ------------------------------------------------------------ decode kernel
