@@ -242,13 +242,15 @@ struct DecodeCfg<float, D, GMAX> {
 // code conversions), so the kernel is bound by per-tile latency rather than
 // by HBM: more decode warps hide more of it.  Up to 8 query rows the state
 // fits 128 registers and 15 decode warps run (one merge buffer to fit shared
-// memory); with 16 rows 14 warps in pairs as above (measured on B200: 15
-// warps 4.49 TB/s, 11 warps 4.25, 8 warps with 4 stages 3.78 on the
-// Llama-3-8B-shaped batch).  Two stages per warp keep 56-120 KB per SM in
-// flight.
+// memory); measured on B200 on the Llama-3-8B-shaped batch: 15 warps 4.49
+// TB/s, 11 warps 4.25, 8 warps with 4 stages 3.78.  With 16 rows one warp
+// holds all of them (11 warps, 168 registers): paired warps would each widen
+// the same codes to f16, and the conversions dominate (spec verification:
+// 11 single warps 2.93 TB/s, 7 pairs 2.49).  Two stages per warp keep
+// 88-120 KB per SM in flight.
 template <int D, int GMAX>
 struct DecodeCfg<pkv::Fp8Kv, D, GMAX> {
-  static constexpr int W = GMAX == 16 ? 14 : 15, S = 2, MB = 1, SPLIT = GMAX == 16 ? 2 : 1;
+  static constexpr int W = GMAX == 16 ? 11 : 15, S = 2, MB = 1, SPLIT = 1;
 };
 
 // Largest dynamic shared memory already enabled per kernel, per device.
