@@ -14,6 +14,11 @@ per-sequence block table, slot_mapping, copy-on-write of shared blocks):
   reshape_and_cache(k, v, k_cache, v_cache, slot_mapping)
   copy_blocks(k_cache, v_cache, pairs)
   slot_mapping(block_tables, context_lens=None, token_seq=None, token_pos=None)
+  DecodePlan(...)            plan once per step (optionally writing the new tokens
+                             in the same launch), run once per layer
+  paged_attention_multi(...) several causal query tokens per sequence
+  *_fp8 variants             FP8 (e4m3) pools with per-pool scales
+  BlockManager               host-side block bookkeeping with prefix caching
   check_device_error()
 """
 from __future__ import annotations

@@ -83,6 +83,23 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Eight bf16 values (16 bytes) to eight e4m3 codes (8 bytes, same order):
+// code = e4m3(value / scale), the division in float (round to nearest even),
+// then round to nearest even onto e4m3, saturating to +-448.
+__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float scale) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint32_t codes[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t p0 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i]), scale),
+                                        __fdiv_rn(bf16hi_to_f32(w[2 * i]), scale));
+    const uint32_t p1 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i + 1]), scale),
+                                        __fdiv_rn(bf16hi_to_f32(w[2 * i + 1]), scale));
+    codes[i] = p0 | (p1 << 16);
+  }
+  return make_uint2(codes[0], codes[1]);
+}
+
 // ------------------------------------------------ reshape_and_cache into FP8
 // One CTA per token: each thread turns 8 bf16 values of the token's K (and V)
 // into 8 e4m3 codes, code = e4m3(value / scale) with the division in float,
@@ -113,18 +130,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       const uint4 x = (c ? v : k)[static_cast<int64_t>(t) * units + u];
-      const float sc = c ? v_scale : k_scale;
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-      uint32_t codes[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint32_t p0 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i]), sc),
-                                            __fdiv_rn(bf16hi_to_f32(w[2 * i]), sc));
-        const uint32_t p1 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i + 1]), sc),
-                                            __fdiv_rn(bf16hi_to_f32(w[2 * i + 1]), sc));
-        codes[i] = p0 | (p1 << 16);
-      }
-      *reinterpret_cast<uint2*>((c ? v_cache : k_cache) + dst) = make_uint2(codes[0], codes[1]);
+      *reinterpret_cast<uint2*>((c ? v_cache : k_cache) + dst) =
+          bf16x8_to_e4m3x8(x, c ? v_scale : k_scale);
     }
   }
 }

@@ -71,24 +71,10 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int32_t within = u % units_per_head;
     const int64_t row = (block * num_kv_heads + h) * kBlock + offset;  // destination row
     if constexpr (kFp8) {
-      // 8 bf16 values -> 8 e4m3 codes (value / scale in float, nearest even, saturated)
+      // 8 bf16 values -> 8 e4m3 codes
       const int64_t dst = row * (units_per_head * 8) + within * 8;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const uint4 x = (c ? vsrc : ksrc)[u];
-        const float sc = c ? v_scale : k_scale;
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t codes[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const uint32_t p0 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i]), sc),
-                                              __fdiv_rn(bf16hi_to_f32(w[2 * i]), sc));
-          const uint32_t p1 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i + 1]), sc),
-                                              __fdiv_rn(bf16hi_to_f32(w[2 * i + 1]), sc));
-          codes[i] = p0 | (p1 << 16);
-        }
-        *reinterpret_cast<uint2*>((c ? v_cache : k_cache) + dst) = make_uint2(codes[0], codes[1]);
-      }
+      *reinterpret_cast<uint2*>(k_cache + dst) = bf16x8_to_e4m3x8(ksrc[u], k_scale);
+      *reinterpret_cast<uint2*>(v_cache + dst) = bf16x8_to_e4m3x8(vsrc[u], v_scale);
     } else {
       const int64_t dst = row * (units_per_head * 16) + within * 16;
       *reinterpret_cast<uint4*>(k_cache + dst) = ksrc[u];
