@@ -167,8 +167,10 @@ pkv_status pkv_paged_attention_decode(void *out, const void *q, const void *k_ca
  * to keys 0 .. L - n + i:
  *   out[row][h] = softmax_{j <= L-n+i}(scale * q[row][h] . K_j) V_j.
  * q, out: [num_q_tokens][Hq][D].  max_query_len (host) bounds every chunk;
- * max_query_len x (Hq/Hkv) must be at most 16 (the query rows of one kv head
- * share an MMA tile).  A chunk longer than max_query_len or than its context
+ * Hq/Hkv must be at most 16.  Chunks of any length are accepted: the rows of
+ * one kv head are taken 16 (whole tokens) at a time, each group of rows
+ * reading only the keys it can see, so a long chunk (a prompt prefilled in
+ * one call) re-reads the KV once per group.  A chunk longer than max_query_len or than its context
  * is clamped, and a chunk reaching outside rows [0, num_q_tokens) is skipped;
  * both are flagged PKV_DEVERR_LEN.  With n = 1 everywhere this is
  * pkv_paged_attention_decode.  Workspace: pkv_multi_workspace_bytes().

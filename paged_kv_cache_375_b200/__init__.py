@@ -253,7 +253,7 @@ def paged_attention_multi(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Ten
 
     q, out: [T][Hq][D]; query_start_loc: int32 [B+1] (sequence s owns rows
     query_start_loc[s] .. query_start_loc[s+1]-1, at positions L-n .. L-1 of its context,
-    L = context_lens[s] including the chunk).  max_query_len * (Hq/Hkv) <= 16.
+    L = context_lens[s] including the chunk).  Any chunk length; Hq/Hkv <= 16.
     """
     dev = q.device
     _need(q, "q", device=dev)

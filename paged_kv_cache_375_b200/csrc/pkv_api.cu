@@ -397,10 +397,14 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
   if (max_query_len < 1) return fail(PKV_ERR_SHAPE, "max_query_len must be >= 1");
   const int group = d->num_q_heads / d->num_kv_heads;
-  const int rows_max = max_query_len * group;
-  if (rows_max > 16)
-    return fail(PKV_ERR_UNSUPPORTED, "chunk length x group = %d > 16 query rows per kv head",
-                rows_max);
+  if (group > 16)
+    return fail(PKV_ERR_UNSUPPORTED, "%d query heads per kv head (at most 16)", group);
+  // Up to 16 query rows per item (an item's rows share one MMA tile); a longer
+  // chunk is split into row groups of whole tokens, each read against the
+  // keys its rows can see.
+  const int group_tokens = max_query_len * group <= 16 ? max_query_len : 16 / group;
+  const int row_groups = (max_query_len + group_tokens - 1) / group_tokens;
+  const int rows_max = group_tokens * group;
   if ((st = bind_device(out, "out")) != PKV_OK) return st;
   CUtensorMap mk, mv;
   if ((st = encode_pool_map(&mk, k_cache, d)) != PKV_OK) return st;
@@ -418,6 +422,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.part_ml = plan.max_parts > 1 ? reinterpret_cast<float*>(ws + plan.part_ml_off) : nullptr;
   prm.query_start_loc = query_start_loc;
   prm.max_query_len = max_query_len;
+  prm.group_tokens = group_tokens;
+  prm.row_groups = row_groups;
   prm.num_q_tokens = plan.num_q_tokens;
   prm.num_q_heads = d->num_q_heads;
   prm.num_kv_heads = d->num_kv_heads;
@@ -428,7 +434,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.part_blocks = plan.part_blocks;
   prm.qk_scale_log2 = scale * pkv::kLog2e * k_scale;
   prm.out_scale = v_scale;
-  const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads;
+  const int64_t units =
+      static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads * row_groups;
   if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_BF16) {
@@ -552,8 +559,7 @@ pkv_status multi_one_shot(void* out, const void* q, const void* k_cache, const v
   if ((st = check_multi_pools(dims, fp8, k_scale, v_scale)) != PKV_OK) return st;
   if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
   if (!query_start_loc) return fail(PKV_ERR_NULL, "query_start_loc is NULL");
-  if (max_query_len < 1 || (max_query_len * (dims->num_q_heads / dims->num_kv_heads)) > 16)
-    return fail(PKV_ERR_UNSUPPORTED, "max_query_len x group must be in [1, 16]");
+  if (max_query_len < 1) return fail(PKV_ERR_SHAPE, "max_query_len must be >= 1");
   if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
   st = pkv_decode_plan(context_lens, dims, max_context_len, partition_tokens, workspace,
                        workspace_bytes, cuda_stream);

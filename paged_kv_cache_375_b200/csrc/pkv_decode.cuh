@@ -165,7 +165,9 @@ struct DecodeParams {
   // Query tokens of sequence s: rows query_start_loc[s] .. query_start_loc[s+1]-1
   // at positions L-n .. L-1 (causal); NULL means one token per sequence, row s.
   const int32_t* query_start_loc;
-  int32_t max_query_len;         // longest chunk; chunk length x group <= GMAX
+  int32_t max_query_len;         // longest chunk (tokens); longer chunks are flagged
+  int32_t group_tokens;          // chunk tokens per item (row group): group_tokens x group <= GMAX
+  int32_t row_groups;            // items per (sequence, partition, kv head)
   int32_t num_q_tokens;          // rows of q and out
   int32_t num_q_heads;
   int32_t num_kv_heads;
@@ -896,7 +898,9 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int g = prm.group;
-  const int rows_max = prm.max_query_len * g;  // query rows of the largest item
+  // query rows of the largest item
+  const int rows_max = (prm.max_query_len < prm.group_tokens ? prm.max_query_len
+                                                              : prm.group_tokens) * g;
   uint8_t* stages = smem + Lay::kStagesOff;
   uint8_t* ring = smem + Lay::kRingOff;
   int32_t* tables = reinterpret_cast<int32_t*>(smem + Lay::kTablesOff);  // [kRing][kMaxItemBlocks]
@@ -932,7 +936,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   const int32_t hkv = prm.num_kv_heads;
   if (warp == W) {
     // ================================ scheduler ================================
-    const uint32_t total = prm.counters[1] * static_cast<uint32_t>(hkv);
+    const uint32_t per_item = static_cast<uint32_t>(hkv) * prm.row_groups;
+    const uint32_t total = prm.counters[1] * per_item;
     uint32_t next = 0;
     if (lane == 0) next = atomicAdd(&prm.counters[0], 1u);
     uint32_t item_seq = 0;
@@ -963,39 +968,52 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
       }
       // fetch the following item now; its value is only needed next time round
       if (lane == 0) next = atomicAdd(&prm.counters[0], 1u);
-      const PlanItem pi = prm.items[widx / hkv];
-      const int32_t kvh = static_cast<int32_t>(widx % hkv);
+      // work index -> (planned item, kv head, row group); a (sequence, partition,
+      // kv head)'s row groups are adjacent, so they read the same tiles close in time
+      const PlanItem pi = prm.items[widx / per_item];
+      const uint32_t rem = widx % per_item;
+      const int32_t kvh = static_cast<int32_t>(rem / prm.row_groups);
+      const int32_t grp = static_cast<int32_t>(rem % prm.row_groups);
       const int32_t blk_begin = pi.part * prm.part_blocks;
-      int32_t nblk = (pi.len + kBlock - 1) / kBlock - blk_begin;
-      nblk = nblk < prm.part_blocks ? nblk : prm.part_blocks;
-      nblk = nblk < 0 ? 0 : nblk;
-      const int32_t* src = prm.block_tables +
-                           static_cast<size_t>(pi.seq) * prm.max_blocks_per_seq + blk_begin;
-      int32_t* dst = tables + r * kMaxItemBlocks;
-      for (int32_t j = lane; j < nblk; j += 32) dst[j] = src[j];
       // the chunk of query tokens: one per sequence unless query_start_loc is given
       int32_t q_start = pi.seq, q_len = 1;
       if (prm.query_start_loc) {
         q_start = prm.query_start_loc[pi.seq];
         q_len = prm.query_start_loc[pi.seq + 1] - q_start;
         const int32_t cap = pi.len < prm.max_query_len ? pi.len : prm.max_query_len;
+        const bool first = lane == 0 && kvh == 0 && pi.part == 0 && grp == 0;
         if (q_len < 0 || q_len > cap) {
-          if (lane == 0 && kvh == 0 && pi.part == 0) raise_error(PKV_DEVERR_LEN);
+          if (first) raise_error(PKV_DEVERR_LEN);
           q_len = q_len < 0 ? 0 : cap;
         }
         if (q_start < 0 || q_start + q_len > prm.num_q_tokens) {  // rows outside q / out
-          if (lane == 0 && kvh == 0 && pi.part == 0) raise_error(PKV_DEVERR_LEN);
+          if (first) raise_error(PKV_DEVERR_LEN);
           q_start = 0;
           q_len = 0;
         }
       }
+      // this row group: chunk tokens t0 .. t0 + tlen - 1; none of its rows sees a
+      // key past position len_eff - 1, so only those blocks are read
+      const int32_t t0 = grp * prm.group_tokens;
+      int32_t tlen = q_len - t0;
+      tlen = tlen < 0 ? 0 : (tlen > prm.group_tokens ? prm.group_tokens : tlen);
+      const int32_t len_eff = tlen > 0 ? pi.len - (q_len - t0 - tlen) : pi.len;
+      int32_t nblk = (len_eff + kBlock - 1) / kBlock - blk_begin;
+      nblk = nblk < prm.part_blocks ? nblk : prm.part_blocks;
+      nblk = nblk < 0 || tlen == 0 ? 0 : nblk;  // a group without rows reads nothing
+      q_start += t0;
+      q_len = tlen;
+      const int32_t* src = prm.block_tables +
+                           static_cast<size_t>(pi.seq) * prm.max_blocks_per_seq + blk_begin;
+      int32_t* dst = tables + r * kMaxItemBlocks;
+      for (int32_t j = lane; j < nblk; j += 32) dst[j] = src[j];
       __syncwarp();
       if (lane == 0) {
         ItemMeta& mt = meta[r];
         mt.seq = pi.seq;
         mt.kv_head = kvh;
         mt.part = pi.part;
-        mt.len = pi.len;
+        mt.len = len_eff;
         mt.nparts = pi.nparts;
         mt.blk_begin = blk_begin;
         mt.nblk = nblk;

@@ -265,7 +265,7 @@ def gpu_fp8_multi(b, partition_tokens=0, plan=False):
 
 
 @pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 4), (8, 8, 16), (16, 2, 2), (12, 4, 5),
-                                             (16, 1, 1)])
+                                             (16, 1, 1), (32, 8, 20), (16, 1, 3)])
 def test_fp8_multi_matches_oracle(cuda_device, hq, hkv, max_chunk):
     rng = np.random.default_rng(hq * 31 + hkv * 7 + max_chunk)
     lens = np.array([1, 2, 15, 16, 17, 33, 64, 100, 257, 300, 31, 48])

@@ -121,3 +121,25 @@ def test_chunk_outside_the_query_rows_is_skipped_and_flagged(cuda_device):
     b.query_start_loc = np.array([0, 2, 9], dtype=np.int32)   # rows 2..8 but q has 5 rows
     gpu_multi(b, max_query_len=16)
     assert pkv.device_error_bits() & pkv.DEVERR_LEN
+
+
+@pytest.mark.parametrize("hq,hkv,chunk_cap,partition", [(32, 8, 40, 0), (8, 8, 100, 0),
+                                                       (6, 2, 17, 0), (32, 8, 64, 256),
+                                                       (16, 1, 9, 48)])
+def test_long_chunks_in_row_groups(cuda_device, hq, hkv, chunk_cap, partition):
+    """Chunks longer than 16 query rows per kv head: split into row groups of whole
+    tokens, each reading only the keys its rows can see."""
+    rng = np.random.default_rng(hq * 13 + chunk_cap)
+    lens = np.array([1, 17, 40, 64, 100, 300, 1000, 33])
+    chunks = np.minimum(rng.integers(1, chunk_cap + 1, size=lens.shape[0]), lens)
+    chunks[1] = min(chunk_cap, lens[1])            # at least one chunk at the cap
+    b = workloads.chunked_batch(800 + hq + chunk_cap, lens, chunks, hq, hkv, 128, "bf16",
+                                device=cuda_device)
+    run_and_check(b, partition, f"rows in groups {hq}/{hkv} chunks<={chunk_cap} p{partition}")
+
+
+def test_whole_prompt_prefill_matches_oracle(cuda_device):
+    """Every sequence's whole context as its chunk (a prompt prefilled in one call)."""
+    lens = np.array([5, 16, 31, 77, 128])
+    b = workloads.chunked_batch(811, lens, lens.copy(), 8, 2, 64, "f32", device=cuda_device)
+    run_and_check(b, 0, "whole-prompt prefill fp32")
