@@ -1,4 +1,4 @@
-"""The C-ABI library loads, exports every entry point its header declares, and
+"""The C-ABI library loads, exports every entry point its headers declare, and
 its host-side logic (argument checks, workspace sizing, partition choice,
 copy-pair validation) behaves as documented.  No GPU is needed: nothing here
 launches a kernel."""
@@ -14,6 +14,8 @@ from paged_kv_cache_375_b200 import build as pkv_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "pkv.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+                 if f.endswith(".h"))
 
 
 @pytest.fixture(scope="module")
@@ -22,14 +24,17 @@ def lib():
     return pkv.load_library()
 
 
-def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+def declared_functions(headers=None):
+    names = set()
+    for h in headers or HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
-    names = declared_functions()
+    assert len(HEADERS) >= 2 and HEADER in HEADERS
+    names = declared_functions([HEADER])
     for required in ("pkv_paged_attention_decode", "pkv_reshape_and_cache", "pkv_copy_blocks",
                      "pkv_slot_mapping", "pkv_check_device_error", "pkv_decode_workspace_bytes"):
         assert required in names
