@@ -7,27 +7,29 @@
 // through the sequence's block table.
 //
 // How it runs on a B200:
-//  * A planning kernel turns context_lens into a work list of items
+//  * A planning step turns context_lens into a work list of items
 //    (sequence, partition), longest first.  A partition is at most
 //    `part_blocks` blocks; a sequence longer than one partition is split
 //    (split-K) and its partial results are merged by log-sum-exp afterwards.
-//  * The decode kernel is persistent (one CTA per SM).  Items (x every kv
-//    head) are handed out through an atomic counter.  Inside a CTA one
-//    producer warp walks the block table and issues a TMA tensor load per
-//    128-byte column chunk of each 16-token K and V tile (the tile of one
-//    (block, kv head) is contiguous in the HND pool) into 128B-swizzled
-//    shared memory, signalling an mbarrier; W consumer warps take the blocks
-//    of an item round-robin, each keeping its own online-softmax state, and
-//    merge their states at the end of the item.  The producer runs ahead
-//    across item boundaries, so the next item's tiles are already in flight
-//    while the current one is merged.
-//  * bf16: all query heads of a GQA group (g <= 16 rows) form the M side of
-//    mma.sync m16n8k16: S = Q K^T per 16-token tile, then O += P V.  Every KV
-//    tile is read from HBM once per group.
+//  * The decode kernel is persistent (one CTA per SM).  Work units (item x kv
+//    head x row group) are handed out through an atomic counter by a
+//    scheduler warp, which publishes each into a ring in shared memory: its
+//    metadata, its q rows (bulk copies) and its slice of the block table.
+//  * The decode warps take the blocks of an item round-robin.  Each warp (or
+//    the lead warp of a pair) owns a few tile stages and issues its own TMA
+//    tensor loads -- one per 128-byte column chunk of the 16-token K and V
+//    tiles, contiguous per (block, kv head) in the HND pool -- into
+//    128B-swizzled shared memory, running ahead across item boundaries.  At
+//    the end of an item the warps merge their online-softmax states.
+//  * bf16 and FP8: per pair of 16-token tiles, S^T = K Q^T on mma.sync
+//    (tile tokens = M, the item's query rows = N, up to 16), online softmax in
+//    log2 units with a lazily moved maximum, P^T through movmatrix, O^T +=
+//    V^T P^T, and the row sums by one more MMA.  Every KV tile is read from
+//    HBM once per GQA group.  FP8 codes are widened to f16 in registers.
 //  * fp32: the same pipeline with a CUDA-core consumer (fp32 has no exact
 //    tensor-core path; TF32 would break the fp32 tolerance).
-//  * Padding slots of the last block are never used: their scores are
-//    selected to -inf and their V values are masked to zero before the MMA
+//  * Padding slots of the last block are never used: their scores are set
+//    to -inf and their V values are masked to zero before the MMA
 //    (0 * NaN would otherwise poison the output).
 #pragma once
 
@@ -241,10 +243,10 @@ struct ItemMeta {
 // ---- consumer state for bf16 (tensor cores) ----
 //
 // Per 16-token tile the scores are computed transposed, S^T = K Q^T, with the
-// tile's tokens as the MMA's M (16) and the group's query heads as N (8 per
-// n-tile), so one m16n8k16 covers a k-step of the whole group.  The output is
-// kept transposed too, O^T += V^T P^T (M = head_dim in tiles of 16, N = the
-// heads, K = the tile's tokens); P^T reaches the B-fragment layout through
+// tile's tokens as the MMA's M (16) and the item's query rows (the GQA group's
+// heads, times the chunk's tokens) as N (8 per n-tile), so one m16n8k16 covers
+// a k-step of all of them.  The output is kept transposed too, O^T += V^T P^T
+// (M = head_dim in tiles of 16, N = the rows, K = the tile's tokens); P^T reaches the B-fragment layout through
 // movmatrix.  Two tiles are processed per step for instruction-level
 // parallelism.  The running max only moves when it grows by more than
 // kRescaleSlack (log2 units): weights then stay below 2^kRescaleSlack and the
@@ -874,9 +876,10 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& prm, const
 
 // The persistent decode kernel.  Warps 0..W-1 decode; warp W schedules.
 //
-// The scheduler warp fetches items from the global work counter and
-// publishes each into a ring slot: its metadata, its q tile (one bulk copy)
-// and the slice of the block table it covers.  Every lead decode warp (the
+// The scheduler warp fetches work units (item x kv head x row group) from the
+// global work counter and publishes each into a ring slot: its metadata, its
+// q rows (one bulk copy per chunk token) and the slice of the block table it
+// covers.  Every lead decode warp (the
 // first W / SPLIT) owns S tile stages and is its own TMA producer: it keeps up
 // to S of its blocks in flight, following its share of the items (blocks l,
 // l+L, ... of each, L = W / SPLIT) and running ahead into the next items
