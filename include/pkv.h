@@ -13,6 +13,11 @@
  *  - blocks shared by several sequences are reference counted and copied on
  *    write ("vLLM 深读：用 PagedAttention 撑起高并发 LLM 推理", section
  *    "先看浪费在哪里").
+ * Beyond one query token per sequence the same decode kernel serves chunks of
+ * several causal query tokens (pkv_paged_attention_multi), and pools of FP8
+ * (e4m3) codes with per-pool scales (the *_fp8 calls).  The host block
+ * manager that produces tables, slots and copy pairs is declared in
+ * pkv_block_manager.h.
  *
  * Conventions for every call:
  *  - Pointers are DEVICE pointers unless the argument says "host".  The caller
@@ -37,6 +42,7 @@
  *
  * Layouts (row-major, innermost last):
  *  - q, out         [num_seqs][num_q_heads][head_dim], dtype of the cache
+ *                   (bf16 for FP8 pools)
  *  - k, v (new)     [num_tokens][num_kv_heads][head_dim]
  *  - k_cache,v_cache[num_blocks][num_kv_heads][16][head_dim]  ("HND": one
  *                   (block, kv head) tile of 16 tokens is contiguous)
