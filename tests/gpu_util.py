@@ -25,10 +25,12 @@ def dev_i32(a: np.ndarray, device) -> torch.Tensor:
 
 
 def host_bits(t: torch.Tensor) -> np.ndarray:
-    """Host copy: float32 as is, bf16 as its uint16 bit patterns."""
+    """Host copy: float32 as is, bf16 as its uint16 bit patterns, e4m3 as its codes."""
     t = t.detach().contiguous().cpu()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.numpy()
 
 
