@@ -373,6 +373,9 @@ def run_ours(args, world, rank, local):
             "new_tokens_per_step": step.T, "cow_pairs_per_step": int(b.cow_pairs.shape[0]),
             "partition_tokens": step.part_tokens, "split_k": step.split,
             "kv_bytes_per_step": kv_bytes,
+            # KV-block usage of the pool (blocks holding tokens / pool size)
+            "blocks_in_use": int(b.meta.get("blocks_in_use", 0)),
+            "pool_usage": round(int(b.meta.get("blocks_in_use", 0)) / b.num_blocks, 4),
             **({"batch_override": args.batch} if args.batch else {}),
             "l2": ("L2 flushed before every step (a 252 MB write outside the timed events; "
                    "the working set is under 4x L2)" if flush else
