@@ -89,12 +89,22 @@ def _load():
             lib.oracle_paged_multi_fp8.argtypes = [P, P, P, P, f32, f32, P, P, P, i32, i32, i32,
                                                    i32, i32, i64, i32, f32, i32]
             lib.oracle_e4m3_quantize.argtypes = [P, i64, f32, P]
+            lib.oracle_e5m2_quantize.argtypes = [P, i64, f32, P]
+            lib.oracle_e5m2_values.argtypes = [P, i64, P]
+            lib.oracle_reshape_and_cache_e5m2.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i64,
+                                                          f32, f32]
+            lib.oracle_paged_decode_e5m2.argtypes = [P, P, P, P, f32, f32, P, P, i32, i32, i32,
+                                                     i32, i32, i64, i32, f32, P, i64, i32]
+            lib.oracle_paged_multi_e5m2.argtypes = [P, P, P, P, f32, f32, P, P, P, i32, i32, i32,
+                                                    i32, i32, i64, i32, f32, i32]
             lib.oracle_e4m3_values.argtypes = [P, i64, P]
             lib.oracle_lse_merge_f32.argtypes = [P, P, P, i32, i32, P]
             for name in ("oracle_slot_mapping", "oracle_reshape_and_cache",
                          "oracle_copy_blocks", "oracle_paged_decode", "oracle_paged_multi",
                          "oracle_paged_decode_fp8", "oracle_reshape_and_cache_fp8",
-                         "oracle_paged_multi_fp8",
+                         "oracle_paged_multi_fp8", "oracle_e5m2_quantize",
+                         "oracle_e5m2_values", "oracle_reshape_and_cache_e5m2",
+                         "oracle_paged_decode_e5m2", "oracle_paged_multi_e5m2",
                          "oracle_e4m3_quantize", "oracle_e4m3_values",
                          "oracle_partition_stats", "oracle_lse_merge",
                          "oracle_lse_merge_f32"):
@@ -213,6 +223,22 @@ def e4m3_quantize(x: np.ndarray, scale: float = 1.0) -> np.ndarray:
     return out
 
 
+def e5m2_quantize(x: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """uint8 e5m2 codes of float32 x / scale (the division in float32)."""
+    xf = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(xf.shape, dtype=np.uint8)
+    _check(_load().oracle_e5m2_quantize(_ptr(xf), xf.size, float(scale), _ptr(out)))
+    return out
+
+
+def e5m2_values(codes: np.ndarray) -> np.ndarray:
+    """Exact values of e5m2 codes (no scale), as float64."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _check(_load().oracle_e5m2_values(_ptr(c), c.size, _ptr(out)))
+    return out
+
+
 def e4m3_values(codes: np.ndarray) -> np.ndarray:
     """Exact values of e4m3 codes (no scale), as float64."""
     c = np.ascontiguousarray(codes, dtype=np.uint8)
@@ -221,23 +247,31 @@ def e4m3_values(codes: np.ndarray) -> np.ndarray:
     return out
 
 
+_FP8 = ("e4m3", "e5m2")
+
+
 def reshape_and_cache_fp8(k: np.ndarray, v: np.ndarray, k_cache: np.ndarray,
                           v_cache: np.ndarray, slot_mapping_: np.ndarray, k_scale: float,
-                          v_scale: float) -> None:
-    """In place on uint8 e4m3 pools [NB][Hkv][BS][D]; k, v are bf16 bits [T][Hkv][D]."""
+                          v_scale: float, fmt: str = "e4m3") -> None:
+    """In place on uint8 FP8 pools [NB][Hkv][BS][D] (fmt "e4m3" or "e5m2"); k, v are bf16
+    bits [T][Hkv][D]."""
+    assert fmt in _FP8
     sm = np.ascontiguousarray(slot_mapping_, dtype=np.int64)
     nb, hkv, bs, d = k_cache.shape
     assert k.dtype == np.uint16 and k_cache.dtype == np.uint8 and k.shape[1:] == (hkv, d)
-    _check(_load().oracle_reshape_and_cache_fp8(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache),
-                                                _ptr(sm), sm.shape[0], hkv, d, bs, nb,
-                                                float(k_scale), float(v_scale)))
+    fn = (_load().oracle_reshape_and_cache_fp8 if fmt == "e4m3" else
+          _load().oracle_reshape_and_cache_e5m2)
+    _check(fn(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(sm), sm.shape[0], hkv, d, bs,
+              nb, float(k_scale), float(v_scale)))
 
 
 def paged_decode_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_scale: float,
                      v_scale: float, block_tables: np.ndarray, context_lens: np.ndarray,
                      scale: float, tasks: np.ndarray | None = None,
-                     threads: int | None = None) -> np.ndarray:
-    """Float64 decode over e4m3 pools (uint8 codes times the pool's scale); q is bf16 bits."""
+                     threads: int | None = None, fmt: str = "e4m3") -> np.ndarray:
+    """Float64 decode over FP8 pools (uint8 codes times the pool's scale; fmt "e4m3" or
+    "e5m2"); q is bf16 bits."""
+    assert fmt in _FP8
     assert q.dtype == np.uint16 and k_cache.dtype == np.uint8 == v_cache.dtype
     B, Hq, D = q.shape
     NB, Hkv, BS, _ = k_cache.shape
@@ -251,18 +285,20 @@ def paged_decode_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_
         tk = np.ascontiguousarray(tasks, dtype=np.int32).reshape(-1, 2)
         out = np.empty((tk.shape[0], D), dtype=np.float64)
         tp, n = _ptr(tk), tk.shape[0]
-    _check(_load().oracle_paged_decode_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                           float(k_scale), float(v_scale), _ptr(bt), _ptr(cl),
-                                           B, Hq, Hkv, D, BS, NB, bt.shape[1], float(scale), tp,
-                                           n, threads))
+    fn = _load().oracle_paged_decode_fp8 if fmt == "e4m3" else _load().oracle_paged_decode_e5m2
+    _check(fn(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale),
+              _ptr(bt), _ptr(cl), B, Hq, Hkv, D, BS, NB, bt.shape[1], float(scale), tp, n,
+              threads))
     return out
 
 
 def paged_multi_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_scale: float,
                     v_scale: float, block_tables: np.ndarray, context_lens: np.ndarray,
                     query_start_loc: np.ndarray, scale: float,
-                    threads: int | None = None) -> np.ndarray:
-    """paged_multi over e4m3 pools (uint8 codes times the pool's scale); q is bf16 bits."""
+                    threads: int | None = None, fmt: str = "e4m3") -> np.ndarray:
+    """paged_multi over FP8 pools (uint8 codes times the pool's scale; fmt "e4m3" or
+    "e5m2"); q is bf16 bits."""
+    assert fmt in _FP8
     assert q.dtype == np.uint16 and k_cache.dtype == np.uint8 == v_cache.dtype
     T, Hq, D = q.shape
     NB, Hkv, BS, _ = k_cache.shape
@@ -272,10 +308,10 @@ def paged_multi_fp8(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_s
     assert qsl.shape[0] == cl.shape[0] + 1 and qsl[-1] <= T
     out = np.zeros((T, Hq, D), dtype=np.float64)
     threads = threads or len(os.sched_getaffinity(0))
-    _check(_load().oracle_paged_multi_fp8(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                          float(k_scale), float(v_scale), _ptr(bt), _ptr(cl),
-                                          _ptr(qsl), cl.shape[0], Hq, Hkv, D, BS, NB,
-                                          bt.shape[1], float(scale), threads))
+    fn = _load().oracle_paged_multi_fp8 if fmt == "e4m3" else _load().oracle_paged_multi_e5m2
+    _check(fn(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale),
+              _ptr(bt), _ptr(cl), _ptr(qsl), cl.shape[0], Hq, Hkv, D, BS, NB, bt.shape[1],
+              float(scale), threads))
     return out
 
 

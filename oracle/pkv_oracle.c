@@ -58,7 +58,12 @@ enum {
     ORACLE_NO_MEMORY = 6
 };
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 2, ORACLE_E5M2 = 3 };
+
+static int is_fp8(int dtype)
+{
+    return dtype == ORACLE_E4M3 || dtype == ORACLE_E5M2;
+}
 
 /* ------------------------------------------------------------------------- */
 /* FP8 E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; no
@@ -115,6 +120,82 @@ static uint8_t e4m3_encode(float y)
     return sign | (uint8_t)(((unbiased + 7) << 3) | ((int)steps - 8));
 }
 
+/* FP8 E5M2 (1 sign bit, 5 exponent bits with bias 15, 2 mantissa bits, the
+ * IEEE-style layout of the upper byte of a binary16: exponent 31 holds the
+ * infinities (mantissa 0) and NaNs, so the largest finite value is
+ * 1.75 * 2^15 = 57344; exponent 0 holds the subnormals m * 2^-16).  The same
+ * reading of "quantise" as for e4m3: divide in single precision, round to the
+ * nearest representable value with ties to even, saturate to +-57344 instead
+ * of overflowing, keep NaN. */
+static double e5m2_value(uint8_t code)
+{
+    const int sign = code >> 7, exp = (code >> 2) & 31, man = code & 3;
+    double v;
+    if (exp == 31) {
+        v = man == 0 ? INFINITY : NAN;
+    } else if (exp == 0) {
+        v = ldexp((double)man, -16);
+    } else {
+        v = ldexp(1.0 + man / 4.0, exp - 15);
+    }
+    return sign ? -v : v;
+}
+
+static uint8_t e5m2_encode(float y)
+{
+    if (isnan(y)) {
+        return 0x7f;
+    }
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a = fabs((double)y);
+    if (a >= 57344.0) {
+        return sign | 0x7b;                       /* saturate (infinities too) */
+    }
+    int e;
+    frexp(a, &e);                                 /* a = f * 2^e, 0.5 <= f < 1 */
+    int unbiased = e - 1;                         /* a in [2^unbiased, 2^(unbiased+1)) */
+    if (a == 0.0 || unbiased < -14) {
+        unbiased = -14;                           /* subnormal range: steps of 2^-16 */
+    }
+    /* number of 2^(unbiased-2) steps, rounded to nearest, ties to even */
+    double steps = rint(ldexp(a, 2 - unbiased));
+    if (steps >= 8.0) {                           /* rounded up into the next binade */
+        unbiased += 1;
+        steps = 4.0;
+    }
+    if (unbiased > 15) {
+        return sign | 0x7b;                       /* beyond 57344 after rounding */
+    }
+    if (steps < 4.0) {                            /* subnormal */
+        return sign | (uint8_t)steps;
+    }
+    return sign | (uint8_t)(((unbiased + 15) << 2) | ((int)steps - 4));
+}
+
+/* Encode n floats: out[i] = e5m2(x[i] / scale), the division in float. */
+int oracle_e5m2_quantize(const float *x, int64_t n, float scale, uint8_t *out)
+{
+    if ((!x || !out) && n > 0) {
+        return 1;
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        out[i] = e5m2_encode(x[i] / scale);
+    }
+    return 0;
+}
+
+/* Decode n e5m2 codes to doubles (exact values, without any scale). */
+int oracle_e5m2_values(const uint8_t *codes, int64_t n, double *out)
+{
+    if ((!codes || !out) && n > 0) {
+        return 1;
+    }
+    for (int64_t i = 0; i < n; ++i) {
+        out[i] = e5m2_value(codes[i]);
+    }
+    return 0;
+}
+
 /* Encode n floats: out[i] = e4m3(x[i] / scale), the division in float. */
 int oracle_e4m3_quantize(const float *x, int64_t n, float scale, uint8_t *out)
 {
@@ -150,6 +231,9 @@ static double widen(const void *base, int64_t index, int dtype)
     }
     if (dtype == ORACLE_E4M3) {
         return e4m3_value(((const uint8_t *)base)[index]);
+    }
+    if (dtype == ORACLE_E5M2) {
+        return e5m2_value(((const uint8_t *)base)[index]);
     }
     uint32_t bits = (uint32_t)((const uint16_t *)base)[index] << 16;
     float f;
@@ -225,11 +309,40 @@ int oracle_reshape_and_cache(const void *k, const void *v, void *k_cache,
 /* reshape_and_cache into FP8 (e4m3) pools: token t's bf16 K and V values are
  * quantised (code = e4m3(value / scale), the division in float) and written
  * at slot_mapping[t]. */
+static int reshape_and_cache_f8(const uint16_t *k, const uint16_t *v, uint8_t *k_cache,
+                                uint8_t *v_cache, const int64_t *slot_mapping,
+                                int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int64_t num_blocks, float k_scale,
+                                float v_scale, uint8_t (*encode)(float));
+
 int oracle_reshape_and_cache_fp8(const uint16_t *k, const uint16_t *v, uint8_t *k_cache,
                                  uint8_t *v_cache, const int64_t *slot_mapping,
                                  int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
                                  int32_t block_size, int64_t num_blocks, float k_scale,
                                  float v_scale)
+{
+    return reshape_and_cache_f8(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                num_kv_heads, head_dim, block_size, num_blocks, k_scale,
+                                v_scale, e4m3_encode);
+}
+
+/* The same into e5m2 pools: code = e5m2(value / scale). */
+int oracle_reshape_and_cache_e5m2(const uint16_t *k, const uint16_t *v, uint8_t *k_cache,
+                                  uint8_t *v_cache, const int64_t *slot_mapping,
+                                  int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t block_size, int64_t num_blocks, float k_scale,
+                                  float v_scale)
+{
+    return reshape_and_cache_f8(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                num_kv_heads, head_dim, block_size, num_blocks, k_scale,
+                                v_scale, e5m2_encode);
+}
+
+static int reshape_and_cache_f8(const uint16_t *k, const uint16_t *v, uint8_t *k_cache,
+                                uint8_t *v_cache, const int64_t *slot_mapping,
+                                int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int64_t num_blocks, float k_scale,
+                                float v_scale, uint8_t (*encode)(float))
 {
     if (!k || !v || !k_cache || !v_cache || !slot_mapping || num_tokens < 0 ||
         num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0) {
@@ -251,8 +364,8 @@ int oracle_reshape_and_cache_fp8(const uint16_t *k, const uint16_t *v, uint8_t *
                 size_t src = ((size_t)t * num_kv_heads + h) * head_dim + d;
                 size_t dst = (((size_t)block * num_kv_heads + h) * block_size + offset) *
                                  head_dim + d;
-                k_cache[dst] = e4m3_encode((float)widen(k, (int64_t)src, ORACLE_BF16) / k_scale);
-                v_cache[dst] = e4m3_encode((float)widen(v, (int64_t)src, ORACLE_BF16) / v_scale);
+                k_cache[dst] = encode((float)widen(k, (int64_t)src, ORACLE_BF16) / k_scale);
+                v_cache[dst] = encode((float)widen(v, (int64_t)src, ORACLE_BF16) / v_scale);
             }
         }
     }
@@ -322,7 +435,7 @@ typedef struct {
 
 static int q_dtype(const problem *pb)
 {
-    return pb->dtype == ORACLE_E4M3 ? ORACLE_BF16 : pb->dtype;
+    return is_fp8(pb->dtype) ? ORACLE_BF16 : pb->dtype;
 }
 
 /* Gather the contiguous K and V rows [0, len) of (seq, kv_head) by walking the
@@ -527,7 +640,7 @@ static int paged_decode_scaled(double *out, const void *q, const void *k_cache,
                                const int32_t *tasks, int64_t num_tasks, int32_t num_threads)
 {
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
-        (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && dtype != ORACLE_E4M3) ||
+        (dtype != ORACLE_F32 && dtype != ORACLE_BF16 && !is_fp8(dtype)) ||
         num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
         num_q_heads % num_kv_heads != 0 || head_dim <= 0 || block_size <= 0 ||
         num_blocks <= 0 || max_blocks_per_seq <= 0 || num_tasks < 0) {
@@ -673,6 +786,21 @@ int oracle_paged_multi(double *out, const void *q, const void *k_cache, const vo
 
 /* The same over FP8 (e4m3) pools: q is bf16; each cached element is its code's
  * value times k_scale (K pool) or v_scale (V pool). */
+/* Decode over e5m2 pools (as oracle_paged_decode_fp8). */
+int oracle_paged_decode_e5m2(double *out, const void *q, const void *k_cache,
+                             const void *v_cache, float k_scale, float v_scale,
+                             const int32_t *block_tables, const int32_t *context_lens,
+                             int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                             int32_t head_dim, int32_t block_size, int64_t num_blocks,
+                             int32_t max_blocks_per_seq, float scale,
+                             const int32_t *tasks, int64_t num_tasks, int32_t num_threads)
+{
+    return paged_decode_scaled(out, q, k_cache, v_cache, ORACLE_E5M2, k_scale, v_scale,
+                               block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                               head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
+                               tasks, num_tasks, num_threads);
+}
+
 int oracle_paged_multi_fp8(double *out, const void *q, const void *k_cache, const void *v_cache,
                            float k_scale, float v_scale, const int32_t *block_tables,
                            const int32_t *context_lens, const int32_t *query_start_loc,
@@ -681,6 +809,21 @@ int oracle_paged_multi_fp8(double *out, const void *q, const void *k_cache, cons
                            int32_t max_blocks_per_seq, float scale, int32_t num_threads)
 {
     return paged_multi_scaled(out, q, k_cache, v_cache, ORACLE_E4M3, k_scale, v_scale,
+                              block_tables, context_lens, query_start_loc, num_seqs, num_q_heads,
+                              num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
+                              scale, num_threads);
+}
+
+/* Several query tokens over e5m2 pools. */
+int oracle_paged_multi_e5m2(double *out, const void *q, const void *k_cache,
+                            const void *v_cache, float k_scale, float v_scale,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            const int32_t *query_start_loc, int32_t num_seqs, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int64_t num_blocks, int32_t max_blocks_per_seq, float scale,
+                            int32_t num_threads)
+{
+    return paged_multi_scaled(out, q, k_cache, v_cache, ORACLE_E5M2, k_scale, v_scale,
                               block_tables, context_lens, query_start_loc, num_seqs, num_q_heads,
                               num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq,
                               scale, num_threads);
@@ -784,7 +927,7 @@ int oracle_partition_stats(const void *q, const void *k_cache, const void *v_cac
     const int32_t kv_head = q_head / (num_q_heads / num_kv_heads);
     for (int32_t d = 0; d < D; ++d) {
         qrow[d] = widen(q, ((int64_t)seq * num_q_heads + q_head) * D + d,
-                        dtype == ORACLE_E4M3 ? ORACLE_BF16 : dtype);
+                        is_fp8(dtype) ? ORACLE_BF16 : dtype);
     }
     st = gather_context(&pb, seq, kv_head, L, K, V);
     if (st == ORACLE_OK) {

@@ -48,6 +48,11 @@ MUTANTS = {
                              "return sign | (uint8_t)(((unbiased + 8) << 3) | ((int)steps - 8));"),
     "e4m3_no_saturation": ("        return sign | 0x7e;                       /* saturate */",
                            "        return sign | 0x7f;                       /* saturate */"),
+    "e5m2_bias_off_by_one": ("return sign | (uint8_t)(((unbiased + 15) << 2) | ((int)steps - 4));",
+                             "return sign | (uint8_t)(((unbiased + 16) << 2) | ((int)steps - 4));"),
+    "e5m2_value_three_mantissa_bits": ("v = ldexp(1.0 + man / 4.0, exp - 15);",
+                                       "v = ldexp(1.0 + man / 8.0, exp - 15);"),
+    "e5m2_subnormal_step": ("v = ldexp((double)man, -16);", "v = ldexp((double)man, -15);"),
     "fp8_scale_dropped": ("V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype) * pb->v_scale;",
                           "V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype);"),
 }

@@ -543,6 +543,109 @@ def test_e4m3_divides_by_the_scale_in_float():
     assert np.array_equal(oracle.e4m3_quantize(x, 0.5), oracle.e4m3_quantize(x / np.float32(0.5)))
 
 
+# ------------------------------------------------------------- FP8 (e5m2) ----
+def test_golden_e5m2_examples():
+    g = _golden("e5m2_examples.json")
+    codes = oracle.e5m2_quantize(np.array(g["values"], dtype=np.float32))
+    assert codes.tolist() == g["codes"]
+
+
+def test_e5m2_every_finite_code_round_trips_and_specials():
+    codes = np.array([c for c in range(256) if (c >> 2) & 31 != 31], dtype=np.uint8)
+    vals = oracle.e5m2_values(codes)
+    assert np.isfinite(vals).all() and np.abs(vals).max() == 57344.0
+    assert np.array_equal(oracle.e5m2_quantize(vals.astype(np.float32)), codes)
+    assert np.isinf(oracle.e5m2_values(np.array([0x7c, 0xfc], dtype=np.uint8))).all()
+    assert np.isnan(oracle.e5m2_values(np.array([0x7d, 0x7e, 0x7f, 0xff], dtype=np.uint8))).all()
+
+
+def test_e5m2_values_are_the_upper_byte_of_binary16():
+    """An e5m2 code is the upper byte of an IEEE binary16 with the lower byte zero."""
+    codes = np.arange(256, dtype=np.uint8)
+    f16 = (codes.astype(np.uint16) << 8).view(np.float16).astype(np.float64)
+    vals = oracle.e5m2_values(codes)
+    same = np.isnan(f16) == np.isnan(vals)
+    assert same.all()
+    ok = ~np.isnan(f16)
+    assert np.array_equal(f16[ok], vals[ok])
+
+
+def test_e5m2_rounds_to_the_nearest_value_ties_to_even():
+    rng = np.random.default_rng(33)
+    x = np.concatenate([rng.standard_normal(3000) * 10.0 ** rng.uniform(-6, 4.5, 3000),
+                        rng.uniform(-60000, 60000, 200)]).astype(np.float32)
+    codes = oracle.e5m2_quantize(x)
+    grid_codes = np.array([c for c in range(256) if (c >> 2) & 31 != 31], dtype=np.uint8)
+    grid = oracle.e5m2_values(grid_codes)
+    for xi, ci in zip(x.astype(np.float64), codes):
+        if abs(xi) >= 57344.0:
+            assert oracle.e5m2_values(np.array([ci]))[0] == np.copysign(57344.0, xi)
+            continue
+        d = np.abs(grid - xi)
+        best = grid_codes[d == d.min()]
+        if len(best) > 1:                                   # a tie: the even mantissa wins
+            best = [c for c in best if (c & 1) == 0 and (c & 0x80) == (ci & 0x80)] or best
+        assert ci in best, (xi, ci, best)
+
+
+def test_e5m2_agrees_with_torch_in_range():
+    """Inside the finite range torch's float32 -> float8_e5m2 cast rounds to nearest even
+    as well (outside it torch overflows to infinity where the KV cache saturates)."""
+    rng = np.random.default_rng(34)
+    x = (rng.standard_normal(5000) * 10.0 ** rng.uniform(-5, 4, 5000)).astype(np.float32)
+    x = x[np.abs(x) < 57344.0]
+    want = torch.from_numpy(x).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e5m2_quantize(x), want)
+
+
+def test_e5m2_decode_and_multi_match_dense_attention():
+    rng = np.random.default_rng(35)
+    lens, chunks = [1, 16, 33, 70], [1, 3, 5, 16]
+    hq, hkv, d = 8, 2, 32
+    q32, kp32, vp32, bt, cl, _, _, _ = random_paged(rng, lens, hq, hkv, d)
+    k_scale, v_scale = np.float32(0.05), np.float32(0.02)
+    kc = oracle.e5m2_quantize(np.nan_to_num(kp32), k_scale)
+    vc = oracle.e5m2_quantize(np.nan_to_num(vp32), v_scale)
+    kd = oracle.e5m2_values(kc) * float(k_scale)
+    vd = oracle.e5m2_values(vc) * float(v_scale)
+    qb = to_bf16_bits(q32)
+    out = oracle.paged_decode_fp8(qb, kc, vc, k_scale, v_scale, bt, cl, 0.125, fmt="e5m2")
+    qf = bf16_bits_to_f64(qb)
+    ctx = []
+    for s, L in enumerate(lens):
+        nb = (L + BS - 1) // BS
+        K = kd[bt[s, :nb]].transpose(0, 2, 1, 3).reshape(nb * BS, hkv, d)[:L]
+        V = vd[bt[s, :nb]].transpose(0, 2, 1, 3).reshape(nb * BS, hkv, d)[:L]
+        ctx.append((K, V))
+        np.testing.assert_allclose(out[s], dense_attention(qf[s], K, V, 0.125), rtol=0,
+                                   atol=1e-12)
+    qsl = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    qm = to_bf16_bits(rng.standard_normal((int(qsl[-1]), hq, d)).astype(np.float32))
+    outm = oracle.paged_multi_fp8(qm, kc, vc, k_scale, v_scale, bt, cl, qsl, 0.2, fmt="e5m2")
+    qmf = bf16_bits_to_f64(qm)
+    for s, (L, n) in enumerate(zip(lens, chunks)):
+        K, V = ctx[s]
+        for i in range(n):
+            p = L - n + i
+            np.testing.assert_allclose(outm[qsl[s] + i], dense_attention(
+                qmf[qsl[s] + i], K[:p + 1], V[:p + 1], 0.2), rtol=0, atol=1e-12)
+
+
+def test_e5m2_reshape_quantises_into_the_slot():
+    rng = np.random.default_rng(36)
+    kf = (rng.standard_normal((3, 2, 16)) * 30).astype(np.float32)
+    vf = (rng.standard_normal((3, 2, 16)) * 30).astype(np.float32)
+    k, v = to_bf16_bits(kf), to_bf16_bits(vf)
+    kf, vf = bf16_bits_to_f64(k).astype(np.float32), bf16_bits_to_f64(v).astype(np.float32)
+    kc = np.zeros((4, 2, 16, 16), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    oracle.reshape_and_cache_fp8(k, v, kc, vc, np.array([5, -1, 50], dtype=np.int64), 0.5,
+                                 0.25, fmt="e5m2")
+    assert np.array_equal(kc[0, :, 5], oracle.e5m2_quantize(kf[0], 0.5))
+    assert np.array_equal(vc[3, :, 2], oracle.e5m2_quantize(vf[2], 0.25))
+    assert kc.astype(np.int64).sum() == oracle.e5m2_quantize(kf[[0, 2]], 0.5).astype(np.int64).sum()
+
+
 def test_fp8_decode_matches_dense_attention_on_dequantised_values():
     rng = np.random.default_rng(31)
     lens = [1, 16, 33, 70]
