@@ -44,7 +44,7 @@ METRIC = "paged decode attn: KV-read GB/s (% of B200 HBM peak), seqs/s at batch"
 UNIT = "GB/s"
 WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shared_prefix",
              "c5": "c5_long_splitk", "c1": "c1_tiny_fp32", "c3spec": "c3_spec_decode",
-             "c3fp8": "c3_fp8", "c3specfp8": "c3_spec_fp8"}
+             "c3fp8": "c3_fp8", "c3specfp8": "c3_spec_fp8", "c3e5m2": "c3_fp8e5m2"}
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 << 20       # B200 L2; working sets below 4x this are flushed between steps
 DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
@@ -247,7 +247,7 @@ class Step:
 
     def write_new(self, slots):
         b = self.b
-        if b.dtype == "fp8":
+        if workloads.fp8_format(b.dtype):
             self.pkv.reshape_and_cache_fp8(b.new_k, b.new_v, b.k_cache, b.v_cache, slots,
                                            b.k_scale, b.v_scale)
         else:
@@ -265,14 +265,14 @@ class Step:
                                             workspace_tensor=self.ws, **extra)
 
     def decode(self):
-        if self.multi and self.b.dtype == "fp8":
+        if self.multi and workloads.fp8_format(self.b.dtype):
             self.plan_obj.run_multi_fp8(self.out, self.b.q, self.b.k_cache, self.b.v_cache,
                                         self.qsl, self.b.max_query_len, self.b.scale,
                                         self.b.k_scale, self.b.v_scale)
         elif self.multi:
             self.plan_obj.run_multi(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.qsl,
                                     self.b.max_query_len, self.b.scale)
-        elif self.b.dtype == "fp8":
+        elif workloads.fp8_format(self.b.dtype):
             self.plan_obj.run_fp8(self.out, self.b.q, self.b.k_cache, self.b.v_cache, self.b.scale,
                                   self.b.k_scale, self.b.v_scale)
         else:
@@ -579,12 +579,13 @@ def oracle_step(b: workloads.Batch, host: dict, seqs: np.ndarray | None, threads
     k, v = host["k_cache"], host["v_cache"]
     if b.cow_pairs.shape[0]:
         oracle.copy_blocks(k, v, b.cow_pairs)
-    fp8 = b.dtype == "fp8"
+    fmt = workloads.fp8_format(b.dtype)
+    fp8 = fmt is not None
     if b.new_seq.shape[0]:
         slots = oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos)
         if fp8:
             oracle.reshape_and_cache_fp8(host["new_k"], host["new_v"], k, v, slots, b.k_scale,
-                                         b.v_scale)
+                                         b.v_scale, fmt=fmt)
         else:
             oracle.reshape_and_cache(host["new_k"], host["new_v"], k, v, slots)
     if b.query_start_loc is not None:          # several query tokens per sequence
@@ -595,14 +596,16 @@ def oracle_step(b: workloads.Batch, host: dict, seqs: np.ndarray | None, threads
         q = np.ascontiguousarray(host["q"][rows])
         if fp8:
             return oracle.paged_multi_fp8(q, k, v, b.k_scale, b.v_scale, b.block_tables[sel],
-                                          b.context_lens[sel], sub_qsl, b.scale, threads=threads)
+                                          b.context_lens[sel], sub_qsl, b.scale, threads=threads,
+                                          fmt=fmt)
         return oracle.paged_multi(q, k, v, b.block_tables[sel], b.context_lens[sel], sub_qsl,
                                   b.scale, threads=threads)
     tasks = None if seqs is None else np.array([(s, h) for s in seqs
                                                 for h in range(b.num_q_heads)], dtype=np.int32)
     if fp8:
         return oracle.paged_decode_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
-                                       b.context_lens, b.scale, tasks=tasks, threads=threads)
+                                       b.context_lens, b.scale, tasks=tasks, threads=threads,
+                                       fmt=fmt)
     return oracle.paged_decode(host["q"], k, v, b.block_tables, b.context_lens, b.scale,
                                tasks=tasks, threads=threads)
 

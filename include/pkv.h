@@ -83,8 +83,10 @@ typedef enum pkv_status {
 typedef enum pkv_dtype {
     PKV_F32 = 0,       /* IEEE binary32 */
     PKV_BF16 = 1,      /* bfloat16; arithmetic in fp32, output rounded to nearest even */
-    PKV_FP8_E4M3 = 2   /* caches hold FP8 e4m3 codes (one byte; value = code x the pool's
+    PKV_FP8_E4M3 = 2,  /* caches hold FP8 e4m3 codes (one byte; value = code x the pool's
                           scale); q, out and the new K/V are bf16; head_dim 128 only */
+    PKV_FP8_E5M2 = 3   /* the same with e5m2 codes (1-5-2, bias 15: the upper byte of an
+                          IEEE binary16; widening to f16 is a byte move) */
 } pkv_dtype;
 
 /* Bits of the per-device error word. */
@@ -307,7 +309,8 @@ pkv_status pkv_decode_prepare_fp8(const void *k, const void *v, void *k_cache, v
  *    over e4m3 pools with their k_scale and v_scale; q and out are bf16.
  *    Arithmetic: codes are widened exactly to f16, q is rounded to f16
  *    (|q| above 65504 saturates), products accumulate in fp32.
- * dims->dtype must be PKV_FP8_E4M3 (the plain calls reject it); copy_blocks,
+ * dims->dtype must be PKV_FP8_E4M3 or PKV_FP8_E5M2 (the plain calls reject
+ * both; for e5m2 read e5m2 for e4m3 above, saturating to +-57344); copy_blocks,
  * slot mapping and the planner work on FP8 pools unchanged.
  */
 pkv_status pkv_reshape_and_cache_fp8(const void *k, const void *v, void *k_cache, void *v_cache,

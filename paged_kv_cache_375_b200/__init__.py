@@ -32,7 +32,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpkv.so")
 
-PKV_F32, PKV_BF16, PKV_FP8_E4M3 = 0, 1, 2
+PKV_F32, PKV_BF16, PKV_FP8_E4M3, PKV_FP8_E5M2 = 0, 1, 2, 3
+FP8_DTYPES = (torch.float8_e4m3fn, torch.float8_e5m2)   # pool dtypes of the *_fp8 calls
 DEVERR_BLOCK, DEVERR_SLOT, DEVERR_LEN, DEVERR_PAIR, DEVERR_POS, DEVERR_TIMEOUT = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
 
@@ -137,7 +138,10 @@ def _dtype_code(t: torch.dtype) -> int:
         return PKV_F32
     if t == torch.float8_e4m3fn:
         return PKV_FP8_E4M3
-    raise TypeError(f"dtype {t} not supported (bfloat16, float32 or float8_e4m3fn caches)")
+    if t == torch.float8_e5m2:
+        return PKV_FP8_E5M2
+    raise TypeError(f"dtype {t} not supported (bfloat16, float32, float8_e4m3fn or float8_e5m2 "
+                    "caches)")
 
 
 def _stream_ptr(device: torch.device):
@@ -146,6 +150,13 @@ def _stream_ptr(device: torch.device):
 
 def _p(t: torch.Tensor | None):
     return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _need_fp8_pools(k_cache: torch.Tensor, v_cache: torch.Tensor, device):
+    _need(k_cache, "k_cache", device=device)
+    if k_cache.dtype not in FP8_DTYPES:
+        raise TypeError(f"k_cache must be float8_e4m3fn or float8_e5m2, got {k_cache.dtype}")
+    _need(v_cache, "v_cache", k_cache.dtype, device)
 
 
 def _need(t: torch.Tensor, name: str, dtype=None, device=None):
@@ -287,8 +298,7 @@ def _check_fp8_decode(out, q, k_cache, v_cache, block_tables, context_lens):
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(out, "out", torch.bfloat16, dev)
-    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
-    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need_fp8_pools(k_cache, v_cache, dev)
     _need(block_tables, "block_tables", torch.int32, dev)
     _need(context_lens, "context_lens", torch.int32, dev)
     if k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
@@ -305,7 +315,7 @@ def paged_attention_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torc
                                v_scale: float, *, max_context_len: int | None = None,
                                partition_tokens: int = 0,
                                workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
-    """paged_attention_decode over FP8 (float8_e4m3fn) caches whose elements stand for
+    """paged_attention_decode over FP8 (float8_e4m3fn or float8_e5m2) caches whose elements stand for
     code * k_scale and code * v_scale; q and out are bfloat16, head_dim 128."""
     _check_fp8_decode(out, q, k_cache, v_cache, block_tables, context_lens)
     dev = q.device
@@ -328,13 +338,12 @@ def paged_attention_multi_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch
                               scale: float, k_scale: float, v_scale: float, max_query_len: int,
                               *, max_context_len: int | None = None, partition_tokens: int = 0,
                               workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
-    """paged_attention_multi over FP8 (float8_e4m3fn) pools with their scales; q and out
+    """paged_attention_multi over FP8 (float8_e4m3fn or float8_e5m2) pools with their scales; q and out
     are bfloat16, head_dim 128."""
     dev = q.device
     _need(q, "q", torch.bfloat16, dev)
     _need(out, "out", torch.bfloat16, dev)
-    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
-    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need_fp8_pools(k_cache, v_cache, dev)
     _need(block_tables, "block_tables", torch.int32, dev)
     _need(context_lens, "context_lens", torch.int32, dev)
     _need(query_start_loc, "query_start_loc", torch.int32, dev)
@@ -400,7 +409,7 @@ class DecodePlan:
                                        _p(self.workspace), self.workspace.numel(),
                                        _stream_ptr(dev)))
             return
-        fp8 = k_cache.dtype == torch.float8_e4m3fn
+        fp8 = k_cache.dtype in FP8_DTYPES
         src = torch.bfloat16 if fp8 else k_cache.dtype
         _need(new_k, "new_k", src, dev)
         _need(new_v, "new_v", src, dev)
@@ -455,8 +464,7 @@ class DecodePlan:
         dev = q.device
         _need(q, "q", torch.bfloat16, dev)
         _need(out, "out", torch.bfloat16, dev)
-        _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
-        _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+        _need_fp8_pools(k_cache, v_cache, dev)
         _need(query_start_loc, "query_start_loc", torch.int32, dev)
         lib = load_library()
         need = lib.pkv_multi_workspace_bytes(ctypes.byref(self.dims), q.shape[0],
@@ -496,7 +504,9 @@ class DecodePlan:
         if q.shape[0] != self.dims.num_seqs or tuple(k_cache.shape) != (
                 self.dims.num_blocks, self.dims.num_kv_heads, 16, self.dims.head_dim):
             raise ValueError("inconsistent shapes")
-        dims = PkvDims(*[getattr(self.dims, f) for f, _ in PkvDims._fields_[:-1]], PKV_FP8_E4M3)
+        # the pools' own FP8 format (the plan itself does not depend on it)
+        dims = PkvDims(*[getattr(self.dims, f) for f, _ in PkvDims._fields_[:-1]],
+                       _dtype_code(k_cache.dtype))
         _check(load_library().pkv_decode_run_fp8(
             _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
             _p(self.context_lens), float(scale), float(k_scale), float(v_scale),
@@ -527,12 +537,12 @@ def reshape_and_cache_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tenso
                           v_cache: torch.Tensor, slot_mapping: torch.Tensor, k_scale: float,
                           v_scale: float) -> None:
     """Quantise bf16 k, v ([T][Hkv][128]) to e4m3 codes (value / scale, nearest even,
-    saturated) and write them into the float8_e4m3fn caches at slot_mapping; -1 skips."""
+    saturated) and write them into the FP8 caches (float8_e4m3fn or float8_e5m2) at
+    slot_mapping; -1 skips."""
     dev = k.device
     _need(k, "k", torch.bfloat16, dev)
     _need(v, "v", torch.bfloat16, dev)
-    _need(k_cache, "k_cache", torch.float8_e4m3fn, dev)
-    _need(v_cache, "v_cache", torch.float8_e4m3fn, dev)
+    _need_fp8_pools(k_cache, v_cache, dev)
     _need(slot_mapping, "slot_mapping", torch.int64, dev)
     T = slot_mapping.shape[0]
     if k.shape != v.shape or k.shape[0] != T or k.shape[1:] != (k_cache.shape[1], k_cache.shape[3]) \

@@ -80,15 +80,16 @@ pkv_status bind_device(const void* p, const char* what) {
   return PKV_OK;
 }
 
-int elem_bytes(pkv_dtype t) { return t == PKV_BF16 ? 2 : (t == PKV_FP8_E4M3 ? 1 : 4); }
+bool is_fp8(int t) { return t == PKV_FP8_E4M3 || t == PKV_FP8_E5M2; }
+int elem_bytes(pkv_dtype t) { return t == PKV_BF16 ? 2 : (is_fp8(t) ? 1 : 4); }
 
 // Checks shared by every call.  `need_seq` also checks the per-sequence fields.
 pkv_status check_dims(const pkv_dims* d, bool need_seq) {
   if (!d) return fail(PKV_ERR_NULL, "dims is NULL");
-  if (d->dtype != PKV_F32 && d->dtype != PKV_BF16 && d->dtype != PKV_FP8_E4M3)
+  if (d->dtype != PKV_F32 && d->dtype != PKV_BF16 && !is_fp8(d->dtype))
     return fail(PKV_ERR_UNSUPPORTED, "dtype %d not supported (fp32, bf16, fp8 e4m3)",
                 (int)d->dtype);
-  if (d->dtype == PKV_FP8_E4M3 && d->head_dim != 128)
+  if (is_fp8(d->dtype) && d->head_dim != 128)
     return fail(PKV_ERR_UNSUPPORTED, "FP8 caches need head_dim 128");
   if (d->block_size != pkv::kBlock)
     return fail(PKV_ERR_UNSUPPORTED, "block_size %d not supported (16)", d->block_size);
@@ -211,7 +212,7 @@ pkv_status encode_pool_map(CUtensorMap* map, const void* pool, const pkv_dims* d
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map,
                    d->dtype == PKV_BF16       ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                   : d->dtype == PKV_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                   : is_fp8(d->dtype)         ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                    2, const_cast<void*>(pool), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -252,6 +253,8 @@ template <int D, int GMAX>
 struct DecodeCfg<pkv::Fp8Kv, D, GMAX> {
   static constexpr int W = GMAX == 16 ? 11 : 15, S = 2, MB = 1, SPLIT = 1;
 };
+template <int D, int GMAX>
+struct DecodeCfg<pkv::Fp8E5m2Kv, D, GMAX> : DecodeCfg<pkv::Fp8Kv, D, GMAX> {};
 
 // Largest dynamic shared memory already enabled per kernel, per device.
 struct SmemAttr {
@@ -438,6 +441,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
       static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads * row_groups;
   if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
+  } else if (d->dtype == PKV_FP8_E5M2) {
+    st = launch_decode_d<pkv::Fp8E5m2Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_BF16) {
     st = d->head_dim == 128
              ? launch_decode_d<__nv_bfloat16, 128>(mk, mv, prm, units, rows_max, stream)
@@ -471,11 +476,11 @@ pkv_status decode_prepare(const void* k, const void* v, void* k_cache, void* v_c
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
   if (fp8) {
-    if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+    if (!is_fp8(dims->dtype)) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
     if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
         !std::isfinite(v_scale))
       return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
-  } else if (dims->dtype == PKV_FP8_E4M3) {
+  } else if (is_fp8(dims->dtype)) {
     return fail(PKV_ERR_UNSUPPORTED, "FP8 pools need their scales: use pkv_decode_prepare_fp8");
   }
   if (dims->num_seqs == 0) return PKV_OK;
@@ -494,7 +499,9 @@ pkv_status decode_prepare(const void* k, const void* v, void* k_cache, void* v_c
   const int seqs_per_cta = pkv::kPlanThreads / per;
   const unsigned grid = 1u + static_cast<unsigned>((dims->num_seqs + seqs_per_cta - 1) / seqs_per_cta);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  auto kern = fp8 ? pkv::decode_prepare_kernel<true> : pkv::decode_prepare_kernel<false>;
+  auto kern = !fp8 ? pkv::decode_prepare_kernel<false, false>
+              : dims->dtype == PKV_FP8_E5M2 ? pkv::decode_prepare_kernel<true, true>
+                                            : pkv::decode_prepare_kernel<true, false>;
   cudaError_t e = launch(kern, dim3(grid), dim3(pkv::kPlanThreads), 0,
                          static_cast<cudaStream_t>(cuda_stream), static_cast<const uint4*>(k),
                          static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
@@ -516,11 +523,11 @@ namespace {
 // entry points (FP8 pools and their scales) or the plain ones (bf16 / fp32).
 pkv_status check_multi_pools(const pkv_dims* dims, bool fp8, float k_scale, float v_scale) {
   if (fp8) {
-    if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+    if (!is_fp8(dims->dtype)) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
     if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
         !std::isfinite(v_scale))
       return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
-  } else if (dims->dtype == PKV_FP8_E4M3) {
+  } else if (is_fp8(dims->dtype)) {
     return fail(PKV_ERR_UNSUPPORTED,
                 "FP8 pools need their scales: use the _fp8 calls for several query tokens");
   }
@@ -649,7 +656,7 @@ pkv_status pkv_decode_run(void* out, const void* q, const void* k_cache, const v
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
-  if (dims->dtype == PKV_FP8_E4M3)
+  if (is_fp8(dims->dtype))
     return fail(PKV_ERR_UNSUPPORTED, "FP8 caches need their scales: use pkv_decode_run_fp8");
   return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
                     dims, plan, workspace, workspace_bytes, cuda_stream);
@@ -664,7 +671,7 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_ca
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
-  if (dims->dtype == PKV_FP8_E4M3)
+  if (is_fp8(dims->dtype))
     return fail(PKV_ERR_UNSUPPORTED,
                 "FP8 caches need their scales: use pkv_paged_attention_decode_fp8");
   if (dims->num_seqs == 0) return PKV_OK;
@@ -752,7 +759,7 @@ pkv_status pkv_decode_run_fp8(void* out, const void* q, const void* k_cache,
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
-  if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+  if (!is_fp8(dims->dtype)) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
   return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
                     dims, plan, workspace, workspace_bytes, cuda_stream, k_scale, v_scale);
 }
@@ -767,7 +774,7 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
   DecodePlan plan;
   pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan);
   if (st != PKV_OK) return st;
-  if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+  if (!is_fp8(dims->dtype)) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
   if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
     return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
   if (dims->num_seqs == 0) return PKV_OK;
@@ -785,7 +792,7 @@ pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache
                                      void* cuda_stream) {
   pkv_status st = check_dims(dims, false);
   if (st != PKV_OK) return st;
-  if (dims->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+  if (!is_fp8(dims->dtype)) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
   if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
     return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
   if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
@@ -797,7 +804,9 @@ pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache
   if ((st = bind_device(k_cache, "k_cache")) != PKV_OK) return st;
   const int units = dims->num_kv_heads * dims->head_dim / 8;
   const int threads = units < 256 ? (units + 31) / 32 * 32 : 256;
-  cudaError_t e = launch(pkv::reshape_and_cache_fp8_kernel, dim3(num_tokens), dim3(threads), 0,
+  auto kern = dims->dtype == PKV_FP8_E5M2 ? pkv::reshape_and_cache_fp8_kernel<true>
+                                          : pkv::reshape_and_cache_fp8_kernel<false>;
+  cudaError_t e = launch(kern, dim3(num_tokens), dim3(threads), 0,
                          static_cast<cudaStream_t>(cuda_stream), static_cast<const uint4*>(k),
                          static_cast<const uint4*>(v), static_cast<uint8_t*>(k_cache),
                          static_cast<uint8_t*>(v_cache), slot_mapping, dims->num_kv_heads,
@@ -832,7 +841,7 @@ pkv_status pkv_reshape_and_cache(const void* k, const void* v, void* k_cache, vo
                                  const pkv_dims* dims, void* cuda_stream) {
   pkv_status st = check_dims(dims, false);
   if (st != PKV_OK) return st;
-  if (dims->dtype == PKV_FP8_E4M3)
+  if (is_fp8(dims->dtype))
     return fail(PKV_ERR_UNSUPPORTED, "FP8 caches quantise on write: use pkv_reshape_and_cache_fp8");
   if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
   if (num_tokens == 0) return PKV_OK;

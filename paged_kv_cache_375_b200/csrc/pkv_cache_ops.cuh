@@ -83,18 +83,22 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Eight bf16 values (16 bytes) to eight e4m3 codes (8 bytes, same order):
+// Eight bf16 values (16 bytes) to eight FP8 codes (8 bytes, same order):
 // code = e4m3(value / scale), the division in float (round to nearest even),
 // then round to nearest even onto e4m3, saturating to +-448.
-__device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float scale) {
+// With kE5m2 the codes are e5m2 (saturating to +-57344).
+template <bool kE5m2 = false>
+__device__ __forceinline__ uint2 bf16x8_to_fp8x8(uint4 x, float scale) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
   uint32_t codes[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const uint32_t p0 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i]), scale),
-                                        __fdiv_rn(bf16hi_to_f32(w[2 * i]), scale));
-    const uint32_t p1 = f32x2_to_e4m3x2(__fdiv_rn(bf16lo_to_f32(w[2 * i + 1]), scale),
-                                        __fdiv_rn(bf16hi_to_f32(w[2 * i + 1]), scale));
+    const float a = __fdiv_rn(bf16lo_to_f32(w[2 * i]), scale);
+    const float b = __fdiv_rn(bf16hi_to_f32(w[2 * i]), scale);
+    const float c = __fdiv_rn(bf16lo_to_f32(w[2 * i + 1]), scale);
+    const float d = __fdiv_rn(bf16hi_to_f32(w[2 * i + 1]), scale);
+    const uint32_t p0 = kE5m2 ? f32x2_to_e5m2x2(a, b) : f32x2_to_e4m3x2(a, b);
+    const uint32_t p1 = kE5m2 ? f32x2_to_e5m2x2(c, d) : f32x2_to_e4m3x2(c, d);
     codes[i] = p0 | (p1 << 16);
   }
   return make_uint2(codes[0], codes[1]);
@@ -102,8 +106,10 @@ __device__ __forceinline__ uint2 bf16x8_to_e4m3x8(uint4 x, float scale) {
 
 // ------------------------------------------------ reshape_and_cache into FP8
 // One CTA per token: each thread turns 8 bf16 values of the token's K (and V)
-// into 8 e4m3 codes, code = e4m3(value / scale) with the division in float,
-// rounded to nearest even and saturated to +-448, and stores them at the slot.
+// into 8 FP8 codes, code = e4m3(value / scale) (or e5m2 with kE5m2) with the
+// division in float, rounded to nearest even and saturated to the largest
+// finite code, and stores them at the slot.
+template <bool kE5m2>
 __global__ void __launch_bounds__(256)
     reshape_and_cache_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                  uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
@@ -131,7 +137,7 @@ __global__ void __launch_bounds__(256)
     for (int c = 0; c < 2; ++c) {
       const uint4 x = (c ? v : k)[static_cast<int64_t>(t) * units + u];
       *reinterpret_cast<uint2*>((c ? v_cache : k_cache) + dst) =
-          bf16x8_to_e4m3x8(x, c ? v_scale : k_scale);
+          bf16x8_to_fp8x8<kE5m2>(x, c ? v_scale : k_scale);
     }
   }
 }

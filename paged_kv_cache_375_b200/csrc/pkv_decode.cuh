@@ -184,6 +184,8 @@ struct DecodeParams {
 
 // Tag type of an FP8 (e4m3) cache: one-byte codes, bf16 q and out.
 struct Fp8Kv {};
+// Tag type of an FP8 (e5m2) cache.
+struct Fp8E5m2Kv {};
 
 // Bytes per q / out element for a cache element type.
 template <typename T>
@@ -485,8 +487,9 @@ __device__ __forceinline__ void bf16_publish(Bf16State<D, GMAX>& st, float* slot
 // Q's fragments are built in the same order.  V fragments come from
 // ldmatrix.trans on 16-bit units (pairs of d-values); a byte permute splits
 // the pairs, so row r of an output m-tile is d = 16mt + 2r and row r+8 is
-// d = 16mt + 2r + 1.  Codes become f16 exactly (cvt.f16x2.e4m3x2); the K
-// scale is folded into the score scale and the V scale into the output.
+// d = 16mt + 2r + 1.  Codes become f16 exactly: e4m3 by cvt.f16x2.e4m3x2,
+// e5m2 (the upper byte of a binary16) by the byte permute alone; the K scale
+// is folded into the score scale and the V scale into the output.
 // (The e4m3 m16n8k32 MMA straight on the codes, with q split into two e4m3
 // terms, was measured slower here: more issued instructions per tile.)
 template <int GMAX>
@@ -536,7 +539,33 @@ __device__ __forceinline__ void fp8_begin_item(Fp8State<GMAX>& st, const uint8_t
   st.lim_min = len - q_len + row0 / g;
 }
 
-template <int GMAX>
+// Four FP8 codes (one 32-bit word, bytes b0..b3) to two f16x2: (b0, b1) to `lo`,
+// (b2, b3) to `hi`.  e4m3 codes are converted (exactly); e5m2 codes are the
+// upper bytes of binary16 values, so a byte permute places them.
+template <bool kE5m2>
+__device__ __forceinline__ void fp8x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  if constexpr (kE5m2) {
+    lo = __byte_perm(x, 0u, 0x1404u);
+    hi = __byte_perm(x, 0u, 0x3424u);
+  } else {
+    e4m3x4_to_f16x2x2(x, lo, hi);
+  }
+}
+
+// The same with the pairs (b0, b2) to `lo` and (b1, b3) to `hi` (the V layout
+// after ldmatrix.trans on 16-bit units).
+template <bool kE5m2>
+__device__ __forceinline__ void fp8x4_to_f16x2x2_interleaved(uint32_t x, uint32_t& lo,
+                                                             uint32_t& hi) {
+  if constexpr (kE5m2) {
+    lo = __byte_perm(x, 0u, 0x2404u);
+    hi = __byte_perm(x, 0u, 0x3414u);
+  } else {
+    e4m3x4_to_f16x2x2(__byte_perm(x, 0u, 0x3120u), lo, hi);
+  }
+}
+
+template <int GMAX, bool kE5m2 = false>
 __device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
                                          const uint8_t* v0, int valid0, int pos0,
                                          const uint8_t* k1, const uint8_t* v1, int valid1,
@@ -562,10 +591,10 @@ __device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
       uint32_t m0, m1, m2, m3;
       ldmatrix_x4(smem_addr(t ? k1 : k0) + tok * 128u + off, m0, m1, m2, m3);
       uint32_t a_lo[4], a_hi[4];
-      e4m3x4_to_f16x2x2(m0, a_lo[0], a_lo[2]);
-      e4m3x4_to_f16x2x2(m1, a_lo[1], a_lo[3]);
-      e4m3x4_to_f16x2x2(m2, a_hi[0], a_hi[2]);
-      e4m3x4_to_f16x2x2(m3, a_hi[1], a_hi[3]);
+      fp8x4_to_f16x2x2<kE5m2>(m0, a_lo[0], a_lo[2]);
+      fp8x4_to_f16x2x2<kE5m2>(m1, a_lo[1], a_lo[3]);
+      fp8x4_to_f16x2x2<kE5m2>(m2, a_hi[0], a_hi[2]);
+      fp8x4_to_f16x2x2<kE5m2>(m3, a_hi[1], a_hi[3]);
 #pragma unroll
       for (int nh = 0; nh < NH; ++nh) {
         mma_f16_16816(s[t][nh], a_lo, st.qb[nh][2 * kp][0], st.qb[nh][2 * kp][1]);
@@ -658,11 +687,9 @@ __device__ __forceinline__ void fp8_step(Fp8State<GMAX>& st, const uint8_t* k0,
       // m0 / m1: tokens 0-7 / 8-15 of granule 2mp; m2 / m3: of granule 2mp+1
 #pragma unroll
       for (int hlf = 0; hlf < 2; ++hlf) {
-        const uint32_t ya = __byte_perm(hlf ? m2 : m0, 0u, 0x3120u);
-        const uint32_t yb = __byte_perm(hlf ? m3 : m1, 0u, 0x3120u);
         uint32_t a[4];
-        e4m3x4_to_f16x2x2(ya, a[0], a[1]);
-        e4m3x4_to_f16x2x2(yb, a[2], a[3]);
+        fp8x4_to_f16x2x2_interleaved<kE5m2>(hlf ? m2 : m0, a[0], a[1]);
+        fp8x4_to_f16x2x2_interleaved<kE5m2>(hlf ? m3 : m1, a[2], a[3]);
         if (partial) {
           a[0] &= mk0;
           a[1] &= mk0;
@@ -1052,7 +1079,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
   // ================================ decode warps ================================
   using Bst = Bf16State<D, RPW>;
   using Fst = F32State<D, GMAX>;
-  constexpr bool kFp8 = std::is_same<T, Fp8Kv>::value;
+  constexpr bool kE5m2 = std::is_same<T, Fp8E5m2Kv>::value;
+  constexpr bool kFp8 = std::is_same<T, Fp8Kv>::value || kE5m2;
   constexpr bool kBf16 = sizeof(T) == 2;
   static_assert(SPLIT == 1 || kFp8 || kBf16, "row split needs the tensor-core states");
   typename std::conditional<kFp8, Fp8State<RPW>,
@@ -1194,8 +1222,8 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
       const int pos0 = (it.blk_begin + b) * kBlock;  // position of the first tile's token 0
       if constexpr (kFp8) {
         if (my_rows > 0)
-          fp8_step<RPW>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
-                        kt[1] + Lay::kTileBytes, valid[1], pos0 + L * kBlock, sc, lane);
+          fp8_step<RPW, kE5m2>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
+                               kt[1] + Lay::kTileBytes, valid[1], pos0 + L * kBlock, sc, lane);
       } else if constexpr (kBf16) {
         if (my_rows > 0)
           bf16_step<D, RPW>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],

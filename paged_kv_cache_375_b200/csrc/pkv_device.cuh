@@ -262,6 +262,17 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Two floats to e5m2x2 codes (round to nearest even, saturating to
+// +-57344); `lo` in the low byte of the result.
+__device__ __forceinline__ uint32_t f32x2_to_e5m2x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 p;\n\tcvt.rn.satfinite.e5m2x2.f32 p, %2, %1;\n\t"
+      "cvt.u32.u16 %0, p;\n\t}"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
+}
+
 // Two floats to a packed f16x2 (round to nearest even, saturating to the
 // largest finite f16); `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {

@@ -17,7 +17,7 @@ namespace pkv {
 // plans; CTA c > 0 writes sequences (c - 1) * seqs_per_cta ... with `per`
 // threads each (per = min(units, kPlanThreads), units = 16-byte source units
 // of one token's K row block).  A sequence with L = 0 has no new token.
-template <bool kFp8>
+template <bool kFp8, bool kE5m2>
 __global__ void __launch_bounds__(kPlanThreads)
     decode_prepare_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                           uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
@@ -71,10 +71,10 @@ __global__ void __launch_bounds__(kPlanThreads)
     const int32_t within = u % units_per_head;
     const int64_t row = (block * num_kv_heads + h) * kBlock + offset;  // destination row
     if constexpr (kFp8) {
-      // 8 bf16 values -> 8 e4m3 codes
+      // 8 bf16 values -> 8 FP8 codes
       const int64_t dst = row * (units_per_head * 8) + within * 8;
-      *reinterpret_cast<uint2*>(k_cache + dst) = bf16x8_to_e4m3x8(ksrc[u], k_scale);
-      *reinterpret_cast<uint2*>(v_cache + dst) = bf16x8_to_e4m3x8(vsrc[u], v_scale);
+      *reinterpret_cast<uint2*>(k_cache + dst) = bf16x8_to_fp8x8<kE5m2>(ksrc[u], k_scale);
+      *reinterpret_cast<uint2*>(v_cache + dst) = bf16x8_to_fp8x8<kE5m2>(vsrc[u], v_scale);
     } else {
       const int64_t dst = row * (units_per_head * 16) + within * 16;
       *reinterpret_cast<uint4*>(k_cache + dst) = ksrc[u];

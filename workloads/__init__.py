@@ -96,7 +96,8 @@ class Batch:
 
     name: str
     seed: int
-    dtype: str                      # "f32", "bf16" or "fp8" (e4m3 caches, bf16 q and new K/V)
+    dtype: str                      # "f32", "bf16", "fp8" (e4m3 caches, bf16 q and new K/V)
+                                    # or "fp8e5m2" (e5m2 caches)
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
@@ -144,7 +145,7 @@ class Batch:
     @property
     def elem_bytes(self) -> int:
         """Bytes of one cache element."""
-        return {"f32": 4, "bf16": 2, "fp8": 1}[self.dtype]
+        return {"f32": 4, "bf16": 2, "fp8": 1, "fp8e5m2": 1}[self.dtype]
 
     @property
     def q_elem_bytes(self) -> int:
@@ -178,7 +179,7 @@ class Batch:
             t = t.detach().contiguous().cpu()
             if t.dtype == torch.bfloat16:
                 return t.view(torch.int16).numpy().view(np.uint16)
-            if t.dtype == torch.float8_e4m3fn:
+            if t.dtype in (torch.float8_e4m3fn, torch.float8_e5m2):
                 return t.view(torch.uint8).numpy()
             return t.numpy()
         return {"q": h(self.q), "k_cache": h(self.k_cache), "v_cache": h(self.v_cache),
@@ -197,7 +198,13 @@ class Batch:
 
 def torch_dtype(dtype: str) -> torch.dtype:
     """Element type of q / out / new K/V (an FP8 configuration's caches are e4m3)."""
-    return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16}[dtype]
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.bfloat16,
+            "fp8e5m2": torch.bfloat16}[dtype]
+
+
+def fp8_format(dtype: str) -> str | None:
+    """The FP8 code format of a configuration's pools ("e4m3", "e5m2"), None if not FP8."""
+    return {"fp8": "e4m3", "fp8e5m2": "e5m2"}.get(dtype)
 
 
 # Scales of the FP8 configurations' pools (exact in float32, different so that
@@ -223,6 +230,22 @@ def _random_codes(shape, gen, device, chunk_rows: int | None = None) -> torch.Te
         c = (sign << 7) | (expo << 3) | mant
         out[r0:r1] = torch.where((c & 0x7F) == E4M3_NAN_CODE, c - 1, c)
     return out.view(torch.float8_e4m3fn)
+
+
+def _random_codes_e5m2(shape, gen, device, chunk_rows: int | None = None) -> torch.Tensor:
+    """Random e5m2 bit patterns: sign, exponent field 8..22 and mantissa drawn uniformly
+    (magnitudes log-uniform over 2^-7 .. 2^7 x 1.75).  A drawing of codes."""
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    rows = shape[0]
+    step = chunk_rows or rows
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        sub = (r1 - r0,) + tuple(shape[1:])
+        sign = torch.randint(0, 2, sub, generator=gen, device=device, dtype=torch.uint8)
+        expo = torch.randint(8, 23, sub, generator=gen, device=device, dtype=torch.uint8)
+        mant = torch.randint(0, 4, sub, generator=gen, device=device, dtype=torch.uint8)
+        out[r0:r1] = (sign << 7) | (expo << 2) | mant
+    return out.view(torch.float8_e5m2)
 
 
 def default_scale(head_dim: int) -> float:
@@ -261,11 +284,12 @@ def _assemble(name: str, seed: int, dtype: str, hq: int, hkv: int, d: int, num_b
     gen.manual_seed(seed)
     shape = (num_blocks, hkv, BLOCK_SIZE, d)
     chunk = max(1, (1 << 26) // (hkv * BLOCK_SIZE * d))
-    fp8 = dtype == "fp8"
+    fp8 = fp8_format(dtype) is not None
     vdt = "bf16" if fp8 else dtype
     if fp8:
-        k_cache = _random_codes(shape, gen, device, chunk)
-        v_cache = _random_codes(shape, gen, device, chunk)
+        draw = _random_codes if dtype == "fp8" else _random_codes_e5m2
+        k_cache = draw(shape, gen, device, chunk)
+        v_cache = draw(shape, gen, device, chunk)
     else:
         k_cache = _randn(shape, gen, device, dtype, chunk)
         v_cache = _randn(shape, gen, device, dtype, chunk)
@@ -391,6 +415,18 @@ def c3_fp8(device="cpu", num_seqs: int = 256) -> Batch:
     return b
 
 
+def c3_fp8e5m2(device="cpu", num_seqs: int = 256) -> Batch:
+    """The Llama-3-8B-shaped GQA decode batch over FP8 e5m2 pools (one scale per pool)."""
+    seed = CONFIG_SEEDS["c3_llama3_8b_gqa"]
+    lens = c3_lens(num_seqs)
+    need = int(sum((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE for L in lens))
+    nb = max(32768, int(math.ceil(1.25 * need)))
+    b = random_batch(seed, lens, 32, 8, 128, "fp8e5m2", num_blocks=nb, device=device,
+                     new_token=True, name="c3_fp8e5m2_llama3_8b_gqa")
+    b.meta["lognormal_sigma"] = C3_LOGNORMAL_SIGMA
+    return b
+
+
 def chunked_batch(seed: int, lens, chunks, hq: int, hkv: int, d: int, dtype: str = "bf16",
                   num_blocks: int | None = None, device="cpu", name: str = "chunked",
                   extra_table: int = 0) -> Batch:
@@ -511,6 +547,8 @@ CONFIGS["c3_spec_decode"] = ("Llama-3-8B-shaped GQA bf16, batch 256, verifying 4
                               "per sequence (causal, 16 query rows per kv head)")
 CONFIGS["c3_spec_fp8"] = ("the speculative-verification batch (256 x 4 draft tokens, causal) over FP8 "
                           "e4m3 pools, bf16 q/out")
+CONFIGS["c3_fp8e5m2"] = ("Llama-3-8B-shaped GQA over FP8 e5m2 pools (one scale per pool), bf16 q/out: "
+                         "batch 256, 32q/8kv, d128, the same lognormal lens")
 CONFIGS["c3_fp8"] = ("Llama-3-8B-shaped GQA over FP8 e4m3 pools (one scale per pool), bf16 q/out: "
                      "batch 256, 32q/8kv, d128, the same lognormal lens, reshape_and_cache_fp8 "
                      "of the new token before attention")
@@ -520,6 +558,7 @@ BUILDERS = {
     "c3_spec_decode": c3_spec_decode,
     "c3_fp8": c3_fp8,
     "c3_spec_fp8": c3_spec_fp8,
+    "c3_fp8e5m2": c3_fp8e5m2,
     "c2_llama2_13b_mha": c2_llama2_13b_mha,
     "c3_llama3_8b_gqa": c3_llama3_8b_gqa,
     "c4_shared_prefix": c4_shared_prefix,
