@@ -1,5 +1,5 @@
 """Seeded random configurations through the whole path against the oracle: dtype
-(fp32, bf16, FP8), head_dim, kv heads and group size, ragged and empty lengths,
+(fp32, bf16, FP8 e4m3 and e5m2), head_dim, kv heads and group size, ragged and empty lengths,
 one or several query tokens, partition size.  Each case draws its own shapes."""
 import numpy as np
 import pytest
@@ -15,8 +15,8 @@ pytestmark = pytest.mark.gpu
 
 def _case(seed):
     rng = np.random.default_rng(10_000 + seed)
-    dtype = ["f32", "bf16", "fp8"][seed % 3]
-    d = 128 if dtype == "fp8" else int(rng.choice([64, 128]))
+    dtype = ["f32", "bf16", "fp8", "fp8e5m2"][seed % 4]
+    d = 128 if workloads.fp8_format(dtype) else int(rng.choice([64, 128]))
     hkv = int(rng.choice([1, 2, 4, 8]))
     g = int(rng.choice([1, 2, 3, 4, 6, 8, 16]))
     n = int(rng.integers(1, 12))
@@ -42,10 +42,11 @@ def test_random_configuration(cuda_device, seed):
                                     device=dev, extra_table=1)
     host = b.host()
     bt, cl = dev_i32(b.block_tables, dev), dev_i32(b.context_lens, dev)
+    fmt = workloads.fp8_format(dtype)
     if b.new_seq.shape[0]:
         slots = pkv.slot_mapping(bt, b.num_blocks, token_seq=dev_i32(b.new_seq, dev),
                                  token_pos=dev_i32(b.new_pos, dev))
-        if dtype == "fp8":
+        if fmt:
             pkv.reshape_and_cache_fp8(b.new_k, b.new_v, b.k_cache, b.v_cache, slots, b.k_scale,
                                       b.v_scale)
         else:
@@ -53,7 +54,7 @@ def test_random_configuration(cuda_device, seed):
     out = torch.empty_like(b.q)
     mcl = max(b.max_context_len, 1)
     if chunks is None:
-        if dtype == "fp8":
+        if fmt:
             pkv.paged_attention_decode_fp8(out, b.q, b.k_cache, b.v_cache, bt, cl, b.scale,
                                            b.k_scale, b.v_scale, max_context_len=mcl,
                                            partition_tokens=partition)
@@ -62,7 +63,7 @@ def test_random_configuration(cuda_device, seed):
                                        max_context_len=mcl, partition_tokens=partition)
     else:
         qsl = dev_i32(b.query_start_loc, dev)
-        if dtype == "fp8":
+        if fmt:
             pkv.paged_attention_multi_fp8(out, b.q, b.k_cache, b.v_cache, bt, cl, qsl, b.scale,
                                           b.k_scale, b.v_scale, b.max_query_len,
                                           max_context_len=mcl, partition_tokens=partition)
@@ -75,19 +76,19 @@ def test_random_configuration(cuda_device, seed):
     k, v = host["k_cache"].copy(), host["v_cache"].copy()
     if b.new_seq.shape[0]:
         sl = oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos)
-        if dtype == "fp8":
+        if fmt:
             oracle.reshape_and_cache_fp8(host["new_k"], host["new_v"], k, v, sl, b.k_scale,
-                                         b.v_scale)
+                                         b.v_scale, fmt=fmt)
         else:
             oracle.reshape_and_cache(host["new_k"], host["new_v"], k, v, sl)
     if chunks is None:
         ref = (oracle.paged_decode_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
-                                       b.context_lens, b.scale) if dtype == "fp8" else
+                                       b.context_lens, b.scale, fmt=fmt) if fmt else
                oracle.paged_decode(host["q"], k, v, b.block_tables, b.context_lens, b.scale))
     else:
         ref = (oracle.paged_multi_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
-                                      b.context_lens, b.query_start_loc, b.scale)
-               if dtype == "fp8" else
+                                      b.context_lens, b.query_start_loc, b.scale, fmt=fmt)
+               if fmt else
                oracle.paged_multi(host["q"], k, v, b.block_tables, b.context_lens,
                                   b.query_start_loc, b.scale))
-    check_close(out, ref, "bf16" if dtype == "fp8" else dtype, what)
+    check_close(out, ref, "bf16" if fmt else dtype, what)
