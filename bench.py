@@ -189,7 +189,7 @@ def whole_job_value(units_per_rank: float, world: int, seconds: float) -> float:
 class Step:
     """The hot path over one batch through the public API (device-resident inputs)."""
 
-    def __init__(self, b: workloads.Batch, partition_tokens: int):
+    def __init__(self, b: workloads.Batch, partition_tokens: int, shared_prefix: bool = True):
         import paged_kv_cache_375_b200 as pkv
         self.pkv, self.b = pkv, b
         dev = b.q.device
@@ -203,10 +203,19 @@ class Step:
         self.part_tokens = pkv.decode_partition_tokens(self.dims, self.mcl, partition_tokens)
         self.split = self.part_tokens < self.mcl
         self.multi = b.query_start_loc is not None
+        # sequences that share a prompt's blocks: read those blocks once per group
+        self.shared = shared_prefix and "group_start" in b.meta and not self.multi
+        if self.shared:
+            self.group_start = torch.tensor(b.meta["group_start"], dtype=torch.int32, device=dev)
+            self.shared_blocks = torch.tensor(b.meta["shared_blocks"], dtype=torch.int32,
+                                              device=dev)
+            self.split = True                           # prefix and own partials are merged
         if self.multi:
             self.qsl = torch.from_numpy(b.query_start_loc).to(dev)
             ws = pkv.load_library().pkv_multi_workspace_bytes(
                 __import__("ctypes").byref(self.dims), b.q.shape[0], self.mcl, partition_tokens)
+        elif self.shared:
+            ws = pkv.decode_shared_workspace_bytes(self.dims, self.mcl, partition_tokens)
         else:
             ws = pkv.decode_workspace_bytes(self.dims, self.mcl, partition_tokens)
         self.ws = torch.empty(ws, dtype=torch.uint8, device=dev)
@@ -219,7 +228,8 @@ class Step:
         self.slots = torch.empty(max(self.T, 1), dtype=torch.int64, device=dev)
         self.pairs = torch.from_numpy(b.cow_pairs).to(dev) if b.cow_pairs.shape[0] else None
         # one new token per sequence at its last position, no copies: the fused prologue
-        self.fused = self.decode_mode and self.pairs is None and not self.multi
+        self.fused = (self.decode_mode and self.pairs is None and not self.multi
+                      and not self.shared)
         if self.pairs is not None:
             pkv.validate_copy_pairs(torch.from_numpy(b.cow_pairs), b.num_blocks)
 
@@ -255,6 +265,12 @@ class Step:
 
     def plan(self):
         b = self.b
+        if self.shared:
+            self.plan_obj = self.pkv.SharedDecodePlan(
+                self.bt, self.cl, self.group_start, self.shared_blocks, b.num_q_heads, b.k_cache,
+                max_context_len=self.mcl, partition_tokens=self.partition,
+                workspace_tensor=self.ws)
+            return
         extra = {}
         if self.fused:   # one launch: the new tokens' slots and writes, and the plan
             extra = dict(new_k=b.new_k, new_v=b.new_v, v_cache=b.v_cache, k_scale=b.k_scale,
@@ -294,7 +310,7 @@ def run_ours(args, world, rank, local):
     name = WORKLOADS[args.workload]
     b = (workloads.BUILDERS[name](device=dev, num_seqs=args.batch) if args.batch else
          workloads.BUILDERS[name](device=dev))
-    step = Step(b, args.partition)
+    step = Step(b, args.partition, shared_prefix=not args.no_shared_prefix)
     alg = algorithmic_bytes(b)
     kv_bytes = b.kv_bytes() if name != "c4_shared_prefix" else b.unique_kv_bytes()
     stream = torch.cuda.current_stream(dev)
@@ -372,6 +388,9 @@ def run_ours(args, world, rank, local):
             "context_tokens": int(b.context_lens.sum()), "max_context_len": b.max_context_len,
             "new_tokens_per_step": step.T, "cow_pairs_per_step": int(b.cow_pairs.shape[0]),
             "partition_tokens": step.part_tokens, "split_k": step.split,
+            **({"shared_prefix": "each prompt's full blocks read once per kv head for its "
+                                 f"{b.meta['samples']} samples (shared-prefix items, "
+                                 "log-sum-exp merge)"} if step.shared else {}),
             "kv_bytes_per_step": kv_bytes,
             # KV-block usage of the pool (blocks holding tokens / pool size)
             "blocks_in_use": int(b.meta.get("blocks_in_use", 0)),
@@ -409,6 +428,32 @@ def run_ours(args, world, rank, local):
     return result
 
 
+def plan_items(step: Step) -> int:
+    """Work items the plan writes: a (sequence, partition) each; with shared prefixes, each
+    sequence's partitions after its prefix plus, per group, its prefix partitions times the
+    items that take the group's members (16 query rows at most per item)."""
+    b = step.b
+    lens = b.context_lens.astype(np.int64)
+    P = step.part_tokens
+
+    def parts(n):
+        return np.maximum(1, (n + P - 1) // P)
+
+    if not step.shared:
+        return int(parts(lens).sum())
+    g = b.num_q_heads // b.num_kv_heads
+    per_item = 16 // g if g <= 8 else 1
+    gs, sb = b.meta["group_start"], b.meta["shared_blocks"]
+    items = 0
+    for i in range(len(sb)):
+        members = lens[gs[i]:gs[i + 1]]
+        pref = min([int(sb[i])] + [int(L) // 16 for L in members]) if len(members) >= 2 else 0
+        items += int(parts(members - 16 * pref).sum())
+        if pref:
+            items += int(parts(np.int64(16 * pref))) * -(-len(members) // per_item)
+    return items
+
+
 def op_bytes(step: Step) -> dict:
     """Algorithmic bytes of each cache-maintenance op of one step (read + write)."""
     b = step.b
@@ -420,9 +465,9 @@ def op_bytes(step: Step) -> dict:
         "slot_mapping": T * (4 + 4 + 8) + (4 * b.num_seqs if step.decode_mode else 8 * T),
         "reshape_and_cache": 2 * T * (row_in + row) + 8 * T,    # K and V, read and write
         "copy_blocks": 2 * 2 * P * block + 16 * P,              # K and V, read and write
-        # reads the lengths, writes one 16-byte work item per (sequence, partition)
-        "plan": 4 * b.num_seqs + 16 * int(np.maximum(
-            1, (b.context_lens.astype(np.int64) + step.part_tokens - 1) // step.part_tokens).sum()),
+        # reads the lengths (and the groups), writes one 32-byte work item per item
+        "plan": 4 * b.num_seqs + 32 * plan_items(step) + (
+            8 * len(step.b.meta["shared_blocks"]) + 4 if step.shared else 0),
     }
     out["decode_prologue"] = out["slot_mapping"] + out["reshape_and_cache"] + out["plan"]
     return out
@@ -434,6 +479,9 @@ def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
     pkv, b = step.pkv, step.b
 
     def plan_only():
+        if step.shared:
+            step.plan()
+            return
         pkv.DecodePlan(step.bt, step.cl, b.num_q_heads, b.k_cache, max_context_len=step.mcl,
                        partition_tokens=step.partition, workspace_tensor=step.ws)
 
@@ -504,19 +552,22 @@ def run_e2e(step: Step, args, world, dev, kv_bytes):
     (q, the new tokens' K/V, context lengths, block tables) and reads the output back to
     pinned host memory, synchronising on it."""
     b = step.b
-    host = {name: t.detach().cpu().pin_memory() for name, t in (
-        ("q", b.q), ("new_k", b.new_k), ("new_v", b.new_v), ("cl", step.cl), ("bt", step.bt))}
+    ins = [("q", b.q), ("new_k", b.new_k), ("new_v", b.new_v), ("cl", step.cl), ("bt", step.bt)]
+    if step.shared:
+        ins += [("gs", step.group_start), ("sb", step.shared_blocks)]
+    host = {name: t.detach().cpu().pin_memory() for name, t in ins}
+    dst = dict(ins)
     out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
     stream = torch.cuda.current_stream(dev)
 
+    def inputs_in():
+        for name, t in host.items():
+            dst[name].copy_(t, non_blocking=True)
+
     def one():
-        b.q.copy_(host["q"], non_blocking=True)
-        b.new_k.copy_(host["new_k"], non_blocking=True)
-        b.new_v.copy_(host["new_v"], non_blocking=True)
-        step.cl.copy_(host["cl"], non_blocking=True)
-        step.bt.copy_(host["bt"], non_blocking=True)
+        inputs_in()
         step()
         out_host.copy_(step.out, non_blocking=True)
         stream.synchronize()
@@ -549,11 +600,7 @@ def run_e2e(step: Step, args, world, dev, kv_bytes):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(graph_stream):
             with torch.cuda.graph(g, stream=graph_stream):
-                b.q.copy_(host["q"], non_blocking=True)
-                b.new_k.copy_(host["new_k"], non_blocking=True)
-                b.new_v.copy_(host["new_v"], non_blocking=True)
-                step.cl.copy_(host["cl"], non_blocking=True)
-                step.bt.copy_(host["bt"], non_blocking=True)
+                inputs_in()
                 step()
                 out_host.copy_(step.out, non_blocking=True)
         torch.cuda.synchronize(dev)
@@ -701,6 +748,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true",
                     help="skip timing the cache ops and the plan alone after the timed region")
+    ap.add_argument("--no-shared-prefix", action="store_true",
+                    help="decode a batch with shared prompt blocks with the plain plan (every "
+                         "sequence reads its whole table)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--batch", type=int, default=0,
                     help="number of sequences (0 = the workload's own); a smaller batch of the "

@@ -96,6 +96,9 @@ typedef enum pkv_dtype {
 #define PKV_DEVERR_PAIR    0x8u   /* copy pair outside [0, num_blocks) */
 #define PKV_DEVERR_POS     0x10u  /* slot-mapping position outside the block table */
 #define PKV_DEVERR_TIMEOUT 0x20u  /* a bounded wait gave up */
+#define PKV_DEVERR_GROUP   0x40u  /* shared-prefix groups: bounds not nondecreasing in
+                                     [0, num_seqs], or a shared block count < 0 or past
+                                     a member's full blocks */
 
 typedef struct pkv_dims {
     int32_t num_seqs;            /* B */
@@ -353,6 +356,85 @@ pkv_status pkv_decode_run_fp8(void *out, const void *q, const void *k_cache,
                               float v_scale, const pkv_dims *dims, int32_t max_context_len,
                               int32_t partition_tokens, void *workspace, size_t workspace_bytes,
                               void *cuda_stream);
+
+/*
+ * Decode for batches whose consecutive sequences share their leading blocks:
+ * parallel samples of one prompt, or requests behind one system prompt (the
+ * pages' prefix sharing with reference counts and copy-on-write: "vLLM 深读：
+ * 用 PagedAttention 撑起高并发 LLM 推理", section "先看浪费在哪里").  The result
+ * is pkv_paged_attention_decode's, but a shared block is read from HBM once
+ * per kv head for its whole group instead of once per sequence.
+ *
+ * Group i covers sequences group_start[i] .. group_start[i+1] - 1
+ * (group_start: int32 [num_groups + 1], device, nondecreasing within
+ * [0, num_seqs]; num_groups <= num_seqs; a sequence in no group has no shared
+ * prefix).  shared_blocks: int32 [num_groups], device.  Definition: every
+ * member s of group i reads its first P = shared_blocks[i] blocks through the
+ * FIRST member's table row and blocks P .. through its own row, i.e.
+ *   out[s][h] = softmax_j(scale * q[s][h] . K_j) V_j   over j < context_lens[s]
+ * with K_j, V_j from block_tables[j < 16P ? first : s][j/16], slot j%16.  When
+ * the members' tables really hold the same first P entries (what a block
+ * manager's fork gives) this is exactly pkv_paged_attention_decode; the
+ * tables are not compared.  Groups of fewer than two members read no shared
+ * prefix (their count is not looked at).  Otherwise P larger than a member's
+ * full blocks (context_len/16, rounded down) is lowered to them and a negative
+ * P raised to 0; both, and group bounds that are not nondecreasing in
+ * [0, num_seqs] (then no group is used), are flagged PKV_DEVERR_GROUP.
+ *
+ * How it runs: the plan makes, per group, items over the shared blocks that
+ * take one query token of each of up to 16/(Hq/Hkv) members at once (all
+ * Hq/Hkv heads of each, at most 16 query rows; one member per item when
+ * Hq/Hkv > 8), and ordinary items over each sequence's own blocks; every
+ * member's prefix and own partial results are merged by log-sum-exp (so the
+ * merge kernel always runs).  Workspace: pkv_decode_shared_workspace_bytes()
+ * (different from the plain decode's).  Plan/run split as pkv_decode_plan /
+ * pkv_decode_run, with the same rules; the plan also depends on group_start
+ * and shared_blocks.  The _fp8 calls take FP8 pools and their scales.
+ * pkv_decode_shared_workspace_layout: offsets of the partial results (as
+ * pkv_decode_workspace_layout) and of seq_prefix, int32 [num_seqs] = P used
+ * for each sequence after the plan (for tests).
+ */
+size_t pkv_decode_shared_workspace_bytes(const pkv_dims *dims, int32_t max_context_len,
+                                         int32_t partition_tokens);
+
+pkv_status pkv_decode_shared_workspace_layout(const pkv_dims *dims, int32_t max_context_len,
+                                              int32_t partition_tokens, int32_t *max_parts,
+                                              size_t *part_o_offset, size_t *part_ml_offset,
+                                              size_t *seq_prefix_offset);
+
+pkv_status pkv_paged_attention_decode_shared(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, const int32_t *group_start,
+    const int32_t *shared_blocks, int32_t num_groups, float scale, const pkv_dims *dims,
+    int32_t max_context_len, int32_t partition_tokens, void *workspace, size_t workspace_bytes,
+    void *cuda_stream);
+
+pkv_status pkv_paged_attention_decode_shared_fp8(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, const int32_t *group_start,
+    const int32_t *shared_blocks, int32_t num_groups, float scale, float k_scale, float v_scale,
+    const pkv_dims *dims, int32_t max_context_len, int32_t partition_tokens, void *workspace,
+    size_t workspace_bytes, void *cuda_stream);
+
+pkv_status pkv_decode_plan_shared(const int32_t *context_lens, const int32_t *group_start,
+                                  const int32_t *shared_blocks, int32_t num_groups,
+                                  const pkv_dims *dims, int32_t max_context_len,
+                                  int32_t partition_tokens, void *workspace,
+                                  size_t workspace_bytes, void *cuda_stream);
+
+pkv_status pkv_decode_run_shared(void *out, const void *q, const void *k_cache,
+                                 const void *v_cache, const int32_t *block_tables,
+                                 const int32_t *context_lens, float scale, const pkv_dims *dims,
+                                 int32_t max_context_len, int32_t partition_tokens,
+                                 void *workspace, size_t workspace_bytes, void *cuda_stream);
+
+pkv_status pkv_decode_run_shared_fp8(void *out, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *block_tables,
+                                     const int32_t *context_lens, float scale, float k_scale,
+                                     float v_scale, const pkv_dims *dims,
+                                     int32_t max_context_len, int32_t partition_tokens,
+                                     void *workspace, size_t workspace_bytes,
+                                     void *cuda_stream);
 
 /*
  * reshape_and_cache: for every token t with slot_mapping[t] >= 0, copy the

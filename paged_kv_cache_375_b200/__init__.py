@@ -17,7 +17,10 @@ per-sequence block table, slot_mapping, copy-on-write of shared blocks):
   DecodePlan(...)            plan once per step (optionally writing the new tokens
                              in the same launch), run once per layer
   paged_attention_multi(...) several causal query tokens per sequence
-  *_fp8 variants             FP8 (e4m3) pools with per-pool scales
+  paged_attention_decode_shared(...), SharedDecodePlan
+                             decode reading a prefix shared by consecutive
+                             sequences once per group
+  *_fp8 variants             FP8 (e4m3 or e5m2) pools with per-pool scales
   BlockManager               host-side block bookkeeping with prefix caching
   check_device_error()
 """
@@ -36,6 +39,7 @@ PKV_F32, PKV_BF16, PKV_FP8_E4M3, PKV_FP8_E5M2 = 0, 1, 2, 3
 FP8_DTYPES = (torch.float8_e4m3fn, torch.float8_e5m2)   # pool dtypes of the *_fp8 calls
 DEVERR_BLOCK, DEVERR_SLOT, DEVERR_LEN, DEVERR_PAIR, DEVERR_POS, DEVERR_TIMEOUT = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20)
+DEVERR_GROUP = 0x40
 
 STATUS_NAMES = {0: "PKV_OK", 1: "PKV_ERR_NULL", 2: "PKV_ERR_SHAPE", 3: "PKV_ERR_UNSUPPORTED",
                 4: "PKV_ERR_WORKSPACE", 5: "PKV_ERR_PAIRS", 6: "PKV_ERR_CUDA",
@@ -98,6 +102,18 @@ def load_library() -> ctypes.CDLL:
                                                              f32, f32, D, i32, i32, P, sz, P]),
             "pkv_multi_run_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, f32, f32, D,
                                                  i32, i32, P, sz, P]),
+            "pkv_decode_shared_workspace_bytes": (sz, [D, i32, i32]),
+            "pkv_decode_shared_workspace_layout": (ctypes.c_int, [D, i32, i32, P, P, P, P]),
+            "pkv_paged_attention_decode_shared": (ctypes.c_int, [P, P, P, P, P, P, P, P, i32,
+                                                                 f32, D, i32, i32, P, sz, P]),
+            "pkv_paged_attention_decode_shared_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, P,
+                                                                     i32, f32, f32, f32, D, i32,
+                                                                     i32, P, sz, P]),
+            "pkv_decode_plan_shared": (ctypes.c_int, [P, P, P, i32, D, i32, i32, P, sz, P]),
+            "pkv_decode_run_shared": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P, sz,
+                                                     P]),
+            "pkv_decode_run_shared_fp8": (ctypes.c_int, [P, P, P, P, P, P, f32, f32, f32, D, i32,
+                                                         i32, P, sz, P]),
             "pkv_copy_blocks": (ctypes.c_int, [P, P, P, i32, D, P]),
             "pkv_validate_copy_pairs": (ctypes.c_int, [P, i32, i32]),
             "pkv_slot_mapping": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
@@ -513,6 +529,156 @@ class DecodePlan:
             ctypes.byref(dims), self.max_context_len, self.partition_tokens, _p(self.workspace),
             self.workspace.numel(), _stream_ptr(q.device)))
         return out
+
+
+def decode_shared_workspace_bytes(dims: PkvDims, max_context_len: int,
+                                  partition_tokens: int = 0) -> int:
+    return load_library().pkv_decode_shared_workspace_bytes(ctypes.byref(dims), max_context_len,
+                                                            partition_tokens)
+
+
+def decode_shared_workspace_layout(dims: PkvDims, max_context_len: int,
+                                   partition_tokens: int = 0):
+    """(max_parts, part_o_offset, part_ml_offset, seq_prefix_offset) in a shared-prefix
+    decode's workspace."""
+    mp = ctypes.c_int32()
+    po, pm, sp = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load_library().pkv_decode_shared_workspace_layout(
+        ctypes.byref(dims), max_context_len, partition_tokens, ctypes.byref(mp),
+        ctypes.byref(po), ctypes.byref(pm), ctypes.byref(sp)))
+    return mp.value, po.value, pm.value, sp.value
+
+
+def _check_groups(group_start: torch.Tensor, shared_blocks: torch.Tensor, dev, num_seqs: int):
+    _need(group_start, "group_start", torch.int32, dev)
+    _need(shared_blocks, "shared_blocks", torch.int32, dev)
+    G = shared_blocks.shape[0]
+    if group_start.dim() != 1 or shared_blocks.dim() != 1 or group_start.shape[0] != G + 1:
+        raise ValueError("group_start must be int32 [num_groups + 1], shared_blocks int32 "
+                         "[num_groups]")
+    if G > num_seqs:
+        raise ValueError("num_groups must be <= num_seqs")
+    return G
+
+
+class SharedDecodePlan:
+    """A decode plan for batches whose consecutive sequences share leading blocks.
+
+    Group i is sequences ``group_start[i] .. group_start[i+1]-1`` (int32 [G+1], device);
+    every member reads its first ``shared_blocks[i]`` blocks (int32 [G], device) through the
+    first member's table row, so the shared blocks are read once per kv head for the whole
+    group.  With tables that really share those blocks the result is exactly
+    paged_attention_decode's.  Plan once per step, ``run`` (``run_fp8``) once per layer."""
+
+    def __init__(self, block_tables: torch.Tensor, context_lens: torch.Tensor,
+                 group_start: torch.Tensor, shared_blocks: torch.Tensor, num_q_heads: int,
+                 k_cache: torch.Tensor, *, max_context_len: int | None = None,
+                 partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None):
+        dev = context_lens.device
+        _need(block_tables, "block_tables", torch.int32, dev)
+        _need(context_lens, "context_lens", torch.int32, dev)
+        B = context_lens.shape[0]
+        G = _check_groups(group_start, shared_blocks, dev, B)
+        self.block_tables, self.context_lens = block_tables, context_lens
+        self.group_start, self.shared_blocks = group_start, shared_blocks
+        self.dims = make_dims(B, num_q_heads, k_cache, block_tables.shape[1])
+        self.max_context_len = (block_tables.shape[1] * k_cache.shape[2] if max_context_len is None
+                                else int(max_context_len))
+        self.partition_tokens = partition_tokens
+        need = decode_shared_workspace_bytes(self.dims, self.max_context_len, partition_tokens)
+        if need == 0:
+            raise PkvError(2, load_library().pkv_last_error_message().decode())
+        if workspace_tensor is None:
+            workspace_tensor = torch.empty(need, dtype=torch.uint8, device=dev)
+        if workspace_tensor.numel() < need:
+            raise ValueError(f"workspace_tensor has {workspace_tensor.numel()} bytes, {need} needed")
+        self.workspace = workspace_tensor
+        _check(load_library().pkv_decode_plan_shared(
+            _p(context_lens), _p(group_start), _p(shared_blocks), G, ctypes.byref(self.dims),
+            self.max_context_len, partition_tokens, _p(self.workspace), self.workspace.numel(),
+            _stream_ptr(dev)))
+
+    def _shapes(self, q, k_cache):
+        if q.shape[0] != self.dims.num_seqs or tuple(k_cache.shape) != (
+                self.dims.num_blocks, self.dims.num_kv_heads, 16, self.dims.head_dim):
+            raise ValueError("inconsistent shapes")
+
+    def run(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+            v_cache: torch.Tensor, scale: float) -> torch.Tensor:
+        dev = q.device
+        _need(q, "q", device=dev)
+        _need(out, "out", q.dtype, dev)
+        _need(k_cache, "k_cache", q.dtype, dev)
+        _need(v_cache, "v_cache", q.dtype, dev)
+        if out.shape != q.shape or v_cache.shape != k_cache.shape:
+            raise ValueError("inconsistent shapes")
+        self._shapes(q, k_cache)
+        _check(load_library().pkv_decode_run_shared(
+            _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
+            _p(self.context_lens), float(scale), ctypes.byref(self.dims), self.max_context_len,
+            self.partition_tokens, _p(self.workspace), self.workspace.numel(), _stream_ptr(dev)))
+        return out
+
+    def run_fp8(self, out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, scale: float, k_scale: float,
+                v_scale: float) -> torch.Tensor:
+        """``run`` over FP8 caches (see paged_attention_decode_fp8)."""
+        _check_fp8_decode(out, q, k_cache, v_cache, self.block_tables, self.context_lens)
+        self._shapes(q, k_cache)
+        dims = PkvDims(*[getattr(self.dims, f) for f, _ in PkvDims._fields_[:-1]],
+                       _dtype_code(k_cache.dtype))
+        _check(load_library().pkv_decode_run_shared_fp8(
+            _p(out), _p(q), _p(k_cache), _p(v_cache), _p(self.block_tables),
+            _p(self.context_lens), float(scale), float(k_scale), float(v_scale),
+            ctypes.byref(dims), self.max_context_len, self.partition_tokens, _p(self.workspace),
+            self.workspace.numel(), _stream_ptr(q.device)))
+        return out
+
+
+def paged_attention_decode_shared(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                                  v_cache: torch.Tensor, block_tables: torch.Tensor,
+                                  context_lens: torch.Tensor, group_start: torch.Tensor,
+                                  shared_blocks: torch.Tensor, scale: float, *,
+                                  k_scale: float | None = None, v_scale: float | None = None,
+                                  max_context_len: int | None = None, partition_tokens: int = 0,
+                                  workspace_tensor: torch.Tensor | None = None) -> torch.Tensor:
+    """Decode with shared prefixes read once per group (see SharedDecodePlan), in one call:
+    the plan, the decode and the merge.  FP8 pools take k_scale and v_scale."""
+    dev = q.device
+    fp8 = k_cache.dtype in FP8_DTYPES
+    if fp8:
+        _check_fp8_decode(out, q, k_cache, v_cache, block_tables, context_lens)
+        if k_scale is None or v_scale is None:
+            raise ValueError("FP8 pools need k_scale and v_scale")
+    else:
+        _need(q, "q", device=dev)
+        _need(out, "out", q.dtype, dev)
+        _need(k_cache, "k_cache", q.dtype, dev)
+        _need(v_cache, "v_cache", q.dtype, dev)
+        _need(block_tables, "block_tables", torch.int32, dev)
+        _need(context_lens, "context_lens", torch.int32, dev)
+    B, hq, d = q.shape
+    if out.shape != q.shape or block_tables.dim() != 2 or block_tables.shape[0] != B \
+            or context_lens.shape != (B,) or k_cache.dim() != 4 or v_cache.shape != k_cache.shape \
+            or k_cache.shape[3] != d:
+        raise ValueError("inconsistent shapes")
+    G = _check_groups(group_start, shared_blocks, dev, B)
+    dims = make_dims(B, hq, k_cache, block_tables.shape[1])
+    mcl = block_tables.shape[1] * k_cache.shape[2] if max_context_len is None else int(max_context_len)
+    need = decode_shared_workspace_bytes(dims, mcl, partition_tokens)
+    if need == 0:
+        raise PkvError(2, load_library().pkv_last_error_message().decode())
+    ws = workspace_tensor if workspace_tensor is not None else workspace(dev, need)
+    lib = load_library()
+    head = [_p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+            _p(group_start), _p(shared_blocks), G, float(scale)]
+    tail = [ctypes.byref(dims), mcl, partition_tokens, _p(ws), ws.numel(), _stream_ptr(dev)]
+    if fp8:
+        _check(lib.pkv_paged_attention_decode_shared_fp8(*head, float(k_scale), float(v_scale),
+                                                         *tail))
+    else:
+        _check(lib.pkv_paged_attention_decode_shared(*head, *tail))
+    return out
 
 
 def reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,

@@ -126,7 +126,11 @@ struct DecodePlan {
   int32_t max_parts = 0;
   int32_t max_len = 0;       // lengths above this are clamped (and flagged)
   int32_t num_q_tokens = 0;  // query rows of q and out (num_seqs for decode)
+  // shared-prefix plans: sequences one shared-prefix item serves (x group <= 16 rows)
+  bool shared = false;
+  int32_t members_per_item = 0;
   size_t items_off = 0, part_o_off = 0, part_ml_off = 0, total = 0;
+  size_t seq_prefix_off = 0, group_pref_off = 0;
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -147,9 +151,12 @@ int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested) 
   return static_cast<int32_t>(p);
 }
 
-// num_q_tokens < 0: one query token per sequence (decode).
+// num_q_tokens < 0: one query token per sequence (decode).  shared: the
+// shared-prefix plan (decode only), whose sequences may have one partial more
+// (the prefix is split from the rest at a block boundary) and whose work list
+// holds up to two items per partial row.
 pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partition_tokens,
-                     DecodePlan* plan, int32_t num_q_tokens = -1) {
+                     DecodePlan* plan, int32_t num_q_tokens = -1, bool shared = false) {
   pkv_status st = check_dims(d, true);
   if (st != PKV_OK) return st;
   if (max_context_len < 0) return fail(PKV_ERR_SHAPE, "max_context_len must be >= 0");
@@ -168,9 +175,23 @@ pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partiti
   p.part_blocks = p.part_tokens / pkv::kBlock;
   p.max_parts = max_len <= 0 ? 1 : (max_len + p.part_tokens - 1) / p.part_tokens;
   const size_t B = static_cast<size_t>(d->num_seqs);
+  size_t max_items = B * p.max_parts;
+  if (shared) {
+    const int group = d->num_q_heads / d->num_kv_heads;
+    p.shared = true;
+    p.members_per_item = group <= 8 ? 16 / group : 1;
+    p.max_parts += 1;
+    max_items = 2 * B * p.max_parts;
+  }
   const size_t rows = static_cast<size_t>(p.num_q_tokens) * d->num_q_heads * p.max_parts;
   p.items_off = 256;
-  size_t off = round_up(p.items_off + B * p.max_parts * sizeof(pkv::PlanItem), 256);
+  size_t off = round_up(p.items_off + max_items * sizeof(pkv::PlanItem), 256);
+  if (shared) {
+    p.seq_prefix_off = off;
+    off = round_up(off + B * sizeof(int32_t), 256);
+    p.group_pref_off = off;
+    off = round_up(off + B * sizeof(int32_t), 256);
+  }
   if (p.max_parts > 1) {
     p.part_o_off = off;
     off = round_up(off + rows * d->head_dim * sizeof(float), 256);
@@ -345,8 +366,10 @@ pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
   const float* pml = reinterpret_cast<const float*>(ws + plan.part_ml_off);
   auto kern = d->head_dim == 128 ? pkv::merge_kernel<T, 128> : pkv::merge_kernel<T, 64>;
   cudaError_t e = launch(kern, dim3(grid), dim3(pkv::kMergeWarps * 32), 0, stream, out, po, pml,
-                         context_lens,
-                         query_start_loc, d->num_seqs, plan.num_q_tokens, d->num_q_heads,
+                         context_lens, query_start_loc,
+                         plan.shared ? reinterpret_cast<const int32_t*>(ws + plan.seq_prefix_off)
+                                     : nullptr,
+                         d->num_seqs, plan.num_q_tokens, d->num_q_heads,
                          plan.max_parts, plan.max_len, plan.part_tokens);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return PKV_OK;
@@ -405,6 +428,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   // Up to 16 query rows per item (an item's rows share one MMA tile); a longer
   // chunk is split into row groups of whole tokens, each read against the
   // keys its rows can see.
+  // A shared-prefix plan serves one token of up to members_per_item sequences per item.
+  if (plan.shared) max_query_len = plan.members_per_item;
   const int group_tokens = max_query_len * group <= 16 ? max_query_len : 16 / group;
   const int row_groups = (max_query_len + group_tokens - 1) / group_tokens;
   const int rows_max = group_tokens * group;
@@ -437,8 +462,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.part_blocks = plan.part_blocks;
   prm.qk_scale_log2 = scale * pkv::kLog2e * k_scale;
   prm.out_scale = v_scale;
-  const int64_t units =
-      static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads * row_groups;
+  const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads *
+                        (plan.shared ? 2 : row_groups);
   if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_FP8_E5M2) {
@@ -574,6 +599,89 @@ pkv_status multi_one_shot(void* out, const void* q, const void* k_cache, const v
   return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
                     max_query_len, scale, dims, plan, workspace, workspace_bytes, cuda_stream,
                     k_scale, v_scale);
+}
+
+}  // namespace
+
+namespace {
+
+// The shared-prefix decode: its plan, and the run over it (bf16 / fp32 pools,
+// or FP8 pools with their scales when `fp8`).
+pkv_status plan_shared(const int32_t* context_lens, const int32_t* group_start,
+                       const int32_t* shared_blocks, int32_t num_groups, const pkv_dims* dims,
+                       int32_t max_context_len, int32_t partition_tokens, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, -1, true);
+  if (st != PKV_OK) return st;
+  if (num_groups < 0 || num_groups > dims->num_seqs)
+    return fail(PKV_ERR_SHAPE, "num_groups must be in [0, num_seqs]");
+  if (dims->num_seqs == 0) return PKV_OK;
+  if (!context_lens || !group_start || (num_groups > 0 && !shared_blocks))
+    return fail(PKV_ERR_NULL, "context_lens, group_start or shared_blocks is NULL");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  if ((st = bind_device(workspace, "workspace")) != PKV_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaError_t e = launch(pkv::plan_shared_kernel, dim3(1), dim3(pkv::kPlanThreads), 0,
+                         static_cast<cudaStream_t>(cuda_stream), context_lens, group_start,
+                         shared_blocks, num_groups, dims->num_seqs, plan.max_len,
+                         plan.part_blocks, plan.members_per_item,
+                         reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off),
+                         reinterpret_cast<uint32_t*>(ws),
+                         reinterpret_cast<int32_t*>(ws + plan.seq_prefix_off),
+                         reinterpret_cast<int32_t*>(ws + plan.group_pref_off));
+  if (e != cudaSuccess) return cuda_fail(e, "shared-prefix plan launch");
+  return PKV_OK;
+}
+
+pkv_status check_pool_kind(const pkv_dims* dims, bool fp8, float k_scale, float v_scale) {
+  if (fp8) {
+    if (!is_fp8(dims->dtype)) return fail(PKV_ERR_UNSUPPORTED, "dims->dtype must be FP8");
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+        !std::isfinite(v_scale))
+      return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive");
+  } else if (is_fp8(dims->dtype)) {
+    return fail(PKV_ERR_UNSUPPORTED, "FP8 pools need their scales: use the _fp8 calls");
+  }
+  return PKV_OK;
+}
+
+pkv_status run_shared(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, const int32_t* context_lens, float scale,
+                      bool fp8, float k_scale, float v_scale, const pkv_dims* dims,
+                      int32_t max_context_len, int32_t partition_tokens, void* workspace,
+                      size_t workspace_bytes, void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, -1, true);
+  if (st != PKV_OK) return st;
+  if ((st = check_pool_kind(dims, fp8, k_scale, v_scale)) != PKV_OK) return st;
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
+                    dims, plan, workspace, workspace_bytes, cuda_stream, k_scale, v_scale);
+}
+
+pkv_status shared_one_shot(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens,
+                           const int32_t* group_start, const int32_t* shared_blocks,
+                           int32_t num_groups, float scale, bool fp8, float k_scale,
+                           float v_scale, const pkv_dims* dims, int32_t max_context_len,
+                           int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                           void* cuda_stream) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, -1, true);
+  if (st != PKV_OK) return st;
+  if ((st = check_pool_kind(dims, fp8, k_scale, v_scale)) != PKV_OK) return st;
+  if (dims->num_seqs == 0) return PKV_OK;
+  // Check everything the run needs before launching the plan.
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  st = plan_shared(context_lens, group_start, shared_blocks, num_groups, dims, max_context_len,
+                   partition_tokens, workspace, workspace_bytes, cuda_stream);
+  if (st != PKV_OK) return st;
+  return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
+                    dims, plan, workspace, workspace_bytes, cuda_stream, k_scale, v_scale);
 }
 
 }  // namespace
@@ -784,6 +892,82 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
   if (st != PKV_OK) return st;
   return run_decode(out, q, k_cache, v_cache, block_tables, context_lens, nullptr, 1, scale,
                     dims, plan, workspace, workspace_bytes, cuda_stream, k_scale, v_scale);
+}
+
+size_t pkv_decode_shared_workspace_bytes(const pkv_dims* dims, int32_t max_context_len,
+                                         int32_t partition_tokens) {
+  DecodePlan plan;
+  if (make_plan(dims, max_context_len, partition_tokens, &plan, -1, true) != PKV_OK) return 0;
+  return plan.total;
+}
+
+pkv_status pkv_decode_shared_workspace_layout(const pkv_dims* dims, int32_t max_context_len,
+                                              int32_t partition_tokens, int32_t* max_parts,
+                                              size_t* part_o_offset, size_t* part_ml_offset,
+                                              size_t* seq_prefix_offset) {
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, -1, true);
+  if (st != PKV_OK) return st;
+  if (max_parts) *max_parts = plan.max_parts;
+  if (part_o_offset) *part_o_offset = plan.part_o_off;
+  if (part_ml_offset) *part_ml_offset = plan.part_ml_off;
+  if (seq_prefix_offset) *seq_prefix_offset = plan.seq_prefix_off;
+  return PKV_OK;
+}
+
+pkv_status pkv_decode_plan_shared(const int32_t* context_lens, const int32_t* group_start,
+                                  const int32_t* shared_blocks, int32_t num_groups,
+                                  const pkv_dims* dims, int32_t max_context_len,
+                                  int32_t partition_tokens, void* workspace,
+                                  size_t workspace_bytes, void* cuda_stream) {
+  return plan_shared(context_lens, group_start, shared_blocks, num_groups, dims,
+                     max_context_len, partition_tokens, workspace, workspace_bytes, cuda_stream);
+}
+
+pkv_status pkv_decode_run_shared(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, float scale, const pkv_dims* dims,
+                                 int32_t max_context_len, int32_t partition_tokens,
+                                 void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  return run_shared(out, q, k_cache, v_cache, block_tables, context_lens, scale, false, 1.f,
+                    1.f, dims, max_context_len, partition_tokens, workspace, workspace_bytes,
+                    cuda_stream);
+}
+
+pkv_status pkv_decode_run_shared_fp8(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, float scale, float k_scale,
+                                     float v_scale, const pkv_dims* dims,
+                                     int32_t max_context_len, int32_t partition_tokens,
+                                     void* workspace, size_t workspace_bytes,
+                                     void* cuda_stream) {
+  return run_shared(out, q, k_cache, v_cache, block_tables, context_lens, scale, true, k_scale,
+                    v_scale, dims, max_context_len, partition_tokens, workspace,
+                    workspace_bytes, cuda_stream);
+}
+
+pkv_status pkv_paged_attention_decode_shared(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
+    const int32_t* shared_blocks, int32_t num_groups, float scale, const pkv_dims* dims,
+    int32_t max_context_len, int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+    void* cuda_stream) {
+  return shared_one_shot(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                         shared_blocks, num_groups, scale, false, 1.f, 1.f, dims,
+                         max_context_len, partition_tokens, workspace, workspace_bytes,
+                         cuda_stream);
+}
+
+pkv_status pkv_paged_attention_decode_shared_fp8(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* group_start,
+    const int32_t* shared_blocks, int32_t num_groups, float scale, float k_scale, float v_scale,
+    const pkv_dims* dims, int32_t max_context_len, int32_t partition_tokens, void* workspace,
+    size_t workspace_bytes, void* cuda_stream) {
+  return shared_one_shot(out, q, k_cache, v_cache, block_tables, context_lens, group_start,
+                         shared_blocks, num_groups, scale, true, k_scale, v_scale, dims,
+                         max_context_len, partition_tokens, workspace, workspace_bytes,
+                         cuda_stream);
 }
 
 pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,

@@ -43,12 +43,21 @@ constexpr int kRing = 4;          // items in flight between producer and consum
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// One unit of planned work: tokens [p*part_blocks*16, ...) of sequence s.
+// One unit of planned work.  An ordinary item covers blocks blk0 .. of
+// sequence `seq` (at most part_blocks of them) for that sequence's own query
+// rows.  A shared-prefix item (q_start >= 0) covers blocks blk0 .. of a
+// prefix that the q_len consecutive sequences q_start .. q_start + q_len - 1
+// share, read through the table of `seq` (the first of them), for one query
+// token of each of those sequences at once.
 struct PlanItem {
-  int32_t seq;
-  int32_t part;
-  int32_t len;     // context length of the sequence, after validation
-  int32_t nparts;  // partitions of the sequence
+  int32_t seq;      // sequence whose block table is read
+  int32_t part;     // partial-result slot of the rows (used when nparts > 1)
+  int32_t len;      // keys at positions < len belong to the item's context
+  int32_t nparts;   // 1: the item is its rows' whole context (output written directly)
+  int32_t blk0;     // first block
+  int32_t q_start;  // shared-prefix items: first query row; -1: the rows of `seq`
+  int32_t q_len;    // shared-prefix items: sequences served
+  int32_t pad;
 };
 
 // Context length after validation against the table width and the host's
@@ -80,28 +89,13 @@ __device__ __forceinline__ int32_t part_size_blocks(int32_t L, int32_t p, int32_
   return rest < part_blocks ? rest : part_blocks;
 }
 
-// The plan, run by one CTA of kPlanThreads threads: counts the work items per
-// size, scans, and writes them sorted by size (largest first).  counters[0] =
-// work counter, counters[1] = items, counters[2] = CTAs finished; the work and
-// finish counters are zeroed here, and the decode kernel's last CTA zeroes
-// them again, so one plan serves any number of runs.  The caller has already
-// passed griddepcontrol.wait.
-__device__ __forceinline__ void plan_body(const int32_t* __restrict__ context_lens,
-                                          int32_t num_seqs, int32_t max_len, int32_t part_blocks,
-                                          PlanItem* __restrict__ items,
-                                          uint32_t* __restrict__ counters, uint32_t* hist,
-                                          uint32_t* warp_sums) {
+// Exclusive scan of the item-size histogram in descending bucket order (one
+// CTA of kPlanThreads threads, thread i owning bucket kPlanBuckets-1-i):
+// afterwards hist[b] is the position of bucket b's first item.  Also sets
+// counters[1] = number of items and zeroes the work and finish counters.
+__device__ __forceinline__ void plan_scan(uint32_t* hist, uint32_t* warp_sums,
+                                          uint32_t* __restrict__ counters) {
   const int tid = threadIdx.x;
-  const int32_t part_tokens = part_blocks * kBlock;
-  for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
-  __syncthreads();
-  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
-    int32_t L = checked_len(context_lens[s], max_len);
-    int32_t n = num_parts(L, part_tokens);
-    for (int32_t p = 0; p < n; ++p) atomicAdd(&hist[plan_bucket(part_size_blocks(L, p, part_blocks))], 1u);
-  }
-  __syncthreads();
-  // Exclusive scan in descending bucket order: thread i owns bucket B-1-i.
   const int bucket = kPlanBuckets - 1 - tid;
   uint32_t v = hist[bucket];
   uint32_t incl = v;
@@ -132,13 +126,37 @@ __device__ __forceinline__ void plan_body(const int32_t* __restrict__ context_le
     counters[2] = 0u;
   }
   __syncthreads();
+}
+
+// The plan, run by one CTA of kPlanThreads threads: counts the work items per
+// size, scans, and writes them sorted by size (largest first).  counters[0] =
+// work counter, counters[1] = items, counters[2] = CTAs finished; the work and
+// finish counters are zeroed here, and the decode kernel's last CTA zeroes
+// them again, so one plan serves any number of runs.  The caller has already
+// passed griddepcontrol.wait.
+__device__ __forceinline__ void plan_body(const int32_t* __restrict__ context_lens,
+                                          int32_t num_seqs, int32_t max_len, int32_t part_blocks,
+                                          PlanItem* __restrict__ items,
+                                          uint32_t* __restrict__ counters, uint32_t* hist,
+                                          uint32_t* warp_sums) {
+  const int tid = threadIdx.x;
+  const int32_t part_tokens = part_blocks * kBlock;
+  for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
+  __syncthreads();
+  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
+    int32_t L = checked_len(context_lens[s], max_len);
+    int32_t n = num_parts(L, part_tokens);
+    for (int32_t p = 0; p < n; ++p) atomicAdd(&hist[plan_bucket(part_size_blocks(L, p, part_blocks))], 1u);
+  }
+  __syncthreads();
+  plan_scan(hist, warp_sums, counters);
   for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
     int32_t L = context_lens[s];
     L = L < 0 ? 0 : (L > max_len ? max_len : L);
     int32_t n = num_parts(L, part_tokens);
     for (int32_t p = 0; p < n; ++p) {
       uint32_t pos = atomicAdd(&hist[plan_bucket(part_size_blocks(L, p, part_blocks))], 1u);
-      items[pos] = PlanItem{s, p, L, n};
+      items[pos] = PlanItem{s, p, L, n, p * part_blocks, -1, 0, 0};
     }
   }
 }
@@ -153,6 +171,148 @@ __global__ void __launch_bounds__(kPlanThreads)
   pdl_wait();
   pdl_trigger();
   plan_body(context_lens, num_seqs, max_len, part_blocks, items, counters, hist, warp_sums);
+}
+
+// ------------------------------------------------------- shared-prefix plan
+// Parallel samples of one prompt (or requests behind one system prompt) hold
+// the same physical blocks at the start of their tables: the pages' prefix
+// sharing with reference counts ("vLLM 深读：用 PagedAttention 撑起高并发 LLM
+// 推理", section "先看浪费在哪里").  This plan reads such a prefix once per kv
+// head for a whole group of sequences: a shared-prefix item multiplies its
+// tiles against one query token of each of up to `members_per_item`
+// sequences, and each sequence's own blocks after the prefix become ordinary
+// items; the two partial results meet in the log-sum-exp merge.
+//
+// Group i covers sequences group_start[i] .. group_start[i+1] - 1 (bounds
+// nondecreasing within [0, num_seqs]; a sequence in no group has no shared
+// prefix).  Every member's first shared_blocks[i] blocks are read through the
+// FIRST member's table.  A group of fewer than two members, or bounds that
+// are not nondecreasing in [0, num_seqs] (flagged PKV_DEVERR_GROUP, then no
+// group is used), give no shared prefix; a negative count, or one beyond a
+// member's full blocks, is raised to 0 or lowered to them and flagged
+// PKV_DEVERR_GROUP.
+//
+// Outputs besides the work list: seq_prefix[s] = shared blocks of sequence s
+// (what the merge needs to count its partials), group_pref[i] scratch.  The
+// partials of a sequence with P shared blocks are slots 0 .. np(P*16) - 1
+// for the prefix and np(P*16) .. for its own tokens, np = num_parts.
+
+// The group holding sequence s (groups 0 .. G-1 with nondecreasing bounds), or -1.
+__device__ __forceinline__ int32_t group_of(const int32_t* __restrict__ group_start, int32_t G,
+                                            int32_t s) {
+  if (G <= 0 || s < group_start[0] || s >= group_start[G]) return -1;
+  int32_t lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int32_t mid = (lo + hi + 1) / 2;
+    if (group_start[mid] <= s) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+    plan_shared_kernel(const int32_t* __restrict__ context_lens,
+                       const int32_t* __restrict__ group_start,
+                       const int32_t* __restrict__ shared_blocks, int32_t num_groups,
+                       int32_t num_seqs, int32_t max_len, int32_t part_blocks,
+                       int32_t members_per_item, PlanItem* __restrict__ items,
+                       uint32_t* __restrict__ counters, int32_t* __restrict__ seq_prefix,
+                       int32_t* group_pref) {
+  __shared__ uint32_t hist[kPlanBuckets];
+  __shared__ uint32_t warp_sums[kPlanThreads / 32];
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const int32_t part_tokens = part_blocks * kBlock;
+  for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
+  // the group bounds
+  int bad = 0;
+  for (int32_t i = tid; i <= num_groups; i += kPlanThreads) {
+    const int32_t a = group_start[i];
+    if (a < 0 || a > num_seqs || (i < num_groups && a > group_start[i + 1])) bad = 1;
+  }
+  const bool groups_ok = __syncthreads_or(bad) == 0;
+  if (!groups_ok && tid == 0) raise_error(PKV_DEVERR_GROUP);
+  const int32_t G = groups_ok ? num_groups : 0;
+  // each group's prefix as given, within the table width; none (and no check)
+  // for a group of fewer than two members
+  for (int32_t i = tid; i < G; i += kPlanThreads) {
+    int32_t p = 0;
+    if (group_start[i + 1] - group_start[i] >= 2) {
+      p = shared_blocks[i];
+      const int32_t cap = max_len / kBlock;
+      if (p < 0 || p > cap) {
+        raise_error(PKV_DEVERR_GROUP);
+        p = p < 0 ? 0 : cap;
+      }
+    }
+    group_pref[i] = p;
+  }
+  __syncthreads();
+  // ... and never past a member's own full blocks
+  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
+    const int32_t gi = group_of(group_start, G, s);
+    if (gi < 0) continue;
+    const int32_t full = checked_len(context_lens[s], max_len) / kBlock;
+    if (full < group_pref[gi]) {
+      raise_error(PKV_DEVERR_GROUP);
+      atomicMin(&group_pref[gi], full);
+    }
+  }
+  __syncthreads();
+  // sizes: each sequence's own partitions, each group's prefix partitions
+  // (one item per members_per_item sequences)
+  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
+    const int32_t gi = group_of(group_start, G, s);
+    const int32_t pref = gi >= 0 ? group_pref[gi] : 0;
+    seq_prefix[s] = pref;
+    const int32_t tail = checked_len(context_lens[s], max_len) - pref * kBlock;
+    const int32_t n = num_parts(tail, part_tokens);
+    for (int32_t p = 0; p < n; ++p)
+      atomicAdd(&hist[plan_bucket(part_size_blocks(tail, p, part_blocks))], 1u);
+  }
+  for (int32_t i = tid; i < G; i += kPlanThreads) {
+    const int32_t pref = group_pref[i];
+    if (pref == 0) continue;
+    const int32_t members = group_start[i + 1] - group_start[i];
+    const uint32_t per = static_cast<uint32_t>((members + members_per_item - 1) / members_per_item);
+    const int32_t n = num_parts(pref * kBlock, part_tokens);
+    for (int32_t p = 0; p < n; ++p)
+      atomicAdd(&hist[plan_bucket(part_size_blocks(pref * kBlock, p, part_blocks))], per);
+  }
+  __syncthreads();
+  plan_scan(hist, warp_sums, counters);
+  for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
+    const int32_t pref = seq_prefix[s];
+    int32_t L = context_lens[s];
+    L = L < 0 ? 0 : (L > max_len ? max_len : L);
+    const int32_t tail = L - pref * kBlock;
+    const int32_t np = pref > 0 ? num_parts(pref * kBlock, part_tokens) : 0;
+    const int32_t n = num_parts(tail, part_tokens);
+    for (int32_t p = 0; p < n; ++p) {
+      const uint32_t pos = atomicAdd(&hist[plan_bucket(part_size_blocks(tail, p, part_blocks))], 1u);
+      items[pos] = PlanItem{s, np + p, L, np + n, pref + p * part_blocks, -1, 0, 0};
+    }
+  }
+  for (int32_t i = tid; i < G; i += kPlanThreads) {
+    const int32_t pref = group_pref[i];
+    if (pref == 0) continue;
+    const int32_t first = group_start[i], members = group_start[i + 1] - first;
+    const int32_t per = (members + members_per_item - 1) / members_per_item;
+    const int32_t n = num_parts(pref * kBlock, part_tokens);
+    for (int32_t p = 0; p < n; ++p) {
+      // the items of one partition sit next to each other: their tiles are
+      // read close in time and mostly served once from HBM
+      const uint32_t pos = atomicAdd(
+          &hist[plan_bucket(part_size_blocks(pref * kBlock, p, part_blocks))], static_cast<uint32_t>(per));
+      for (int32_t j = 0; j < per; ++j) {
+        const int32_t q0 = first + j * members_per_item;
+        const int32_t qn = members - j * members_per_item < members_per_item
+                               ? members - j * members_per_item
+                               : members_per_item;
+        items[pos + j] = PlanItem{first, p, pref * kBlock, 2, p * part_blocks, q0, qn, 0};
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------ decode kernel
@@ -240,7 +400,11 @@ struct DecodeLayout {
 struct ItemMeta {
   int32_t seq, kv_head, part, len, nparts, blk_begin, nblk;
   int32_t q_start, q_len;        // query rows of the chunk and its length
+  // rows of token i see keys up to len - q_causal + i: q_causal = q_len for a
+  // causal chunk, 1 for a shared prefix (every row sees every key of it)
+  int32_t q_causal;
 };
+static_assert(sizeof(ItemMeta) <= 64, "a ring slot's metadata area is 64 bytes");
 
 // ---- consumer state for bf16 (tensor cores) ----
 //
@@ -1004,10 +1168,20 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
       const uint32_t rem = widx % per_item;
       const int32_t kvh = static_cast<int32_t>(rem / prm.row_groups);
       const int32_t grp = static_cast<int32_t>(rem % prm.row_groups);
-      const int32_t blk_begin = pi.part * prm.part_blocks;
-      // the chunk of query tokens: one per sequence unless query_start_loc is given
+      const int32_t blk_begin = pi.blk0;
+      // the chunk of query tokens: one per sequence unless query_start_loc is
+      // given; a shared-prefix item serves one token of each of q_len sequences
       int32_t q_start = pi.seq, q_len = 1;
-      if (prm.query_start_loc) {
+      const bool shared = pi.q_start >= 0;
+      if (shared) {
+        q_start = pi.q_start;
+        q_len = pi.q_len;
+        if (q_len < 0 || q_len > prm.group_tokens || q_start + q_len > prm.num_q_tokens) {
+          if (lane == 0 && kvh == 0) raise_error(PKV_DEVERR_GROUP);
+          q_start = 0;
+          q_len = 0;
+        }
+      } else if (prm.query_start_loc) {
         q_start = prm.query_start_loc[pi.seq];
         q_len = prm.query_start_loc[pi.seq + 1] - q_start;
         const int32_t cap = pi.len < prm.max_query_len ? pi.len : prm.max_query_len;
@@ -1049,6 +1223,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
         mt.nblk = nblk;
         mt.q_start = q_start;
         mt.q_len = q_len;
+        mt.q_causal = shared ? 1 : q_len;
         const uint32_t row_bytes = static_cast<uint32_t>(g * D * QELEM);  // one token's group
         if (q_len > 0) {
           mbar_arrive_expect_tx(&item_full[r], row_bytes * q_len);
@@ -1188,11 +1363,11 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
                                    : (rows - row0 < 0 ? 0 : (rows - row0 < RPW ? rows - row0 : RPW));
     const uint8_t* my_qs = qs + row0 * D * QELEM;
     if constexpr (kFp8) {
-      fp8_begin_item<RPW>(st, my_qs, my_rows, g, it.len, it.q_len, lane, row0);
+      fp8_begin_item<RPW>(st, my_qs, my_rows, g, it.len, it.q_causal, lane, row0);
     } else if constexpr (kBf16) {
-      bf16_begin_item<D, RPW>(st, my_qs, my_rows, g, it.len, it.q_len, lane, row0);
+      bf16_begin_item<D, RPW>(st, my_qs, my_rows, g, it.len, it.q_causal, lane, row0);
     } else {
-      f32_begin_item<D, GMAX>(st, rows, g, it.len, it.q_len);
+      f32_begin_item<D, GMAX>(st, rows, g, it.len, it.q_causal);
     }
     // bf16 consumes the blocks two at a time (b and b + L), fp32 one at a time.
     constexpr int kStep = (kBf16 || kFp8) ? 2 : 1;
@@ -1289,7 +1464,7 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 
 // ------------------------------------------------------------- merge kernel
 // One CTA of kMergeWarps warps per (query token, query head) row whose
-// sequence was split: combine the partitions' (m, l, o) by log-sum-exp and
+// sequence was split (or read a shared prefix separately): combine the partitions' (m, l, o) by log-sum-exp and
 // store the final output.  Every warp finds the common maximum M, takes every
 // kMergeWarps-th partition (so a row's partials stream in on several warps at
 // once), and warp 0 adds the warps' sums in a fixed order.  Partitions a causal
@@ -1300,7 +1475,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(void* __restrict__ out, const float* __restrict__ part_o,
                  const float* __restrict__ part_ml, const int32_t* __restrict__ context_lens,
-                 const int32_t* __restrict__ query_start_loc, int32_t num_seqs,
+                 const int32_t* __restrict__ query_start_loc,
+                 const int32_t* __restrict__ seq_prefix, int32_t num_seqs,
                  int32_t num_q_tokens, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
                  int32_t part_tokens) {
   constexpr int VEC = D / 32;  // floats per lane
@@ -1324,7 +1500,10 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   }
   int32_t L = context_lens[s];
   L = L < 0 ? 0 : (L > max_len ? max_len : L);
-  const int32_t n = num_parts(L, part_tokens);
+  // partials: those of a shared prefix of P blocks (if any), then the sequence's own
+  const int32_t P = seq_prefix ? seq_prefix[s] : 0;
+  const int32_t n = (P > 0 ? num_parts(P * kBlock, part_tokens) : 0) +
+                    num_parts(L - P * kBlock, part_tokens);
   if (n <= 1) return;  // the decode kernel wrote this row directly (uniform over the CTA)
   const float* ml = part_ml + row * max_parts * 2;
   float M = -INFINITY;

@@ -525,8 +525,12 @@ def c4_shared_prefix(device="cpu", prompts: int = 32, samples: int = 8, prefix: 
             lens.append(L)
             seq_ids.extend([s] * (L - P0))
             positions.extend(range(P0, L))
+    # the samples of prompt i are sequences i*samples .. (i+1)*samples - 1; all of them
+    # keep the prompt's full blocks (the partial last one is copied on a sample's first write)
     meta = {"prompts": prompts, "samples": samples, "prefix_lens": prefix_lens.tolist(),
-            "tails": tails.reshape(-1).tolist(), "blocks_in_use": bm.blocks_in_use()}
+            "tails": tails.reshape(-1).tolist(), "blocks_in_use": bm.blocks_in_use(),
+            "group_start": [i * samples for i in range(prompts + 1)],
+            "shared_blocks": [int(p) // BLOCK_SIZE for p in prefix_lens]}
     return _assemble("c4_shared_prefix", seed, "bf16", 32, 8, 128, nb, np.array(lens),
                      tables, initial, np.array(prefill), np.array(seq_ids, dtype=np.int64),
                      np.array(positions, dtype=np.int64), bm.cow_pairs, device, meta)
