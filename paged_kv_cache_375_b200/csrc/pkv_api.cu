@@ -355,16 +355,24 @@ pkv_status check_workspace(const DecodePlan& plan, const void* workspace, size_t
   return PKV_OK;
 }
 
+// The merge: one warp per row when a row has at most 8 partials (the common
+// case: a few partitions, or a shared prefix and the sequence's own blocks),
+// else the CTA's kMergeWarps warps per row.
 template <typename T>
 pkv_status launch_merge(void* out, const DecodePlan& plan, uint8_t* ws,
                         const int32_t* context_lens, const int32_t* query_start_loc,
                         const pkv_dims* d, cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(plan.num_q_tokens) * d->num_q_heads;
   if (rows > 0x7fffffff) return fail(PKV_ERR_UNSUPPORTED, "too many query rows for the merge");
-  const unsigned grid = static_cast<unsigned>(rows);  // one CTA per row
+  const bool warp_rows = plan.max_parts <= 8;
+  const int64_t per_cta = warp_rows ? pkv::kMergeWarps : 1;
+  const unsigned grid = static_cast<unsigned>((rows + per_cta - 1) / per_cta);
   const float* po = reinterpret_cast<const float*>(ws + plan.part_o_off);
   const float* pml = reinterpret_cast<const float*>(ws + plan.part_ml_off);
-  auto kern = d->head_dim == 128 ? pkv::merge_kernel<T, 128> : pkv::merge_kernel<T, 64>;
+  const bool d128 = d->head_dim == 128;
+  auto kern = warp_rows ? (d128 ? pkv::merge_kernel<T, 128, 1> : pkv::merge_kernel<T, 64, 1>)
+                        : (d128 ? pkv::merge_kernel<T, 128, pkv::kMergeWarps>
+                                : pkv::merge_kernel<T, 64, pkv::kMergeWarps>);
   cudaError_t e = launch(kern, dim3(grid), dim3(pkv::kMergeWarps * 32), 0, stream, out, po, pml,
                          context_lens, query_start_loc,
                          plan.shared ? reinterpret_cast<const int32_t*>(ws + plan.seq_prefix_off)

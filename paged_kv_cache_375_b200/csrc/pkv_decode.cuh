@@ -11,6 +11,10 @@
 //    (sequence, partition), longest first.  A partition is at most
 //    `part_blocks` blocks; a sequence longer than one partition is split
 //    (split-K) and its partial results are merged by log-sum-exp afterwards.
+//    A second planner serves batches whose consecutive sequences share their
+//    leading blocks: a shared-prefix item reads those blocks once for one
+//    query token of each of several sequences, and their partial results
+//    are merged with those of each sequence's own blocks.
 //  * The decode kernel is persistent (one CTA per SM).  Work units (item x kv
 //    head x row group) are handed out through an atomic counter by a
 //    scheduler warp, which publishes each into a ring in shared memory: its
@@ -198,8 +202,9 @@ __global__ void __launch_bounds__(kPlanThreads)
 // for the prefix and np(P*16) .. for its own tokens, np = num_parts.
 
 // The group holding sequence s (groups 0 .. G-1 with nondecreasing bounds), or -1.
-__device__ __forceinline__ int32_t group_of(const int32_t* __restrict__ group_start, int32_t G,
-                                            int32_t s) {
+constexpr int kPlanGroupCache = 2048;
+
+__device__ __forceinline__ int32_t group_of(const int32_t* group_start, int32_t G, int32_t s) {
   if (G <= 0 || s < group_start[0] || s >= group_start[G]) return -1;
   int32_t lo = 0, hi = G - 1;
   while (lo < hi) {
@@ -219,25 +224,29 @@ __global__ void __launch_bounds__(kPlanThreads)
                        int32_t* group_pref) {
   __shared__ uint32_t hist[kPlanBuckets];
   __shared__ uint32_t warp_sums[kPlanThreads / 32];
+  __shared__ int32_t gs_cache[kPlanGroupCache];  // the group bounds, when they fit
   pdl_wait();
   pdl_trigger();
   const int tid = threadIdx.x;
   const int32_t part_tokens = part_blocks * kBlock;
   for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
-  // the group bounds
+  // the group bounds (kept in shared memory for the searches below if they fit)
+  const bool cached = num_groups < kPlanGroupCache;
   int bad = 0;
   for (int32_t i = tid; i <= num_groups; i += kPlanThreads) {
     const int32_t a = group_start[i];
     if (a < 0 || a > num_seqs || (i < num_groups && a > group_start[i + 1])) bad = 1;
+    if (cached) gs_cache[i] = a;
   }
   const bool groups_ok = __syncthreads_or(bad) == 0;
   if (!groups_ok && tid == 0) raise_error(PKV_DEVERR_GROUP);
   const int32_t G = groups_ok ? num_groups : 0;
+  const int32_t* gsp = cached ? gs_cache : group_start;
   // each group's prefix as given, within the table width; none (and no check)
   // for a group of fewer than two members
   for (int32_t i = tid; i < G; i += kPlanThreads) {
     int32_t p = 0;
-    if (group_start[i + 1] - group_start[i] >= 2) {
+    if (gsp[i + 1] - gsp[i] >= 2) {
       p = shared_blocks[i];
       const int32_t cap = max_len / kBlock;
       if (p < 0 || p > cap) {
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   __syncthreads();
   // ... and never past a member's own full blocks
   for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
-    const int32_t gi = group_of(group_start, G, s);
+    const int32_t gi = group_of(gsp, G, s);
     if (gi < 0) continue;
     const int32_t full = checked_len(context_lens[s], max_len) / kBlock;
     if (full < group_pref[gi]) {
@@ -262,7 +271,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   // sizes: each sequence's own partitions, each group's prefix partitions
   // (one item per members_per_item sequences)
   for (int32_t s = tid; s < num_seqs; s += kPlanThreads) {
-    const int32_t gi = group_of(group_start, G, s);
+    const int32_t gi = group_of(gsp, G, s);
     const int32_t pref = gi >= 0 ? group_pref[gi] : 0;
     seq_prefix[s] = pref;
     const int32_t tail = checked_len(context_lens[s], max_len) - pref * kBlock;
@@ -273,7 +282,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   for (int32_t i = tid; i < G; i += kPlanThreads) {
     const int32_t pref = group_pref[i];
     if (pref == 0) continue;
-    const int32_t members = group_start[i + 1] - group_start[i];
+    const int32_t members = gsp[i + 1] - gsp[i];
     const uint32_t per = static_cast<uint32_t>((members + members_per_item - 1) / members_per_item);
     const int32_t n = num_parts(pref * kBlock, part_tokens);
     for (int32_t p = 0; p < n; ++p)
@@ -296,7 +305,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   for (int32_t i = tid; i < G; i += kPlanThreads) {
     const int32_t pref = group_pref[i];
     if (pref == 0) continue;
-    const int32_t first = group_start[i], members = group_start[i + 1] - first;
+    const int32_t first = gsp[i], members = gsp[i + 1] - first;
     const int32_t per = (members + members_per_item - 1) / members_per_item;
     const int32_t n = num_parts(pref * kBlock, part_tokens);
     for (int32_t p = 0; p < n; ++p) {
@@ -1463,15 +1472,18 @@ __global__ void __launch_bounds__((W + 1) * 32, 1)
 }
 
 // ------------------------------------------------------------- merge kernel
-// One CTA of kMergeWarps warps per (query token, query head) row whose
-// sequence was split (or read a shared prefix separately): combine the partitions' (m, l, o) by log-sum-exp and
-// store the final output.  Every warp finds the common maximum M, takes every
-// kMergeWarps-th partition (so a row's partials stream in on several warps at
-// once), and warp 0 adds the warps' sums in a fixed order.  Partitions a causal
-// row cannot see carry l = 0 and no weight.
+// Combines the partial results (m, l, o) of a (query token, query head) row
+// whose sequence was split (or read a shared prefix separately) by
+// log-sum-exp and stores the final output.  WPR warps serve one row (CTAs of
+// kMergeWarps warps, so kMergeWarps / WPR rows per CTA): every warp finds the
+// common maximum M and takes every WPR-th partition, so a long row's partials
+// stream in on several warps at once; with WPR > 1 warp 0 adds the warps'
+// sums in a fixed order.  WPR = 1 suits rows with a few partials (one warp
+// per row, no shared-memory step).  Partitions a causal row cannot see carry
+// l = 0 and no weight.
 constexpr int kMergeWarps = 4;
 
-template <typename T, int D>
+template <typename T, int D, int WPR>
 __global__ void __launch_bounds__(kMergeWarps * 32)
     merge_kernel(void* __restrict__ out, const float* __restrict__ part_o,
                  const float* __restrict__ part_ml, const int32_t* __restrict__ context_lens,
@@ -1479,13 +1491,17 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
                  const int32_t* __restrict__ seq_prefix, int32_t num_seqs,
                  int32_t num_q_tokens, int32_t num_q_heads, int32_t max_parts, int32_t max_len,
                  int32_t part_tokens) {
+  static_assert(WPR == 1 || WPR == kMergeWarps, "one warp per row, or the whole CTA");
   constexpr int VEC = D / 32;  // floats per lane
+  constexpr int RPC = kMergeWarps / WPR;  // rows per CTA
   __shared__ __align__(16) float red[kMergeWarps][D];
   __shared__ float red_w[kMergeWarps];
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = blockIdx.x;
+  const int sub = warp % WPR;  // which of the row's partitions this warp takes
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * RPC + warp / WPR;
+  // (returns below are uniform over the warps that share a row)
   if (row >= static_cast<int64_t>(num_q_tokens) * num_q_heads) return;
   const int32_t t = static_cast<int32_t>(row / num_q_heads);  // query token
   int32_t s = t;                                                // its sequence
@@ -1504,7 +1520,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   const int32_t P = seq_prefix ? seq_prefix[s] : 0;
   const int32_t n = (P > 0 ? num_parts(P * kBlock, part_tokens) : 0) +
                     num_parts(L - P * kBlock, part_tokens);
-  if (n <= 1) return;  // the decode kernel wrote this row directly (uniform over the CTA)
+  if (n <= 1) return;  // the decode kernel wrote this row directly
   const float* ml = part_ml + row * max_parts * 2;
   float M = -INFINITY;
   for (int p = lane; p < n; p += 32) M = fmaxf(M, ml[2 * p]);
@@ -1517,7 +1533,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
   const float* po = part_o + row * max_parts * D + lane * VEC;
   if (M != -INFINITY) {
 #pragma unroll 4
-    for (int p = warp; p < n; p += kMergeWarps) {
+    for (int p = sub; p < n; p += WPR) {
       const float lp = ml[2 * p + 1];
       const float w = lp > 0.f ? lp * exp2f((ml[2 * p] - M) * kLog2e) : 0.f;
       wsum += w;
@@ -1534,20 +1550,23 @@ __global__ void __launch_bounds__(kMergeWarps * 32)
       }
     }
   }
+  float tot = wsum;
+  if constexpr (WPR > 1) {
 #pragma unroll
-  for (int i = 0; i < VEC; ++i) red[warp][lane * VEC + i] = acc[i];
-  if (lane == 0) red_w[warp] = wsum;
-  __syncthreads();
-  if (warp != 0) return;
-  float tot = 0.f;
+    for (int i = 0; i < VEC; ++i) red[warp][lane * VEC + i] = acc[i];
+    if (lane == 0) red_w[warp] = wsum;
+    __syncthreads();
+    if (warp != 0) return;
+    tot = 0.f;
 #pragma unroll
-  for (int w = 0; w < kMergeWarps; ++w) tot += red_w[w];
+    for (int w = 0; w < kMergeWarps; ++w) tot += red_w[w];
 #pragma unroll
-  for (int i = 0; i < VEC; ++i) {
-    float a = 0.f;
+    for (int i = 0; i < VEC; ++i) {
+      float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kMergeWarps; ++w) a += red[w][lane * VEC + i];
-    acc[i] = a;
+      for (int w = 0; w < kMergeWarps; ++w) a += red[w][lane * VEC + i];
+      acc[i] = a;
+    }
   }
   const float inv = tot > 0.f ? 1.f / tot : 0.f;
   if constexpr (sizeof(T) == 2) {
