@@ -84,6 +84,22 @@ int32_t pkv_bm_take_copies(pkv_block_manager *bm, int64_t *pairs_out, int32_t ma
 pkv_status pkv_bm_block_tables(pkv_block_manager *bm, const int64_t *seq_ids, int32_t n,
                                int32_t max_blocks, int32_t *tables_out, int32_t *lens_out);
 
+/* Groups for pkv_paged_attention_decode_shared over n sequences taken in the
+ * order of seq_ids (the rows of the tables pkv_bm_block_tables exports in the
+ * same order): maximal runs of consecutive sequences that hold the same
+ * physical blocks at the start of their tables -- what fork gives parallel
+ * samples of one prompt, or prefix caching gives requests with one system
+ * prompt.  A run starting at sequence i takes the next sequences while they
+ * keep at least min_shared_blocks (>= 1) leading blocks in common with
+ * sequence i, counting only blocks that are full in both.  For run r:
+ * group_start_out[r] .. group_start_out[r+1] - 1 are its positions in seq_ids
+ * and shared_blocks_out[r] the leading blocks all its members share (0 for a
+ * run of one).  group_start_out needs n + 1 entries, shared_blocks_out n;
+ * *num_groups_out receives the number of runs. */
+pkv_status pkv_bm_shared_prefix_groups(pkv_block_manager *bm, const int64_t *seq_ids, int32_t n,
+                                       int32_t min_shared_blocks, int32_t *group_start_out,
+                                       int32_t *shared_blocks_out, int32_t *num_groups_out);
+
 /* Counts: free blocks (never used or returned), cached blocks held by nobody
  * (evictable), blocks referenced by at least one sequence, live sequences. */
 pkv_status pkv_bm_stats(const pkv_block_manager *bm, int32_t *free_blocks,

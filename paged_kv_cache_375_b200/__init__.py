@@ -131,6 +131,7 @@ def load_library() -> ctypes.CDLL:
             "pkv_bm_block_tables": (ctypes.c_int, [P, P, i32, i32, P, P]),
             "pkv_bm_stats": (ctypes.c_int, [P, P, P, P, P]),
             "pkv_bm_refcount": (i32, [P, i32]),
+            "pkv_bm_shared_prefix_groups": (ctypes.c_int, [P, P, i32, i32, P, P, P]),
             "pkv_last_error_message": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -899,6 +900,20 @@ class BlockManager:
                                                 tables.ctypes.data_as(ctypes.c_void_p),
                                                 lens.ctypes.data_as(ctypes.c_void_p)))
         return tables, lens
+
+    def shared_prefix_groups(self, seq_ids, min_shared_blocks: int = 1):
+        """(group_start int32 [G+1], shared_blocks int32 [G]) for paged_attention_decode_shared
+        over these sequences in this order: runs of consecutive sequences whose tables begin
+        with the same physical blocks (at least min_shared_blocks full ones)."""
+        s, sp = self._arr(seq_ids, self._np.int64)
+        n = s.shape[0]
+        gs = self._np.empty(n + 1, dtype=self._np.int32)
+        sb = self._np.empty(max(n, 1), dtype=self._np.int32)
+        g = ctypes.c_int32()
+        _bm_check(self._lib.pkv_bm_shared_prefix_groups(
+            self._h, sp, n, int(min_shared_blocks), gs.ctypes.data_as(ctypes.c_void_p),
+            sb.ctypes.data_as(ctypes.c_void_p), ctypes.byref(g)))
+        return gs[:g.value + 1].copy(), sb[:g.value].copy()
 
     def stats(self) -> dict:
         v = [ctypes.c_int32() for _ in range(4)]

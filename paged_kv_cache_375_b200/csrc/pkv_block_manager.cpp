@@ -312,6 +312,46 @@ pkv_status pkv_bm_block_tables(pkv_block_manager* bm, const int64_t* seq_ids, in
   return PKV_OK;
 }
 
+pkv_status pkv_bm_shared_prefix_groups(pkv_block_manager* bm, const int64_t* seq_ids, int32_t n,
+                                       int32_t min_shared_blocks, int32_t* group_start_out,
+                                       int32_t* shared_blocks_out, int32_t* num_groups_out) {
+  if (!bm || !group_start_out || !num_groups_out || ((!seq_ids || !shared_blocks_out) && n > 0))
+    return PKV_ERR_NULL;
+  if (n < 0 || min_shared_blocks < 1) return PKV_ERR_SHAPE;
+  std::vector<const Sequence*> seqs(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end()) return PKV_ERR_NOT_FOUND;
+    seqs[i] = &it->second;
+  }
+  // leading physical blocks two sequences hold in common, among the full
+  // blocks of both
+  auto common = [&](const Sequence& a, const Sequence& b) {
+    const size_t full = std::min(a.tokens.size(), b.tokens.size()) / static_cast<size_t>(bm->bs);
+    size_t c = 0;
+    while (c < full && c < a.table.size() && c < b.table.size() && a.table[c] == b.table[c]) ++c;
+    return static_cast<int32_t>(c);
+  };
+  int32_t g = 0;
+  group_start_out[0] = 0;
+  for (int32_t i = 0; i < n;) {
+    // a run starts at i and takes the following sequences while they keep at
+    // least min_shared_blocks leading blocks in common with its first member
+    int32_t shared = 0, j = i + 1;
+    for (; j < n; ++j) {
+      const int32_t c = common(*seqs[i], *seqs[j]);
+      const int32_t p = j == i + 1 ? c : std::min(shared, c);
+      if (p < min_shared_blocks) break;
+      shared = p;
+    }
+    shared_blocks_out[g] = j - i >= 2 ? shared : 0;
+    group_start_out[++g] = j;
+    i = j;
+  }
+  *num_groups_out = g;
+  return PKV_OK;
+}
+
 pkv_status pkv_bm_stats(const pkv_block_manager* bm, int32_t* free_blocks,
                         int32_t* evictable_blocks, int32_t* used_blocks, int32_t* sequences) {
   if (!bm) return PKV_ERR_NULL;

@@ -190,3 +190,86 @@ def test_exhaustion_is_reported_and_changes_nothing():
     assert e.value.status == 11
     with pytest.raises(pkv.PkvError):
         bm.add_sequence(0, [1])                  # id already in use
+
+
+def _lcp_full(tables, lens, a, b):
+    full = min(lens[a], lens[b]) // BS
+    c = 0
+    while c < full and tables[a, c] == tables[b, c]:
+        c += 1
+    return c
+
+
+def check_groups(bm, ids, min_shared):
+    """Runs of consecutive sequences with common leading blocks, checked by brute force:
+    they tile the list in order, every member holds the run's first P table entries, P is
+    the exact minimum over members of the blocks common with the first member (full ones
+    only), and no run could take its next sequence."""
+    gs, sb = bm.shared_prefix_groups(ids, min_shared)
+    tables, lens = bm.block_tables(ids, max_blocks=256)
+    n = len(ids)
+    assert gs[0] == 0 and gs[-1] == n and (np.diff(gs) >= 1).all() and len(sb) == len(gs) - 1
+    for r in range(len(sb)):
+        a, e = int(gs[r]), int(gs[r + 1])
+        if e - a == 1:
+            assert sb[r] == 0
+        else:
+            p = min(_lcp_full(tables, lens, a, m) for m in range(a + 1, e))
+            assert sb[r] == p >= min_shared
+            for m in range(a, e):
+                assert (tables[m, :p] == tables[a, :p]).all() and p <= lens[m] // BS
+        if e < n:
+            ext = _lcp_full(tables, lens, a, e)
+            if e - a >= 2:
+                ext = min(ext, int(sb[r]))
+            assert ext < min_shared
+    return gs, sb
+
+
+def test_shared_prefix_groups_of_forks_and_cached_prompts():
+    bm = pkv.BlockManager(400, BS, seed=9, prefix_caching=True)
+    bm.add_sequence(0, list(range(40)))            # 2 full blocks + a partial one
+    for c in (1, 2, 3):
+        bm.fork(0, c)
+    bm.add_sequence(10, list(range(1000, 1100)))   # 6 full blocks + a partial one
+    bm.fork(10, 11)
+    bm.add_sequence(20, list(range(5000, 5010)))   # shares nothing
+    prompt = list(range(7000, 7048))               # 3 full blocks, cached on first use
+    bm.add_sequence(30, prompt + [1])
+    bm.add_sequence(31, prompt + [2, 3])           # prefix caching shares the 3 full blocks
+    ids = [0, 1, 2, 3, 10, 11, 20, 30, 31]
+    bm.append_tokens(ids, [5] * len(ids))          # copies the shared partial blocks
+    bm.take_copies()
+    gs, sb = check_groups(bm, ids, 1)
+    assert gs.tolist() == [0, 4, 6, 7, 9] and sb.tolist() == [2, 6, 0, 3]
+    gs, sb = check_groups(bm, ids, 3)
+    assert gs.tolist() == [0, 1, 2, 3, 4, 6, 7, 9] and sb.tolist() == [0, 0, 0, 0, 6, 0, 3]
+    # another order splits the runs
+    check_groups(bm, [0, 10, 1, 11, 2, 3], 1)
+    with pytest.raises(pkv.PkvError):
+        bm.shared_prefix_groups([0, 99], 1)
+    with pytest.raises(pkv.PkvError):
+        bm.shared_prefix_groups([0, 1], 0)
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3, 4])
+def test_shared_prefix_groups_random_forest(seed):
+    rng = np.random.default_rng(seed)
+    bm = pkv.BlockManager(3000, BS, seed=seed)
+    ids = []
+    for p in range(12):
+        root = 100 * p
+        bm.add_sequence(root, rng.integers(0, 1000, size=int(rng.integers(1, 120))).tolist())
+        fam = [root]
+        for c in range(int(rng.integers(0, 6))):
+            parent = int(rng.choice(fam))
+            bm.fork(parent, root + c + 1)
+            fam.append(root + c + 1)
+            steps = int(rng.integers(0, 40))
+            for _ in range(steps):
+                bm.append_tokens([root + c + 1], [int(rng.integers(0, 1000))])
+        ids += fam
+    bm.take_copies()
+    for m in (1, 2, 4):
+        check_groups(bm, ids, m)
+        check_groups(bm, list(rng.permutation(ids)), m)

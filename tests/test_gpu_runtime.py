@@ -116,3 +116,51 @@ def test_decode_step_captured_in_a_cuda_graph_matches_eager(cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
     assert pkv.device_error_bits() == 0
+
+
+def test_shared_prefix_step_in_a_cuda_graph(cuda_device):
+    """The shared-prefix step (copy-on-write, new tokens, shared plan, decode, merge)
+    captured once and replayed gives bit-identical results to eager launches."""
+    b = workloads.c4_shared_prefix(device=cuda_device, prompts=3, samples=5, prefix=300,
+                                   max_tail=60, num_blocks=500)
+    dev = cuda_device
+    bt = dev_i32(b.block_tables, dev)
+    cl = dev_i32(b.context_lens, dev)
+    gs = dev_i32(np.asarray(b.meta["group_start"]), dev)
+    sb = dev_i32(np.asarray(b.meta["shared_blocks"]), dev)
+    mcl = b.max_context_len
+    ws = torch.empty(pkv.decode_shared_workspace_bytes(
+        pkv.make_dims(b.num_seqs, b.num_q_heads, b.k_cache, b.max_blocks_per_seq), mcl),
+        dtype=torch.uint8, device=dev)
+    pairs = torch.from_numpy(b.cow_pairs).to(dev)
+    seq, pos = dev_i32(b.new_seq, dev), dev_i32(b.new_pos, dev)
+    slots = torch.empty(b.new_seq.shape[0], dtype=torch.int64, device=dev)
+    out = torch.empty_like(b.q)
+
+    def step():
+        pkv.copy_blocks(b.k_cache, b.v_cache, pairs, validate=False)
+        pkv.slot_mapping(bt, b.num_blocks, token_seq=seq, token_pos=pos, out=slots)
+        pkv.reshape_and_cache(b.new_k, b.new_v, b.k_cache, b.v_cache, slots)
+        plan = pkv.SharedDecodePlan(bt, cl, gs, sb, b.num_q_heads, b.k_cache,
+                                    max_context_len=mcl, workspace_tensor=ws)
+        plan.run(out, b.q, b.k_cache, b.v_cache, b.scale)
+
+    step()
+    torch.cuda.synchronize()
+    eager = out.clone()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        step()
+        torch.cuda.synchronize()
+        out.zero_()
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    assert pkv.device_error_bits() == 0

@@ -254,3 +254,55 @@ def test_shared_prefix_workload_full_size_sampled(cuda_device):
     got = out[torch.from_numpy(tasks[:, 0]).long(), torch.from_numpy(tasks[:, 1]).long()]
     check_close(got, ref, "bf16", "c4 full size, shared prefix")
     assert torch.isfinite(out).all()
+
+
+def test_block_manager_groups_drive_the_shared_decode(cuda_device):
+    """Forks and prefix caching in the host block manager, its tables, slots and groups,
+    then the KV written through reshape_and_cache (copies first) and the shared decode,
+    against the oracle over the manager's own tables."""
+    dev = cuda_device
+    hq, hkv, d, nb = 32, 8, 128, 600
+    rng = np.random.default_rng(77)
+    bm = pkv.BlockManager(nb, 16, seed=3, prefix_caching=True)
+    ids, prompts = [], {}
+    for p, (plen, samples) in enumerate([(70, 4), (200, 8), (33, 1), (160, 3)]):
+        root = 100 * p
+        prompts[root] = plen
+        bm.add_sequence(root, rng.integers(0, 30000, size=plen).tolist())
+        ids.append(root)
+        for c in range(1, samples):
+            bm.fork(root, root + c)
+            ids.append(root + c)
+    # every sequence decodes a few tokens of its own (copy-on-write of shared partial blocks)
+    for _ in range(5):
+        bm.append_tokens(ids, rng.integers(0, 30000, size=len(ids)).astype(np.int32))
+    pairs = bm.take_copies()
+    tables, lens = bm.block_tables(ids, max_blocks=32)
+    gs, sb = bm.shared_prefix_groups(ids, 1)
+    assert (sb > 0).sum() == 3
+    # K/V for every written position, through the manager's slots
+    gen = torch.Generator(device=dev).manual_seed(5)
+    k_cache = torch.full((nb, hkv, 16, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    v_cache = torch.full_like(k_cache, float("nan"))
+    slots = np.concatenate([bm.slots(s, 0, int(L)) for s, L in zip(ids, lens)])
+    # positions shared by several sequences have one slot: write each slot once
+    slots = np.unique(slots)
+    T = slots.shape[0]
+    k = torch.randn((T, hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    v = torch.randn((T, hkv, d), generator=gen, device=dev).to(torch.bfloat16)
+    if pairs.shape[0]:
+        pkv.copy_blocks(k_cache, v_cache, torch.from_numpy(pairs))
+    pkv.reshape_and_cache(k, v, k_cache, v_cache, torch.from_numpy(slots).to(dev))
+    q = torch.randn((len(ids), hq, d), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    scale = float(np.float32(1.0 / np.sqrt(d)))
+    pkv.paged_attention_decode_shared(out, q, k_cache, v_cache, dev_i32(tables, dev),
+                                      dev_i32(lens, dev), dev_i32(gs, dev), dev_i32(sb, dev),
+                                      scale, max_context_len=int(lens.max()))
+    assert pkv.device_error_bits() == 0
+
+    def bits(t):
+        return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+    ref = oracle.paged_decode(bits(q), bits(k_cache), bits(v_cache), tables, lens, scale)
+    check_close(out, ref, "bf16", "block manager groups")
