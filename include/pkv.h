@@ -14,10 +14,12 @@
  *    write ("vLLM 深读：用 PagedAttention 撑起高并发 LLM 推理", section
  *    "先看浪费在哪里").
  * Beyond one query token per sequence the same decode kernel serves chunks of
- * several causal query tokens (pkv_paged_attention_multi), and pools of FP8
- * (e4m3) codes with per-pool scales (the *_fp8 calls).  The host block
- * manager that produces tables, slots and copy pairs is declared in
- * pkv_block_manager.h.
+ * several causal query tokens (pkv_paged_attention_multi), batches whose
+ * consecutive sequences share their leading blocks, each such block read once
+ * for the group (pkv_paged_attention_decode_shared), and pools of FP8 (e4m3
+ * or e5m2) codes with per-pool scales (the *_fp8 calls).  The host block
+ * manager that produces tables, slots, copy pairs and shared-prefix groups is
+ * declared in pkv_block_manager.h.
  *
  * Conventions for every call:
  *  - Pointers are DEVICE pointers unless the argument says "host".  The caller
