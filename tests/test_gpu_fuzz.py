@@ -92,3 +92,54 @@ def test_random_configuration(cuda_device, seed):
                oracle.paged_multi(host["q"], k, v, b.block_tables, b.context_lens,
                                   b.query_start_loc, b.scale))
     check_close(out, ref, "bf16" if fmt else dtype, what)
+
+
+@pytest.mark.parametrize("seed", range(32))
+def test_random_shared_prefix_configuration(cuda_device, seed):
+    """The shared-prefix decode on random groups: sizes, prefix blocks (sometimes past a
+    member's full blocks, then lowered and flagged), tails, tables that share or not, all
+    pool dtypes, partitions; the oracle reads the tables as the call defines them."""
+    from test_gpu_shared_prefix import substituted_tables
+    rng = np.random.default_rng(30_000 + seed)
+    dtype = ["f32", "bf16", "fp8", "fp8e5m2"][seed % 4]
+    d = 128 if workloads.fp8_format(dtype) else int(rng.choice([64, 128]))
+    hkv = int(rng.choice([1, 2, 4, 8]))
+    g = int(rng.choice([1, 2, 3, 4, 8, 16]))
+    sizes = rng.integers(1, 13, size=int(rng.integers(1, 6)))
+    pref = rng.integers(0, 21, size=sizes.shape[0])
+    lens = []
+    for n, p in zip(sizes, pref):
+        lens += (16 * p + rng.integers(0, 300, size=n)).tolist()
+    claimed = pref + (rng.random(pref.shape[0]) < 0.2) * rng.integers(1, 4, size=pref.shape[0])
+    partition = int(rng.choice([0, 16, 48, 256]))
+    share = bool(rng.random() < 0.7)
+    b = workloads.random_batch(40_000 + seed, lens, g * hkv, hkv, d, dtype, device="cpu",
+                               extra_table=1)
+    gs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    sb = claimed.astype(np.int32)
+    if share:
+        b.block_tables = substituted_tables(b.block_tables, gs, sb, b.context_lens)
+    b = b.to(cuda_device)
+    host = b.host()
+    dev = cuda_device
+    out = torch.empty_like(b.q)
+    fmt = workloads.fp8_format(dtype)
+    kw = dict(k_scale=b.k_scale, v_scale=b.v_scale) if fmt else {}
+    pkv.paged_attention_decode_shared(out, b.q, b.k_cache, b.v_cache, dev_i32(b.block_tables, dev),
+                                      dev_i32(b.context_lens, dev), dev_i32(gs, dev),
+                                      dev_i32(sb, dev), b.scale,
+                                      max_context_len=max(b.max_context_len, 1),
+                                      partition_tokens=partition, **kw)
+    bits = pkv.device_error_bits()
+    lowered = any(sizes[i] >= 2 and min(lens[gs[i]:gs[i + 1]]) // 16 < sb[i]
+                  for i in range(len(sizes)))
+    what = f"seed {seed}: {dtype} d{d} {g * hkv}/{hkv} sizes {sizes.tolist()} P {sb.tolist()}"
+    assert bits == (pkv.DEVERR_GROUP if lowered else 0), what
+    tables = substituted_tables(b.block_tables, gs, sb, b.context_lens)
+    if fmt:
+        ref = oracle.paged_decode_fp8(host["q"], host["k_cache"], host["v_cache"], b.k_scale,
+                                      b.v_scale, tables, b.context_lens, b.scale, fmt=fmt)
+    else:
+        ref = oracle.paged_decode(host["q"], host["k_cache"], host["v_cache"], tables,
+                                  b.context_lens, b.scale)
+    check_close(out, ref, "f32" if dtype == "f32" else "bf16", what)
