@@ -186,10 +186,15 @@ def whole_job_value(units_per_rank: float, world: int, seconds: float) -> float:
 
 
 # ------------------------------------------------------------------ our arm
+# New tokens per step up to which the writes share a launch with the plan.
+TOKEN_PROLOGUE_MAX = 4096
+
+
 class Step:
     """The hot path over one batch through the public API (device-resident inputs)."""
 
-    def __init__(self, b: workloads.Batch, partition_tokens: int, shared_prefix: bool = True):
+    def __init__(self, b: workloads.Batch, partition_tokens: int, shared_prefix: bool = True,
+                 token_prologue: bool = False):
         import paged_kv_cache_375_b200 as pkv
         self.pkv, self.b = pkv, b
         dev = b.q.device
@@ -230,14 +235,17 @@ class Step:
         # one new token per sequence at its last position, no copies: the fused prologue
         self.fused = (self.decode_mode and self.pairs is None and not self.multi
                       and not self.shared)
+        # any other short list of new tokens (a few per sequence): written in the same
+        # launch as the plan.  A long list (the parallel-sampling tails) keeps
+        # reshape_and_cache, whose many small CTAs stream the rows at the copy bandwidth.
+        self.fused_tokens = (self.T > 0 and not self.fused
+                             and (token_prologue or self.T <= TOKEN_PROLOGUE_MAX))
         if self.pairs is not None:
             pkv.validate_copy_pairs(torch.from_numpy(b.cow_pairs), b.num_blocks)
 
     def launches_per_step(self) -> int:
-        if self.fused:                                 # prologue, decode (, merge)
-            return 2 + (1 if self.split else 0)
-        n = 2 + (1 if self.split else 0)              # plan, decode (, merge)
-        n += 2 if self.T else 0                        # slot indexing, reshape_and_cache
+        n = 2 + (1 if self.split else 0)              # plan or prologue, decode (, merge)
+        n += 2 if self.T and not (self.fused or self.fused_tokens) else 0  # slots, reshape
         n += 1 if self.pairs is not None else 0        # copy_blocks
         return n
 
@@ -247,7 +255,7 @@ class Step:
             return                                     # done by the prologue in plan()
         if self.pairs is not None:
             pkv.copy_blocks(b.k_cache, b.v_cache, self.pairs, validate=False)
-        if self.T:
+        if self.T and not self.fused_tokens:
             if self.decode_mode:
                 pkv.slot_mapping(self.bt, b.num_blocks, context_lens=self.cl, out=self.slots)
             else:
@@ -265,16 +273,19 @@ class Step:
 
     def plan(self):
         b = self.b
+        extra = {}
+        if self.fused or self.fused_tokens:
+            # one launch: the new tokens' slots and writes, and the plan
+            extra = dict(new_k=b.new_k, new_v=b.new_v, v_cache=b.v_cache, k_scale=b.k_scale,
+                         v_scale=b.v_scale, slot_mapping_out=self.slots[:self.T])
+            if self.fused_tokens:
+                extra.update(token_seq=self.seq, token_pos=self.pos)
         if self.shared:
             self.plan_obj = self.pkv.SharedDecodePlan(
                 self.bt, self.cl, self.group_start, self.shared_blocks, b.num_q_heads, b.k_cache,
                 max_context_len=self.mcl, partition_tokens=self.partition,
-                workspace_tensor=self.ws)
+                workspace_tensor=self.ws, **extra)
             return
-        extra = {}
-        if self.fused:   # one launch: the new tokens' slots and writes, and the plan
-            extra = dict(new_k=b.new_k, new_v=b.new_v, v_cache=b.v_cache, k_scale=b.k_scale,
-                         v_scale=b.v_scale, slot_mapping_out=self.slots[:self.T])
         self.plan_obj = self.pkv.DecodePlan(self.bt, self.cl, b.num_q_heads, b.k_cache,
                                             max_context_len=self.mcl,
                                             partition_tokens=self.partition,
@@ -310,7 +321,8 @@ def run_ours(args, world, rank, local):
     name = WORKLOADS[args.workload]
     b = (workloads.BUILDERS[name](device=dev, num_seqs=args.batch) if args.batch else
          workloads.BUILDERS[name](device=dev))
-    step = Step(b, args.partition, shared_prefix=not args.no_shared_prefix)
+    step = Step(b, args.partition, shared_prefix=not args.no_shared_prefix,
+                token_prologue=args.token_prologue)
     alg = algorithmic_bytes(b)
     kv_bytes = b.kv_bytes() if name != "c4_shared_prefix" else b.unique_kv_bytes()
     stream = torch.cuda.current_stream(dev)
@@ -480,13 +492,15 @@ def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
 
     def plan_only():
         if step.shared:
-            step.plan()
+            pkv.SharedDecodePlan(step.bt, step.cl, step.group_start, step.shared_blocks,
+                                 b.num_q_heads, b.k_cache, max_context_len=step.mcl,
+                                 partition_tokens=step.partition, workspace_tensor=step.ws)
             return
         pkv.DecodePlan(step.bt, step.cl, b.num_q_heads, b.k_cache, max_context_len=step.mcl,
                        partition_tokens=step.partition, workspace_tensor=step.ws)
 
     ops = {"plan": plan_only}
-    if step.fused:
+    if step.fused or step.fused_tokens:
         ops["decode_prologue"] = step.plan
     if step.T:
         if step.decode_mode:
@@ -555,6 +569,8 @@ def run_e2e(step: Step, args, world, dev, kv_bytes):
     ins = [("q", b.q), ("new_k", b.new_k), ("new_v", b.new_v), ("cl", step.cl), ("bt", step.bt)]
     if step.shared:
         ins += [("gs", step.group_start), ("sb", step.shared_blocks)]
+    if step.fused_tokens:
+        ins += [("seq", step.seq), ("pos", step.pos)]
     host = {name: t.detach().cpu().pin_memory() for name, t in ins}
     dst = dict(ins)
     out_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
@@ -751,6 +767,9 @@ def main(argv=None):
     ap.add_argument("--no-shared-prefix", action="store_true",
                     help="decode a batch with shared prompt blocks with the plain plan (every "
                          "sequence reads its whole table)")
+    ap.add_argument("--token-prologue", action="store_true",
+                    help="write any number of new tokens in the plan's launch (by default only "
+                         f"up to {TOKEN_PROLOGUE_MAX} a step)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--batch", type=int, default=0,
                     help="number of sequences (0 = the workload's own); a smaller batch of the "

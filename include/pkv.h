@@ -303,6 +303,36 @@ pkv_status pkv_decode_prepare_fp8(const void *k, const void *v, void *k_cache, v
                                   size_t workspace_bytes, void *cuda_stream);
 
 /*
+ * The prologue for any list of new tokens in one launch: the tails of parallel
+ * samples, a chunk of several query tokens per sequence.  Token t (k[t], v[t],
+ * [num_tokens][Hkv][D]) of sequence token_seq[t] at position token_pos[t]
+ * (int32 [num_tokens] each, device) is written into its slot
+ * block_tables[seq][pos/16] * 16 + pos % 16 exactly as pkv_slot_mapping (token
+ * mode) followed by pkv_reshape_and_cache (or pkv_reshape_and_cache_fp8 for
+ * FP8 pools, with k_scale and v_scale; they are ignored otherwise) does, with
+ * the same device-side checks (PKV_DEVERR_POS, PKV_DEVERR_BLOCK; a flagged
+ * token is skipped); slot_mapping_out (int64 [num_tokens], may be NULL)
+ * receives the slots, -1 for flagged tokens.  In the same launch one CTA
+ * builds the decode plan from context_lens: with group_start == NULL the plan
+ * of pkv_decode_plan (follow with pkv_decode_run, pkv_multi_run or their
+ * _fp8 forms; workspace sized for that run), else the shared-prefix plan of
+ * pkv_decode_plan_shared over (group_start, shared_blocks, num_groups)
+ * (follow with pkv_decode_run_shared or its _fp8 form; workspace
+ * pkv_decode_shared_workspace_bytes).  Copy-on-write copies (pkv_copy_blocks)
+ * issued before it on the stream complete before any token is written.
+ * Two tokens with the same slot leave it unspecified.
+ */
+pkv_status pkv_decode_prepare_tokens(const void *k, const void *v, void *k_cache, void *v_cache,
+                                     const int32_t *block_tables, const int32_t *context_lens,
+                                     const int32_t *token_seq, const int32_t *token_pos,
+                                     int32_t num_tokens, int64_t *slot_mapping_out,
+                                     float k_scale, float v_scale, const int32_t *group_start,
+                                     const int32_t *shared_blocks, int32_t num_groups,
+                                     const pkv_dims *dims, int32_t max_context_len,
+                                     int32_t partition_tokens, void *workspace,
+                                     size_t workspace_bytes, void *cuda_stream);
+
+/*
  * FP8 KV cache.  The pages list FP8 among the quantisation formats and note
  * that memory saved holds more KV blocks ("vLLM 深读", section "引擎的分层结构";
  * "vllm" by vampireachao, "第三层：图、核、量化"); here the cache itself is FP8:

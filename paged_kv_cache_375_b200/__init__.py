@@ -102,6 +102,8 @@ def load_library() -> ctypes.CDLL:
                                                              f32, f32, D, i32, i32, P, sz, P]),
             "pkv_multi_run_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, f32, f32, D,
                                                  i32, i32, P, sz, P]),
+            "pkv_decode_prepare_tokens": (ctypes.c_int, [P, P, P, P, P, P, P, P, i32, P, f32, f32,
+                                                         P, P, i32, D, i32, i32, P, sz, P]),
             "pkv_decode_shared_workspace_bytes": (sz, [D, i32, i32]),
             "pkv_decode_shared_workspace_layout": (ctypes.c_int, [D, i32, i32, P, P, P, P]),
             "pkv_paged_attention_decode_shared": (ctypes.c_int, [P, P, P, P, P, P, P, P, i32,
@@ -386,6 +388,39 @@ def paged_attention_multi_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch
     return out
 
 
+def _prepare_tokens(lib, dims, k_cache, v_cache, block_tables, context_lens, new_k, new_v,
+                    token_seq, token_pos, k_scale, v_scale, slot_mapping_out, group_start,
+                    shared_blocks, num_groups, max_context_len, partition_tokens, ws, dev):
+    """The token-list prologue (pkv_decode_prepare_tokens): writes and plan in one launch."""
+    fp8 = k_cache.dtype in FP8_DTYPES
+    src = torch.bfloat16 if fp8 else k_cache.dtype
+    _need(new_k, "new_k", src, dev)
+    _need(new_v, "new_v", src, dev)
+    _need(token_seq, "token_seq", torch.int32, dev)
+    _need(token_pos, "token_pos", torch.int32, dev)
+    _need(k_cache, "k_cache", device=dev)
+    if v_cache is None:
+        raise ValueError("v_cache is needed to write the new tokens")
+    _need(v_cache, "v_cache", k_cache.dtype, dev)
+    T = token_seq.shape[0]
+    if new_k.shape != (T, k_cache.shape[1], k_cache.shape[3]) or new_v.shape != new_k.shape \
+            or token_pos.shape != (T,) or v_cache.shape != k_cache.shape:
+        raise ValueError("new_k, new_v must be [num_tokens][num_kv_heads][head_dim], "
+                         "token_seq and token_pos int32 [num_tokens]")
+    if slot_mapping_out is not None:
+        _need(slot_mapping_out, "slot_mapping_out", torch.int64, dev)
+        if slot_mapping_out.shape != (T,):
+            raise ValueError("slot_mapping_out must be int64 [num_tokens]")
+    if fp8 and (k_scale is None or v_scale is None):
+        raise ValueError("FP8 pools need k_scale and v_scale")
+    _check(lib.pkv_decode_prepare_tokens(
+        _p(new_k), _p(new_v), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+        _p(token_seq), _p(token_pos), T, _p(slot_mapping_out),
+        float(k_scale) if fp8 else 1.0, float(v_scale) if fp8 else 1.0, _p(group_start),
+        _p(shared_blocks), num_groups, ctypes.byref(dims), max_context_len, partition_tokens,
+        _p(ws), ws.numel(), _stream_ptr(dev)))
+
+
 class DecodePlan:
     """A decode plan for one step: the work list built from context_lens, kept in a
     workspace.  ``run`` decodes one layer's cache pools with it; plan once per step, run
@@ -395,14 +430,17 @@ class DecodePlan:
     launch also writes every sequence's new token (position L - 1) into its slot of
     ``k_cache``/``v_cache`` (quantised with ``k_scale``/``v_scale`` for FP8 pools) and,
     if given, each slot into ``slot_mapping_out`` (int64 [B]): slot indexing,
-    reshape_and_cache and the plan in one launch."""
+    reshape_and_cache and the plan in one launch.  With ``token_seq``/``token_pos`` (int32
+    [T]) the new tokens are any list instead ([T][Hkv][D]; ``slot_mapping_out`` int64 [T]),
+    e.g. the chunks of several query tokens per sequence."""
 
     def __init__(self, block_tables: torch.Tensor, context_lens: torch.Tensor, num_q_heads: int,
                  k_cache: torch.Tensor, *, max_context_len: int | None = None,
                  partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None,
                  new_k: torch.Tensor | None = None, new_v: torch.Tensor | None = None,
                  v_cache: torch.Tensor | None = None, k_scale: float | None = None,
-                 v_scale: float | None = None, slot_mapping_out: torch.Tensor | None = None):
+                 v_scale: float | None = None, slot_mapping_out: torch.Tensor | None = None,
+                 token_seq: torch.Tensor | None = None, token_pos: torch.Tensor | None = None):
         dev = context_lens.device
         _need(block_tables, "block_tables", torch.int32, dev)
         _need(context_lens, "context_lens", torch.int32, dev)
@@ -425,6 +463,11 @@ class DecodePlan:
                                        self.max_context_len, partition_tokens,
                                        _p(self.workspace), self.workspace.numel(),
                                        _stream_ptr(dev)))
+            return
+        if token_seq is not None:
+            _prepare_tokens(lib, self.dims, k_cache, v_cache, block_tables, context_lens, new_k,
+                            new_v, token_seq, token_pos, k_scale, v_scale, slot_mapping_out, None,
+                            None, 0, self.max_context_len, partition_tokens, self.workspace, dev)
             return
         fp8 = k_cache.dtype in FP8_DTYPES
         src = torch.bfloat16 if fp8 else k_cache.dtype
@@ -569,12 +612,19 @@ class SharedDecodePlan:
     every member reads its first ``shared_blocks[i]`` blocks (int32 [G], device) through the
     first member's table row, so the shared blocks are read once per kv head for the whole
     group.  With tables that really share those blocks the result is exactly
-    paged_attention_decode's.  Plan once per step, ``run`` (``run_fp8``) once per layer."""
+    paged_attention_decode's.  Plan once per step, ``run`` (``run_fp8``) once per layer.
+    With ``new_k``/``new_v`` ([T][Hkv][D]), ``v_cache`` and ``token_seq``/``token_pos``
+    (int32 [T]) the same launch also writes those tokens into their slots (quantised with
+    ``k_scale``/``v_scale`` for FP8 pools), as slot indexing + reshape_and_cache would."""
 
     def __init__(self, block_tables: torch.Tensor, context_lens: torch.Tensor,
                  group_start: torch.Tensor, shared_blocks: torch.Tensor, num_q_heads: int,
                  k_cache: torch.Tensor, *, max_context_len: int | None = None,
-                 partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None):
+                 partition_tokens: int = 0, workspace_tensor: torch.Tensor | None = None,
+                 new_k: torch.Tensor | None = None, new_v: torch.Tensor | None = None,
+                 v_cache: torch.Tensor | None = None, token_seq: torch.Tensor | None = None,
+                 token_pos: torch.Tensor | None = None, k_scale: float | None = None,
+                 v_scale: float | None = None, slot_mapping_out: torch.Tensor | None = None):
         dev = context_lens.device
         _need(block_tables, "block_tables", torch.int32, dev)
         _need(context_lens, "context_lens", torch.int32, dev)
@@ -594,6 +644,12 @@ class SharedDecodePlan:
         if workspace_tensor.numel() < need:
             raise ValueError(f"workspace_tensor has {workspace_tensor.numel()} bytes, {need} needed")
         self.workspace = workspace_tensor
+        if new_k is not None:
+            _prepare_tokens(load_library(), self.dims, k_cache, v_cache, block_tables,
+                            context_lens, new_k, new_v, token_seq, token_pos, k_scale, v_scale,
+                            slot_mapping_out, group_start, shared_blocks, G,
+                            self.max_context_len, partition_tokens, self.workspace, dev)
+            return
         _check(load_library().pkv_decode_plan_shared(
             _p(context_lens), _p(group_start), _p(shared_blocks), G, ctypes.byref(self.dims),
             self.max_context_len, partition_tokens, _p(self.workspace), self.workspace.numel(),

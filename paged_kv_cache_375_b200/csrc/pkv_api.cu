@@ -613,6 +613,94 @@ pkv_status multi_one_shot(void* out, const void* q, const void* k_cache, const v
 
 namespace {
 
+// The token-list prologue (see pkv_decode_prepare_tokens).
+pkv_status prepare_tokens(const void* k, const void* v, void* k_cache, void* v_cache,
+                          const int32_t* block_tables, const int32_t* context_lens,
+                          const int32_t* token_seq, const int32_t* token_pos, int32_t num_tokens,
+                          int64_t* slot_mapping_out, float k_scale, float v_scale,
+                          const int32_t* group_start, const int32_t* shared_blocks,
+                          int32_t num_groups, const pkv_dims* dims, int32_t max_context_len,
+                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                          void* cuda_stream) {
+  const bool shared = group_start != nullptr;
+  DecodePlan plan;
+  pkv_status st = make_plan(dims, max_context_len, partition_tokens, &plan, -1, shared);
+  if (st != PKV_OK) return st;
+  const bool fp8 = is_fp8(dims->dtype);
+  if (fp8 && (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) ||
+              !std::isfinite(v_scale)))
+    return fail(PKV_ERR_SHAPE, "k_scale and v_scale must be finite and positive for FP8 pools");
+  if (num_tokens < 0) return fail(PKV_ERR_SHAPE, "num_tokens must be >= 0");
+  if (shared && (num_groups < 0 || num_groups > dims->num_seqs))
+    return fail(PKV_ERR_SHAPE, "num_groups must be in [0, num_seqs]");
+  if (dims->num_seqs == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (num_tokens > 0 && (!k || !v || !token_seq || !token_pos))
+    return fail(PKV_ERR_NULL, "k, v, token_seq or token_pos is NULL");
+  if (shared && num_groups > 0 && !shared_blocks) return fail(PKV_ERR_NULL, "shared_blocks is NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "k, v and the caches must be 16-byte aligned");
+  if ((st = check_workspace(plan, workspace, workspace_bytes)) != PKV_OK) return st;
+  if ((st = bind_device(k_cache, "k_cache")) != PKV_OK) return st;
+  // 16-byte units of one head's source row: bf16 / fp32 rows as stored, FP8
+  // rows as their bf16 inputs
+  const int units_per_head = dims->head_dim * (fp8 ? 2 : elem_bytes(dims->dtype)) / 16;
+  const int units = dims->num_kv_heads * units_per_head;
+  const int per = units < pkv::kPlanThreads ? units : pkv::kPlanThreads;
+  const int toks_per_cta = pkv::kPlanThreads / per;
+  const unsigned grid =
+      1u + static_cast<unsigned>((static_cast<int64_t>(num_tokens) + toks_per_cta - 1) / toks_per_cta);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::TokenPrepare a{};
+  a.k = static_cast<const uint4*>(k);
+  a.v = static_cast<const uint4*>(v);
+  a.k_cache = static_cast<uint8_t*>(k_cache);
+  a.v_cache = static_cast<uint8_t*>(v_cache);
+  a.block_tables = block_tables;
+  a.token_seq = token_seq;
+  a.token_pos = token_pos;
+  a.slots_out = slot_mapping_out;
+  a.num_tokens = num_tokens;
+  a.num_seqs = dims->num_seqs;
+  a.num_kv_heads = dims->num_kv_heads;
+  a.units_per_head = units_per_head;
+  a.max_blocks_per_seq = dims->max_blocks_per_seq;
+  a.num_blocks = dims->num_blocks;
+  a.toks_per_cta = toks_per_cta;
+  a.per = per;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.context_lens = context_lens;
+  a.max_len = plan.max_len;
+  a.part_blocks = plan.part_blocks;
+  a.items = reinterpret_cast<pkv::PlanItem*>(ws + plan.items_off);
+  a.counters = reinterpret_cast<uint32_t*>(ws);
+  if (shared) {
+    a.group_start = group_start;
+    a.shared_blocks = shared_blocks;
+    a.num_groups = num_groups;
+    a.members_per_item = plan.members_per_item;
+    a.seq_prefix = reinterpret_cast<int32_t*>(ws + plan.seq_prefix_off);
+    a.group_pref = reinterpret_cast<int32_t*>(ws + plan.group_pref_off);
+  }
+  const bool e5m2 = dims->dtype == PKV_FP8_E5M2;
+  auto kern = shared ? (!fp8 ? pkv::token_prepare_kernel<false, false, true>
+                             : e5m2 ? pkv::token_prepare_kernel<true, true, true>
+                                    : pkv::token_prepare_kernel<true, false, true>)
+                     : (!fp8 ? pkv::token_prepare_kernel<false, false, false>
+                             : e5m2 ? pkv::token_prepare_kernel<true, true, false>
+                                    : pkv::token_prepare_kernel<true, false, false>);
+  cudaError_t e = launch(kern, dim3(grid), dim3(pkv::kPlanThreads), 0,
+                         static_cast<cudaStream_t>(cuda_stream), a);
+  if (e != cudaSuccess) return cuda_fail(e, "token prologue launch");
+  return PKV_OK;
+}
+
+}  // namespace
+
+namespace {
+
 // The shared-prefix decode: its plan, and the run over it (bf16 / fp32 pools,
 // or FP8 pools with their scales when `fp8`).
 pkv_status plan_shared(const int32_t* context_lens, const int32_t* group_start,
@@ -976,6 +1064,21 @@ pkv_status pkv_paged_attention_decode_shared_fp8(
                          shared_blocks, num_groups, scale, true, k_scale, v_scale, dims,
                          max_context_len, partition_tokens, workspace, workspace_bytes,
                          cuda_stream);
+}
+
+pkv_status pkv_decode_prepare_tokens(const void* k, const void* v, void* k_cache, void* v_cache,
+                                     const int32_t* block_tables, const int32_t* context_lens,
+                                     const int32_t* token_seq, const int32_t* token_pos,
+                                     int32_t num_tokens, int64_t* slot_mapping_out,
+                                     float k_scale, float v_scale, const int32_t* group_start,
+                                     const int32_t* shared_blocks, int32_t num_groups,
+                                     const pkv_dims* dims, int32_t max_context_len,
+                                     int32_t partition_tokens, void* workspace,
+                                     size_t workspace_bytes, void* cuda_stream) {
+  return prepare_tokens(k, v, k_cache, v_cache, block_tables, context_lens, token_seq, token_pos,
+                        num_tokens, slot_mapping_out, k_scale, v_scale, group_start,
+                        shared_blocks, num_groups, dims, max_context_len, partition_tokens,
+                        workspace, workspace_bytes, cuda_stream);
 }
 
 pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache, void* v_cache,

@@ -214,19 +214,15 @@ __device__ __forceinline__ int32_t group_of(const int32_t* group_start, int32_t 
   return lo;
 }
 
-__global__ void __launch_bounds__(kPlanThreads)
-    plan_shared_kernel(const int32_t* __restrict__ context_lens,
-                       const int32_t* __restrict__ group_start,
-                       const int32_t* __restrict__ shared_blocks, int32_t num_groups,
-                       int32_t num_seqs, int32_t max_len, int32_t part_blocks,
-                       int32_t members_per_item, PlanItem* __restrict__ items,
-                       uint32_t* __restrict__ counters, int32_t* __restrict__ seq_prefix,
-                       int32_t* group_pref) {
-  __shared__ uint32_t hist[kPlanBuckets];
-  __shared__ uint32_t warp_sums[kPlanThreads / 32];
-  __shared__ int32_t gs_cache[kPlanGroupCache];  // the group bounds, when they fit
-  pdl_wait();
-  pdl_trigger();
+// The shared-prefix plan, run by one CTA of kPlanThreads threads (the caller
+// has passed griddepcontrol.wait); gs_cache holds kPlanGroupCache ints of
+// shared memory.
+__device__ __forceinline__ void plan_shared_body(
+    const int32_t* __restrict__ context_lens, const int32_t* __restrict__ group_start,
+    const int32_t* __restrict__ shared_blocks, int32_t num_groups, int32_t num_seqs,
+    int32_t max_len, int32_t part_blocks, int32_t members_per_item, PlanItem* __restrict__ items,
+    uint32_t* __restrict__ counters, int32_t* __restrict__ seq_prefix, int32_t* group_pref,
+    uint32_t* hist, uint32_t* warp_sums, int32_t* gs_cache) {
   const int tid = threadIdx.x;
   const int32_t part_tokens = part_blocks * kBlock;
   for (int b = tid; b < kPlanBuckets; b += kPlanThreads) hist[b] = 0;
@@ -322,6 +318,24 @@ __global__ void __launch_bounds__(kPlanThreads)
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(kPlanThreads)
+    plan_shared_kernel(const int32_t* __restrict__ context_lens,
+                       const int32_t* __restrict__ group_start,
+                       const int32_t* __restrict__ shared_blocks, int32_t num_groups,
+                       int32_t num_seqs, int32_t max_len, int32_t part_blocks,
+                       int32_t members_per_item, PlanItem* __restrict__ items,
+                       uint32_t* __restrict__ counters, int32_t* __restrict__ seq_prefix,
+                       int32_t* group_pref) {
+  __shared__ uint32_t hist[kPlanBuckets];
+  __shared__ uint32_t warp_sums[kPlanThreads / 32];
+  __shared__ int32_t gs_cache[kPlanGroupCache];  // the group bounds, when they fit
+  pdl_wait();
+  pdl_trigger();
+  plan_shared_body(context_lens, group_start, shared_blocks, num_groups, num_seqs, max_len,
+                   part_blocks, members_per_item, items, counters, seq_prefix, group_pref, hist,
+                   warp_sums, gs_cache);
 }
 
 // ------------------------------------------------------------ decode kernel
