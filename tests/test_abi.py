@@ -163,3 +163,79 @@ def test_product_path_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), f
+
+
+def test_shared_prefix_workspace_sizes():
+    """The shared-prefix plan keeps partials even when the plain decode is single pass, one
+    partial more per row, room for two items per (sequence, partition) and the per-sequence
+    and per-group block counts."""
+    d = dims(B=256, hq=32, hkv=8, nb=40000, mb=512)
+    assert pkv.decode_workspace_bytes(d, 1600) < pkv.decode_shared_workspace_bytes(d, 1600)
+    max_parts, po, pm, sp = pkv.decode_shared_workspace_layout(d, 1600)
+    assert max_parts == 2
+    assert sp % 256 == 0 and po % 256 == 0 and pm % 256 == 0
+    assert sp >= 256 + 2 * 256 * 2 * 32            # counters, then 2*B*max_parts items
+    assert po >= sp + 2 * 256 * 4                  # seq_prefix, group block counts
+    assert pm >= po + 256 * 32 * 2 * 128 * 4
+    assert pkv.decode_shared_workspace_bytes(d, 1600) >= pm + 256 * 32 * 2 * 2 * 4
+    # split-K: one partial more than the plain decode's
+    d = dims(B=8, hq=64, hkv=8, nb=81920, mb=8192)
+    assert pkv.decode_shared_workspace_layout(d, 131072, 512)[0] == \
+        pkv.decode_workspace_layout(d, 131072, 512)[0] + 1
+    assert pkv.decode_shared_workspace_bytes(dims(bs=8), 64) == 0
+
+
+def test_shared_prefix_calls_reject_bad_arguments(lib):
+    d = dims()
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any launch
+    big = 1 << 24
+
+    def one_shot(num_groups, dd=d, fp8=False, ws=big):
+        args = [fake] * 8 + [num_groups, 1.0]
+        if fp8:
+            return lib.pkv_paged_attention_decode_shared_fp8(*args, 1.0, 1.0, ctypes.byref(dd),
+                                                             64, 0, fake, ws, null)
+        return lib.pkv_paged_attention_decode_shared(*args, ctypes.byref(dd), 64, 0, fake, ws,
+                                                     null)
+
+    assert pkv.STATUS_NAMES[one_shot(d.num_seqs + 1)] == "PKV_ERR_SHAPE"
+    assert pkv.STATUS_NAMES[one_shot(-1)] == "PKV_ERR_SHAPE"
+    assert pkv.STATUS_NAMES[one_shot(2, ws=64)] == "PKV_ERR_WORKSPACE"
+    assert pkv.STATUS_NAMES[one_shot(2, fp8=True)] == "PKV_ERR_UNSUPPORTED"   # bf16 pools
+    fp8 = dims(dtype=pkv.PKV_FP8_E4M3)
+    assert pkv.STATUS_NAMES[one_shot(2, dd=fp8)] == "PKV_ERR_UNSUPPORTED"     # scales needed
+    st = lib.pkv_paged_attention_decode_shared(null, *[fake] * 7, 2, 1.0, ctypes.byref(d), 64,
+                                               0, fake, big, null)
+    assert pkv.STATUS_NAMES[st] == "PKV_ERR_NULL"
+    st = lib.pkv_decode_plan_shared(fake, null, fake, 2, ctypes.byref(d), 64, 0, fake, big, null)
+    assert pkv.STATUS_NAMES[st] == "PKV_ERR_NULL"
+    empty = dims(B=0)
+    assert lib.pkv_paged_attention_decode_shared(*[null] * 8, 0, 1.0, ctypes.byref(empty), 0, 0,
+                                                 null, 0, null) == 0
+
+
+def test_token_prologue_rejects_bad_arguments(lib):
+    d = dims()
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    big = 1 << 24
+
+    def call(k=fake, T=4, ks=1.0, vs=1.0, gs=null, G=0, dd=d, ws=big):
+        return pkv.STATUS_NAMES[lib.pkv_decode_prepare_tokens(
+            k, fake, fake, fake, fake, fake, fake, fake, T, null, ks, vs, gs, fake, G,
+            ctypes.byref(dd), 64, 0, fake, ws, null)]
+
+    assert call(T=-1) == "PKV_ERR_SHAPE"
+    assert call(k=null) == "PKV_ERR_NULL"
+    assert call(k=odd) == "PKV_ERR_ALIGN"
+    assert call(ws=64) == "PKV_ERR_WORKSPACE"
+    assert call(gs=fake, G=d.num_seqs + 1) == "PKV_ERR_SHAPE"
+    fp8 = dims(dtype=pkv.PKV_FP8_E5M2)
+    assert call(dd=fp8, ks=0.0) == "PKV_ERR_SHAPE"
+    assert call(dd=fp8, vs=float("inf")) == "PKV_ERR_SHAPE"
+    # the shared plan needs the larger workspace
+    need_plain = pkv.decode_workspace_bytes(d, 64)
+    assert call(gs=fake, G=2, ws=need_plain) == "PKV_ERR_WORKSPACE"
+    assert call(dd=dims(B=0)) == "PKV_OK"
