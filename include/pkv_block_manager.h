@@ -84,6 +84,14 @@ int32_t pkv_bm_take_copies(pkv_block_manager *bm, int64_t *pairs_out, int32_t ma
 pkv_status pkv_bm_block_tables(pkv_block_manager *bm, const int64_t *seq_ids, int32_t n,
                                int32_t max_blocks, int32_t *tables_out, int32_t *lens_out);
 
+/* An order of n sequences (order_out[i] = a position in seq_ids) in which
+ * sequences that begin with the same physical blocks are consecutive: the
+ * tables' full blocks sorted lexicographically, ties in the given order.
+ * Laying out a step's rows (q, out, tables) in this order makes the runs of
+ * pkv_bm_shared_prefix_groups as long as the sharing allows. */
+pkv_status pkv_bm_prefix_order(pkv_block_manager *bm, const int64_t *seq_ids, int32_t n,
+                               int32_t *order_out);
+
 /* Groups for pkv_paged_attention_decode_shared over n sequences taken in the
  * order of seq_ids (the rows of the tables pkv_bm_block_tables exports in the
  * same order): maximal runs of consecutive sequences that hold the same

@@ -134,6 +134,7 @@ def load_library() -> ctypes.CDLL:
             "pkv_bm_stats": (ctypes.c_int, [P, P, P, P, P]),
             "pkv_bm_refcount": (i32, [P, i32]),
             "pkv_bm_shared_prefix_groups": (ctypes.c_int, [P, P, i32, i32, P, P, P]),
+            "pkv_bm_prefix_order": (ctypes.c_int, [P, P, i32, P]),
             "pkv_last_error_message": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sig.items():
@@ -956,6 +957,15 @@ class BlockManager:
                                                 tables.ctypes.data_as(ctypes.c_void_p),
                                                 lens.ctypes.data_as(ctypes.c_void_p)))
         return tables, lens
+
+    def prefix_order(self, seq_ids):
+        """Positions of seq_ids in an order where sequences beginning with the same physical
+        blocks are consecutive (int32 [n]); lay out q, out and the tables in it."""
+        s, sp = self._arr(seq_ids, self._np.int64)
+        out = self._np.empty(s.shape[0], dtype=self._np.int32)
+        _bm_check(self._lib.pkv_bm_prefix_order(self._h, sp, s.shape[0],
+                                                out.ctypes.data_as(ctypes.c_void_p)))
+        return out
 
     def shared_prefix_groups(self, seq_ids, min_shared_blocks: int = 1):
         """(group_start int32 [G+1], shared_blocks int32 [G]) for paged_attention_decode_shared

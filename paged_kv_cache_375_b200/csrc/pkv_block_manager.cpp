@@ -312,6 +312,34 @@ pkv_status pkv_bm_block_tables(pkv_block_manager* bm, const int64_t* seq_ids, in
   return PKV_OK;
 }
 
+pkv_status pkv_bm_prefix_order(pkv_block_manager* bm, const int64_t* seq_ids, int32_t n,
+                               int32_t* order_out) {
+  if (!bm || ((!seq_ids || !order_out) && n > 0)) return PKV_ERR_NULL;
+  if (n < 0) return PKV_ERR_SHAPE;
+  std::vector<const Sequence*> seqs(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end()) return PKV_ERR_NOT_FOUND;
+    seqs[i] = &it->second;
+  }
+  // lexicographic order of the full blocks' physical ids: sequences that
+  // begin with the same blocks end up next to each other, and the longer the
+  // common run the closer (ties keep the given order)
+  std::vector<int32_t> idx(static_cast<size_t>(n));
+  for (int32_t i = 0; i < n; ++i) idx[i] = i;
+  const size_t bs = static_cast<size_t>(bm->bs);
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t x, int32_t y) {
+    const Sequence& a = *seqs[x];
+    const Sequence& b = *seqs[y];
+    const size_t fa = std::min(a.tokens.size() / bs, a.table.size());
+    const size_t fb = std::min(b.tokens.size() / bs, b.table.size());
+    return std::lexicographical_compare(a.table.begin(), a.table.begin() + fa, b.table.begin(),
+                                        b.table.begin() + fb);
+  });
+  std::copy(idx.begin(), idx.end(), order_out);
+  return PKV_OK;
+}
+
 pkv_status pkv_bm_shared_prefix_groups(pkv_block_manager* bm, const int64_t* seq_ids, int32_t n,
                                        int32_t min_shared_blocks, int32_t* group_start_out,
                                        int32_t* shared_blocks_out, int32_t* num_groups_out) {

@@ -273,3 +273,35 @@ def test_shared_prefix_groups_random_forest(seed):
     for m in (1, 2, 4):
         check_groups(bm, ids, m)
         check_groups(bm, list(rng.permutation(ids)), m)
+
+
+@pytest.mark.parametrize("seed", [5, 6, 7])
+def test_prefix_order_puts_sharers_together(seed):
+    """In the prefix order every family of forks (sharing at least one full block) forms
+    one run, whatever order the step's rows came in; the order is a permutation."""
+    rng = np.random.default_rng(seed)
+    bm = pkv.BlockManager(4000, BS, seed=seed)
+    fams = []
+    for p in range(10):
+        root = 100 * p
+        bm.add_sequence(root, rng.integers(0, 1000, size=int(rng.integers(16, 200))).tolist())
+        fam = [root]
+        for c in range(int(rng.integers(1, 6))):
+            bm.fork(root, root + c + 1)
+            fam.append(root + c + 1)
+        for s in fam:
+            for _ in range(int(rng.integers(0, 30))):
+                bm.append_tokens([s], [int(rng.integers(0, 1000))])
+        fams.append(fam)
+    bm.take_copies()
+    ids = [s for f in fams for s in f]
+    shuffled = list(rng.permutation(ids))
+    order = bm.prefix_order(shuffled)
+    assert sorted(order.tolist()) == list(range(len(ids)))
+    ordered = [int(shuffled[i]) for i in order]
+    gs, sb = check_groups(bm, ordered, 1)
+    runs = [set(ordered[gs[r]:gs[r + 1]]) for r in range(len(sb))]
+    for f in fams:
+        assert set(f) in runs, f"family {f} split over runs"
+    with pytest.raises(pkv.PkvError):
+        bm.prefix_order([0, 12345])
