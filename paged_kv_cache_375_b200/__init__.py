@@ -21,7 +21,9 @@ per-sequence block table, slot_mapping, copy-on-write of shared blocks):
                              decode reading a prefix shared by consecutive
                              sequences once per group
   *_fp8 variants             FP8 (e4m3 or e5m2) pools with per-pool scales
-  BlockManager               host-side block bookkeeping with prefix caching
+  BlockManager               host-side block bookkeeping with prefix caching; its
+                             prefix_order / shared_prefix_groups feed the
+                             shared-prefix decode
   check_device_error()
 """
 from __future__ import annotations
