@@ -78,3 +78,23 @@ def test_algorithmic_bytes_count_every_context_token_once_per_kv_head():
     assert a["kv"] == (17 + 40) * 2 * 64 * 2 * 2
     assert a["table"] == (2 + 3) * 4
     assert a["total"] == a["kv"] + a["q_out"] + a["table"] + a["lens"]
+
+
+def test_plan_item_accounting():
+    """The bench's count of planned work items (the plan kernel's written bytes) for the
+    plain and the shared-prefix plans of the parallel-sampling batch."""
+    import types
+    import bench
+    import workloads
+    b = workloads.c4_shared_prefix(prompts=4, samples=8, prefix=256, max_tail=100,
+                                   num_blocks=2000)
+    lens = b.context_lens.astype(np.int64)
+    P = int(((int(lens.max()) + 15) // 16) * 16)          # single pass
+    plain = types.SimpleNamespace(b=b, part_tokens=P, shared=False)
+    assert bench.plan_items(plain) == b.num_seqs
+    shared = types.SimpleNamespace(b=b, part_tokens=P, shared=True)
+    # per prompt: 2 prefix items (4 samples x 4 heads = 16 rows each) + 8 own-block items
+    assert bench.plan_items(shared) == 4 * (2 + 8)
+    split = types.SimpleNamespace(b=b, part_tokens=64, shared=True)
+    n_own = int(np.maximum(1, (lens - 256 + 63) // 64).sum())
+    assert bench.plan_items(split) == 4 * (256 // 64) * 2 + n_own
