@@ -5,7 +5,10 @@ One step = one pass of the whole path over one synthetic batch, with every
 input already resident in HBM:
   slot indexing of the new tokens -> reshape_and_cache -> decode plan ->
   decode (-> log-sum-exp merge when sequences are split)
-(the shared-prefix workload also runs copy_blocks first).
+The first three share one launch when the new tokens are one per sequence
+or a short list (the fused prologues).  The shared-prefix workload runs
+copy_blocks first and decodes with the shared-prefix plan: each prompt's
+blocks read once for its samples, merged with each sample's own blocks.
 
 The default workload is the Llama-3-8B-shaped GQA batch (256 sequences, 32 q /
 8 kv heads, head_dim 128, bf16, lognormal context lengths with median 1000),
@@ -14,7 +17,7 @@ KV pools (about 2.3 GB) are far larger than the 126 MB L2, so no flush is
 needed between steps.
 
 Usage:
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c5]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c3|c2|c4|c5|...]
   python bench.py --impl reference ...      # the float64 CPU oracle, timed
 For N > 1 launch one process per GPU with torch.distributed.run; every rank
 decodes its own replica of the batch (the path has no exchange step), the
