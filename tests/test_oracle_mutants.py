@@ -53,6 +53,9 @@ MUTANTS = {
     "e5m2_value_three_mantissa_bits": ("v = ldexp(1.0 + man / 4.0, exp - 15);",
                                        "v = ldexp(1.0 + man / 8.0, exp - 15);"),
     "e5m2_subnormal_step": ("v = ldexp((double)man, -16);", "v = ldexp((double)man, -15);"),
+    "merge_f32_m_and_l_swapped": ("        md[p] = (double)m[p];\n", "        md[p] = (double)l[p];\n"),
+    "merge_f32_o_transposed": ("od[(int64_t)p * head_dim + d] = (double)o[(int64_t)p * head_dim + d];",
+                               "od[(int64_t)p * head_dim + d] = (double)o[(int64_t)d * nparts + p];"),
     "fp8_scale_dropped": ("V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype) * pb->v_scale;",
                           "V[(int64_t)j * D + d] = widen(pb->v_cache, row + d, pb->dtype);"),
 }

@@ -366,6 +366,55 @@ def test_merge_ignores_empty_parts():
     assert np.array_equal(oracle.lse_merge(m[[0]], l[[0]], o[[0]]), np.zeros(2))
 
 
+def test_golden_lse_merge_from_float32_partials():
+    """The hand-derived two-part merge, entered as single-precision partials (the
+    form a GPU writes them in): only the rounding of ln 3 to float32 remains."""
+    g = _golden("lse_merge_two_parts.json")
+    out = oracle.lse_merge(np.array(g["m"], dtype=np.float32), np.array(g["l"], dtype=np.float32),
+                           np.array(g["o"], dtype=np.float32))
+    np.testing.assert_allclose(out, g["expected"], rtol=0, atol=1e-6)
+
+
+def test_float32_merge_is_the_merge_of_the_widened_partials():
+    """Single-precision partials (with empty parts and rows whose every part is
+    empty) merge exactly as their values widened to float64 by numpy do; the
+    float64 merge is pinned on its own above (fixture, associativity)."""
+    rng = np.random.default_rng(31)
+    for trial in range(40):
+        P = int(rng.integers(1, 12))
+        D = int(rng.choice([1, 3, 64, 128]))
+        m = (rng.standard_normal(P) * 6).astype(np.float32)
+        l = (rng.random(P) * 50 + 0.5).astype(np.float32)
+        o = rng.standard_normal((P, D)).astype(np.float32)
+        empty = rng.random(P) < (1.0 if trial % 10 == 9 else 0.3)
+        m[empty] = -np.inf
+        l[empty] = 0.0
+        o[empty] = np.nan
+        got = oracle.lse_merge(m, l, o)
+        want = oracle.lse_merge(m.astype(np.float64), l.astype(np.float64), o.astype(np.float64))
+        assert np.array_equal(got, want, equal_nan=False), trial
+        if empty.all():
+            assert np.array_equal(got, np.zeros(D))
+
+
+def test_float32_merge_of_rounded_partitions_matches_single_pass():
+    """Partition statistics rounded to float32 and merged through the
+    single-precision entry stay within float32 rounding of the single pass."""
+    rng = np.random.default_rng(32)
+    lens = [5, 33, 700]
+    q, kp, vp, bt, cl, _, _, _ = random_paged(rng, lens, 4, 2, 16)
+    full = oracle.paged_decode(q, kp, vp, bt, cl, 0.25)
+    for s, L in enumerate(lens):
+        for h in range(4):
+            parts = [oracle.partition_stats(q, kp, vp, bt, cl, 0.25, s, h, t0, min(L, t0 + 64))
+                     for t0 in range(0, L, 64)]
+            m = np.array([p[0] for p in parts], dtype=np.float32)
+            l = np.array([p[1] for p in parts], dtype=np.float32)
+            o = np.array([p[2] for p in parts], dtype=np.float32)
+            merged = oracle.lse_merge(m, l, o)
+            np.testing.assert_allclose(merged, full[s, h], rtol=0, atol=2e-6)
+
+
 # ------------------------------------------------- reshape_and_cache, slots ----
 def test_reshape_then_decode_equals_dense():
     """Write a whole context token by token through slot_mapping + reshape_and_cache into a
