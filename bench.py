@@ -191,6 +191,11 @@ def whole_job_value(units_per_rank: float, world: int, seconds: float) -> float:
 # ------------------------------------------------------------------ our arm
 # New tokens per step up to which the writes share a launch with the plan.
 TOKEN_PROLOGUE_MAX = 4096
+# The roofline's decode duration: at least this many bracketed launches and this many
+# seconds after the timed region (at most ROOF_MAX_LAUNCHES).
+ROOF_LAUNCHES = 200
+ROOF_SECONDS = 0.3
+ROOF_MAX_LAUNCHES = 5000
 
 
 class Step:
@@ -337,9 +342,9 @@ def run_ours(args, world, rank, local):
 
     # Timed region: K steps back to back.  Events between launches would break
     # the overlap of consecutive launches (programmatic dependent launch), so
-    # only every SAMPLE-th step has its decode launch bracketed by events; those
-    # give the decode kernel's duration for the roofline (slightly pessimistic:
-    # a bracketed launch cannot overlap the plan kernel before it).
+    # only every SAMPLE-th step has its decode launch bracketed by events (a
+    # bracketed launch cannot overlap the plan kernel before it); the roofline's
+    # decode duration comes from a longer loop right after the region.
     #
     # A working set that L2 could hold a good part of (the tiny fp32 batch, the
     # shared-prefix batch's unique bytes) is flushed before every step by a
@@ -356,7 +361,8 @@ def run_ours(args, world, rank, local):
     sampler = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with sampler:
+    sampler.__enter__()
+    try:
         step_ev[0][0].record(stream)
         for i in range(K):
             if flush:
@@ -375,10 +381,32 @@ def run_ours(args, world, rank, local):
         if not flush:
             step_ev[0][1].record(stream)
         torch.cuda.synchronize(dev)
+        total_ms = sum(a.elapsed_time(z) for a, z in step_ev)
+        # Roofline sample, right after the timed region and under the same clock
+        # sampling: the decode launch of at least ROOF_LAUNCHES further steps (and
+        # ROOF_SECONDS), each bracketed by events, so the duration does not rest on
+        # the few launches a short timed region samples.  Each decode follows its
+        # step's own cache ops and plan (the decode consumes the plan's work
+        # counters) and, for flushed workloads, the L2 flush.
+        n_roof = int(min(ROOF_MAX_LAUNCHES,
+                         max(ROOF_LAUNCHES, ROOF_SECONDS * 1e3 / max(total_ms / K, 1e-3))))
+        roof_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(n_roof)]
+        for i in range(n_roof):
+            if flush:
+                flush_buf.fill_(i & 0xff)
+            step.cache_ops()
+            step.plan()
+            roof_ev[i][0].record(stream)
+            step.decode()
+            roof_ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    finally:
+        sampler.__exit__(None, None, None)
     barrier(world)
     pkv.check_device_error(dev)
-    total_ms = sum(a.elapsed_time(z) for a, z in step_ev)
-    decode_samples = sorted(a.elapsed_time(z) for a, z in ev.values())
+    region_samples = sorted(a.elapsed_time(z) for a, z in ev.values())
+    decode_samples = sorted(a.elapsed_time(z) for a, z in roof_ev)
     decode_ms = statistics.mean(decode_samples)
     ops = None if args.no_breakdown else breakdown(step, stream, dev)
     total_ms = max_over_ranks(total_ms, world, dev)
@@ -397,7 +425,10 @@ def run_ours(args, world, rank, local):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": b.dtype, "data": "synthetic",
         "config": {
-            "workload": f"{name}: {workloads.CONFIGS[name]}",
+            "workload": f"{name}: {workloads.CONFIGS[name]}; " + (
+                f"split-K, {step.part_tokens}-token partitions this run" if step.split
+                and not step.shared else "single pass this run" if not step.split else
+                "shared-prefix plan this run"),
             "batch": b.num_seqs, "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads,
             "head_dim": b.head_dim, "block_size": 16, "num_blocks": b.num_blocks,
             "context_tokens": int(b.context_lens.sum()), "max_context_len": b.max_context_len,
@@ -418,10 +449,15 @@ def run_ours(args, world, rank, local):
         },
         "pct_of_hbm_peak": round(100.0 * value / world / peak, 2),
         "seqs_per_s": round(whole_job_value(b.num_seqs * K, world, seconds), 1),
-        "breakdown": {"decode_ms_sampled": round(decode_ms, 5),
+        "breakdown": {"decode_ms_mean": round(decode_ms, 5),
                       "decode_ms_median": round(statistics.median(decode_samples), 5),
-                      "decode_ms_best": round(decode_samples[0], 5), "ops_alone": ops,
-                      "note": "decode: every 8th step of the timed region bracketed by events; "
+                      "decode_ms_best": round(decode_samples[0], 5),
+                      "decode_launches_sampled": len(decode_samples),
+                      "decode_ms_in_region_mean": round(statistics.mean(region_samples), 5),
+                      "decode_launches_in_region": len(region_samples), "ops_alone": ops,
+                      "note": "decode: each of the roofline loop's launches after the timed "
+                              "region bracketed by events (in the timed region, every 8th "
+                              "step's decode is bracketed too: decode_ms_in_region_mean); "
                               "other ops: each timed alone (50 launches) after the timed region"},
         "roofline": {
             "kernel": "decode_kernel" + (" + merge_kernel" if step.split else ""),

@@ -248,9 +248,14 @@ pkv_status pkv_decode_run(void *out, const void *q, const void *k_cache, const v
  * same arguments as pkv_paged_attention_decode minus the workspace: the
  * scratch is a fixed array of PKV_STATIC_WORKSPACE_BYTES inside the library,
  * reserved on every GPU that loads the library until the process exits.
- *  - The call allocates nothing.  The first call on a device looks up that
- *    array's device address (cudaGetSymbolAddress, with that device current)
- *    and caches it; make that first call before any stream capture.
+ *  - The call allocates nothing.  It runs on the device that owns `out`;
+ *    q, the caches, block_tables and context_lens must be on that device too
+ *    (else PKV_ERR_SHAPE).  The first call on a device makes that device
+ *    current for the library, looks up the array's device address there
+ *    (cudaGetSymbolAddress) and caches it for the rest of the process; make
+ *    that first call before any stream capture (a first call on a capturing
+ *    stream returns PKV_ERR_UNSUPPORTED).  The cached address does not
+ *    survive a cudaDeviceReset of that device.
  *  - A decode whose pkv_decode_workspace_bytes() exceeds
  *    PKV_STATIC_WORKSPACE_BYTES is rejected with PKV_ERR_WORKSPACE (the
  *    message gives both sizes); use pkv_paged_attention_decode with a

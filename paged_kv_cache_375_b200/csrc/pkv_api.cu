@@ -393,20 +393,54 @@ std::mutex g_static_ws_mu;
 void* g_static_ws_ptr[kMaxDevices] = {};
 
 // Device address of g_static_workspace on the current device, looked up once
-// per device (host code cannot use the array's name as a device pointer).
-pkv_status static_workspace(void** ptr) {
+// per device (host code cannot use the array's name as a device pointer).  The
+// caller binds the device first.  The lookup may load the module, which a
+// stream capture does not allow, so the first call on a device refuses a
+// capturing stream.  The cached address belongs to the device's primary
+// context: it does not survive a cudaDeviceReset.
+pkv_status static_workspace(cudaStream_t stream, void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_UNSUPPORTED, "device %d out of range", dev);
   std::lock_guard<std::mutex> lock(g_static_ws_mu);
   if (!g_static_ws_ptr[dev]) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (cap != cudaStreamCaptureStatusNone)
+      return fail(PKV_ERR_UNSUPPORTED,
+                  "the first pkv_paged_attention_decode_static call on device %d looks up the "
+                  "built-in scratch and must not be made while its stream is being captured",
+                  dev);
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
     g_static_ws_ptr[dev] = p;
   }
   *ptr = g_static_ws_ptr[dev];
+  return PKV_OK;
+}
+
+// Every operand of a call must live on the device that owns `out` (the device
+// bind_device made current): the kernels run there and read all of them.
+pkv_status check_same_device(const void* const* ptrs, const char* const* names, int n) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  for (int i = 0; i < n; ++i) {
+    cudaPointerAttributes a;
+    e = cudaPointerGetAttributes(&a, ptrs[i]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "cudaPointerGetAttributes");
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+      return fail(PKV_ERR_SHAPE, "%s is not device memory", names[i]);
+    if (a.device != dev)
+      return fail(PKV_ERR_SHAPE, "%s is on device %d but out is on device %d", names[i],
+                  a.device, dev);
+  }
   return PKV_OK;
 }
 
@@ -1124,8 +1158,17 @@ pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const voi
                 "this decode needs %zu bytes of scratch but the built-in scratch holds %u; "
                 "call pkv_paged_attention_decode with a workspace of your own",
                 plan.total, (unsigned)PKV_STATIC_WORKSPACE_BYTES);
+  if (dims->num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  // The scratch address is per device: bind the device that owns `out` (the
+  // device the kernels run on) before looking it up.
+  if ((st = bind_device(out, "out")) != PKV_OK) return st;
+  const void* const ptrs[] = {q, k_cache, v_cache, block_tables, context_lens};
+  const char* const names[] = {"q", "k_cache", "v_cache", "block_tables", "context_lens"};
+  if ((st = check_same_device(ptrs, names, 5)) != PKV_OK) return st;
   void* ws = nullptr;
-  if ((st = static_workspace(&ws)) != PKV_OK) return st;
+  if ((st = static_workspace(static_cast<cudaStream_t>(cuda_stream), &ws)) != PKV_OK) return st;
   return pkv_paged_attention_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                                     dims, max_context_len, partition_tokens, ws,
                                     PKV_STATIC_WORKSPACE_BYTES, cuda_stream);

@@ -25,11 +25,11 @@ def dev_i32(a: np.ndarray, device) -> torch.Tensor:
 
 
 def host_bits(t: torch.Tensor) -> np.ndarray:
-    """Host copy: float32 as is, bf16 as its uint16 bit patterns, e4m3 as its codes."""
+    """Host copy: float32 as is, bf16 as its uint16 bit patterns, FP8 as its codes."""
     t = t.detach().contiguous().cpu()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
-    if t.dtype == torch.float8_e4m3fn:
+    if t.dtype in (torch.float8_e4m3fn, torch.float8_e5m2):
         return t.view(torch.uint8).numpy()
     return t.numpy()
 
@@ -83,6 +83,20 @@ def check_close(out_gpu: torch.Tensor, ref: np.ndarray, dtype: str, what: str = 
         worst = (err / bound).max()
         assert worst <= 1.0, f"{what}: error {worst:.3f} of the bound (max abs {err.max():.3e})"
     return float(err.max())
+
+
+def compact_all(b: workloads.Batch, k_cache: torch.Tensor, v_cache: torch.Tensor):
+    """Host copies of every block some sequence references (each block once, shared
+    blocks included) and the block tables renumbered onto them, so the oracle can
+    recompute every output of a full-size batch without copying the whole pool back."""
+    nblk = (b.context_lens.astype(np.int64) + 15) // 16
+    used = np.arange(b.block_tables.shape[1])[None, :] < nblk[:, None]
+    uniq, inv = np.unique(b.block_tables[used], return_inverse=True)
+    bt = np.full(b.block_tables.shape, -1, dtype=np.int32)
+    bt[used] = inv.astype(np.int32)
+    idx = torch.from_numpy(uniq if uniq.size else np.zeros(1, np.int64)).long()
+    idx = idx.to(k_cache.device)
+    return host_bits(k_cache.index_select(0, idx)), host_bits(v_cache.index_select(0, idx)), bt
 
 
 def sample_tasks(b: workloads.Batch, n: int, seed: int = 0) -> np.ndarray:

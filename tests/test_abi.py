@@ -131,6 +131,26 @@ def test_decode_rejects_null_and_small_workspace(lib):
     assert pkv.STATUS_NAMES[st] == "PKV_ERR_ALIGN"
 
 
+def test_static_decode_binds_the_output_device_before_the_scratch_lookup(lib):
+    """The built-in scratch's address is per device, so the no-allocation decode must make
+    the device that owns `out` current before looking it up.  With host buffers and a
+    nonzero batch the call therefore fails while binding `out` (at the pointer query on a
+    machine without a GPU, with 'not device memory' on one), never at the lookup."""
+    import numpy as np
+    fn = lib.pkv_paged_attention_decode_static
+    P, i32 = ctypes.c_void_p, ctypes.c_int32
+    fn.argtypes = [P, P, P, P, P, P, ctypes.c_float, ctypes.POINTER(pkv.PkvDims), i32, i32, P]
+    fn.restype = ctypes.c_int
+    d = dims()
+    bufs = [np.zeros(1 << 14, dtype=np.uint8) for _ in range(6)]
+    ptrs = [P(b.ctypes.data) for b in bufs]
+    st = fn(*ptrs, 1.0, ctypes.byref(d), 64, 0, P(0))
+    msg = lib.pkv_last_error_message()
+    assert st != 0
+    assert b"cudaGetSymbolAddress" not in msg and b"cudaGetDevice" not in msg, msg
+    assert b"cudaPointerGetAttributes" in msg or b"out is not device memory" in msg, msg
+
+
 def test_empty_batch_is_a_no_op(lib):
     d = dims(B=0)
     null = ctypes.c_void_p(0)

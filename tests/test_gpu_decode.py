@@ -5,8 +5,8 @@ Covers: the tiny fp32 workload, randomised small shapes (head_dim 64/128,
 group sizes 1..16, lengths around block boundaries, empty contexts), single-pass
 vs split-K vs oracle, the split-K partials against the oracle's merge, the
 paging invariants on the GPU (placement permutation and shared-vs-private are
-bitwise), poisoned padding, device-side index errors, and the full-size
-workloads on sampled outputs.
+bitwise), poisoned padding, device-side index errors, and every output of the
+full-size workloads.
 """
 import numpy as np
 import pytest
@@ -15,8 +15,8 @@ import torch
 import oracle
 import paged_kv_cache_375_b200 as pkv
 import workloads
-from gpu_util import (check_close, compact_for_tasks, dev_i32, gpu_step, host_bits,
-                      oracle_caches_after_step, sample_tasks, to_f64)
+from gpu_util import (check_close, dev_i32, gpu_step, host_bits,
+                      oracle_caches_after_step, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -172,23 +172,39 @@ def test_context_longer_than_hint_is_flagged(cuda_device):
     assert pkv.device_error_bits() & pkv.DEVERR_LEN
 
 
-@pytest.mark.parametrize("name,n_tasks,partition", [
-    ("c2_llama2_13b_mha", 48, 0),
-    ("c3_llama3_8b_gqa", 64, 0),
-    ("c3_llama3_8b_gqa", 32, 512),
-    ("c4_shared_prefix", 48, 0),
-    ("c5_long_splitk", 12, 0),
+@pytest.mark.parametrize("name,partition", [
+    ("c2_llama2_13b_mha", 0),
+    ("c3_llama3_8b_gqa", 0),
+    ("c3_llama3_8b_gqa", 512),
+    ("c4_shared_prefix", 0),
+    ("c5_long_splitk", 0),
+    ("c5_long_splitk", 512),
 ])
-def test_full_size_workloads_sampled(cuda_device, name, n_tasks, partition):
-    """Full-size workloads in the launch configuration the benchmark uses; the oracle
-    recomputes sampled (sequence, head) outputs one by one."""
+def test_full_size_workloads_every_output(cuda_device, name, partition):
+    """Full-size workloads in the launch configurations the benchmark uses (the Llama-3-8B
+    batch through the fused decode prologue; the long-context batch with the automatic
+    partition and with its configured 512-token partitions, about 1,300 partials per
+    row): the pools after the step's copies and writes equal the oracle's byte for byte,
+    and every output is recomputed by the oracle on all host cores."""
     b = workloads.BUILDERS[name](device=cuda_device)
-    out, kc, vc = gpu_step(b, partition)
+    host = b.host()                                    # the pools before the step
+    k_ref, v_ref = oracle_caches_after_step(b, host)
+    if name == "c3_llama3_8b_gqa" and partition == 0:
+        dev = b.q.device
+        bt, cl = dev_i32(b.block_tables, dev), dev_i32(b.context_lens, dev)
+        plan = pkv.DecodePlan(bt, cl, b.num_q_heads, b.k_cache, max_context_len=b.max_context_len,
+                              new_k=b.new_k, new_v=b.new_v, v_cache=b.v_cache)
+        out = torch.empty_like(b.q)
+        plan.run(out, b.q, b.k_cache, b.v_cache, b.scale)
+        kc, vc = b.k_cache, b.v_cache
+    else:
+        out, kc, vc = gpu_step(b, partition)
+    if partition:
+        assert pkv.decode_partition_tokens(
+            pkv.make_dims(b.num_seqs, b.num_q_heads, b.k_cache, b.max_blocks_per_seq),
+            b.max_context_len, partition) == partition
     assert pkv.device_error_bits() == 0
-    tasks = sample_tasks(b, n_tasks, seed=len(name))
-    kh, vh, bt = compact_for_tasks(b, kc, vc, tasks)
-    ref = oracle.paged_decode(host_bits(b.q), kh, vh, bt, b.context_lens, b.scale, tasks=tasks,
-                              threads=4)
-    got = out[torch.from_numpy(tasks[:, 0]).long(), torch.from_numpy(tasks[:, 1]).long()]
-    check_close(got, ref, b.dtype, name)
-    assert torch.isfinite(out).all()
+    assert np.array_equal(host_bits(kc), k_ref)
+    assert np.array_equal(host_bits(vc), v_ref)
+    ref = oracle.paged_decode(host["q"], k_ref, v_ref, b.block_tables, b.context_lens, b.scale)
+    check_close(out, ref, b.dtype, f"{name} partition {partition}")

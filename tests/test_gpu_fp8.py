@@ -190,34 +190,26 @@ def test_fp8_dims_rejected_where_unsupported(cuda_device):
         pkv.paged_attention_decode_fp8(out, b.q, b.k_cache, b.v_cache, bt, cl, b.scale, 0.0, 1.0)
 
 
-def test_c3_fp8_full_size_sampled(cuda_device):
-    """The full Llama-3-8B-shaped batch over FP8 pools; the new tokens' codes are compared
-    bit for bit and sampled (sequence, head) outputs are recomputed by the oracle."""
+def test_c3_fp8_full_size_every_output(cuda_device):
+    """The full Llama-3-8B-shaped batch over FP8 pools, through the fused decode prologue
+    the benchmark times: both pools bit for bit against the oracle's quantising writes,
+    and every output against the oracle on all host cores."""
     b = workloads.c3_fp8(device=cuda_device)
-    new_k = b.new_k.cpu().view(torch.int16).numpy().view(np.uint16)
-    new_v = b.new_v.cpu().view(torch.int16).numpy().view(np.uint16)
-    out = gpu_fp8_step(b)
+    host = b.host()
+    k_ref, v_ref = oracle_fp8_caches(b, host)
+    dev = b.q.device
+    bt, cl = dev_i32(b.block_tables, dev), dev_i32(b.context_lens, dev)
+    plan = pkv.DecodePlan(bt, cl, b.num_q_heads, b.k_cache, max_context_len=b.max_context_len,
+                          new_k=b.new_k, new_v=b.new_v, v_cache=b.v_cache, k_scale=b.k_scale,
+                          v_scale=b.v_scale)
+    out = torch.empty_like(b.q)
+    plan.run_fp8(out, b.q, b.k_cache, b.v_cache, b.scale, b.k_scale, b.v_scale)
     assert pkv.device_error_bits() == 0
-    # the new tokens' codes, gathered from their slots
-    slots = oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos)
-    blk, off = slots // 16, slots % 16
-    kc, vc = codes(b.k_cache), codes(b.v_cache)
-    got_k = kc[blk, :, off, :]
-    got_v = vc[blk, :, off, :]
-    # bf16 bits shifted into the upper half of a float32 are the exact values
-    want_k = oracle.e4m3_quantize((new_k.astype(np.uint32) << 16).view(np.float32), b.k_scale)
-    want_v = oracle.e4m3_quantize((new_v.astype(np.uint32) << 16).view(np.float32), b.v_scale)
-    np.testing.assert_array_equal(got_k, want_k)
-    np.testing.assert_array_equal(got_v, want_v)
-    rng = np.random.default_rng(35)
-    seqs = np.unique(np.concatenate([[int(np.argmax(b.context_lens))],
-                                     rng.integers(0, b.num_seqs, 5)]))
-    tasks = np.array([(s, h) for s in seqs for h in rng.integers(0, 32, 3)], dtype=np.int32)
-    q = b.q.cpu().view(torch.int16).numpy().view(np.uint16)
-    ref = oracle.paged_decode_fp8(q, kc, vc, b.k_scale, b.v_scale, b.block_tables,
-                                  b.context_lens, b.scale, tasks=tasks, threads=8)
-    got = out[torch.from_numpy(tasks[:, 0]).long(), torch.from_numpy(tasks[:, 1]).long()]
-    check_close(got, ref, "bf16", "c3 fp8 sampled")
+    np.testing.assert_array_equal(codes(b.k_cache), k_ref)
+    np.testing.assert_array_equal(codes(b.v_cache), v_ref)
+    ref = oracle.paged_decode_fp8(host["q"], k_ref, v_ref, b.k_scale, b.v_scale, b.block_tables,
+                                  b.context_lens, b.scale)
+    check_close(out, ref, "bf16", "c3 fp8, every output")
 
 
 def test_plain_multi_call_rejects_fp8_pools(cuda_device):
@@ -312,21 +304,3 @@ def test_fp8_one_token_chunks_equal_fp8_decode_bitwise(cuda_device):
                                    dev_i32(b.context_lens, cuda_device), b.scale, b.k_scale,
                                    b.v_scale, max_context_len=b.max_context_len)
     assert torch.equal(multi.view(torch.int16), out.view(torch.int16))
-
-
-def test_fp8_spec_decode_workload_sampled(cuda_device):
-    b = workloads.c3_spec_fp8(device=cuda_device)
-    out = gpu_fp8_multi(b)
-    assert pkv.device_error_bits() == 0
-    assert torch.isfinite(out.float()).all()
-    rng = np.random.default_rng(36)
-    seqs = np.unique(np.concatenate([[int(np.argmax(b.context_lens))],
-                                     rng.integers(0, b.num_seqs, 5)]))
-    qsl = b.query_start_loc
-    rows = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in seqs])
-    sub_qsl = np.concatenate([[0], np.cumsum(qsl[seqs + 1] - qsl[seqs])]).astype(np.int32)
-    q = b.q.cpu().view(torch.int16).numpy().view(np.uint16)[rows]
-    ref = oracle.paged_multi_fp8(np.ascontiguousarray(q), codes(b.k_cache), codes(b.v_cache),
-                                 b.k_scale, b.v_scale, b.block_tables[seqs],
-                                 b.context_lens[seqs], sub_qsl, b.scale, threads=8)
-    check_close(out[torch.from_numpy(rows).long()], ref, "bf16", "fp8 spec decode")

@@ -8,7 +8,7 @@ import torch
 import oracle
 import paged_kv_cache_375_b200 as pkv
 import workloads
-from gpu_util import check_close, compact_for_tasks, dev_i32, host_bits, oracle_caches_after_step
+from gpu_util import check_close, dev_i32, oracle_caches_after_step
 
 pytestmark = pytest.mark.gpu
 
@@ -89,30 +89,6 @@ def test_chunk_longer_than_its_context_is_flagged(cuda_device):
     b.query_start_loc = np.array([0, 2, 5], dtype=np.int32)
     gpu_multi(b, max_query_len=2)     # the second chunk (3 tokens) exceeds max_query_len
     assert pkv.device_error_bits() & pkv.DEVERR_LEN
-
-
-def test_spec_decode_workload_sampled(cuda_device):
-    """The full Llama-3-8B-shaped batch verifying 4 draft tokens per sequence; sampled
-    query rows recomputed by the oracle."""
-    b = workloads.c3_spec_decode(device=cuda_device)
-    out = gpu_multi(b)
-    assert pkv.device_error_bits() == 0
-    assert torch.isfinite(out).all()
-    rng = np.random.default_rng(5)
-    seqs = np.unique(np.concatenate([[int(np.argmax(b.context_lens))],
-                                     rng.integers(0, b.num_seqs, 6)]))
-    # the oracle on the sampled sequences only, over their compacted blocks
-    tasks = np.array([(s, 0) for s in seqs], dtype=np.int32)
-    kh, vh, bt = compact_for_tasks(b, b.k_cache, b.v_cache, tasks)
-    sub_bt = bt[seqs]
-    sub_cl = b.context_lens[seqs]
-    qsl = b.query_start_loc
-    rows = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in seqs])
-    sub_qsl = np.concatenate([[0], np.cumsum(qsl[seqs + 1] - qsl[seqs])]).astype(np.int32)
-    q_rows = host_bits(b.q)[rows]
-    ref = oracle.paged_multi(np.ascontiguousarray(q_rows), kh, vh, sub_bt, sub_cl, sub_qsl,
-                             b.scale, threads=4)
-    check_close(out[torch.from_numpy(rows).long()], ref, "bf16", "spec decode")
 
 
 def test_chunk_outside_the_query_rows_is_skipped_and_flagged(cuda_device):

@@ -76,10 +76,12 @@ def test_fused_prologue_equals_the_separate_calls(cuda_device, dtype, hq, hkv, d
                                      b.k_scale, b.v_scale)
         ref = oracle.paged_decode_fp8(host["q"], kh, vh, b.k_scale, b.v_scale, b.block_tables,
                                       b.context_lens, b.scale)
-        np.testing.assert_array_equal(_bits(k2), kh)
     else:
         kh, vh = oracle_caches_after_step(b, host)
         ref = oracle.paged_decode(host["q"], kh, vh, b.block_tables, b.context_lens, b.scale)
+    # the pools byte for byte against the oracle's writes, in every dtype
+    np.testing.assert_array_equal(_bits(k2), kh.view(np.uint8))
+    np.testing.assert_array_equal(_bits(v2), vh.view(np.uint8))
     check_close(out2, ref, "bf16" if dtype == "fp8" else dtype, f"fused {dtype}")
 
 
@@ -129,7 +131,12 @@ def test_bad_table_entry_is_flagged_and_not_written(cuda_device):
 
 
 def test_full_size_batch_fused_equals_separate(cuda_device):
+    """The full Llama-3-8B-shaped batch: the fused prologue and the three separate calls
+    give the same pools, slots and outputs, and both meet the oracle: the pools byte for
+    byte, the slots exactly, every output within the bf16 tolerance."""
     b = workloads.c3_llama3_8b_gqa(device=cuda_device)
+    host = b.host()
+    k_ref, v_ref = oracle_caches_after_step(b, host)
     k1, v1 = b.k_cache.clone(), b.v_cache.clone()
     out1, s1 = separate(b, k1, v1)
     k2, v2 = b.k_cache.clone(), b.v_cache.clone()
@@ -139,6 +146,12 @@ def test_full_size_batch_fused_equals_separate(cuda_device):
     assert pkv.device_error_bits() == 0
     assert torch.equal(s1, s2)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    np.testing.assert_array_equal(_bits(k2), k_ref.view(np.uint8))
+    np.testing.assert_array_equal(_bits(v2), v_ref.view(np.uint8))
+    np.testing.assert_array_equal(s2.cpu().numpy(),
+                                  oracle.slot_mapping(b.block_tables, b.new_seq, b.new_pos))
+    ref = oracle.paged_decode(host["q"], k_ref, v_ref, b.block_tables, b.context_lens, b.scale)
+    check_close(out2, ref, "bf16", "c3 fused prologue, every output")
 
 
 # ---------------------------------------------------------------- token lists

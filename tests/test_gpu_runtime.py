@@ -1,14 +1,16 @@
 """Runtime behaviour on the GPU: a plan reused for several runs (several layers'
 pools), back-to-back decodes on one stream, and the bounded-wait failure path
 (a wait that nothing completes turns into an error status, and the context
-stays usable)."""
+stays usable), and decode steps captured in CUDA graphs and replayed, checked
+against eager launches and against the oracle."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_375_b200 as pkv
 import workloads
-from gpu_util import check_close, dev_i32
+from gpu_util import check_close, dev_i32, host_bits, oracle_caches_after_step
 
 pytestmark = pytest.mark.gpu
 
@@ -64,7 +66,6 @@ def test_expired_wait_reports_timeout_and_context_survives(cuda_device):
     # the context is still usable: a decode afterwards is correct
     b = workloads.c1_tiny_fp32(device=cuda_device)
     host = b.host()
-    import oracle
     out = torch.empty_like(b.q)
     pkv.paged_attention_decode(out, b.q, b.k_cache, b.v_cache, dev_i32(b.block_tables, cuda_device),
                                dev_i32(b.context_lens, cuda_device), b.scale, b.num_kv_heads,
@@ -77,9 +78,13 @@ def test_expired_wait_reports_timeout_and_context_survives(cuda_device):
 
 def test_decode_step_captured_in_a_cuda_graph_matches_eager(cuda_device):
     """Slot indexing, reshape_and_cache, plan and decode captured once into a CUDA graph
-    and replayed give bit-identical results to eager launches."""
+    and replayed give bit-identical results to eager launches, and every replay meets
+    the tolerance against the oracle (pools byte for byte)."""
     b = workloads.random_batch(74, [5, 17, 300, 1200, 2100], 32, 8, 128, "bf16",
                                device=cuda_device, new_token=True)
+    host = b.host()
+    k_ref, v_ref = oracle_caches_after_step(b, host)
+    ref = oracle.paged_decode(host["q"], k_ref, v_ref, b.block_tables, b.context_lens, b.scale)
     bt = dev_i32(b.block_tables, cuda_device)
     cl = dev_i32(b.context_lens, cuda_device)
     mcl = b.max_context_len
@@ -115,14 +120,21 @@ def test_decode_step_captured_in_a_cuda_graph_matches_eager(cuda_device):
         g.replay()
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+        check_close(out, ref, "bf16", "graph replay")
     assert pkv.device_error_bits() == 0
+    assert np.array_equal(host_bits(b.k_cache), k_ref)
+    assert np.array_equal(host_bits(b.v_cache), v_ref)
 
 
 def test_shared_prefix_step_in_a_cuda_graph(cuda_device):
     """The shared-prefix step (copy-on-write, new tokens, shared plan, decode, merge)
-    captured once and replayed gives bit-identical results to eager launches."""
+    captured once and replayed gives bit-identical results to eager launches, and every
+    replay meets the tolerance against the oracle."""
     b = workloads.c4_shared_prefix(device=cuda_device, prompts=3, samples=5, prefix=300,
                                    max_tail=60, num_blocks=500)
+    host = b.host()
+    k_ref, v_ref = oracle_caches_after_step(b, host)
+    ref = oracle.paged_decode(host["q"], k_ref, v_ref, b.block_tables, b.context_lens, b.scale)
     dev = cuda_device
     bt = dev_i32(b.block_tables, dev)
     cl = dev_i32(b.context_lens, dev)
@@ -163,4 +175,5 @@ def test_shared_prefix_step_in_a_cuda_graph(cuda_device):
         g.replay()
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+        check_close(out, ref, "bf16", "shared-prefix graph replay")
     assert pkv.device_error_bits() == 0

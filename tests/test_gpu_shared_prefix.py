@@ -232,30 +232,6 @@ def test_shared_prefix_workload_small(cuda_device):
     check_close(out, ref, "bf16", "c4 small")
 
 
-def test_shared_prefix_workload_full_size_sampled(cuda_device):
-    """The full parallel-sampling batch (32 prompts x 8 samples) in the launch configuration
-    the benchmark times: sampled outputs recomputed by the oracle one by one."""
-    from gpu_util import compact_for_tasks, host_bits, sample_tasks
-    b = workloads.c4_shared_prefix(device=cuda_device)
-    gpu_step(b)   # copy-on-write and the tails' writes (and a plain decode)
-    dev = b.q.device
-    out = torch.empty_like(b.q)
-    gs = np.asarray(b.meta["group_start"], dtype=np.int32)
-    sb = np.asarray(b.meta["shared_blocks"], dtype=np.int32)
-    pkv.paged_attention_decode_shared(out, b.q, b.k_cache, b.v_cache,
-                                      dev_i32(b.block_tables, dev), dev_i32(b.context_lens, dev),
-                                      dev_i32(gs, dev), dev_i32(sb, dev), b.scale,
-                                      max_context_len=b.max_context_len)
-    assert pkv.device_error_bits() == 0
-    tasks = sample_tasks(b, 48, seed=4)
-    kh, vh, bt = compact_for_tasks(b, b.k_cache, b.v_cache, tasks)
-    ref = oracle.paged_decode(host_bits(b.q), kh, vh, bt, b.context_lens, b.scale, tasks=tasks,
-                              threads=4)
-    got = out[torch.from_numpy(tasks[:, 0]).long(), torch.from_numpy(tasks[:, 1]).long()]
-    check_close(got, ref, "bf16", "c4 full size, shared prefix")
-    assert torch.isfinite(out).all()
-
-
 def test_block_manager_groups_drive_the_shared_decode(cuda_device):
     """Forks and prefix caching in the host block manager, its tables, slots and groups,
     then the KV written through reshape_and_cache (copies first) and the shared decode,

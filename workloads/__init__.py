@@ -40,7 +40,8 @@ CONFIGS = {
                         "[16,8192], reshape_and_cache of the new token before attention",
     "c4_shared_prefix": "parallel sampling bf16 GQA 32q/8kv d128: 32 prompts x 8 samples sharing 1024+r prefix "
                         "tokens, tails U[0,512], copy-on-write via copy_blocks, then decode",
-    "c5_long_splitk": "long context bf16 GQA 64q/8kv d128: batch 8, lens U[32768,131072], 512-token partitions",
+    "c5_long_splitk": "long context bf16 GQA 64q/8kv d128: batch 8, lens U[32768,131072], split-K partitions "
+                      "merged by log-sum-exp (512 tokens as configured; the automatic size is 4096)",
 }
 CONFIG_SEEDS = {name: i + 1 for i, name in enumerate(CONFIGS)}
 
