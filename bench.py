@@ -47,8 +47,14 @@ METRIC = "paged decode attn: KV-read GB/s (% of B200 HBM peak), seqs/s at batch"
 UNIT = "GB/s"
 WORKLOADS = {"c3": "c3_llama3_8b_gqa", "c2": "c2_llama2_13b_mha", "c4": "c4_shared_prefix",
              "c5": "c5_long_splitk", "c1": "c1_tiny_fp32", "c3spec": "c3_spec_decode",
-             "c3fp8": "c3_fp8", "c3specfp8": "c3_spec_fp8", "c3e5m2": "c3_fp8e5m2"}
+             "c3fp8": "c3_fp8", "c3specfp8": "c3_spec_fp8", "c3e5m2": "c3_fp8e5m2",
+             "c3prefill": "c3_prefill"}
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0            # burst; about 1400 sustained under the power cap
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+# Chunks with more query rows per kv head than this run on the tcgen05 prefill kernel
+# (128-row query tiles); shorter ones on the decode kernel (at most 16 rows per item).
+PREFILL_MIN_ROWS = 64
 L2_BYTES = 126 << 20       # B200 L2; working sets below 4x this are flushed between steps
 DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")  # JSON text
@@ -62,6 +68,32 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """(burst, sustained, kind) dense bf16 TFLOP/s of this machine's B200s."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        burst = float(d["bf16_tflops"])
+        return burst, float(d.get("bf16_tflops_sustained", burst)), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+
+
+def attention_flops(b: workloads.Batch) -> int:
+    """Multiply-adds x 2 of S = q K^T and O = P V over the keys each query row can see:
+    4 * head_dim per (query row, query head, visible key); chunk token i of an n-token
+    chunk sees L - n + i + 1 keys."""
+    lens = b.context_lens.astype(np.int64)
+    if b.query_start_loc is None:
+        visible = int(lens.sum())
+    else:
+        n = np.diff(b.query_start_loc).astype(np.int64)
+        # sum over i < n of (L - n + i + 1) = n (L - n) + n (n + 1) / 2
+        visible = int((n * (lens - n) + n * (n + 1) // 2).sum())
+    return 4 * b.head_dim * b.num_q_heads * visible
 
 
 def decode_source_hash() -> str:
@@ -202,7 +234,7 @@ class Step:
     """The hot path over one batch through the public API (device-resident inputs)."""
 
     def __init__(self, b: workloads.Batch, partition_tokens: int, shared_prefix: bool = True,
-                 token_prologue: bool = False):
+                 token_prologue: bool = False, multi_kernel: str = "auto"):
         import paged_kv_cache_375_b200 as pkv
         self.pkv, self.b = pkv, b
         dev = b.q.device
@@ -223,6 +255,13 @@ class Step:
             self.shared_blocks = torch.tensor(b.meta["shared_blocks"], dtype=torch.int32,
                                               device=dev)
             self.split = True                           # prefix and own partials are merged
+        # long chunks (chunked prefill) on the tcgen05 kernel, short ones on the decode kernel
+        g = b.num_q_heads // b.num_kv_heads
+        self.prefill = self.multi and b.dtype == "bf16" and (
+            multi_kernel == "prefill" or
+            (multi_kernel == "auto" and b.max_query_len * g > PREFILL_MIN_ROWS))
+        if self.prefill:
+            self.split = False
         if self.multi:
             self.qsl = torch.from_numpy(b.query_start_loc).to(dev)
             ws = pkv.load_library().pkv_multi_workspace_bytes(
@@ -246,12 +285,14 @@ class Step:
         # any other short list of new tokens (a few per sequence): written in the same
         # launch as the plan.  A long list (the parallel-sampling tails) keeps
         # reshape_and_cache, whose many small CTAs stream the rows at the copy bandwidth.
-        self.fused_tokens = (self.T > 0 and not self.fused
+        self.fused_tokens = (self.T > 0 and not self.fused and not self.prefill
                              and (token_prologue or self.T <= TOKEN_PROLOGUE_MAX))
         if self.pairs is not None:
             pkv.validate_copy_pairs(torch.from_numpy(b.cow_pairs), b.num_blocks)
 
     def launches_per_step(self) -> int:
+        if self.prefill:                               # slots, reshape, prefill
+            return 1 + (2 if self.T else 0)
         n = 2 + (1 if self.split else 0)              # plan or prologue, decode (, merge)
         n += 2 if self.T and not (self.fused or self.fused_tokens) else 0  # slots, reshape
         n += 1 if self.pairs is not None else 0        # copy_blocks
@@ -281,6 +322,8 @@ class Step:
 
     def plan(self):
         b = self.b
+        if self.prefill:
+            return                                     # the prefill kernel needs no plan
         extra = {}
         if self.fused or self.fused_tokens:
             # one launch: the new tokens' slots and writes, and the plan
@@ -300,7 +343,11 @@ class Step:
                                             workspace_tensor=self.ws, **extra)
 
     def decode(self):
-        if self.multi and workloads.fp8_format(self.b.dtype):
+        if self.prefill:
+            b = self.b
+            self.pkv.paged_prefill(self.out, b.q, b.k_cache, b.v_cache, self.bt, self.cl,
+                                   self.qsl, b.scale, b.num_kv_heads, max_context_len=self.mcl)
+        elif self.multi and workloads.fp8_format(self.b.dtype):
             self.plan_obj.run_multi_fp8(self.out, self.b.q, self.b.k_cache, self.b.v_cache,
                                         self.qsl, self.b.max_query_len, self.b.scale,
                                         self.b.k_scale, self.b.v_scale)
@@ -330,7 +377,7 @@ def run_ours(args, world, rank, local):
     b = (workloads.BUILDERS[name](device=dev, num_seqs=args.batch) if args.batch else
          workloads.BUILDERS[name](device=dev))
     step = Step(b, args.partition, shared_prefix=not args.no_shared_prefix,
-                token_prologue=args.token_prologue)
+                token_prologue=args.token_prologue, multi_kernel=args.multi_kernel)
     alg = algorithmic_bytes(b)
     kv_bytes = b.kv_bytes() if name != "c4_shared_prefix" else b.unique_kv_bytes()
     stream = torch.cuda.current_stream(dev)
@@ -459,14 +506,7 @@ def run_ours(args, world, rank, local):
                               "region bracketed by events (in the timed region, every 8th "
                               "step's decode is bracketed too: decode_ms_in_region_mean); "
                               "other ops: each timed alone (50 launches) after the timed region"},
-        "roofline": {
-            "kernel": "decode_kernel" + (" + merge_kernel" if step.split else ""),
-            "bound": "hbm", "achieved": round(alg["total"] / (decode_ms / 1e3) / 1e9, 2),
-            "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)",
-            "unit": "GB/s", "frac": round(alg["total"] / (decode_ms / 1e3) / 1e9 / peak, 4),
-            "traffic": recorded_traffic(args.workload),
-            "algorithmic_bytes_per_launch": alg,
-        },
+        "roofline": roofline(step, alg, decode_ms, peak, peak_kind, args.workload),
         "gpu_launches": step.launches_per_step() * K,
         "clocks": sampler.summary(),
     }
@@ -477,6 +517,32 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
     return result
+
+
+def roofline(step: Step, alg: dict, decode_ms: float, peak: float, peak_kind: str,
+             workload: str) -> dict:
+    """The dominant kernel against its roofline: HBM for decode (algorithmic bytes per
+    launch / launch time), the bf16 tensor cores for the prefill kernel (attention
+    flops per launch / launch time; its HBM bytes reported beside)."""
+    gbs = alg["total"] / (decode_ms / 1e3) / 1e9
+    if step.prefill:
+        burst, sustained, kind = tensor_peak()
+        flops = attention_flops(step.b)
+        tf = flops / (decode_ms / 1e3) / 1e12
+        return {"kernel": "prefill_kernel (tcgen05, TMEM accumulators)", "bound": "tensor",
+                "achieved": round(tf, 2), "peak": burst,
+                "peak_kind": f"{kind} bf16_tflops (dense, burst)", "unit": "TFLOP/s",
+                "frac": round(tf / burst, 4), "frac_of_sustained": round(tf / sustained, 4),
+                "peak_sustained": sustained, "traffic": recorded_traffic(workload),
+                "algorithmic_flops_per_launch": flops,
+                "hbm": {"achieved_GBps": round(gbs, 2), "peak": peak,
+                        "frac": round(gbs / peak, 4)},
+                "algorithmic_bytes_per_launch": alg}
+    return {"kernel": "decode_kernel" + (" + merge_kernel" if step.split else ""),
+            "bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
+            "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)", "unit": "GB/s",
+            "frac": round(gbs / peak, 4), "traffic": recorded_traffic(workload),
+            "algorithmic_bytes_per_launch": alg}
 
 
 def plan_items(step: Step) -> int:
@@ -538,7 +604,7 @@ def breakdown(step: Step, stream, dev, n: int = 50) -> dict:
         pkv.DecodePlan(step.bt, step.cl, b.num_q_heads, b.k_cache, max_context_len=step.mcl,
                        partition_tokens=step.partition, workspace_tensor=step.ws)
 
-    ops = {"plan": plan_only}
+    ops = {} if step.prefill else {"plan": plan_only}
     if step.fused or step.fused_tokens:
         ops["decode_prologue"] = step.plan
     if step.T:
@@ -809,6 +875,10 @@ def main(argv=None):
     ap.add_argument("--token-prologue", action="store_true",
                     help="write any number of new tokens in the plan's launch (by default only "
                          f"up to {TOKEN_PROLOGUE_MAX} a step)")
+    ap.add_argument("--multi-kernel", choices=["auto", "prefill", "decode"], default="auto",
+                    help="several query tokens per sequence: the tcgen05 prefill kernel "
+                         f"(auto: chunks of more than {PREFILL_MIN_ROWS} rows per kv head) or "
+                         "the decode kernel's row groups")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--batch", type=int, default=0,
                     help="number of sequences (0 = the workload's own); a smaller batch of the "

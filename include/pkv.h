@@ -203,6 +203,32 @@ pkv_status pkv_paged_attention_multi(void *out, const void *q, const void *k_cac
                                      size_t workspace_bytes, void *cuda_stream);
 
 /*
+ * The same operation as pkv_paged_attention_multi, for long chunks (chunked
+ * prefill: vampireachao.github.io "vllm", section "第二层：请求不该排队等整批";
+ * the flattened layout of the "vLLM" wiki entry, section "Flattened 布局与
+ * slot_mapping"): chunk token i of sequence s, at position L - n + i of its
+ * context, attends to keys 0 .. L - n + i found block by block through the
+ * table.  Runs on the tcgen05 tensor cores with the accumulators in tensor
+ * memory: a work unit is 128 query rows (floor(128/g) chunk tokens times the
+ * g query heads of one kv head), and every 128-key tile of K and V is read
+ * once per unit.  For chunks of a few tokens the decode kernel behind
+ * pkv_paged_attention_multi is the better fit.
+ *  - bf16 pools only (PKV_ERR_UNSUPPORTED otherwise); head_dim 64 or 128;
+ *    Hq/Hkv at most 16; at most 2048 sequences a call.
+ *  - q, out: bf16 [num_q_tokens][Hq][D]; query_start_loc int32 [B+1] (device).
+ *  - No workspace, no split-K: the call allocates nothing and needs none.
+ *  - Device-side errors as for the multi call: a chunk longer than its
+ *    context or outside [0, num_q_tokens) is skipped and flags
+ *    PKV_DEVERR_LEN; a length past the table or max_context_len is clamped
+ *    and flagged PKV_DEVERR_LEN; a table entry outside [0, num_blocks) is
+ *    read as block 0 and flags PKV_DEVERR_BLOCK.
+ */
+pkv_status pkv_paged_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, const int32_t *context_lens,
+                             const int32_t *query_start_loc, int32_t num_q_tokens, float scale,
+                             const pkv_dims *dims, int32_t max_context_len, void *cuda_stream);
+
+/*
  * The run half of pkv_paged_attention_multi, over a plan made by
  * pkv_decode_plan (the plan depends only on the context lengths); the same
  * rules as pkv_decode_run apply, with the workspace sized by

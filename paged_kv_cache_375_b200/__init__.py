@@ -94,6 +94,7 @@ def load_library() -> ctypes.CDLL:
             "pkv_paged_attention_multi": (ctypes.c_int, [P, P, P, P, P, P, P, i32, i32, f32, D,
                                                          i32, i32, P, sz, P]),
             "pkv_decode_run": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P, sz, P]),
+            "pkv_paged_prefill": (ctypes.c_int, [P, P, P, P, P, P, P, i32, f32, D, i32, P]),
             "pkv_reshape_and_cache": (ctypes.c_int, [P, P, P, P, P, i32, D, P]),
             "pkv_reshape_and_cache_fp8": (ctypes.c_int, [P, P, P, P, P, i32, f32, f32, D, P]),
             "pkv_paged_attention_decode_fp8": (ctypes.c_int, [P, P, P, P, P, P, f32, f32, f32, D,
@@ -313,6 +314,38 @@ def paged_attention_multi(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Ten
         _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
         _p(query_start_loc), T, int(max_query_len), float(scale), ctypes.byref(dims), mcl,
         partition_tokens, _p(ws), ws.numel(), _stream_ptr(dev)))
+    return out
+
+
+def paged_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                  v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+                  query_start_loc: torch.Tensor, scale: float, num_kv_heads: int, *,
+                  max_context_len: int | None = None) -> torch.Tensor:
+    """The same causal attention as paged_attention_multi, on the tcgen05 tensor cores
+    with 128-row query tiles: for long chunks (chunked prefill, whole prompts).
+
+    bf16 only; q, out: [T][Hq][D]; query_start_loc: int32 [B+1].  Needs no workspace.
+    """
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, dev)
+    _need(block_tables, "block_tables", torch.int32, dev)
+    _need(context_lens, "context_lens", torch.int32, dev)
+    _need(query_start_loc, "query_start_loc", torch.int32, dev)
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape or k_cache.shape[1] != num_kv_heads:
+        raise ValueError("k_cache and v_cache must be [num_blocks][num_kv_heads][16][head_dim]")
+    T, hq, d = q.shape
+    B = context_lens.shape[0]
+    if out.shape != q.shape or query_start_loc.shape != (B + 1,) or block_tables.shape[0] != B \
+            or k_cache.shape[3] != d:
+        raise ValueError("inconsistent shapes")
+    dims = make_dims(B, hq, k_cache, block_tables.shape[1])
+    mcl = block_tables.shape[1] * k_cache.shape[2] if max_context_len is None else int(max_context_len)
+    _check(load_library().pkv_paged_prefill(
+        _p(out), _p(q), _p(k_cache), _p(v_cache), _p(block_tables), _p(context_lens),
+        _p(query_start_loc), T, float(scale), ctypes.byref(dims), mcl, _stream_ptr(dev)))
     return out
 
 

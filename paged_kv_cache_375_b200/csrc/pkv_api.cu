@@ -16,6 +16,7 @@
 #include "pkv_cache_ops.cuh"
 #include "pkv_decode.cuh"
 #include "pkv_device.cuh"
+#include "pkv_prefill.cuh"
 #include "pkv_prepare.cuh"
 
 namespace {
@@ -816,6 +817,48 @@ pkv_status shared_one_shot(void* out, const void* q, const void* k_cache, const 
 
 }  // namespace
 
+namespace {
+
+// A 3-D view of q [num_q_tokens][Hq][D] (bf16) for the prefill kernel: the box
+// is {64 columns, the g heads of one kv head, tokens_per_tile tokens}, so one
+// load brings the tile's 128 query rows (token-major, head-minor) of one
+// 128-byte column half, 128-byte swizzled.
+pkv_status encode_q_map(CUtensorMap* map, const void* q, int32_t num_q_tokens, const pkv_dims* d,
+                        int group, int tokens_per_tile) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d->head_dim),
+                        static_cast<cuuint64_t>(d->num_q_heads),
+                        static_cast<cuuint64_t>(num_q_tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d->head_dim) * 2,
+                           static_cast<cuuint64_t>(d->num_q_heads) * d->head_dim * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(group),
+                       static_cast<cuuint32_t>(tokens_per_tile)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (q) failed (%d)", (int)r);
+  return PKV_OK;
+}
+
+template <int D>
+pkv_status launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const pkv::PrefillParams& prm, int64_t units_bound,
+                          cudaStream_t stream) {
+  auto kern = pkv::prefill_kernel<D>;
+  constexpr int smem = pkv::PfLayout<D>::kTotal;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+  const int64_t sms = device_sm_count();
+  const int grid = static_cast<int>(units_bound < sms ? units_bound : sms);
+  e = launch(kern, dim3(grid), dim3(pkv::kPfThreads), smem, stream, mq, mk, mv, prm);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return PKV_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t pkv_decode_partition_tokens(const pkv_dims* dims, int32_t max_context_len,
@@ -1143,6 +1186,56 @@ pkv_status pkv_reshape_and_cache_fp8(const void* k, const void* v, void* k_cache
                          k_scale, v_scale);
   if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache_fp8 launch");
   return PKV_OK;
+}
+
+pkv_status pkv_paged_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             const int32_t* query_start_loc, int32_t num_q_tokens, float scale,
+                             const pkv_dims* dims, int32_t max_context_len, void* cuda_stream) {
+  pkv_status st = check_dims(dims, true);
+  if (st != PKV_OK) return st;
+  if (dims->dtype != PKV_BF16)
+    return fail(PKV_ERR_UNSUPPORTED, "pkv_paged_prefill runs on bf16 pools only");
+  if (dims->num_seqs > pkv::kPfMaxSeqs)
+    return fail(PKV_ERR_UNSUPPORTED, "pkv_paged_prefill takes at most %d sequences a call",
+                pkv::kPfMaxSeqs);
+  if (num_q_tokens < 0 || max_context_len < 0)
+    return fail(PKV_ERR_SHAPE, "num_q_tokens and max_context_len must be >= 0");
+  if (dims->num_seqs == 0 || num_q_tokens == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
+    return fail(PKV_ERR_NULL, "a tensor pointer is NULL");
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(PKV_ERR_ALIGN, "out, q and the caches must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(PKV_ERR_SHAPE, "scale must be finite");
+  if ((st = bind_device(out, "out")) != PKV_OK) return st;
+  const int group = dims->num_q_heads / dims->num_kv_heads;
+  const int tpt = pkv::kPfRows / group;
+  CUtensorMap mq, mk, mv;
+  if ((st = encode_q_map(&mq, q, num_q_tokens, dims, group, tpt)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&mk, k_cache, dims)) != PKV_OK) return st;
+  if ((st = encode_pool_map(&mv, v_cache, dims)) != PKV_OK) return st;
+  const int64_t table_len = static_cast<int64_t>(dims->max_blocks_per_seq) * pkv::kBlock;
+  pkv::PrefillParams prm;
+  prm.out = out;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.query_start_loc = query_start_loc;
+  prm.num_seqs = dims->num_seqs;
+  prm.num_q_tokens = num_q_tokens;
+  prm.num_q_heads = dims->num_q_heads;
+  prm.num_kv_heads = dims->num_kv_heads;
+  prm.group = group;
+  prm.tokens_per_tile = tpt;
+  prm.max_blocks_per_seq = dims->max_blocks_per_seq;
+  prm.num_blocks = dims->num_blocks;
+  prm.max_len = static_cast<int32_t>(max_context_len < table_len ? max_context_len : table_len);
+  prm.qk_scale_log2 = scale * pkv::kLog2e;
+  // tiles of all chunks together: at most ceil(T / tpt) + B
+  const int64_t units_bound =
+      (static_cast<int64_t>(num_q_tokens + tpt - 1) / tpt + dims->num_seqs) * dims->num_kv_heads;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  return dims->head_dim == 128 ? launch_prefill<128>(mq, mk, mv, prm, units_bound, stream)
+                               : launch_prefill<64>(mq, mk, mv, prm, units_bound, stream);
 }
 
 pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_cache,

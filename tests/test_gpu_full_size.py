@@ -5,7 +5,9 @@ Each case builds the workload at its full size, runs one step through the
 benchmark's own ``Step`` (the fused decode prologue for one new token per
 sequence; the token prologue for draft verification; copy_blocks, slot
 indexing and reshape_and_cache before the shared-prefix plan for parallel
-sampling; the decode and, where sequences are split, the log-sum-exp merge),
+sampling; the decode and, where sequences are split, the log-sum-exp merge;
+slot indexing, reshape_and_cache and the tcgen05 prefill kernel for the
+chunked-prefill step),
 then runs the oracle's pass over the same step on all host cores.  Both pools
 must equal the oracle's byte for byte (copy-on-write copies, the new tokens'
 writes, FP8 quantisation), and every output row must meet the tolerance: max
@@ -29,7 +31,7 @@ from gpu_util import check_close, host_bits
 pytestmark = pytest.mark.gpu
 
 CASES = [("c2", 0), ("c3", 0), ("c3", 512), ("c4", 0), ("c5", 0), ("c5", 512), ("c3fp8", 0),
-         ("c3e5m2", 0), ("c3spec", 0), ("c3specfp8", 0)]
+         ("c3e5m2", 0), ("c3spec", 0), ("c3specfp8", 0), ("c3prefill", 0)]
 
 
 @pytest.mark.parametrize("workload,partition", CASES)
@@ -40,6 +42,7 @@ def test_bench_step_every_output(cuda_device, workload, partition):
     step = bench.Step(b, partition)
     if partition:
         assert step.part_tokens == partition and step.split
+    assert step.prefill == (workload == "c3prefill")     # long chunks: the tcgen05 kernel
     step()
     torch.cuda.synchronize(cuda_device)
     assert pkv.device_error_bits(cuda_device) == 0

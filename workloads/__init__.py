@@ -482,6 +482,26 @@ def c3_spec_fp8(device="cpu", num_seqs: int = 256, draft: int = 4) -> Batch:
     return c3_spec_decode(device, num_seqs, draft, "fp8")
 
 
+def c3_prefill(device="cpu", num_seqs: int = 16, chunk: int = 1024,
+               max_cached: int = 3072) -> Batch:
+    """A chunked-prefill step of the Llama-3-8B-shaped model (32 q / 8 kv heads, d128,
+    bf16): each of `num_seqs` prompts processes its next `chunk` tokens over a cached
+    prefix of U[0, max_cached] tokens (multiples of 16 tokens: earlier chunks filled
+    whole blocks), so the chunk is the last `chunk` positions of a context of
+    prefix + chunk tokens; the chunk's K/V are written by reshape_and_cache, then every
+    chunk token attends causally."""
+    seed = CONFIG_SEEDS["c3_llama3_8b_gqa"] + 200
+    rng = np.random.default_rng(seed)
+    cached = rng.integers(0, max_cached // BLOCK_SIZE, size=num_seqs, endpoint=True) * BLOCK_SIZE
+    lens = cached + chunk
+    need = int(sum((int(L) + BLOCK_SIZE - 1) // BLOCK_SIZE for L in lens))
+    b = chunked_batch(seed, lens, np.full(num_seqs, chunk), 32, 8, 128, "bf16",
+                      num_blocks=max(4096, int(math.ceil(1.25 * need))), device=device,
+                      name="c3_prefill")
+    b.meta["chunk"] = chunk
+    return b
+
+
 def c4_shared_prefix(device="cpu", prompts: int = 32, samples: int = 8, prefix: int = 1024,
                      max_tail: int = 512, num_blocks: int | None = None) -> Batch:
     """Parallel sampling with a shared prefix.
@@ -548,6 +568,8 @@ def c5_long_splitk(device="cpu", num_seqs: int = 8) -> Batch:
                         device=device, name="c5_long_splitk")
 
 
+CONFIGS["c3_prefill"] = ("chunked prefill, Llama-3-8B-shaped GQA bf16 (32q/8kv, d128): 16 prompts x "
+                          "1024-token chunks over cached prefixes U[0, 3072] (causal)")
 CONFIGS["c3_spec_decode"] = ("Llama-3-8B-shaped GQA bf16, batch 256, verifying 4 speculative tokens "
                               "per sequence (causal, 16 query rows per kv head)")
 CONFIGS["c3_spec_fp8"] = ("the speculative-verification batch (256 x 4 draft tokens, causal) over FP8 "
@@ -561,6 +583,7 @@ CONFIGS["c3_fp8"] = ("Llama-3-8B-shaped GQA over FP8 e4m3 pools (one scale per p
 BUILDERS = {
     "c1_tiny_fp32": c1_tiny_fp32,
     "c3_spec_decode": c3_spec_decode,
+    "c3_prefill": c3_prefill,
     "c3_fp8": c3_fp8,
     "c3_spec_fp8": c3_spec_fp8,
     "c3_fp8e5m2": c3_fp8e5m2,
