@@ -15,6 +15,7 @@
 #include "pkv.h"
 #include "pkv_cache_ops.cuh"
 #include "pkv_decode.cuh"
+#include "pkv_decode_warp.cuh"
 #include "pkv_device.cuh"
 #include "pkv_prefill.cuh"
 #include "pkv_prepare.cuh"
@@ -335,6 +336,28 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
   return PKV_OK;
 }
 
+// Short items (split-K partitions of at most kWarpItemMaxBlocks blocks, the
+// shared-prefix plan) of bf16 head_dim-128 decode: one warp per item, eight
+// warps per CTA, 3 tile stages each for up to 8 query rows, 2 for 16.
+template <int GMAX>
+pkv_status launch_decode_warp(const CUtensorMap& mk, const CUtensorMap& mv,
+                              const pkv::DecodeParams& prm, int64_t work_units,
+                              cudaStream_t stream) {
+  constexpr int W = 8, S = GMAX <= 8 ? 3 : 2;
+  using Lay = pkv::WarpDecodeLayout<GMAX, W, S>;
+  auto kern = pkv::decode_warp_kernel<GMAX, W, S>;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), Lay::kTotal);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_warp)");
+  int64_t grid = device_sm_count();
+  const int64_t need = (work_units + W - 1) / W;
+  if (grid > need) grid = need;
+  if (grid < 1) grid = 1;
+  e = launch(kern, dim3(static_cast<unsigned>(grid)), dim3(W * 32), Lay::kTotal, stream, mk, mv,
+             prm);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_warp launch");
+  return PKV_OK;
+}
+
 // The query rows of an item (chunk length x group) go on the MMA's N side:
 // up to 8 or up to 16 rows.
 template <typename T, int D>
@@ -511,6 +534,13 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_FP8_E5M2) {
     st = launch_decode_d<pkv::Fp8E5m2Kv, 128>(mk, mv, prm, units, rows_max, stream);
+  } else if (d->dtype == PKV_BF16 && d->head_dim == 128 &&
+             (!query_start_loc || max_query_len == 1) &&
+             rows_max <= 16 && plan.part_blocks <= pkv::kWarpItemMaxBlocks &&
+             (plan.max_parts > 1 || plan.shared)) {
+    // short items: a warp per item, no merge across warps
+    st = rows_max <= 8 ? launch_decode_warp<8>(mk, mv, prm, units, stream)
+                       : launch_decode_warp<16>(mk, mv, prm, units, stream);
   } else if (d->dtype == PKV_BF16) {
     st = d->head_dim == 128
              ? launch_decode_d<__nv_bfloat16, 128>(mk, mv, prm, units, rows_max, stream)

@@ -19,22 +19,27 @@
 //   O += P V     (M 128 rows, N = head_dim, K = 128 keys) into TMEM
 //
 // Roles in a CTA of 8 warps (one CTA per SM, persistent over work units):
-//  * warp 0, one lane: TMA producer.  Loads the unit's Q tile (a 3-D tensor
-//    map over q [T][Hq][D], box {64 d, g heads, tokens}) and, per KV tile of
-//    128 keys, the tile's 8 blocks of K and of V through the block table (the
-//    2-D pool map, one box per block and 64-column half), into 128-byte
-//    swizzled stages laid out [half][128 keys][128 B].
+//  * warp 0, two lanes: TMA producers.  Lane 0 loads the unit's Q tile (a 3-D
+//    tensor map over q [T][Hq][D], box {64 d, g heads, tokens}) and, per KV
+//    tile of 128 keys, the tile's 8 blocks of K through the block table (the
+//    2-D pool map, one box per block and 64-column half); lane 1 does the same
+//    for V.  Stages are 128-byte swizzled, laid out [half][128 keys][128 B]; a
+//    K stage is released when its scores are computed, a V stage when its
+//    P V is.
 //  * warp 1: TMEM allocation; one lane issues the MMAs and commits them to
 //    mbarriers; the warp zeroes the value rows past the context in the last
 //    block of the context (NaN padding times a zero weight is still NaN on a
 //    tensor core).
-//  * warps 4-7 (a warpgroup; warp w reads TMEM lanes 32(w-4) ...): softmax.
-//    Thread r owns query row r: it reads its 128 scores from TMEM, masks keys
-//    past its causal limit, keeps a running maximum in log2 units that moves
-//    only when it grows by more than 8 (the output row in TMEM is rescaled
-//    then), writes P in bf16 into shared memory (the A operand of P V) and
-//    sums the rounded weights.  At the end it reads its output row from TMEM,
-//    divides by the sum and stores bf16.
+//  * warps 4-11 (two warpgroups; warp w reads TMEM lanes 32(w%4) ...): softmax.
+//    Query row r belongs to one thread of each warpgroup, which take keys 0-63
+//    and 64-127 of every tile.  Each reads its 64 scores from TMEM, masks keys
+//    past the row's causal limit, swaps its maximum with its partner through
+//    shared memory, keeps a running maximum in log2 units that moves only when
+//    it grows by more than 8 (the output row in TMEM is then rescaled, each
+//    thread its half of the columns), writes its half of P in bf16 into shared
+//    memory (the A operand of P V) and sums its weights.  At the end the two
+//    sums are added, and each thread reads its half of the output row from
+//    TMEM, divides by the sum and stores bf16.
 // S is double-buffered in TMEM, so the MMA of the next tile's scores runs
 // while the softmax works on this tile's.
 #pragma once
@@ -47,7 +52,8 @@ constexpr int kPfRows = 128;       // query rows per tile: the MMA's M
 constexpr int kPfKeys = 128;       // keys per KV tile: N of S = Q K^T, K of O += P V
 constexpr int kPfBlocksPerTile = kPfKeys / kBlock;
 constexpr int kPfStages = 2;       // KV tile stages
-constexpr int kPfThreads = 256;    // warp 0 producer, warp 1 MMA, warps 4-7 softmax
+constexpr int kPfThreads = 384;    // warp 0 producers, warp 1 MMA, warps 4-11 softmax
+constexpr int kPfSoftmaxWarps = 8;  // two warpgroups: keys 0-63 and 64-127 of every row
 constexpr int kPfMaxSeqs = 2048;   // sequences per call (per-CTA tile prefix in shared memory)
 constexpr uint32_t kPfTmemCols = 512;  // S buffers at columns 0 and 128, O at 256
 constexpr float kPfRescaleSlack = 8.f; // the running max moves when it grows by more (log2)
@@ -76,11 +82,14 @@ struct PfLayout {
   static constexpr int kVOff = kKOff + kPfStages * kKvBytes;
   static constexpr int kPrefixOff = kVOff + kPfStages * kKvBytes;
   static constexpr int kBarsOff = kPrefixOff + (kPfMaxSeqs + 8) * 4;
-  // q_full, q_empty, k_full[S], v_full[S], kv_empty[S], s_full[2], s_free[2], p_full,
-  // o_done, final
-  static constexpr int kNumBars = 2 + 3 * kPfStages + 4 + 3;
+  // q_full, q_empty, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], s_free[2],
+  // p_full, o_done, final, xchg[4] (the two softmax warps of each row quarter)
+  static constexpr int kNumBars = 2 + 4 * kPfStages + 4 + 3 + 4;
   static constexpr int kMiscOff = kBarsOff + kNumBars * 8;     // tmem base, abort flag
-  static constexpr int kTotal = kMiscOff + 16 + 1024;          // + alignment slack
+  // row maxima exchanged between the two softmax warpgroups: [parity][half][row],
+  // then the row sums [half][row]
+  static constexpr int kXchgOff = kMiscOff + 16;
+  static constexpr int kTotal = kXchgOff + (4 + 2) * kPfRows * 4 + 1024;  // + alignment slack
 };
 
 // ------------------------------------------------------------ tcgen05 helpers
@@ -136,6 +145,20 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, float (&v)[32]) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane, loaded and waited
+// for in one statement.
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // 128 consecutive fp32 columns of this thread's TMEM lane, loaded and waited
@@ -294,12 +317,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
   uint64_t* v_full = k_full + kPfStages;
-  uint64_t* kv_empty = v_full + kPfStages;
-  uint64_t* s_full = kv_empty + kPfStages;
+  uint64_t* k_empty = v_full + kPfStages;
+  uint64_t* v_empty = k_empty + kPfStages;
+  uint64_t* s_full = v_empty + kPfStages;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_done = p_full + 1;
   uint64_t* fin = o_done + 1;
+  uint64_t* xchg = fin + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::kMiscOff);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -310,15 +335,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int i = 0; i < kPfStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], kPfSoftmaxWarps);
     }
-    mbar_init(p_full, 4);
+    mbar_init(p_full, kPfSoftmaxWarps);
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&xchg[i], 2);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -368,25 +395,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t qrow_bytes = 128u * static_cast<uint32_t>(g * p.tokens_per_tile);
 
   if (warp == 0) {
-    // ===================================================== TMA producer
-    if (lane == 0) {
-      prefetch_tensormap(&map_q);
-      prefetch_tensormap(&map_k);
-      prefetch_tensormap(&map_v);
+    // ===================================================== TMA producers
+    // Lane 0 loads Q and the K tiles, lane 1 the V tiles: a K stage is free
+    // once the tile's scores are computed, a V stage only once its P V is,
+    // so the next K tiles are not held up behind the current P V.
+    if (lane < 2) {
+      const bool is_k = lane == 0;
+      const CUtensorMap* map = is_k ? &map_k : &map_v;
+      uint8_t* stage_base = is_k ? sK : sV;
+      uint64_t* full_bar = is_k ? k_full : v_full;
+      uint64_t* empty_bar = is_k ? k_empty : v_empty;
+      if (is_k) prefetch_tensormap(&map_q);
+      prefetch_tensormap(map);
       uint32_t qc = 0, kvc = 0;
       bool ok = true;
       for (int32_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const PfUnit w = pf_unit(p, prefix, u);
-        if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(q_full, qrow_bytes * H);
-#pragma unroll
-        for (int h = 0; h < H; ++h)
-          tma_load_3d(sQ + h * (kPfRows * 128), &map_q, h * 64, w.kv_head * g, w.q_row0, q_full);
-        ++qc;
         const int32_t* table = p.block_tables + static_cast<int64_t>(w.seq) * p.max_blocks_per_seq;
         for (int32_t j = 0; j < w.ntiles; ++j, ++kvc) {
           const int st = kvc % kPfStages;
-          if (kvc >= kPfStages && !mbar_wait(&kv_empty[st], ((kvc / kPfStages) + 1) & 1)) {
+          if (kvc >= kPfStages && !mbar_wait(&empty_bar[st], ((kvc / kPfStages) + 1) & 1)) {
             ok = false;
             break;
           }
@@ -396,24 +424,29 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int b = 0; b < nblk; ++b) {
             int32_t pb = table[blk0 + b];
             if (pb < 0 || pb >= p.num_blocks) {
-              raise_error(PKV_DEVERR_BLOCK);
+              if (is_k) raise_error(PKV_DEVERR_BLOCK);
               pb = 0;
             }
             rows[b] = (pb * p.num_kv_heads + w.kv_head) * kBlock;
           }
-          const uint32_t bytes = static_cast<uint32_t>(nblk) * H * (kBlock * 128);
-          mbar_arrive_expect_tx(&k_full[st], bytes);
+          mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(nblk) * H * (kBlock * 128));
           for (int b = 0; b < nblk; ++b)
 #pragma unroll
             for (int h = 0; h < H; ++h)
-              tma_load_2d(sK + st * Lay::kKvBytes + h * (kPfKeys * 128) + b * (kBlock * 128),
-                          &map_k, h * 64, rows[b], &k_full[st]);
-          mbar_arrive_expect_tx(&v_full[st], bytes);
-          for (int b = 0; b < nblk; ++b)
+              tma_load_2d(stage_base + st * Lay::kKvBytes + h * (kPfKeys * 128) +
+                              b * (kBlock * 128),
+                          map, h * 64, rows[b], &full_bar[st]);
+          if (is_k && j == 0) {
+            // the unit's Q tile, once the previous unit's last scores are done
+            // (its first K tile is already on its way)
+            if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1)) { ok = false; break; }
+            mbar_arrive_expect_tx(q_full, qrow_bytes * H);
 #pragma unroll
             for (int h = 0; h < H; ++h)
-              tma_load_2d(sV + st * Lay::kKvBytes + h * (kPfKeys * 128) + b * (kBlock * 128),
-                          &map_v, h * 64, rows[b], &v_full[st]);
+              tma_load_3d(sQ + h * (kPfRows * 128), &map_q, h * 64, w.kv_head * g, w.q_row0,
+                          q_full);
+            ++qc;
+          }
         }
       }
       if (!ok) *abort_flag = 1u;
@@ -449,6 +482,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                      ks > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[sb]);
+          umma_commit(&k_empty[st]);  // the K tile is free once the scores are
         }
         __syncwarp();
         ++sc;
@@ -495,7 +529,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                      umma_desc_sw128(v_base + st * Lay::kKvBytes + voff, kPfKeys * 128, 1024),
                      idesc_o, (j > 0 || b > 0) ? 1u : 0u);
           }
-          umma_commit(&kv_empty[st]);
+          umma_commit(&v_empty[st]);
           umma_commit(o_done);
         }
         __syncwarp();
@@ -511,8 +545,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ===================================================== softmax
-    const int r = threadIdx.x - 128;  // query row of the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+    // Warp w reads TMEM lanes 32 (w % 4) ..: thread r owns query row r; the
+    // warpgroup `half` takes keys 64 half .. 64 half + 63 of every tile and
+    // columns D/2 half .. of the output.  The partner warps (w and w + 4) swap
+    // their row maxima each tile through shared memory, meeting at an mbarrier
+    // (two arrivals, a bounded wait like every other).
+    const int r = (warp & 3) * 32 + lane;  // query row of the tile = TMEM lane
+    const int half = (warp - 4) >> 2;
+    constexpr int KH = kPfKeys / 2;          // keys per half
+    constexpr int DH = D / 2;                // output columns per half
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(sm + Lay::kXchgOff);  // [2][2][128]
+    float* xsum = xmax + 4 * kPfRows;                            // [2][128]
+    uint64_t* my_xchg = &xchg[warp & 3];
+    uint32_t xc = 0;  // uses of my_xchg
     const float sc_log2 = p.qk_scale_log2;
     const int32_t rows_used = g * p.tokens_per_tile;
     const int i_tok = r / g, h_in = r - (r / g) * g;
@@ -522,66 +568,93 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const PfUnit w = pf_unit(p, prefix, u);
       const bool row_ok = r < rows_used && i_tok < w.ntok;
       const int32_t lim = row_ok ? w.L - w.q_len + w.tok0 + i_tok : -1;  // last visible key
+      // smallest limit over the warp's rows: tiles wholly below it need no mask
+      int32_t lim_min = lim;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lim_min = min(lim_min, __shfl_xor_sync(0xffffffffu, lim_min, o));
       float m = -INFINITY, l = 0.f;
       for (int32_t j = 0; j < w.ntiles; ++j) {
         const int sb = sc & 1;
         if (!warp_wait(&s_full[sb], (sc >> 1) & 1)) { ok = false; break; }
         ++sc;
         tc_fence_after();
-        float s[kPfKeys];
-        tmem_ld128_wait(lane_base + sb * kPfKeys, s);
+        float s[KH];
+        tmem_ld64_wait(lane_base + sb * kPfKeys + half * KH, s);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
         // scores in log2 units; keys past the row's causal limit (and past the
         // context, and past the blocks loaded for a short last tile) get -inf
-        const int32_t pos0 = j * kPfKeys;
-        float mx = -INFINITY;
+        const int32_t pos0 = j * kPfKeys + half * KH;
+        float mxp[8];
 #pragma unroll
-        for (int c = 0; c < kPfKeys; ++c) {
-          s[c] = pos0 + c <= lim ? s[c] * sc_log2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
+        if (pos0 + KH - 1 <= lim_min) {
+#pragma unroll
+          for (int c = 0; c < KH; ++c) {
+            s[c] *= sc_log2;
+            mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);  // eight independent chains
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < KH; ++c) {
+            s[c] = pos0 + c <= lim ? s[c] * sc_log2 : -INFINITY;
+            mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);
+          }
         }
+        float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        // the row's maximum over both halves
+        xmax[((j & 1) * 2 + half) * kPfRows + r] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(my_xchg);
+        if (!warp_wait(my_xchg, xc & 1)) { ok = false; break; }
+        ++xc;
+        mx = fmaxf(mx, xmax[((j & 1) * 2 + (half ^ 1)) * kPfRows + r]);
         const bool grow = mx > m + kPfRescaleSlack;
         const float alpha = grow ? fast_exp2(m - mx) : 1.f;  // 0 when m = -inf
         if (grow) m = mx;
         // P = 2^(s - m) in bf16 (packed pairs, in registers) and the sum of the
-        // rounded weights, before waiting for the previous tile's P V: the
-        // exponentials overlap that MMA
+        // weights, before waiting for the previous tile's P V: the exponentials
+        // overlap that MMA
         const float mu = m == -INFINITY ? 0.f : m;
-        uint32_t pk[kPfKeys / 2];
-        float lsum = 0.f;
+        uint32_t pk[KH / 2];
+        float lsp[8];
 #pragma unroll
-        for (int c = 0; c < kPfKeys / 2; ++c) {
-          pk[c] = pack_bf16x2(fast_exp2(s[2 * c] - mu), fast_exp2(s[2 * c + 1] - mu));
-          lsum += bf16lo_to_f32(pk[c]) + bf16hi_to_f32(pk[c]);
+        for (int e = 0; e < 8; ++e) lsp[e] = 0.f;
+#pragma unroll
+        for (int c = 0; c < KH / 2; ++c) {
+          const float p0 = fast_exp2(s[2 * c] - mu), p1 = fast_exp2(s[2 * c + 1] - mu);
+          pk[c] = pack_bf16x2(p0, p1);
+          lsp[c & 7] += p0 + p1;
         }
+        const float lsum = ((lsp[0] + lsp[1]) + (lsp[2] + lsp[3])) +
+                           ((lsp[4] + lsp[5]) + (lsp[6] + lsp[7]));
         l = l * alpha + lsum;
         // P and O may be touched only once the previous tile's P V has completed
         if (j > 0) {
           if (!warp_wait(o_done, od & 1)) { ok = false; break; }
           ++od;
           tc_fence_after();
-          // rows whose maximum moved rescale their output row (warp-uniform:
+          // rows whose maximum moved rescale their output columns (warp-uniform:
           // the other rows of the warp multiply by 1)
           if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < DH / 32; ++c) {
               float o[32];
-              tmem_ld32_wait(lane_base + 2 * kPfKeys + c * 32, o);
+              tmem_ld32_wait(lane_base + 2 * kPfKeys + half * DH + c * 32, o);
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] *= alpha;
-              tmem_st32(lane_base + 2 * kPfKeys + c * 32, o);
+              tmem_st32(lane_base + 2 * kPfKeys + half * DH + c * 32, o);
             }
             tmem_wait_st();
           }
         }
-        // P row r in [key half][row][128 B] with the 128-byte swizzle
+        // this half's 64 keys of row r: [key half][row][128 B] with the
+        // 128-byte swizzle
 #pragma unroll
-        for (int k = 0; k < kPfKeys / 8; ++k) {
-          const int half = k >> 3, chunk = k & 7;
-          *reinterpret_cast<uint4*>(sP + half * (kPfRows * 128) + r * 128 +
-                                    ((chunk ^ (r & 7)) << 4)) =
+        for (int k = 0; k < 8; ++k) {
+          *reinterpret_cast<uint4*>(sP + half * (kPfRows * 128) + r * 128 + ((k ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
         fence_proxy_async_smem();
@@ -591,17 +664,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       if (!ok) break;
       if (w.ntiles > 0) {
+        // the row's weight sum over both halves
+        xsum[half * kPfRows + r] = l;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(my_xchg);
+        if (!warp_wait(my_xchg, xc & 1)) { ok = false; break; }
+        ++xc;
+        l += xsum[(half ^ 1) * kPfRows + r];
         if (!warp_wait(o_done, od & 1)) { ok = false; break; }
         ++od;
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
                               (static_cast<int64_t>(w.q_row0 + i_tok) * p.num_q_heads +
-                               w.kv_head * g + h_in) * D;
+                               w.kv_head * g + h_in) * D + half * DH;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < DH / 32; ++c) {
           float o[32];
-          tmem_ld32_wait(lane_base + 2 * kPfKeys + c * 32, o);
+          tmem_ld32_wait(lane_base + 2 * kPfKeys + half * DH + c * 32, o);
           if (row_ok) {
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
