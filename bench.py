@@ -251,6 +251,8 @@ class Step:
         # sequences that share a prompt's blocks: read those blocks once per group
         self.shared = shared_prefix and "group_start" in b.meta and not self.multi
         if self.shared:
+            self.part_tokens = pkv.decode_shared_partition_tokens(self.dims, self.mcl,
+                                                                  partition_tokens)
             self.group_start = torch.tensor(b.meta["group_start"], dtype=torch.int32, device=dev)
             self.shared_blocks = torch.tensor(b.meta["shared_blocks"], dtype=torch.int32,
                                               device=dev)

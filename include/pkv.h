@@ -457,6 +457,17 @@ pkv_status pkv_decode_run_fp8(void *out, const void *q, const void *k_cache,
  * pkv_decode_workspace_layout) and of seq_prefix, int32 [num_seqs] = P used
  * for each sequence after the plan (for tests).
  */
+/*
+ * Partition size (tokens) the shared-prefix plan uses for these arguments
+ * (0 = automatic; otherwise the request).  Its automatic choice differs from
+ * pkv_decode_partition_tokens for bf16 head_dim-128 caches: those plans run
+ * one warp per work item, so the prefix and the sequences' own blocks are cut
+ * finer (about 16 items per warp, at least 512 tokens each).  Returns 0 for
+ * invalid dims.
+ */
+int32_t pkv_decode_shared_partition_tokens(const pkv_dims *dims, int32_t max_context_len,
+                                           int32_t partition_tokens);
+
 size_t pkv_decode_shared_workspace_bytes(const pkv_dims *dims, int32_t max_context_len,
                                          int32_t partition_tokens);
 

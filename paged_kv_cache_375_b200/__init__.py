@@ -80,6 +80,7 @@ def load_library() -> ctypes.CDLL:
         D = ctypes.POINTER(PkvDims)
         sig = {
             "pkv_decode_partition_tokens": (i32, [D, i32, i32]),
+            "pkv_decode_shared_partition_tokens": (i32, [D, i32, i32]),
             "pkv_decode_workspace_bytes": (sz, [D, i32, i32]),
             "pkv_decode_workspace_layout": (ctypes.c_int, [D, i32, i32, P, P, P]),
             "pkv_paged_attention_decode": (ctypes.c_int, [P, P, P, P, P, P, f32, D, i32, i32, P,
@@ -203,6 +204,13 @@ def make_dims(num_seqs: int, num_q_heads: int, k_cache: torch.Tensor,
 def decode_partition_tokens(dims: PkvDims, max_context_len: int, partition_tokens: int = 0) -> int:
     return load_library().pkv_decode_partition_tokens(ctypes.byref(dims), max_context_len,
                                                       partition_tokens)
+
+
+def decode_shared_partition_tokens(dims: PkvDims, max_context_len: int,
+                                   partition_tokens: int = 0) -> int:
+    """Partition size of the shared-prefix plan (see pkv_decode_shared_partition_tokens)."""
+    return load_library().pkv_decode_shared_partition_tokens(ctypes.byref(dims), max_context_len,
+                                                             partition_tokens)
 
 
 def decode_workspace_bytes(dims: PkvDims, max_context_len: int, partition_tokens: int = 0) -> int:

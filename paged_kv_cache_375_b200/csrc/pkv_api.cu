@@ -141,10 +141,16 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // length: P = the power of two >= B*Hkv*max_len / (16*SMs), within
 // [512, 8192] tokens.  When that covers the longest sequence the decode is
 // single-pass (the planner then orders whole sequences longest first).
-int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested) {
+//
+// Shared-prefix plans of bf16 head_dim-128 caches run on decode_warp_kernel,
+// whose work is handed out per warp: there the aim is about 16 items per
+// warp (eight per SM), so a long prefix is cut into several items that
+// different warps read at once.
+int32_t choose_partition(const pkv_dims* d, int32_t max_len, int32_t requested,
+                         bool per_warp = false) {
   if (requested > 0) return requested;
   const int64_t units = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
-  const int64_t target = units * max_len / (16ll * device_sm_count());
+  const int64_t target = units * max_len / (16ll * device_sm_count() * (per_warp ? 8 : 1));
   int64_t p = 512;
   while (p < target && p < pkv::kMaxItemBlocks * pkv::kBlock) p *= 2;
   if (p >= max_len)
@@ -173,7 +179,8 @@ pkv_status make_plan(const pkv_dims* d, int32_t max_context_len, int32_t partiti
   DecodePlan p;
   p.max_len = max_len;
   p.num_q_tokens = num_q_tokens < 0 ? d->num_seqs : num_q_tokens;
-  p.part_tokens = choose_partition(d, max_len, partition_tokens);
+  p.part_tokens = choose_partition(d, max_len, partition_tokens,
+                                   shared && d->dtype == PKV_BF16 && d->head_dim == 128);
   p.part_blocks = p.part_tokens / pkv::kBlock;
   p.max_parts = max_len <= 0 ? 1 : (max_len + p.part_tokens - 1) / p.part_tokens;
   const size_t B = static_cast<size_t>(d->num_seqs);
@@ -337,13 +344,16 @@ pkv_status launch_decode(const CUtensorMap& mk, const CUtensorMap& mv,
 }
 
 // Short items (split-K partitions of at most kWarpItemMaxBlocks blocks, the
-// shared-prefix plan) of bf16 head_dim-128 decode: one warp per item, eight
-// warps per CTA, 3 tile stages each for up to 8 query rows, 2 for 16.
+// shared-prefix plan) of bf16 head_dim-128 decode: one warp per item; for up
+// to 8 query rows eight warps per CTA with 3 tile stages each, for 16 rows
+// (the 16-row state needs 239 registers) six warps with 4 stages (measured on
+// the parallel-sampling batch: 8 x 2 stages 0.116 ms, 7 x 3 0.110, 6 x 4
+// 0.106; on the long-context batch at 512-token partitions 8 x 3 beat 6 x 4).
 template <int GMAX>
 pkv_status launch_decode_warp(const CUtensorMap& mk, const CUtensorMap& mv,
                               const pkv::DecodeParams& prm, int64_t work_units,
                               cudaStream_t stream) {
-  constexpr int W = 8, S = GMAX <= 8 ? 3 : 2;
+  constexpr int W = GMAX <= 8 ? 8 : 6, S = GMAX <= 8 ? 3 : 4;
   using Lay = pkv::WarpDecodeLayout<GMAX, W, S>;
   auto kern = pkv::decode_warp_kernel<GMAX, W, S>;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), Lay::kTotal);
@@ -895,6 +905,13 @@ int32_t pkv_decode_partition_tokens(const pkv_dims* dims, int32_t max_context_le
                                     int32_t partition_tokens) {
   DecodePlan plan;
   if (make_plan(dims, max_context_len, partition_tokens, &plan) != PKV_OK) return 0;
+  return plan.part_tokens;
+}
+
+int32_t pkv_decode_shared_partition_tokens(const pkv_dims* dims, int32_t max_context_len,
+                                           int32_t partition_tokens) {
+  DecodePlan plan;
+  if (make_plan(dims, max_context_len, partition_tokens, &plan, -1, true) != PKV_OK) return 0;
   return plan.part_tokens;
 }
 

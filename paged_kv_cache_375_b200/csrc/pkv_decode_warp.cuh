@@ -24,6 +24,8 @@
 // blocks.
 #pragma once
 
+#include <type_traits>
+
 #include "pkv_decode.cuh"
 
 namespace pkv {
@@ -101,7 +103,6 @@ __global__ void __launch_bounds__(W * 32, 1)
                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
   using Lay = WarpDecodeLayout<GMAX, W, S>;
   constexpr int D = 128;
-  using St = Bf16State<D, GMAX>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -218,15 +219,17 @@ __global__ void __launch_bounds__(W * 32, 1)
     }
   };
 
-  St st;
   bool ok = true;
   uint32_t qc = 0;               // q loads consumed
-  while (has_cur) {
-    produce();
-    if (!mbar_wait(qbar, qc & 1)) { ok = false; break; }
-    ++qc;
+  // One item with a state of G rows (G = 8 for items of at most 8 query rows,
+  // so a 16-row kernel does not spend half its MMAs and exponentials on empty
+  // rows; else GMAX).
+  auto run_item = [&](auto rows_tag) {
+    constexpr int G = decltype(rows_tag)::value;
+    using Sg = Bf16State<D, G>;
+    Sg st;
     const int rows = cur.q_len * g;
-    bf16_begin_item<D, GMAX>(st, qbuf, rows, g, cur.len, 1, lane);
+    bf16_begin_item<D, G>(st, qbuf, rows, g, cur.len, 1, lane);
     __syncwarp();                // every lane has its q fragments: the buffer is free
     if (has_nxt) load_q(nxt);
     for (int32_t b = 0; b < cur.nblk; b += 2) {
@@ -245,20 +248,19 @@ __global__ void __launch_bounds__(W * 32, 1)
           valid[x] = v > kBlock ? kBlock : v;
         }
       }
-      if (!ok) break;
+      if (!ok) return;
       const int pos0 = (cur.blk_begin + b) * kBlock;
       if (rows > 0)
-        bf16_step<D, GMAX>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
-                           kt[1] + Lay::kTileBytes, valid[1], pos0 + kBlock, sc, lane);
+        bf16_step<D, G>(st, kt[0], kt[0] + Lay::kTileBytes, valid[0], pos0, kt[1],
+                        kt[1] + Lay::kTileBytes, valid[1], pos0 + kBlock, sc, lane);
       __syncwarp();
       cctr += n;
       produce();
     }
-    if (!ok) break;
     // ---- the item's result, straight from the fragments: row n = nh*8 + qd + hc,
     // column d = 16 mt + r (and + 8) ----
 #pragma unroll
-    for (int nh = 0; nh < St::NH; ++nh)
+    for (int nh = 0; nh < Sg::NH; ++nh)
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
         const int n = nh * 8 + qd + hc;
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(W * 32, 1)
           if (cur.nparts == 1) {
             uint16_t* o16 = reinterpret_cast<uint16_t*>(prm.out) + row * D;
 #pragma unroll
-            for (int mt = 0; mt < St::MT; ++mt) {
+            for (int mt = 0; mt < Sg::MT; ++mt) {
               o16[mt * 16 + r] = static_cast<uint16_t>(pack_bf16x2(st.o[nh][mt][hc] * inv, 0.f));
               o16[mt * 16 + r + 8] =
                   static_cast<uint16_t>(pack_bf16x2(st.o[nh][mt][hc + 2] * inv, 0.f));
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(W * 32, 1)
             const size_t prow = row * prm.max_parts + cur.part;
             float* po = prm.part_o + prow * D;
 #pragma unroll
-            for (int mt = 0; mt < St::MT; ++mt) {
+            for (int mt = 0; mt < Sg::MT; ++mt) {
               po[mt * 16 + r] = st.o[nh][mt][hc] * inv;
               po[mt * 16 + r + 8] = st.o[nh][mt][hc + 2] * inv;
             }
@@ -291,6 +293,17 @@ __global__ void __launch_bounds__(W * 32, 1)
           }
         }
       }
+  };
+  while (has_cur) {
+    produce();
+    if (!mbar_wait(qbar, qc & 1)) { ok = false; break; }
+    ++qc;
+    if (GMAX > 8 && cur.q_len * g <= 8) {
+      run_item(std::integral_constant<int, 8>{});
+    } else {
+      run_item(std::integral_constant<int, GMAX>{});
+    }
+    if (!ok) break;
     // ---- next item ----
     if (!has_nxt) break;
     cur = nxt;

@@ -407,47 +407,73 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint64_t* empty_bar = is_k ? k_empty : v_empty;
       if (is_k) prefetch_tensormap(&map_q);
       prefetch_tensormap(map);
+      // The stream of (unit, KV tile) this CTA loads.  The block-table entries
+      // of the next tile are read before waiting for a free stage, so their
+      // latency is off the critical path.
+      int32_t u = blockIdx.x, j = 0;
+      PfUnit w{};
+      if (u < total_units) w = pf_unit(p, prefix, u);
+      auto read_rows = [&](const PfUnit& wu, int32_t jj, int32_t (&rows)[kPfBlocksPerTile],
+                           int32_t& nblk) {
+        const int32_t* table = p.block_tables + static_cast<int64_t>(wu.seq) * p.max_blocks_per_seq;
+        const int32_t blk0 = jj * kPfBlocksPerTile;
+        nblk = min(kPfBlocksPerTile, (wu.nkv - jj * kPfKeys + kBlock - 1) / kBlock);
+#pragma unroll
+        for (int b = 0; b < kPfBlocksPerTile; ++b) rows[b] = b < nblk ? table[blk0 + b] : 0;
+      };
+      int32_t rows[kPfBlocksPerTile], nblk = 0;
+      if (u < total_units) read_rows(w, 0, rows, nblk);
       uint32_t qc = 0, kvc = 0;
       bool ok = true;
-      for (int32_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const PfUnit w = pf_unit(p, prefix, u);
-        const int32_t* table = p.block_tables + static_cast<int64_t>(w.seq) * p.max_blocks_per_seq;
-        for (int32_t j = 0; j < w.ntiles; ++j, ++kvc) {
-          const int st = kvc % kPfStages;
-          if (kvc >= kPfStages && !mbar_wait(&empty_bar[st], ((kvc / kPfStages) + 1) & 1)) {
-            ok = false;
-            break;
-          }
-          const int32_t blk0 = j * kPfBlocksPerTile;
-          const int32_t nblk = min(kPfBlocksPerTile, (w.nkv - j * kPfKeys + kBlock - 1) / kBlock);
-          int32_t rows[kPfBlocksPerTile];
-          for (int b = 0; b < nblk; ++b) {
-            int32_t pb = table[blk0 + b];
-            if (pb < 0 || pb >= p.num_blocks) {
-              if (is_k) raise_error(PKV_DEVERR_BLOCK);
-              pb = 0;
-            }
-            rows[b] = (pb * p.num_kv_heads + w.kv_head) * kBlock;
-          }
-          mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(nblk) * H * (kBlock * 128));
-          for (int b = 0; b < nblk; ++b)
-#pragma unroll
-            for (int h = 0; h < H; ++h)
-              tma_load_2d(stage_base + st * Lay::kKvBytes + h * (kPfKeys * 128) +
-                              b * (kBlock * 128),
-                          map, h * 64, rows[b], &full_bar[st]);
-          if (is_k && j == 0) {
-            // the unit's Q tile, once the previous unit's last scores are done
-            // (its first K tile is already on its way)
-            if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1)) { ok = false; break; }
-            mbar_arrive_expect_tx(q_full, qrow_bytes * H);
-#pragma unroll
-            for (int h = 0; h < H; ++h)
-              tma_load_3d(sQ + h * (kPfRows * 128), &map_q, h * 64, w.kv_head * g, w.q_row0,
-                          q_full);
-            ++qc;
-          }
+      while (u < total_units) {
+        // the tile after this one (possibly the first of the next unit)
+        int32_t un = u, jn = j + 1;
+        PfUnit wn = w;
+        if (jn >= w.ntiles) {
+          un = u + gridDim.x;
+          jn = 0;
+          if (un < total_units) wn = pf_unit(p, prefix, un);
         }
+        int32_t rows_n[kPfBlocksPerTile], nblk_n = 0;
+        if (un < total_units) read_rows(wn, jn, rows_n, nblk_n);
+        // this tile
+        const int st = kvc % kPfStages;
+        if (kvc >= kPfStages && !mbar_wait(&empty_bar[st], ((kvc / kPfStages) + 1) & 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(nblk) * H * (kBlock * 128));
+        for (int b = 0; b < nblk; ++b) {
+          int32_t pb = rows[b];
+          if (pb < 0 || pb >= p.num_blocks) {
+            if (is_k) raise_error(PKV_DEVERR_BLOCK);
+            pb = 0;
+          }
+          const int32_t y = (pb * p.num_kv_heads + w.kv_head) * kBlock;
+#pragma unroll
+          for (int h = 0; h < H; ++h)
+            tma_load_2d(stage_base + st * Lay::kKvBytes + h * (kPfKeys * 128) +
+                            b * (kBlock * 128),
+                        map, h * 64, y, &full_bar[st]);
+        }
+        ++kvc;
+        if (is_k && j == 0) {
+          // the unit's Q tile, once the previous unit's last scores are done
+          // (its first K tile is already on its way)
+          if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(q_full, qrow_bytes * H);
+#pragma unroll
+          for (int h = 0; h < H; ++h)
+            tma_load_3d(sQ + h * (kPfRows * 128), &map_q, h * 64, w.kv_head * g, w.q_row0,
+                        q_full);
+          ++qc;
+        }
+        u = un;
+        j = jn;
+        w = wn;
+        nblk = nblk_n;
+#pragma unroll
+        for (int b = 0; b < kPfBlocksPerTile; ++b) rows[b] = rows_n[b];
       }
       if (!ok) *abort_flag = 1u;
     }

@@ -191,13 +191,18 @@ def test_shared_prefix_workspace_sizes():
     and per-group block counts."""
     d = dims(B=256, hq=32, hkv=8, nb=40000, mb=512)
     assert pkv.decode_workspace_bytes(d, 1600) < pkv.decode_shared_workspace_bytes(d, 1600)
+    # bf16 head_dim 128: the automatic partition aims at ~16 items per warp (one warp per
+    # item), at least 512 tokens: 512 here, so 4 partitions of the context + 1
+    assert pkv.decode_shared_partition_tokens(d, 1600) == 512
+    assert pkv.decode_partition_tokens(d, 1600) >= 1600       # the plain plan: single pass
     max_parts, po, pm, sp = pkv.decode_shared_workspace_layout(d, 1600)
-    assert max_parts == 2
+    assert max_parts == 5
+    assert pkv.decode_shared_workspace_layout(d, 1600, 2048)[0] == 2
     assert sp % 256 == 0 and po % 256 == 0 and pm % 256 == 0
-    assert sp >= 256 + 2 * 256 * 2 * 32            # counters, then 2*B*max_parts items
+    assert sp >= 256 + 2 * 256 * 5 * 32            # counters, then 2*B*max_parts items
     assert po >= sp + 2 * 256 * 4                  # seq_prefix, group block counts
-    assert pm >= po + 256 * 32 * 2 * 128 * 4
-    assert pkv.decode_shared_workspace_bytes(d, 1600) >= pm + 256 * 32 * 2 * 2 * 4
+    assert pm >= po + 256 * 32 * 5 * 128 * 4
+    assert pkv.decode_shared_workspace_bytes(d, 1600) >= pm + 256 * 32 * 5 * 2 * 4
     # split-K: one partial more than the plain decode's
     d = dims(B=8, hq=64, hkv=8, nb=81920, mb=8192)
     assert pkv.decode_shared_workspace_layout(d, 131072, 512)[0] == \
