@@ -19,11 +19,11 @@
 //   O += P V     (M 128 rows, N = head_dim, K = 128 keys) into TMEM
 //
 // Roles in a CTA of 8 warps (one CTA per SM, persistent over work units):
-//  * warp 0, two lanes: TMA producers.  Lane 0 loads the unit's Q tile (a 3-D
-//    tensor map over q [T][Hq][D], box {64 d, g heads, tokens}) and, per KV
-//    tile of 128 keys, the tile's 8 blocks of K through the block table (the
-//    2-D pool map, one box per block and 64-column half); lane 1 does the same
-//    for V.  Stages are 128-byte swizzled, laid out [half][128 keys][128 B]; a
+//  * warps 0 and 2, one lane each: TMA producers.  Warp 0 loads the unit's Q
+//    tile (a 3-D tensor map over q [T][Hq][D], box {64 d, g heads, tokens})
+//    and, per KV tile of 128 keys, the tile's 8 blocks of K through the block
+//    table (the 2-D pool map, one box per block and 64-column half); warp 2
+//    does the same for V.  Stages are 128-byte swizzled, laid out [half][128 keys][128 B]; a
 //    K stage is released when its scores are computed, a V stage when its
 //    P V is.
 //  * warp 1: TMEM allocation; one lane issues the MMAs and commits them to
@@ -51,11 +51,14 @@ namespace pkv {
 constexpr int kPfRows = 128;       // query rows per tile: the MMA's M
 constexpr int kPfKeys = 128;       // keys per KV tile: N of S = Q K^T, K of O += P V
 constexpr int kPfBlocksPerTile = kPfKeys / kBlock;
-constexpr int kPfStages = 2;       // KV tile stages
-constexpr int kPfThreads = 384;    // warp 0 producers, warp 1 MMA, warps 4-11 softmax
+constexpr int kPfKStages = 3;      // K tile stages (a K stage frees as soon as its scores are done)
+constexpr int kPfVStages = 2;      // V tile stages
+constexpr int kPfThreads = 384;    // warps 0, 2 producers, warp 1 MMA, warps 4-11 softmax
 constexpr int kPfSoftmaxWarps = 8;  // two warpgroups: keys 0-63 and 64-127 of every row
 constexpr int kPfMaxSeqs = 2048;   // sequences per call (per-CTA tile prefix in shared memory)
-constexpr uint32_t kPfTmemCols = 512;  // S buffers at columns 0 and 128, O at 256
+constexpr uint32_t kPfTmemCols = 512;  // S buffers at columns 0 and 128, O at 256, P at 384
+constexpr uint32_t kPfTmemO = 2 * kPfKeys;        // O: head_dim columns of fp32
+constexpr uint32_t kPfTmemP = 3 * kPfKeys;        // P: bf16 pairs, kPfKeys / 2 columns
 constexpr float kPfRescaleSlack = 8.f; // the running max moves when it grows by more (log2)
 
 struct PrefillParams {
@@ -74,17 +77,15 @@ template <int D>
 struct PfLayout {
   static constexpr int kHalves = D / 64;                       // 128-byte column halves
   static constexpr int kQBytes = kHalves * kPfRows * 128;      // [half][128 rows][128 B]
-  static constexpr int kPBytes = (kPfKeys / 64) * kPfRows * 128;  // [key half][128 rows][128 B]
   static constexpr int kKvBytes = kHalves * kPfKeys * 128;     // one K (or V) stage
   static constexpr int kQOff = 0;
-  static constexpr int kPOff = kQOff + kQBytes;
-  static constexpr int kKOff = kPOff + kPBytes;
-  static constexpr int kVOff = kKOff + kPfStages * kKvBytes;
-  static constexpr int kPrefixOff = kVOff + kPfStages * kKvBytes;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + kPfKStages * kKvBytes;
+  static constexpr int kPrefixOff = kVOff + kPfVStages * kKvBytes;
   static constexpr int kBarsOff = kPrefixOff + (kPfMaxSeqs + 8) * 4;
-  // q_full, q_empty, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], s_free[2],
-  // p_full, o_done, final, xchg[4] (the two softmax warps of each row quarter)
-  static constexpr int kNumBars = 2 + 4 * kPfStages + 4 + 3 + 4;
+  // q_full, q_empty, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2],
+  // s_free[2], p_full, o_done, final, xchg[4] (the two softmax warps of each row quarter)
+  static constexpr int kNumBars = 2 + 2 * kPfKStages + 2 * kPfVStages + 4 + 3 + 4;
   static constexpr int kMiscOff = kBarsOff + kNumBars * 8;     // tmem base, abort flag
   // row maxima exchanged between the two softmax warpgroups: [parity][half][row],
   // then the row sums [half][row]
@@ -121,6 +122,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same with A in tensor memory (M rows on the lanes, two 16-bit
+// elements per 32-bit column along K).
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -192,6 +204,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  float f[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+  tmem_st32(taddr, f);
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
@@ -308,7 +327,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = sm + Lay::kQOff;
-  uint8_t* sP = sm + Lay::kPOff;
   uint8_t* sK = sm + Lay::kKOff;
   uint8_t* sV = sm + Lay::kVOff;
   int32_t* prefix = reinterpret_cast<int32_t*>(sm + Lay::kPrefixOff);
@@ -316,10 +334,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  uint64_t* v_full = k_full + kPfStages;
-  uint64_t* k_empty = v_full + kPfStages;
-  uint64_t* v_empty = k_empty + kPfStages;
-  uint64_t* s_full = v_empty + kPfStages;
+  uint64_t* k_empty = k_full + kPfKStages;
+  uint64_t* v_full = k_empty + kPfKStages;
+  uint64_t* v_empty = v_full + kPfVStages;
+  uint64_t* s_full = v_empty + kPfVStages;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* o_done = p_full + 1;
@@ -332,10 +350,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < kPfStages; ++i) {
+    for (int i = 0; i < kPfKStages; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kPfVStages; ++i) {
+      mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -394,17 +414,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int g = p.group;
   const uint32_t qrow_bytes = 128u * static_cast<uint32_t>(g * p.tokens_per_tile);
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2) {
     // ===================================================== TMA producers
-    // Lane 0 loads Q and the K tiles, lane 1 the V tiles: a K stage is free
-    // once the tile's scores are computed, a V stage only once its P V is,
-    // so the next K tiles are not held up behind the current P V.
-    if (lane < 2) {
-      const bool is_k = lane == 0;
+    // Warp 0 (one lane) loads Q and the K tiles, warp 2 the V tiles: a K
+    // stage is free once the tile's scores are computed, a V stage only once
+    // its P V is, so the next K tiles are not held up behind the current P V.
+    // (Two lanes of one warp would not do: while one waits on its barrier
+    // the other's path does not run.)
+    if (lane == 0) {
+      const bool is_k = warp == 0;
       const CUtensorMap* map = is_k ? &map_k : &map_v;
       uint8_t* stage_base = is_k ? sK : sV;
       uint64_t* full_bar = is_k ? k_full : v_full;
       uint64_t* empty_bar = is_k ? k_empty : v_empty;
+      const uint32_t nst = is_k ? kPfKStages : kPfVStages;
       if (is_k) prefetch_tensormap(&map_q);
       prefetch_tensormap(map);
       // The stream of (unit, KV tile) this CTA loads.  The block-table entries
@@ -437,8 +460,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int32_t rows_n[kPfBlocksPerTile], nblk_n = 0;
         if (un < total_units) read_rows(wn, jn, rows_n, nblk_n);
         // this tile
-        const int st = kvc % kPfStages;
-        if (kvc >= kPfStages && !mbar_wait(&empty_bar[st], ((kvc / kPfStages) + 1) & 1)) {
+        const int st = kvc % nst;
+        if (kvc >= nst && !mbar_wait(&empty_bar[st], ((kvc / nst) + 1) & 1)) {
           ok = false;
           break;
         }
@@ -481,7 +504,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ===================================================== MMA issue
     constexpr uint32_t idesc_s = umma_idesc_bf16(kPfRows, kPfKeys, false);
     constexpr uint32_t idesc_o = umma_idesc_bf16(kPfRows, D, true);
-    const uint32_t q_base = smem_addr(sQ), p_base = smem_addr(sP);
+    const uint32_t q_base = smem_addr(sQ);
     const uint32_t k_base = smem_addr(sK), v_base = smem_addr(sV);
     uint32_t qc = 0, kvc = 0, sc = 0, pc = 0;
     bool ok = true;
@@ -493,8 +516,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // S_j = Q K_j^T into S buffer sc % 2
       auto issue_s = [&](int32_t j) -> bool {
         const uint32_t c = kv0 + j;
-        const int st = c % kPfStages;
-        if (!warp_wait(&k_full[st], (c / kPfStages) & 1)) return false;
+        const int st = c % kPfKStages;
+        if (!warp_wait(&k_full[st], (c / kPfKStages) & 1)) return false;
         const int sb = sc & 1;
         if (sc >= 2 && !warp_wait(&s_free[sb], ((sc >> 1) + 1) & 1)) return false;
         tc_fence_after();
@@ -522,10 +545,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           __syncwarp();
         }
         const uint32_t c = kv0 + j;
-        const int st = c % kPfStages;
+        const int st = c % kPfVStages;
         if (!warp_wait(p_full, pc & 1)) { ok = false; break; }
         ++pc;
-        if (!warp_wait(&v_full[st], (c / kPfStages) & 1)) { ok = false; break; }
+        if (!warp_wait(&v_full[st], (c / kPfVStages) & 1)) { ok = false; break; }
         const int32_t nblk = min(kPfBlocksPerTile, (w.nkv - j * kPfKeys + kBlock - 1) / kBlock);
         // value rows past the context in the context's last block: zero them
         // (their weights are zero, but NaN or Inf there would still poison O)
@@ -549,11 +572,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         if (lane == 0) {
           for (int b = 0; b < nblk; ++b) {
-            const uint32_t poff = (b >> 2) * (kPfRows * 128) + (b & 3) * 32;
+            // A = P from tensor memory: the 16 keys of block b are columns 8b .. 8b+7
             const uint32_t voff = b * (kBlock * 128);
-            umma_f16(tmem + 2 * kPfKeys, umma_desc_sw128(p_base + poff, 16, 1024),
-                     umma_desc_sw128(v_base + st * Lay::kKvBytes + voff, kPfKeys * 128, 1024),
-                     idesc_o, (j > 0 || b > 0) ? 1u : 0u);
+            umma_f16_tmem_a(tmem + kPfTmemO, tmem + kPfTmemP + b * (kBlock / 2),
+                            umma_desc_sw128(v_base + st * Lay::kKvBytes + voff, kPfKeys * 128,
+                                            1024),
+                            idesc_o, (j > 0 || b > 0) ? 1u : 0u);
           }
           umma_commit(&v_empty[st]);
           umma_commit(o_done);
@@ -668,22 +692,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll 1
             for (int c = 0; c < DH / 32; ++c) {
               float o[32];
-              tmem_ld32_wait(lane_base + 2 * kPfKeys + half * DH + c * 32, o);
+              tmem_ld32_wait(lane_base + kPfTmemO + half * DH + c * 32, o);
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] *= alpha;
-              tmem_st32(lane_base + 2 * kPfKeys + half * DH + c * 32, o);
+              tmem_st32(lane_base + kPfTmemO + half * DH + c * 32, o);
             }
             tmem_wait_st();
           }
         }
-        // this half's 64 keys of row r: [key half][row][128 B] with the
-        // 128-byte swizzle
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          *reinterpret_cast<uint4*>(sP + half * (kPfRows * 128) + r * 128 + ((k ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-        }
-        fence_proxy_async_smem();
+        // this half's 64 keys of row r into tensor memory, two bf16 a column
+        // (keys 2c and 2c+1 in column c, the lower key in the low half): the
+        // A operand of P V
+        tmem_st32u(lane_base + kPfTmemP + half * (KH / 2), pk);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full);
@@ -707,7 +728,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < DH / 32; ++c) {
           float o[32];
-          tmem_ld32_wait(lane_base + 2 * kPfKeys + half * DH + c * 32, o);
+          tmem_ld32_wait(lane_base + kPfTmemO + half * DH + c * 32, o);
           if (row_ok) {
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
