@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpkv.so")
 SOURCES = ["pkv_api.cu", "pkv_block_manager.cpp"]
 DEPS = SOURCES + ["pkv_device.cuh", "pkv_decode.cuh", "pkv_cache_ops.cuh", "pkv_prepare.cuh",
-                  "pkv_prefill.cuh", "pkv_decode_warp.cuh"]
+                  "pkv_prefill.cuh", "pkv_decode_warp.cuh", "pkv_decode_fp8tc.cuh"]
 HEADERS = ["pkv.h", "pkv_block_manager.h"]
 
 NVCC_FLAGS = [

@@ -15,6 +15,7 @@
 #include "pkv.h"
 #include "pkv_cache_ops.cuh"
 #include "pkv_decode.cuh"
+#include "pkv_decode_fp8tc.cuh"
 #include "pkv_decode_warp.cuh"
 #include "pkv_device.cuh"
 #include "pkv_prefill.cuh"
@@ -368,6 +369,27 @@ pkv_status launch_decode_warp(const CUtensorMap& mk, const CUtensorMap& mv,
   return PKV_OK;
 }
 
+// Decode over e4m3 pools on the tcgen05 tensor cores (one query token per
+// sequence, plain or split-K plans).
+template <int RM>
+pkv_status launch_decode_fp8tc(const CUtensorMap& mk, const CUtensorMap& mv,
+                               const pkv::DecodeParams& prm, int64_t work_units,
+                               cudaStream_t stream) {
+  constexpr int ST = pkv::tc_stages<RM>();
+  auto kern = pkv::decode_fp8tc_kernel<RM, ST>;
+  constexpr int smem = pkv::TcLayout<ST>::kTotal;
+  cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_fp8tc)");
+  // persistent: two CTAs per SM with three stages each, else one
+  int64_t grid = static_cast<int64_t>(device_sm_count()) * (ST <= 3 ? 2 : 1);
+  if (grid > work_units) grid = work_units;
+  if (grid < 1) grid = 1;
+  e = launch(kern, dim3(static_cast<unsigned>(grid)), dim3(pkv::kTcThreads), smem, stream, mk,
+             mv, prm);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_fp8tc launch");
+  return PKV_OK;
+}
+
 // The query rows of an item (chunk length x group) go on the MMA's N side:
 // up to 8 or up to 16 rows.
 template <typename T, int D>
@@ -540,7 +562,13 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.out_scale = v_scale;
   const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads *
                         (plan.shared ? 2 : row_groups);
-  if (d->dtype == PKV_FP8_E4M3) {
+  if (d->dtype == PKV_FP8_E4M3 && (!query_start_loc || max_query_len == 1) && !plan.shared &&
+      group <= 16) {
+    // one query token per sequence over e4m3 codes: the tensor-core path
+    st = group <= 4   ? launch_decode_fp8tc<4>(mk, mv, prm, units, stream)
+         : group <= 8 ? launch_decode_fp8tc<8>(mk, mv, prm, units, stream)
+                      : launch_decode_fp8tc<16>(mk, mv, prm, units, stream);
+  } else if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_FP8_E5M2) {
     st = launch_decode_d<pkv::Fp8E5m2Kv, 128>(mk, mv, prm, units, rows_max, stream);
