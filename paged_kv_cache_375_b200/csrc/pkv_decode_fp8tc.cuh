@@ -452,68 +452,92 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
       const int b = n & 1;
       if (!warp_wait(&bq_full[b], (n >> 1) & 1)) { ok = false; break; }
       const uint32_t c0 = c;
-      auto issue_s = [&](int32_t j) -> bool {
-        const uint32_t cc = c0 + j;
-        const int st = cc % ST;
-        if (!warp_wait(&k_full[st], (cc / ST) & 1)) return false;
-        const int sb = sc & 1;
-        if (sc >= 2 && !warp_wait(&s_free[sb], ((sc >> 1) + 1) & 1)) return false;
-        tc_fence_after();
-        if (lane == 0) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            umma_f8(tmem + sb * kTcN,
-                    umma_desc(k_base + st * Lay::kTileBytes + ks * 32, 16, 1024, 2),
-                    umma_desc(bq_base + b * Lay::kBqBytes + ks * 32, 16, 1024, 2), idesc_s,
-                    ks > 0 ? 1u : 0u);
-          umma_commit(&s_full[sb]);
-          umma_commit(&k_empty[st]);
-        }
-        __syncwarp();
-        ++sc;
-        return true;
-      };
-      if (w.ntiles > 0 && !issue_s(0)) { ok = false; break; }
       if (w.ntiles == 0) {
         if (lane == 0) umma_commit(&bq_empty[b]);
         __syncwarp();
       }
-      for (int32_t j = 0; j < w.ntiles; ++j) {
-        if (j + 1 < w.ntiles && !issue_s(j + 1)) { ok = false; break; }
-        if (j + 1 == w.ntiles) {
-          if (lane == 0) umma_commit(&bq_empty[b]);  // the unit's last scores read Bq
-          __syncwarp();
-        }
-        const uint32_t cc = c0 + j;
-        const int st = cc % ST;
-        if (!warp_wait(p_full, pc & 1)) { ok = false; break; }
-        ++pc;
-        if (!warp_wait(&v_full[st], (cc / ST) & 1)) { ok = false; break; }
-        // keys of this tile inside the context; P V runs over whole 32-key steps,
-        // the value rows past the context within them are zeroed first
-        const int32_t valid = min(kTcKeys, w.end - (w.blk_begin + j * kTcBlocks) * kBlock);
-        const int ksteps = (valid + 31) / 32;
-        const int zero_end = ksteps * 32;
-        uint8_t* vt = sV + st * Lay::kTileBytes;
-        if (valid < zero_end) {
-          for (int i = lane; i < (zero_end - valid) * 8; i += 32) {
-            const int row = valid + i / 8, ch = i % 8;
-            *reinterpret_cast<uint4*>(vt + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+      // Two streams of MMAs, issued as their inputs arrive: the scores of
+      // tile ns (up to two tiles ahead: S has two buffers) once its K stage
+      // is full and its S buffer free, and P V of tile np once P and the V
+      // stage are ready.  Neither waits behind the other, so a late K tile
+      // does not hold back the P V that the softmax needs before its next P.
+      // The warp polls (every lane tests, so each one has observed a phase
+      // before it touches the data behind it); a poll that sees no progress
+      // for kWaitLimitCycles flags a timeout.
+      int32_t ns = 0, np = 0;
+      long long idle_since = -1;
+      while (np < w.ntiles) {
+        bool progress = false;
+        if (np < ns) {
+          const uint32_t cc = c0 + np;
+          const int st = cc % ST;
+          if (__all_sync(0xffffffffu, mbar_test(p_full, pc & 1) &&
+                                          mbar_test(&v_full[st], (cc / ST) & 1))) {
+            ++pc;
+            // keys of this tile inside the context; P V runs over whole 32-key
+            // steps, the value rows past the context within them are zeroed first
+            const int32_t valid = min(kTcKeys, w.end - (w.blk_begin + np * kTcBlocks) * kBlock);
+            const int ksteps = (valid + 31) / 32;
+            const int zero_end = ksteps * 32;
+            uint8_t* vt = sV + st * Lay::kTileBytes;
+            if (valid < zero_end) {
+              for (int i = lane; i < (zero_end - valid) * 8; i += 32) {
+                const int row = valid + i / 8, ch = i % 8;
+                *reinterpret_cast<uint4*>(vt + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              for (int kk = 0; kk < ksteps; ++kk)
+                umma_f8(tmem + kTcTmemO,
+                        umma_desc(v_base + st * Lay::kTileBytes + kk * 4096, 16384, 1024, 2),
+                        umma_desc(p_base + kk * 1024, 16, 256, 6), idesc_o,
+                        (np > 0 || kk > 0) ? 1u : 0u);
+              umma_commit(&v_empty[st]);
+              umma_commit(o_done);
+            }
+            __syncwarp();
+            ++np;
+            progress = true;
           }
-          fence_proxy_async_smem();
-          __syncwarp();
         }
-        tc_fence_after();
-        if (lane == 0) {
-          for (int kk = 0; kk < ksteps; ++kk)
-            umma_f8(tmem + kTcTmemO, umma_desc(v_base + st * Lay::kTileBytes + kk * 4096, 16384, 1024, 2),
-                    umma_desc(p_base + kk * 1024, 16, 256, 6), idesc_o,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&v_empty[st]);
-          umma_commit(o_done);
+        if (ns < w.ntiles && ns <= np + 2) {
+          const uint32_t cc = c0 + ns;
+          const int st = cc % ST;
+          const int sb = sc & 1;
+          if (__all_sync(0xffffffffu, mbar_test(&k_full[st], (cc / ST) & 1) &&
+                                          (sc < 2 || mbar_test(&s_free[sb], ((sc >> 1) + 1) & 1)))) {
+            tc_fence_after();
+            if (lane == 0) {
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                umma_f8(tmem + sb * kTcN,
+                        umma_desc(k_base + st * Lay::kTileBytes + ks * 32, 16, 1024, 2),
+                        umma_desc(bq_base + b * Lay::kBqBytes + ks * 32, 16, 1024, 2), idesc_s,
+                        ks > 0 ? 1u : 0u);
+              umma_commit(&s_full[sb]);
+              umma_commit(&k_empty[st]);
+              if (ns + 1 == w.ntiles) umma_commit(&bq_empty[b]);  // the unit's last scores read Bq
+            }
+            __syncwarp();
+            ++sc;
+            ++ns;
+            progress = true;
+          }
         }
-        __syncwarp();
+        if (progress) {
+          idle_since = -1;
+        } else if (idle_since < 0) {
+          idle_since = clock64();
+        } else if (clock64() - idle_since > kWaitLimitCycles) {
+          if (lane == 0) raise_error(PKV_DEVERR_TIMEOUT);
+          ok = false;
+          break;
+        }
       }
+      if (!ok) break;
       c = c0 + w.ntiles;
     }
     if (lane == 0) {
