@@ -56,7 +56,10 @@ FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 # (128-row query tiles); shorter ones on the decode kernel (at most 16 rows per item).
 PREFILL_MIN_ROWS = 64
 L2_BYTES = 126 << 20       # B200 L2; working sets below 4x this are flushed between steps
-DECODE_SOURCES = ["pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"]
+# the sources of every kernel a step can launch and of their launch configuration: a
+# recorded traffic figure holds only for the code it was taken on
+DECODE_SOURCES = ["pkv_decode.cuh", "pkv_decode_warp.cuh", "pkv_decode_fp8tc.cuh",
+                  "pkv_prefill.cuh", "pkv_device.cuh", "pkv_api.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")  # JSON text
 
 
@@ -104,15 +107,20 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
-    the current decode sources and this workload; else None."""
+def traffic_key(workload: str, partition: int) -> str:
+    """The traffic record of a workload (and an explicit partition size, when given)."""
+    return workload if not partition else f"{workload}@{partition}"
+
+
+def recorded_traffic(key: str):
+    """DRAM bytes per launch of the step's dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel sources and this workload; else None."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    entry = rec.get(workload)
+    entry = rec.get(key)
     if not entry or entry.get("source_hash") != decode_source_hash():
         return None
     return entry.get("dram_bytes_per_launch")
@@ -521,6 +529,23 @@ def run_ours(args, world, rank, local):
     return result
 
 
+def dominant_kernel(step: Step) -> str:
+    """The kernel the library launches for the step's attention (the dispatch of
+    run_decode and pkv_paged_prefill in pkv_api.cu, restated)."""
+    b = step.b
+    if step.prefill:
+        return "prefill_kernel"
+    g = b.num_q_heads // b.num_kv_heads
+    one_token = not step.multi or b.max_query_len == 1
+    if b.dtype == "fp8" and one_token and not step.shared and g <= 16:
+        return "decode_fp8tc_kernel"
+    rows = (16 // g) * g if step.shared else g
+    if (b.dtype == "bf16" and b.head_dim == 128 and one_token and rows <= 16
+            and step.part_tokens // 16 <= 128 and (step.split or step.shared)):
+        return "decode_warp_kernel"
+    return "decode_kernel"
+
+
 def roofline(step: Step, alg: dict, decode_ms: float, peak: float, peak_kind: str,
              workload: str) -> dict:
     """The dominant kernel against its roofline: HBM for decode (algorithmic bytes per
@@ -531,19 +556,21 @@ def roofline(step: Step, alg: dict, decode_ms: float, peak: float, peak_kind: st
         burst, sustained, kind = tensor_peak()
         flops = attention_flops(step.b)
         tf = flops / (decode_ms / 1e3) / 1e12
-        return {"kernel": "prefill_kernel (tcgen05, TMEM accumulators)", "bound": "tensor",
+        return {"kernel": "prefill_kernel", "bound": "tensor",
                 "achieved": round(tf, 2), "peak": burst,
                 "peak_kind": f"{kind} bf16_tflops (dense, burst)", "unit": "TFLOP/s",
                 "frac": round(tf / burst, 4), "frac_of_sustained": round(tf / sustained, 4),
-                "peak_sustained": sustained, "traffic": recorded_traffic(workload),
+                "peak_sustained": sustained,
+                "traffic": recorded_traffic(traffic_key(workload, step.partition)),
                 "algorithmic_flops_per_launch": flops,
                 "hbm": {"achieved_GBps": round(gbs, 2), "peak": peak,
                         "frac": round(gbs / peak, 4)},
                 "algorithmic_bytes_per_launch": alg}
-    return {"kernel": "decode_kernel" + (" + merge_kernel" if step.split else ""),
+    return {"kernel": dominant_kernel(step) + (" + merge_kernel" if step.split else ""),
             "bound": "hbm", "achieved": round(gbs, 2), "peak": peak,
             "peak_kind": f"{peak_kind} hbm_gbs (copy bandwidth)", "unit": "GB/s",
-            "frac": round(gbs / peak, 4), "traffic": recorded_traffic(workload),
+            "frac": round(gbs / peak, 4),
+            "traffic": recorded_traffic(traffic_key(workload, step.partition)),
             "algorithmic_bytes_per_launch": alg}
 
 

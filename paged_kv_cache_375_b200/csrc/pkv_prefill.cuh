@@ -513,77 +513,99 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!warp_wait(q_full, qc & 1)) { ok = false; break; }
       ++qc;
       const uint32_t kv0 = kvc;
-      // S_j = Q K_j^T into S buffer sc % 2
-      auto issue_s = [&](int32_t j) -> bool {
-        const uint32_t c = kv0 + j;
-        const int st = c % kPfKStages;
-        if (!warp_wait(&k_full[st], (c / kPfKStages) & 1)) return false;
-        const int sb = sc & 1;
-        if (sc >= 2 && !warp_wait(&s_free[sb], ((sc >> 1) + 1) & 1)) return false;
-        tc_fence_after();
-        if (lane == 0) {
+      // Two streams of MMAs, issued as their inputs arrive: S_ns = Q K_ns^T
+      // into S buffer sc % 2 (up to two tiles ahead of P V: S has two
+      // buffers) and O += P_np V_np.  Neither waits behind the other, so a
+      // finished P goes to the tensor core at once.  Every lane tests the
+      // barriers, so each one has observed a phase before it touches the data
+      // behind it; no progress for kWaitLimitCycles flags a timeout.
+      int32_t ns = 0, np = 0;
+      long long idle_since = -1;
+      while (np < w.ntiles) {
+        bool progress = false;
+        if (np < ns) {
+          const uint32_t c = kv0 + np;
+          const int st = c % kPfVStages;
+          if (__all_sync(0xffffffffu, mbar_test(p_full, pc & 1) &&
+                                          mbar_test(&v_full[st], (c / kPfVStages) & 1))) {
+            ++pc;
+            const int32_t j = np;
+            const int32_t nblk =
+                min(kPfBlocksPerTile, (w.nkv - j * kPfKeys + kBlock - 1) / kBlock);
+            // value rows past the context in the context's last block: zero them
+            // (their weights are zero, but NaN or Inf there would still poison O)
+            const int32_t last_blk = (w.L - 1) / kBlock;
+            const int32_t tail = w.L % kBlock;
+            if (tail != 0 && last_blk >= j * kPfBlocksPerTile &&
+                last_blk < j * kPfBlocksPerTile + nblk) {
+              const int b = last_blk - j * kPfBlocksPerTile;
+              const int nrows = kBlock - tail;
+              for (int i = lane; i < nrows * 8 * H; i += 32) {
+                const int h = i / (nrows * 8);
+                const int rr = (i / 8) % nrows + tail;
+                const int chunk = i % 8;
+                *reinterpret_cast<uint4*>(sV + st * Lay::kKvBytes + h * (kPfKeys * 128) +
+                                          (b * kBlock + rr) * 128 + chunk * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              for (int b = 0; b < nblk; ++b) {
+                // A = P from tensor memory: the 16 keys of block b are columns 8b .. 8b+7
+                const uint32_t voff = b * (kBlock * 128);
+                umma_f16_tmem_a(tmem + kPfTmemO, tmem + kPfTmemP + b * (kBlock / 2),
+                                umma_desc_sw128(v_base + st * Lay::kKvBytes + voff,
+                                                kPfKeys * 128, 1024),
+                                idesc_o, (j > 0 || b > 0) ? 1u : 0u);
+              }
+              umma_commit(&v_empty[st]);
+              umma_commit(o_done);
+            }
+            __syncwarp();
+            ++np;
+            progress = true;
+          }
+        }
+        if (ns < w.ntiles && ns <= np + 2) {
+          const uint32_t c = kv0 + ns;
+          const int st = c % kPfKStages;
+          const int sb = sc & 1;
+          if (__all_sync(0xffffffffu, mbar_test(&k_full[st], (c / kPfKStages) & 1) &&
+                                          (sc < 2 || mbar_test(&s_free[sb], ((sc >> 1) + 1) & 1)))) {
+            tc_fence_after();
+            if (lane == 0) {
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * (kPfRows * 128) + (ks & 3) * 32;
-            const uint32_t koff = (ks >> 2) * (kPfKeys * 128) + (ks & 3) * 32;
-            umma_f16(tmem + sb * kPfKeys, umma_desc_sw128(q_base + off, 16, 1024),
-                     umma_desc_sw128(k_base + st * Lay::kKvBytes + koff, 16, 1024), idesc_s,
-                     ks > 0 ? 1u : 0u);
+              for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t off = (ks >> 2) * (kPfRows * 128) + (ks & 3) * 32;
+                const uint32_t koff = (ks >> 2) * (kPfKeys * 128) + (ks & 3) * 32;
+                umma_f16(tmem + sb * kPfKeys, umma_desc_sw128(q_base + off, 16, 1024),
+                         umma_desc_sw128(k_base + st * Lay::kKvBytes + koff, 16, 1024), idesc_s,
+                         ks > 0 ? 1u : 0u);
+              }
+              umma_commit(&s_full[sb]);
+              umma_commit(&k_empty[st]);  // the K tile is free once the scores are
+              if (ns + 1 == w.ntiles) umma_commit(q_empty);  // the unit's last S reads Q
+            }
+            __syncwarp();
+            ++sc;
+            ++ns;
+            progress = true;
           }
-          umma_commit(&s_full[sb]);
-          umma_commit(&k_empty[st]);  // the K tile is free once the scores are
         }
-        __syncwarp();
-        ++sc;
-        return true;
-      };
-      if (w.ntiles > 0 && !issue_s(0)) { ok = false; break; }
-      for (int32_t j = 0; j < w.ntiles; ++j) {
-        if (j + 1 < w.ntiles && !issue_s(j + 1)) { ok = false; break; }
-        if (j + 1 == w.ntiles) {
-          if (lane == 0) umma_commit(q_empty);  // the unit's last S reads Q
-          __syncwarp();
+        if (progress) {
+          idle_since = -1;
+        } else if (idle_since < 0) {
+          idle_since = clock64();
+        } else if (clock64() - idle_since > kWaitLimitCycles) {
+          if (lane == 0) raise_error(PKV_DEVERR_TIMEOUT);
+          ok = false;
+          break;
         }
-        const uint32_t c = kv0 + j;
-        const int st = c % kPfVStages;
-        if (!warp_wait(p_full, pc & 1)) { ok = false; break; }
-        ++pc;
-        if (!warp_wait(&v_full[st], (c / kPfVStages) & 1)) { ok = false; break; }
-        const int32_t nblk = min(kPfBlocksPerTile, (w.nkv - j * kPfKeys + kBlock - 1) / kBlock);
-        // value rows past the context in the context's last block: zero them
-        // (their weights are zero, but NaN or Inf there would still poison O)
-        const int32_t last_blk = (w.L - 1) / kBlock;
-        const int32_t tail = w.L % kBlock;
-        if (tail != 0 && last_blk >= j * kPfBlocksPerTile &&
-            last_blk < j * kPfBlocksPerTile + nblk) {
-          const int b = last_blk - j * kPfBlocksPerTile;
-          const int nrows = kBlock - tail;
-          for (int i = lane; i < nrows * 8 * H; i += 32) {
-            const int h = i / (nrows * 8);
-            const int rr = (i / 8) % nrows + tail;
-            const int chunk = i % 8;
-            *reinterpret_cast<uint4*>(sV + st * Lay::kKvBytes + h * (kPfKeys * 128) +
-                                      (b * kBlock + rr) * 128 + chunk * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          for (int b = 0; b < nblk; ++b) {
-            // A = P from tensor memory: the 16 keys of block b are columns 8b .. 8b+7
-            const uint32_t voff = b * (kBlock * 128);
-            umma_f16_tmem_a(tmem + kPfTmemO, tmem + kPfTmemP + b * (kBlock / 2),
-                            umma_desc_sw128(v_base + st * Lay::kKvBytes + voff, kPfKeys * 128,
-                                            1024),
-                            idesc_o, (j > 0 || b > 0) ? 1u : 0u);
-          }
-          umma_commit(&v_empty[st]);
-          umma_commit(o_done);
-        }
-        __syncwarp();
       }
+      if (!ok) break;
       kvc = kv0 + w.ntiles;
     }
     if (!ok) *abort_flag = 1u;
