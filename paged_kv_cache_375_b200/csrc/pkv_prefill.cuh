@@ -18,30 +18,33 @@
 //   S  = Q K^T   (M 128 rows, N 128 keys, K = head_dim)   into TMEM
 //   O += P V     (M 128 rows, N = head_dim, K = 128 keys) into TMEM
 //
-// Roles in a CTA of 8 warps (one CTA per SM, persistent over work units):
+// Roles in a CTA of 12 warps (one CTA per SM, persistent over work units):
 //  * warps 0 and 2, one lane each: TMA producers.  Warp 0 loads the unit's Q
 //    tile (a 3-D tensor map over q [T][Hq][D], box {64 d, g heads, tokens})
 //    and, per KV tile of 128 keys, the tile's 8 blocks of K through the block
 //    table (the 2-D pool map, one box per block and 64-column half); warp 2
-//    does the same for V.  Stages are 128-byte swizzled, laid out [half][128 keys][128 B]; a
-//    K stage is released when its scores are computed, a V stage when its
-//    P V is.
+//    does the same for V.  Stages are 128-byte swizzled, laid out
+//    [half][128 keys][128 B]; a K stage is released when its scores are
+//    computed, a V stage when its P V is.
 //  * warp 1: TMEM allocation; one lane issues the MMAs and commits them to
-//    mbarriers; the warp zeroes the value rows past the context in the last
-//    block of the context (NaN padding times a zero weight is still NaN on a
-//    tensor core).
+//    mbarriers, polling two streams (the scores of the next tiles, P V of the
+//    tile whose P is ready) so that neither waits behind the other; the warp
+//    zeroes the value rows past the context in the last block of the context
+//    (NaN padding times a zero weight is still NaN on a tensor core).
 //  * warps 4-11 (two warpgroups; warp w reads TMEM lanes 32(w%4) ...): softmax.
 //    Query row r belongs to one thread of each warpgroup, which take keys 0-63
 //    and 64-127 of every tile.  Each reads its 64 scores from TMEM, masks keys
 //    past the row's causal limit, swaps its maximum with its partner through
 //    shared memory, keeps a running maximum in log2 units that moves only when
 //    it grows by more than 8 (the output row in TMEM is then rescaled, each
-//    thread its half of the columns), writes its half of P in bf16 into shared
-//    memory (the A operand of P V) and sums its weights.  At the end the two
-//    sums are added, and each thread reads its half of the output row from
+//    thread its half of the columns), writes its half of P in bf16 pairs into
+//    tensor memory (the A operand of P V) and sums its weights.  At the end the
+//    two sums are added, and each thread reads its half of the output row from
 //    TMEM, divides by the sum and stores bf16.
-// S is double-buffered in TMEM, so the MMA of the next tile's scores runs
-// while the softmax works on this tile's.
+// TMEM: S double-buffered at columns 0 and 128 (the MMA of the next tile's
+// scores runs while the softmax works on this tile's), O at 256, P
+// double-buffered at 384 and 448 (the softmax writes the next tile's P while
+// the tensor core still reads this one's).
 #pragma once
 
 #include "pkv_device.cuh"
@@ -56,9 +59,9 @@ constexpr int kPfVStages = 2;      // V tile stages
 constexpr int kPfThreads = 384;    // warps 0, 2 producers, warp 1 MMA, warps 4-11 softmax
 constexpr int kPfSoftmaxWarps = 8;  // two warpgroups: keys 0-63 and 64-127 of every row
 constexpr int kPfMaxSeqs = 2048;   // sequences per call (per-CTA tile prefix in shared memory)
-constexpr uint32_t kPfTmemCols = 512;  // S buffers at columns 0 and 128, O at 256, P at 384
+constexpr uint32_t kPfTmemCols = 512;  // S buffers at columns 0 and 128, O at 256, P at 384 and 448
 constexpr uint32_t kPfTmemO = 2 * kPfKeys;        // O: head_dim columns of fp32
-constexpr uint32_t kPfTmemP = 3 * kPfKeys;        // P: bf16 pairs, kPfKeys / 2 columns
+constexpr uint32_t kPfTmemP = 3 * kPfKeys;        // P: two buffers of bf16 pairs, kPfKeys / 2 columns each
 constexpr float kPfRescaleSlack = 8.f; // the running max moves when it grows by more (log2)
 
 struct PrefillParams {
@@ -84,8 +87,9 @@ struct PfLayout {
   static constexpr int kPrefixOff = kVOff + kPfVStages * kKvBytes;
   static constexpr int kBarsOff = kPrefixOff + (kPfMaxSeqs + 8) * 4;
   // q_full, q_empty, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2],
-  // s_free[2], p_full, o_done, final, xchg[4] (the two softmax warps of each row quarter)
-  static constexpr int kNumBars = 2 + 2 * kPfKStages + 2 * kPfVStages + 4 + 3 + 4;
+  // s_free[2], p_full[2], pv_done[2], final, xchg[4] (the two softmax warps of each row
+  // quarter)
+  static constexpr int kNumBars = 2 + 2 * kPfKStages + 2 * kPfVStages + 4 + 5 + 4;
   static constexpr int kMiscOff = kBarsOff + kNumBars * 8;     // tmem base, abort flag
   // row maxima exchanged between the two softmax warpgroups: [parity][half][row],
   // then the row sums [half][row]
@@ -340,8 +344,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* s_full = v_empty + kPfVStages;
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* fin = o_done + 1;
+  // [tile & 1]: the softmax warps have written that tile's P.  One barrier per
+  // P buffer: the warps of different row quarters may be a tile apart.
+  uint64_t* pv_done = p_full + 2;  // [tile & 1]: that tile's P V has completed
+  uint64_t* fin = pv_done + 2;
   uint64_t* xchg = fin + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Lay::kMiscOff);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -362,8 +368,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], kPfSoftmaxWarps);
     }
-    mbar_init(p_full, kPfSoftmaxWarps);
-    mbar_init(o_done, 1);
+    mbar_init(&p_full[0], kPfSoftmaxWarps);
+    mbar_init(&p_full[1], kPfSoftmaxWarps);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(fin, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&xchg[i], 2);
     *abort_flag = 0u;
@@ -506,7 +514,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     constexpr uint32_t idesc_o = umma_idesc_bf16(kPfRows, D, true);
     const uint32_t q_base = smem_addr(sQ);
     const uint32_t k_base = smem_addr(sK), v_base = smem_addr(sV);
-    uint32_t qc = 0, kvc = 0, sc = 0, pc = 0;
+    uint32_t qc = 0, kvc = 0, sc = 0;
     bool ok = true;
     for (int32_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       const PfUnit w = pf_unit(p, prefix, u);
@@ -526,9 +534,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (np < ns) {
           const uint32_t c = kv0 + np;
           const int st = c % kPfVStages;
-          if (__all_sync(0xffffffffu, mbar_test(p_full, pc & 1) &&
+          if (__all_sync(0xffffffffu, mbar_test(&p_full[c & 1], (c >> 1) & 1) &&
                                           mbar_test(&v_full[st], (c / kPfVStages) & 1))) {
-            ++pc;
             const int32_t j = np;
             const int32_t nblk =
                 min(kPfBlocksPerTile, (w.nkv - j * kPfKeys + kBlock - 1) / kBlock);
@@ -556,13 +563,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               for (int b = 0; b < nblk; ++b) {
                 // A = P from tensor memory: the 16 keys of block b are columns 8b .. 8b+7
                 const uint32_t voff = b * (kBlock * 128);
-                umma_f16_tmem_a(tmem + kPfTmemO, tmem + kPfTmemP + b * (kBlock / 2),
+                umma_f16_tmem_a(tmem + kPfTmemO,
+                                tmem + kPfTmemP + (c & 1) * (kPfKeys / 2) + b * (kBlock / 2),
                                 umma_desc_sw128(v_base + st * Lay::kKvBytes + voff,
                                                 kPfKeys * 128, 1024),
                                 idesc_o, (j > 0 || b > 0) ? 1u : 0u);
               }
               umma_commit(&v_empty[st]);
-              umma_commit(o_done);
+              umma_commit(&pv_done[c & 1]);
             }
             __syncwarp();
             ++np;
@@ -634,7 +642,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const float sc_log2 = p.qk_scale_log2;
     const int32_t rows_used = g * p.tokens_per_tile;
     const int i_tok = r / g, h_in = r - (r / g) * g;
-    uint32_t sc = 0, od = 0;
+    uint32_t sc = 0;
     bool ok = true;
     for (int32_t u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
       const PfUnit w = pf_unit(p, prefix, u);
@@ -647,6 +655,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       float m = -INFINITY, l = 0.f;
       for (int32_t j = 0; j < w.ntiles; ++j) {
         const int sb = sc & 1;
+        const uint32_t t = sc;  // this tile's place in the CTA's sequence of tiles
         if (!warp_wait(&s_full[sb], (sc >> 1) & 1)) { ok = false; break; }
         ++sc;
         tc_fence_after();
@@ -703,14 +712,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const float lsum = ((lsp[0] + lsp[1]) + (lsp[2] + lsp[3])) +
                            ((lsp[4] + lsp[5]) + (lsp[6] + lsp[7]));
         l = l * alpha + lsum;
-        // P and O may be touched only once the previous tile's P V has completed
-        if (j > 0) {
-          if (!warp_wait(o_done, od & 1)) { ok = false; break; }
-          ++od;
+        // P buffer t & 1 is free once P V of tile t - 2 has completed (tile k's
+        // P V completes phase k / 2 of pv_done[k & 1]); O may be rescaled only
+        // once P V of tile t - 1 has
+        if (t >= 2) {
+          if (!warp_wait(&pv_done[t & 1], ((t - 2) >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
+        }
+        if (j > 0) {
           // rows whose maximum moved rescale their output columns (warp-uniform:
           // the other rows of the warp multiply by 1)
           if (__any_sync(0xffffffffu, grow)) {
+            if (!warp_wait(&pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < DH / 32; ++c) {
               float o[32];
@@ -725,11 +739,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // this half's 64 keys of row r into tensor memory, two bf16 a column
         // (keys 2c and 2c+1 in column c, the lower key in the low half): the
         // A operand of P V
-        tmem_st32u(lane_base + kPfTmemP + half * (KH / 2), pk);
+        tmem_st32u(lane_base + kPfTmemP + (t & 1) * (kPfKeys / 2) + half * (KH / 2), pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[t & 1]);
       }
       if (!ok) break;
       if (w.ntiles > 0) {
@@ -740,8 +754,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!warp_wait(my_xchg, xc & 1)) { ok = false; break; }
         ++xc;
         l += xsum[(half ^ 1) * kPfRows + r];
-        if (!warp_wait(o_done, od & 1)) { ok = false; break; }
-        ++od;
+        // the unit's last P V (tile sc - 1)
+        if (!warp_wait(&pv_done[(sc - 1) & 1], ((sc - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
