@@ -380,8 +380,8 @@ pkv_status launch_decode_fp8tc(const CUtensorMap& mk, const CUtensorMap& mv,
   constexpr int smem = pkv::TcLayout<ST>::kTotal;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_fp8tc)");
-  // persistent: two CTAs per SM with three stages each, else one
-  int64_t grid = static_cast<int64_t>(device_sm_count()) * (ST <= 3 ? 2 : 1);
+  // persistent: two CTAs per SM
+  int64_t grid = static_cast<int64_t>(device_sm_count()) * 2;
   if (grid > work_units) grid = work_units;
   if (grid < 1) grid = 1;
   e = launch(kern, dim3(static_cast<unsigned>(grid)), dim3(pkv::kTcThreads), smem, stream, mk,
@@ -562,12 +562,13 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.out_scale = v_scale;
   const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads *
                         (plan.shared ? 2 : row_groups);
-  if (d->dtype == PKV_FP8_E4M3 && (!query_start_loc || max_query_len == 1) && !plan.shared &&
-      group <= 16) {
-    // one query token per sequence over e4m3 codes: the tensor-core path
-    st = group <= 4   ? launch_decode_fp8tc<4>(mk, mv, prm, units, stream)
-         : group <= 8 ? launch_decode_fp8tc<8>(mk, mv, prm, units, stream)
-                      : launch_decode_fp8tc<16>(mk, mv, prm, units, stream);
+  if (d->dtype == PKV_FP8_E4M3 && !plan.shared && row_groups == 1 && rows_max <= 8) {
+    // e4m3 codes, every sequence's query rows (chunk tokens x group) in one
+    // unit of at most 8: the tensor-core path.  (16-row units ran slower
+    // there than on decode_kernel: the softmax's per-key work grows with the
+    // rows while the bytes stay.)
+    st = rows_max <= 4 ? launch_decode_fp8tc<4>(mk, mv, prm, units, stream)
+                       : launch_decode_fp8tc<8>(mk, mv, prm, units, stream);
   } else if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_FP8_E5M2) {

@@ -19,9 +19,11 @@
 // are likewise 16 high and 16 low columns of the weights.  S and O therefore
 // come out of tensor memory as 32 columns, and s = s_hi + s_lo / 16 (so for O).
 //
-// Roles in a CTA of 8 warps (persistent over work units, the plan's items x kv
-// heads; two CTAs per SM with three K and three V stages each for up to 8
-// query rows, one CTA with six stages for 16):
+// Units of up to 8 query rows (one token per sequence with up to 8 heads per
+// kv head, or chunks of a few tokens: row r = token r / g, head r % g, each
+// token seeing the keys up to its own position).  Roles in a CTA of 8 warps
+// (persistent over work units, the plan's items x kv heads; two CTAs per SM
+// with three K and three V stages each):
 //  * warp 0 (one lane) and warp 2 (one lane): TMA producers of the K and the V
 //    tiles (one box per 16-token block, 128 one-byte codes wide), the next
 //    tile's table entries read ahead.  The K producer also claims the units:
@@ -34,7 +36,7 @@
 //    weight times a NaN code is NaN on a tensor core too);
 //  * warps 4-7: thread t owns key t of every tile (TMEM lane t of S) and column
 //    t of the output (TMEM lane t of O^T).  Per tile it forms the scaled
-//    scores of up to 16 query rows, finds each row's maximum over the 128
+//    scores of the unit's rows, finds each row's maximum over the 128
 //    keys (a reduce-scatter over the warp, then the four warps' maxima meet in
 //    shared memory at a bounded mbarrier), keeps the lazily moved running
 //    maximum of decode_kernel (O^T rescaled in tensor memory when it moves by
@@ -115,12 +117,13 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return f16lo_to_f32(e4m3x2_to_f16x2(code));
 }
 
-// A work unit: planned item x kv head (decode plans: one query token per
-// sequence, or chunks of at most one token).
+// A work unit: planned item x kv head.  Its rows: q_len query tokens (rows
+// q_start .. of q and out, the last q_len positions of the context) x the
+// group's heads, row r = token r / g, head r % g; at most 16.
 struct TcUnit {
   int32_t seq, kv_head, part, len, nparts, blk_begin, nblk, ntiles;
   int32_t end;    // keys at positions < end belong to the unit (its partition's end)
-  int32_t q_row;  // the query token's row of q and out; rows < 0: no query token
+  int32_t q_start, q_len;
 };
 
 __device__ __forceinline__ TcUnit tc_unit(const DecodeParams& prm, int32_t u) {
@@ -132,10 +135,10 @@ __device__ __forceinline__ TcUnit tc_unit(const DecodeParams& prm, int32_t u) {
   w.len = pi.len;
   w.nparts = pi.nparts;
   w.blk_begin = pi.blk0;
-  w.q_row = pi.seq;
+  w.q_start = pi.seq;
   int32_t q_len = 1;
   if (prm.query_start_loc) {
-    // a chunk of at most one token: the scheduler's checks of decode_kernel
+    // a chunk of several tokens: the scheduler's checks of decode_kernel
     const int32_t q0 = prm.query_start_loc[pi.seq];
     q_len = prm.query_start_loc[pi.seq + 1] - q0;
     const int32_t cap = pi.len < prm.max_query_len ? pi.len : prm.max_query_len;
@@ -148,8 +151,9 @@ __device__ __forceinline__ TcUnit tc_unit(const DecodeParams& prm, int32_t u) {
       if (first) raise_error(PKV_DEVERR_LEN);
       q_len = 0;
     }
-    w.q_row = q_len > 0 ? q0 : -1;
+    w.q_start = q0;
   }
+  w.q_len = q_len;
   int32_t nblk = (pi.len + kBlock - 1) / kBlock - pi.blk0;
   nblk = nblk < prm.part_blocks ? nblk : prm.part_blocks;
   w.nblk = (nblk < 0 || q_len == 0) ? 0 : nblk;
@@ -192,16 +196,17 @@ __device__ __forceinline__ float scatter_max(const float (&z)[RM], int lane, int
   return r;
 }
 
-// RM: query rows the softmax handles (4, 8 or 16, at least the group size);
-// the operand layouts always hold 16 high and 16 low rows.
-// Stages per CTA: 3 when two CTAs share an SM (up to 8 query rows), else 6.
+// RM: query rows the softmax handles (4 or 8, at least the unit's rows); the
+// operand layouts hold 16 high and 16 low rows.  ST: K and V stages per CTA,
+// three, with two CTAs per SM.
 template <int RM>
-constexpr int tc_stages() { return RM <= 8 ? 3 : 6; }
+constexpr int tc_stages() { return 3; }
 
 template <int RM, int ST = tc_stages<RM>()>
-__global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
+__global__ void __launch_bounds__(kTcThreads, 2)
     decode_fp8tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
+  static_assert(RM == 4 || RM == 8, "4 or 8 query rows per unit");
   using Lay = TcLayout<ST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -382,13 +387,16 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
       if (n >= 2 && !warp_wait(&bq_empty[b], ((n >> 1) + 1) & 1)) { ok = false; break; }
       uint8_t* bq = sBq + b * Lay::kBqBytes;
       if (lane < kTcRows) {
-        // query row `lane` of the group: high terms in row lane, low in 16 + lane
+        // the unit's row `lane` (token lane / g, head lane % g): high terms in
+        // row lane, low in 16 + lane
         float c = 1.f;
+        const bool live = lane < w.q_len * g;
+        const size_t qrow = live ? static_cast<size_t>(w.q_start + lane / g) * prm.num_q_heads +
+                                       w.kv_head * g + lane % g
+                                 : 0;
         const uint4* src = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(prm.q) +
-            (static_cast<size_t>(w.q_row < 0 ? 0 : w.q_row) * prm.num_q_heads + w.kv_head * g +
-             lane) * 128);
-        if (lane < g && w.q_row >= 0) {
+            static_cast<const __nv_bfloat16*>(prm.q) + qrow * 128);
+        if (live) {
           float mx = 0.f;
 #pragma unroll 4
           for (int i = 0; i < 16; ++i) {
@@ -410,7 +418,7 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
 #pragma unroll 2
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
-          if (lane < g && w.q_row >= 0) {
+          if (live) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
               const uint4 v = src[2 * ch + half];
@@ -558,6 +566,7 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
       if (!take_unit(n, u)) { ok = false; break; }
       if (u < 0) break;
       const TcUnit w = tc_unit(prm, u);
+      const int rows = w.q_len * g;  // the unit's query rows
       const int b = n & 1;
       float m[RM], l[RM], ic[RM];
 #pragma unroll
@@ -582,12 +591,17 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
+        // key pos is seen by the rows of tokens i >= pos - (len - q_len), i.e.
+        // rows r >= thr (all rows for keys before the chunk)
         const int32_t pos = (w.blk_begin + j * kTcBlocks) * kBlock + t;
         const bool in_ctx = pos < w.end;
+        const int32_t thr = (pos - (w.len - w.q_len)) * g;
         float z[RM];
 #pragma unroll
         for (int r = 0; r < RM; ++r)
-          z[r] = (in_ctx && r < g) ? fmaf(s[kTcRows + r], 0.0625f, s[r]) * ic[r] : -INFINITY;
+          z[r] = (in_ctx && r < rows && r >= thr)
+                     ? fmaf(s[kTcRows + r], 0.0625f, s[r]) * ic[r]
+                     : -INFINITY;
         // each row's maximum over the warp's 32 keys: reduce-scatter
         int row;
         const float v1 = scatter_max<RM>(z, lane, row);
@@ -609,14 +623,19 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
           any_grow |= grow;
         }
         // this key's weights, high and low e4m3 terms, and the running sums
+        // two rows at a time: one conversion makes both rows' codes
         uint32_t ph[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int r = 0; r < RM; ++r) {
-          const float mu = m[r] == -INFINITY ? 0.f : m[r];
-          const float p = fast_exp2(z[r] - mu);
-          l[r] = fmaf(l[r], alpha[r], p);
-          const uint32_t hc = e4m3_code(p);
-          const uint32_t lc = e4m3_code((p - e4m3_value(hc)) * 16.f);
+        for (int r = 0; r < RM; r += 2) {
+          const float mu0 = m[r] == -INFINITY ? 0.f : m[r];
+          const float mu1 = m[r + 1] == -INFINITY ? 0.f : m[r + 1];
+          const float p0 = fast_exp2(z[r] - mu0), p1 = fast_exp2(z[r + 1] - mu1);
+          l[r] = fmaf(l[r], alpha[r], p0);
+          l[r + 1] = fmaf(l[r + 1], alpha[r + 1], p1);
+          const uint32_t hc = f32x2_to_e4m3x2(p0, p1);
+          const uint32_t hv = e4m3x2_to_f16x2(hc);
+          const uint32_t lc = f32x2_to_e4m3x2((p0 - f16lo_to_f32(hv)) * 16.f,
+                                              (p1 - f16hi_to_f32(hv)) * 16.f);
           ph[r >> 2] |= hc << (8 * (r & 3));
           pl[r >> 2] |= lc << (8 * (r & 3));
         }
@@ -678,17 +697,18 @@ __global__ void __launch_bounds__(kTcThreads, ST <= 3 ? 2 : 1)
         tc_fence_after();
         tmem_ld32_wait(lane_base + kTcTmemO, o);
       }
-      const size_t row0 = static_cast<size_t>(w.q_row) * prm.num_q_heads + w.kv_head * g;
 #pragma unroll
       for (int r = 0; r < RM; ++r) {
-        if (r < g && w.q_row >= 0) {
+        if (r < rows) {
+          const size_t qrow = static_cast<size_t>(w.q_start + r / g) * prm.num_q_heads +
+                              w.kv_head * g + r % g;
           const float acc = fmaf(o[kTcRows + r], 0.0625f, o[r]);
           const float inv = l[r] > 0.f ? prm.out_scale / l[r] : 0.f;
           if (w.nparts == 1) {
-            reinterpret_cast<uint16_t*>(prm.out)[(row0 + r) * 128 + t] =
+            reinterpret_cast<uint16_t*>(prm.out)[qrow * 128 + t] =
                 static_cast<uint16_t>(pack_bf16x2(acc * inv, 0.f));
           } else {
-            const size_t prow = (row0 + r) * prm.max_parts + w.part;
+            const size_t prow = qrow * prm.max_parts + w.part;
             prm.part_o[prow * 128 + t] = acc * inv;
             if (t == 0) {
               prm.part_ml[prow * 2 + 0] = m[r] == -INFINITY ? -INFINITY : m[r] * kLn2;

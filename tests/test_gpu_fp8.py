@@ -256,7 +256,10 @@ def gpu_fp8_multi(b, partition_tokens=0, plan=False):
     return out
 
 
-@pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 4), (8, 8, 16), (16, 2, 2), (12, 4, 5),
+# chunks x group <= 8 rows run on the tensor-core kernel (the first four), up to
+# 16 on decode_kernel, longer chunks in row groups
+@pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 2), (8, 8, 8), (16, 8, 4), (24, 8, 2),
+                                             (32, 8, 4), (8, 8, 16), (16, 2, 2), (12, 4, 5),
                                              (16, 1, 1), (32, 8, 20), (16, 1, 3)])
 def test_fp8_multi_matches_oracle(cuda_device, hq, hkv, max_chunk):
     rng = np.random.default_rng(hq * 31 + hkv * 7 + max_chunk)
@@ -274,10 +277,13 @@ def test_fp8_multi_matches_oracle(cuda_device, hq, hkv, max_chunk):
     check_close(out, ref, "bf16", f"fp8 multi {hq}/{hkv} chunks<={max_chunk}")
 
 
-@pytest.mark.parametrize("partition", [16, 256])
-def test_fp8_multi_split_k_and_plan_run(cuda_device, partition):
+@pytest.mark.parametrize("partition,chunks", [(16, (4, 3, 4, 1, 2)), (256, (4, 3, 4, 1, 2)),
+                                              (16, (2, 1, 2, 2, 1)), (256, (2, 1, 2, 2, 1))])
+def test_fp8_multi_split_k_and_plan_run(cuda_device, partition, chunks):
+    """Split-K and plan/run for chunks of up to 4 tokens (16 rows: decode_kernel) and of
+    up to 2 (8 rows: the tensor-core kernel)."""
     lens = np.array([40, 300, 1000, 2100, 5])
-    chunks = np.array([4, 3, 4, 1, 2])
+    chunks = np.array(chunks)
     b = workloads.chunked_batch(995 + partition, lens, chunks, 32, 8, 128, "fp8",
                                 device=cuda_device)
     b.k_scale, b.v_scale = workloads.FP8_K_SCALE, workloads.FP8_V_SCALE
