@@ -18,14 +18,14 @@
 //   S  = Q K^T   (M 128 rows, N 128 keys, K = head_dim)   into TMEM
 //   O += P V     (M 128 rows, N = head_dim, K = 128 keys) into TMEM
 //
-// Roles in a CTA of 12 warps (one CTA per SM, persistent over work units):
-//  * warps 0 and 2, one lane each: TMA producers.  Warp 0 loads the unit's Q
-//    tile (a 3-D tensor map over q [T][Hq][D], box {64 d, g heads, tokens})
-//    and, per KV tile of 128 keys, the tile's 8 blocks of K through the block
-//    table (the 2-D pool map, one box per block and 64-column half); warp 2
-//    does the same for V.  Stages are 128-byte swizzled, laid out
-//    [half][128 keys][128 B]; a K stage is released when its scores are
-//    computed, a V stage when its P V is.
+// Roles in a CTA of 13 warps (one CTA per SM, persistent over work units):
+//  * warps 0, 3 (K) and 2, 12 (V), one lane each: TMA producers.  Warp 0
+//    loads the unit's Q tile (a 3-D tensor map over q [T][Hq][D], box {64 d,
+//    g heads, tokens}); per KV tile of 128 keys, warps 0 and 3 load blocks 0-3
+//    and 4-7 of K through the block table (the 2-D pool map, one box per
+//    block and 64-column half), warps 2 and 12 the same of V.  Stages are
+//    128-byte swizzled, laid out [half][128 keys][128 B]; a K stage is
+//    released when its scores are computed, a V stage when its P V is.
 //  * warp 1: TMEM allocation; one lane issues the MMAs and commits them to
 //    mbarriers, polling two streams (the scores of the next tiles, P V of the
 //    tile whose P is ready) so that neither waits behind the other; the warp
@@ -56,7 +56,10 @@ constexpr int kPfKeys = 128;       // keys per KV tile: N of S = Q K^T, K of O +
 constexpr int kPfBlocksPerTile = kPfKeys / kBlock;
 constexpr int kPfKStages = 3;      // K tile stages (a K stage frees as soon as its scores are done)
 constexpr int kPfVStages = 2;      // V tile stages
-constexpr int kPfThreads = 384;    // warps 0, 2 producers, warp 1 MMA, warps 4-11 softmax
+constexpr int kPfThreads = 416;    // warps 0, 3 (K) and 2, 12 (V) producers, warp 1 MMA,
+                                   // warps 4-11 softmax
+constexpr int kPfKProducers = 2;
+constexpr int kPfVProducers = 2;
 constexpr int kPfSoftmaxWarps = 8;  // two warpgroups: keys 0-63 and 64-127 of every row
 constexpr int kPfMaxSeqs = 2048;   // sequences per call (per-CTA tile prefix in shared memory)
 constexpr uint32_t kPfTmemCols = 512;  // S buffers at columns 0 and 128, O at 256, P at 384 and 448
@@ -357,11 +360,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < kPfKStages; ++i) {
-      mbar_init(&k_full[i], 1);
+      mbar_init(&k_full[i], kPfKProducers);  // every producer warp of the stream
       mbar_init(&k_empty[i], 1);
     }
     for (int i = 0; i < kPfVStages; ++i) {
-      mbar_init(&v_full[i], 1);
+      mbar_init(&v_full[i], kPfVProducers);
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -422,15 +425,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int g = p.group;
   const uint32_t qrow_bytes = 128u * static_cast<uint32_t>(g * p.tokens_per_tile);
 
-  if (warp == 0 || warp == 2) {
+  if (warp == 0 || warp == 2 || warp == 3 || warp == 12) {
     // ===================================================== TMA producers
-    // Warp 0 (one lane) loads Q and the K tiles, warp 2 the V tiles: a K
-    // stage is free once the tile's scores are computed, a V stage only once
-    // its P V is, so the next K tiles are not held up behind the current P V.
-    // (Two lanes of one warp would not do: while one waits on its barrier
-    // the other's path does not run.)
+    // Warps 0 and 3 (one lane each) load the K tiles, blocks 0-3 and 4-7 of
+    // each, warp 0 also the Q tile; warps 2 and 12 load the V tiles the same
+    // way.  A K stage is free once the tile's scores are computed, a V stage
+    // only once its P V is, so the next K tiles are not held up behind the
+    // current P V.  Two warps per stream: one warp issues tensor copies at
+    // about 14 bytes a cycle, below what the tile pipeline consumes (four K
+    // and three V warps measured slower again).  (Two lanes of one warp would
+    // not do: while one waits on its barrier the other's path does not run.)
     if (lane == 0) {
-      const bool is_k = warp == 0;
+      const bool is_k = warp == 0 || warp == 3;
+      const int nprod = is_k ? kPfKProducers : kPfVProducers;
+      const int part = (warp == 3 || warp == 12) ? 1 : 0;
       const CUtensorMap* map = is_k ? &map_k : &map_v;
       uint8_t* stage_base = is_k ? sK : sV;
       uint64_t* full_bar = is_k ? k_full : v_full;
@@ -473,8 +481,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(nblk) * H * (kBlock * 128));
-        for (int b = 0; b < nblk; ++b) {
+        // this warp's blocks of the tile: [8 part / nprod, 8 (part + 1) / nprod)
+        const int b0 = part * kPfBlocksPerTile / nprod;
+        const int b1 = min(nblk, (part + 1) * kPfBlocksPerTile / nprod);
+        mbar_arrive_expect_tx(&full_bar[st],
+                              static_cast<uint32_t>(max(b1 - b0, 0)) * H * (kBlock * 128));
+        for (int b = b0; b < b1; ++b) {
           int32_t pb = rows[b];
           if (pb < 0 || pb >= p.num_blocks) {
             if (is_k) raise_error(PKV_DEVERR_BLOCK);
@@ -488,7 +500,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         map, h * 64, y, &full_bar[st]);
         }
         ++kvc;
-        if (is_k && j == 0) {
+        if (is_k && part == 0 && j == 0) {
           // the unit's Q tile, once the previous unit's last scores are done
           // (its first K tile is already on its way)
           if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1)) { ok = false; break; }

@@ -164,3 +164,13 @@ def test_rejects_what_it_does_not_run(cuda_device):
     assert pkv.STATUS_NAMES[st] == "PKV_ERR_UNSUPPORTED"
     with pytest.raises(TypeError):
         gpu_prefill(b)
+
+
+def test_many_sequences(cuda_device):
+    """More sequences than the two-tile kernel's prefix holds (256): the one-tile
+    kernel serves the call, with the same results."""
+    rng = np.random.default_rng(3100)
+    lens = rng.integers(1, 200, size=300)
+    chunks = np.minimum(rng.integers(1, 150, size=300), lens)
+    b = workloads.chunked_batch(3100, lens, chunks, 32, 8, 128, "bf16", device=cuda_device)
+    run_and_check(b, "300 sequences")
