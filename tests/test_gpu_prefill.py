@@ -167,8 +167,8 @@ def test_rejects_what_it_does_not_run(cuda_device):
 
 
 def test_many_sequences(cuda_device):
-    """More sequences than the two-tile kernel's prefix holds (256): the one-tile
-    kernel serves the call, with the same results."""
+    """300 short sequences: many units per CTA, the per-CTA tile prefix over all of
+    them, chunks from 1 token to 150."""
     rng = np.random.default_rng(3100)
     lens = rng.integers(1, 200, size=300)
     chunks = np.minimum(rng.integers(1, 150, size=300), lens)
