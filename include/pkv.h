@@ -373,13 +373,13 @@ pkv_status pkv_decode_prepare_tokens(const void *k, const void *v, void *k_cache
  *    even, saturate to +-448); slots as in pkv_reshape_and_cache.
  *  - pkv_paged_attention_decode_fp8 / pkv_decode_run_fp8: as the bf16 calls,
  *    over e4m3 pools with their k_scale and v_scale; q and out are bf16.
- *    Arithmetic over e4m3 pools, one query token per sequence: the codes
- *    enter the tensor cores as they are, q (times a power of two per row)
- *    and the softmax weights as two e4m3 terms each (the rounded value and
- *    16 x its rounding remainder, about 8 significant bits), products
- *    accumulate in fp32.  Over e5m2 pools, and for several query tokens or
- *    shared prefixes: codes are widened exactly to f16, q is rounded to f16
- *    (|q| above 65504 saturates), products accumulate in fp32.
+ *    Arithmetic when a sequence's query rows (chunk tokens x heads per kv
+ *    head) number at most 8 and there is no shared prefix: the codes (e4m3
+ *    or e5m2) enter the tensor cores as they are, q (times a power of two per
+ *    row) and the softmax weights as two e4m3 terms each (the rounded value
+ *    and 16 x its rounding remainder, about 8 significant bits), products
+ *    accumulate in fp32.  Otherwise: codes are widened exactly to f16, q is
+ *    rounded to f16 (|q| above 65504 saturates), products accumulate in fp32.
  * dims->dtype must be PKV_FP8_E4M3 or PKV_FP8_E5M2 (the plain calls reject
  * both; for e5m2 read e5m2 for e4m3 above, saturating to +-57344); copy_blocks,
  * slot mapping and the planner work on FP8 pools unchanged.

@@ -369,14 +369,14 @@ pkv_status launch_decode_warp(const CUtensorMap& mk, const CUtensorMap& mv,
   return PKV_OK;
 }
 
-// Decode over e4m3 pools on the tcgen05 tensor cores (one query token per
-// sequence, plain or split-K plans).
-template <int RM>
+// Decode over FP8 pools on the tcgen05 tensor cores (units of up to RM query
+// rows, plain or split-K plans); AF: 0 e4m3 pools, 1 e5m2.
+template <int RM, int AF>
 pkv_status launch_decode_fp8tc(const CUtensorMap& mk, const CUtensorMap& mv,
                                const pkv::DecodeParams& prm, int64_t work_units,
                                cudaStream_t stream) {
   constexpr int ST = pkv::tc_stages<RM>();
-  auto kern = pkv::decode_fp8tc_kernel<RM, ST>;
+  auto kern = pkv::decode_fp8tc_kernel<RM, AF, ST>;
   constexpr int smem = pkv::TcLayout<ST>::kTotal;
   cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_fp8tc)");
@@ -562,13 +562,17 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.out_scale = v_scale;
   const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads *
                         (plan.shared ? 2 : row_groups);
-  if (d->dtype == PKV_FP8_E4M3 && !plan.shared && row_groups == 1 && rows_max <= 8) {
-    // e4m3 codes, every sequence's query rows (chunk tokens x group) in one
+  if (is_fp8(d->dtype) && !plan.shared && row_groups == 1 && rows_max <= 8) {
+    // FP8 codes, every sequence's query rows (chunk tokens x group) in one
     // unit of at most 8: the tensor-core path.  (16-row units ran slower
     // there than on decode_kernel: the softmax's per-key work grows with the
     // rows while the bytes stay.)
-    st = rows_max <= 4 ? launch_decode_fp8tc<4>(mk, mv, prm, units, stream)
-                       : launch_decode_fp8tc<8>(mk, mv, prm, units, stream);
+    if (d->dtype == PKV_FP8_E4M3)
+      st = rows_max <= 4 ? launch_decode_fp8tc<4, 0>(mk, mv, prm, units, stream)
+                         : launch_decode_fp8tc<8, 0>(mk, mv, prm, units, stream);
+    else
+      st = rows_max <= 4 ? launch_decode_fp8tc<4, 1>(mk, mv, prm, units, stream)
+                         : launch_decode_fp8tc<8, 1>(mk, mv, prm, units, stream);
   } else if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_FP8_E5M2) {

@@ -103,12 +103,15 @@ __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_
       : "memory");
 }
 
-// Instruction descriptor of kind::f8f6f4, e4m3 x e4m3 -> fp32 (bits 4-5 = 1,
-// A and B formats 0), A / B major (bits 15 / 16: 1 = MN-major), N >> 3 in
-// bits 17-22, M >> 4 in bits 24-28.
-__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// Instruction descriptor of kind::f8f6f4 -> fp32 (bits 4-5 = 1): A's format
+// in bits 7-9 (0 e4m3, 1 e5m2; the instruction takes A's and B's formats
+// separately), B e4m3 (bits 10-12 = 0), A / B major (bits 15 / 16: 1 =
+// MN-major), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t umma_idesc_f8(int M, int N, int a_fmt, bool a_mn,
+                                                     bool b_mn) {
+  return (1u << 4) | (static_cast<uint32_t>(a_fmt) << 7) | (a_mn ? (1u << 15) : 0u) |
+         (b_mn ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // e4m3 code of x (round to nearest even, saturating) and its value.
@@ -202,11 +205,13 @@ __device__ __forceinline__ float scatter_max(const float (&z)[RM], int lane, int
 template <int RM>
 constexpr int tc_stages() { return 3; }
 
-template <int RM, int ST = tc_stages<RM>()>
+// AF: the pools' code format, A of both products (0 e4m3, 1 e5m2).
+template <int RM, int AF, int ST = tc_stages<RM>()>
 __global__ void __launch_bounds__(kTcThreads, 2)
     decode_fp8tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
   static_assert(RM == 4 || RM == 8, "4 or 8 query rows per unit");
+  static_assert(AF == 0 || AF == 1, "e4m3 or e5m2 pools");
   using Lay = TcLayout<ST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -446,8 +451,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
   } else if (warp == 1) {
     // ===================================================== MMA issue
-    constexpr uint32_t idesc_s = umma_idesc_e4m3(kTcKeys, kTcN, false, false);
-    constexpr uint32_t idesc_o = umma_idesc_e4m3(128, kTcN, true, true);
+    constexpr uint32_t idesc_s = umma_idesc_f8(kTcKeys, kTcN, AF, false, false);
+    constexpr uint32_t idesc_o = umma_idesc_f8(128, kTcN, AF, true, true);
     const uint32_t k_base = smem_addr(sK), v_base = smem_addr(sV);
     const uint32_t bq_base = smem_addr(sBq), p_base = smem_addr(sP);
     uint32_t n = 0, c = 0, sc = 0, pc = 0;
