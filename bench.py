@@ -538,7 +538,7 @@ def dominant_kernel(step: Step) -> str:
     g = b.num_q_heads // b.num_kv_heads
     one_token = not step.multi or b.max_query_len == 1
     chunk_rows = (b.max_query_len if step.multi else 1) * g
-    if b.dtype in ("fp8", "fp8e5m2") and not step.shared and chunk_rows <= 8:
+    if b.dtype in ("fp8", "fp8e5m2") and not step.shared and chunk_rows <= 16:
         return "decode_fp8tc_kernel"
     rows = (16 // g) * g if step.shared else g
     if (b.dtype == "bf16" and b.head_dim == 128 and one_token and rows <= 16

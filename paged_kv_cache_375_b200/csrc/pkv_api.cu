@@ -562,17 +562,17 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   prm.out_scale = v_scale;
   const int64_t units = static_cast<int64_t>(d->num_seqs) * plan.max_parts * d->num_kv_heads *
                         (plan.shared ? 2 : row_groups);
-  if (is_fp8(d->dtype) && !plan.shared && row_groups == 1 && rows_max <= 8) {
-    // FP8 codes, every sequence's query rows (chunk tokens x group) in one
-    // unit of at most 8: the tensor-core path.  (16-row units ran slower
-    // there than on decode_kernel: the softmax's per-key work grows with the
-    // rows while the bytes stay.)
+  if (is_fp8(d->dtype) && !plan.shared && row_groups == 1) {
+    // FP8 codes, every sequence's query rows (chunk tokens x group, at most
+    // 16) in one unit: the tensor-core path
     if (d->dtype == PKV_FP8_E4M3)
-      st = rows_max <= 4 ? launch_decode_fp8tc<4, 0>(mk, mv, prm, units, stream)
-                         : launch_decode_fp8tc<8, 0>(mk, mv, prm, units, stream);
+      st = rows_max <= 4   ? launch_decode_fp8tc<4, 0>(mk, mv, prm, units, stream)
+           : rows_max <= 8 ? launch_decode_fp8tc<8, 0>(mk, mv, prm, units, stream)
+                           : launch_decode_fp8tc<16, 0>(mk, mv, prm, units, stream);
     else
-      st = rows_max <= 4 ? launch_decode_fp8tc<4, 1>(mk, mv, prm, units, stream)
-                         : launch_decode_fp8tc<8, 1>(mk, mv, prm, units, stream);
+      st = rows_max <= 4   ? launch_decode_fp8tc<4, 1>(mk, mv, prm, units, stream)
+           : rows_max <= 8 ? launch_decode_fp8tc<8, 1>(mk, mv, prm, units, stream)
+                           : launch_decode_fp8tc<16, 1>(mk, mv, prm, units, stream);
   } else if (d->dtype == PKV_FP8_E4M3) {
     st = launch_decode_d<pkv::Fp8Kv, 128>(mk, mv, prm, units, rows_max, stream);
   } else if (d->dtype == PKV_FP8_E5M2) {

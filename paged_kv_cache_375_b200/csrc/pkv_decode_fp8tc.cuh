@@ -19,9 +19,10 @@
 // are likewise 16 high and 16 low columns of the weights.  S and O therefore
 // come out of tensor memory as 32 columns, and s = s_hi + s_lo / 16 (so for O).
 //
-// Units of up to 8 query rows (one token per sequence with up to 8 heads per
-// kv head, or chunks of a few tokens: row r = token r / g, head r % g, each
-// token seeing the keys up to its own position).  Roles in a CTA of 8 warps
+// Units of up to 16 query rows (one token per sequence with up to 16 heads
+// per kv head, or chunks of a few tokens, such as the draft tokens of a
+// speculative step: row r = token r / g, head r % g, each token seeing the
+// keys up to its own position).  Roles in a CTA of 8 warps
 // (persistent over work units, the plan's items x kv heads; two CTAs per SM
 // with three K and three V stages each):
 //  * warp 0 (one lane) and warp 2 (one lane): TMA producers of the K and the V
@@ -36,12 +37,15 @@
 //    weight times a NaN code is NaN on a tensor core too);
 //  * warps 4-7: thread t owns key t of every tile (TMEM lane t of S) and column
 //    t of the output (TMEM lane t of O^T).  Per tile it forms the scaled
-//    scores of the unit's rows, finds each row's maximum over the 128
-//    keys (a reduce-scatter over the warp, then the four warps' maxima meet in
-//    shared memory at a bounded mbarrier), keeps the lazily moved running
-//    maximum of decode_kernel (O^T rescaled in tensor memory when it moves by
-//    more than 2^8), accumulates its own share of each row's weight sum,
-//    writes its key's 32 P bytes and arrives.  At the end of a unit the sums
+//    scores of the unit's rows against the lazily moved running maximum of
+//    decode_kernel.  In a tile that every row sees whole, where no score
+//    passes its row's maximum by more than the slack (2^8), the four warps
+//    only exchange one flag; otherwise (a unit's first tile, a masked tile, a
+//    maximum that moves) each row's maximum over the 128 keys is formed (a
+//    reduce-scatter over the warp, then the four warps' maxima meet in shared
+//    memory at a bounded mbarrier) and O^T is rescaled in tensor memory where
+//    it moved.  The thread accumulates its own share of each row's weight
+//    sum, writes its key's 32 P bytes and arrives.  At the end of a unit the sums
 //    are reduced over the 128 threads and each thread writes its output
 //    column (or the partial o / l, m, l of a split sequence).
 // S is double-buffered in tensor memory, so the next tile's scores run on the
@@ -61,6 +65,7 @@ constexpr int kTcN = 2 * kTcRows;                // MMA N: high and low terms
 constexpr int kTcThreads = 256;
 constexpr uint32_t kTcTmemCols = 128;            // S at columns 0 and 32, O^T at 64
 constexpr uint32_t kTcTmemO = 64;
+constexpr float kNoMax = 1e30f;                  // a running maximum not yet set
 
 // ST = K stages = V stages.
 template <int ST>
@@ -73,7 +78,7 @@ struct TcLayout {
   static constexpr int kPOff = kBqOff + 2 * kBqBytes;            // [128 keys][32 B], 32-byte swizzle
   static constexpr int kPBytes = kTcKeys * kTcN;
   static constexpr int kXOff = kPOff + kPBytes;                  // exchange floats
-  // xmax [2][4 warps][16], xsum [2][4][16], inv_c [2][16]
+  // xmax [2][4 warps][16], xsum [2][4][16], row scales [2][16]
   static constexpr int kXFloats = 2 * 4 * kTcRows + 2 * 4 * kTcRows + 2 * kTcRows;
   static constexpr int kRingOff = kXOff + kXFloats * 4;         // unit indices [kTcRing]
   static constexpr int kBarsOff = kRingOff + kTcRing * 4;
@@ -118,6 +123,54 @@ __host__ __device__ constexpr uint32_t umma_idesc_f8(int M, int N, int a_fmt, bo
 __device__ __forceinline__ uint32_t e4m3_code(float x) { return f32x2_to_e4m3x2(x, 0.f) & 0xffu; }
 __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return f16lo_to_f32(e4m3x2_to_f16x2(code));
+}
+
+// The weights p0, p1 of two rows as two-term e4m3 codes, formed in f16x2: the
+// high pair hi = e4m3(p) and the low pair e4m3(16 (p - hi)), p0 in the low
+// byte of each.  p - hi is exact in f16 (hi is p rounded to 4 significant
+// bits), so the pair keeps about 8 bits of each weight, as through f32.
+__device__ __forceinline__ void p_codes2(float p0, float p1, uint32_t& hc, uint32_t& lc) {
+  asm("{\n\t.reg .b32 ph, hv, dl, k16;\n\t.reg .b16 h, l;\n\t"
+      "cvt.rn.f16x2.f32 ph, %3, %2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 h, ph;\n\t"
+      "cvt.rn.f16x2.e4m3x2 hv, h;\n\t"
+      "mov.b32 k16, 0x4C004C00;\n\t"
+      "sub.rn.f16x2 dl, ph, hv;\n\t"
+      "mul.rn.f16x2 dl, dl, k16;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 l, dl;\n\t"
+      "cvt.u32.u16 %0, h;\n\t"
+      "cvt.u32.u16 %1, l;\n\t}"
+      : "=r"(hc), "=r"(lc)
+      : "f"(p0), "f"(p1));
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane: load (waited for in
+// the same statement) and store.
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
 }
 
 // A work unit: planned item x kv head.  Its rows: q_len query tokens (rows
@@ -199,7 +252,7 @@ __device__ __forceinline__ float scatter_max(const float (&z)[RM], int lane, int
   return r;
 }
 
-// RM: query rows the softmax handles (4 or 8, at least the unit's rows); the
+// RM: query rows the softmax handles (4, 8 or 16, at least the unit's rows); the
 // operand layouts hold 16 high and 16 low rows.  ST: K and V stages per CTA,
 // three, with two CTAs per SM.
 template <int RM>
@@ -210,7 +263,7 @@ template <int RM, int AF, int ST = tc_stages<RM>()>
 __global__ void __launch_bounds__(kTcThreads, 2)
     decode_fp8tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, const DecodeParams prm) {
-  static_assert(RM == 4 || RM == 8, "4 or 8 query rows per unit");
+  static_assert(RM == 4 || RM == 8 || RM == 16, "4, 8 or 16 query rows per unit");
   static_assert(AF == 0 || AF == 1, "e4m3 or e5m2 pools");
   using Lay = TcLayout<ST>;
   extern __shared__ uint8_t smem_raw[];
@@ -222,7 +275,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   uint8_t* sP = sm + Lay::kPOff;
   float* xmax = reinterpret_cast<float*>(sm + Lay::kXOff);  // [2][4][16]
   float* xsum = xmax + 2 * 4 * kTcRows;                      // [2][4][16]
-  float* inv_c = xsum + 2 * 4 * kTcRows;                     // [2][16]
+  // [Bq buffer][row]: the score scale of the row in log2 units over its c, 0
+  // for rows past the unit's
+  float* row_sc = xsum + 2 * 4 * kTcRows;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBarsOff);
   uint64_t* k_full = bars;
   uint64_t* k_empty = k_full + ST;
@@ -443,7 +498,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           *reinterpret_cast<uint4*>(bq + swz128(kTcRows + lane, ch * 16)) =
               make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        inv_c[b * kTcRows + lane] = 1.f / c;
+        row_sc[b * kTcRows + lane] = live ? prm.qk_scale_log2 / c : 0.f;
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -563,7 +618,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int t = threadIdx.x - 128;  // key of a tile, and output column
     const int wi = warp - 4;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wi * 32) << 16);
-    const float sc_log2 = prm.qk_scale_log2;
     uint32_t n = 0, sc = 0, od = 0, xc = 0;
     bool ok = true;
     for (; ok; ++n) {
@@ -573,19 +627,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const TcUnit w = tc_unit(prm, u);
       const int rows = w.q_len * g;  // the unit's query rows
       const int b = n & 1;
-      float m[RM], l[RM], ic[RM];
+      // nm: minus the running maximum (lazily moved, log2 units); kNoMax
+      // marks a row without a visible key yet, and rows past the unit's
+      // (zero rows of Bq, scale 0) are pinned so that they never move nor weigh
+      float nm[RM], l[RM];
 #pragma unroll
       for (int r = 0; r < RM; ++r) {
-        m[r] = -INFINITY;
+        nm[r] = r < rows ? kNoMax : -kNoMax;
         l[r] = 0.f;
       }
-      // the unit's row scales; the buffer is released once read (and once the
-      // MMAs that read Bq are done)
+      // the unit's row scales, read from shared memory at every tile; the Bq
+      // buffer is released at the end of the unit (and once the MMAs that
+      // read it are done)
       if (!warp_wait(&bq_full[b], (n >> 1) & 1)) { ok = false; break; }
-#pragma unroll
-      for (int r = 0; r < RM; ++r) ic[r] = inv_c[b * kTcRows + r] * sc_log2;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bq_empty[b]);
+      const float* ic = row_sc + b * kTcRows;
       for (int32_t j = 0; j < w.ntiles; ++j) {
         const int sb = sc & 1;
         if (!warp_wait(&s_full[sb], (sc >> 1) & 1)) { ok = false; break; }
@@ -596,69 +651,105 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
-        // key pos is seen by the rows of tokens i >= pos - (len - q_len), i.e.
-        // rows r >= thr (all rows for keys before the chunk)
-        const int32_t pos = (w.blk_begin + j * kTcBlocks) * kBlock + t;
-        const bool in_ctx = pos < w.end;
-        const int32_t thr = (pos - (w.len - w.q_len)) * g;
-        float z[RM];
+        const int32_t pos0 = (w.blk_begin + j * kTcBlocks) * kBlock;  // the tile's first key
+        // every key of the tile in the context and before the chunk: every
+        // row sees all of them
+        const bool full = pos0 + kTcKeys <= w.end && pos0 + kTcKeys - 1 <= w.len - w.q_len;
+        float tt[RM];  // the scores, high and low terms joined
 #pragma unroll
-        for (int r = 0; r < RM; ++r)
-          z[r] = (in_ctx && r < rows && r >= thr)
-                     ? fmaf(s[kTcRows + r], 0.0625f, s[r]) * ic[r]
-                     : -INFINITY;
-        // each row's maximum over the warp's 32 keys: reduce-scatter
-        int row;
-        const float v1 = scatter_max<RM>(z, lane, row);
-        float* xm = xmax + (j & 1) * 4 * kTcRows;
-        if ((lane & (32 / RM - 1)) == 0) xm[wi * kTcRows + row] = v1;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(xbar);
-        if (!warp_wait(xbar, xc & 1)) { ok = false; break; }
-        ++xc;
-        float alpha[RM];
-        bool any_grow = false;
+        for (int r = 0; r < RM; ++r) tt[r] = fmaf(s[kTcRows + r], 0.0625f, s[r]);
+        // Common case: an unmasked tile in which no row's maximum moves by
+        // more than the slack; the warps then only agree on that (one flag
+        // each).  Otherwise (a unit's first tile, a masked tile, a moved
+        // maximum) the rows' maxima over the tile are formed and exchanged.
+        bool slow = j == 0 || !full;
+        if (!slow) {
+          bool up = false;
 #pragma unroll
-        for (int r = 0; r < RM; ++r) {
-          const float mt = fmaxf(fmaxf(xm[r], xm[kTcRows + r]),
-                                 fmaxf(xm[2 * kTcRows + r], xm[3 * kTcRows + r]));
-          const bool grow = mt > m[r] + kRescaleSlack;
-          alpha[r] = grow ? fast_exp2(m[r] - mt) : 1.f;  // 0 when m = -inf
-          if (grow) m[r] = mt;
-          any_grow |= grow;
+          for (int r = 0; r < RM; ++r) up |= fmaf(tt[r], ic[r], nm[r]) > kRescaleSlack;
+          const bool wup = __any_sync(0xffffffffu, up);
+          float* xf = xmax + (xc & 1) * 4 * kTcRows;
+          if (lane == 0) xf[wi * kTcRows] = wup ? 1.f : 0.f;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xbar);
+          if (!warp_wait(xbar, xc & 1)) { ok = false; break; }
+          ++xc;
+          slow = (xf[0] + xf[kTcRows]) + (xf[2 * kTcRows] + xf[3 * kTcRows]) != 0.f;
         }
-        // this key's weights, high and low e4m3 terms, and the running sums
-        // two rows at a time: one conversion makes both rows' codes
+        float dd[RM];  // scaled score minus the running maximum (log2 units)
+        bool waited = false;
+        if (!slow) {
+#pragma unroll
+          for (int r = 0; r < RM; ++r) dd[r] = fmaf(tt[r], ic[r], nm[r]);
+        } else {
+          // key pos is seen by the rows of tokens i >= pos - (len - q_len),
+          // i.e. rows r >= thr (all rows for keys before the chunk)
+          const int32_t pos = pos0 + t;
+          const bool in_ctx = pos < w.end;
+          const int32_t thr = (pos - (w.len - w.q_len)) * g;
+          float z[RM];
+#pragma unroll
+          for (int r = 0; r < RM; ++r)
+            z[r] = (in_ctx && r < rows && r >= thr) ? tt[r] * ic[r] : -INFINITY;
+          // each row's maximum over the warp's 32 keys: reduce-scatter; then
+          // the four warps' maxima meet in shared memory
+          int row;
+          const float v1 = scatter_max<RM>(z, lane, row);
+          float* xm = xmax + (xc & 1) * 4 * kTcRows;
+          if ((lane & (32 / RM - 1)) == 0) xm[wi * kTcRows + row] = v1;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xbar);
+          if (!warp_wait(xbar, xc & 1)) { ok = false; break; }
+          ++xc;
+          float alpha[RM];
+          bool any_grow = false;
+#pragma unroll
+          for (int r = 0; r < RM; ++r) {
+            const float mt = fmaxf(fmaxf(xm[r], xm[kTcRows + r]),
+                                   fmaxf(xm[2 * kTcRows + r], xm[3 * kTcRows + r]));
+            const bool grow = mt > kRescaleSlack - nm[r];
+            alpha[r] = grow ? fast_exp2(-(nm[r] + mt)) : 1.f;  // 0 without an earlier key
+            if (grow) nm[r] = -mt;
+            any_grow |= grow;
+            l[r] *= alpha[r];
+            dd[r] = z[r] + nm[r];  // -inf for masked keys
+          }
+          if (j > 0 && any_grow) {  // the same decision in every thread
+            // O^T rescaled once the P V of the tile before has completed
+            if (!warp_wait(o_done, od & 1)) { ok = false; break; }
+            ++od;
+            waited = true;
+            tc_fence_after();
+            // the high columns (0 .. 15), then the low ones
+#pragma unroll 1
+            for (int hl = 0; hl < 2; ++hl) {
+              float o[16];
+              tmem_ld16_wait(lane_base + kTcTmemO + hl * kTcRows, o);
+#pragma unroll
+              for (int r = 0; r < RM; ++r) o[r] *= alpha[r];
+              tmem_st16(lane_base + kTcTmemO + hl * kTcRows, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        // this key's weights (at most 2^slack), high and low e4m3 terms, and
+        // the running sums, two rows per conversion
         uint32_t ph[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int r = 0; r < RM; r += 2) {
-          const float mu0 = m[r] == -INFINITY ? 0.f : m[r];
-          const float mu1 = m[r + 1] == -INFINITY ? 0.f : m[r + 1];
-          const float p0 = fast_exp2(z[r] - mu0), p1 = fast_exp2(z[r + 1] - mu1);
-          l[r] = fmaf(l[r], alpha[r], p0);
-          l[r + 1] = fmaf(l[r + 1], alpha[r + 1], p1);
-          const uint32_t hc = f32x2_to_e4m3x2(p0, p1);
-          const uint32_t hv = e4m3x2_to_f16x2(hc);
-          const uint32_t lc = f32x2_to_e4m3x2((p0 - f16lo_to_f32(hv)) * 16.f,
-                                              (p1 - f16hi_to_f32(hv)) * 16.f);
+          const float p0 = fast_exp2(dd[r]), p1 = fast_exp2(dd[r + 1]);
+          l[r] += p0;
+          l[r + 1] += p1;
+          uint32_t hc, lc;
+          p_codes2(p0, p1, hc, lc);
           ph[r >> 2] |= hc << (8 * (r & 3));
           pl[r >> 2] |= lc << (8 * (r & 3));
         }
-        if (j > 0) {
+        if (j > 0 && !waited) {
+          // P is single-buffered: the P V of the tile before must be done
           if (!warp_wait(o_done, od & 1)) { ok = false; break; }
           ++od;
           tc_fence_after();
-          if (any_grow) {  // the same decision in every thread
-            float o[32];
-            tmem_ld32_wait(lane_base + kTcTmemO, o);
-#pragma unroll
-            for (int r = 0; r < RM; ++r) {
-              o[r] *= alpha[r];
-              o[kTcRows + r] *= alpha[r];
-            }
-            tmem_st32(lane_base + kTcTmemO, o);
-            tmem_wait_st();
-          }
         }
         // key t's row of P: [16 high | 16 low] bytes, 32-byte swizzle
         const uint32_t swz = (static_cast<uint32_t>(t) >> 2) & 1u;
@@ -672,6 +763,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         if (lane == 0) mbar_arrive(p_full);
       }
       if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bq_empty[b]);
       // ---- the unit's result ----
       // row sums over the 128 threads (each holds its keys' share)
 #pragma unroll
@@ -716,7 +809,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             const size_t prow = qrow * prm.max_parts + w.part;
             prm.part_o[prow * 128 + t] = acc * inv;
             if (t == 0) {
-              prm.part_ml[prow * 2 + 0] = m[r] == -INFINITY ? -INFINITY : m[r] * kLn2;
+              prm.part_ml[prow * 2 + 0] = nm[r] >= kNoMax ? -INFINITY : -nm[r] * kLn2;
               prm.part_ml[prow * 2 + 1] = l[r];
             }
           }

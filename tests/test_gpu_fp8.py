@@ -256,8 +256,8 @@ def gpu_fp8_multi(b, partition_tokens=0, plan=False):
     return out
 
 
-# chunks x group <= 8 rows run on the tensor-core kernel (the first four), up to
-# 16 on decode_kernel, longer chunks in row groups
+# chunks x group <= 16 rows run on the tensor-core kernel (4-, 8- and 16-row units),
+# longer chunks in row groups on decode_kernel
 @pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 2), (8, 8, 8), (16, 8, 4), (24, 8, 2),
                                              (32, 8, 4), (8, 8, 16), (16, 2, 2), (12, 4, 5),
                                              (16, 1, 1), (32, 8, 20), (16, 1, 3)])
@@ -280,8 +280,8 @@ def test_fp8_multi_matches_oracle(cuda_device, hq, hkv, max_chunk):
 @pytest.mark.parametrize("partition,chunks", [(16, (4, 3, 4, 1, 2)), (256, (4, 3, 4, 1, 2)),
                                               (16, (2, 1, 2, 2, 1)), (256, (2, 1, 2, 2, 1))])
 def test_fp8_multi_split_k_and_plan_run(cuda_device, partition, chunks):
-    """Split-K and plan/run for chunks of up to 4 tokens (16 rows: decode_kernel) and of
-    up to 2 (8 rows: the tensor-core kernel)."""
+    """Split-K and plan/run for chunks of up to 4 tokens (16-row units) and of up to 2
+    (8-row units), both on the tensor-core kernel."""
     lens = np.array([40, 300, 1000, 2100, 5])
     chunks = np.array(chunks)
     b = workloads.chunked_batch(995 + partition, lens, chunks, 32, 8, 128, "fp8",
@@ -310,3 +310,28 @@ def test_fp8_one_token_chunks_equal_fp8_decode_bitwise(cuda_device):
                                    dev_i32(b.context_lens, cuda_device), b.scale, b.k_scale,
                                    b.v_scale, max_context_len=b.max_context_len)
     assert torch.equal(multi.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("hq,hkv,max_chunk", [(32, 8, 1), (32, 8, 4), (16, 1, 1), (8, 8, 16)])
+def test_fp8_running_max_moves_in_later_tiles(cuda_device, hq, hkv, max_chunk):
+    """Scores scaled up (softmax scale 1.0, about 11 times 1/sqrt(128)) over contexts of
+    many 128-key tiles: the rows' maxima keep moving by more than the rescale slack after
+    a unit's first tile, so the tensor-core kernel's softmax leaves its one-flag path and
+    rescales O in tensor memory mid-unit (4- and 16-row units), beside units that never
+    move."""
+    lens = np.array([700, 1500, 2600, 4100, 130, 257, 16, 3000])
+    chunks = np.minimum(np.full(lens.shape[0], max_chunk), lens)
+    b = workloads.chunked_batch(1201 + hq + max_chunk, lens, chunks, hq, hkv, 128, "fp8",
+                                device=cuda_device)
+    b.k_scale, b.v_scale = workloads.FP8_K_SCALE, workloads.FP8_V_SCALE
+    b.scale = 1.0
+    host = b.host()
+    out = gpu_fp8_multi(b)
+    assert pkv.device_error_bits() == 0
+    k, v = oracle_fp8_caches(b, host)
+    ref = oracle.paged_multi_fp8(host["q"], k, v, b.k_scale, b.v_scale, b.block_tables,
+                                 b.context_lens, b.query_start_loc, b.scale)
+    check_close(out, ref, "bf16", f"fp8 moving maxima {hq}/{hkv} chunks {max_chunk}")
+    split = gpu_fp8_multi(b, 256)
+    assert pkv.device_error_bits() == 0
+    check_close(split, ref, "bf16", f"fp8 moving maxima, 256-token partitions {hq}/{hkv}")
