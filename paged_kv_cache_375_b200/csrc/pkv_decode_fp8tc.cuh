@@ -119,12 +119,6 @@ __host__ __device__ constexpr uint32_t umma_idesc_f8(int M, int N, int a_fmt, bo
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// e4m3 code of x (round to nearest even, saturating) and its value.
-__device__ __forceinline__ uint32_t e4m3_code(float x) { return f32x2_to_e4m3x2(x, 0.f) & 0xffu; }
-__device__ __forceinline__ float e4m3_value(uint32_t code) {
-  return f16lo_to_f32(e4m3x2_to_f16x2(code));
-}
-
 // The weights p0, p1 of two rows as two-term e4m3 codes, formed in f16x2: the
 // high pair hi = e4m3(p) and the low pair e4m3(16 (p - hi)), p0 in the low
 // byte of each.  p - hi is exact in f16 (hi is p rounded to 4 significant
@@ -219,36 +213,42 @@ __device__ __forceinline__ TcUnit tc_unit(const DecodeParams& prm, int32_t u) {
   return w;
 }
 
-// One halving step of a reduce-scatter of row maxima over the warp: lanes with
-// bit `off` set keep the upper HALF rows, the others the lower, each taking
-// the maximum with its partner's copy.
-template <int HALF>
+// One halving step of a reduce-scatter of per-row values over the warp
+// (maxima, or sums if SUM): lanes with bit `off` set keep the upper HALF rows,
+// the others the lower, each combining them with its partner's copy.
+template <int HALF, bool SUM>
 __device__ __forceinline__ void scatter_step(float* v, int lane, int off, int& row) {
   const bool upper = lane & off;
 #pragma unroll
   for (int i = 0; i < HALF; ++i) {
     const float send = upper ? v[i] : v[HALF + i];
     const float keep = upper ? v[HALF + i] : v[i];
-    v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+    const float other = __shfl_xor_sync(0xffffffffu, send, off);
+    v[i] = SUM ? keep + other : fmaxf(keep, other);
   }
   if (upper) row += HALF;
 }
 
-// The maxima of RM rows over the warp's 32 lanes: afterwards the lanes whose
-// low bits (below 32 / RM) are zero hold the maximum of row `row`.
-template <int RM>
-__device__ __forceinline__ float scatter_max(const float (&z)[RM], int lane, int& row) {
+// The maxima (or sums if SUM) of RM rows over the warp's 32 lanes, in RM - 1
+// + log2(32 / RM) shuffles: afterwards every lane holds the result for row
+// `row`, and the lanes whose low bits (below 32 / RM) are zero are the first
+// of each row.
+template <int RM, bool SUM = false>
+__device__ __forceinline__ float scatter_reduce(const float (&z)[RM], int lane, int& row) {
   float v[RM];
 #pragma unroll
   for (int i = 0; i < RM; ++i) v[i] = z[i];
   row = 0;
   int off = 16;
-  if constexpr (RM >= 16) { scatter_step<8>(v, lane, off, row); off >>= 1; }
-  if constexpr (RM >= 8) { scatter_step<4>(v, lane, off, row); off >>= 1; }
-  if constexpr (RM >= 4) { scatter_step<2>(v, lane, off, row); off >>= 1; }
-  if constexpr (RM >= 2) { scatter_step<1>(v, lane, off, row); off >>= 1; }
+  if constexpr (RM >= 16) { scatter_step<8, SUM>(v, lane, off, row); off >>= 1; }
+  if constexpr (RM >= 8) { scatter_step<4, SUM>(v, lane, off, row); off >>= 1; }
+  if constexpr (RM >= 4) { scatter_step<2, SUM>(v, lane, off, row); off >>= 1; }
+  if constexpr (RM >= 2) { scatter_step<1, SUM>(v, lane, off, row); off >>= 1; }
   float r = v[0];
-  for (; off > 0; off >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, off));
+  for (; off > 0; off >>= 1) {
+    const float other = __shfl_xor_sync(0xffffffffu, r, off);
+    r = SUM ? r + other : fmaxf(r, other);
+  }
   return r;
 }
 
@@ -446,59 +446,66 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const int b = n & 1;
       if (n >= 2 && !warp_wait(&bq_empty[b], ((n >> 1) + 1) & 1)) { ok = false; break; }
       uint8_t* bq = sBq + b * Lay::kBqBytes;
-      if (lane < kTcRows) {
-        // the unit's row `lane` (token lane / g, head lane % g): high terms in
-        // row lane, low in 16 + lane
+      {
+        // the unit's row `row` (token row / g, head row % g), its codes 0-63
+        // from lane row and 64-127 from lane 16 + row: high terms in row
+        // `row` of Bq, low in 16 + row
+        const int row = lane & (kTcRows - 1), part = lane >> 4;
         float c = 1.f;
-        const bool live = lane < w.q_len * g;
-        const size_t qrow = live ? static_cast<size_t>(w.q_start + lane / g) * prm.num_q_heads +
-                                       w.kv_head * g + lane % g
+        const bool live = row < w.q_len * g;
+        const size_t qrow = live ? static_cast<size_t>(w.q_start + row / g) * prm.num_q_heads +
+                                       w.kv_head * g + row % g
                                  : 0;
         const uint4* src = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(prm.q) + qrow * 128);
+                               static_cast<const __nv_bfloat16*>(prm.q) + qrow * 128) +
+                           part * 8;
+        float mx = 0.f;
         if (live) {
-          float mx = 0.f;
 #pragma unroll 4
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             const uint4 v = src[i];
             const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               mx = fmaxf(mx, fmaxf(fabsf(bf16lo_to_f32(vv[k])), fabsf(bf16hi_to_f32(vv[k]))));
           }
-          // c = 2^(7 - e) with mx = f 2^e, f in [0.5, 1): |c q| < 128
-          if (mx > 0.f && isfinite(mx)) {
-            int e;
-            frexpf(mx, &e);
-            c = ldexpf(1.f, 7 - e);
-          }
         }
-        // 16 codes (one 16-byte chunk of each of the two rows) per step;
-        // rows of 128 codes with the 128-byte swizzle
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the row's other half
+        // c = 2^(7 - e) with mx = f 2^e, f in [0.5, 1): |c q| < 128
+        if (live && mx > 0.f && isfinite(mx)) {
+          int e;
+          frexpf(mx, &e);
+          c = ldexpf(1.f, 7 - e);
+        }
+        // 16 codes (one 16-byte chunk of each of the two rows) per step, two
+        // per conversion; rows of 128 codes with the 128-byte swizzle
 #pragma unroll 2
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int cq = 0; cq < 4; ++cq) {
+          const int ch = part * 4 + cq;
           uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
           if (live) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-              const uint4 v = src[2 * ch + half];
+              const uint4 v = src[2 * cq + half];
               const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const float x = (k & 1 ? bf16hi_to_f32(vv[k >> 1]) : bf16lo_to_f32(vv[k >> 1])) * c;
-                const uint32_t hc = e4m3_code(x);
-                const uint32_t lc = e4m3_code((x - e4m3_value(hc)) * 16.f);
-                const int byte = half * 8 + k;
+              for (int k = 0; k < 4; ++k) {
+                const float x0 = bf16lo_to_f32(vv[k]) * c, x1 = bf16hi_to_f32(vv[k]) * c;
+                const uint32_t hc = f32x2_to_e4m3x2(x0, x1);
+                const uint32_t hv = e4m3x2_to_f16x2(hc);
+                const uint32_t lc = f32x2_to_e4m3x2((x0 - f16lo_to_f32(hv)) * 16.f,
+                                                    (x1 - f16hi_to_f32(hv)) * 16.f);
+                const int byte = half * 8 + 2 * k;  // even: the pair fills half a word
                 hi[byte >> 2] |= hc << (8 * (byte & 3));
                 lo[byte >> 2] |= lc << (8 * (byte & 3));
               }
             }
           }
-          *reinterpret_cast<uint4*>(bq + swz128(lane, ch * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(bq + swz128(kTcRows + lane, ch * 16)) =
+          *reinterpret_cast<uint4*>(bq + swz128(row, ch * 16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(bq + swz128(kTcRows + row, ch * 16)) =
               make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        row_sc[b * kTcRows + lane] = live ? prm.qk_scale_log2 / c : 0.f;
+        if (part == 0) row_sc[b * kTcRows + row] = live ? prm.qk_scale_log2 / c : 0.f;
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -694,7 +701,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           // each row's maximum over the warp's 32 keys: reduce-scatter; then
           // the four warps' maxima meet in shared memory
           int row;
-          const float v1 = scatter_max<RM>(z, lane, row);
+          const float v1 = scatter_reduce<RM>(z, lane, row);
           float* xm = xmax + (xc & 1) * 4 * kTcRows;
           if ((lane & (32 / RM - 1)) == 0) xm[wi * kTcRows + row] = v1;
           __syncwarp();
@@ -766,26 +773,27 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bq_empty[b]);
       // ---- the unit's result ----
-      // row sums over the 128 threads (each holds its keys' share)
-#pragma unroll
-      for (int r = 0; r < RM; ++r) {
-        float v = l[r];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        l[r] = v;
-      }
+      // row sums over the 128 threads (each holds its keys' share): a
+      // reduce-scatter over the warp, then the four warps' sums meet in
+      // shared memory
+      int srow;
+      const float lw = scatter_reduce<RM, true>(l, lane, srow);
       float* xs = xsum + b * 4 * kTcRows;
-      if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < RM; ++r) xs[wi * kTcRows + r] = l[r];
-      }
+      if ((lane & (32 / RM - 1)) == 0) xs[wi * kTcRows + srow] = lw;
       __syncwarp();
       if (lane == 0) mbar_arrive(xbar);
       if (!warp_wait(xbar, xc & 1)) { ok = false; break; }
       ++xc;
-#pragma unroll
-      for (int r = 0; r < RM; ++r)
-        l[r] = (xs[r] + xs[kTcRows + r]) + (xs[2 * kTcRows + r] + xs[3 * kTcRows + r]);
+      // lane r < RM works out row r's sum, output factor and output row once;
+      // the loop below takes them from that lane
+      float l_my = 0.f, inv_my = 0.f;
+      int64_t qrow_my = 0;
+      if (lane < RM) {
+        l_my = (xs[lane] + xs[kTcRows + lane]) + (xs[2 * kTcRows + lane] + xs[3 * kTcRows + lane]);
+        inv_my = l_my > 0.f ? prm.out_scale / l_my : 0.f;
+        qrow_my = static_cast<int64_t>(w.q_start + lane / g) * prm.num_q_heads +
+                  w.kv_head * g + lane % g;
+      }
       float o[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -797,20 +805,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       }
 #pragma unroll
       for (int r = 0; r < RM; ++r) {
-        if (r < rows) {
-          const size_t qrow = static_cast<size_t>(w.q_start + r / g) * prm.num_q_heads +
-                              w.kv_head * g + r % g;
+        if (r < rows) {  // the same in every thread
+          const size_t qrow = static_cast<size_t>(__shfl_sync(0xffffffffu, qrow_my, r));
+          const float inv = __shfl_sync(0xffffffffu, inv_my, r);
           const float acc = fmaf(o[kTcRows + r], 0.0625f, o[r]);
-          const float inv = l[r] > 0.f ? prm.out_scale / l[r] : 0.f;
           if (w.nparts == 1) {
             reinterpret_cast<uint16_t*>(prm.out)[qrow * 128 + t] =
                 static_cast<uint16_t>(pack_bf16x2(acc * inv, 0.f));
           } else {
             const size_t prow = qrow * prm.max_parts + w.part;
+            const float lr = __shfl_sync(0xffffffffu, l_my, r);
             prm.part_o[prow * 128 + t] = acc * inv;
             if (t == 0) {
               prm.part_ml[prow * 2 + 0] = nm[r] >= kNoMax ? -INFINITY : -nm[r] * kLn2;
-              prm.part_ml[prow * 2 + 1] = l[r];
+              prm.part_ml[prow * 2 + 1] = lr;
             }
           }
         }
