@@ -682,11 +682,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         float mxp[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
-        if (pos0 + KH - 1 <= lim_min) {
+        float ks = 1.f;  // the part of the scale still to apply, inside the exponent
+        if (pos0 + KH - 1 <= lim_min && sc_log2 >= 0.f) {
+          // unmasked, scale >= 0: the maximum of the raw scores, scaled once;
+          // each score's scaling joins its exponent's subtraction
+#pragma unroll
+          for (int c = 0; c < KH; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);  // eight chains
+          ks = sc_log2;
+        } else if (pos0 + KH - 1 <= lim_min) {
 #pragma unroll
           for (int c = 0; c < KH; ++c) {
             s[c] *= sc_log2;
-            mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);  // eight independent chains
+            mxp[c & 7] = fmaxf(mxp[c & 7], s[c]);
           }
         } else {
 #pragma unroll
@@ -696,7 +703,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
         float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+                         fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * ks;
         // the row's maximum over both halves
         xmax[((j & 1) * 2 + half) * kPfRows + r] = mx;
         __syncwarp();
@@ -717,7 +724,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int e = 0; e < 8; ++e) lsp[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < KH / 2; ++c) {
-          const float p0 = fast_exp2(s[2 * c] - mu), p1 = fast_exp2(s[2 * c + 1] - mu);
+          const float p0 = fast_exp2(fmaf(s[2 * c], ks, -mu));
+          const float p1 = fast_exp2(fmaf(s[2 * c + 1], ks, -mu));
           pk[c] = pack_bf16x2(p0, p1);
           lsp[c & 7] += p0 + p1;
         }
