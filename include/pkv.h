@@ -373,8 +373,9 @@ pkv_status pkv_decode_prepare_tokens(const void *k, const void *v, void *k_cache
  *    even, saturate to +-448); slots as in pkv_reshape_and_cache.
  *  - pkv_paged_attention_decode_fp8 / pkv_decode_run_fp8: as the bf16 calls,
  *    over e4m3 pools with their k_scale and v_scale; q and out are bf16.
- *    Arithmetic when a sequence's query rows (chunk tokens x heads per kv
- *    head) number at most 8 and there is no shared prefix: the codes (e4m3
+ *    Arithmetic when every sequence's query rows (its chunk's tokens x heads
+ *    per kv head, for the longest chunk) number at most 16 and there is no
+ *    shared prefix: the codes (e4m3
  *    or e5m2) enter the tensor cores as they are, q (times a power of two per
  *    row) and the softmax weights as two e4m3 terms each (the rounded value
  *    and 16 x its rounding remainder, about 8 significant bits), products
