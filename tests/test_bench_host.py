@@ -98,3 +98,31 @@ def test_plan_item_accounting():
     split = types.SimpleNamespace(b=b, part_tokens=64, shared=True)
     n_own = int(np.maximum(1, (lens - 256 + 63) // 64).sum())
     assert bench.plan_items(split) == 4 * (256 // 64) * 2 + n_own
+
+
+def test_dominant_kernel_follows_the_dispatch():
+    """The kernel bench.py names in `roofline` is the one pkv_api.cu launches: FP8
+    units of up to 16 query rows (one token x g, or a few draft tokens x g) on the
+    tensor-core kernel, longer chunks and shared-prefix plans on decode_kernel, short
+    bf16 items on the warp kernel, long chunks on the prefill kernel."""
+    from types import SimpleNamespace as NS
+
+    def step(dtype, hq, hkv, qlen=None, shared=False, split=False, part_tokens=4096,
+             prefill=False):
+        b = NS(dtype=dtype, num_q_heads=hq, num_kv_heads=hkv, head_dim=128,
+               max_query_len=qlen or 1)
+        return NS(b=b, multi=qlen is not None, shared=shared, split=split,
+                  part_tokens=part_tokens, prefill=prefill)
+
+    dk = bench.dominant_kernel
+    assert dk(step("fp8", 32, 8)) == "decode_fp8tc_kernel"                 # 4 rows
+    assert dk(step("fp8e5m2", 32, 8)) == "decode_fp8tc_kernel"
+    assert dk(step("fp8", 32, 8, qlen=4)) == "decode_fp8tc_kernel"         # 16 rows
+    assert dk(step("fp8", 16, 1)) == "decode_fp8tc_kernel"                 # g = 16
+    assert dk(step("fp8", 32, 8, qlen=5)) == "decode_kernel"               # row groups
+    assert dk(step("fp8", 32, 8, shared=True)) == "decode_kernel"
+    assert dk(step("bf16", 32, 8)) == "decode_kernel"                      # single pass
+    assert dk(step("bf16", 32, 8, split=True, part_tokens=512)) == "decode_warp_kernel"
+    assert dk(step("bf16", 32, 8, shared=True, part_tokens=512)) == "decode_warp_kernel"
+    assert dk(step("bf16", 32, 8, qlen=4)) == "decode_kernel"
+    assert dk(step("bf16", 32, 8, qlen=1024, prefill=True)) == "prefill_kernel"
