@@ -587,6 +587,37 @@ def test_e4m3_rounds_to_the_nearest_value_ties_to_even():
         assert ci in best, (xi, ci, best)
 
 
+def test_two_term_e4m3_keeps_eight_bits():
+    """The reading of the FP8 tensor-core arithmetic: q (scaled by a power of two so that
+    |c q| < 128) and the weights (at most 2^8 under the lazy maximum) enter as
+    high = e4m3(x) and low = e4m3(16 (x - high)), x ~ high + low / 16.  From e4m3's
+    definition: 3 stored mantissa bits per term, the low term 4 binades finer, so for
+    |x| in [2^-6, 2^8) the pair is within 2^-8 relative (about 8 significant bits, as
+    bf16); below 2^-6 the low term reaches e4m3's subnormals and the error stays under
+    2^-14 absolute.  The weights are first rounded to f16 (11 bits), which adds at most
+    2^-11 relative."""
+    rng = np.random.default_rng(31)
+    n = 200000
+    sign = rng.choice([-1.0, 1.0], n)
+
+    def pair(x):
+        hi = oracle.e4m3_values(oracle.e4m3_quantize(x))
+        lo = oracle.e4m3_values(oracle.e4m3_quantize(16.0 * (x - hi)))
+        return hi + lo / 16.0
+
+    x = np.exp2(rng.uniform(-6, 8, n)) * sign
+    rel = np.abs(pair(x) - x) / np.abs(x)
+    assert rel.max() <= 2.0 ** -8
+    x16 = x.astype(np.float16).astype(np.float64)          # the weights' f16 step
+    rel16 = np.abs(pair(x16) - x) / np.abs(x)
+    assert rel16.max() <= 2.0 ** -8 + 2.0 ** -11
+    small = np.exp2(rng.uniform(-24, -6, n)) * sign
+    assert np.abs(pair(small) - small).max() <= 2.0 ** -14
+    # one term alone is only 4 bits: the pair is what makes the tolerance hold
+    one = oracle.e4m3_values(oracle.e4m3_quantize(x))
+    assert (np.abs(one - x) / np.abs(x)).max() > 2.0 ** -5
+
+
 def test_e4m3_divides_by_the_scale_in_float():
     x = np.array([1.0, 3.0, -7.5], dtype=np.float32)
     assert np.array_equal(oracle.e4m3_quantize(x, 0.5), oracle.e4m3_quantize(x / np.float32(0.5)))
